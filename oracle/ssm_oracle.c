@@ -1,0 +1,318 @@
+/*
+ * Float64 CPU oracle for the selective diagonal state-space scan and its exact gradient.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, the package's smoke check and the bench's CPU-baseline
+ * leg may load this file's library.  It shares no code, header, table or helper with the CUDA
+ * path: it is the plain definition, written as a sequential loop over time per independent
+ * channel, plus the hand-derived reverse-time adjoint.  No blocking, fusion or reordering of the
+ * arithmetic beyond "channels are independent" (OpenMP runs whole channels on separate threads;
+ * the cross-channel sums dB, dC, dr, dphi are added per thread, then thread by thread in index
+ * order, so a fixed thread count gives a bitwise-fixed result).  Build without -ffast-math.
+ *
+ * Real mode.  The selective SSM of "选择性状态空间模型(S3M)原理与工程实践" §1.1 (step size
+ * delta = softplus(projection), decay A = -exp(log_A), transition exp(A·delta)), with the Euler
+ * input term delta·B_t·x_t:
+ *     delta_t = softplus(delta_raw_t),  A_n = -exp(A_log_n),  a_{t,n} = exp(delta_t A_n)
+ *     h_{t,n} = a_{t,n} h_{t-1,n} + delta_t Bm_{t,n} x_t,   h_{-1} = 0
+ *     y_t     = sum_n Cm_{t,n} h_{t,n} + Dskip x_t
+ * The gradient is the exact reverse-time adjoint of "Breaking the Memory Wall: Exact Analytical
+ * Differentiation via Tiled Operator-Space Evolution" (abstract: exact analytical derivatives in
+ * the state space, no stored graph), derived by hand for the loss L = sum dy·y:
+ *     g_t    = Cm_t dy_t + a_{t+1} g_{t+1},  g_{L-1} = Cm_{L-1} dy_{L-1}     (g_t = dL/dh_t)
+ *     q_t    = g_t a_t h_{t-1}                                               (dL/d log a_t)
+ *     dx_t   = Dskip dy_t + delta_t sum_n g_t Bm_t
+ *     ddelta = sum_n A_n q_t + x_t sum_n g_t Bm_t;   ddelta_raw = ddelta · sigmoid(delta_raw)
+ *     dBm_t  = sum_d g_t delta_t x_t;   dCm_t = sum_d dy_t h_t
+ *     dA_log = A_n sum_{b,t} delta_t q_t;   dDskip = sum_{b,t} dy_t x_t
+ *
+ * Complex mode.  "SPARC: Shared Phase and Retention Control for Efficient Adaptive Spectral
+ * Recurrence" (abstract: two input-dependent scalars, retention r_t and phase phi_t, drive all
+ * complex modes, each with its own timescale lambda_k and frequency omega_k; diagonal affine
+ * recurrence):
+ *     s_t = softplus(r_t),  a_{t,k} = exp(-lambda_k s_t + i omega_k phi_t),  h_t = a_t h_{t-1} + u_t
+ * Loss L = Re sum conj(g) h; complex gradients use d/dRe + i d/dIm (PyTorch's .grad convention):
+ *     mu_t = g_t + conj(a_{t+1}) mu_{t+1};  du_t = mu_t;  q_t = mu_t conj(a_t h_{t-1})
+ *     dlambda_k = -sum s_t Re q;  dr_t = sigmoid(r_t) (-sum_k lambda_k Re q)
+ *     domega_k  =  sum phi_t Im q;  dphi_t = sum_k omega_k Im q
+ */
+#include <complex.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double softplus(double z) { return z > 0.0 ? z + log1p(exp(-z)) : log1p(exp(z)); }
+
+static double sigmoid(double z) {
+    if (z >= 0.0) return 1.0 / (1.0 + exp(-z));
+    double e = exp(z);
+    return e / (1.0 + e);
+}
+
+int ssm_oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static int pick_threads(int nthreads) {
+    int m = ssm_oracle_max_threads();
+    if (nthreads <= 0 || nthreads > m) nthreads = m;
+    return nthreads;
+}
+
+/*
+ * Real mode, channels d in [d_lo, d_hi).  Inputs (row-major, float64):
+ *   x, draw, dy [B,L,D]; Bm, Cm [B,L,N]; A_log [D,N]; Dskip [D].  dy may be NULL (forward only).
+ * Outputs (NULL to skip): y [B,L,D] and, when dy is given, dx, ddraw [B,L,D] — only entries with
+ * d in range are written; ckpt [B, ceil(L/T), D, N] holds h at the last step of every chunk of T
+ * steps; dA_log [D,N] and dD [D] rows in range (summed over all b); dB, dC [B,L,N] are fully
+ * overwritten with the sums over the channels in range.
+ * Returns 0, or -1 on a bad argument / allocation failure.
+ */
+int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
+                    const double* x, const double* draw, const double* A_log, const double* Bm,
+                    const double* Cm, const double* Dskip, const double* dy,
+                    int64_t d_lo, int64_t d_hi, int nthreads,
+                    double* y, double* ckpt, double* dx, double* ddraw,
+                    double* dA_log, double* dB, double* dC, double* dD) {
+    if (B < 0 || L < 0 || D <= 0 || N <= 0 || T <= 0 || d_lo < 0 || d_hi > D || d_lo > d_hi)
+        return -1;
+    const int64_t nC = (L + T - 1) / T;
+    const int bwd = dy != NULL;
+    nthreads = pick_threads(nthreads);
+    const size_t bln = (size_t)B * (size_t)L * (size_t)N;
+    double** part_dB = NULL;
+    double** part_dC = NULL;
+    int fail = 0;
+    if (bwd) {
+        part_dB = (double**)calloc((size_t)nthreads, sizeof(double*));
+        part_dC = (double**)calloc((size_t)nthreads, sizeof(double*));
+        if (!part_dB || !part_dC) { free(part_dB); free(part_dC); return -1; }
+    }
+
+#pragma omp parallel num_threads(nthreads)
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        tid = omp_get_thread_num();
+#endif
+        double* hh = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * (size_t)N);
+        double* aa = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * (size_t)N);
+        double* A = (double*)malloc(sizeof(double) * (size_t)N);
+        double* h = (double*)malloc(sizeof(double) * (size_t)N);
+        double* v = (double*)malloc(sizeof(double) * (size_t)N);
+        double* dAsum = (double*)malloc(sizeof(double) * (size_t)N);
+        double* myB = NULL;
+        double* myC = NULL;
+        if (bwd) {
+            myB = (double*)calloc(bln > 0 ? bln : 1, sizeof(double));
+            myC = (double*)calloc(bln > 0 ? bln : 1, sizeof(double));
+            part_dB[tid] = myB;
+            part_dC[tid] = myC;
+        }
+        if (!hh || !aa || !A || !h || !v || !dAsum || (bwd && (!myB || !myC))) {
+#pragma omp atomic write
+            fail = 1;
+        }
+#pragma omp barrier
+        if (!fail) {
+#pragma omp for schedule(static)
+            for (int64_t d = d_lo; d < d_hi; ++d) {
+                for (int64_t n = 0; n < N; ++n) {
+                    A[n] = -exp(A_log[d * N + n]);
+                    dAsum[n] = 0.0;
+                }
+                double dDsum = 0.0;
+                for (int64_t b = 0; b < B; ++b) {
+                    /* forward: sequential recurrence, full history of a and h kept */
+                    for (int64_t n = 0; n < N; ++n) h[n] = 0.0;
+                    for (int64_t t = 0; t < L; ++t) {
+                        const int64_t i = (b * L + t) * D + d;
+                        const double* Bt = Bm + (b * L + t) * N;
+                        const double* Ct = Cm + (b * L + t) * N;
+                        const double delta = softplus(draw[i]);
+                        double acc = 0.0;
+                        for (int64_t n = 0; n < N; ++n) {
+                            const double a = exp(delta * A[n]);
+                            h[n] = a * h[n] + delta * Bt[n] * x[i];
+                            aa[t * N + n] = a;
+                            hh[t * N + n] = h[n];
+                            acc += Ct[n] * h[n];
+                        }
+                        if (y) y[i] = acc + Dskip[d] * x[i];
+                        if (ckpt && (t == L - 1 || (t + 1) % T == 0)) {
+                            double* ck = ckpt + ((b * nC + t / T) * D + d) * N;
+                            for (int64_t n = 0; n < N; ++n) ck[n] = h[n];
+                        }
+                    }
+                    if (!bwd) continue;
+                    /* backward: reverse-time adjoint; v = a_{t+1} g_{t+1} */
+                    for (int64_t n = 0; n < N; ++n) v[n] = 0.0;
+                    for (int64_t t = L - 1; t >= 0; --t) {
+                        const int64_t i = (b * L + t) * D + d;
+                        const double* Bt = Bm + (b * L + t) * N;
+                        const double* Ct = Cm + (b * L + t) * N;
+                        const double delta = softplus(draw[i]);
+                        double sum_gB = 0.0, sum_Aq = 0.0;
+                        for (int64_t n = 0; n < N; ++n) {
+                            const double a = aa[t * N + n];
+                            const double hprev = t > 0 ? hh[(t - 1) * N + n] : 0.0;
+                            const double g = Ct[n] * dy[i] + v[n];
+                            const double q = g * a * hprev;
+                            sum_Aq += A[n] * q;
+                            sum_gB += g * Bt[n];
+                            dAsum[n] += delta * q;
+                            myB[(b * L + t) * N + n] += g * delta * x[i];
+                            myC[(b * L + t) * N + n] += dy[i] * hh[t * N + n];
+                            v[n] = a * g;
+                        }
+                        if (dx) dx[i] = Dskip[d] * dy[i] + delta * sum_gB;
+                        if (ddraw) ddraw[i] = (sum_Aq + x[i] * sum_gB) * sigmoid(draw[i]);
+                        dDsum += dy[i] * x[i];
+                    }
+                }
+                if (bwd) {
+                    if (dA_log)
+                        for (int64_t n = 0; n < N; ++n) dA_log[d * N + n] = A[n] * dAsum[n];
+                    if (dD) dD[d] = dDsum;
+                }
+            }
+        }
+        free(hh); free(aa); free(A); free(h); free(v); free(dAsum);
+    }
+
+    if (bwd) {
+        if (!fail) {
+            if (dB) memset(dB, 0, sizeof(double) * bln);
+            if (dC) memset(dC, 0, sizeof(double) * bln);
+            for (int tt = 0; tt < nthreads; ++tt) {
+                for (size_t j = 0; j < bln; ++j) {
+                    if (dB) dB[j] += part_dB[tt][j];
+                    if (dC) dC[j] += part_dC[tt][j];
+                }
+            }
+        }
+        for (int tt = 0; tt < nthreads; ++tt) { free(part_dB[tt]); free(part_dC[tt]); }
+        free(part_dB);
+        free(part_dC);
+    }
+    return fail ? -1 : 0;
+}
+
+/*
+ * Complex mode, modes k in [k_lo, k_hi).  u, g, h, du are [B,L,K] complex (interleaved re, im
+ * doubles); r, phi [B,L]; lambda, omega [K].  g may be NULL (forward only).  h, du entries with k
+ * in range are written; dlambda, domega entries in range; dr, dphi [B,L] are fully overwritten
+ * with the sums over the modes in range.  Returns 0 or -1.
+ */
+int ssm_oracle_complex(int64_t B, int64_t L, int64_t K,
+                       const double* u_, const double* r, const double* phi,
+                       const double* lambda, const double* omega, const double* g_,
+                       int64_t k_lo, int64_t k_hi, int nthreads,
+                       double* h_, double* du_, double* dr, double* dphi,
+                       double* dlambda, double* domega) {
+    if (B < 0 || L < 0 || K <= 0 || k_lo < 0 || k_hi > K || k_lo > k_hi) return -1;
+    const double complex* u = (const double complex*)u_;
+    const double complex* g = (const double complex*)g_;
+    double complex* hout = (double complex*)h_;
+    double complex* du = (double complex*)du_;
+    const int bwd = g != NULL;
+    nthreads = pick_threads(nthreads);
+    const size_t bl = (size_t)B * (size_t)L;
+    double** part_r = NULL;
+    double** part_p = NULL;
+    int fail = 0;
+    if (bwd) {
+        part_r = (double**)calloc((size_t)nthreads, sizeof(double*));
+        part_p = (double**)calloc((size_t)nthreads, sizeof(double*));
+        if (!part_r || !part_p) { free(part_r); free(part_p); return -1; }
+    }
+
+#pragma omp parallel num_threads(nthreads)
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        tid = omp_get_thread_num();
+#endif
+        const size_t Lp = (size_t)(L > 0 ? L : 1);
+        double complex* hh = (double complex*)malloc(sizeof(double complex) * Lp);
+        double complex* aa = (double complex*)malloc(sizeof(double complex) * Lp);
+        double* myr = NULL;
+        double* myp = NULL;
+        if (bwd) {
+            myr = (double*)calloc(bl > 0 ? bl : 1, sizeof(double));
+            myp = (double*)calloc(bl > 0 ? bl : 1, sizeof(double));
+            part_r[tid] = myr;
+            part_p[tid] = myp;
+        }
+        if (!hh || !aa || (bwd && (!myr || !myp))) {
+#pragma omp atomic write
+            fail = 1;
+        }
+#pragma omp barrier
+        if (!fail) {
+#pragma omp for schedule(static)
+            for (int64_t k = k_lo; k < k_hi; ++k) {
+                const double lam = lambda[k], om = omega[k];
+                double dlam = 0.0, dom = 0.0;
+                for (int64_t b = 0; b < B; ++b) {
+                    double complex h = 0.0;
+                    for (int64_t t = 0; t < L; ++t) {
+                        const int64_t j = b * L + t;
+                        const double s = softplus(r[j]);
+                        const double complex a = cexp(-lam * s + I * (om * phi[j]));
+                        h = a * h + u[j * K + k];
+                        aa[t] = a;
+                        hh[t] = h;
+                        if (hout) hout[j * K + k] = h;
+                    }
+                    if (!bwd) continue;
+                    double complex mu_next = 0.0; /* conj(a_{t+1}) mu_{t+1} */
+                    for (int64_t t = L - 1; t >= 0; --t) {
+                        const int64_t j = b * L + t;
+                        const double s = softplus(r[j]);
+                        const double complex mu = g[j * K + k] + mu_next;
+                        const double complex hprev = t > 0 ? hh[t - 1] : 0.0;
+                        const double complex q = mu * conj(aa[t] * hprev);
+                        if (du) du[j * K + k] = mu;
+                        dlam += -s * creal(q);
+                        dom += phi[j] * cimag(q);
+                        myr[j] += -lam * creal(q);
+                        myp[j] += om * cimag(q);
+                        mu_next = conj(aa[t]) * mu;
+                    }
+                }
+                if (bwd) {
+                    if (dlambda) dlambda[k] = dlam;
+                    if (domega) domega[k] = dom;
+                }
+            }
+        }
+        free(hh); free(aa);
+    }
+
+    if (bwd) {
+        if (!fail) {
+            if (dr) memset(dr, 0, sizeof(double) * bl);
+            if (dphi) memset(dphi, 0, sizeof(double) * bl);
+            for (int tt = 0; tt < nthreads; ++tt) {
+                for (size_t j = 0; j < bl; ++j) {
+                    if (dr) dr[j] += part_r[tt][j];
+                    if (dphi) dphi[j] += part_p[tt][j];
+                }
+            }
+            if (dr)
+                for (size_t j = 0; j < bl; ++j) dr[j] *= sigmoid(r[j]);
+        }
+        for (int tt = 0; tt < nthreads; ++tt) { free(part_r[tt]); free(part_p[tt]); }
+        free(part_r);
+        free(part_p);
+    }
+    return fail ? -1 : 0;
+}
