@@ -1,0 +1,343 @@
+#!/usr/bin/env python
+"""Throughput of the selective scan's forward + exact backward on B200.
+
+One step = ssm_scan_fwd + ssm_scan_bwd over one batch of the workload (inputs resident in HBM),
+plus, with more than one rank, the data-parallel all-reduce of the parameter gradients
+(dA_log, dD).  Each rank owns a full batch of the workload (weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Rank 0 prints one JSON line.  ``value`` is state-updates/s over all ranks (B*L*D*N per rank per
+step), device-timed with CUDA events, max over ranks; L2 is flushed (a 256 MiB write) before every
+timed step, outside the events.  ``e2e`` is the same metric through the same calls with the inputs
+copied in from pinned host memory and every output copied back inside the timed region.
+``--impl reference`` times the float64 CPU oracle on the host cores instead (bounded sample).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd scan state-updates/s (B·L·D·N/s); achieved HBM GB/s vs B200 peak"
+UNIT = "state-updates/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mamba130m_layer")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seg-chunks", type=int, default=0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w):
+    """Minimum bytes the method moves per step (fwd + bwd), split by call."""
+    from selective_state_space_bwd_b200 import inputs as gen
+    s = 2 if w.io == gen.BF16 else 4
+    E = w.batch * w.seqlen * w.dim
+    BLN = w.batch * w.seqlen * w.dstate
+    nC = -(-w.seqlen // w.chunk)
+    ck = w.batch * nC * w.dim * w.dstate * 4
+    fwd = 3 * E * s + 2 * BLN * s + ck           # x, delta_raw in; y out; Bm, Cm in; ckpt out
+    bwd = 5 * E * s + 4 * BLN * s + ck           # x, delta_raw, dy in; dx, ddelta_raw out;
+    return fwd, bwd                              # Bm, Cm in; dB, dC out; ckpt in
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(w, inp, budget_s=(10.0, 30.0)):
+    """Time the float64 oracle on the host cores: whole batch rows of the workload, repeated
+    until about budget_s[0] seconds of work (stops before budget_s[1])."""
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    rows = 0
+    t_total = 0.0
+    b = 0
+    while t_total < budget_s[0]:
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        oracle.real(inp["x"][sl], inp["delta_raw"][sl], inp["A_log"], inp["Bm"][sl], inp["Cm"][sl],
+                    inp["Dskip"], inp["dy"][sl], chunk=w.chunk, threads=threads)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        rows += 1
+        b = (b + 1) % w.batch
+        if t_total + dt > budget_s[1]:
+            break
+    upd = rows * w.seqlen * w.dim * w.dstate
+    return {"value": upd / t_total, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, D={w.dim}, N={w.dstate}), "
+                      f"fwd+bwd in float64, {t_total:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from selective_state_space_bwd_b200 import inputs as gen
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    inp = gen.real_inputs(1, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed=0)
+    upd = w.seqlen * w.dim * w.dstate
+    times = []
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.real(inp["x"], inp["delta_raw"], inp["A_log"], inp["Bm"], inp["Cm"], inp["Dskip"],
+                    inp["dy"], chunk=w.chunk, threads=threads)
+        dt = time.perf_counter() - t0
+        if k >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = upd * len(times) / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
+                       "sample": "one batch row per step", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"1 of {w.batch} batch rows of {w.name} per step, float64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from selective_state_space_bwd_b200 import inputs as gen
+    w = gen.WORKLOADS[args.workload]
+    if isinstance(w, gen.ComplexWorkload):
+        raise SystemExit("bench.py times the real-mode workloads")
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_bwd_b200 import build, ssm_scan as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    S.lib()
+
+    dt = torch.bfloat16 if w.io == gen.BF16 else torch.float32
+    inp = gen.real_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed=rank)
+    host = {k: torch.from_numpy(v).to(dt if k not in ("A_log", "Dskip") else torch.float32)
+            for k, v in inp.items()}
+    host = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    shape = S.real_shape(w.batch, w.seqlen, w.dim, w.dstate, w.chunk,
+                         S.SSM_BF16 if w.io == gen.BF16 else S.SSM_F32, args.seg_chunks)
+    nC = -(-w.seqlen // w.chunk)
+    y = torch.empty_like(d["x"])
+    ckpt = torch.empty((w.batch, nC, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    out = dict(dx=torch.empty_like(d["x"]), ddelta_raw=torch.empty_like(d["x"]),
+               dA_log=torch.empty_like(d["A_log"]), dB=torch.empty_like(d["Bm"]),
+               dC=torch.empty_like(d["Cm"]), dD=torch.empty_like(d["Dskip"]))
+    wsf = torch.empty(S.workspace_bytes(shape, False), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(S.workspace_bytes(shape, True), dtype=torch.uint8, device=dev)
+    gbuf = torch.empty(w.dim * w.dstate + w.dim, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        S.ssm_scan_fwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
+                       chunk=w.chunk, seg_chunks=args.seg_chunks, y=y, ckpt=ckpt, ws=wsf,
+                       stream=stream)
+
+    def bwd():
+        S.ssm_scan_bwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"], ckpt,
+                       d["dy"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
+                       stream=stream)
+
+    def allreduce():
+        if world > 1:
+            gbuf[: w.dim * w.dstate].copy_(out["dA_log"].view(-1))
+            gbuf[w.dim * w.dstate:].copy_(out["dD"])
+            dist.all_reduce(gbuf)
+
+    for _ in range(max(3, args.warmup)):
+        fwd(); bwd(); allreduce()
+    torch.cuda.synchronize()
+    if S.ssm_scan_status(wsb) != 0 or S.ssm_scan_status(wsf) != 0:
+        raise SystemExit("device status word reports a non-finite state")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream); fwd(); e[1].record(stream); bwd(); e[2].record(stream)
+        allreduce(); e[3].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / 1e3
+    tt = torch.tensor([t_step, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    t_step, t_fwd, t_bwd = tt.tolist()
+
+    # end to end: host inputs in, every output back, inside the timed region
+    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = hy.numel() * hy.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+
+    def e2e_step():
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        fwd(); bwd(); allreduce()
+        hy.copy_(y, non_blocking=True)
+        for k, v in out.items():
+            hout[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    t_e2e = float(t_e2e)
+
+    upd_rank = w.batch * w.seqlen * w.dim * w.dstate
+    value = world * upd_rank * args.steps / t_step
+    hbm, peak_kind = peaks()
+    fb, bb = algorithmic_bytes(w)
+    launches = (S.kernel_launches(shape, False) + S.kernel_launches(shape, True)) * args.steps
+    bwd_gbs = bb / (t_bwd / args.steps) / 1e9
+    fwd_gbs = fb / (t_fwd / args.steps) / 1e9
+    step_gbs = (fb + bb) / ((t_fwd + t_bwd) / args.steps) / 1e9
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.io == gen.BF16 else "f32",
+            "data": "synthetic (seeded generator, workload value distributions)",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
+                       "state": "fp32", "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (weak: one full batch per rank; "
+                                      "dA_log/dD all-reduced)" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": "ssm_scan_bwd (chunk-recompute adjoint + "
+                         "fixed-order reductions)", "achieved": bwd_gbs, "peak": hbm,
+                         "unit": "GB/s", "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+            "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_step": step_gbs / hbm,
+            "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
+            "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_sample(w, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * ssm_scan.h — C ABI of the B200 selective diagonal state-space scan and its exact gradient.
+ *
+ * What the calls compute
+ * ----------------------
+ * Real mode (the selective SSM of "选择性状态空间模型(S3M)原理与工程实践" §1.1: step size
+ * delta = softplus(projection), decay A = -exp(log_A), transition exp(A·delta); input term taken
+ * as the Euler form delta·B_t·x_t), per batch b and channel d, for states n = 0..N-1:
+ *
+ *     delta_t = softplus(delta_raw_t)          A_n = -exp(A_log[d,n])
+ *     h_t,n   = exp(delta_t A_n) h_{t-1,n} + delta_t Bm_t,n x_t          h_{-1} = 0
+ *     y_t     = sum_n Cm_t,n h_t,n + Dskip[d] x_t
+ *
+ * ssm_scan_bwd returns the exact gradient of sum(dy·y) by a reverse-time adjoint scan ("Breaking
+ * the Memory Wall: Exact Analytical Differentiation via Tiled Operator-Space Evolution", abstract:
+ * exact analytical derivatives without materialising the graph; tiled operator-space evolution).
+ * Only the state at the end of every chunk of T steps is stored (the checkpoint buffer, O(L/T));
+ * the backward recomputes each chunk from its checkpoint.  The time-parallel structure (local scan
+ * of a chunk, carry across chunks, correction) follows the three-phase scan described for Flash
+ * PD-SSM ("Flash PD-SSM", technical summary, hardware-aware implementation, phases A–C).
+ *
+ * Complex mode ("SPARC: Shared Phase and Retention Control for Efficient Adaptive Spectral
+ * Recurrence", abstract: two shared input-dependent scalars drive every complex mode, each mode
+ * keeps its own timescale and frequency; diagonal affine recurrence), per batch b and mode k:
+ *
+ *     s_t = softplus(r_t)      a_t,k = exp(-lambda_k s_t + i omega_k phi_t)
+ *     h_t,k = a_t,k h_{t-1,k} + u_t,k                                   h_{-1} = 0
+ *
+ * and ssm_scan_complex_bwd returns the gradient of Re sum conj(g)·h with respect to u (complex,
+ * as d/dRe + i d/dIm), r, phi, lambda and omega.
+ *
+ * Conventions (all calls)
+ * -----------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller, except the shape structs,
+ *   which are host pointers read during the call only.  The library allocates no memory and
+ *   keeps no state between calls; calls on different streams with different buffers may overlap.
+ * - Arrays are dense row-major (C order), no strides.  Every array pointer must be 16-byte
+ *   aligned (SSM_ERR_MISALIGNED otherwise).
+ * - Calls enqueue kernels on `stream` and return without synchronising.  Argument errors are
+ *   detected on the host before anything is enqueued (nothing is written).  A failed launch
+ *   returns SSM_ERR_CUDA.  Conditions found on the device (non-finite state) are recorded in a
+ *   status word at the start of the workspace; ssm_scan_status() reads it.  Each fwd/bwd call
+ *   resets that word when it starts.
+ * - Gradients overwrite their outputs (they do not accumulate).  All outputs are deterministic:
+ *   the same inputs give bitwise the same outputs on every run (no floating-point atomics).
+ * - Workspace: a caller-owned device buffer of at least ssm_scan_*_workspace_bytes() bytes,
+ *   used as scratch by one call at a time (do not share one workspace between overlapping calls).
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_SCAN_ABI_VERSION 1
+
+/* Same underlying type as cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st* ssm_stream_t;
+
+typedef enum ssm_status {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,          /* null pointer, negative size, reserved field not zero */
+    SSM_ERR_UNSUPPORTED = 2,          /* dstate not in {4,8,16}, chunk not in {16..256}, bad io */
+    SSM_ERR_MISALIGNED = 3,           /* pointer not 16-byte aligned, or dim*sizeof(io) % 16 != 0 */
+    SSM_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the size query's answer */
+    SSM_ERR_CUDA = 5,                 /* a kernel launch or CUDA runtime call failed */
+    SSM_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (reserved) */
+    SSM_ERR_NONFINITE = 7             /* a NaN or Inf reached a carried state (device-side) */
+} ssm_status;
+
+typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+/* Real-mode problem size. */
+typedef struct ssm_shape {
+    int64_t batch;      /* B >= 0 */
+    int64_t seqlen;     /* L >= 0 (0 is a valid empty problem) */
+    int64_t dim;        /* D >= 1; D * sizeof(io) must be a multiple of 16 bytes */
+    int64_t dstate;     /* N, one of 4, 8, 16 */
+    int32_t chunk;      /* T, one of 16, 32, 64, 128, 256: checkpoint spacing in steps */
+    int32_t io;         /* ssm_dtype of x, delta_raw, Bm, Cm, y, dy, dx, ddelta_raw, dB, dC */
+    int32_t seg_chunks; /* time-parallel split, in chunks per segment; 0 = automatic.  A tuning
+                           knob only: results agree to rounding for every value. */
+    int32_t reserved;   /* must be 0 */
+} ssm_shape;
+
+/* Complex-mode problem size. */
+typedef struct ssm_cshape {
+    int64_t batch;      /* B >= 0 */
+    int64_t seqlen;     /* L >= 0 */
+    int64_t modes;      /* K >= 1, even */
+    int32_t chunk;      /* time-split granularity in steps, one of 16..256 */
+    int32_t seg_chunks; /* chunks per time segment; 0 = automatic (tuning knob only) */
+} ssm_cshape;
+
+/* ABI version of the loaded library (SSM_SCAN_ABI_VERSION at build time). */
+int ssm_scan_abi_version(void);
+
+/* Bytes of the checkpoint buffer: B * ceil(L/T) * D * N * sizeof(float).  Layout
+ * [B, ceil(L/T), D, N] fp32; entry c holds h at the last step of chunk c (step min((c+1)T, L)-1).
+ * Returns 0 for an invalid shape. */
+size_t ssm_scan_checkpoint_bytes(const ssm_shape* shape);
+
+/* Workspace bytes for ssm_scan_fwd (backward == 0) or ssm_scan_bwd (backward != 0); at least
+ * 256.  Returns 0 for an invalid shape. */
+size_t ssm_scan_workspace_bytes(const ssm_shape* shape, int backward);
+
+/*
+ * Forward scan.
+ *   x, delta_raw  [B, L, D]  io dtype           Bm, Cm  [B, L, N]  io dtype
+ *   A_log         [D, N]     fp32               Dskip   [D]        fp32
+ * Outputs:
+ *   y             [B, L, D]  io dtype
+ *   ckpt          [B, ceil(L/T), D, N] fp32 (ssm_scan_checkpoint_bytes); keep it for the backward
+ * Returns an ssm_status.
+ */
+int ssm_scan_fwd(const ssm_shape* shape,
+                 const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip,
+                 void* y, float* ckpt,
+                 void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/*
+ * Backward: exact gradient of sum(dy * y) for the forward above.
+ *   inputs as for ssm_scan_fwd, plus ckpt (written by ssm_scan_fwd on the same inputs) and
+ *   dy [B, L, D] io dtype.
+ * Outputs (overwritten):
+ *   dx, ddelta_raw [B, L, D] io dtype;   dB, dC [B, L, N] io dtype;
+ *   dA_log [D, N] fp32;                  dD [D] fp32.
+ * Returns an ssm_status.
+ */
+int ssm_scan_bwd(const ssm_shape* shape,
+                 const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip,
+                 const float* ckpt, const void* dy,
+                 void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC, float* dD,
+                 void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/* Workspace bytes for the complex calls (at least 256); 0 for an invalid shape. */
+size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward);
+
+/*
+ * Complex forward.
+ *   u       [B, L, K] complex64 (interleaved re, im fp32)
+ *   r, phi  [B, L] fp32          lambda, omega [K] fp32
+ * Output:
+ *   h       [B, L, K] complex64: the whole state trajectory (the output of this mode)
+ */
+int ssm_scan_complex_fwd(const ssm_cshape* shape,
+                         const void* u, const float* r, const float* phi,
+                         const float* lambda, const float* omega,
+                         void* h, void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/*
+ * Complex backward: gradient of Re sum conj(g)·h.
+ *   h       [B, L, K] complex64, the trajectory written by ssm_scan_complex_fwd.  Because the
+ *           trajectory is this mode's output it is already resident, so the backward reads it
+ *           (h_{t-1} at step t) instead of recomputing it.
+ *   r, phi, lambda, omega as for the forward;  g [B, L, K] complex64 (dLoss/dh).
+ * Outputs (overwritten):
+ *   du [B, L, K] complex64;  dr, dphi [B, L] fp32;  dlambda, domega [K] fp32.
+ */
+int ssm_scan_complex_bwd(const ssm_cshape* shape,
+                         const void* h, const float* r, const float* phi,
+                         const float* lambda, const float* omega, const void* g,
+                         void* du, float* dr, float* dphi, float* dlambda, float* domega,
+                         void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
+ * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */
+int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);
+
+/* Same for the complex calls. */
+int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward);
+
+/* Waits for `stream`, then returns the status word the last call on `ws` left (SSM_OK,
+ * SSM_ERR_NONFINITE or SSM_ERR_TIMEOUT), or SSM_ERR_CUDA if the copy itself fails. */
+int ssm_scan_status(const void* ws, ssm_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* ssm_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

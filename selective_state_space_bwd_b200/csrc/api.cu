@@ -1,0 +1,321 @@
+// C-ABI entry points (include/ssm_scan.h): argument validation on the host, workspace layout,
+// kernel launches.  Nothing here allocates memory or keeps state between calls.
+#include "../../include/ssm_scan.h"
+#include "ssm_internal.h"
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr int kTargetCtas = 296;  // 2 x 148 SMs: below this many CTAs, split time into segments
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool valid_chunk(int T) { return T == 16 || T == 32 || T == 64 || T == 128 || T == 256; }
+
+int pick_segments(int64_t ctas_per_seg, int nC, int forced, int* seg_chunks) {
+    if (nC <= 0) {
+        *seg_chunks = 1;
+        return 1;
+    }
+    int sc;
+    if (forced > 0) {
+        sc = forced < nC ? forced : nC;
+    } else {
+        int64_t nseg = 1;
+        if (ctas_per_seg < kTargetCtas) nseg = (kTargetCtas + ctas_per_seg - 1) / ctas_per_seg;
+        if (nseg > nC) nseg = nC;
+        sc = (int)((nC + nseg - 1) / nseg);
+    }
+    *seg_chunks = sc;
+    return (nC + sc - 1) / sc;
+}
+
+struct RealPlan {
+    int B, L, D, N, T, nC, ndt, seg_chunks, nseg, esz;
+    // workspace offsets (bytes); fwd and bwd use separate layouts
+    size_t f_sumP, f_sumS, f_hin, f_end;
+    size_t b_gP, b_gG, b_vin, b_part, b_dA, b_dD, b_end;
+};
+
+int plan_real(const ssm_shape* s, RealPlan* p) {
+    if (!s) return SSM_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->dim < 1 || s->reserved != 0 || s->seg_chunks < 0)
+        return SSM_ERR_INVALID_ARG;
+    if (s->dstate != 4 && s->dstate != 8 && s->dstate != 16) return SSM_ERR_UNSUPPORTED;
+    if (!valid_chunk(s->chunk)) return SSM_ERR_UNSUPPORTED;
+    if (s->io != SSM_F32 && s->io != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    // index arithmetic inside the kernels is 32-bit for per-row offsets and grid sizes
+    if (s->batch > 65535 || s->seqlen > (int64_t)1 << 30 || s->dim > (int64_t)1 << 24)
+        return SSM_ERR_UNSUPPORTED;
+    p->esz = s->io == SSM_BF16 ? 2 : 4;
+    if ((s->dim * p->esz) % 16 != 0) return SSM_ERR_MISALIGNED;
+    p->B = (int)s->batch;
+    p->L = (int)s->seqlen;
+    p->D = (int)s->dim;
+    p->N = (int)s->dstate;
+    p->T = s->chunk;
+    p->nC = (p->L + p->T - 1) / p->T;
+    const int DT = ssm::real_dt(p->N);
+    p->ndt = (p->D + DT - 1) / DT;
+    p->nseg = pick_segments((int64_t)p->B * p->ndt, p->nC, s->seg_chunks, &p->seg_chunks);
+    if (p->nseg > 65535) return SSM_ERR_UNSUPPORTED;
+
+    const size_t B = p->B, DN = (size_t)p->D * p->N, S = p->nseg;
+    size_t o = kStatusBytes;
+    const size_t summ = S > 1 ? B * (S - 1) * DN * 4 : 0;
+    p->f_sumP = o; o = align256(o + summ);
+    p->f_sumS = o; o = align256(o + summ);
+    p->f_hin = o;  o = align256(o + (S > 1 ? B * S * DN * 4 : 0));
+    p->f_end = o;
+    o = kStatusBytes;
+    p->b_gP = o;   o = align256(o + summ);
+    p->b_gG = o;   o = align256(o + summ);
+    p->b_vin = o;  o = align256(o + (S > 1 ? B * S * DN * 4 : 0));
+    p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->L * 2 * p->N * 4);
+    p->b_dA = o;   o = align256(o + B * S * DN * 4);
+    p->b_dD = o;   o = align256(o + B * S * (size_t)p->D * 4);
+    p->b_end = o;
+    return SSM_OK;
+}
+
+struct CplxPlan {
+    int B, L, K, T, nC, nkt, seg_chunks, nseg;
+    size_t f_sumP, f_sumS, f_hin, f_end;
+    size_t b_gP, b_gG, b_win, b_rp, b_lo, b_end;
+};
+
+int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
+    if (!s) return SSM_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->modes < 1 || s->seg_chunks < 0)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_chunk(s->chunk)) return SSM_ERR_UNSUPPORTED;
+    if (s->batch > 65535 || s->seqlen > (int64_t)1 << 30 || s->modes > (int64_t)1 << 26)
+        return SSM_ERR_UNSUPPORTED;
+    if (s->modes % 2 != 0) return SSM_ERR_MISALIGNED;
+    p->B = (int)s->batch;
+    p->L = (int)s->seqlen;
+    p->K = (int)s->modes;
+    p->T = s->chunk;
+    p->nC = (p->L + p->T - 1) / p->T;
+    p->nkt = (p->K + ssm::kCplxKT - 1) / ssm::kCplxKT;
+    p->nseg = pick_segments((int64_t)p->B * p->nkt, p->nC, s->seg_chunks, &p->seg_chunks);
+    if (p->nseg > 65535) return SSM_ERR_UNSUPPORTED;
+    const size_t B = p->B, K = p->K, S = p->nseg;
+    const size_t summ = S > 1 ? B * (S - 1) * K * 8 : 0;
+    size_t o = kStatusBytes;
+    p->f_sumP = o; o = align256(o + summ);
+    p->f_sumS = o; o = align256(o + summ);
+    p->f_hin = o;  o = align256(o + (S > 1 ? B * S * K * 8 : 0));
+    p->f_end = o;
+    o = kStatusBytes;
+    p->b_gP = o;  o = align256(o + summ);
+    p->b_gG = o;  o = align256(o + summ);
+    p->b_win = o; o = align256(o + (S > 1 ? B * S * K * 8 : 0));
+    p->b_rp = o;  o = align256(o + (size_t)p->nkt * B * (size_t)p->L * 8);
+    p->b_lo = o;  o = align256(o + B * S * K * 8);
+    p->b_end = o;
+    return SSM_OK;
+}
+
+// A pointer may be null only when the array it describes is empty.
+bool ptr_ok(const void* ptr, size_t count) { return count == 0 || ptr != nullptr; }
+
+int check_arrays(const void* const* ptrs, const size_t* counts, int n) {
+    for (int i = 0; i < n; ++i) {
+        if (!ptr_ok(ptrs[i], counts[i])) return SSM_ERR_INVALID_ARG;
+        if (counts[i] && !aligned16(ptrs[i])) return SSM_ERR_MISALIGNED;
+    }
+    return SSM_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_scan_abi_version(void) { return SSM_SCAN_ABI_VERSION; }
+
+size_t ssm_scan_checkpoint_bytes(const ssm_shape* shape) {
+    RealPlan p;
+    if (plan_real(shape, &p) != SSM_OK) return 0;
+    return (size_t)p.B * p.nC * p.D * p.N * sizeof(float);
+}
+
+size_t ssm_scan_workspace_bytes(const ssm_shape* shape, int backward) {
+    RealPlan p;
+    if (plan_real(shape, &p) != SSM_OK) return 0;
+    return backward ? p.b_end : p.f_end;
+}
+
+int ssm_scan_fwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip, void* y, float* ckpt, void* ws,
+                 size_t ws_bytes, ssm_stream_t stream) {
+    RealPlan p;
+    int st = plan_real(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLD = (size_t)p.B * p.L * p.D, BLN = (size_t)p.B * p.L * p.N;
+    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN;
+    const void* ptrs[] = {x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt, ws};
+    const size_t counts[] = {BLD, BLD, DN, BLN, BLN, (size_t)p.D, BLD, ck, 1};
+    if ((st = check_arrays(ptrs, counts, 9)) != SSM_OK) return st;
+    if (ws_bytes < p.f_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) return SSM_OK;
+    ssm::RealArgs a = {};
+    a.B = p.B; a.L = p.L; a.D = p.D; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.ndt = p.ndt;
+    a.x = x; a.draw = delta_raw; a.A_log = A_log; a.Bm = Bm; a.Cm = Cm; a.Dskip = Dskip;
+    a.y = y; a.ckpt = ckpt;
+    a.sumP = at<float>(ws, p.f_sumP); a.sumS = at<float>(ws, p.f_sumS); a.hin = at<float>(ws, p.f_hin);
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_real_fwd(a, shape->io == SSM_BF16, p.N, s) == cudaSuccess ? SSM_OK
+                                                                                : SSM_ERR_CUDA;
+}
+
+int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip, const float* ckpt,
+                 const void* dy, void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC,
+                 float* dD, void* ws, size_t ws_bytes, ssm_stream_t stream) {
+    RealPlan p;
+    int st = plan_real(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLD = (size_t)p.B * p.L * p.D, BLN = (size_t)p.B * p.L * p.N;
+    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN;
+    const void* ptrs[] = {x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy,
+                          dx, ddelta_raw, dA_log, dB, dC, dD, ws};
+    const size_t counts[] = {BLD, BLD, DN, BLN, BLN, (size_t)p.D, ck, BLD,
+                             BLD, BLD, DN, BLN, BLN, (size_t)p.D, 1};
+    if ((st = check_arrays(ptrs, counts, 15)) != SSM_OK) return st;
+    if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) {
+        if (cudaMemsetAsync(dA_log, 0, DN * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (cudaMemsetAsync(dD, 0, (size_t)p.D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::RealArgs a = {};
+    a.B = p.B; a.L = p.L; a.D = p.D; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.ndt = p.ndt;
+    a.x = x; a.draw = delta_raw; a.A_log = A_log; a.Bm = Bm; a.Cm = Cm; a.Dskip = Dskip;
+    a.ckpt_in = ckpt; a.dy = dy; a.dx = dx; a.ddraw = ddelta_raw;
+    a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.vin = at<float>(ws, p.b_vin);
+    a.dBC_part = at<float>(ws, p.b_part); a.dA_part = at<float>(ws, p.b_dA);
+    a.dD_part = at<float>(ws, p.b_dD);
+    a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_real_bwd(a, shape->io == SSM_BF16, p.N, s) == cudaSuccess ? SSM_OK
+                                                                                : SSM_ERR_CUDA;
+}
+
+int ssm_scan_kernel_launches(const ssm_shape* shape, int backward) {
+    RealPlan p;
+    if (plan_real(shape, &p) != SSM_OK) return -1;
+    if (p.B == 0 || p.L == 0) return 0;
+    const int seg = p.nseg > 1 ? 2 : 0;  // segment summary + carry
+    return backward ? 3 + seg : 1 + seg;  // bwd: main + dB/dC reduce + dA_log/dD reduce
+}
+
+int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward) {
+    CplxPlan p;
+    if (plan_cplx(shape, &p) != SSM_OK) return -1;
+    if (p.B == 0 || p.L == 0) return 0;
+    const int seg = p.nseg > 1 ? 2 : 0;
+    return backward ? 3 + seg : 1 + seg;
+}
+
+size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward) {
+    CplxPlan p;
+    if (plan_cplx(shape, &p) != SSM_OK) return 0;
+    return backward ? p.b_end : p.f_end;
+}
+
+int ssm_scan_complex_fwd(const ssm_cshape* shape, const void* u, const float* r, const float* phi,
+                         const float* lambda, const float* omega, void* h, void* ws,
+                         size_t ws_bytes, ssm_stream_t stream) {
+    CplxPlan p;
+    int st = plan_cplx(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLK = (size_t)p.B * p.L * p.K, BL = (size_t)p.B * p.L;
+    const void* ptrs[] = {u, r, phi, lambda, omega, h, ws};
+    const size_t counts[] = {BLK, BL, BL, (size_t)p.K, (size_t)p.K, BLK, 1};
+    if ((st = check_arrays(ptrs, counts, 7)) != SSM_OK) return st;
+    if (ws_bytes < p.f_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) return SSM_OK;
+    ssm::CplxArgs a = {};
+    a.B = p.B; a.L = p.L; a.K = p.K; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.nkt = p.nkt;
+    a.u = static_cast<const float*>(u); a.r = r; a.phi = phi; a.lam = lambda; a.om = omega;
+    a.h = static_cast<float*>(h);
+    a.sumP = at<float>(ws, p.f_sumP); a.sumS = at<float>(ws, p.f_sumS); a.hin = at<float>(ws, p.f_hin);
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_cplx_fwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_scan_complex_bwd(const ssm_cshape* shape, const void* h, const float* r, const float* phi,
+                         const float* lambda, const float* omega, const void* g, void* du,
+                         float* dr, float* dphi, float* dlambda, float* domega, void* ws,
+                         size_t ws_bytes, ssm_stream_t stream) {
+    CplxPlan p;
+    int st = plan_cplx(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLK = (size_t)p.B * p.L * p.K, BL = (size_t)p.B * p.L, K = p.K;
+    const void* ptrs[] = {h, r, phi, lambda, omega, g, du, dr, dphi, dlambda, domega, ws};
+    const size_t counts[] = {BLK, BL, BL, K, K, BLK, BLK, BL, BL, K, K, 1};
+    if ((st = check_arrays(ptrs, counts, 12)) != SSM_OK) return st;
+    if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) {
+        if (cudaMemsetAsync(dlambda, 0, K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (cudaMemsetAsync(domega, 0, K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::CplxArgs a = {};
+    a.B = p.B; a.L = p.L; a.K = p.K; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.nkt = p.nkt;
+    a.r = r; a.phi = phi; a.lam = lambda; a.om = omega;
+    a.h_in = static_cast<const float*>(h); a.g = static_cast<const float*>(g);
+    a.du = static_cast<float*>(du); a.dr = dr; a.dphi = dphi; a.dlam = dlambda; a.dom = domega;
+    a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.win = at<float>(ws, p.b_win);
+    a.rp_part = at<float>(ws, p.b_rp); a.lo_part = at<float>(ws, p.b_lo);
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_cplx_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_scan_status(const void* ws, ssm_stream_t stream) {
+    if (!ws) return SSM_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SSM_ERR_CUDA;
+    return (int)v;
+}
+
+const char* ssm_status_string(int status) {
+    switch (status) {
+        case SSM_OK: return "SSM_OK";
+        case SSM_ERR_INVALID_ARG: return "SSM_ERR_INVALID_ARG: null pointer, negative size or nonzero reserved field";
+        case SSM_ERR_UNSUPPORTED: return "SSM_ERR_UNSUPPORTED: dstate, chunk, io dtype or size outside the supported set";
+        case SSM_ERR_MISALIGNED: return "SSM_ERR_MISALIGNED: pointer not 16-byte aligned or row not a multiple of 16 bytes";
+        case SSM_ERR_WORKSPACE_TOO_SMALL: return "SSM_ERR_WORKSPACE_TOO_SMALL: workspace below the size query's answer";
+        case SSM_ERR_CUDA: return "SSM_ERR_CUDA: a CUDA launch or runtime call failed";
+        case SSM_ERR_TIMEOUT: return "SSM_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case SSM_ERR_NONFINITE: return "SSM_ERR_NONFINITE: a NaN or Inf reached a carried state";
+        default: return "unknown ssm_status";
+    }
+}
+
+}  // extern "C"

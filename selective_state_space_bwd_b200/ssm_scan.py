@@ -1,0 +1,230 @@
+"""ctypes binding of libssm_scan.so (include/ssm_scan.h), over torch device tensors.
+
+Argument marshalling only: every step of the scan runs in the library's CUDA kernels.  If the
+library is missing, or the tensors are not on a CUDA device, the calls raise — there is no CPU
+fallback.  Names mirror the C ABI: ``ssm_scan_fwd``, ``ssm_scan_bwd``, ``ssm_scan_complex_fwd``,
+``ssm_scan_complex_bwd``, ``ssm_scan_status``; the workspace / checkpoint size queries are exposed
+as ``workspace_bytes`` and friends.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
+
+SSM_OK = 0
+SSM_F32, SSM_BF16 = 0, 1
+STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
+                3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_WORKSPACE_TOO_SMALL", 5: "SSM_ERR_CUDA",
+                6: "SSM_ERR_TIMEOUT", 7: "SSM_ERR_NONFINITE"}
+
+
+class SsmShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("chunk", ctypes.c_int32), ("io", ctypes.c_int32),
+                ("seg_chunks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class SsmCShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("modes", ctypes.c_int64),
+                ("chunk", ctypes.c_int32), ("seg_chunks", ctypes.c_int32)]
+
+
+class SsmError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_workspace_bytes",
+            "ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_complex_workspace_bytes",
+            "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
+            "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string"]
+
+
+def lib():
+    """Open libssm_scan.so (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m selective_state_space_bwd_b200.build` (no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            P, Z, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+            SP, CP = ctypes.POINTER(SsmShape), ctypes.POINTER(SsmCShape)
+            L.ssm_scan_abi_version.argtypes, L.ssm_scan_abi_version.restype = [], I
+            L.ssm_scan_checkpoint_bytes.argtypes, L.ssm_scan_checkpoint_bytes.restype = [SP], Z
+            L.ssm_scan_workspace_bytes.argtypes, L.ssm_scan_workspace_bytes.restype = [SP, I], Z
+            L.ssm_scan_fwd.argtypes = [SP] + [P] * 9 + [Z, P]
+            L.ssm_scan_fwd.restype = I
+            L.ssm_scan_bwd.argtypes = [SP] + [P] * 15 + [Z, P]
+            L.ssm_scan_bwd.restype = I
+            L.ssm_scan_complex_workspace_bytes.argtypes = [CP, I]
+            L.ssm_scan_complex_workspace_bytes.restype = Z
+            L.ssm_scan_complex_fwd.argtypes = [CP] + [P] * 7 + [Z, P]
+            L.ssm_scan_complex_fwd.restype = I
+            L.ssm_scan_complex_bwd.argtypes = [CP] + [P] * 12 + [Z, P]
+            L.ssm_scan_complex_bwd.restype = I
+            L.ssm_scan_kernel_launches.argtypes = [SP, I]
+            L.ssm_scan_kernel_launches.restype = I
+            L.ssm_scan_complex_kernel_launches.argtypes = [CP, I]
+            L.ssm_scan_complex_kernel_launches.restype = I
+            L.ssm_scan_status.argtypes, L.ssm_scan_status.restype = [P, P], I
+            L.ssm_status_string.argtypes, L.ssm_status_string.restype = [I], ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def _check(code, what):
+    if code != SSM_OK:
+        raise SsmError(code, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("ssm_scan: every tensor must live on a CUDA device")
+
+
+def real_shape(batch, seqlen, dim, dstate, chunk=128, io=SSM_F32, seg_chunks=0):
+    return SsmShape(int(batch), int(seqlen), int(dim), int(dstate), int(chunk), int(io),
+                    int(seg_chunks), 0)
+
+
+def complex_shape(batch, seqlen, modes, chunk=128, seg_chunks=0):
+    return SsmCShape(int(batch), int(seqlen), int(modes), int(chunk), int(seg_chunks))
+
+
+def checkpoint_bytes(shape: SsmShape) -> int:
+    return int(lib().ssm_scan_checkpoint_bytes(ctypes.byref(shape)))
+
+
+def workspace_bytes(shape: SsmShape, backward: bool) -> int:
+    return int(lib().ssm_scan_workspace_bytes(ctypes.byref(shape), int(bool(backward))))
+
+
+def complex_workspace_bytes(shape: SsmCShape, backward: bool) -> int:
+    return int(lib().ssm_scan_complex_workspace_bytes(ctypes.byref(shape), int(bool(backward))))
+
+
+def kernel_launches(shape: SsmShape, backward: bool) -> int:
+    return int(lib().ssm_scan_kernel_launches(ctypes.byref(shape), int(bool(backward))))
+
+
+def complex_kernel_launches(shape: SsmCShape, backward: bool) -> int:
+    return int(lib().ssm_scan_complex_kernel_launches(ctypes.byref(shape), int(bool(backward))))
+
+
+def _io_of(t):
+    if t.dtype == torch.float32:
+        return SSM_F32
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    raise ValueError(f"unsupported io dtype {t.dtype}")
+
+
+def _workspace(nbytes, device, ws):
+    if ws is not None:
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def ssm_scan_fwd(x, delta_raw, A_log, Bm, Cm, Dskip, chunk=128, seg_chunks=0, y=None, ckpt=None,
+                 ws=None, stream=None):
+    """Forward scan.  x, delta_raw [B,L,D] and Bm, Cm [B,L,N] share one io dtype (fp32 / bf16);
+    A_log [D,N], Dskip [D] fp32.  Returns (y [B,L,D], ckpt [B,ceil(L/T),D,N] fp32)."""
+    _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip)
+    B, L, D = x.shape
+    N = A_log.shape[1]
+    shape = real_shape(B, L, D, N, chunk, _io_of(x), seg_chunks)
+    if y is None:
+        y = torch.empty_like(x)
+    nC = -(-L // chunk)
+    if ckpt is None:
+        ckpt = torch.empty((B, nC, D, N), dtype=torch.float32, device=x.device)
+    ws = _workspace(workspace_bytes(shape, False), x.device, ws)
+    code = lib().ssm_scan_fwd(ctypes.byref(shape), _p(x), _p(delta_raw), _p(A_log), _p(Bm), _p(Cm),
+                              _p(Dskip), _p(y), _p(ckpt), _p(ws), ws.numel() * ws.element_size(),
+                              _stream(stream))
+    _check(code, "ssm_scan_fwd")
+    return y, ckpt
+
+
+def ssm_scan_bwd(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, chunk=128, seg_chunks=0, out=None,
+                 ws=None, stream=None):
+    """Backward.  Returns dict dx, ddelta_raw [B,L,D], dA_log [D,N], dB, dC [B,L,N], dD [D]."""
+    _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy)
+    B, L, D = x.shape
+    N = A_log.shape[1]
+    shape = real_shape(B, L, D, N, chunk, _io_of(x), seg_chunks)
+    if out is None:
+        out = dict(dx=torch.empty_like(x), ddelta_raw=torch.empty_like(x),
+                   dA_log=torch.empty_like(A_log), dB=torch.empty_like(Bm), dC=torch.empty_like(Cm),
+                   dD=torch.empty_like(Dskip))
+    ws = _workspace(workspace_bytes(shape, True), x.device, ws)
+    code = lib().ssm_scan_bwd(ctypes.byref(shape), _p(x), _p(delta_raw), _p(A_log), _p(Bm), _p(Cm),
+                              _p(Dskip), _p(ckpt), _p(dy), _p(out["dx"]), _p(out["ddelta_raw"]),
+                              _p(out["dA_log"]), _p(out["dB"]), _p(out["dC"]), _p(out["dD"]),
+                              _p(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_scan_bwd")
+    return out
+
+
+def ssm_scan_complex_fwd(u, r, phi, lam, omega, chunk=128, seg_chunks=0, h=None, ws=None,
+                         stream=None):
+    """Complex forward.  u [B,L,K] complex64; r, phi [B,L]; lam, omega [K].  Returns h."""
+    _need_cuda(u, r, phi, lam, omega)
+    if u.dtype != torch.complex64:
+        raise ValueError("u must be complex64")
+    B, L, K = u.shape
+    shape = complex_shape(B, L, K, chunk, seg_chunks)
+    if h is None:
+        h = torch.empty_like(u)
+    ws = _workspace(complex_workspace_bytes(shape, False), u.device, ws)
+    code = lib().ssm_scan_complex_fwd(ctypes.byref(shape), _p(u), _p(r), _p(phi), _p(lam),
+                                      _p(omega), _p(h), _p(ws), ws.numel() * ws.element_size(),
+                                      _stream(stream))
+    _check(code, "ssm_scan_complex_fwd")
+    return h
+
+
+def ssm_scan_complex_bwd(h, r, phi, lam, omega, g, chunk=128, seg_chunks=0, out=None, ws=None,
+                         stream=None):
+    """Complex backward of Re sum conj(g) h.  Returns dict du, dr, dphi, dlambda, domega."""
+    _need_cuda(h, r, phi, lam, omega, g)
+    B, L, K = h.shape
+    shape = complex_shape(B, L, K, chunk, seg_chunks)
+    if out is None:
+        out = dict(du=torch.empty_like(g), dr=torch.empty_like(r), dphi=torch.empty_like(phi),
+                   dlambda=torch.empty_like(lam), domega=torch.empty_like(omega))
+    ws = _workspace(complex_workspace_bytes(shape, True), h.device, ws)
+    code = lib().ssm_scan_complex_bwd(ctypes.byref(shape), _p(h), _p(r), _p(phi), _p(lam),
+                                      _p(omega), _p(g), _p(out["du"]), _p(out["dr"]),
+                                      _p(out["dphi"]), _p(out["dlambda"]), _p(out["domega"]),
+                                      _p(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_scan_complex_bwd")
+    return out
+
+
+def ssm_scan_status(ws, stream=None) -> int:
+    """Synchronise the stream and return the device status word a call left in ``ws``."""
+    return int(lib().ssm_scan_status(_p(ws), _stream(stream)))

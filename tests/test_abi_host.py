@@ -1,0 +1,154 @@
+"""Host-side checks of the C ABI: the library builds for sm_100a, loads without a GPU, exports every
+function declared in include/ssm_scan.h, answers size queries by their documented formulas and
+rejects bad arguments with the documented status before touching the device.  No call here
+reaches a CUDA runtime function (every case fails validation first)."""
+
+import ctypes
+import os
+import re
+import shutil
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_scan.h")
+
+pytestmark = pytest.mark.skipif(shutil.which("nvcc") is None and not os.path.exists(
+    os.path.join(ROOT, "selective_state_space_bwd_b200", "libssm_scan.so")),
+    reason="needs nvcc or a prebuilt libssm_scan.so")
+
+
+@pytest.fixture(scope="module")
+def S():
+    from selective_state_space_bwd_b200 import build, ssm_scan
+    build.build()
+    ssm_scan.lib()
+    return ssm_scan
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(ssm_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(S):
+    names = _declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(S.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(S.EXPORTED)
+
+
+def test_abi_version_and_status_strings(S):
+    L = S.lib()
+    assert L.ssm_scan_abi_version() == 1
+    for code in range(8):
+        assert L.ssm_status_string(code).decode().startswith(S.STATUS_NAMES[code])
+    assert L.ssm_status_string(99) == b"unknown ssm_status"
+
+
+@pytest.mark.parametrize("B,L,D,N,T", [(1, 256, 4, 4, 128), (8, 2048, 1536, 16, 128),
+                                       (1, 128000, 1024, 16, 128), (3, 1000, 40, 8, 64),
+                                       (2, 0, 16, 16, 32)])
+def test_checkpoint_and_workspace_sizes(S, B, L, D, N, T):
+    shp = S.real_shape(B, L, D, N, T, S.SSM_F32)
+    nC = -(-L // T)
+    assert S.checkpoint_bytes(shp) == B * nC * D * N * 4
+    fw, bw = S.workspace_bytes(shp, False), S.workspace_bytes(shp, True)
+    assert fw >= 256 and bw >= 256 and fw % 256 == 0 and bw % 256 == 0
+    # backward workspace holds at least the per-channel-tile dB/dC partials
+    DT = 32
+    ndt = -(-D // DT)
+    assert bw >= ndt * B * L * 2 * N * 4
+
+
+def test_segment_knob_changes_only_workspace(S):
+    a = S.real_shape(1, 4096, 64, 16, 128, S.SSM_F32, seg_chunks=1)
+    b = S.real_shape(1, 4096, 64, 16, 128, S.SSM_F32, seg_chunks=32)
+    assert S.checkpoint_bytes(a) == S.checkpoint_bytes(b)
+    assert S.workspace_bytes(a, False) > S.workspace_bytes(b, False)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dstate", 12, 2), ("dstate", 32, 2), ("chunk", 100, 2), ("chunk", 512, 2), ("io", 3, 2),
+    ("batch", -1, 1), ("seqlen", -5, 1), ("dim", 0, 1), ("reserved", 1, 1), ("seg_chunks", -1, 1),
+    ("dim", 6, 3),  # 6 * 4 bytes is not a multiple of 16
+])
+def test_invalid_shapes_rejected(S, field, value, code):
+    shp = S.real_shape(2, 64, 16, 16, 32, S.SSM_F32)
+    setattr(shp, field, value)
+    L = S.lib()
+    assert L.ssm_scan_workspace_bytes(ctypes.byref(shp), 0) == 0
+    assert L.ssm_scan_checkpoint_bytes(ctypes.byref(shp)) == 0
+    fake = ctypes.c_void_p(0x10000)
+    rc = L.ssm_scan_fwd(ctypes.byref(shp), *([fake] * 9), 1 << 20, None)
+    assert rc == code
+
+
+def test_bf16_row_alignment(S):
+    L = S.lib()
+    ok = S.real_shape(1, 8, 8, 16, 16, S.SSM_BF16)       # 8 * 2 = 16 bytes
+    bad = S.real_shape(1, 8, 4, 16, 16, S.SSM_BF16)      # 4 * 2 = 8 bytes
+    assert L.ssm_scan_workspace_bytes(ctypes.byref(ok), 1) > 0
+    assert L.ssm_scan_workspace_bytes(ctypes.byref(bad), 1) == 0
+
+
+def _fake_ptrs(n, base=0x100000):
+    return [ctypes.c_void_p(base + 0x1000 * i) for i in range(n)]
+
+
+def test_null_misaligned_and_small_workspace(S):
+    L = S.lib()
+    shp = S.real_shape(2, 64, 16, 16, 32, S.SSM_F32)
+    need = S.workspace_bytes(shp, False)
+    p = _fake_ptrs(9)
+    q = list(p)
+    q[0] = None
+    assert L.ssm_scan_fwd(ctypes.byref(shp), *q, need, None) == 1
+    q = list(p)
+    q[3] = ctypes.c_void_p(0x100008)
+    assert L.ssm_scan_fwd(ctypes.byref(shp), *q, need, None) == 3
+    assert L.ssm_scan_fwd(ctypes.byref(shp), *p, need - 1, None) == 4
+    pb = _fake_ptrs(15)
+    needb = S.workspace_bytes(shp, True)
+    assert L.ssm_scan_bwd(ctypes.byref(shp), *pb, needb - 256, None) == 4
+    qb = list(pb)
+    qb[7] = None  # dy
+    assert L.ssm_scan_bwd(ctypes.byref(shp), *qb, needb, None) == 1
+
+
+def test_complex_validation(S):
+    L = S.lib()
+    shp = S.complex_shape(2, 64, 16, 32)
+    need_f = S.complex_workspace_bytes(shp, False)
+    need_b = S.complex_workspace_bytes(shp, True)
+    assert need_f >= 256 and need_b >= need_f
+    odd = S.complex_shape(2, 64, 15, 32)
+    assert S.complex_workspace_bytes(odd, True) == 0
+    badT = S.complex_shape(2, 64, 16, 48)
+    assert S.complex_workspace_bytes(badT, False) == 0
+    p = _fake_ptrs(7)
+    assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *p, need_f - 1, None) == 4
+    q = list(p)
+    q[1] = None
+    assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *q, need_f, None) == 1
+    pb = _fake_ptrs(12)
+    pb[5] = ctypes.c_void_p(0x100004)
+    assert L.ssm_scan_complex_bwd(ctypes.byref(shp), *pb, need_b, None) == 3
+
+
+def test_status_null_workspace(S):
+    assert S.lib().ssm_scan_status(None, None) == 1
+
+
+def test_kernel_launch_counts(S):
+    one = S.real_shape(8, 2048, 1536, 16, 128, S.SSM_BF16)        # enough CTAs: no time split
+    assert S.kernel_launches(one, False) == 1 and S.kernel_launches(one, True) == 3
+    split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)     # few CTAs: segment + carry
+    assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 5
+    assert S.kernel_launches(S.real_shape(2, 0, 32, 16, 128), True) == 0
+    assert S.kernel_launches(S.real_shape(2, 8, 32, 12, 128), True) == -1
+    assert S.complex_kernel_launches(S.complex_shape(16, 4096, 2048, 128), True) == 3
