@@ -39,7 +39,7 @@ struct RealPlan {
     int B, L, D, N, T, nC, ndt, seg_chunks, nseg, esz;
     // workspace offsets (bytes); fwd and bwd use separate layouts
     size_t f_sumP, f_sumS, f_hin, f_end;
-    size_t b_gP, b_gG, b_vin, b_part, b_dA, b_dD, b_end;
+    size_t b_gP, b_gG, b_vin, b_part, b_dA, b_dD, b_bnd, b_end;
 };
 
 int plan_real(const ssm_shape* s, RealPlan* p) {
@@ -79,6 +79,7 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->L * 2 * p->N * 4);
     p->b_dA = o;   o = align256(o + B * S * DN * 4);
     p->b_dD = o;   o = align256(o + B * S * (size_t)p->D * 4);
+    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * S * ssm::real_bnd_floats_per_cta(p->N) * 4);
     p->b_end = o;
     return SSM_OK;
 }
@@ -212,6 +213,7 @@ int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, c
     a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.vin = at<float>(ws, p.b_vin);
     a.dBC_part = at<float>(ws, p.b_part); a.dA_part = at<float>(ws, p.b_dA);
     a.dD_part = at<float>(ws, p.b_dD);
+    a.bnd_scratch = at<float>(ws, p.b_bnd);
     a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
     a.status = at<unsigned>(ws, 0);
     return ssm::launch_real_bwd(a, shape->io == SSM_BF16, p.N, s) == cudaSuccess ? SSM_OK

@@ -7,41 +7,114 @@
 // state at every chunk end is kept; each chunk is recomputed from its checkpoint and the exact
 // adjoint g_t = C_t dy_t + a_{t+1} g_{t+1} is swept backwards through it.
 //
-// Work decomposition.  Thread = (channel d, S consecutive states).  A CTA owns DT channels of one
-// batch row and one time segment (a run of whole chunks).  When a segment does not start at t=0
-// its entering state comes from a carry pass over per-segment summaries (prod a, local end state)
-// — the local-scan / carry / correction structure of the three-phase scan in "Flash PD-SSM"
-// (technical summary, hardware-aware implementation).  The backward mirrors it in reverse time.
+// Work decomposition.  Thread = (channel d, S consecutive states), arithmetic on state pairs with
+// the packed fp32x2 instructions; NG = N / S lanes (adjacent) cover a channel; a CTA covers 32
+// channels of one batch row and one time segment (a run of whole chunks).  Steps are processed in
+// groups of 4 so that the loads and exponentials of a group issue ahead of its dependent chain.
+// When a segment does not start at t = 0 its entering state comes from a carry pass over
+// per-segment summaries (prod a, local end state): the local-scan / carry / correction structure
+// of the three-phase scan in "Flash PD-SSM" (technical summary, hardware-aware implementation).
+// The backward mirrors it in reverse time.
 #include "ssm_device.cuh"
 #include "ssm_internal.h"
 
 namespace ssm {
 namespace {
 
-template <int N>
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int N, int S_>
 struct RealCfg {
-    static constexpr int S = kRealS;
-    static constexpr int NG = N / S;
-    static constexpr int DT = kRealDT;
-    static constexpr int NT = DT * NG;
-    static constexpr int TS = kRealTS;
+    static constexpr int S = S_;            // states per thread
+    static constexpr int P2 = S / 2;        // state pairs per thread
+    static constexpr int NG = N / S;        // lanes per channel
+    static constexpr int DT = kRealDT;      // channels per CTA
+    static constexpr int NT = DT * NG;      // threads per CTA
+    static constexpr int TS = S == 4 ? 8 : 4;  // backward window: steps of (a, a h_prev) in registers
+    static constexpr int U = 4;             // steps per unrolled group (= dB/dC flush period)
+    static constexpr int Q = NT / (2 * N);  // channel parts in the dB/dC column sums
+    static_assert(S == 4 || S == 8, "states per thread");
     static_assert(N % S == 0 && NG >= 1 && NG <= 4, "dstate must be 4, 8 or 16");
+    static_assert(Q >= 1 && (DT % Q) == 0, "column-sum split");
 };
 
-__device__ __forceinline__ bool all_finite4(const float* v) {
-    return isfinite(v[0]) && isfinite(v[1]) && isfinite(v[2]) && isfinite(v[3]);
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// exp2 of both halves on the MUFU unit
+__device__ __forceinline__ float2 ex2_pair(float2 e) { return make_float2(ex2_mufu(e.x), ex2_mufu(e.y)); }
+
+// S consecutive floats from shared / global memory as S/2 pairs (16-byte vector accesses)
+template <int S>
+__device__ __forceinline__ void ld_pairs(float2 (&o)[S / 2], const float* p) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(p)[i];
+        o[2 * i] = make_float2(v.x, v.y);
+        o[2 * i + 1] = make_float2(v.z, v.w);
+    }
+}
+template <int S>
+__device__ __forceinline__ void st_pairs(float* p, const float2 (&o)[S / 2]) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i)
+        reinterpret_cast<float4*>(p)[i] = make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
+}
+template <int S>
+__device__ __forceinline__ void st_pairs_cg(float* p, const float2 (&o)[S / 2]) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i)
+        __stcg(reinterpret_cast<float4*>(p) + i,
+               make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y));
+}
+template <int S>
+__device__ __forceinline__ void ld_pairs_cg(float2 (&o)[S / 2], const float* p) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
+        o[2 * i] = make_float2(v.x, v.y);
+        o[2 * i + 1] = make_float2(v.z, v.w);
+    }
+}
+
+template <int S>
+__device__ __forceinline__ bool all_finite(const float2 (&v)[S / 2]) {
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < S / 2; ++i) ok = ok && isfinite(v[i].x) && isfinite(v[i].y);
+    return ok;
+}
+
+// Reduce-scatter of V per-lane values over the NG adjacent lanes of a channel: on return lane
+// `ng` holds, in v[0 .. V/NG), the channel totals of values [ng*V/NG, (ng+1)*V/NG).
+template <int V, int NG>
+__device__ __forceinline__ void reduce_scatter(float (&v)[V], int ng) {
+    int c = V;
+#pragma unroll
+    for (int m = NG / 2; m >= 1; m >>= 1) {
+        const bool up = (ng & m) != 0;
+        const int h = c / 2;
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) {
+            if (i < h) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(kFull, send, m);
+            }
+        }
+        c = h;
+    }
 }
 
 // ------------------------------------------------------------------------------------------------
 // Forward.  SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end
-// state).  SUMMARY = false: the real scan from the segment's entering state, writing y and the
+// state).  SUMMARY = false: the scan from the segment's entering state, writing y and the
 // chunk-end checkpoints.
-// Shared memory: x, delta_raw raw tiles [T][DT] (delta_raw's is reused for y), B, C as float
-// [T][N], (delta, delta*x) pairs [T][DT].
-template <typename E, int N, bool SUMMARY>
-__global__ void __launch_bounds__(RealCfg<N>::NT) real_fwd_kernel(RealArgs p) {
-    using Cfg = RealCfg<N>;
-    constexpr int S = Cfg::S, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT;
+// Shared memory: x and delta_raw raw tiles [T][DT] (delta_raw's is reused for y), B and C as
+// float [T][N], (delta, delta*x) pairs [T][DT].
+template <typename E, int N, int S, bool SUMMARY>
+__global__ void __launch_bounds__(RealCfg<N, S>::NT) real_fwd_kernel(RealArgs p) {
+    using Cfg = RealCfg<N, S>;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, U = Cfg::U;
     extern __shared__ __align__(16) unsigned char smem[];
     const int T = p.T;
     E* sx = reinterpret_cast<E*>(smem);
@@ -57,18 +130,16 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     const int c_begin = seg * p.seg_chunks;
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
 
-    float A2[S], h[S], P[S];
+    float2 A2[P2], h[P2], P[P2];
 #pragma unroll
-    for (int j = 0; j < S; ++j) {
-        A2[j] = dv ? -expf(p.A_log[d * N + n0 + j]) * kLog2e : 0.0f;
-        h[j] = 0.0f;
-        P[j] = 1.0f;
+    for (int i = 0; i < P2; ++i) {
+        A2[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]) * kLog2e,
+                                 -expf(p.A_log[d * N + n0 + 2 * i + 1]) * kLog2e)
+                   : make_float2(0.0f, 0.0f);
+        h[i] = make_float2(0.0f, 0.0f);
+        P[i] = make_float2(1.0f, 1.0f);
     }
-    if (!SUMMARY && seg > 0 && dv) {
-        const float4 hv = *reinterpret_cast<const float4*>(
-            p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
-        h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
-    }
+    if (!SUMMARY && seg > 0 && dv) ld_pairs<S>(h, p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
     const size_t boff = (size_t)b * p.L;
     const E* xb = static_cast<const E*>(p.x) + boff * p.D;
     const E* drb = static_cast<const E*>(p.draw) + boff * p.D;
@@ -80,48 +151,59 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     for (int c = c_begin; c < c_end; ++c) {
         const int t0 = c * T;
         const int rows = min(T, p.L - t0);
+        const int rows4 = (rows + U - 1) / U * U;
         __syncthreads();
-        load_tile<E, DT>(sx, xb, t0, rows, p.L, d0, p.D, tid, NT);
-        load_tile<E, DT>(sdr, drb, t0, rows, p.L, d0, p.D, tid, NT);
-        load_rows_f32<E, N>(sB, Bb, t0, rows, p.L, tid, NT);
-        if (!SUMMARY) load_rows_f32<E, N>(sC, Cb, t0, rows, p.L, tid, NT);
+        load_tile<E, DT>(sx, xb, t0, rows4, p.L, d0, p.D, tid, NT);
+        load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
+        load_rows_f32<E, N>(sB, Bb, t0, rows4, p.L, tid, NT);
+        if (!SUMMARY) load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
         __syncthreads();
-        for (int i = tid; i < rows * DT; i += NT) {
-            const float dlt = softplus_acc(Elem<E>::to_f(sdr[i]));
+        // steps past the sequence end get delta = 0: a = 1 and no input, i.e. they change nothing
+        for (int i = tid; i < rows4 * DT; i += NT) {
+            const float dlt = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
             sdd[i] = make_float2(dlt, dlt * Elem<E>::to_f(sx[i]));
         }
         __syncthreads();
-        for (int r = 0; r < rows; ++r) {
-            const float2 dd = sdd[r * DT + dl];
-            const float4 bv = *reinterpret_cast<const float4*>(sB + r * N + n0);
-            const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
-            if (SUMMARY) {
+        for (int r0 = 0; r0 < rows; r0 += U) {
+            float yp[U];
 #pragma unroll
-                for (int j = 0; j < S; ++j) {
-                    const float a = ex2_mufu(dd.x * A2[j]);
-                    h[j] = fmaf(a, h[j], dd.y * bj[j]);
-                    P[j] *= a;
+            for (int u = 0; u < U; ++u) {
+                const int r = r0 + u;
+                const float2 dd = sdd[r * DT + dl];
+                float2 bq[P2];
+                ld_pairs<S>(bq, sB + r * N + n0);
+                if (SUMMARY) {
+#pragma unroll
+                    for (int i = 0; i < P2; ++i) {
+                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
+                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
+                        P[i] = __fmul2_rn(P[i], a);
+                    }
+                } else {
+                    float2 cq[P2];
+                    ld_pairs<S>(cq, sC + r * N + n0);
+                    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int i = 0; i < P2; ++i) {
+                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
+                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
+                        acc = __ffma2_rn(cq[i], h[i], acc);
+                    }
+                    yp[u] = acc.x + acc.y;
                 }
-            } else {
-                const float4 cv = *reinterpret_cast<const float4*>(sC + r * N + n0);
-                const float cj[4] = {cv.x, cv.y, cv.z, cv.w};
-                float yp = 0.0f;
+            }
+            if (!SUMMARY) {
+                reduce_scatter<U, NG>(yp, ng);
 #pragma unroll
-                for (int j = 0; j < S; ++j) {
-                    const float a = ex2_mufu(dd.x * A2[j]);
-                    h[j] = fmaf(a, h[j], dd.y * bj[j]);
-                    yp = fmaf(cj[j], h[j], yp);
+                for (int j = 0; j < U / NG; ++j) {
+                    const int r = r0 + ng * (U / NG) + j;
+                    if (r < rows)
+                        sdr[r * DT + dl] = Elem<E>::from_f(fmaf(dsk, Elem<E>::to_f(sx[r * DT + dl]), yp[j]));
                 }
-#pragma unroll
-                for (int o = 1; o < NG; o <<= 1) yp += __shfl_xor_sync(0xffffffffu, yp, o);
-                if (ng == 0)
-                    sdr[r * DT + dl] = Elem<E>::from_f(fmaf(dsk, Elem<E>::to_f(sx[r * DT + dl]), yp));
             }
         }
         if (!SUMMARY) {
-            if (dv)
-                *reinterpret_cast<float4*>(p.ckpt + (((size_t)b * p.nC + c) * p.D + d) * N + n0) =
-                    make_float4(h[0], h[1], h[2], h[3]);
+            if (dv) st_pairs<S>(p.ckpt + (((size_t)b * p.nC + c) * p.D + d) * N + n0, h);
             __syncthreads();
             store_tile<E, DT>(yb, sdr, t0, rows, p.L, d0, p.D, tid, NT);
         }
@@ -129,10 +211,10 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     if (SUMMARY) {
         if (dv) {
             const size_t o = (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N + n0;
-            *reinterpret_cast<float4*>(p.sumP + o) = make_float4(P[0], P[1], P[2], P[3]);
-            *reinterpret_cast<float4*>(p.sumS + o) = make_float4(h[0], h[1], h[2], h[3]);
+            st_pairs<S>(p.sumP + o, P);
+            st_pairs<S>(p.sumS + o, h);
         }
-    } else if (dv && !all_finite4(h)) {
+    } else if (dv && !all_finite<S>(h)) {
         flag_status(p.status, kStatusNonFinite);
     }
 }
@@ -156,10 +238,10 @@ __global__ void real_carry_fwd_kernel(int B, int nseg, int DN, const float* __re
 // ------------------------------------------------------------------------------------------------
 // Backward segment summary (segments 1..nseg-1): local reverse adjoint from zero over the
 // segment, v <- a_t (C_t dy_t + v), and P = prod a over the segment.
-template <typename E, int N>
-__global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_summary_kernel(RealArgs p) {
-    using Cfg = RealCfg<N>;
-    constexpr int S = Cfg::S, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT;
+template <typename E, int N, int S>
+__global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(RealArgs p) {
+    using Cfg = RealCfg<N, S>;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, U = Cfg::U;
     extern __shared__ __align__(16) unsigned char smem[];
     const int T = p.T;
     E* sdy = reinterpret_cast<E*>(smem);
@@ -174,12 +256,14 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_summary_kernel(RealAr
     const int c_begin = seg * p.seg_chunks;
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
 
-    float A2[S], v[S], P[S];
+    float2 A2[P2], v[P2], P[P2];
 #pragma unroll
-    for (int j = 0; j < S; ++j) {
-        A2[j] = dv ? -expf(p.A_log[d * N + n0 + j]) * kLog2e : 0.0f;
-        v[j] = 0.0f;
-        P[j] = 1.0f;
+    for (int i = 0; i < P2; ++i) {
+        A2[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]) * kLog2e,
+                                 -expf(p.A_log[d * N + n0 + 2 * i + 1]) * kLog2e)
+                   : make_float2(0.0f, 0.0f);
+        v[i] = make_float2(0.0f, 0.0f);
+        P[i] = make_float2(1.0f, 1.0f);
     }
     const size_t boff = (size_t)b * p.L;
     const E* dyb = static_cast<const E*>(p.dy) + boff * p.D;
@@ -189,30 +273,36 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_summary_kernel(RealAr
     for (int c = c_end - 1; c >= c_begin; --c) {
         const int t0 = c * T;
         const int rows = min(T, p.L - t0);
+        const int rows4 = (rows + U - 1) / U * U;
         __syncthreads();
-        load_tile<E, DT>(sdy, dyb, t0, rows, p.L, d0, p.D, tid, NT);
-        load_tile<E, DT>(sdr, drb, t0, rows, p.L, d0, p.D, tid, NT);
-        load_rows_f32<E, N>(sC, Cb, t0, rows, p.L, tid, NT);
+        load_tile<E, DT>(sdy, dyb, t0, rows4, p.L, d0, p.D, tid, NT);
+        load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
+        load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
         __syncthreads();
-        for (int i = tid; i < rows * DT; i += NT) sdel[i] = softplus_acc(Elem<E>::to_f(sdr[i]));
+        for (int i = tid; i < rows4 * DT; i += NT)
+            sdel[i] = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
         __syncthreads();
-        for (int r = rows - 1; r >= 0; --r) {
-            const float dlt = sdel[r * DT + dl];
-            const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-            const float4 cv = *reinterpret_cast<const float4*>(sC + r * N + n0);
-            const float cj[4] = {cv.x, cv.y, cv.z, cv.w};
+        for (int r0 = rows4 - U; r0 >= 0; r0 -= U) {
 #pragma unroll
-            for (int j = 0; j < S; ++j) {
-                const float a = ex2_mufu(dlt * A2[j]);
-                v[j] = a * fmaf(cj[j], dyv, v[j]);
-                P[j] *= a;
+            for (int u = U - 1; u >= 0; --u) {
+                const int r = r0 + u;
+                const float dlt = sdel[r * DT + dl];
+                const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
+                float2 cq[P2];
+                ld_pairs<S>(cq, sC + r * N + n0);
+#pragma unroll
+                for (int i = 0; i < P2; ++i) {
+                    const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
+                    v[i] = __fmul2_rn(a, __ffma2_rn(cq[i], f2(dyv), v[i]));
+                    P[i] = __fmul2_rn(P[i], a);
+                }
             }
         }
     }
     if (dv) {
         const size_t o = (((size_t)b * (p.nseg - 1) + (seg - 1)) * p.D + d) * N + n0;
-        *reinterpret_cast<float4*>(p.gsumP + o) = make_float4(P[0], P[1], P[2], P[3]);
-        *reinterpret_cast<float4*>(p.gsumG + o) = make_float4(v[0], v[1], v[2], v[3]);
+        st_pairs<S>(p.gsumP + o, P);
+        st_pairs<S>(p.gsumG + o, v);
     }
 }
 
@@ -233,53 +323,21 @@ __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __re
     }
 }
 
-// Reduce 8 per-lane values over the lanes that share (lane % NG).  On return v[0] holds the total
-// of value index ((lane>>4)&1)*4 + ((lane>>3)&1)*2 + ((lane>>2)&1).
-template <int NG>
-__device__ __forceinline__ void transpose_reduce8(float (&v)[8]) {
-    const int lane = threadIdx.x & 31;
-    {
-        const bool up = lane & 16;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float send = up ? v[i] : v[i + 4];
-            const float keep = up ? v[i + 4] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-    }
-    {
-        const bool up = lane & 8;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float send = up ? v[i] : v[i + 2];
-            const float keep = up ? v[i + 2] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-    }
-    {
-        const bool up = lane & 4;
-        const float send = up ? v[0] : v[1];
-        const float keep = up ? v[1] : v[0];
-        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    if (NG <= 2) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
-    if (NG <= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-}
-
 // ------------------------------------------------------------------------------------------------
 // Backward main kernel.  For every stretch of TB <= 128 steps (a chunk, or half a 256-step
 // chunk), in reverse order:
-//   pass A: recompute h forward from the chunk checkpoint, saving h every TS steps (smem);
-//   pass B: for each TS-step piece in reverse, recompute (a_t, a_t h_{t-1}) into registers and
-//           sweep the adjoint backwards, emitting dx, ddelta_raw (per channel), per-CTA sums of
-//           dB, dC (over the CTA's channels) and per-thread sums for dA_log, dD.
-// Shared memory: x, delta_raw, dy raw tiles [TB][DT]; B, C float [TB][N]; delta [TB][DT];
-// saved states [TB/TS][NT] float4; cross-warp dB/dC sums [TS][warps][2N].
-template <typename E, int N>
-__global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_kernel(RealArgs p) {
-    using Cfg = RealCfg<N>;
-    constexpr int S = Cfg::S, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TS = Cfg::TS;
-    constexpr int NW = NT / 32, N2 = 2 * N;
+//   pass A: recompute h forward from the chunk checkpoint; the state at the start of every
+//           TS-step window goes to an L2-resident scratch region owned by this CTA;
+//   pass B: for each window in reverse, recompute (a_t, a_t h_{t-1}) into registers and sweep
+//           the adjoint backwards in groups of 4 steps, emitting dx and ddelta_raw per channel,
+//           the sums of dB and dC over the CTA's 32 channels, and per-thread sums for dA_log, dD.
+// Shared memory: x, delta_raw, dy raw tiles [TB][DT] (x's and delta_raw's reused for dx and
+// ddelta_raw); B, C float [TB][N]; delta [TB][DT]; dB/dC values of one 4-step group [4][DT][2N].
+template <typename E, int N, int S>
+__global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_kernel(RealArgs p) {
+    using Cfg = RealCfg<N, S>;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TS = Cfg::TS;
+    constexpr int U = Cfg::U, Q = Cfg::Q, N2 = 2 * N;
     extern __shared__ __align__(16) unsigned char smem[];
     const int T = p.T;
     const int TB = min(T, kRealMaxTB);
@@ -289,35 +347,29 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     float* sB = reinterpret_cast<float*>(sdy + TB * DT);
     float* sC = sB + TB * N;
     float* sdel = sC + TB * N;
-    float4* sbnd = reinterpret_cast<float4*>(sdel + TB * DT);
-    float* sred = reinterpret_cast<float*>(sbnd + (TB / TS) * NT);
+    float* sred = sdel + TB * DT;
 
     const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
-    const int lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.y, seg = blockIdx.z;
     const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * S;
     const bool dv = d < p.D;
     const int c_begin = seg * p.seg_chunks;
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    // which of the 2N (dB, dC) sums this lane carries after transpose_reduce8, and whether it
-    // is the lane that writes it
-    const int ridx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-    const int rout = ridx < S ? n0 + ridx : N + n0 + (ridx - S);
-    const bool rwriter = (NG == 4) || (NG == 2 && !(lane & 2)) || (NG == 1 && !(lane & 3));
+    // column-sum roles: `part` sums channels [part*DT/Q, ...) of output quad `quad`
+    const int cs_part = (tid >> 3) % Q;
+    const int cs_quad = (tid & 7) + 8 * (tid / (8 * Q));
+    const int cs_u = cs_quad / (N2 / 4), cs_o = 4 * (cs_quad % (N2 / 4));
 
-    float A[S], A2[S], v[S], dA[S];
+    float2 A[P2], A2[P2], v[P2], dA[P2];
 #pragma unroll
-    for (int j = 0; j < S; ++j) {
-        A[j] = dv ? -expf(p.A_log[d * N + n0 + j]) : 0.0f;
-        A2[j] = A[j] * kLog2e;
-        v[j] = 0.0f;
-        dA[j] = 0.0f;
+    for (int i = 0; i < P2; ++i) {
+        A[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]), -expf(p.A_log[d * N + n0 + 2 * i + 1]))
+                  : make_float2(0.0f, 0.0f);
+        A2[i] = __fmul2_rn(A[i], f2(kLog2e));
+        v[i] = make_float2(0.0f, 0.0f);
+        dA[i] = make_float2(0.0f, 0.0f);
     }
-    if (seg < p.nseg - 1 && dv) {
-        const float4 vv = *reinterpret_cast<const float4*>(
-            p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
-        v[0] = vv.x; v[1] = vv.y; v[2] = vv.z; v[3] = vv.w;
-    }
+    if (seg < p.nseg - 1 && dv) ld_pairs<S>(v, p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
     float dDacc = 0.0f;
     const float dsk = dv ? p.Dskip[d] : 0.0f;
     const size_t boff = (size_t)b * p.L;
@@ -329,6 +381,8 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     E* dxb = static_cast<E*>(p.dx) + boff * p.D;
     E* ddrb = static_cast<E*>(p.ddraw) + boff * p.D;
     float* partb = p.dBC_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L * N2;
+    const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    float* bnd = p.bnd_scratch + cta * (size_t)(kRealMaxTB / TS) * NT * S + (size_t)tid * S;
 
     const int per_chunk = T / TB;  // 1, or 2 for 256-step chunks
     for (int c = c_end - 1; c >= c_begin; --c) {
@@ -336,17 +390,16 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_kernel(RealArgs p) {
             const int t0 = c * T + part * TB;
             if (t0 >= p.L) continue;
             const int rows = min(TB, p.L - t0);
+            const int rows4 = (rows + U - 1) / U * U;
             // state entering this stretch
-            float h[S];
+            float2 h[P2];
             if (c > 0 && dv) {
-                const float4 hv = *reinterpret_cast<const float4*>(
-                    p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
-                h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
+                ld_pairs<S>(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
             } else {
 #pragma unroll
-                for (int j = 0; j < S; ++j) h[j] = 0.0f;
+                for (int i = 0; i < P2; ++i) h[i] = make_float2(0.0f, 0.0f);
             }
-            for (int pre = 0; pre < part; ++pre) {  // advance through earlier stretches of the chunk
+            for (int pre = 0; pre < part; ++pre) {  // advance through the chunk's earlier stretch
                 const int tp = c * T + pre * TB;
                 __syncthreads();
                 load_tile<E, DT>(sx, xb, tp, TB, p.L, d0, p.D, tid, NT);
@@ -354,128 +407,171 @@ __global__ void __launch_bounds__(RealCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                 load_rows_f32<E, N>(sB, Bb, tp, TB, p.L, tid, NT);
                 __syncthreads();
                 for (int r = 0; r < TB; ++r) {
-                    const float dlt = softplus_acc(Elem<E>::to_f(sdr[r * DT + dl]));
+                    const float dlt = softplus_fast(Elem<E>::to_f(sdr[r * DT + dl]));
                     const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    const float4 bv = *reinterpret_cast<const float4*>(sB + r * N + n0);
-                    const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
+                    float2 bq[P2];
+                    ld_pairs<S>(bq, sB + r * N + n0);
 #pragma unroll
-                    for (int j = 0; j < S; ++j) h[j] = fmaf(ex2_mufu(dlt * A2[j]), h[j], dxv * bj[j]);
+                    for (int i = 0; i < P2; ++i)
+                        h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dlt), A2[i])), h[i], __fmul2_rn(f2(dxv), bq[i]));
                 }
             }
             __syncthreads();
-            load_tile<E, DT>(sx, xb, t0, rows, p.L, d0, p.D, tid, NT);
-            load_tile<E, DT>(sdr, drb, t0, rows, p.L, d0, p.D, tid, NT);
-            load_tile<E, DT>(sdy, dyb, t0, rows, p.L, d0, p.D, tid, NT);
-            load_rows_f32<E, N>(sB, Bb, t0, rows, p.L, tid, NT);
-            load_rows_f32<E, N>(sC, Cb, t0, rows, p.L, tid, NT);
+            load_tile<E, DT>(sx, xb, t0, rows4, p.L, d0, p.D, tid, NT);
+            load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
+            load_tile<E, DT>(sdy, dyb, t0, rows4, p.L, d0, p.D, tid, NT);
+            load_rows_f32<E, N>(sB, Bb, t0, rows4, p.L, tid, NT);
+            load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
             __syncthreads();
-            for (int i = tid; i < rows * DT; i += NT) sdel[i] = softplus_acc(Elem<E>::to_f(sdr[i]));
+            // steps past the sequence end get delta = 0 (a = 1, no input): they pass state and
+            // adjoint through unchanged
+            for (int i = tid; i < rows4 * DT; i += NT)
+                sdel[i] = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
             __syncthreads();
 
-            // pass A: forward recompute, saving the state at the start of every TS-step piece
-            const int npieces = (rows + TS - 1) / TS;
-            for (int k = 0; k < npieces; ++k) {
-                sbnd[k * NT + tid] = make_float4(h[0], h[1], h[2], h[3]);
-                const int r1 = min(rows, (k + 1) * TS);
-                for (int r = k * TS; r < r1; ++r) {
+            // pass A
+            const int nwin = (rows4 + TS - 1) / TS;
+            for (int k = 0; k < nwin; ++k) {
+                st_pairs_cg<S>(bnd + (size_t)k * NT * S, h);
+#pragma unroll
+                for (int ts = 0; ts < TS; ++ts) {
+                    const int r = k * TS + ts;
+                    if (TS > U && r >= rows4) break;
                     const float dlt = sdel[r * DT + dl];
                     const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    const float4 bv = *reinterpret_cast<const float4*>(sB + r * N + n0);
-                    const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
+                    float2 bq[P2];
+                    ld_pairs<S>(bq, sB + r * N + n0);
 #pragma unroll
-                    for (int j = 0; j < S; ++j) h[j] = fmaf(ex2_mufu(dlt * A2[j]), h[j], dxv * bj[j]);
+                    for (int i = 0; i < P2; ++i)
+                        h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dlt), A2[i])), h[i], __fmul2_rn(f2(dxv), bq[i]));
                 }
             }
 
-            // pass B: pieces in reverse
-            for (int k = npieces - 1; k >= 0; --k) {
-                const int r0 = k * TS;
-                const int nr = min(TS, rows - r0);
-                float aa[TS][S], pp[TS][S];
+            // pass B
+            float2 hw[P2];
+            ld_pairs_cg<S>(hw, bnd + (size_t)(nwin - 1) * NT * S);
+            for (int k = nwin - 1; k >= 0; --k) {
+                float2 aa[TS][P2], pp[TS][P2];
                 {
-                    const float4 hv = sbnd[k * NT + tid];
-                    float hc[S] = {hv.x, hv.y, hv.z, hv.w};
+                    float2 hc[P2];
+#pragma unroll
+                    for (int i = 0; i < P2; ++i) hc[i] = hw[i];
+                    if (k > 0) ld_pairs_cg<S>(hw, bnd + (size_t)(k - 1) * NT * S);  // prefetch
 #pragma unroll
                     for (int ts = 0; ts < TS; ++ts) {
-                        if (ts < nr) {
-                            const int r = r0 + ts;
-                            const float dlt = sdel[r * DT + dl];
-                            const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                            const float4 bv = *reinterpret_cast<const float4*>(sB + r * N + n0);
-                            const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
+                        const int r = k * TS + ts;
+                        const float dlt = (TS > U && r >= rows4) ? 0.0f : sdel[r * DT + dl];
+                        const float dxv = (TS > U && r >= rows4) ? 0.0f : dlt * Elem<E>::to_f(sx[r * DT + dl]);
+                        float2 bq[P2];
+                        if (TS > U && r >= rows4) {
 #pragma unroll
-                            for (int j = 0; j < S; ++j) {
-                                const float a = ex2_mufu(dlt * A2[j]);
-                                const float pr = a * hc[j];
-                                aa[ts][j] = a;
-                                pp[ts][j] = pr;
-                                hc[j] = fmaf(dxv, bj[j], pr);
-                            }
+                            for (int i = 0; i < P2; ++i) bq[i] = make_float2(0.0f, 0.0f);
+                        } else {
+                            ld_pairs<S>(bq, sB + r * N + n0);
+                        }
+#pragma unroll
+                        for (int i = 0; i < P2; ++i) {
+                            const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
+                            const float2 pr = __fmul2_rn(a, hc[i]);
+                            aa[ts][i] = a;
+                            pp[ts][i] = pr;
+                            hc[i] = __ffma2_rn(f2(dxv), bq[i], pr);
                         }
                     }
                 }
 #pragma unroll
-                for (int ts = TS - 1; ts >= 0; --ts) {
-                    if (ts < nr) {
-                        const int r = r0 + ts;
+                for (int g4 = TS / U - 1; g4 >= 0; --g4) {
+                    const int rg = k * TS + g4 * U;
+                    if (TS > U && rg >= rows4) continue;
+                    float sv[2 * U];
+#pragma unroll
+                    for (int u = U - 1; u >= 0; --u) {
+                        const int ts = g4 * U + u;
+                        const int r = rg + u;
                         const float dlt = sdel[r * DT + dl];
-                        const float xv = Elem<E>::to_f(sx[r * DT + dl]);
-                        const float dxv = dlt * xv;
+                        const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
                         const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-                        const float4 bv = *reinterpret_cast<const float4*>(sB + r * N + n0);
-                        const float4 cv = *reinterpret_cast<const float4*>(sC + r * N + n0);
-                        const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
-                        const float cj[4] = {cv.x, cv.y, cv.z, cv.w};
-                        float sgB = 0.0f, sAq = 0.0f;
-                        float red[8];
+                        float2 bq[P2], cq[P2];
+                        ld_pairs<S>(bq, sB + r * N + n0);
+                        ld_pairs<S>(cq, sC + r * N + n0);
+                        float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
+                        float2 rB[P2], rC[P2];
 #pragma unroll
-                        for (int j = 0; j < S; ++j) {
-                            const float g = fmaf(cj[j], dyv, v[j]);
-                            const float hj = fmaf(dxv, bj[j], pp[ts][j]);
-                            const float q = g * pp[ts][j];
-                            dA[j] = fmaf(dlt, q, dA[j]);
-                            sAq = fmaf(A[j], q, sAq);
-                            sgB = fmaf(g, bj[j], sgB);
-                            red[j] = g * dxv;
-                            red[S + j] = dyv * hj;
-                            v[j] = aa[ts][j] * g;
+                        for (int i = 0; i < P2; ++i) {
+                            const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);
+                            const float2 hj = __ffma2_rn(f2(dxv), bq[i], pp[ts][i]);
+                            const float2 q = __fmul2_rn(g, pp[ts][i]);
+                            dA[i] = __ffma2_rn(f2(dlt), q, dA[i]);
+                            sa = __ffma2_rn(A[i], q, sa);
+                            sg = __ffma2_rn(g, bq[i], sg);
+                            rB[i] = __fmul2_rn(g, f2(dxv));
+                            rC[i] = __fmul2_rn(f2(dyv), hj);
+                            v[i] = __fmul2_rn(aa[ts][i], g);
                         }
+                        sv[2 * u] = sg.x + sg.y;
+                        sv[2 * u + 1] = sa.x + sa.y;
+                        float* sr = sred + (u * DT + dl) * N2 + n0;
+                        st_pairs<S>(sr, rB);
+                        st_pairs<S>(sr + N, rC);
+                    }
+                    // per-channel sums over the NG lanes: lane ng gets steps [ng*U/NG, ...)
+                    reduce_scatter<2 * U, NG>(sv, ng);
 #pragma unroll
-                        for (int o = 1; o < NG; o <<= 1) {
-                            sgB += __shfl_xor_sync(0xffffffffu, sgB, o);
-                            sAq += __shfl_xor_sync(0xffffffffu, sAq, o);
-                        }
-                        transpose_reduce8<NG>(red);
-                        if (rwriter) sred[(ts * NW + warp) * N2 + rout] = red[0];
-                        if (ng == 0) {
-                            const float zr = Elem<E>::to_f(sdr[r * DT + dl]);
-                            const float dxo = fmaf(dsk, dyv, dlt * sgB);
-                            const float ddel = fmaf(xv, sgB, sAq);
-                            sx[r * DT + dl] = Elem<E>::from_f(dxo);          // x no longer needed
-                            sdr[r * DT + dl] = Elem<E>::from_f(ddel * sigmoid_acc(zr));
+                    for (int j = 0; j < U / NG; ++j) {
+                        const int r = rg + ng * (U / NG) + j;
+                        if (r < rows) {
+                            const float dlt = sdel[r * DT + dl];
+                            const float xv = Elem<E>::to_f(sx[r * DT + dl]);
+                            const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
+                            const float sgB = sv[2 * j], sAq = sv[2 * j + 1];
+                            const float sig = sigmoid_fast(Elem<E>::to_f(sdr[r * DT + dl]));
+                            sx[r * DT + dl] = Elem<E>::from_f(fmaf(dsk, dyv, dlt * sgB));
+                            sdr[r * DT + dl] = Elem<E>::from_f(fmaf(xv, sgB, sAq) * sig);
                             dDacc = fmaf(dyv, xv, dDacc);
                         }
                     }
-                }
-                __syncthreads();
-                for (int i = tid; i < nr * N2; i += NT) {
-                    const int ts = i / N2, o = i - ts * N2;
-                    float s = 0.0f;
+                    __syncthreads();
+                    {   // dB, dC: sum the group's values over the CTA's channels
+                        const float* src = sred + (cs_u * DT + cs_part * (DT / Q)) * N2 + cs_o;
+                        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
 #pragma unroll
-                    for (int w = 0; w < NW; ++w) s += sred[(ts * NW + w) * N2 + o];
-                    partb[(size_t)(t0 + r0 + ts) * N2 + o] = s;
+                        for (int ch = 0; ch < DT / Q; ch += 2) {
+                            const float4 a0 = *reinterpret_cast<const float4*>(src + ch * N2);
+                            const float4 a1 = *reinterpret_cast<const float4*>(src + (ch + 1) * N2);
+                            s0 = __fadd2_rn(s0, make_float2(a0.x, a0.y));
+                            s1 = __fadd2_rn(s1, make_float2(a0.z, a0.w));
+                            s2 = __fadd2_rn(s2, make_float2(a1.x, a1.y));
+                            s3 = __fadd2_rn(s3, make_float2(a1.z, a1.w));
+                        }
+                        s0 = __fadd2_rn(s0, s2);
+                        s1 = __fadd2_rn(s1, s3);
+#pragma unroll
+                        for (int m = 8; m < 8 * Q; m <<= 1) {
+                            s0.x += __shfl_xor_sync(kFull, s0.x, m);
+                            s0.y += __shfl_xor_sync(kFull, s0.y, m);
+                            s1.x += __shfl_xor_sync(kFull, s1.x, m);
+                            s1.y += __shfl_xor_sync(kFull, s1.y, m);
+                        }
+                        const int r = rg + cs_u;
+                        if (cs_part == 0 && r < rows)
+                            *reinterpret_cast<float4*>(partb + (size_t)(t0 + r) * N2 + cs_o) =
+                                make_float4(s0.x, s0.y, s1.x, s1.y);
+                    }
+                    __syncthreads();
                 }
-                __syncthreads();
             }
             store_tile<E, DT>(dxb, sx, t0, rows, p.L, d0, p.D, tid, NT);
             store_tile<E, DT>(ddrb, sdr, t0, rows, p.L, d0, p.D, tid, NT);
         }
     }
+    // each lane of a channel accumulated dD over its own subset of steps
+#pragma unroll
+    for (int m = 1; m < NG; m <<= 1) dDacc += __shfl_xor_sync(kFull, dDacc, m);
     if (dv) {
         const size_t o = (((size_t)b * p.nseg + seg) * p.D + d) * N + n0;
-        *reinterpret_cast<float4*>(p.dA_part + o) = make_float4(dA[0], dA[1], dA[2], dA[3]);
+        st_pairs<S>(p.dA_part + o, dA);
         if (ng == 0) p.dD_part[((size_t)b * p.nseg + seg) * p.D + d] = dDacc;
-        if (!all_finite4(v)) flag_status(p.status, kStatusNonFinite);
+        if (!all_finite<S>(v)) flag_status(p.status, kStatusNonFinite);
     }
 }
 
@@ -514,19 +610,19 @@ __global__ void real_reduce_params_kernel(RealArgs p, int N) {
     }
 }
 
-size_t fwd_smem(int T, int N, int esz) {
-    const int DT = kRealDT;
-    return (size_t)T * DT * esz * 2 + (size_t)T * N * 4 * 2 + (size_t)T * DT * 8;
+template <int N, int S>
+size_t fwd_smem(int T, int esz) {
+    return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 * 2 + (size_t)T * kRealDT * 8;
 }
-size_t bwd_summary_smem(int T, int N, int esz) {
-    const int DT = kRealDT;
-    return (size_t)T * DT * esz * 2 + (size_t)T * N * 4 + (size_t)T * DT * 4;
+template <int N, int S>
+size_t bwd_summary_smem(int T, int esz) {
+    return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 + (size_t)T * kRealDT * 4;
 }
-size_t bwd_smem(int T, int N, int esz) {
-    const int DT = kRealDT, NT = real_threads(N);
+template <int N, int S>
+size_t bwd_smem(int T, int esz) {
     const int TB = T < kRealMaxTB ? T : kRealMaxTB;
-    return (size_t)TB * DT * esz * 3 + (size_t)TB * N * 4 * 2 + (size_t)TB * DT * 4 +
-           (size_t)(TB / kRealTS) * NT * 16 + (size_t)kRealTS * (NT / 32) * 2 * N * 4;
+    return (size_t)TB * kRealDT * esz * 3 + (size_t)TB * N * 4 * 2 + (size_t)TB * kRealDT * 4 +
+           (size_t)RealCfg<N, S>::U * kRealDT * 2 * N * 4;
 }
 
 template <typename K>
@@ -534,45 +630,44 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename E, int N>
+template <typename E, int N, int S>
 cudaError_t real_fwd_impl(const RealArgs& a, cudaStream_t st) {
-    const dim3 block(real_threads(N));
-    const size_t esz = sizeof(E);
+    const dim3 block(RealCfg<N, S>::NT);
+    const int esz = (int)sizeof(E);
     cudaError_t e;
+    const size_t sm = fwd_smem<N, S>(a.T, esz);
     if (a.nseg > 1) {
-        const size_t sm = fwd_smem(a.T, N, (int)esz);
-        if ((e = set_smem(real_fwd_kernel<E, N, true>, sm)) != cudaSuccess) return e;
-        real_fwd_kernel<E, N, true><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
+        if ((e = set_smem(real_fwd_kernel<E, N, S, true>, sm)) != cudaSuccess) return e;
+        real_fwd_kernel<E, N, S, true><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
                                                                             a.sumP, a.sumS, a.hin);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t sm = fwd_smem(a.T, N, (int)esz);
-    if ((e = set_smem(real_fwd_kernel<E, N, false>, sm)) != cudaSuccess) return e;
-    real_fwd_kernel<E, N, false><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
+    if ((e = set_smem(real_fwd_kernel<E, N, S, false>, sm)) != cudaSuccess) return e;
+    real_fwd_kernel<E, N, S, false><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
     return cudaGetLastError();
 }
 
-template <typename E, int N>
+template <typename E, int N, int S>
 cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
-    const dim3 block(real_threads(N));
+    const dim3 block(RealCfg<N, S>::NT);
     const int esz = (int)sizeof(E);
     cudaError_t e;
     if (a.nseg > 1) {
-        const size_t sm = bwd_summary_smem(a.T, N, esz);
-        if ((e = set_smem(real_bwd_summary_kernel<E, N>, sm)) != cudaSuccess) return e;
-        real_bwd_summary_kernel<E, N><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
+        const size_t sm = bwd_summary_smem<N, S>(a.T, esz);
+        if ((e = set_smem(real_bwd_summary_kernel<E, N, S>, sm)) != cudaSuccess) return e;
+        real_bwd_summary_kernel<E, N, S><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
                                                                             a.gsumP, a.gsumG, a.vin);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t sm = bwd_smem(a.T, N, esz);
-    if ((e = set_smem(real_bwd_kernel<E, N>, sm)) != cudaSuccess) return e;
-    real_bwd_kernel<E, N><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
+    const size_t sm = bwd_smem<N, S>(a.T, esz);
+    if ((e = set_smem(real_bwd_kernel<E, N, S>, sm)) != cudaSuccess) return e;
+    real_bwd_kernel<E, N, S><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t nbc = (int64_t)a.B * a.L * 2 * N;
     if (nbc > 0) {
@@ -584,28 +679,27 @@ cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <typename E>
+cudaError_t fwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
+    if (N == 4) return real_fwd_impl<E, 4, 4>(a, st);
+    if (N == 8) return real_fwd_impl<E, 8, kRealStates8>(a, st);
+    return real_fwd_impl<E, 16, kRealStates16>(a, st);
+}
+template <typename E>
+cudaError_t bwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
+    if (N == 4) return real_bwd_impl<E, 4, 4>(a, st);
+    if (N == 8) return real_bwd_impl<E, 8, kRealStates8>(a, st);
+    return real_bwd_impl<E, 16, kRealStates16>(a, st);
+}
+
 }  // namespace
 
 cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st) {
-    if (io_bf16) {
-        if (N == 4) return real_fwd_impl<__nv_bfloat16, 4>(a, st);
-        if (N == 8) return real_fwd_impl<__nv_bfloat16, 8>(a, st);
-        return real_fwd_impl<__nv_bfloat16, 16>(a, st);
-    }
-    if (N == 4) return real_fwd_impl<float, 4>(a, st);
-    if (N == 8) return real_fwd_impl<float, 8>(a, st);
-    return real_fwd_impl<float, 16>(a, st);
+    return io_bf16 ? fwd_dispatch<__nv_bfloat16>(a, N, st) : fwd_dispatch<float>(a, N, st);
 }
 
 cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st) {
-    if (io_bf16) {
-        if (N == 4) return real_bwd_impl<__nv_bfloat16, 4>(a, st);
-        if (N == 8) return real_bwd_impl<__nv_bfloat16, 8>(a, st);
-        return real_bwd_impl<__nv_bfloat16, 16>(a, st);
-    }
-    if (N == 4) return real_bwd_impl<float, 4>(a, st);
-    if (N == 8) return real_bwd_impl<float, 8>(a, st);
-    return real_bwd_impl<float, 16>(a, st);
+    return io_bf16 ? bwd_dispatch<__nv_bfloat16>(a, N, st) : bwd_dispatch<float>(a, N, st);
 }
 
 }  // namespace ssm

@@ -29,6 +29,28 @@ __device__ __forceinline__ float softplus_acc(float z) {
     return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
 }
 
+// softplus(z) = max(z, 0) + log1p(e), e = exp(-|z|) in [0, 1], using the identity
+// log1p(e) = 2 atanh(s) with s = e / (2 + e) in [0, 1/3] and a polynomial in w = s^2 for
+// 2 atanh(s) / s, fitted here (iteratively reweighted least squares towards minimax, max relative
+// error 4.5e-9 on [0, 1/9]).  With the MUFU exp2 the result is within ~6e-7 relative of softplus.
+__device__ __forceinline__ float softplus_fast(float z) {
+    const float e = ex2_mufu(-fabsf(z) * kLog2e);
+    const float s = __fdividef(e, 2.0f + e);
+    const float w = s * s;
+    float q = fmaf(w, 0.28011780977249146f, 0.2800184488296509f);
+    q = fmaf(w, q, 0.4002152383327484f);
+    q = fmaf(w, q, 0.666664183139801f);
+    q = fmaf(w, q, 2.0f);
+    return fmaf(s, q, fmaxf(z, 0.0f));
+}
+
+// sigmoid(z) = 1 / (1 + exp(-z)) from e = exp(-|z|); within ~5e-7 relative.
+__device__ __forceinline__ float sigmoid_fast(float z) {
+    const float e = ex2_mufu(-fabsf(z) * kLog2e);
+    const float r = __fdividef(1.0f, 1.0f + e);
+    return z >= 0.0f ? r : e * r;
+}
+
 // sigmoid(z) = d softplus / dz, evaluated without overflow for either sign of z.
 __device__ __forceinline__ float sigmoid_acc(float z) {
     const float e = expf(-fabsf(z));

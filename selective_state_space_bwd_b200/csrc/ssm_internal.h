@@ -7,16 +7,23 @@
 
 namespace ssm {
 
-// Thread layout of the real-mode kernels: every thread owns S consecutive states of one channel,
-// NG = N / S threads cover a channel, a CTA covers DT = 32 channels with 32 * NG threads.  The
-// backward holds TS steps of (a_t, a_t h_{t-1}) per state in registers.
-constexpr int kRealS = 4;
+// Thread layout of the real-mode kernels: every thread owns S consecutive states of one channel
+// (S = 4 or 8 for N = 16), NG = N / S adjacent lanes cover a channel, a CTA covers DT = 32
+// channels with 32 * NG threads.  The backward holds a window of TS steps of (a_t, a_t h_{t-1})
+// per state in registers (TS * S = 32) and parks the state at every window start in an
+// L2-resident scratch region of the workspace.
 constexpr int kRealDT = 32;
-constexpr int kRealTS = 8;
 constexpr int kRealMaxTB = 128;  // longest stretch of steps the backward stages at once
+constexpr int kRealStates16 = 4;
+constexpr int kRealStates8 = 4;
 
 inline int real_dt(int) { return kRealDT; }
-inline int real_threads(int N) { return kRealDT * (N / kRealS); }
+inline int real_states(int N) { return N == 16 ? kRealStates16 : (N == 8 ? kRealStates8 : 4); }
+inline int real_threads(int N) { return kRealDT * (N / real_states(N)); }
+inline int real_window(int N) { return real_states(N) == 4 ? 8 : 4; }
+inline size_t real_bnd_floats_per_cta(int N) {
+    return (size_t)(kRealMaxTB / real_window(N)) * real_threads(N) * real_states(N);
+}
 
 // Complex mode: one thread per mode, kCplxKT modes per CTA, kCplxTT steps staged per tile.
 constexpr int kCplxKT = 64;
@@ -45,6 +52,7 @@ struct RealArgs {
     float* dBC_part;  // [ndt][B][L][2N] per-CTA sums over its channels (dB then dC)
     float* dA_part;   // [B][nseg][D][N] sum over the segment of delta * q
     float* dD_part;   // [B][nseg][D]
+    float* bnd_scratch;  // per-CTA window-start states of the backward (L2-resident)
     void* dB;
     void* dC;
     float* dA_log;
