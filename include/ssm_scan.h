@@ -139,6 +139,27 @@ int ssm_scan_bwd(const ssm_shape* shape,
                  void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC, float* dD,
                  void* ws, size_t ws_bytes, ssm_stream_t stream);
 
+/*
+ * Forward scan for callers that cannot allocate device memory (the pages describe no such call;
+ * it exists for integrators whose device memory is owned by someone else, or whose code path may
+ * not call cudaMalloc).  Same inputs, outputs and results as ssm_scan_fwd, but no workspace
+ * argument: the scratch is a fixed 8 MiB array compiled into the library, held on every GPU that
+ * loads it until the process exits.
+ * - Shapes whose forward workspace (ssm_scan_workspace_bytes(shape, 0)) exceeds 8 MiB are
+ *   rejected with SSM_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  Only problems that
+ *   the library splits into many time segments need more than 256 bytes.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.
+ * - Every call on a device shares the one array and leaves its contents behind; calls that
+ *   overlap on the GPU (other streams, other host threads) race on it.  Serialise them.
+ * - The device status word is kept in that array and is not readable through ssm_scan_status.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+int ssm_scan_fwd_noalloc(const ssm_shape* shape,
+                         const void* x, const void* delta_raw, const float* A_log,
+                         const void* Bm, const void* Cm, const float* Dskip,
+                         void* y, float* ckpt, ssm_stream_t stream);
+
 /* Workspace bytes for the complex calls (at least 256); 0 for an invalid shape. */
 size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward);
 

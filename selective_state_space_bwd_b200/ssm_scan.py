@@ -48,7 +48,8 @@ _lib = None
 EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_workspace_bytes",
             "ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_complex_workspace_bytes",
             "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
-            "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string"]
+            "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
+            "ssm_scan_fwd_noalloc"]
 
 
 def lib():
@@ -81,6 +82,8 @@ def lib():
             L.ssm_scan_complex_kernel_launches.restype = I
             L.ssm_scan_status.argtypes, L.ssm_scan_status.restype = [P, P], I
             L.ssm_status_string.argtypes, L.ssm_status_string.restype = [I], ctypes.c_char_p
+            L.ssm_scan_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P]
+            L.ssm_scan_fwd_noalloc.restype = I
             _lib = L
     return _lib
 
@@ -166,6 +169,23 @@ def ssm_scan_fwd(x, delta_raw, A_log, Bm, Cm, Dskip, chunk=128, seg_chunks=0, y=
                               _p(Dskip), _p(y), _p(ckpt), _p(ws), ws.numel() * ws.element_size(),
                               _stream(stream))
     _check(code, "ssm_scan_fwd")
+    return y, ckpt
+
+
+def ssm_scan_fwd_noalloc(x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt, chunk=128, seg_chunks=0,
+                         stream=None):
+    """Forward scan without a workspace, for callers that cannot allocate device memory: the
+    scratch is the library's built-in 8 MiB device array (shared by every call on a device, so
+    overlapping calls race).  The caller passes preallocated ``y`` and ``ckpt``; this function
+    allocates nothing.  Raises SsmError(SSM_ERR_WORKSPACE_TOO_SMALL) when the problem needs more
+    scratch than the array holds."""
+    _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt)
+    B, L, D = x.shape
+    N = A_log.shape[1]
+    shape = real_shape(B, L, D, N, chunk, _io_of(x), seg_chunks)
+    code = lib().ssm_scan_fwd_noalloc(ctypes.byref(shape), _p(x), _p(delta_raw), _p(A_log), _p(Bm),
+                                      _p(Cm), _p(Dskip), _p(y), _p(ckpt), _stream(stream))
+    _check(code, "ssm_scan_fwd_noalloc")
     return y, ckpt
 
 
