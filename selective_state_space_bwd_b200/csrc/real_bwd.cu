@@ -1,239 +1,20 @@
-// Real-mode selective scan: forward with chunk checkpoints, exact chunk-recomputing backward.
+// Real-mode exact backward: chunk recompute from checkpoints and reverse-time adjoint.
 //
-// Recurrence (selective SSM, "选择性状态空间模型(S3M)原理与工程实践" §1.1, Euler input term):
-//   h_t = exp(delta_t A) h_{t-1} + delta_t B_t x_t,   y_t = C_t . h_t + D x_t,
-//   delta = softplus(delta_raw), A = -exp(A_log).
-// Backward ("Breaking the Memory Wall ... Tiled Operator-Space Evolution", abstract): only the
-// state at every chunk end is kept; each chunk is recomputed from its checkpoint and the exact
-// adjoint g_t = C_t dy_t + a_{t+1} g_{t+1} is swept backwards through it.
-//
-// Work decomposition.  Thread = (channel d, S consecutive states), arithmetic on state pairs with
-// the packed fp32x2 instructions; NG = N / S lanes (adjacent) cover a channel; a CTA covers 32
-// channels of one batch row and one time segment (a run of whole chunks).  Steps are processed in
-// groups of 4 so that the loads and exponentials of a group issue ahead of its dependent chain.
-// When a segment does not start at t = 0 its entering state comes from a carry pass over
-// per-segment summaries (prod a, local end state): the local-scan / carry / correction structure
-// of the three-phase scan in "Flash PD-SSM" (technical summary, hardware-aware implementation).
-// The backward mirrors it in reverse time.
-#include "ssm_device.cuh"
-#include "ssm_internal.h"
+// Gradient of sum(dy * y) for the selective scan of real_fwd.cu ("Breaking the Memory Wall:
+// Exact Analytical Differentiation via Tiled Operator-Space Evolution", abstract: exact analytical
+// derivatives without materialising the graph; only chunk-end states are stored).  With
+// g_t = dL/dh_t = C_t dy_t + a_{t+1} g_{t+1} and q_t = g_t a_t h_{t-1}:
+//   dx = D dy + delta sum_n g B,  ddelta = sum_n A q + x sum_n g B,  ddelta_raw = ddelta sigmoid,
+//   dB = sum_d g delta x,  dC = sum_d dy h,  dA_log = A sum_{b,t} delta q,  dD = sum_{b,t} dy x.
+// Thread = (channel, S consecutive states), state pairs in packed fp32x2 arithmetic; NG = N / S
+// adjacent lanes per channel; 32 channels per CTA; a CTA walks its time segment's chunks in
+// reverse.  Time segments other than the last take their entering adjoint from a reverse
+// summary + carry pass (three-phase structure of "Flash PD-SSM", technical summary).
+#include "real_common.cuh"
 
 namespace ssm {
+namespace real {
 namespace {
-
-constexpr unsigned kFull = 0xffffffffu;
-
-template <int N, int S_>
-struct RealCfg {
-    static constexpr int S = S_;            // states per thread
-    static constexpr int P2 = S / 2;        // state pairs per thread
-    static constexpr int NG = N / S;        // lanes per channel
-    static constexpr int DT = kRealDT;      // channels per CTA
-    static constexpr int NT = DT * NG;      // threads per CTA
-    static constexpr int TS = S == 4 ? 8 : 4;  // backward window: steps of (a, a h_prev) in registers
-    static constexpr int U = 4;             // steps per unrolled group (= dB/dC flush period)
-    static constexpr int Q = NT / (2 * N);  // channel parts in the dB/dC column sums
-    static_assert(S == 4 || S == 8, "states per thread");
-    static_assert(N % S == 0 && NG >= 1 && NG <= 4, "dstate must be 4, 8 or 16");
-    static_assert(Q >= 1 && (DT % Q) == 0, "column-sum split");
-};
-
-__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
-
-// exp2 of both halves on the MUFU unit
-__device__ __forceinline__ float2 ex2_pair(float2 e) { return make_float2(ex2_mufu(e.x), ex2_mufu(e.y)); }
-
-// S consecutive floats from shared / global memory as S/2 pairs (16-byte vector accesses)
-template <int S>
-__device__ __forceinline__ void ld_pairs(float2 (&o)[S / 2], const float* p) {
-#pragma unroll
-    for (int i = 0; i < S / 4; ++i) {
-        const float4 v = reinterpret_cast<const float4*>(p)[i];
-        o[2 * i] = make_float2(v.x, v.y);
-        o[2 * i + 1] = make_float2(v.z, v.w);
-    }
-}
-template <int S>
-__device__ __forceinline__ void st_pairs(float* p, const float2 (&o)[S / 2]) {
-#pragma unroll
-    for (int i = 0; i < S / 4; ++i)
-        reinterpret_cast<float4*>(p)[i] = make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
-}
-template <int S>
-__device__ __forceinline__ void st_pairs_cg(float* p, const float2 (&o)[S / 2]) {
-#pragma unroll
-    for (int i = 0; i < S / 4; ++i)
-        __stcg(reinterpret_cast<float4*>(p) + i,
-               make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y));
-}
-template <int S>
-__device__ __forceinline__ void ld_pairs_cg(float2 (&o)[S / 2], const float* p) {
-#pragma unroll
-    for (int i = 0; i < S / 4; ++i) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
-        o[2 * i] = make_float2(v.x, v.y);
-        o[2 * i + 1] = make_float2(v.z, v.w);
-    }
-}
-
-template <int S>
-__device__ __forceinline__ bool all_finite(const float2 (&v)[S / 2]) {
-    bool ok = true;
-#pragma unroll
-    for (int i = 0; i < S / 2; ++i) ok = ok && isfinite(v[i].x) && isfinite(v[i].y);
-    return ok;
-}
-
-// Reduce-scatter of V per-lane values over the NG adjacent lanes of a channel: on return lane
-// `ng` holds, in v[0 .. V/NG), the channel totals of values [ng*V/NG, (ng+1)*V/NG).
-template <int V, int NG>
-__device__ __forceinline__ void reduce_scatter(float (&v)[V], int ng) {
-    int c = V;
-#pragma unroll
-    for (int m = NG / 2; m >= 1; m >>= 1) {
-        const bool up = (ng & m) != 0;
-        const int h = c / 2;
-#pragma unroll
-        for (int i = 0; i < V / 2; ++i) {
-            if (i < h) {
-                const float send = up ? v[i] : v[i + h];
-                const float keep = up ? v[i + h] : v[i];
-                v[i] = keep + __shfl_xor_sync(kFull, send, m);
-            }
-        }
-        c = h;
-    }
-}
-
-// ------------------------------------------------------------------------------------------------
-// Forward.  SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end
-// state).  SUMMARY = false: the scan from the segment's entering state, writing y and the
-// chunk-end checkpoints.
-// Shared memory: x and delta_raw raw tiles [T][DT] (delta_raw's is reused for y), B and C as
-// float [T][N], (delta, delta*x) pairs [T][DT].
-template <typename E, int N, int S, bool SUMMARY>
-__global__ void __launch_bounds__(RealCfg<N, S>::NT) real_fwd_kernel(RealArgs p) {
-    using Cfg = RealCfg<N, S>;
-    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, U = Cfg::U;
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int T = p.T;
-    E* sx = reinterpret_cast<E*>(smem);
-    E* sdr = sx + T * DT;
-    float* sB = reinterpret_cast<float*>(sdr + T * DT);
-    float* sC = sB + T * N;
-    float2* sdd = reinterpret_cast<float2*>(sC + T * N);
-
-    const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
-    const int b = blockIdx.y, seg = blockIdx.z;
-    const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * S;
-    const bool dv = d < p.D;
-    const int c_begin = seg * p.seg_chunks;
-    const int c_end = min(p.nC, c_begin + p.seg_chunks);
-
-    float2 A2[P2], h[P2], P[P2];
-#pragma unroll
-    for (int i = 0; i < P2; ++i) {
-        A2[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]) * kLog2e,
-                                 -expf(p.A_log[d * N + n0 + 2 * i + 1]) * kLog2e)
-                   : make_float2(0.0f, 0.0f);
-        h[i] = make_float2(0.0f, 0.0f);
-        P[i] = make_float2(1.0f, 1.0f);
-    }
-    if (!SUMMARY && seg > 0 && dv) ld_pairs<S>(h, p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
-    const size_t boff = (size_t)b * p.L;
-    const E* xb = static_cast<const E*>(p.x) + boff * p.D;
-    const E* drb = static_cast<const E*>(p.draw) + boff * p.D;
-    const E* Bb = static_cast<const E*>(p.Bm) + boff * N;
-    const E* Cb = static_cast<const E*>(p.Cm) + boff * N;
-    E* yb = SUMMARY ? nullptr : static_cast<E*>(p.y) + boff * p.D;
-    const float dsk = (!SUMMARY && dv) ? p.Dskip[d] : 0.0f;
-
-    for (int c = c_begin; c < c_end; ++c) {
-        const int t0 = c * T;
-        const int rows = min(T, p.L - t0);
-        const int rows4 = (rows + U - 1) / U * U;
-        __syncthreads();
-        load_tile<E, DT>(sx, xb, t0, rows4, p.L, d0, p.D, tid, NT);
-        load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
-        load_rows_f32<E, N>(sB, Bb, t0, rows4, p.L, tid, NT);
-        if (!SUMMARY) load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
-        __syncthreads();
-        // steps past the sequence end get delta = 0: a = 1 and no input, i.e. they change nothing
-        for (int i = tid; i < rows4 * DT; i += NT) {
-            const float dlt = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
-            sdd[i] = make_float2(dlt, dlt * Elem<E>::to_f(sx[i]));
-        }
-        __syncthreads();
-        for (int r0 = 0; r0 < rows; r0 += U) {
-            float yp[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = r0 + u;
-                const float2 dd = sdd[r * DT + dl];
-                float2 bq[P2];
-                ld_pairs<S>(bq, sB + r * N + n0);
-                if (SUMMARY) {
-#pragma unroll
-                    for (int i = 0; i < P2; ++i) {
-                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
-                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
-                        P[i] = __fmul2_rn(P[i], a);
-                    }
-                } else {
-                    float2 cq[P2];
-                    ld_pairs<S>(cq, sC + r * N + n0);
-                    float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-                    for (int i = 0; i < P2; ++i) {
-                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
-                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
-                        acc = __ffma2_rn(cq[i], h[i], acc);
-                    }
-                    yp[u] = acc.x + acc.y;
-                }
-            }
-            if (!SUMMARY) {
-                reduce_scatter<U, NG>(yp, ng);
-#pragma unroll
-                for (int j = 0; j < U / NG; ++j) {
-                    const int r = r0 + ng * (U / NG) + j;
-                    if (r < rows)
-                        sdr[r * DT + dl] = Elem<E>::from_f(fmaf(dsk, Elem<E>::to_f(sx[r * DT + dl]), yp[j]));
-                }
-            }
-        }
-        if (!SUMMARY) {
-            if (dv) st_pairs<S>(p.ckpt + (((size_t)b * p.nC + c) * p.D + d) * N + n0, h);
-            __syncthreads();
-            store_tile<E, DT>(yb, sdr, t0, rows, p.L, d0, p.D, tid, NT);
-        }
-    }
-    if (SUMMARY) {
-        if (dv) {
-            const size_t o = (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N + n0;
-            st_pairs<S>(p.sumP + o, P);
-            st_pairs<S>(p.sumS + o, h);
-        }
-    } else if (dv && !all_finite<S>(h)) {
-        flag_status(p.status, kStatusNonFinite);
-    }
-}
-
-// State entering each segment: h_in[0] = 0, h_in[s+1] = P_s h_in[s] + S_s.
-__global__ void real_carry_fwd_kernel(int B, int nseg, int DN, const float* __restrict__ P,
-                                      const float* __restrict__ Sv, float* __restrict__ hin) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)B * DN) return;
-    const int b = (int)(i / DN), k = (int)(i % DN);
-    float h = 0.0f;
-    for (int s = 0; s < nseg; ++s) {
-        hin[((size_t)b * nseg + s) * DN + k] = h;
-        if (s < nseg - 1) {
-            const size_t j = ((size_t)b * (nseg - 1) + s) * DN + k;
-            h = fmaf(P[j], h, Sv[j]);
-        }
-    }
-}
 
 // ------------------------------------------------------------------------------------------------
 // Backward segment summary (segments 1..nseg-1): local reverse adjoint from zero over the
@@ -611,10 +392,6 @@ __global__ void real_reduce_params_kernel(RealArgs p, int N) {
 }
 
 template <int N, int S>
-size_t fwd_smem(int T, int esz) {
-    return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 * 2 + (size_t)T * kRealDT * 8;
-}
-template <int N, int S>
 size_t bwd_summary_smem(int T, int esz) {
     return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 + (size_t)T * kRealDT * 4;
 }
@@ -628,26 +405,6 @@ size_t bwd_smem(int T, int esz) {
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
-
-template <typename E, int N, int S>
-cudaError_t real_fwd_impl(const RealArgs& a, cudaStream_t st) {
-    const dim3 block(RealCfg<N, S>::NT);
-    const int esz = (int)sizeof(E);
-    cudaError_t e;
-    const size_t sm = fwd_smem<N, S>(a.T, esz);
-    if (a.nseg > 1) {
-        if ((e = set_smem(real_fwd_kernel<E, N, S, true>, sm)) != cudaSuccess) return e;
-        real_fwd_kernel<E, N, S, true><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const int64_t n = (int64_t)a.B * a.D * N;
-        real_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
-                                                                            a.sumP, a.sumS, a.hin);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    if ((e = set_smem(real_fwd_kernel<E, N, S, false>, sm)) != cudaSuccess) return e;
-    real_fwd_kernel<E, N, S, false><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
-    return cudaGetLastError();
 }
 
 template <typename E, int N, int S>
@@ -680,12 +437,6 @@ cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
 }
 
 template <typename E>
-cudaError_t fwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
-    if (N == 4) return real_fwd_impl<E, 4, 4>(a, st);
-    if (N == 8) return real_fwd_impl<E, 8, kRealStates8>(a, st);
-    return real_fwd_impl<E, 16, kRealStates16>(a, st);
-}
-template <typename E>
 cudaError_t bwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
     if (N == 4) return real_bwd_impl<E, 4, 4>(a, st);
     if (N == 8) return real_bwd_impl<E, 8, kRealStates8>(a, st);
@@ -693,13 +444,10 @@ cudaError_t bwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
 }
 
 }  // namespace
-
-cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st) {
-    return io_bf16 ? fwd_dispatch<__nv_bfloat16>(a, N, st) : fwd_dispatch<float>(a, N, st);
-}
+}  // namespace real
 
 cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st) {
-    return io_bf16 ? bwd_dispatch<__nv_bfloat16>(a, N, st) : bwd_dispatch<float>(a, N, st);
+    return io_bf16 ? real::bwd_dispatch<__nv_bfloat16>(a, N, st) : real::bwd_dispatch<float>(a, N, st);
 }
 
 }  // namespace ssm

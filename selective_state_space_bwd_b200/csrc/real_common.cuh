@@ -1,0 +1,127 @@
+// Device helpers shared by the real-mode forward and backward kernels.
+#pragma once
+
+#include "ssm_device.cuh"
+#include "ssm_internal.h"
+
+namespace ssm {
+namespace real {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int N, int S_>
+struct RealCfg {
+    static constexpr int S = S_;            // states per thread
+    static constexpr int P2 = S / 2;        // state pairs per thread
+    static constexpr int NG = N / S;        // lanes per channel
+    static constexpr int DT = kRealDT;      // channels per CTA
+    static constexpr int NT = DT * NG;      // threads per CTA
+    static constexpr int TS = S == 4 ? 8 : 4;  // backward window: steps of (a, a h_prev) in registers
+    static constexpr int U = 4;             // steps per unrolled group (= dB/dC flush period)
+    static constexpr int Q = NT / (2 * N);  // channel parts in the dB/dC column sums
+    static_assert(S == 4 || S == 8, "states per thread");
+    static_assert(N % S == 0 && NG >= 1 && NG <= 4, "dstate must be 4, 8 or 16");
+    static_assert(Q >= 1 && (DT % Q) == 0, "column-sum split");
+};
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// exp2 of both halves on the MUFU unit
+__device__ __forceinline__ float2 ex2_pair(float2 e) { return make_float2(ex2_mufu(e.x), ex2_mufu(e.y)); }
+
+// S consecutive floats from shared / global memory as S/2 pairs (16-byte vector accesses)
+template <int S>
+__device__ __forceinline__ void ld_pairs(float2 (&o)[S / 2], const float* p) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(p)[i];
+        o[2 * i] = make_float2(v.x, v.y);
+        o[2 * i + 1] = make_float2(v.z, v.w);
+    }
+}
+template <int S>
+__device__ __forceinline__ void st_pairs(float* p, const float2 (&o)[S / 2]) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i)
+        reinterpret_cast<float4*>(p)[i] = make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
+}
+template <int S>
+__device__ __forceinline__ void st_pairs_cg(float* p, const float2 (&o)[S / 2]) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i)
+        __stcg(reinterpret_cast<float4*>(p) + i,
+               make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y));
+}
+template <int S>
+__device__ __forceinline__ void ld_pairs_cg(float2 (&o)[S / 2], const float* p) {
+#pragma unroll
+    for (int i = 0; i < S / 4; ++i) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
+        o[2 * i] = make_float2(v.x, v.y);
+        o[2 * i + 1] = make_float2(v.z, v.w);
+    }
+}
+
+template <int S>
+__device__ __forceinline__ bool all_finite(const float2 (&v)[S / 2]) {
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < S / 2; ++i) ok = ok && isfinite(v[i].x) && isfinite(v[i].y);
+    return ok;
+}
+
+// Reduce-scatter of V per-lane values over the NG adjacent lanes of a channel: on return lane
+// `ng` holds, in v[0 .. V/NG), the channel totals of values [ng*V/NG, (ng+1)*V/NG).
+template <int V, int NG>
+__device__ __forceinline__ void reduce_scatter(float (&v)[V], int ng) {
+    int c = V;
+#pragma unroll
+    for (int m = NG / 2; m >= 1; m >>= 1) {
+        const bool up = (ng & m) != 0;
+        const int h = c / 2;
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) {
+            if (i < h) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(kFull, send, m);
+            }
+        }
+        c = h;
+    }
+}
+
+
+// ---------------------------------------------------------------- asynchronous copies (LDGSTS)
+// 16 bytes global -> shared; with valid == false nothing is read and the destination is zeroed.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, bool valid) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int PENDING>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(PENDING));
+}
+
+// Asynchronously copy rows [t0, t0 + rows) x columns [c0, c0 + COLS) of a row-major [*, ncol]
+// array into dst[rows][COLS]; out-of-range rows / columns are zero-filled.  ncol is a multiple of
+// 16 / sizeof(E), so every 16-byte vector is wholly in or out of range.
+template <typename E, int COLS>
+__device__ __forceinline__ void cp_async_tile(E* __restrict__ dst, const E* __restrict__ src, int t0,
+                                              int rows, int nrow, int c0, int ncol, int tid,
+                                              int nthreads) {
+    constexpr int VEC = 16 / sizeof(E);
+    constexpr int VPR = COLS / VEC;
+    static_assert(COLS % VEC == 0, "tile width must be whole 16-byte vectors");
+    for (int i = tid; i < rows * VPR; i += nthreads) {
+        const int r = i / VPR, v = i - r * VPR;
+        const int t = t0 + r, c = c0 + v * VEC;
+        const bool ok = t < nrow && c < ncol;
+        cp_async16(dst + r * COLS + v * VEC, ok ? src + (size_t)t * ncol + c : src, ok);
+    }
+}
+
+}  // namespace real
+}  // namespace ssm
