@@ -79,7 +79,7 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->L * 2 * p->N * 4);
     p->b_dA = o;   o = align256(o + B * S * DN * 4);
     p->b_dD = o;   o = align256(o + B * S * (size_t)p->D * 4);
-    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * S * ssm::real_bnd_floats_per_cta(p->N) * 4);
+    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * S * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
     p->b_end = o;
     return SSM_OK;
 }

@@ -105,38 +105,64 @@ __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __re
 }
 
 // ------------------------------------------------------------------------------------------------
-// Backward main kernel.  For every stretch of TB <= 128 steps (a chunk, or half a 256-step
-// chunk), in reverse order:
-//   pass A: recompute h forward from the chunk checkpoint; the state at the start of every
-//           TS-step window goes to an L2-resident scratch region owned by this CTA;
-//   pass B: for each window in reverse, recompute (a_t, a_t h_{t-1}) into registers and sweep
-//           the adjoint backwards in groups of 4 steps, emitting dx and ddelta_raw per channel,
-//           the sums of dB and dC over the CTA's 32 channels, and per-thread sums for dA_log, dD.
-// Shared memory: x, delta_raw, dy raw tiles [TB][DT] (x's and delta_raw's reused for dx and
-// ddelta_raw); B, C float [TB][N]; delta [TB][DT]; dB/dC values of one 4-step group [4][DT][2N].
-template <typename E, int N, int S>
-__global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_kernel(RealArgs p) {
-    using Cfg = RealCfg<N, S>;
-    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TS = Cfg::TS;
-    constexpr int U = Cfg::U, Q = Cfg::Q, N2 = 2 * N;
+// Backward main kernel.  Chunks of the segment in reverse order; per chunk:
+//   pass A: stream the chunk forward in 32-step sub-tiles (asynchronous two-stage ring).  Per
+//           sub-tile: delta and sigmoid(delta_raw) from one exp per (t, d); (delta, delta) and
+//           the state at every 4-step window start go to this CTA's L2-resident workspace region;
+//           the recurrence advances through the sub-tile.
+//   pass B: stream the sub-tiles in reverse.  Windows are software-pipelined: the reverse sweep
+//           of window q runs interleaved with the recompute of window q-1 (its (a_t, a_t h_{t-1})
+//           into registers), so the exponentials of one overlap the FMA chain of the other.
+//           After each window: reduce-scatter of the per-channel sums over the NG lanes, dx and
+//           ddelta_raw stored directly, and the window's dB / dC values (double-buffered shared
+//           memory) summed over the CTA's 32 channels into its partial-sum rows.
+template <int N>
+struct BwdCfg {
+    static constexpr int S = 4;            // states per thread
+    static constexpr int P2 = 2;           // state pairs per thread
+    static constexpr int NG = N / S;       // lanes per channel
+    static constexpr int DT = kRealDT;     // channels per CTA
+    static constexpr int NT = DT * NG;     // threads per CTA
+    static constexpr int W = 4;            // steps per window
+    static constexpr int TT = 32;          // steps per staged sub-tile
+    static constexpr int Q = NT / (2 * N); // channel parts in the dB/dC column sums
+};
+
+template <typename E, int N>
+struct BwdSmem {
+    static constexpr int TT = BwdCfg<N>::TT, DT = BwdCfg<N>::DT, W = BwdCfg<N>::W;
+    static constexpr int XE = TT * DT, BE = TT * N;
+    // pass A stage: x, delta_raw, B (raw)
+    static constexpr int A_STAGE = (2 * XE + BE) * (int)sizeof(E);
+    static constexpr int A_DD = 2 * A_STAGE;              // (delta, delta*x) float2 [TT][DT]
+    static constexpr int A_BF = A_DD + XE * 8;            // B fp32 [TT][N]
+    static constexpr int A_END = A_BF + BE * 4;
+    // pass B stage: (delta, sigma) float2, x, dy, B, C (raw)
+    static constexpr int B_STAGE = XE * 8 + (2 * XE + 2 * BE) * (int)sizeof(E);
+    static constexpr int B_BF = 2 * B_STAGE;              // B fp32
+    static constexpr int B_CF = B_BF + BE * 4;            // C fp32
+    static constexpr int B_RED = B_CF + BE * 4;           // dB/dC values, 2 x [W][DT][2N]
+    static constexpr int B_END = B_RED + 2 * W * DT * 2 * N * 4;
+    static constexpr int BYTES = A_END > B_END ? A_END : B_END;
+};
+
+template <typename E, int N>
+__global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
+    using Cfg = BwdCfg<N>;
+    using Sm = BwdSmem<E, N>;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;
+    constexpr int TT = Cfg::TT, Q = Cfg::Q, N2 = 2 * N;
     extern __shared__ __align__(16) unsigned char smem[];
-    const int T = p.T;
-    const int TB = min(T, kRealMaxTB);
-    E* sx = reinterpret_cast<E*>(smem);
-    E* sdr = sx + TB * DT;
-    E* sdy = sdr + TB * DT;
-    float* sB = reinterpret_cast<float*>(sdy + TB * DT);
-    float* sC = sB + TB * N;
-    float* sdel = sC + TB * N;
-    float* sred = sdel + TB * DT;
 
     const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
     const int b = blockIdx.y, seg = blockIdx.z;
-    const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * S;
+    const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * Cfg::S;
     const bool dv = d < p.D;
+    const int T = p.T;
+    const int TTe = T < TT ? T : TT;
     const int c_begin = seg * p.seg_chunks;
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    // column-sum roles: `part` sums channels [part*DT/Q, ...) of output quad `quad`
+    // column-sum roles: `cs_part` sums channels [cs_part*DT/Q, ...) of output quad `cs_quad`
     const int cs_part = (tid >> 3) % Q;
     const int cs_quad = (tid & 7) + 8 * (tid / (8 * Q));
     const int cs_u = cs_quad / (N2 / 4), cs_o = 4 * (cs_quad % (N2 / 4));
@@ -150,7 +176,7 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_kernel(RealArgs p)
         v[i] = make_float2(0.0f, 0.0f);
         dA[i] = make_float2(0.0f, 0.0f);
     }
-    if (seg < p.nseg - 1 && dv) ld_pairs<S>(v, p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
+    if (seg < p.nseg - 1 && dv) ld_pairs<4>(v, p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
     float dDacc = 0.0f;
     const float dsk = dv ? p.Dskip[d] : 0.0f;
     const size_t boff = (size_t)b * p.L;
@@ -163,186 +189,270 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_kernel(RealArgs p)
     E* ddrb = static_cast<E*>(p.ddraw) + boff * p.D;
     float* partb = p.dBC_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L * N2;
     const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    float* bnd = p.bnd_scratch + cta * (size_t)(kRealMaxTB / TS) * NT * S + (size_t)tid * S;
+    float* scr = p.bnd_scratch + cta * real_bwd_scratch_floats(N, T);
+    float* bnd = scr + (size_t)tid * 4;                        // window starts: [T/W][NT][4]
+    float2* dsg = reinterpret_cast<float2*>(scr + (size_t)(T / W) * NT * 4);  // (delta, sigma) [T][DT]
 
-    const int per_chunk = T / TB;  // 1, or 2 for 256-step chunks
     for (int c = c_end - 1; c >= c_begin; --c) {
-        for (int part = per_chunk - 1; part >= 0; --part) {
-            const int t0 = c * T + part * TB;
-            if (t0 >= p.L) continue;
-            const int rows = min(TB, p.L - t0);
-            const int rows4 = (rows + U - 1) / U * U;
-            // state entering this stretch
+        const int tc = c * T;
+        const int rows_c = min(T, p.L - tc);
+        const int nsub = (rows_c + TTe - 1) / TTe;
+
+        // ------------------------------------------------------------------ pass A
+        {
             float2 h[P2];
             if (c > 0 && dv) {
-                ld_pairs<S>(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
+                ld_pairs<4>(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
             } else {
 #pragma unroll
                 for (int i = 0; i < P2; ++i) h[i] = make_float2(0.0f, 0.0f);
             }
-            for (int pre = 0; pre < part; ++pre) {  // advance through the chunk's earlier stretch
-                const int tp = c * T + pre * TB;
-                __syncthreads();
-                load_tile<E, DT>(sx, xb, tp, TB, p.L, d0, p.D, tid, NT);
-                load_tile<E, DT>(sdr, drb, tp, TB, p.L, d0, p.D, tid, NT);
-                load_rows_f32<E, N>(sB, Bb, tp, TB, p.L, tid, NT);
-                __syncthreads();
-                for (int r = 0; r < TB; ++r) {
-                    const float dlt = softplus_fast(Elem<E>::to_f(sdr[r * DT + dl]));
-                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    float2 bq[P2];
-                    ld_pairs<S>(bq, sB + r * N + n0);
-#pragma unroll
-                    for (int i = 0; i < P2; ++i)
-                        h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dlt), A2[i])), h[i], __fmul2_rn(f2(dxv), bq[i]));
+            float2* sdd = reinterpret_cast<float2*>(smem + Sm::A_DD);
+            float* sBf = reinterpret_cast<float*>(smem + Sm::A_BF);
+            auto stage = [&](int k) { return reinterpret_cast<E*>(smem + k * Sm::A_STAGE); };
+            auto issue = [&](int j, int k) {
+                const int t0 = tc + j * TTe;
+                E* sx = stage(k);
+                cp_async_tile<E, DT>(sx, xb, t0, TTe, p.L, d0, p.D, tid, NT);
+                cp_async_tile<E, DT>(sx + Sm::XE, drb, t0, TTe, p.L, d0, p.D, tid, NT);
+                cp_async_flat<E>(sx + 2 * Sm::XE, Bb, (size_t)t0 * N, TTe * N, (size_t)p.L * N, tid, NT);
+                cp_async_commit();
+            };
+            __syncthreads();  // previous users of the stage buffers are done
+            issue(0, 0);
+            for (int j = 0; j < nsub; ++j) {
+                const int k = j & 1;
+                if (j + 1 < nsub) {
+                    issue(j + 1, k ^ 1);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
                 }
-            }
-            __syncthreads();
-            load_tile<E, DT>(sx, xb, t0, rows4, p.L, d0, p.D, tid, NT);
-            load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
-            load_tile<E, DT>(sdy, dyb, t0, rows4, p.L, d0, p.D, tid, NT);
-            load_rows_f32<E, N>(sB, Bb, t0, rows4, p.L, tid, NT);
-            load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
-            __syncthreads();
-            // steps past the sequence end get delta = 0 (a = 1, no input): they pass state and
-            // adjoint through unchanged
-            for (int i = tid; i < rows4 * DT; i += NT)
-                sdel[i] = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
-            __syncthreads();
-
-            // pass A
-            const int nwin = (rows4 + TS - 1) / TS;
-            for (int k = 0; k < nwin; ++k) {
-                st_pairs_cg<S>(bnd + (size_t)k * NT * S, h);
-#pragma unroll
-                for (int ts = 0; ts < TS; ++ts) {
-                    const int r = k * TS + ts;
-                    if (TS > U && r >= rows4) break;
-                    const float dlt = sdel[r * DT + dl];
-                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    float2 bq[P2];
-                    ld_pairs<S>(bq, sB + r * N + n0);
-#pragma unroll
-                    for (int i = 0; i < P2; ++i)
-                        h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dlt), A2[i])), h[i], __fmul2_rn(f2(dxv), bq[i]));
+                __syncthreads();
+                const int t0 = tc + j * TTe;
+                const int rows = min(TTe, p.L - t0);
+                const E* sx = stage(k);
+                const E* sdr = sx + Sm::XE;
+                const E* sB = sx + 2 * Sm::XE;
+                // one exp per (t, d) gives delta and sigmoid; steps past the end get delta = 0
+                for (int i = tid; i < TTe * DT; i += NT) {
+                    const int r = i / DT;
+                    float dlt = 0.0f, sig = 0.0f;
+                    if (r < rows) {
+                        const float z = Elem<E>::to_f(sdr[i]);
+                        softplus_sigmoid(z, dlt, sig);
+                    }
+                    sdd[i] = make_float2(dlt, dlt * Elem<E>::to_f(sx[i]));
+                    __stcg(&dsg[(size_t)(j * TTe) * DT + i], make_float2(dlt, sig));
                 }
-            }
-
-            // pass B
-            float2 hw[P2];
-            ld_pairs_cg<S>(hw, bnd + (size_t)(nwin - 1) * NT * S);
-            for (int k = nwin - 1; k >= 0; --k) {
-                float2 aa[TS][P2], pp[TS][P2];
-                {
-                    float2 hc[P2];
+                for (int i = tid; i < TTe * N; i += NT) sBf[i] = Elem<E>::to_f(sB[i]);
+                __syncthreads();
+                for (int w = 0; w < TTe / W; ++w) {
+                    __stcg(reinterpret_cast<float4*>(bnd + (size_t)((j * TTe) / W + w) * NT * 4),
+                           make_float4(h[0].x, h[0].y, h[1].x, h[1].y));
 #pragma unroll
-                    for (int i = 0; i < P2; ++i) hc[i] = hw[i];
-                    if (k > 0) ld_pairs_cg<S>(hw, bnd + (size_t)(k - 1) * NT * S);  // prefetch
-#pragma unroll
-                    for (int ts = 0; ts < TS; ++ts) {
-                        const int r = k * TS + ts;
-                        const float dlt = (TS > U && r >= rows4) ? 0.0f : sdel[r * DT + dl];
-                        const float dxv = (TS > U && r >= rows4) ? 0.0f : dlt * Elem<E>::to_f(sx[r * DT + dl]);
+                    for (int u = 0; u < W; ++u) {
+                        const int r = w * W + u;
+                        const float2 dd = sdd[r * DT + dl];
                         float2 bq[P2];
-                        if (TS > U && r >= rows4) {
+                        ld_pairs<4>(bq, sBf + r * N + n0);
 #pragma unroll
-                            for (int i = 0; i < P2; ++i) bq[i] = make_float2(0.0f, 0.0f);
-                        } else {
-                            ld_pairs<S>(bq, sB + r * N + n0);
-                        }
-#pragma unroll
-                        for (int i = 0; i < P2; ++i) {
-                            const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
-                            const float2 pr = __fmul2_rn(a, hc[i]);
-                            aa[ts][i] = a;
-                            pp[ts][i] = pr;
-                            hc[i] = __ffma2_rn(f2(dxv), bq[i], pr);
-                        }
+                        for (int i = 0; i < P2; ++i)
+                            h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dd.x), A2[i])), h[i],
+                                              __fmul2_rn(f2(dd.y), bq[i]));
                     }
                 }
+                __syncthreads();  // stage k and sdd are free again
+            }
+        }
+
+        // ------------------------------------------------------------------ pass B
+        {
+            float* sBf = reinterpret_cast<float*>(smem + Sm::B_BF);
+            float* sCf = reinterpret_cast<float*>(smem + Sm::B_CF);
+            float* sred = reinterpret_cast<float*>(smem + Sm::B_RED);
+            auto stage = [&](int k) { return smem + k * Sm::B_STAGE; };
+            auto issue = [&](int j, int k) {
+                const int t0 = tc + j * TTe;
+                unsigned char* st = stage(k);
+                // (delta, sigma) of this chunk's rows, written by pass A (always in range)
+                {
+                    const float* src = reinterpret_cast<const float*>(dsg + (size_t)(j * TTe) * DT);
+                    float* dst = reinterpret_cast<float*>(st);
+                    for (int i = tid; i < TTe * DT * 2 / 4; i += NT)
+                        cp_async16(dst + 4 * i, src + 4 * i, true);
+                }
+                E* sx = reinterpret_cast<E*>(st + Sm::XE * 8);
+                cp_async_tile<E, DT>(sx, xb, t0, TTe, p.L, d0, p.D, tid, NT);
+                cp_async_tile<E, DT>(sx + Sm::XE, dyb, t0, TTe, p.L, d0, p.D, tid, NT);
+                cp_async_flat<E>(sx + 2 * Sm::XE, Bb, (size_t)t0 * N, TTe * N, (size_t)p.L * N, tid, NT);
+                cp_async_flat<E>(sx + 2 * Sm::XE + Sm::BE, Cb, (size_t)t0 * N, TTe * N, (size_t)p.L * N, tid, NT);
+                cp_async_commit();
+            };
+            __syncthreads();
+            issue(nsub - 1, (nsub - 1) & 1);
+            float2 hw[P2];  // state at the start of the next window to recompute
+            ld_pairs_cg<4>(hw, bnd + (size_t)((nsub - 1) * TTe / W + TTe / W - 1) * NT * 4);
+            for (int j = nsub - 1; j >= 0; --j) {
+                const int k = j & 1;
+                if (j > 0) {
+                    issue(j - 1, k ^ 1);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
+                __syncthreads();
+                const int t0 = tc + j * TTe;
+                const int rows = min(TTe, p.L - t0);
+                const float2* sds = reinterpret_cast<const float2*>(stage(k));
+                const E* sx = reinterpret_cast<const E*>(stage(k) + Sm::XE * 8);
+                const E* sdy = sx + Sm::XE;
+                const E* sB = sx + 2 * Sm::XE;
+                const E* sC = sB + Sm::BE;
+                for (int i = tid; i < TTe * N; i += NT) {
+                    sBf[i] = Elem<E>::to_f(sB[i]);
+                    sCf[i] = Elem<E>::to_f(sC[i]);
+                }
+                __syncthreads();
+                const int nw = TTe / W;  // 4 or 8 windows, even
+                const int wbase = (j * TTe) / W;
+
+                float2 aaA[W][P2], ppA[W][P2], aaB[W][P2], ppB[W][P2];
+                // recompute window `q` of this sub-tile from hw into (aa, pp); hw <- next start
+                auto recompute_step = [&](float2 (&aa)[W][P2], float2 (&pp)[W][P2], float2 (&hc)[P2],
+                                          int q, int u) {
+                    const int r = q * W + u;
+                    const float dlt = sds[r * DT + dl].x;
+                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
+                    float2 bq[P2];
+                    ld_pairs<4>(bq, sBf + r * N + n0);
 #pragma unroll
-                for (int g4 = TS / U - 1; g4 >= 0; --g4) {
-                    const int rg = k * TS + g4 * U;
-                    if (TS > U && rg >= rows4) continue;
-                    float sv[2 * U];
-#pragma unroll
-                    for (int u = U - 1; u >= 0; --u) {
-                        const int ts = g4 * U + u;
-                        const int r = rg + u;
-                        const float dlt = sdel[r * DT + dl];
-                        const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                        const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-                        float2 bq[P2], cq[P2];
-                        ld_pairs<S>(bq, sB + r * N + n0);
-                        ld_pairs<S>(cq, sC + r * N + n0);
-                        float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
-                        float2 rB[P2], rC[P2];
-#pragma unroll
-                        for (int i = 0; i < P2; ++i) {
-                            const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);
-                            const float2 hj = __ffma2_rn(f2(dxv), bq[i], pp[ts][i]);
-                            const float2 q = __fmul2_rn(g, pp[ts][i]);
-                            dA[i] = __ffma2_rn(f2(dlt), q, dA[i]);
-                            sa = __ffma2_rn(A[i], q, sa);
-                            sg = __ffma2_rn(g, bq[i], sg);
-                            rB[i] = __fmul2_rn(g, f2(dxv));
-                            rC[i] = __fmul2_rn(f2(dyv), hj);
-                            v[i] = __fmul2_rn(aa[ts][i], g);
-                        }
-                        sv[2 * u] = sg.x + sg.y;
-                        sv[2 * u + 1] = sa.x + sa.y;
-                        float* sr = sred + (u * DT + dl) * N2 + n0;
-                        st_pairs<S>(sr, rB);
-                        st_pairs<S>(sr + N, rC);
+                    for (int i = 0; i < P2; ++i) {
+                        const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
+                        const float2 pr = __fmul2_rn(a, hc[i]);
+                        aa[u][i] = a;
+                        pp[u][i] = pr;
+                        hc[i] = __ffma2_rn(f2(dxv), bq[i], pr);
                     }
-                    // per-channel sums over the NG lanes: lane ng gets steps [ng*U/NG, ...)
-                    reduce_scatter<2 * U, NG>(sv, ng);
+                };
+                auto reverse_step = [&](const float2 (&aa)[W][P2], const float2 (&pp)[W][P2], int q,
+                                        int uu, float (&sv)[2 * W], float* red) {
+                    const int r = q * W + uu;
+                    const float dlt = sds[r * DT + dl].x;
+                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
+                    const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
+                    float2 bq[P2], cq[P2];
+                    ld_pairs<4>(bq, sBf + r * N + n0);
+                    ld_pairs<4>(cq, sCf + r * N + n0);
+                    float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
+                    float2 rB[P2], rC[P2];
 #pragma unroll
-                    for (int j = 0; j < U / NG; ++j) {
-                        const int r = rg + ng * (U / NG) + j;
-                        if (r < rows) {
-                            const float dlt = sdel[r * DT + dl];
+                    for (int i = 0; i < P2; ++i) {
+                        const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);
+                        const float2 hj = __ffma2_rn(f2(dxv), bq[i], pp[uu][i]);
+                        const float2 qv = __fmul2_rn(g, pp[uu][i]);
+                        dA[i] = __ffma2_rn(f2(dlt), qv, dA[i]);
+                        sa = __ffma2_rn(A[i], qv, sa);
+                        sg = __ffma2_rn(g, bq[i], sg);
+                        rB[i] = __fmul2_rn(g, f2(dxv));
+                        rC[i] = __fmul2_rn(f2(dyv), hj);
+                        v[i] = __fmul2_rn(aa[uu][i], g);
+                    }
+                    sv[2 * uu] = sg.x + sg.y;
+                    sv[2 * uu + 1] = sa.x + sa.y;
+                    float* sr = red + (uu * DT + dl) * N2 + n0;
+                    st_pairs<4>(sr, rB);
+                    st_pairs<4>(sr + N, rC);
+                };
+                // after a window's reverse sweep: outputs, then its dB/dC column sums
+                auto finish_window = [&](int q, float (&sv)[2 * W], const float* red) {
+                    reduce_scatter<2 * W, NG>(sv, ng);
+#pragma unroll
+                    for (int jj = 0; jj < W / NG; ++jj) {
+                        const int uu = ng * (W / NG) + jj;
+                        const int r = q * W + uu;
+                        if (r < rows && dv) {
+                            const float2 ds = sds[r * DT + dl];
                             const float xv = Elem<E>::to_f(sx[r * DT + dl]);
                             const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-                            const float sgB = sv[2 * j], sAq = sv[2 * j + 1];
-                            const float sig = sigmoid_fast(Elem<E>::to_f(sdr[r * DT + dl]));
-                            sx[r * DT + dl] = Elem<E>::from_f(fmaf(dsk, dyv, dlt * sgB));
-                            sdr[r * DT + dl] = Elem<E>::from_f(fmaf(xv, sgB, sAq) * sig);
+                            const float sgB = sv[2 * jj], sAq = sv[2 * jj + 1];
+                            const size_t o = (size_t)(t0 + r) * p.D + d;
+                            dxb[o] = Elem<E>::from_f(fmaf(dsk, dyv, ds.x * sgB));
+                            ddrb[o] = Elem<E>::from_f(fmaf(xv, sgB, sAq) * ds.y);
                             dDacc = fmaf(dyv, xv, dDacc);
                         }
                     }
-                    __syncthreads();
-                    {   // dB, dC: sum the group's values over the CTA's channels
-                        const float* src = sred + (cs_u * DT + cs_part * (DT / Q)) * N2 + cs_o;
-                        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
+                    __syncthreads();  // the window's dB/dC values are in `red`
+                    const float* src = red + (cs_u * DT + cs_part * (DT / Q)) * N2 + cs_o;
+                    float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
 #pragma unroll
-                        for (int ch = 0; ch < DT / Q; ch += 2) {
-                            const float4 a0 = *reinterpret_cast<const float4*>(src + ch * N2);
-                            const float4 a1 = *reinterpret_cast<const float4*>(src + (ch + 1) * N2);
-                            s0 = __fadd2_rn(s0, make_float2(a0.x, a0.y));
-                            s1 = __fadd2_rn(s1, make_float2(a0.z, a0.w));
-                            s2 = __fadd2_rn(s2, make_float2(a1.x, a1.y));
-                            s3 = __fadd2_rn(s3, make_float2(a1.z, a1.w));
-                        }
-                        s0 = __fadd2_rn(s0, s2);
-                        s1 = __fadd2_rn(s1, s3);
-#pragma unroll
-                        for (int m = 8; m < 8 * Q; m <<= 1) {
-                            s0.x += __shfl_xor_sync(kFull, s0.x, m);
-                            s0.y += __shfl_xor_sync(kFull, s0.y, m);
-                            s1.x += __shfl_xor_sync(kFull, s1.x, m);
-                            s1.y += __shfl_xor_sync(kFull, s1.y, m);
-                        }
-                        const int r = rg + cs_u;
-                        if (cs_part == 0 && r < rows)
-                            *reinterpret_cast<float4*>(partb + (size_t)(t0 + r) * N2 + cs_o) =
-                                make_float4(s0.x, s0.y, s1.x, s1.y);
+                    for (int ch = 0; ch < DT / Q; ch += 2) {
+                        const float4 a0 = *reinterpret_cast<const float4*>(src + ch * N2);
+                        const float4 a1 = *reinterpret_cast<const float4*>(src + (ch + 1) * N2);
+                        s0 = __fadd2_rn(s0, make_float2(a0.x, a0.y));
+                        s1 = __fadd2_rn(s1, make_float2(a0.z, a0.w));
+                        s2 = __fadd2_rn(s2, make_float2(a1.x, a1.y));
+                        s3 = __fadd2_rn(s3, make_float2(a1.z, a1.w));
                     }
-                    __syncthreads();
+                    s0 = __fadd2_rn(s0, s2);
+                    s1 = __fadd2_rn(s1, s3);
+#pragma unroll
+                    for (int m = 8; m < 8 * Q; m <<= 1) {
+                        s0.x += __shfl_xor_sync(kFull, s0.x, m);
+                        s0.y += __shfl_xor_sync(kFull, s0.y, m);
+                        s1.x += __shfl_xor_sync(kFull, s1.x, m);
+                        s1.y += __shfl_xor_sync(kFull, s1.y, m);
+                    }
+                    const int r = q * W + cs_u;
+                    if (cs_part == 0 && r < rows)
+                        *reinterpret_cast<float4*>(partb + (size_t)(t0 + r) * N2 + cs_o) =
+                            make_float4(s0.x, s0.y, s1.x, s1.y);
+                };
+
+                // prologue: recompute the last window of the sub-tile
+                {
+                    float2 hc[P2] = {hw[0], hw[1]};
+                    if (nw >= 2) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + nw - 2) * NT * 4);
+#pragma unroll
+                    for (int u = 0; u < W; ++u) recompute_step(aaA, ppA, hc, nw - 1, u);
                 }
+                for (int q = nw - 1; q >= 1; q -= 2) {
+                    // reverse window q (set A) while recomputing window q-1 (set B)
+                    {
+                        float sv[2 * W];
+                        float* red = sred + (q & 1) * W * DT * N2;
+                        float2 hc[P2] = {hw[0], hw[1]};
+                        if (q >= 2) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 2) * NT * 4);
+#pragma unroll
+                        for (int u = 0; u < W; ++u) {
+                            reverse_step(aaA, ppA, q, W - 1 - u, sv, red);
+                            recompute_step(aaB, ppB, hc, q - 1, u);
+                        }
+                        finish_window(q, sv, red);
+                    }
+                    // reverse window q-1 (set B) while recomputing window q-2 (set A)
+                    {
+                        float sv[2 * W];
+                        float* red = sred + ((q - 1) & 1) * W * DT * N2;
+                        if (q >= 2) {
+                            float2 hc[P2] = {hw[0], hw[1]};
+                            if (q >= 3) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 3) * NT * 4);
+#pragma unroll
+                            for (int u = 0; u < W; ++u) {
+                                reverse_step(aaB, ppB, q - 1, W - 1 - u, sv, red);
+                                recompute_step(aaA, ppA, hc, q - 2, u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < W; ++u) reverse_step(aaB, ppB, q - 1, W - 1 - u, sv, red);
+                        }
+                        finish_window(q - 1, sv, red);
+                    }
+                }
+                // state at the start of the last window of the previous sub-tile
+                if (j > 0) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase - 1) * NT * 4);
+                __syncthreads();  // stage k, sBf/sCf and sred are free again
             }
-            store_tile<E, DT>(dxb, sx, t0, rows, p.L, d0, p.D, tid, NT);
-            store_tile<E, DT>(ddrb, sdr, t0, rows, p.L, d0, p.D, tid, NT);
         }
     }
     // each lane of a channel accumulated dD over its own subset of steps
@@ -350,9 +460,9 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_kernel(RealArgs p)
     for (int m = 1; m < NG; m <<= 1) dDacc += __shfl_xor_sync(kFull, dDacc, m);
     if (dv) {
         const size_t o = (((size_t)b * p.nseg + seg) * p.D + d) * N + n0;
-        st_pairs<S>(p.dA_part + o, dA);
+        st_pairs<4>(p.dA_part + o, dA);
         if (ng == 0) p.dD_part[((size_t)b * p.nseg + seg) * p.D + d] = dDacc;
-        if (!all_finite<S>(v)) flag_status(p.status, kStatusNonFinite);
+        if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
     }
 }
 
@@ -395,36 +505,28 @@ template <int N, int S>
 size_t bwd_summary_smem(int T, int esz) {
     return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 + (size_t)T * kRealDT * 4;
 }
-template <int N, int S>
-size_t bwd_smem(int T, int esz) {
-    const int TB = T < kRealMaxTB ? T : kRealMaxTB;
-    return (size_t)TB * kRealDT * esz * 3 + (size_t)TB * N * 4 * 2 + (size_t)TB * kRealDT * 4 +
-           (size_t)RealCfg<N, S>::U * kRealDT * 2 * N * 4;
-}
-
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename E, int N, int S>
+template <typename E, int N>
 cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
-    const dim3 block(RealCfg<N, S>::NT);
     const int esz = (int)sizeof(E);
     cudaError_t e;
     if (a.nseg > 1) {
-        const size_t sm = bwd_summary_smem<N, S>(a.T, esz);
-        if ((e = set_smem(real_bwd_summary_kernel<E, N, S>, sm)) != cudaSuccess) return e;
-        real_bwd_summary_kernel<E, N, S><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
+        const size_t sm = bwd_summary_smem<N, 4>(a.T, esz);
+        if ((e = set_smem(real_bwd_summary_kernel<E, N, 4>, sm)) != cudaSuccess) return e;
+        real_bwd_summary_kernel<E, N, 4><<<dim3(a.ndt, a.B, a.nseg - 1), dim3(RealCfg<N, 4>::NT), sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
                                                                             a.gsumP, a.gsumG, a.vin);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t sm = bwd_smem<N, S>(a.T, esz);
-    if ((e = set_smem(real_bwd_kernel<E, N, S>, sm)) != cudaSuccess) return e;
-    real_bwd_kernel<E, N, S><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
+    const size_t sm = BwdSmem<E, N>::BYTES;
+    if ((e = set_smem(real_bwd_kernel<E, N>, sm)) != cudaSuccess) return e;
+    real_bwd_kernel<E, N><<<dim3(a.ndt, a.B, a.nseg), dim3(BwdCfg<N>::NT), sm, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t nbc = (int64_t)a.B * a.L * 2 * N;
     if (nbc > 0) {
@@ -438,9 +540,9 @@ cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
 
 template <typename E>
 cudaError_t bwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
-    if (N == 4) return real_bwd_impl<E, 4, 4>(a, st);
-    if (N == 8) return real_bwd_impl<E, 8, kRealStates8>(a, st);
-    return real_bwd_impl<E, 16, kRealStates16>(a, st);
+    if (N == 4) return real_bwd_impl<E, 4>(a, st);
+    if (N == 8) return real_bwd_impl<E, 8>(a, st);
+    return real_bwd_impl<E, 16>(a, st);
 }
 
 }  // namespace

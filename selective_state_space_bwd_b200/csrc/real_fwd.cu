@@ -47,42 +47,6 @@ struct FwdSmem {
     static constexpr int BYTES = Y + XE * (int)sizeof(E);
 };
 
-// 1-D asynchronous copy of elements [e0, e0 + ne) of a contiguous array of `etotal` elements,
-// zero-filling past the end.  ne * sizeof(E) is a multiple of 16.  The pieces are 16 bytes when
-// the source start is 16-byte aligned, else 8 or 4 bytes (a [B, L, N] bf16 array with N = 4 and
-// odd L starts odd batch rows on an 8-byte boundary).
-template <int G, typename E>
-__device__ __forceinline__ void cp_async_pieces(E* __restrict__ dst, const E* __restrict__ src,
-                                                size_t e0, int ne, size_t etotal, int tid,
-                                                int nthreads) {
-    constexpr int VEC = G / sizeof(E);
-    for (int i = tid; i < ne / VEC; i += nthreads) {
-        const size_t e = e0 + (size_t)i * VEC;
-        const size_t left = e < etotal ? etotal - e : 0;
-        const int bytes = left >= (size_t)VEC ? G : (int)(left * sizeof(E));
-        const unsigned s = (unsigned)__cvta_generic_to_shared(dst + i * VEC);
-        const E* g = bytes > 0 ? src + e : src;
-        if (G == 16)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(g), "r"(bytes));
-        else if (G == 8)
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(g), "r"(bytes));
-        else
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(g), "r"(bytes));
-    }
-}
-template <typename E>
-__device__ __forceinline__ void cp_async_flat(E* __restrict__ dst, const E* __restrict__ src,
-                                              size_t e0, int ne, size_t etotal, int tid,
-                                              int nthreads) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(src + e0);
-    if ((a & 15) == 0)
-        cp_async_pieces<16>(dst, src, e0, ne, etotal, tid, nthreads);
-    else if ((a & 7) == 0)
-        cp_async_pieces<8>(dst, src, e0, ne, etotal, tid, nthreads);
-    else
-        cp_async_pieces<4>(dst, src, e0, ne, etotal, tid, nthreads);
-}
-
 // SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end state).
 // SUMMARY = false: the scan from the segment's entering state, writing y and checkpoints.
 template <typename E, int N, bool SUMMARY>

@@ -44,6 +44,20 @@ __device__ __forceinline__ float softplus_fast(float z) {
     return fmaf(s, q, fmaxf(z, 0.0f));
 }
 
+// softplus(z) and sigmoid(z) = d softplus / dz from one shared exp(-|z|).
+__device__ __forceinline__ void softplus_sigmoid(float z, float& sp, float& sg) {
+    const float e = ex2_mufu(-fabsf(z) * kLog2e);
+    const float s = __fdividef(e, 2.0f + e);
+    const float w = s * s;
+    float q = fmaf(w, 0.28011780977249146f, 0.2800184488296509f);
+    q = fmaf(w, q, 0.4002152383327484f);
+    q = fmaf(w, q, 0.666664183139801f);
+    q = fmaf(w, q, 2.0f);
+    sp = fmaf(s, q, fmaxf(z, 0.0f));
+    const float r = __fdividef(1.0f, 1.0f + e);
+    sg = z >= 0.0f ? r : e * r;
+}
+
 // sigmoid(z) = 1 / (1 + exp(-z)) from e = exp(-|z|); within ~5e-7 relative.
 __device__ __forceinline__ float sigmoid_fast(float z) {
     const float e = ex2_mufu(-fabsf(z) * kLog2e);

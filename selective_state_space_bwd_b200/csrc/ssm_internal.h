@@ -7,22 +7,16 @@
 
 namespace ssm {
 
-// Thread layout of the real-mode kernels: every thread owns S consecutive states of one channel
-// (S = 4 or 8 for N = 16), NG = N / S adjacent lanes cover a channel, a CTA covers DT = 32
-// channels with 32 * NG threads.  The backward holds a window of TS steps of (a_t, a_t h_{t-1})
-// per state in registers (TS * S = 32) and parks the state at every window start in an
-// L2-resident scratch region of the workspace.
+// Real-mode kernels: a thread owns 4 consecutive states of one channel, N / 4 adjacent lanes
+// cover a channel and a CTA covers kRealDT channels of one batch row.
 constexpr int kRealDT = 32;
-constexpr int kRealMaxTB = 128;  // longest stretch of steps the backward stages at once
-constexpr int kRealStates16 = 4;
-constexpr int kRealStates8 = 4;
 
 inline int real_dt(int) { return kRealDT; }
-inline int real_states(int N) { return N == 16 ? kRealStates16 : (N == 8 ? kRealStates8 : 4); }
-inline int real_threads(int N) { return kRealDT * (N / real_states(N)); }
-inline int real_window(int N) { return real_states(N) == 4 ? 8 : 4; }
-inline size_t real_bnd_floats_per_cta(int N) {
-    return (size_t)(kRealMaxTB / real_window(N)) * real_threads(N) * real_states(N);
+
+// Backward scratch per CTA (floats): the state at every 4-step window start of one chunk
+// ([T/4][threads][4]) and (delta, sigmoid(delta_raw)) of one chunk ([T][32] float2).
+__host__ __device__ inline size_t real_bwd_scratch_floats(int N, int T) {
+    return (size_t)T * (kRealDT * (N / 4)) + (size_t)T * kRealDT * 2;
 }
 
 // Complex mode: one thread per mode, kCplxKT modes per CTA, kCplxTT steps staged per tile.
@@ -52,7 +46,7 @@ struct RealArgs {
     float* dBC_part;  // [ndt][B][L][2N] per-CTA sums over its channels (dB then dC)
     float* dA_part;   // [B][nseg][D][N] sum over the segment of delta * q
     float* dD_part;   // [B][nseg][D]
-    float* bnd_scratch;  // per-CTA window-start states of the backward (L2-resident)
+    float* bnd_scratch;  // per-CTA backward scratch (L2-resident), real_bwd_scratch_floats each
     void* dB;
     void* dC;
     float* dA_log;
