@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seg-chunks", type=int, default=0)
+    ap.add_argument("--memory-curve", action="store_true",
+                    help="peak device memory of fwd+bwd vs L for the stiff workload's shape")
     return ap.parse_args()
 
 
@@ -143,6 +145,63 @@ def oracle_sample(w, inp, budget_s=(10.0, 30.0)):
                       f"fwd+bwd in float64, {t_total:.1f} s"}
 
 
+def measured_traffic(kernel_file, workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu capture summary,
+    if that capture was taken on the current kernel source; else None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p))
+        src = open(os.path.join(ROOT, "selective_state_space_bwd_b200", "csrc", kernel_file), "rb").read()
+        if rec.get("workload") != workload or rec.get("source_sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def memory_curve():
+    """Peak device memory of one fwd+bwd at the stiff workload's width (B=1, D=1024, N=16,
+    fp32, T=128) for growing L, minus the inputs and outputs themselves."""
+    import torch
+    from selective_state_space_bwd_b200 import build, ssm_scan as S
+    build.build()
+    dev = torch.device("cuda", 0)
+    B, D, N, T = 1, 1024, 16, 128
+    rows = []
+    for L in (8000, 16000, 32000, 64000, 128000):
+        torch.cuda.empty_cache()
+        x = torch.randn(B, L, D, device=dev)
+        dr = torch.rand(B, L, D, device=dev) * 7.4 - 6.9
+        dy = torch.randn(B, L, D, device=dev)
+        A_log = torch.rand(D, N, device=dev) * 4.6 - 0.7
+        Bm, Cm = torch.randn(B, L, N, device=dev), torch.randn(B, L, N, device=dev)
+        Dskip = torch.randn(D, device=dev)
+        y = torch.empty_like(x)
+        out = dict(dx=torch.empty_like(x), ddelta_raw=torch.empty_like(x),
+                   dA_log=torch.empty_like(A_log), dB=torch.empty_like(Bm), dC=torch.empty_like(Cm),
+                   dD=torch.empty_like(Dskip))
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        y, ck = S.ssm_scan_fwd(x, dr, A_log, Bm, Cm, Dskip, chunk=T, y=y)
+        S.ssm_scan_bwd(x, dr, A_log, Bm, Cm, Dskip, ck, dy, chunk=T, out=out)
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated() - base
+        shape = S.real_shape(B, L, D, N, T, S.SSM_F32)
+        rows.append({"L": L, "extra_peak_bytes": peak,
+                     "checkpoint_bytes": S.checkpoint_bytes(shape),
+                     "fwd_workspace_bytes": S.workspace_bytes(shape, False),
+                     "bwd_workspace_bytes": S.workspace_bytes(shape, True),
+                     "every_state_bytes": L * D * N * 4})
+        del x, dr, dy, Bm, Cm, y, out, ck
+    print(json.dumps({"metric": "peak device memory beyond inputs/outputs, fwd+bwd",
+                      "shape": {"batch": B, "dim": D, "dstate": N, "chunk": T, "io": "f32"},
+                      "curve": rows}), flush=True)
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -178,6 +237,8 @@ def run_reference(args, w):
 
 def main():
     args = parse()
+    if args.memory_curve:
+        return memory_curve()
     from selective_state_space_bwd_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
     if isinstance(w, gen.ComplexWorkload):
@@ -187,7 +248,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from selective_state_space_bwd_b200 import build, ssm_scan as S
+    from selective_state_space_bwd_b200 import build, dp, ssm_scan as S
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -236,9 +297,7 @@ def main():
 
     def allreduce():
         if world > 1:
-            gbuf[: w.dim * w.dstate].copy_(out["dA_log"].view(-1))
-            gbuf[w.dim * w.dstate:].copy_(out["dD"])
-            dist.all_reduce(gbuf)
+            dp.allreduce_param_grads(out["dA_log"], out["dD"], buf=gbuf)
 
     for _ in range(max(3, args.warmup)):
         fwd(); bwd(); allreduce()
@@ -323,7 +382,8 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "ssm_scan_bwd (chunk-recompute adjoint + "
                          "fixed-order reductions)", "achieved": bwd_gbs, "peak": hbm,
                          "unit": "GB/s", "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+                         "algorithmic_bytes_per_launch": bb,
+                         "traffic": measured_traffic("real_bwd.cu", w.name)},
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_step": step_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,

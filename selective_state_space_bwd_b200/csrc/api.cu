@@ -37,6 +37,9 @@ int pick_segments(int64_t ctas_per_seg, int nC, int forced, int* seg_chunks) {
 
 struct RealPlan {
     int B, L, D, N, T, nC, ndt, seg_chunks, nseg, esz;
+    // backward: its own segmentation (see real_bwd_impl): b_nseg segments of b_seg_chunks
+    // chunks, concurrent (b_seq = 0, b_group per launch) or sequential blocks (b_seq = 1)
+    int b_nseg, b_seg_chunks, b_seq, b_group, b_rows, b_launches;
     // workspace offsets (bytes); fwd and bwd use separate layouts
     size_t f_sumP, f_sumS, f_hin, f_end;
     size_t b_gP, b_gG, b_vin, b_part, b_dA, b_dD, b_bnd, b_end;
@@ -72,14 +75,60 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->f_sumS = o; o = align256(o + summ);
     p->f_hin = o;  o = align256(o + (S > 1 ? B * S * DN * 4 : 0));
     p->f_end = o;
+
+    // Backward.  The per-CTA dB/dC partial sums cover the steps of one launch; time is walked
+    // in launches whose partial buffer fits max(checkpoint bytes, 128 MiB), so the backward's
+    // memory stays O(L / T) however long the sequence.
+    const size_t per_chunk = (size_t)p->ndt * B * p->T * 2 * p->N * 4;
+    const size_t ckpt = B * (size_t)p->nC * DN * 4;
+    const size_t cap = ckpt > ((size_t)128 << 20) ? ckpt : ((size_t)128 << 20);
+    const int64_t ctas_per_seg = (int64_t)B * p->ndt;
+    const size_t chunks_cap = per_chunk > 0 ? cap / per_chunk : (size_t)p->nC;  // per launch
+    const int nC1 = p->nC > 0 ? p->nC : 1;
+    auto clampi = [](size_t v, size_t lo, size_t hi) { return (int)(v < lo ? lo : (v > hi ? hi : v)); };
+    if (s->seg_chunks > 0) {
+        // forced time split: concurrent segments, as many per launch as the cap allows
+        p->b_seg_chunks = s->seg_chunks < nC1 ? s->seg_chunks : nC1;
+        p->b_nseg = (nC1 + p->b_seg_chunks - 1) / p->b_seg_chunks;
+        p->b_seq = 0;
+        p->b_group = clampi(chunks_cap / p->b_seg_chunks, 1, p->b_nseg);
+    } else if (ctas_per_seg >= kTargetCtas || nC1 <= 1) {
+        // enough CTAs without splitting time: one pass, or sequential blocks if the partial sums
+        // of the whole sequence would exceed the cap
+        if (chunks_cap >= (size_t)nC1) {
+            p->b_nseg = 1;
+            p->b_seg_chunks = nC1;
+            p->b_seq = 0;
+        } else {
+            p->b_seg_chunks = clampi(chunks_cap, 1, nC1);
+            p->b_nseg = (nC1 + p->b_seg_chunks - 1) / p->b_seg_chunks;
+            p->b_seq = 1;
+        }
+        p->b_group = 1;
+    } else {
+        // few CTAs: concurrent segments (summary + carry), `g` of them per launch for
+        // parallelism, each short enough that a launch's partial sums fit the cap
+        const int g = (int)((kTargetCtas + ctas_per_seg - 1) / ctas_per_seg);
+        p->b_seg_chunks = clampi(chunks_cap / g, 1, (size_t)((nC1 + g - 1) / g));
+        p->b_nseg = (nC1 + p->b_seg_chunks - 1) / p->b_seg_chunks;
+        p->b_seq = 0;
+        p->b_group = g < p->b_nseg ? g : p->b_nseg;
+    }
+    if (p->b_nseg > 65535) return SSM_ERR_UNSUPPORTED;
+    const size_t BS = p->b_nseg;
+    const int per = p->b_seq ? 1 : p->b_group;
+    p->b_launches = (p->b_nseg + per - 1) / per;
+    const size_t rows = (size_t)per * p->b_seg_chunks * p->T;
+    p->b_rows = (int)(rows < (size_t)p->L ? rows : (size_t)p->L);
+    const size_t bsumm = (BS > 1 && !p->b_seq) ? B * (BS - 1) * DN * 4 : 0;
     o = kStatusBytes;
-    p->b_gP = o;   o = align256(o + summ);
-    p->b_gG = o;   o = align256(o + summ);
-    p->b_vin = o;  o = align256(o + (S > 1 ? B * S * DN * 4 : 0));
-    p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->L * 2 * p->N * 4);
-    p->b_dA = o;   o = align256(o + B * S * DN * 4);
-    p->b_dD = o;   o = align256(o + B * S * (size_t)p->D * 4);
-    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * S * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
+    p->b_gP = o;   o = align256(o + bsumm);
+    p->b_gG = o;   o = align256(o + bsumm);
+    p->b_vin = o;  o = align256(o + (BS > 1 ? B * BS * DN * 4 : 0));
+    p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->b_rows * 2 * p->N * 4);
+    p->b_dA = o;   o = align256(o + B * BS * DN * 4);
+    p->b_dD = o;   o = align256(o + B * BS * (size_t)p->D * 4);
+    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * per * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
     p->b_end = o;
     return SSM_OK;
 }
@@ -207,7 +256,8 @@ int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, c
     }
     ssm::RealArgs a = {};
     a.B = p.B; a.L = p.L; a.D = p.D; a.T = p.T; a.nC = p.nC;
-    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.ndt = p.ndt;
+    a.seg_chunks = p.b_seg_chunks; a.nseg = p.b_nseg; a.ndt = p.ndt;
+    a.seq_blocks = p.b_seq; a.part_rows = p.b_rows;
     a.x = x; a.draw = delta_raw; a.A_log = A_log; a.Bm = Bm; a.Cm = Cm; a.Dskip = Dskip;
     a.ckpt_in = ckpt; a.dy = dy; a.dx = dx; a.ddraw = ddelta_raw;
     a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.vin = at<float>(ws, p.b_vin);
@@ -216,16 +266,18 @@ int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, c
     a.bnd_scratch = at<float>(ws, p.b_bnd);
     a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
     a.status = at<unsigned>(ws, 0);
-    return ssm::launch_real_bwd(a, shape->io == SSM_BF16, p.N, s) == cudaSuccess ? SSM_OK
-                                                                                : SSM_ERR_CUDA;
+    return ssm::launch_real_bwd(a, shape->io == SSM_BF16, p.N, p.b_group, s) == cudaSuccess
+               ? SSM_OK
+               : SSM_ERR_CUDA;
 }
 
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward) {
     RealPlan p;
     if (plan_real(shape, &p) != SSM_OK) return -1;
     if (p.B == 0 || p.L == 0) return 0;
-    const int seg = p.nseg > 1 ? 2 : 0;  // segment summary + carry
-    return backward ? 3 + seg : 1 + seg;  // bwd: main + dB/dC reduce + dA_log/dD reduce
+    if (!backward) return p.nseg > 1 ? 3 : 1;  // [segment summary + carry] + scan
+    // [summary + carry] + per launch (main + dB/dC reduce) + dA_log/dD reduce
+    return (p.b_nseg > 1 && !p.b_seq ? 2 : 0) + 2 * p.b_launches + 1;
 }
 
 int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward) {

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     extern __shared__ __align__(16) unsigned char smem[];
 
     const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
-    const int b = blockIdx.y, seg = blockIdx.z;
+    const int b = blockIdx.y, seg = p.seg0 + blockIdx.z;
     const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * Cfg::S;
     const bool dv = d < p.D;
     const int T = p.T;
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     const E* Cb = static_cast<const E*>(p.Cm) + boff * N;
     E* dxb = static_cast<E*>(p.dx) + boff * p.D;
     E* ddrb = static_cast<E*>(p.ddraw) + boff * p.D;
-    float* partb = p.dBC_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L * N2;
+    float* partb = p.dBC_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.part_rows * N2 -
+                   (size_t)p.part_t0 * N2;  // indexed by absolute step t
     const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
     float* scr = p.bnd_scratch + cta * real_bwd_scratch_floats(N, T);
     float* bnd = scr + (size_t)tid * 4;                        // window starts: [T/W][NT][4]
@@ -462,22 +463,29 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
         const size_t o = (((size_t)b * p.nseg + seg) * p.D + d) * N + n0;
         st_pairs<4>(p.dA_part + o, dA);
         if (ng == 0) p.dD_part[((size_t)b * p.nseg + seg) * p.D + d] = dDacc;
+        // sequential blocks: the adjoint leaving this block's start enters the previous block
+        if (p.seq_blocks && seg > 0)
+            st_pairs<4>(p.vin + (((size_t)b * p.nseg + (seg - 1)) * p.D + d) * N + n0, v);
         if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
     }
 }
 
-// dB, dC: fixed-order sums of the per-CTA partials over the channel tiles.
+// dB, dC for the steps [part_t0, part_t0 + rows) of the current launch: fixed-order sums of the
+// per-CTA partials over the channel tiles.
 template <typename E, int N>
-__global__ void real_reduce_dbc_kernel(RealArgs p) {
+__global__ void real_reduce_dbc_kernel(RealArgs p, int rows) {
     constexpr int N2 = 2 * N;
-    const int64_t total = (int64_t)p.B * p.L * N2;
+    const int64_t total = (int64_t)p.B * rows * N2;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= total) return;
-    const int64_t bl = i / N2;
-    const int o = (int)(i - bl * N2);
-    const size_t stride = (size_t)p.B * p.L * N2;
+    const int o = (int)(i % N2);
+    const int64_t r = (i / N2) % rows;
+    const int64_t b = i / ((int64_t)N2 * rows);
+    const size_t stride = (size_t)p.B * p.part_rows * N2;
+    const float* src = p.dBC_part + ((size_t)b * p.part_rows + r) * N2 + o;
     float s = 0.0f;
-    for (int t = 0; t < p.ndt; ++t) s += p.dBC_part[(size_t)t * stride + i];
+    for (int t = 0; t < p.ndt; ++t) s += src[(size_t)t * stride];
+    const size_t bl = (size_t)b * p.L + p.part_t0 + r;
     if (o < N)
         static_cast<E*>(p.dB)[bl * N + o] = Elem<E>::from_f(s);
     else
@@ -510,11 +518,18 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Launch plan: segments [0, nseg) of seg_chunks chunks each.  Concurrent segments (seq_blocks
+// == 0) get their entering adjoints from the summary + carry pass and run `group` segments per
+// launch; sequential blocks (seq_blocks == 1) run one per launch from the end, each writing the
+// adjoint entering the previous one.  Either way the dB/dC partial buffer holds the rows of one
+// launch only, so its size does not grow with L.
 template <typename E, int N>
-cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
+cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
     const int esz = (int)sizeof(E);
     cudaError_t e;
-    if (a.nseg > 1) {
+    RealArgs a = a0;
+    if (a.nseg > 1 && !a.seq_blocks) {
+        a.seg0 = 1;
         const size_t sm = bwd_summary_smem<N, 4>(a.T, esz);
         if ((e = set_smem(real_bwd_summary_kernel<E, N, 4>, sm)) != cudaSuccess) return e;
         real_bwd_summary_kernel<E, N, 4><<<dim3(a.ndt, a.B, a.nseg - 1), dim3(RealCfg<N, 4>::NT), sm, st>>>(a);
@@ -526,12 +541,20 @@ cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
     }
     const size_t sm = BwdSmem<E, N>::BYTES;
     if ((e = set_smem(real_bwd_kernel<E, N>, sm)) != cudaSuccess) return e;
-    real_bwd_kernel<E, N><<<dim3(a.ndt, a.B, a.nseg), dim3(BwdCfg<N>::NT), sm, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int64_t nbc = (int64_t)a.B * a.L * 2 * N;
-    if (nbc > 0) {
-        real_reduce_dbc_kernel<E, N><<<(unsigned)((nbc + 255) / 256), 256, 0, st>>>(a);
+    const int per = a.seq_blocks ? 1 : group;
+    for (int hi = a.nseg; hi > 0; hi -= per) {
+        const int lo = hi - per > 0 ? hi - per : 0;
+        a.seg0 = lo;
+        a.part_t0 = lo * a.seg_chunks * a.T;
+        const int t_hi = min(a.L, hi * a.seg_chunks * a.T);
+        const int rows = t_hi - a.part_t0;
+        real_bwd_kernel<E, N><<<dim3(a.ndt, a.B, hi - lo), dim3(BwdCfg<N>::NT), sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t nbc = (int64_t)a.B * rows * 2 * N;
+        if (nbc > 0) {
+            real_reduce_dbc_kernel<E, N><<<(unsigned)((nbc + 255) / 256), 256, 0, st>>>(a, rows);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
     }
     const int64_t np = (int64_t)a.D * N;
     real_reduce_params_kernel<<<(unsigned)((np + 255) / 256), 256, 0, st>>>(a, N);
@@ -539,17 +562,18 @@ cudaError_t real_bwd_impl(const RealArgs& a, cudaStream_t st) {
 }
 
 template <typename E>
-cudaError_t bwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
-    if (N == 4) return real_bwd_impl<E, 4>(a, st);
-    if (N == 8) return real_bwd_impl<E, 8>(a, st);
-    return real_bwd_impl<E, 16>(a, st);
+cudaError_t bwd_dispatch(const RealArgs& a, int N, int group, cudaStream_t st) {
+    if (N == 4) return real_bwd_impl<E, 4>(a, group, st);
+    if (N == 8) return real_bwd_impl<E, 8>(a, group, st);
+    return real_bwd_impl<E, 16>(a, group, st);
 }
 
 }  // namespace
 }  // namespace real
 
-cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st) {
-    return io_bf16 ? real::bwd_dispatch<__nv_bfloat16>(a, N, st) : real::bwd_dispatch<float>(a, N, st);
+cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cudaStream_t st) {
+    return io_bf16 ? real::bwd_dispatch<__nv_bfloat16>(a, N, group, st)
+                   : real::bwd_dispatch<float>(a, N, group, st);
 }
 
 }  // namespace ssm

@@ -43,10 +43,15 @@ struct RealArgs {
     float* gsumP;     // backward segment summaries [B][nseg-1][D][N] (segments 1..nseg-1)
     float* gsumG;
     float* vin;       // scaled adjoint a_{t+1} g_{t+1} entering each segment from its end
-    float* dBC_part;  // [ndt][B][L][2N] per-CTA sums over its channels (dB then dC)
+    float* dBC_part;  // [ndt][B][part_rows][2N] per-CTA sums over its channels (dB then dC),
+                      // rows relative to part_t0 (the first step of the current launch)
     float* dA_part;   // [B][nseg][D][N] sum over the segment of delta * q
     float* dD_part;   // [B][nseg][D]
     float* bnd_scratch;  // per-CTA backward scratch (L2-resident), real_bwd_scratch_floats each
+    int seg0;         // backward: first segment handled by this launch (blockIdx.z offset)
+    int seq_blocks;   // backward: segments run as sequential launches, each handing its
+                      // entering adjoint to the next through vin
+    int part_t0, part_rows;
     void* dB;
     void* dC;
     float* dA_log;
@@ -82,7 +87,7 @@ struct CplxArgs {
 
 // Launchers (return cudaGetLastError() of the last launch).
 cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st);
-cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st);
+cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cudaStream_t st);
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st);
 cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st);
 

@@ -59,10 +59,22 @@ def test_checkpoint_and_workspace_sizes(S, B, L, D, N, T):
     assert S.checkpoint_bytes(shp) == B * nC * D * N * 4
     fw, bw = S.workspace_bytes(shp, False), S.workspace_bytes(shp, True)
     assert fw >= 256 and bw >= 256 and fw % 256 == 0 and bw % 256 == 0
-    # backward workspace holds at least the per-channel-tile dB/dC partials
-    DT = 32
-    ndt = -(-D // DT)
-    assert bw >= ndt * B * L * 2 * N * 4
+    # the backward's dB/dC partial sums cover one launch's steps, capped at
+    # max(checkpoint bytes, 128 MiB); the rest of its workspace is per-CTA scratch
+    cap = max(S.checkpoint_bytes(shp), 128 << 20)
+    assert bw <= cap + (160 << 20)
+
+
+def test_backward_workspace_is_o_of_l_over_t(S):
+    """Growing L 4x at the stiff workload's width grows the backward workspace by no more than
+    the checkpoints grow (the O(L/T) memory of the chunk-tiled backward)."""
+    a = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
+    b = S.real_shape(1, 512000, 1024, 16, 128, S.SSM_F32)
+    dw = S.workspace_bytes(b, True) - S.workspace_bytes(a, True)
+    dc = S.checkpoint_bytes(b) - S.checkpoint_bytes(a)
+    assert dw <= dc
+    every_state = 512000 * 1024 * 16 * 4
+    assert S.workspace_bytes(b, True) + S.checkpoint_bytes(b) < every_state / 10
 
 
 def test_segment_knob_changes_only_workspace(S):
@@ -147,8 +159,14 @@ def test_status_null_workspace(S):
 def test_kernel_launch_counts(S):
     one = S.real_shape(8, 2048, 1536, 16, 128, S.SSM_BF16)        # enough CTAs: no time split
     assert S.kernel_launches(one, False) == 1 and S.kernel_launches(one, True) == 3
-    split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)     # few CTAs: segment + carry
-    assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 5
+    # few CTAs: concurrent segments + carry; the backward uses 40 shorter segments (25 chunks),
+    # 10 per launch (320 CTAs) so that each launch's dB/dC partial sums stay under the cap:
+    # summary + carry + 4 x (main + reduce) + params = 11
+    split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
+    assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 11
+    # long and wide: the backward walks time in 4 sequential blocks
+    blocks = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)
+    assert S.kernel_launches(blocks, False) == 1 and S.kernel_launches(blocks, True) == 9
     assert S.kernel_launches(S.real_shape(2, 0, 32, 16, 128), True) == 0
     assert S.kernel_launches(S.real_shape(2, 8, 32, 12, 128), True) == -1
     assert S.complex_kernel_launches(S.complex_shape(16, 4096, 2048, 128), True) == 3
