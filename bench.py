@@ -57,6 +57,26 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+# FP32-pipe lane operations per state update (an FMA counts as one), the minimum the arithmetic
+# of the method needs, with per-(t, d) and per-(t, n) terms (O(1/N), O(1/D)) left out:
+#   forward:  delta*A'; u*B; h = a*h + u*B; y += C*h                                      -> 4
+#   backward: recompute delta*A', p = a*h_prev, h = p + u*B (3); g = C*dy + v; v = a*g;
+#             dB += u*g; dC += dy*h; q = g*p; dA += delta*q; sum A*q; sum g*B (8)           -> 11
+# plus one exp2 (MUFU) per update in each direction.
+FWD_OPS_PER_UPDATE = 4
+BWD_OPS_PER_UPDATE = 11
+SMS, FP32_LANES_PER_SM = 148, 128
+
+
+def alu_peak_tops():
+    """FP32-pipe lane operations per second at the maximum SM clock: 148 SMs x 128 lanes x f."""
+    mhz = 1965.0
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        mhz = float(json.load(open(p)).get("sm_max_mhz", mhz))
+    return SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12, mhz
+
+
 def algorithmic_bytes(w):
     """Minimum bytes the method moves per step (fwd + bwd), split by call."""
     from selective_state_space_bwd_b200 import inputs as gen
@@ -366,6 +386,9 @@ def main():
     bwd_gbs = bb / (t_bwd / args.steps) / 1e9
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
     step_gbs = (fb + bb) / ((t_fwd + t_bwd) / args.steps) / 1e9
+    alu_peak, alu_mhz = alu_peak_tops()
+    fo, bo = FWD_OPS_PER_UPDATE * upd_rank, BWD_OPS_PER_UPDATE * upd_rank
+    bwd_tops = bo / (t_bwd / args.steps) / 1e12
 
     if rank == 0:
         line = {
@@ -379,12 +402,19 @@ def main():
                        "state": "fp32", "l2": "flushed (256 MiB write) before every timed step",
                        "parallelism": f"dp{world} (weak: one full batch per rank; "
                                       "dA_log/dD all-reduced)" if world > 1 else "single GPU"},
-            "roofline": {"bound": "hbm", "kernel": "ssm_scan_bwd (chunk-recompute adjoint + "
-                         "fixed-order reductions)", "achieved": bwd_gbs, "peak": hbm,
-                         "unit": "GB/s", "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
+            "roofline": {"bound": "alu", "kernel": "ssm_scan_bwd call (real_bwd_kernel + "
+                         "dB/dC and parameter reductions)", "achieved": bwd_tops, "peak": alu_peak,
+                         "unit": "Top/s", "frac": bwd_tops / alu_peak,
+                         "peak_kind": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                                      f"{alu_mhz:.0f} MHz (FMA = 1 op)",
+                         "algorithmic_ops_per_launch": bo,
                          "algorithmic_bytes_per_launch": bb,
                          "traffic": measured_traffic("real_bwd.cu", w.name)},
+            "hbm": {"achieved_bwd": bwd_gbs, "achieved_fwd": fwd_gbs, "achieved_step": step_gbs,
+                    "peak": hbm, "unit": "GB/s", "peak_kind": peak_kind},
+            "hbm_frac_bwd": bwd_gbs / hbm,
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_step": step_gbs / hbm,
+            "alu_frac_fwd": fo / (t_fwd / args.steps) / 1e12 / alu_peak,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -128,6 +128,14 @@ struct BwdCfg {
     static constexpr int Q = NT / (2 * N); // channel parts in the dB/dC column sums
 };
 
+// Quad swizzle of the dB/dC rows: a quarter-warp (8 lanes) covers 32/N channels; channel rows are
+// N/2 quads long, so rows 16/N apart start on the same bank.  XOR-ing the quad index with N/4 for
+// every other such group spreads the quarter-warp over all 32 banks.
+template <int N>
+__host__ __device__ constexpr int red_swz(int ch) {
+    return ((ch / (16 / N)) & 1) * (N / 4);
+}
+
 template <typename E, int N>
 struct BwdSmem {
     static constexpr int TT = BwdCfg<N>::TT, DT = BwdCfg<N>::DT, W = BwdCfg<N>::W;
@@ -361,9 +369,12 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                     }
                     sv[2 * uu] = sg.x + sg.y;
                     sv[2 * uu + 1] = sa.x + sa.y;
-                    float* sr = red + (uu * DT + dl) * N2 + n0;
-                    st_pairs<4>(sr, rB);
-                    st_pairs<4>(sr + N, rC);
+                    // rows of 2N floats; odd channel groups swap their dB and dC halves so that a
+                    // quarter-warp's 16-byte stores fall in distinct banks
+                    float* sr = red + (uu * DT + dl) * N2;
+                    const int sw = red_swz<N>(dl);
+                    st_pairs<4>(sr + 4 * (ng ^ sw), rB);
+                    st_pairs<4>(sr + 4 * ((NG + ng) ^ sw), rC);
                 };
                 // after a window's reverse sweep: outputs, then its dB/dC column sums
                 auto finish_window = [&](int q, float (&sv)[2 * W], const float* red) {
@@ -384,12 +395,16 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                         }
                     }
                     __syncthreads();  // the window's dB/dC values are in `red`
-                    const float* src = red + (cs_u * DT + cs_part * (DT / Q)) * N2 + cs_o;
+                    const float* src = red + (cs_u * DT + cs_part * (DT / Q)) * N2;
+                    const int cq = cs_o >> 2;
                     float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
 #pragma unroll
                     for (int ch = 0; ch < DT / Q; ch += 2) {
-                        const float4 a0 = *reinterpret_cast<const float4*>(src + ch * N2);
-                        const float4 a1 = *reinterpret_cast<const float4*>(src + (ch + 1) * N2);
+                        // DT / Q is a multiple of 8, so the swizzle of channel ch is red_swz(ch)
+                        const float4 a0 = *reinterpret_cast<const float4*>(
+                            src + ch * N2 + 4 * (cq ^ red_swz<N>(ch)));
+                        const float4 a1 = *reinterpret_cast<const float4*>(
+                            src + (ch + 1) * N2 + 4 * (cq ^ red_swz<N>(ch + 1)));
                         s0 = __fadd2_rn(s0, make_float2(a0.x, a0.y));
                         s1 = __fadd2_rn(s1, make_float2(a0.z, a0.w));
                         s2 = __fadd2_rn(s2, make_float2(a1.x, a1.y));
