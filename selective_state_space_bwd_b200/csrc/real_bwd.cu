@@ -110,9 +110,9 @@ __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __re
 //           sub-tile: delta and sigmoid(delta_raw) from one exp per (t, d); (delta, delta) and
 //           the state at every 4-step window start go to this CTA's L2-resident workspace region;
 //           the recurrence advances through the sub-tile.
-//   pass B: stream the sub-tiles in reverse.  Windows are software-pipelined: the reverse sweep
-//           of window q runs interleaved with the recompute of window q-1 (its (a_t, a_t h_{t-1})
-//           into registers), so the exponentials of one overlap the FMA chain of the other.
+//   pass B: stream the sub-tiles in reverse.  For each 4-step window, last first: recompute
+//           (a_t, a_t h_{t-1}) forward from the window's start state into registers, then sweep
+//           the adjoint back through the window.
 //           After each window: reduce-scatter of the per-channel sums over the NG lanes, dx and
 //           ddelta_raw stored directly, and the window's dB / dC values (double-buffered shared
 //           memory) summed over the CTA's 32 channels into its partial-sum rows.
@@ -326,56 +326,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                 const int nw = TTe / W;  // 4 or 8 windows, even
                 const int wbase = (j * TTe) / W;
 
-                float2 aaA[W][P2], ppA[W][P2], aaB[W][P2], ppB[W][P2];
-                // recompute window `q` of this sub-tile from hw into (aa, pp); hw <- next start
-                auto recompute_step = [&](float2 (&aa)[W][P2], float2 (&pp)[W][P2], float2 (&hc)[P2],
-                                          int q, int u) {
-                    const int r = q * W + u;
-                    const float dlt = sds[r * DT + dl].x;
-                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    float2 bq[P2];
-                    ld_pairs<4>(bq, sBf + r * N + n0);
-#pragma unroll
-                    for (int i = 0; i < P2; ++i) {
-                        const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
-                        const float2 pr = __fmul2_rn(a, hc[i]);
-                        aa[u][i] = a;
-                        pp[u][i] = pr;
-                        hc[i] = __ffma2_rn(f2(dxv), bq[i], pr);
-                    }
-                };
-                auto reverse_step = [&](const float2 (&aa)[W][P2], const float2 (&pp)[W][P2], int q,
-                                        int uu, float (&sv)[2 * W], float* red) {
-                    const int r = q * W + uu;
-                    const float dlt = sds[r * DT + dl].x;
-                    const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                    const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-                    float2 bq[P2], cq[P2];
-                    ld_pairs<4>(bq, sBf + r * N + n0);
-                    ld_pairs<4>(cq, sCf + r * N + n0);
-                    float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
-                    float2 rB[P2], rC[P2];
-#pragma unroll
-                    for (int i = 0; i < P2; ++i) {
-                        const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);
-                        const float2 hj = __ffma2_rn(f2(dxv), bq[i], pp[uu][i]);
-                        const float2 qv = __fmul2_rn(g, pp[uu][i]);
-                        dA[i] = __ffma2_rn(f2(dlt), qv, dA[i]);
-                        sa = __ffma2_rn(A[i], qv, sa);
-                        sg = __ffma2_rn(g, bq[i], sg);
-                        rB[i] = __fmul2_rn(g, f2(dxv));
-                        rC[i] = __fmul2_rn(f2(dyv), hj);
-                        v[i] = __fmul2_rn(aa[uu][i], g);
-                    }
-                    sv[2 * uu] = sg.x + sg.y;
-                    sv[2 * uu + 1] = sa.x + sa.y;
-                    // rows of 2N floats; odd channel groups swap their dB and dC halves so that a
-                    // quarter-warp's 16-byte stores fall in distinct banks
-                    float* sr = red + (uu * DT + dl) * N2;
-                    const int sw = red_swz<N>(dl);
-                    st_pairs<4>(sr + 4 * (ng ^ sw), rB);
-                    st_pairs<4>(sr + 4 * ((NG + ng) ^ sw), rC);
-                };
+                float2 aa[W][P2], pp[W][P2];  // (a_t, a_t h_{t-1}) of the current window
                 // after a window's reverse sweep: outputs, then its dB/dC column sums
                 auto finish_window = [&](int q, float (&sv)[2 * W], const float* red) {
                     reduce_scatter<2 * W, NG>(sv, ng);
@@ -425,45 +376,63 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                             make_float4(s0.x, s0.y, s1.x, s1.y);
                 };
 
-                // prologue: recompute the last window of the sub-tile
-                {
+                // windows in reverse: recompute (a_t, a_t h_{t-1}) forward from the window's start
+                // state, keeping B_t, delta_t and delta_t x_t in registers for the reverse sweep
+                for (int q = nw - 1; q >= 0; --q) {
                     float2 hc[P2] = {hw[0], hw[1]};
-                    if (nw >= 2) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + nw - 2) * NT * 4);
+                    if (q >= 1) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 1) * NT * 4);
+                    float2 bqs[W][P2];
+                    float dls[W], dxs[W];
 #pragma unroll
-                    for (int u = 0; u < W; ++u) recompute_step(aaA, ppA, hc, nw - 1, u);
-                }
-                for (int q = nw - 1; q >= 1; q -= 2) {
-                    // reverse window q (set A) while recomputing window q-1 (set B)
-                    {
-                        float sv[2 * W];
-                        float* red = sred + (q & 1) * W * DT * N2;
-                        float2 hc[P2] = {hw[0], hw[1]};
-                        if (q >= 2) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 2) * NT * 4);
+                    for (int u = 0; u < W; ++u) {
+                        const int r = q * W + u;
+                        const float dlt = sds[r * DT + dl].x;
+                        const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
+                        ld_pairs<4>(bqs[u], sBf + r * N + n0);
+                        dls[u] = dlt;
+                        dxs[u] = dxv;
 #pragma unroll
-                        for (int u = 0; u < W; ++u) {
-                            reverse_step(aaA, ppA, q, W - 1 - u, sv, red);
-                            recompute_step(aaB, ppB, hc, q - 1, u);
+                        for (int i = 0; i < P2; ++i) {
+                            const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
+                            const float2 pr = __fmul2_rn(a, hc[i]);
+                            aa[u][i] = a;
+                            pp[u][i] = pr;
+                            hc[i] = __ffma2_rn(f2(dxv), bqs[u][i], pr);
                         }
-                        finish_window(q, sv, red);
                     }
-                    // reverse window q-1 (set B) while recomputing window q-2 (set A)
-                    {
-                        float sv[2 * W];
-                        float* red = sred + ((q - 1) & 1) * W * DT * N2;
-                        if (q >= 2) {
-                            float2 hc[P2] = {hw[0], hw[1]};
-                            if (q >= 3) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 3) * NT * 4);
+                    float sv[2 * W];
+                    float* red = sred + (q & 1) * W * DT * N2;
 #pragma unroll
-                            for (int u = 0; u < W; ++u) {
-                                reverse_step(aaB, ppB, q - 1, W - 1 - u, sv, red);
-                                recompute_step(aaA, ppA, hc, q - 2, u);
-                            }
-                        } else {
+                    for (int uu = W - 1; uu >= 0; --uu) {
+                        const int r = q * W + uu;
+                        const float dlt = dls[uu], dxv = dxs[uu];
+                        const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
+                        float2 cq[P2];
+                        ld_pairs<4>(cq, sCf + r * N + n0);
+                        float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
+                        float2 rB[P2], rC[P2];
 #pragma unroll
-                            for (int u = 0; u < W; ++u) reverse_step(aaB, ppB, q - 1, W - 1 - u, sv, red);
+                        for (int i = 0; i < P2; ++i) {
+                            const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);      // adjoint g_t
+                            const float2 hj = __ffma2_rn(f2(dxv), bqs[uu][i], pp[uu][i]);  // h_t
+                            const float2 qv = __fmul2_rn(g, pp[uu][i]);
+                            dA[i] = __ffma2_rn(f2(dlt), qv, dA[i]);
+                            sa = __ffma2_rn(A[i], qv, sa);
+                            sg = __ffma2_rn(g, bqs[uu][i], sg);
+                            rB[i] = __fmul2_rn(g, f2(dxv));
+                            rC[i] = __fmul2_rn(f2(dyv), hj);
+                            v[i] = __fmul2_rn(aa[uu][i], g);                        // a_t g_t
                         }
-                        finish_window(q - 1, sv, red);
+                        sv[2 * uu] = sg.x + sg.y;
+                        sv[2 * uu + 1] = sa.x + sa.y;
+                        // rows of 2N floats; odd channel groups swap their dB and dC halves so
+                        // that a quarter-warp's 16-byte stores fall in distinct banks
+                        float* sr = red + (uu * DT + dl) * N2;
+                        const int sw = red_swz<N>(dl);
+                        st_pairs<4>(sr + 4 * (ng ^ sw), rB);
+                        st_pairs<4>(sr + 4 * ((NG + ng) ^ sw), rC);
                     }
+                    finish_window(q, sv, red);
                 }
                 // state at the start of the last window of the previous sub-tile
                 if (j > 0) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase - 1) * NT * 4);
