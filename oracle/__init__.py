@@ -45,6 +45,9 @@ def _load():
             I64 = ctypes.c_int64
             lib.ssm_oracle_real.argtypes = [I64, I64, I64, I64, I64] + [P] * 7 + [I64, I64, ctypes.c_int] + [P] * 8
             lib.ssm_oracle_real.restype = ctypes.c_int
+            lib.ssm_oracle_real_ex.argtypes = ([I64, I64, I64, I64, I64] + [P] * 7 +
+                                               [I64, I64, ctypes.c_int, ctypes.c_int] + [P] * 12)
+            lib.ssm_oracle_real_ex.restype = ctypes.c_int
             lib.ssm_oracle_complex.argtypes = [I64, I64, I64] + [P] * 6 + [I64, I64, ctypes.c_int] + [P] * 6
             lib.ssm_oracle_complex.restype = ctypes.c_int
             lib.ssm_oracle_max_threads.argtypes = []
@@ -70,14 +73,16 @@ def _ptr(a):
 
 
 def real(x, delta_raw, A_log, Bm, Cm, Dskip, dy=None, chunk=128, d_range=None, threads=0,
-         want_ckpt=False):
+         want_ckpt=False, zoh=False, h0=None, dhL=None):
     """Real-mode forward (and, if ``dy`` is given, backward) in float64.
 
-    Shapes: x, delta_raw, dy [B,L,D]; Bm, Cm [B,L,N]; A_log [D,N]; Dskip [D].
-    Returns a dict with y [B,L,D] (and ckpt [B,ceil(L/chunk),D,N] if asked), plus dx, ddelta_raw
-    [B,L,D], dA_log [D,N], dB, dC [B,L,N], dD [D] when ``dy`` is given.  With ``d_range=(lo, hi)``
-    only channels lo..hi-1 are computed: other entries of the per-channel outputs are NaN and
-    dB/dC are the sums over those channels only.
+    Shapes: x, delta_raw, dy [B,L,D]; Bm, Cm [B,L,N]; A_log [D,N]; Dskip [D]; h0, dhL [B,D,N].
+    Returns a dict with y [B,L,D] and the final state hL [B,D,N] (and ckpt [B,ceil(L/chunk),D,N] if
+    asked), plus dx, ddelta_raw [B,L,D], dA_log [D,N], dB, dC [B,L,N], dD [D] and dh0 [B,D,N] when
+    ``dy`` is given.  ``zoh`` selects the zero-order-hold input term; ``h0`` is the initial state
+    (default zero) and ``dhL`` the upstream gradient of the final state (default zero).  With
+    ``d_range=(lo, hi)`` only channels lo..hi-1 are computed: other entries of the per-channel
+    outputs are NaN and dB/dC are the sums over those channels only.
     """
     lib = _load()
     x, delta_raw, A_log, Bm, Cm, Dskip = map(_f64, (x, delta_raw, A_log, Bm, Cm, Dskip))
@@ -87,7 +92,13 @@ def real(x, delta_raw, A_log, Bm, Cm, Dskip, dy=None, chunk=128, d_range=None, t
     assert A_log.shape == (D, N) and Dskip.shape == (D,)
     lo, hi = (0, D) if d_range is None else (int(d_range[0]), int(d_range[1]))
     nC = (L + chunk - 1) // chunk
-    out = {"y": np.full((B, L, D), np.nan)}
+    if h0 is not None:
+        h0 = _f64(h0)
+        assert h0.shape == (B, D, N)
+    if dhL is not None:
+        dhL = _f64(dhL)
+        assert dhL.shape == (B, D, N)
+    out = {"y": np.full((B, L, D), np.nan), "hL": np.full((B, D, N), np.nan)}
     if want_ckpt:
         out["ckpt"] = np.full((B, nC, D, N), np.nan)
     if dy is not None:
@@ -95,12 +106,15 @@ def real(x, delta_raw, A_log, Bm, Cm, Dskip, dy=None, chunk=128, d_range=None, t
         assert dy.shape == (B, L, D)
         out.update(dx=np.full((B, L, D), np.nan), ddelta_raw=np.full((B, L, D), np.nan),
                    dA_log=np.full((D, N), np.nan), dB=np.zeros((B, L, N)),
-                   dC=np.zeros((B, L, N)), dD=np.full((D,), np.nan))
-    rc = lib.ssm_oracle_real(B, L, D, N, int(chunk), _ptr(x), _ptr(delta_raw), _ptr(A_log),
-                             _ptr(Bm), _ptr(Cm), _ptr(Dskip), _ptr(dy), lo, hi, int(threads),
-                             _ptr(out["y"]), _ptr(out.get("ckpt")), _ptr(out.get("dx")),
-                             _ptr(out.get("ddelta_raw")), _ptr(out.get("dA_log")),
-                             _ptr(out.get("dB")), _ptr(out.get("dC")), _ptr(out.get("dD")))
+                   dC=np.zeros((B, L, N)), dD=np.full((D,), np.nan),
+                   dh0=np.full((B, D, N), np.nan))
+    rc = lib.ssm_oracle_real_ex(B, L, D, N, int(chunk), _ptr(x), _ptr(delta_raw), _ptr(A_log),
+                                _ptr(Bm), _ptr(Cm), _ptr(Dskip), _ptr(dy), lo, hi, int(threads),
+                                int(bool(zoh)), _ptr(h0), _ptr(dhL),
+                                _ptr(out["y"]), _ptr(out.get("ckpt")), _ptr(out.get("dx")),
+                                _ptr(out.get("ddelta_raw")), _ptr(out.get("dA_log")),
+                                _ptr(out.get("dB")), _ptr(out.get("dC")), _ptr(out.get("dD")),
+                                _ptr(out["hL"]), _ptr(out.get("dh0")))
     if rc != 0:
         raise RuntimeError("ssm_oracle_real failed (bad argument or out of memory)")
     return out

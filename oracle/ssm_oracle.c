@@ -25,6 +25,16 @@
  *     dBm_t  = sum_d g_t delta_t x_t;   dCm_t = sum_d dy_t h_t
  *     dA_log = A_n sum_{b,t} delta_t q_t;   dDskip = sum_{b,t} dy_t x_t
  *
+ * Options of the real mode (ssm_oracle_real_ex):
+ *   - initial state h_{-1} = h0 [B,D,N] instead of zero, and the final state hL = h_{L-1} out;
+ *     with an upstream gradient dhL of the final state the loss becomes L = sum dy·y + sum dhL·hL,
+ *     so g_{L-1} = Cm dy + dhL, and dh0 = dL/dh0 = a_0 g_0 is returned (h_{-1} = h0 enters q_0);
+ *   - zero-order-hold input term, the blog's §1.1 discretisation B̄ = (delta A)^{-1}(exp(delta A) - 1)
+ *     delta B, which for a diagonal A is phi_{t,n} Bm_{t,n} x_t with phi = expm1(delta A) / A.
+ *     Then dphi/ddelta = a and dphi/dA = (delta a - phi) / A, so
+ *       dx_t = Dskip dy_t + sum_n g phi Bm;   ddelta = sum_n A q + x_t sum_n g a Bm;
+ *       dBm_t = sum_d g phi x;   dA_n gets, beside delta q, g Bm x (delta a - phi) / A.
+ *
  * Complex mode.  "SPARC: Shared Phase and Retention Control for Efficient Adaptive Spectral
  * Recurrence" (abstract: two input-dependent scalars, retention r_t and phase phi_t, drive all
  * complex modes, each with its own timescale lambda_k and frequency omega_k; diagonal affine
@@ -75,12 +85,20 @@ static int pick_threads(int nthreads) {
  * overwritten with the sums over the channels in range.
  * Returns 0, or -1 on a bad argument / allocation failure.
  */
-int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
-                    const double* x, const double* draw, const double* A_log, const double* Bm,
-                    const double* Cm, const double* Dskip, const double* dy,
-                    int64_t d_lo, int64_t d_hi, int nthreads,
-                    double* y, double* ckpt, double* dx, double* ddraw,
-                    double* dA_log, double* dB, double* dC, double* dD) {
+/*
+ * As above, with the options: zoh != 0 selects the zero-order-hold input term; h0 [B,D,N] (NULL:
+ * zero) is the initial state; hL [B,D,N] (NULL: skip) receives the final state; dhL [B,D,N] (NULL:
+ * zero) is the upstream gradient of the final state; dh0 [B,D,N] (NULL: skip) receives the gradient
+ * with respect to h0 (both only for d in range).
+ */
+int ssm_oracle_real_ex(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
+                       const double* x, const double* draw, const double* A_log, const double* Bm,
+                       const double* Cm, const double* Dskip, const double* dy,
+                       int64_t d_lo, int64_t d_hi, int nthreads, int zoh,
+                       const double* h0, const double* dhL,
+                       double* y, double* ckpt, double* dx, double* ddraw,
+                       double* dA_log, double* dB, double* dC, double* dD,
+                       double* hL, double* dh0) {
     if (B < 0 || L < 0 || D <= 0 || N <= 0 || T <= 0 || d_lo < 0 || d_hi > D || d_lo > d_hi)
         return -1;
     const int64_t nC = (L + T - 1) / T;
@@ -131,7 +149,8 @@ int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
                 double dDsum = 0.0;
                 for (int64_t b = 0; b < B; ++b) {
                     /* forward: sequential recurrence, full history of a and h kept */
-                    for (int64_t n = 0; n < N; ++n) h[n] = 0.0;
+                    const int64_t s0 = (b * D + d) * N;  /* offset of this row in h0/hL/dhL/dh0 */
+                    for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[s0 + n] : 0.0;
                     for (int64_t t = 0; t < L; ++t) {
                         const int64_t i = (b * L + t) * D + d;
                         const double* Bt = Bm + (b * L + t) * N;
@@ -140,7 +159,8 @@ int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
                         double acc = 0.0;
                         for (int64_t n = 0; n < N; ++n) {
                             const double a = exp(delta * A[n]);
-                            h[n] = a * h[n] + delta * Bt[n] * x[i];
+                            const double w = zoh ? expm1(delta * A[n]) / A[n] : delta;
+                            h[n] = a * h[n] + w * Bt[n] * x[i];
                             aa[t * N + n] = a;
                             hh[t * N + n] = h[n];
                             acc += Ct[n] * h[n];
@@ -151,31 +171,42 @@ int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
                             for (int64_t n = 0; n < N; ++n) ck[n] = h[n];
                         }
                     }
+                    if (hL)
+                        for (int64_t n = 0; n < N; ++n) hL[s0 + n] = h[n];
                     if (!bwd) continue;
-                    /* backward: reverse-time adjoint; v = a_{t+1} g_{t+1} */
-                    for (int64_t n = 0; n < N; ++n) v[n] = 0.0;
+                    /* backward: reverse-time adjoint; v = a_{t+1} g_{t+1}, dhL beyond the end */
+                    for (int64_t n = 0; n < N; ++n) v[n] = dhL ? dhL[s0 + n] : 0.0;
                     for (int64_t t = L - 1; t >= 0; --t) {
                         const int64_t i = (b * L + t) * D + d;
                         const double* Bt = Bm + (b * L + t) * N;
                         const double* Ct = Cm + (b * L + t) * N;
                         const double delta = softplus(draw[i]);
-                        double sum_gB = 0.0, sum_Aq = 0.0;
+                        /* sum_gwB: sum_n g w Bm (w = delta, or phi for zoh); sum_gdB: sum_n g
+                         * (dw/ddelta) Bm (dw/ddelta = 1, or a for zoh) */
+                        double sum_gwB = 0.0, sum_gdB = 0.0, sum_Aq = 0.0;
                         for (int64_t n = 0; n < N; ++n) {
                             const double a = aa[t * N + n];
-                            const double hprev = t > 0 ? hh[(t - 1) * N + n] : 0.0;
+                            const double hprev =
+                                t > 0 ? hh[(t - 1) * N + n] : (h0 ? h0[s0 + n] : 0.0);
                             const double g = Ct[n] * dy[i] + v[n];
                             const double q = g * a * hprev;
+                            const double w = zoh ? expm1(delta * A[n]) / A[n] : delta;
+                            const double dw_ddelta = zoh ? a : 1.0;
                             sum_Aq += A[n] * q;
-                            sum_gB += g * Bt[n];
+                            sum_gwB += g * w * Bt[n];
+                            sum_gdB += g * dw_ddelta * Bt[n];
                             dAsum[n] += delta * q;
-                            myB[(b * L + t) * N + n] += g * delta * x[i];
+                            if (zoh) dAsum[n] += g * Bt[n] * x[i] * (delta * a - w) / A[n];
+                            myB[(b * L + t) * N + n] += g * w * x[i];
                             myC[(b * L + t) * N + n] += dy[i] * hh[t * N + n];
                             v[n] = a * g;
                         }
-                        if (dx) dx[i] = Dskip[d] * dy[i] + delta * sum_gB;
-                        if (ddraw) ddraw[i] = (sum_Aq + x[i] * sum_gB) * sigmoid(draw[i]);
+                        if (dx) dx[i] = Dskip[d] * dy[i] + sum_gwB;
+                        if (ddraw) ddraw[i] = (sum_Aq + x[i] * sum_gdB) * sigmoid(draw[i]);
                         dDsum += dy[i] * x[i];
                     }
+                    if (dh0)
+                        for (int64_t n = 0; n < N; ++n) dh0[s0 + n] = v[n];
                 }
                 if (bwd) {
                     if (dA_log)
@@ -203,6 +234,17 @@ int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
         free(part_dC);
     }
     return fail ? -1 : 0;
+}
+
+int ssm_oracle_real(int64_t B, int64_t L, int64_t D, int64_t N, int64_t T,
+                    const double* x, const double* draw, const double* A_log, const double* Bm,
+                    const double* Cm, const double* Dskip, const double* dy,
+                    int64_t d_lo, int64_t d_hi, int nthreads,
+                    double* y, double* ckpt, double* dx, double* ddraw,
+                    double* dA_log, double* dB, double* dC, double* dD) {
+    return ssm_oracle_real_ex(B, L, D, N, T, x, draw, A_log, Bm, Cm, Dskip, dy, d_lo, d_hi,
+                              nthreads, 0, NULL, NULL, y, ckpt, dx, ddraw, dA_log, dB, dC, dD,
+                              NULL, NULL);
 }
 
 /*
