@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define SSM_SCAN_ABI_VERSION 1
+#define SSM_SCAN_ABI_VERSION 2
 
 /* Same underlying type as cudaStream_t (NULL = the legacy default stream). */
 typedef struct CUstream_st* ssm_stream_t;
@@ -138,6 +138,46 @@ int ssm_scan_bwd(const ssm_shape* shape,
                  const float* ckpt, const void* dy,
                  void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC, float* dD,
                  void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/* Input-term discretisation.  SSM_EULER: b_t = delta_t B_t x_t (the form used above).
+ * SSM_ZOH: zero-order hold, the discretisation B̄ = (delta A)^{-1} (exp(delta A) - 1) delta B of
+ * "选择性状态空间模型(S3M)原理与工程实践" §1.1, which for a diagonal A is
+ * b_{t,n} = (exp(delta_t A_n) - 1) / A_n * B_{t,n} x_t. */
+typedef enum ssm_discretization { SSM_EULER = 0, SSM_ZOH = 1 } ssm_discretization;
+
+/* Options of the real-mode calls (all zero / NULL = the plain calls above).  The pointers are
+ * device pointers owned by the caller, [B, D, N] fp32 row-major, 16-byte aligned, or NULL.
+ * The forward and the backward of one pair must get the same discretization and h0. */
+typedef struct ssm_scan_options {
+    int32_t discretization; /* ssm_discretization */
+    int32_t reserved;       /* must be 0 */
+    const float* h0;        /* initial state h_{-1} (NULL: zero); read by forward and backward */
+    float* hL;              /* forward: final state h_{L-1} written here (NULL: not written);
+                               with L = 0 it is h0 */
+    const float* dhL;       /* backward: upstream gradient of hL (NULL: zero); the loss is then
+                               sum(dy * y) + sum(dhL * hL) */
+    float* dh0;             /* backward: gradient of the loss w.r.t. h0 written here (NULL: not
+                               written); with L = 0 it is dhL */
+} ssm_scan_options;
+
+/* ssm_scan_fwd with options (opts may be NULL).  Carrying hL of one call into h0 of the next
+ * streams a long sequence through several calls with the same result as one call (to rounding).
+ * Returns an ssm_status; SSM_ERR_INVALID_ARG for an unknown discretization or reserved != 0. */
+int ssm_scan_fwd_ex(const ssm_shape* shape, const ssm_scan_options* opts,
+                    const void* x, const void* delta_raw, const float* A_log,
+                    const void* Bm, const void* Cm, const float* Dskip,
+                    void* y, float* ckpt,
+                    void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/* ssm_scan_bwd with options (opts may be NULL): the exact gradient of
+ * sum(dy * y) + sum(dhL * hL), plus dh0.  ckpt must come from ssm_scan_fwd_ex with the same
+ * discretization and h0.  Workspace as for ssm_scan_bwd. */
+int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts,
+                    const void* x, const void* delta_raw, const float* A_log,
+                    const void* Bm, const void* Cm, const float* Dskip,
+                    const float* ckpt, const void* dy,
+                    void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC, float* dD,
+                    void* ws, size_t ws_bytes, ssm_stream_t stream);
 
 /*
  * Forward scan for callers that cannot allocate device memory (the pages describe no such call;

@@ -183,6 +183,20 @@ int check_arrays(const void* const* ptrs, const size_t* counts, int n) {
     return SSM_OK;
 }
 
+int check_options(const ssm_scan_options& o) {
+    if (o.reserved != 0) return SSM_ERR_INVALID_ARG;
+    if (o.discretization != SSM_EULER && o.discretization != SSM_ZOH) return SSM_ERR_INVALID_ARG;
+    return SSM_OK;
+}
+
+// dst <- src (n floats), or zeros when src is null; nothing when dst is null.
+int copy_or_zero(float* dst, const float* src, size_t n, cudaStream_t s) {
+    if (!dst || n == 0) return SSM_OK;
+    const cudaError_t e = src ? cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(dst, 0, n * sizeof(float), s);
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
@@ -206,21 +220,27 @@ size_t ssm_scan_workspace_bytes(const ssm_shape* shape, int backward) {
     return backward ? p.b_end : p.f_end;
 }
 
-int ssm_scan_fwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
-                 const void* Bm, const void* Cm, const float* Dskip, void* y, float* ckpt, void* ws,
-                 size_t ws_bytes, ssm_stream_t stream) {
+int ssm_scan_fwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const void* x,
+                    const void* delta_raw, const float* A_log, const void* Bm, const void* Cm,
+                    const float* Dskip, void* y, float* ckpt, void* ws, size_t ws_bytes,
+                    ssm_stream_t stream) {
     RealPlan p;
     int st = plan_real(shape, &p);
     if (st != SSM_OK) return st;
+    const ssm_scan_options o = opts ? *opts : ssm_scan_options{};
+    if ((st = check_options(o)) != SSM_OK) return st;
     const size_t BLD = (size_t)p.B * p.L * p.D, BLN = (size_t)p.B * p.L * p.N;
-    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN;
-    const void* ptrs[] = {x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt, ws};
-    const size_t counts[] = {BLD, BLD, DN, BLN, BLN, (size_t)p.D, BLD, ck, 1};
-    if ((st = check_arrays(ptrs, counts, 9)) != SSM_OK) return st;
+    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN, BDN = (size_t)p.B * DN;
+    const void* ptrs[] = {x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt, ws, o.h0, o.hL};
+    const size_t counts[] = {BLD, BLD, DN, BLN, BLN, (size_t)p.D, BLD, ck, 1,
+                             o.h0 ? BDN : 0, o.hL ? BDN : 0};
+    if ((st = check_arrays(ptrs, counts, 11)) != SSM_OK) return st;
     if (ws_bytes < p.f_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
-    if (p.B == 0 || p.L == 0) return SSM_OK;
+    if (p.B == 0) return SSM_OK;
+    if (p.L == 0)  // the final state is the initial one
+        return copy_or_zero(o.hL, o.h0, BDN, s);
     ssm::RealArgs a = {};
     a.B = p.B; a.L = p.L; a.D = p.D; a.T = p.T; a.nC = p.nC;
     a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.ndt = p.ndt;
@@ -228,31 +248,43 @@ int ssm_scan_fwd(const ssm_shape* shape, const void* x, const void* delta_raw, c
     a.y = y; a.ckpt = ckpt;
     a.sumP = at<float>(ws, p.f_sumP); a.sumS = at<float>(ws, p.f_sumS); a.hin = at<float>(ws, p.f_hin);
     a.status = at<unsigned>(ws, 0);
+    a.h0 = o.h0; a.hL = o.hL; a.zoh = o.discretization == SSM_ZOH;
     return ssm::launch_real_fwd(a, shape->io == SSM_BF16, p.N, s) == cudaSuccess ? SSM_OK
                                                                                 : SSM_ERR_CUDA;
 }
 
-int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
-                 const void* Bm, const void* Cm, const float* Dskip, const float* ckpt,
-                 const void* dy, void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC,
-                 float* dD, void* ws, size_t ws_bytes, ssm_stream_t stream) {
+int ssm_scan_fwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip, void* y, float* ckpt, void* ws,
+                 size_t ws_bytes, ssm_stream_t stream) {
+    return ssm_scan_fwd_ex(shape, nullptr, x, delta_raw, A_log, Bm, Cm, Dskip, y, ckpt, ws,
+                           ws_bytes, stream);
+}
+
+int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const void* x,
+                    const void* delta_raw, const float* A_log, const void* Bm, const void* Cm,
+                    const float* Dskip, const float* ckpt, const void* dy, void* dx,
+                    void* ddelta_raw, float* dA_log, void* dB, void* dC, float* dD, void* ws,
+                    size_t ws_bytes, ssm_stream_t stream) {
     RealPlan p;
     int st = plan_real(shape, &p);
     if (st != SSM_OK) return st;
+    const ssm_scan_options o = opts ? *opts : ssm_scan_options{};
+    if ((st = check_options(o)) != SSM_OK) return st;
     const size_t BLD = (size_t)p.B * p.L * p.D, BLN = (size_t)p.B * p.L * p.N;
-    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN;
+    const size_t DN = (size_t)p.D * p.N, ck = (size_t)p.B * p.nC * DN, BDN = (size_t)p.B * DN;
     const void* ptrs[] = {x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy,
-                          dx, ddelta_raw, dA_log, dB, dC, dD, ws};
+                          dx, ddelta_raw, dA_log, dB, dC, dD, ws, o.h0, o.dhL, o.dh0};
     const size_t counts[] = {BLD, BLD, DN, BLN, BLN, (size_t)p.D, ck, BLD,
-                             BLD, BLD, DN, BLN, BLN, (size_t)p.D, 1};
-    if ((st = check_arrays(ptrs, counts, 15)) != SSM_OK) return st;
+                             BLD, BLD, DN, BLN, BLN, (size_t)p.D, 1,
+                             o.h0 ? BDN : 0, o.dhL ? BDN : 0, o.dh0 ? BDN : 0};
+    if ((st = check_arrays(ptrs, counts, 18)) != SSM_OK) return st;
     if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
     if (p.B == 0 || p.L == 0) {
         if (cudaMemsetAsync(dA_log, 0, DN * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
         if (cudaMemsetAsync(dD, 0, (size_t)p.D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
-        return SSM_OK;
+        return copy_or_zero(o.dh0, o.dhL, BDN, s);  // with no steps, dL/dh0 = dL/dhL
     }
     ssm::RealArgs a = {};
     a.B = p.B; a.L = p.L; a.D = p.D; a.T = p.T; a.nC = p.nC;
@@ -266,9 +298,18 @@ int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, c
     a.bnd_scratch = at<float>(ws, p.b_bnd);
     a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
     a.status = at<unsigned>(ws, 0);
+    a.h0 = o.h0; a.dhL = o.dhL; a.dh0 = o.dh0; a.zoh = o.discretization == SSM_ZOH;
     return ssm::launch_real_bwd(a, shape->io == SSM_BF16, p.N, p.b_group, s) == cudaSuccess
                ? SSM_OK
                : SSM_ERR_CUDA;
+}
+
+int ssm_scan_bwd(const ssm_shape* shape, const void* x, const void* delta_raw, const float* A_log,
+                 const void* Bm, const void* Cm, const float* Dskip, const float* ckpt,
+                 const void* dy, void* dx, void* ddelta_raw, float* dA_log, void* dB, void* dC,
+                 float* dD, void* ws, size_t ws_bytes, ssm_stream_t stream) {
+    return ssm_scan_bwd_ex(shape, nullptr, x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, dx,
+                           ddelta_raw, dA_log, dB, dC, dD, ws, ws_bytes, stream);
 }
 
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward) {

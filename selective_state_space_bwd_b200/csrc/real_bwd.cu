@@ -87,14 +87,15 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(Rea
     }
 }
 
-// Scaled adjoint entering each segment from its end: v_in[nseg-1] = 0,
+// Scaled adjoint entering each segment from its end: v_in[nseg-1] = dhL (or 0),
 // v_in[s-1] = G_s + P_s v_in[s].
 __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __restrict__ P,
-                                      const float* __restrict__ G, float* __restrict__ vin) {
+                                      const float* __restrict__ G, float* __restrict__ vin,
+                                      const float* __restrict__ dhL) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)B * DN) return;
     const int b = (int)(i / DN), k = (int)(i % DN);
-    float v = 0.0f;
+    float v = dhL ? dhL[i] : 0.0f;
     for (int s = nseg - 1; s >= 0; --s) {
         vin[((size_t)b * nseg + s) * DN + k] = v;
         if (s > 0) {
@@ -154,11 +155,14 @@ struct BwdSmem {
     static constexpr int BYTES = A_END > B_END ? A_END : B_END;
 };
 
-template <typename E, int N>
+template <typename E, int N, bool ZOH>
 __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N>;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;
+    // per-step channel sums over the states: sum g w' B (dx), sum A q, and for zero-order hold
+    // also sum g a B (ddelta; with Euler it equals the first)
+    constexpr int SV = ZOH ? 3 : 2;
     constexpr int TT = Cfg::TT, Q = Cfg::Q, N2 = 2 * N;
     extern __shared__ __align__(16) unsigned char smem[];
 
@@ -176,15 +180,27 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
     const int cs_u = cs_quad / (N2 / 4), cs_o = 4 * (cs_quad % (N2 / 4));
 
     float2 A[P2], A2[P2], v[P2], dA[P2];
+    float2 Ar[P2];  // zero-order hold: 1 / A
 #pragma unroll
     for (int i = 0; i < P2; ++i) {
         A[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]), -expf(p.A_log[d * N + n0 + 2 * i + 1]))
                   : make_float2(0.0f, 0.0f);
         A2[i] = __fmul2_rn(A[i], f2(kLog2e));
+        if (ZOH)
+            Ar[i] = dv ? make_float2(-expf(-p.A_log[d * N + n0 + 2 * i]),
+                                     -expf(-p.A_log[d * N + n0 + 2 * i + 1]))
+                       : make_float2(0.0f, 0.0f);
         v[i] = make_float2(0.0f, 0.0f);
         dA[i] = make_float2(0.0f, 0.0f);
     }
-    if (seg < p.nseg - 1 && dv) ld_pairs<4>(v, p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
+    if (dv) {
+        // the adjoint entering from the segment's end: handed over by the carry or by the later
+        // block, or, for the last segment, the upstream gradient of the final state (or zero)
+        const float* src = seg < p.nseg - 1 ? p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0
+                           : p.dhL          ? p.dhL + ((size_t)b * p.D + d) * N + n0
+                                            : nullptr;
+        if (src) ld_pairs<4>(v, src);
+    }
     float dDacc = 0.0f;
     const float dsk = dv ? p.Dskip[d] : 0.0f;
     const size_t boff = (size_t)b * p.L;
@@ -212,6 +228,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
             float2 h[P2];
             if (c > 0 && dv) {
                 ld_pairs<4>(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
+            } else if (p.h0 && dv) {
+                ld_pairs<4>(h, p.h0 + ((size_t)b * p.D + d) * N + n0);
             } else {
 #pragma unroll
                 for (int i = 0; i < P2; ++i) h[i] = make_float2(0.0f, 0.0f);
@@ -266,9 +284,15 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                         float2 bq[P2];
                         ld_pairs<4>(bq, sBf + r * N + n0);
 #pragma unroll
-                        for (int i = 0; i < P2; ++i)
-                            h[i] = __ffma2_rn(ex2_pair(__fmul2_rn(f2(dd.x), A2[i])), h[i],
-                                              __fmul2_rn(f2(dd.y), bq[i]));
+                        for (int i = 0; i < P2; ++i) {
+                            const float2 zl2 = __fmul2_rn(f2(dd.x), A2[i]);
+                            const float2 a = ex2_pair(zl2);
+                            float2 w = f2(dd.y);  // input weight times x: delta x, or phi x
+                            if constexpr (ZOH)
+                                w = __fmul2_rn(w, zoh_e1(__fmul2_rn(zl2, f2(kLn2)), a,
+                                                         __fmul2_rn(f2(__fdividef(1.0f, dd.x)), Ar[i])));
+                            h[i] = __ffma2_rn(a, h[i], __fmul2_rn(w, bq[i]));
+                        }
                     }
                 }
                 __syncthreads();  // stage k and sdd are free again
@@ -328,8 +352,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
 
                 float2 aa[W][P2], pp[W][P2];  // (a_t, a_t h_{t-1}) of the current window
                 // after a window's reverse sweep: outputs, then its dB/dC column sums
-                auto finish_window = [&](int q, float (&sv)[2 * W], const float* red) {
-                    reduce_scatter<2 * W, NG>(sv, ng);
+                auto finish_window = [&](int q, float (&sv)[SV * W], const float* red) {
+                    reduce_scatter<SV * W, NG>(sv, ng);
 #pragma unroll
                     for (int jj = 0; jj < W / NG; ++jj) {
                         const int uu = ng * (W / NG) + jj;
@@ -338,10 +362,11 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                             const float2 ds = sds[r * DT + dl];
                             const float xv = Elem<E>::to_f(sx[r * DT + dl]);
                             const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
-                            const float sgB = sv[2 * jj], sAq = sv[2 * jj + 1];
+                            const float sgB = sv[SV * jj], sAq = sv[SV * jj + 1];
+                            const float sgaB = ZOH ? sv[SV * jj + 2] : sgB;
                             const size_t o = (size_t)(t0 + r) * p.D + d;
                             dxb[o] = Elem<E>::from_f(fmaf(dsk, dyv, ds.x * sgB));
-                            ddrb[o] = Elem<E>::from_f(fmaf(xv, sgB, sAq) * ds.y);
+                            ddrb[o] = Elem<E>::from_f(fmaf(xv, sgaB, sAq) * ds.y);
                             dDacc = fmaf(dyv, xv, dDacc);
                         }
                     }
@@ -382,7 +407,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                     float2 hc[P2] = {hw[0], hw[1]};
                     if (q >= 1) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 1) * NT * 4);
                     float2 bqs[W][P2];
-                    float dls[W], dxs[W];
+                    float2 e1s[ZOH ? W : 1][P2];  // zero-order hold: E1(delta A) per step
+                    float dls[W], dxs[W], rds[ZOH ? W : 1];
 #pragma unroll
                     for (int u = 0; u < W; ++u) {
                         const int r = q * W + u;
@@ -391,16 +417,25 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                         ld_pairs<4>(bqs[u], sBf + r * N + n0);
                         dls[u] = dlt;
                         dxs[u] = dxv;
+                        if constexpr (ZOH) rds[u] = __fdividef(1.0f, dlt);
 #pragma unroll
                         for (int i = 0; i < P2; ++i) {
-                            const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
+                            const float2 zl2 = __fmul2_rn(f2(dlt), A2[i]);
+                            const float2 a = ex2_pair(zl2);
                             const float2 pr = __fmul2_rn(a, hc[i]);
                             aa[u][i] = a;
                             pp[u][i] = pr;
-                            hc[i] = __ffma2_rn(f2(dxv), bqs[u][i], pr);
+                            if constexpr (ZOH) {
+                                const float2 e1 = zoh_e1(__fmul2_rn(zl2, f2(kLn2)), a,
+                                                         __fmul2_rn(f2(rds[u]), Ar[i]));
+                                e1s[u][i] = e1;
+                                hc[i] = __ffma2_rn(__fmul2_rn(f2(dxv), e1), bqs[u][i], pr);
+                            } else {
+                                hc[i] = __ffma2_rn(f2(dxv), bqs[u][i], pr);
+                            }
                         }
                     }
-                    float sv[2 * W];
+                    float sv[SV * W];
                     float* red = sred + (q & 1) * W * DT * N2;
 #pragma unroll
                     for (int uu = W - 1; uu >= 0; --uu) {
@@ -410,21 +445,41 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
                         float2 cq[P2];
                         ld_pairs<4>(cq, sCf + r * N + n0);
                         float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
+                        float2 sga = make_float2(0.0f, 0.0f);
                         float2 rB[P2], rC[P2];
 #pragma unroll
                         for (int i = 0; i < P2; ++i) {
                             const float2 g = __ffma2_rn(cq[i], f2(dyv), v[i]);      // adjoint g_t
-                            const float2 hj = __ffma2_rn(f2(dxv), bqs[uu][i], pp[uu][i]);  // h_t
                             const float2 qv = __fmul2_rn(g, pp[uu][i]);
                             dA[i] = __ffma2_rn(f2(dlt), qv, dA[i]);
                             sa = __ffma2_rn(A[i], qv, sa);
-                            sg = __ffma2_rn(g, bqs[uu][i], sg);
-                            rB[i] = __fmul2_rn(g, f2(dxv));
-                            rC[i] = __fmul2_rn(f2(dyv), hj);
-                            v[i] = __fmul2_rn(aa[uu][i], g);                        // a_t g_t
+                            if constexpr (ZOH) {
+                                // input weight phi = delta E1; d phi / ddelta = a;
+                                // d phi / dA = delta^2 E2
+                                const float2 e1 = e1s[uu][i];
+                                const float2 hj = __ffma2_rn(__fmul2_rn(f2(dxv), e1), bqs[uu][i],
+                                                             pp[uu][i]);           // h_t
+                                const float2 e2 = zoh_e2(
+                                    __fmul2_rn(__fmul2_rn(f2(dlt), A2[i]), f2(kLn2)), aa[uu][i],
+                                    e1, __fmul2_rn(f2(rds[uu]), Ar[i]));
+                                const float2 gb = __fmul2_rn(g, bqs[uu][i]);
+                                dA[i] = __ffma2_rn(gb, __fmul2_rn(f2(dxv * dlt), e2), dA[i]);
+                                sg = __ffma2_rn(gb, e1, sg);
+                                rB[i] = __fmul2_rn(__fmul2_rn(g, e1), f2(dxv));
+                                rC[i] = __fmul2_rn(f2(dyv), hj);
+                                v[i] = __fmul2_rn(aa[uu][i], g);                    // a_t g_t
+                                sga = __ffma2_rn(v[i], bqs[uu][i], sga);
+                            } else {
+                                const float2 hj = __ffma2_rn(f2(dxv), bqs[uu][i], pp[uu][i]);  // h_t
+                                sg = __ffma2_rn(g, bqs[uu][i], sg);
+                                rB[i] = __fmul2_rn(g, f2(dxv));
+                                rC[i] = __fmul2_rn(f2(dyv), hj);
+                                v[i] = __fmul2_rn(aa[uu][i], g);                    // a_t g_t
+                            }
                         }
-                        sv[2 * uu] = sg.x + sg.y;
-                        sv[2 * uu + 1] = sa.x + sa.y;
+                        sv[SV * uu] = sg.x + sg.y;
+                        sv[SV * uu + 1] = sa.x + sa.y;
+                        if constexpr (ZOH) sv[SV * uu + 2] = sga.x + sga.y;
                         // rows of 2N floats; odd channel groups swap their dB and dC halves so
                         // that a quarter-warp's 16-byte stores fall in distinct banks
                         float* sr = red + (uu * DT + dl) * N2;
@@ -450,6 +505,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT) real_bwd_kernel(RealArgs p) {
         // sequential blocks: the adjoint leaving this block's start enters the previous block
         if (p.seq_blocks && seg > 0)
             st_pairs<4>(p.vin + (((size_t)b * p.nseg + (seg - 1)) * p.D + d) * N + n0, v);
+        // the first segment ends at t = -1: its adjoint a_0 g_0 is the gradient of h0
+        if (p.dh0 && seg == 0) st_pairs<4>(p.dh0 + ((size_t)b * p.D + d) * N + n0, v);
         if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
     }
 }
@@ -507,7 +564,7 @@ cudaError_t set_smem(K kern, size_t bytes) {
 // launch; sequential blocks (seq_blocks == 1) run one per launch from the end, each writing the
 // adjoint entering the previous one.  Either way the dB/dC partial buffer holds the rows of one
 // launch only, so its size does not grow with L.
-template <typename E, int N>
+template <typename E, int N, bool ZOH>
 cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
     const int esz = (int)sizeof(E);
     cudaError_t e;
@@ -520,11 +577,12 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
-                                                                            a.gsumP, a.gsumG, a.vin);
+                                                                            a.gsumP, a.gsumG, a.vin,
+                                                                            a.dhL);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const size_t sm = BwdSmem<E, N>::BYTES;
-    if ((e = set_smem(real_bwd_kernel<E, N>, sm)) != cudaSuccess) return e;
+    if ((e = set_smem(real_bwd_kernel<E, N, ZOH>, sm)) != cudaSuccess) return e;
     const int per = a.seq_blocks ? 1 : group;
     for (int hi = a.nseg; hi > 0; hi -= per) {
         const int lo = hi - per > 0 ? hi - per : 0;
@@ -532,7 +590,7 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         a.part_t0 = lo * a.seg_chunks * a.T;
         const int t_hi = min(a.L, hi * a.seg_chunks * a.T);
         const int rows = t_hi - a.part_t0;
-        real_bwd_kernel<E, N><<<dim3(a.ndt, a.B, hi - lo), dim3(BwdCfg<N>::NT), sm, st>>>(a);
+        real_bwd_kernel<E, N, ZOH><<<dim3(a.ndt, a.B, hi - lo), dim3(BwdCfg<N>::NT), sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t nbc = (int64_t)a.B * rows * 2 * N;
         if (nbc > 0) {
@@ -545,11 +603,16 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <typename E, bool ZOH>
+cudaError_t bwd_dispatch_n(const RealArgs& a, int N, int group, cudaStream_t st) {
+    if (N == 4) return real_bwd_impl<E, 4, ZOH>(a, group, st);
+    if (N == 8) return real_bwd_impl<E, 8, ZOH>(a, group, st);
+    return real_bwd_impl<E, 16, ZOH>(a, group, st);
+}
+
 template <typename E>
 cudaError_t bwd_dispatch(const RealArgs& a, int N, int group, cudaStream_t st) {
-    if (N == 4) return real_bwd_impl<E, 4>(a, group, st);
-    if (N == 8) return real_bwd_impl<E, 8>(a, group, st);
-    return real_bwd_impl<E, 16>(a, group, st);
+    return a.zoh ? bwd_dispatch_n<E, true>(a, N, group, st) : bwd_dispatch_n<E, false>(a, N, group, st);
 }
 
 }  // namespace

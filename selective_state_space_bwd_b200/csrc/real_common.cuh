@@ -70,6 +70,42 @@ __device__ __forceinline__ bool all_finite(const float2 (&v)[S / 2]) {
     return ok;
 }
 
+// ---------------------------------------------------------------- zero-order hold
+// For a pair of exponents z = delta * A <= 0 (natural units), with a = exp(z) and rz = 1 / z:
+//   E1(z) = expm1(z) / z           the input weight is phi = (exp(delta A) - 1) / A = delta E1(z)
+//   E2(z) = (exp(z) - E1(z)) / z   d phi / dA = (delta a - phi) / A = delta^2 E2(z)
+// Below |z| = 1/2 both come from their Taylor series about 0 (E1 = sum_k z^k / (k+1)!,
+// E2 = sum_k z^(k-1) k / (k+1)!, eight terms each, remainder under 3e-8 relative); above it from
+// the quotients, where a - 1 and a - E1 do not cancel.  delta = 0 (padding) gives rz = inf and
+// z = 0, which selects the series.
+constexpr float kZohSeries = -0.5f;
+
+__device__ __forceinline__ float2 zoh_e1(float2 z, float2 a, float2 rz) {
+    float2 p = f2(1.0f / 40320.0f);
+    p = __ffma2_rn(p, z, f2(1.0f / 5040.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 720.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 120.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 24.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 6.0f));
+    p = __ffma2_rn(p, z, f2(0.5f));
+    p = __ffma2_rn(p, z, f2(1.0f));
+    const float2 q = __fmul2_rn(__fadd2_rn(a, f2(-1.0f)), rz);
+    return make_float2(z.x > kZohSeries ? p.x : q.x, z.y > kZohSeries ? p.y : q.y);
+}
+
+__device__ __forceinline__ float2 zoh_e2(float2 z, float2 a, float2 e1, float2 rz) {
+    float2 p = f2(1.0f / 45360.0f);
+    p = __ffma2_rn(p, z, f2(1.0f / 5760.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 840.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 144.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 30.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 8.0f));
+    p = __ffma2_rn(p, z, f2(1.0f / 3.0f));
+    p = __ffma2_rn(p, z, f2(0.5f));
+    const float2 q = __fmul2_rn(__ffma2_rn(e1, f2(-1.0f), a), rz);
+    return make_float2(z.x > kZohSeries ? p.x : q.x, z.y > kZohSeries ? p.y : q.y);
+}
+
 // Reduce-scatter of V per-lane values over the NG adjacent lanes of a channel: on return lane
 // `ng` holds, in v[0 .. V/NG), the channel totals of values [ng*V/NG, (ng+1)*V/NG).
 template <int V, int NG>

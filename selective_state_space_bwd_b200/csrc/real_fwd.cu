@@ -49,7 +49,7 @@ struct FwdSmem {
 
 // SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end state).
 // SUMMARY = false: the scan from the segment's entering state, writing y and checkpoints.
-template <typename E, int N, bool SUMMARY>
+template <typename E, int N, bool SUMMARY, bool ZOH>
 __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     using Cfg = FwdCfg<N>;
     using Sm = FwdSmem<E, N>;
@@ -71,15 +71,26 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     const int ntiles = (t_end - t_begin + TTe - 1) / TTe;
 
     float2 A2[P2], h[P2], P[P2];
+    float2 Ar[P2];  // zero-order hold: 1 / A
 #pragma unroll
     for (int i = 0; i < P2; ++i) {
         A2[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]) * kLog2e,
                                  -expf(p.A_log[d * N + n0 + 2 * i + 1]) * kLog2e)
                    : make_float2(0.0f, 0.0f);
+        if (ZOH)
+            Ar[i] = dv ? make_float2(-expf(-p.A_log[d * N + n0 + 2 * i]),
+                                     -expf(-p.A_log[d * N + n0 + 2 * i + 1]))
+                       : make_float2(0.0f, 0.0f);
         h[i] = make_float2(0.0f, 0.0f);
         P[i] = make_float2(1.0f, 1.0f);
     }
-    if (!SUMMARY && seg > 0 && dv) ld_pairs<4>(h, p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0);
+    if (!SUMMARY && dv) {
+        // the state entering this segment: from the carry when split in time, else h0 (or zero)
+        const float* src = p.nseg > 1 ? p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0
+                           : p.h0   ? p.h0 + ((size_t)b * p.D + d) * N + n0
+                                    : nullptr;
+        if (src) ld_pairs<4>(h, src);
+    }
     const size_t boff = (size_t)b * p.L;
     const E* xb = static_cast<const E*>(p.x) + boff * p.D;
     const E* drb = static_cast<const E*>(p.draw) + boff * p.D;
@@ -100,6 +111,18 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
             cp_async_flat<E>(sx + 2 * Sm::XE + Sm::BE, Cb, (size_t)t0 * N, rows4 * N,
                              (size_t)p.L * N, tid, NT);
         cp_async_commit();
+    };
+
+    // input term w B_t x_t for a pair of states given (delta, delta x), a = exp(delta A) and
+    // zl2 = delta A log2(e): w = delta (Euler) or (exp(delta A) - 1) / A (zero-order hold)
+    auto input_term = [&](float2 dd, float2 a, float2 zl2, float2 bq, int i) {
+        if constexpr (ZOH) {
+            const float2 z = __fmul2_rn(zl2, f2(kLn2));
+            const float2 rz = __fmul2_rn(f2(__fdividef(1.0f, dd.x)), Ar[i]);
+            return __fmul2_rn(__fmul2_rn(f2(dd.y), zoh_e1(z, a, rz)), bq);
+        } else {
+            return __fmul2_rn(f2(dd.y), bq);
+        }
     };
 
     if (ntiles > 0) issue(0, 0);
@@ -140,8 +163,9 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
                 if (SUMMARY) {
 #pragma unroll
                     for (int i = 0; i < P2; ++i) {
-                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
-                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
+                        const float2 zl2 = __fmul2_rn(f2(dd.x), A2[i]);
+                        const float2 a = ex2_pair(zl2);
+                        h[i] = __ffma2_rn(a, h[i], input_term(dd, a, zl2, bq[i], i));
                         P[i] = __fmul2_rn(P[i], a);
                     }
                 } else {
@@ -150,8 +174,9 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
                     float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
                     for (int i = 0; i < P2; ++i) {
-                        const float2 a = ex2_pair(__fmul2_rn(f2(dd.x), A2[i]));
-                        h[i] = __ffma2_rn(a, h[i], __fmul2_rn(f2(dd.y), bq[i]));
+                        const float2 zl2 = __fmul2_rn(f2(dd.x), A2[i]);
+                        const float2 a = ex2_pair(zl2);
+                        h[i] = __ffma2_rn(a, h[i], input_term(dd, a, zl2, bq[i], i));
                         acc = __ffma2_rn(cq[i], h[i], acc);
                     }
                     yp[u] = acc.x + acc.y;
@@ -168,8 +193,10 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
             }
         }
         const bool chunk_end = (t0 + rows) % T == 0 || t0 + rows == p.L;
-        if (!SUMMARY && dv && chunk_end)
+        if (!SUMMARY && dv && chunk_end) {
             st_pairs<4>(p.ckpt + (((size_t)b * p.nC + t0 / T) * p.D + d) * N + n0, h);
+            if (p.hL && t0 + rows == p.L) st_pairs<4>(p.hL + ((size_t)b * p.D + d) * N + n0, h);
+        }
         __syncthreads();
         if (!SUMMARY) store_tile<E, DT>(yb, sy, t0, rows, p.L, d0, p.D, tid, NT);
     }
@@ -184,13 +211,14 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     }
 }
 
-// State entering each segment: h_in[0] = 0, h_in[s+1] = P_s h_in[s] + S_s.
+// State entering each segment: h_in[0] = h0 (or 0), h_in[s+1] = P_s h_in[s] + S_s.
 __global__ void real_carry_fwd_kernel(int B, int nseg, int DN, const float* __restrict__ P,
-                                      const float* __restrict__ Sv, float* __restrict__ hin) {
+                                      const float* __restrict__ Sv, float* __restrict__ hin,
+                                      const float* __restrict__ h0) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)B * DN) return;
     const int b = (int)(i / DN), k = (int)(i % DN);
-    float h = 0.0f;
+    float h = h0 ? h0[i] : 0.0f;
     for (int s = 0; s < nseg; ++s) {
         hin[((size_t)b * nseg + s) * DN + k] = h;
         if (s < nseg - 1) {
@@ -205,30 +233,36 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename E, int N>
+template <typename E, int N, bool ZOH>
 cudaError_t real_fwd_impl(const RealArgs& a, cudaStream_t st) {
     const dim3 block(FwdCfg<N>::NT);
     const size_t sm = FwdSmem<E, N>::BYTES;
     cudaError_t e;
     if (a.nseg > 1) {
-        if ((e = set_smem(real_fwd_kernel<E, N, true>, sm)) != cudaSuccess) return e;
-        real_fwd_kernel<E, N, true><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
+        if ((e = set_smem(real_fwd_kernel<E, N, true, ZOH>, sm)) != cudaSuccess) return e;
+        real_fwd_kernel<E, N, true, ZOH><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
-                                                                            a.sumP, a.sumS, a.hin);
+                                                                            a.sumP, a.sumS, a.hin,
+                                                                            a.h0);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = set_smem(real_fwd_kernel<E, N, false>, sm)) != cudaSuccess) return e;
-    real_fwd_kernel<E, N, false><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
+    if ((e = set_smem(real_fwd_kernel<E, N, false, ZOH>, sm)) != cudaSuccess) return e;
+    real_fwd_kernel<E, N, false, ZOH><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
     return cudaGetLastError();
+}
+
+template <typename E, bool ZOH>
+cudaError_t fwd_dispatch_n(const RealArgs& a, int N, cudaStream_t st) {
+    if (N == 4) return real_fwd_impl<E, 4, ZOH>(a, st);
+    if (N == 8) return real_fwd_impl<E, 8, ZOH>(a, st);
+    return real_fwd_impl<E, 16, ZOH>(a, st);
 }
 
 template <typename E>
 cudaError_t fwd_dispatch(const RealArgs& a, int N, cudaStream_t st) {
-    if (N == 4) return real_fwd_impl<E, 4>(a, st);
-    if (N == 8) return real_fwd_impl<E, 8>(a, st);
-    return real_fwd_impl<E, 16>(a, st);
+    return a.zoh ? fwd_dispatch_n<E, true>(a, N, st) : fwd_dispatch_n<E, false>(a, N, st);
 }
 
 }  // namespace

@@ -57,6 +57,14 @@ struct RealArgs {
     float* dA_log;
     float* dD;
     unsigned* status;
+    // options: initial state h0 and final state hL ([B][D][N] fp32, may be null); upstream
+    // gradient dhL of the final state and gradient dh0 of the initial state (backward, may be null);
+    // zoh != 0 selects the zero-order-hold input term
+    const float* h0;
+    float* hL;
+    const float* dhL;
+    float* dh0;
+    int zoh;
 };
 
 struct CplxArgs {

@@ -36,6 +36,15 @@ class SsmCShape(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("seg_chunks", ctypes.c_int32)]
 
 
+SSM_EULER, SSM_ZOH = 0, 1
+
+
+class SsmOptions(ctypes.Structure):
+    _fields_ = [("discretization", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("h0", ctypes.c_void_p), ("hL", ctypes.c_void_p), ("dhL", ctypes.c_void_p),
+                ("dh0", ctypes.c_void_p)]
+
+
 class SsmError(RuntimeError):
     def __init__(self, code, what):
         self.code = code
@@ -49,7 +58,7 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_complex_workspace_bytes",
             "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
             "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
-            "ssm_scan_fwd_noalloc"]
+            "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex"]
 
 
 def lib():
@@ -84,6 +93,11 @@ def lib():
             L.ssm_status_string.argtypes, L.ssm_status_string.restype = [I], ctypes.c_char_p
             L.ssm_scan_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P]
             L.ssm_scan_fwd_noalloc.restype = I
+            OP = ctypes.POINTER(SsmOptions)
+            L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
+            L.ssm_scan_fwd_ex.restype = I
+            L.ssm_scan_bwd_ex.argtypes = [SP, OP] + [P] * 15 + [Z, P]
+            L.ssm_scan_bwd_ex.restype = I
             _lib = L
     return _lib
 
@@ -206,6 +220,64 @@ def ssm_scan_bwd(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, chunk=128, seg_ch
                               _p(out["dA_log"]), _p(out["dB"]), _p(out["dC"]), _p(out["dD"]),
                               _p(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_scan_bwd")
+    return out
+
+
+def _options(zoh, h0=None, hL=None, dhL=None, dh0=None):
+    for t in (h0, hL, dhL, dh0):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError("h0, hL, dhL, dh0 must be contiguous float32 [B, D, N]")
+    return SsmOptions(SSM_ZOH if zoh else SSM_EULER, 0, None if h0 is None else h0.data_ptr(),
+                      None if hL is None else hL.data_ptr(), None if dhL is None else dhL.data_ptr(),
+                      None if dh0 is None else dh0.data_ptr())
+
+
+def ssm_scan_fwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, zoh=False, h0=None, chunk=128,
+                    seg_chunks=0, y=None, ckpt=None, hL=None, ws=None, stream=None):
+    """Forward scan with options: ``zoh`` selects the zero-order-hold input term, ``h0`` [B,D,N]
+    fp32 is the initial state (None: zero).  Returns (y, ckpt, hL) with hL [B,D,N] the final
+    state.  The backward must get the same ``zoh`` and ``h0``."""
+    _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip, h0)
+    B, L, D = x.shape
+    N = A_log.shape[1]
+    shape = real_shape(B, L, D, N, chunk, _io_of(x), seg_chunks)
+    if y is None:
+        y = torch.empty_like(x)
+    if ckpt is None:
+        ckpt = torch.empty((B, -(-L // chunk), D, N), dtype=torch.float32, device=x.device)
+    if hL is None:
+        hL = torch.empty((B, D, N), dtype=torch.float32, device=x.device)
+    opts = _options(zoh, h0=h0, hL=hL)
+    ws = _workspace(workspace_bytes(shape, False), x.device, ws)
+    code = lib().ssm_scan_fwd_ex(ctypes.byref(shape), ctypes.byref(opts), _p(x), _p(delta_raw),
+                                 _p(A_log), _p(Bm), _p(Cm), _p(Dskip), _p(y), _p(ckpt), _p(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_scan_fwd_ex")
+    return y, ckpt, hL
+
+
+def ssm_scan_bwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, zoh=False, h0=None, dhL=None,
+                    chunk=128, seg_chunks=0, out=None, ws=None, stream=None):
+    """Backward with options: the gradient of sum(dy y) + sum(dhL hL).  Returns the dict of
+    ssm_scan_bwd plus dh0 [B,D,N] (the gradient with respect to h0)."""
+    _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, h0, dhL)
+    B, L, D = x.shape
+    N = A_log.shape[1]
+    shape = real_shape(B, L, D, N, chunk, _io_of(x), seg_chunks)
+    if out is None:
+        out = dict(dx=torch.empty_like(x), ddelta_raw=torch.empty_like(x),
+                   dA_log=torch.empty_like(A_log), dB=torch.empty_like(Bm), dC=torch.empty_like(Cm),
+                   dD=torch.empty_like(Dskip))
+    if out.get("dh0") is None:
+        out["dh0"] = torch.empty((B, D, N), dtype=torch.float32, device=x.device)
+    opts = _options(zoh, h0=h0, dhL=dhL, dh0=out["dh0"])
+    ws = _workspace(workspace_bytes(shape, True), x.device, ws)
+    code = lib().ssm_scan_bwd_ex(ctypes.byref(shape), ctypes.byref(opts), _p(x), _p(delta_raw),
+                                 _p(A_log), _p(Bm), _p(Cm), _p(Dskip), _p(ckpt), _p(dy),
+                                 _p(out["dx"]), _p(out["ddelta_raw"]), _p(out["dA_log"]),
+                                 _p(out["dB"]), _p(out["dC"]), _p(out["dD"]), _p(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_scan_bwd_ex")
     return out
 
 

@@ -44,7 +44,7 @@ def test_exports_every_declared_symbol(S):
 
 def test_abi_version_and_status_strings(S):
     L = S.lib()
-    assert L.ssm_scan_abi_version() == 1
+    assert L.ssm_scan_abi_version() == 2
     for code in range(8):
         assert L.ssm_status_string(code).decode().startswith(S.STATUS_NAMES[code])
     assert L.ssm_status_string(99) == b"unknown ssm_status"
@@ -130,6 +130,28 @@ def test_null_misaligned_and_small_workspace(S):
     qb = list(pb)
     qb[7] = None  # dy
     assert L.ssm_scan_bwd(ctypes.byref(shp), *qb, needb, None) == 1
+
+
+def test_option_validation(S):
+    """The option-taking calls reject an unknown discretization, a non-zero reserved field and a
+    misaligned state pointer before anything is enqueued; NULL options equal the plain calls'
+    validation."""
+    L = S.lib()
+    shp = S.real_shape(2, 64, 16, 16, 32, S.SSM_F32)
+    need, needb = S.workspace_bytes(shp, False), S.workspace_bytes(shp, True)
+    p, pb = _fake_ptrs(9), _fake_ptrs(15)
+    bad_disc = S.SsmOptions(2, 0, None, None, None, None)
+    bad_res = S.SsmOptions(S.SSM_ZOH, 7, None, None, None, None)
+    mis_h0 = S.SsmOptions(S.SSM_EULER, 0, 0x100004, None, None, None)
+    mis_dh0 = S.SsmOptions(S.SSM_ZOH, 0, None, None, None, 0x100008)
+    for o in (bad_disc, bad_res):
+        assert L.ssm_scan_fwd_ex(ctypes.byref(shp), ctypes.byref(o), *p, need, None) == 1
+        assert L.ssm_scan_bwd_ex(ctypes.byref(shp), ctypes.byref(o), *pb, needb, None) == 1
+    assert L.ssm_scan_fwd_ex(ctypes.byref(shp), ctypes.byref(mis_h0), *p, need, None) == 3
+    assert L.ssm_scan_bwd_ex(ctypes.byref(shp), ctypes.byref(mis_dh0), *pb, needb, None) == 3
+    # NULL options: same checks as the plain calls (here: workspace too small)
+    assert L.ssm_scan_fwd_ex(ctypes.byref(shp), None, *p, need - 1, None) == 4
+    assert L.ssm_scan_bwd_ex(ctypes.byref(shp), None, *pb, needb - 256, None) == 4
 
 
 def test_complex_validation(S):
