@@ -44,6 +44,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seg-chunks", type=int, default=0)
+    ap.add_argument("--zoh", action="store_true",
+                    help="zero-order-hold input term instead of Euler (ssm_scan_*_ex)")
+    ap.add_argument("--state", action="store_true",
+                    help="pass an initial state h0 and an upstream final-state gradient dhL")
     ap.add_argument("--memory-curve", action="store_true",
                     help="peak device memory of fwd+bwd vs L for the stiff workload's shape")
     return ap.parse_args()
@@ -65,6 +69,10 @@ def peaks():
 # plus one exp2 (MUFU) per update in each direction.
 FWD_OPS_PER_UPDATE = 4
 BWD_OPS_PER_UPDATE = 11
+# zero-order hold adds, per update: phi = (a - 1) / A (2) and x phi (1) forward; in the backward
+# the same 2 in the recompute, psi = (delta a - phi) / A (3), g B x psi into dA (2), sum g a B (1)
+ZOH_FWD_OPS_PER_UPDATE = 7
+ZOH_BWD_OPS_PER_UPDATE = 19
 SMS, FP32_LANES_PER_SM = 148, 128
 
 
@@ -139,7 +147,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def oracle_sample(w, inp, budget_s=(10.0, 30.0)):
+def oracle_sample(w, inp, budget_s=(10.0, 30.0), zoh=False):
     """Time the float64 oracle on the host cores: whole batch rows of the workload, repeated
     until about budget_s[0] seconds of work (stops before budget_s[1])."""
     import oracle
@@ -152,7 +160,7 @@ def oracle_sample(w, inp, budget_s=(10.0, 30.0)):
         sl = slice(b, b + 1)
         t0 = time.perf_counter()
         oracle.real(inp["x"][sl], inp["delta_raw"][sl], inp["A_log"], inp["Bm"][sl], inp["Cm"][sl],
-                    inp["Dskip"], inp["dy"][sl], chunk=w.chunk, threads=threads)
+                    inp["Dskip"], inp["dy"][sl], chunk=w.chunk, threads=threads, zoh=zoh)
         dt = time.perf_counter() - t0
         t_total += dt
         rows += 1
@@ -305,15 +313,35 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    use_ex = args.zoh or args.state
+    h0 = dhL = hL = None
+    if args.state:
+        g = torch.Generator(device="cpu").manual_seed(1234 + rank)
+        h0 = torch.randn((w.batch, w.dim, w.dstate), generator=g).to(dev)
+        dhL = torch.randn((w.batch, w.dim, w.dstate), generator=g).to(dev)
+    if use_ex:
+        hL = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+        out["dh0"] = torch.empty_like(hL)
+
     def fwd():
-        S.ssm_scan_fwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
-                       chunk=w.chunk, seg_chunks=args.seg_chunks, y=y, ckpt=ckpt, ws=wsf,
-                       stream=stream)
+        if use_ex:
+            S.ssm_scan_fwd_ex(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
+                              zoh=args.zoh, h0=h0, chunk=w.chunk, seg_chunks=args.seg_chunks,
+                              y=y, ckpt=ckpt, hL=hL, ws=wsf, stream=stream)
+        else:
+            S.ssm_scan_fwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
+                           chunk=w.chunk, seg_chunks=args.seg_chunks, y=y, ckpt=ckpt, ws=wsf,
+                           stream=stream)
 
     def bwd():
-        S.ssm_scan_bwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"], ckpt,
-                       d["dy"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
-                       stream=stream)
+        if use_ex:
+            S.ssm_scan_bwd_ex(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
+                              ckpt, d["dy"], zoh=args.zoh, h0=h0, dhL=dhL, chunk=w.chunk,
+                              seg_chunks=args.seg_chunks, out=out, ws=wsb, stream=stream)
+        else:
+            S.ssm_scan_bwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"], ckpt,
+                           d["dy"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
+                           stream=stream)
 
     def allreduce():
         if world > 1:
@@ -387,7 +415,10 @@ def main():
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
     step_gbs = (fb + bb) / ((t_fwd + t_bwd) / args.steps) / 1e9
     alu_peak, alu_mhz = alu_peak_tops()
-    fo, bo = FWD_OPS_PER_UPDATE * upd_rank, BWD_OPS_PER_UPDATE * upd_rank
+    if args.zoh:
+        fo, bo = ZOH_FWD_OPS_PER_UPDATE * upd_rank, ZOH_BWD_OPS_PER_UPDATE * upd_rank
+    else:
+        fo, bo = FWD_OPS_PER_UPDATE * upd_rank, BWD_OPS_PER_UPDATE * upd_rank
     bwd_tops = bo / (t_bwd / args.steps) / 1e12
 
     if rank == 0:
@@ -399,6 +430,8 @@ def main():
             "data": "synthetic (seeded generator, workload value distributions)",
             "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
                        "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
+                       "discretization": "zoh" if args.zoh else "euler",
+                       "initial_state": bool(args.state),
                        "state": "fp32", "l2": "flushed (256 MiB write) before every timed step",
                        "parallelism": f"dp{world} (weak: one full batch per rank; "
                                       "dA_log/dD all-reduced)" if world > 1 else "single GPU"},
@@ -422,7 +455,7 @@ def main():
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_sample(w, inp)
+            line["cpu_baseline"] = oracle_sample(w, inp, zoh=args.zoh)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
