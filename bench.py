@@ -238,13 +238,22 @@ def run_reference(args, w):
     import oracle
     oracle.build()
     threads = oracle.max_threads()
-    inp = gen.real_inputs(1, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed=0)
-    upd = w.seqlen * w.dim * w.dstate
+    cplx = isinstance(w, gen.ComplexWorkload)
+    if cplx:
+        inp = gen.complex_inputs(1, w.seqlen, w.modes, seed=0)
+        upd = w.seqlen * w.modes
+    else:
+        inp = gen.real_inputs(1, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed=0)
+        upd = w.seqlen * w.dim * w.dstate
     times = []
     for k in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.real(inp["x"], inp["delta_raw"], inp["A_log"], inp["Bm"], inp["Cm"], inp["Dskip"],
-                    inp["dy"], chunk=w.chunk, threads=threads)
+        if cplx:
+            oracle.complex_(inp["u"], inp["r"], inp["phi"], inp["lam"], inp["omega"], inp["g"],
+                            threads=threads)
+        else:
+            oracle.real(inp["x"], inp["delta_raw"], inp["A_log"], inp["Bm"], inp["Cm"],
+                        inp["Dskip"], inp["dy"], chunk=w.chunk, threads=threads)
         dt = time.perf_counter() - t0
         if k >= args.warmup:
             times.append(dt)
@@ -254,13 +263,188 @@ def run_reference(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
-                       "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
-                       "sample": "one batch row per step", "l2": "n/a (CPU)"},
+            "config": ({"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                        "modes": w.modes, "chunk": w.chunk, "io": "complex64"} if cplx else
+                       {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                        "dstate": w.dstate, "chunk": w.chunk, "io": w.io})
+                      | {"sample": "one batch row per step", "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"1 of {w.batch} batch rows of {w.name} per step, float64"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def complex_algorithmic_bytes(w):
+    """Minimum bytes of one complex fwd + bwd: u read and h written by the forward; h and g read,
+    du written by the backward (8 B each, complex64); r and phi read by both, dr and dphi
+    written (4 B each)."""
+    BLK, BL = w.batch * w.seqlen * w.modes, w.batch * w.seqlen
+    return 16 * BLK + 8 * BL, 24 * BLK + 16 * BL
+
+
+def oracle_sample_complex(w, inp, budget_s=(10.0, 30.0)):
+    """Time the float64 oracle's complex mode on whole batch rows (about budget_s[0] seconds)."""
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    rows, t_total, b = 0, 0.0, 0
+    while t_total < budget_s[0]:
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        oracle.complex_(inp["u"][sl], inp["r"][sl], inp["phi"][sl], inp["lam"], inp["omega"],
+                        inp["g"][sl], threads=threads)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        rows += 1
+        b = (b + 1) % w.batch
+        if t_total + dt > budget_s[1]:
+            break
+    upd = rows * w.seqlen * w.modes
+    return {"value": upd / t_total, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, K={w.modes}), fwd+bwd in "
+                      f"float64 / complex128, {t_total:.1f} s"}
+
+
+def main_complex(args, w):
+    """The complex-mode (shared retention/phase) scan: ssm_scan_complex_fwd + _bwd per step."""
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_bwd_b200 import build, ssm_scan as S
+    from selective_state_space_bwd_b200 import inputs as gen
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    S.lib()
+    inp = gen.complex_inputs(w.batch, w.seqlen, w.modes, seed=rank)
+    host = {k: torch.from_numpy(v).pin_memory() for k, v in inp.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    shape = S.complex_shape(w.batch, w.seqlen, w.modes, w.chunk, args.seg_chunks)
+    h = torch.empty_like(d["u"])
+    out = dict(du=torch.empty_like(d["g"]), dr=torch.empty_like(d["r"]),
+               dphi=torch.empty_like(d["phi"]), dlambda=torch.empty_like(d["lam"]),
+               domega=torch.empty_like(d["omega"]))
+    wsf = torch.empty(S.complex_workspace_bytes(shape, False), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(S.complex_workspace_bytes(shape, True), dtype=torch.uint8, device=dev)
+    gbuf = torch.empty(2 * w.modes, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        S.ssm_scan_complex_fwd(d["u"], d["r"], d["phi"], d["lam"], d["omega"], chunk=w.chunk,
+                               seg_chunks=args.seg_chunks, h=h, ws=wsf, stream=stream)
+
+    def bwd():
+        S.ssm_scan_complex_bwd(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"], chunk=w.chunk,
+                               seg_chunks=args.seg_chunks, out=out, ws=wsb, stream=stream)
+
+    def allreduce():
+        if world > 1:  # dlambda, domega sum over the batch rows of every rank
+            gbuf[:w.modes].copy_(out["dlambda"])
+            gbuf[w.modes:].copy_(out["domega"])
+            dist.all_reduce(gbuf)
+            out["dlambda"].copy_(gbuf[:w.modes])
+            out["domega"].copy_(gbuf[w.modes:])
+
+    for _ in range(max(3, args.warmup)):
+        fwd(); bwd(); allreduce()
+    torch.cuda.synchronize()
+    if S.ssm_scan_status(wsb) != 0 or S.ssm_scan_status(wsf) != 0:
+        raise SystemExit("device status word reports a non-finite state")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream); fwd(); e[1].record(stream); bwd(); e[2].record(stream)
+        allreduce(); e[3].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / 1e3
+    tt = torch.tensor([t_step, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    t_step, t_fwd, t_bwd = tt.tolist()
+
+    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    hh = torch.empty(h.shape, dtype=h.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = hh.numel() * hh.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+
+    def e2e_step():
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        fwd(); bwd(); allreduce()
+        hh.copy_(h, non_blocking=True)
+        for k, v in out.items():
+            hout[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    t_e2e = float(t_e2e)
+
+    upd_rank = w.batch * w.seqlen * w.modes
+    value = world * upd_rank * args.steps / t_step
+    hbm, peak_kind = peaks()
+    fb, bb = complex_algorithmic_bytes(w)
+    bwd_gbs = bb / (t_bwd / args.steps) / 1e9
+    fwd_gbs = fb / (t_fwd / args.steps) / 1e9
+    launches = (S.complex_kernel_launches(shape, False) + S.complex_kernel_launches(shape, True)) * args.steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "c64",
+            "data": "synthetic (seeded generator, workload value distributions)",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                       "modes": w.modes, "chunk": w.chunk, "io": "complex64",
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (weak: one full batch per rank; "
+                                      "dlambda/domega all-reduced)" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": "ssm_scan_complex_bwd call (cplx_bwd_kernel + "
+                         "reductions)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+            "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
+            "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
+            "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_sample_complex(w, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def main():
@@ -269,10 +453,10 @@ def main():
         return memory_curve()
     from selective_state_space_bwd_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
-    if isinstance(w, gen.ComplexWorkload):
-        raise SystemExit("bench.py times the real-mode workloads")
     if args.impl == "reference":
         return run_reference(args, w)
+    if isinstance(w, gen.ComplexWorkload):
+        return main_complex(args, w)
 
     import torch
     import torch.distributed as dist
