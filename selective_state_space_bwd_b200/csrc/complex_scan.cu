@@ -6,14 +6,24 @@
 //   mu_t = g_t + w_{t+1},  w_t = conj(a_t) mu_t,  q_t = mu_t conj(a_t h_{t-1}) = w_t conj(h_{t-1}),
 //   du = mu,  dlambda = -sum s Re q,  dr = sigmoid(r) (-sum_k lambda Re q),
 //   domega = sum phi Im q,  dphi = sum_k omega Im q.
-// Thread = one mode of one batch row; CTA = kCplxKT modes x one time segment.  Segments other than
-// the first (forward) / last (backward) take their entering carry from a summary + carry pass,
-// as in the real mode.
-#include "ssm_device.cuh"
-#include "ssm_internal.h"
+// Thread = one mode of one batch row; CTA = kCplxKT modes x one time segment.  Tiles of steps are
+// streamed through a two-stage cp.async ring; the per-step sums over the modes (dr, dphi) go
+// through shared memory, one column per step.  Segments other than the first (forward) / last
+// (backward) take their entering carry from a summary + carry pass, as in the real mode.
+#include "real_common.cuh"
 
 namespace ssm {
 namespace {
+
+using real::cp_async_commit;
+using real::cp_async_flat;
+using real::cp_async_tile;
+using real::cp_async_wait;
+
+constexpr int KT = kCplxKT;
+constexpr int TTF = kCplxTT;   // forward tile: steps per stage
+constexpr int TTB = 16;        // backward tile (two input tiles per stage)
+constexpr int CB = 8;          // transitions computed together (independent of the state)
 
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
     return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
@@ -27,32 +37,98 @@ __device__ __forceinline__ float2 cmul_cb(float2 a, float2 b) {
     return make_float2(fmaf(a.x, b.x, a.y * b.y), fmaf(a.y, b.x, -a.x * b.y));
 }
 
-// exp(-lam s + i om ph).  The phase product is split into its rounded value and exact residual
-// (one fma), and the residual is applied to the sine/cosine to first order, so the phase carries
-// no fp32 rounding of om*ph.
-__device__ __forceinline__ float2 transition(float lam, float om, float s, float ph) {
+// sin and cos of a phase th.  Reduction by pi/2 with pi/2 split into three floats (the first two
+// carry 12 significant bits, so kq times either is exact while |kq| < 4096), then the Taylor
+// series of sin (to x^9) and cos (to x^10) on [-pi/4, pi/4], whose remainders are below 2e-9 and
+// 1.1e-10 there.  Branch-free; `far` reports |th| beyond the reduction's range (|th| > ~6400),
+// where the result is not used (see transitions()).
+__device__ __forceinline__ void sincos_phase(float th, float& sn, float& cs, bool& far) {
+    float kq = rintf(th * 0x1.45f306p-1f);  // th * 2/pi
+    far = fabsf(kq) >= 4096.0f;
+    kq = fminf(fmaxf(kq, -4095.0f), 4095.0f);
+    float x = fmaf(-kq, 0x1.92p+0f, th);
+    x = fmaf(-kq, 0x1.fb4p-12f, x);
+    x = fmaf(-kq, 0x1.4442d2p-24f, x);
+    const float x2 = x * x;
+    float ps = fmaf(x2, 1.0f / 362880.0f, -1.0f / 5040.0f);
+    ps = fmaf(x2, ps, 1.0f / 120.0f);
+    ps = fmaf(x2, ps, -1.0f / 6.0f);
+    const float s = fmaf(x * x2, ps, x);
+    float pc = fmaf(x2, -1.0f / 3628800.0f, 1.0f / 40320.0f);
+    pc = fmaf(x2, pc, -1.0f / 720.0f);
+    pc = fmaf(x2, pc, 1.0f / 24.0f);
+    pc = fmaf(x2, pc, -0.5f);
+    const float c = fmaf(x2, pc, 1.0f);
+    const int q = static_cast<int>(kq) & 3;
+    sn = q == 0 ? s : (q == 1 ? c : (q == 2 ? -s : -c));
+    cs = q == 0 ? c : (q == 1 ? -s : (q == 2 ? -c : s));
+}
+
+// exp(-lam s + i om ph) from given sin/cos of the rounded phase th = om*ph.  The exact residual
+// of the phase product (one fma) is applied to the sine/cosine to first order, so the phase
+// carries no fp32 rounding of om*ph.
+__device__ __forceinline__ float2 transition_from(float lam, float om, float s, float ph, float th,
+                                                  float sn, float cs) {
     const float rho = expf(-lam * s);
-    const float th = om * ph;
     const float tl = fmaf(om, ph, -th);
-    float sn, cs;
-    sincosf(th, &sn, &cs);
     const float c2 = fmaf(-tl, sn, cs);
     const float s2 = fmaf(tl, cs, sn);
     return make_float2(rho * c2, rho * s2);
 }
 
+// The transitions a_{t,k} of CB consecutive steps (ss/sph at r0..r0+CB-1), computed together:
+// they do not depend on the state, so their arithmetic overlaps.  Phases out of the reduction's
+// range (never for |omega phi| < 6400) are redone with the library sincosf, warp-uniformly.
+template <int CB>
+__device__ __forceinline__ void transitions(float2 (&a)[CB], float lam, float om, const float* ss,
+                                            const float* sph, int r0) {
+    bool any_far = false;
+#pragma unroll
+    for (int u = 0; u < CB; ++u) {
+        const float ph = sph[r0 + u], th = om * ph;
+        float sn, cs;
+        bool far;
+        sincos_phase(th, sn, cs, far);
+        any_far |= far;
+        a[u] = transition_from(lam, om, ss[r0 + u], ph, th, sn, cs);
+    }
+    if (__any_sync(0xffffffffu, any_far)) {
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const float ph = sph[r0 + u], th = om * ph;
+            if (fabsf(th * 0x1.45f306p-1f) >= 4095.5f) {
+                float sn, cs;
+                sincosf(th, &sn, &cs);
+                a[u] = transition_from(lam, om, ss[r0 + u], ph, th, sn, cs);
+            }
+        }
+    }
+}
+
+// Per-step scalars of a staged tile: s = softplus(r) and phi, for `rows` steps.
+__device__ __forceinline__ void step_scalars(const float* sr, const float* sp, float* ss, float* sph,
+                                             int rows, int tid) {
+    if (tid < rows) {
+        ss[tid] = softplus_acc(sr[tid]);
+        sph[tid] = sp[tid];
+    }
+}
+
+// Forward.  SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end
+// state).  SUMMARY = false: the scan from the segment's entering state, writing h.
 template <bool SUMMARY>
-__global__ void __launch_bounds__(kCplxKT) cplx_fwd_kernel(CplxArgs p) {
-    constexpr int KT = kCplxKT, TT = kCplxTT;
-    __shared__ __align__(16) float2 su[TT * KT];
-    __shared__ float ss[TT], sph[TT];
+__global__ void __launch_bounds__(KT) cplx_fwd_kernel(CplxArgs p) {
+    __shared__ __align__(16) float2 su[2][TTF * KT];
+    __shared__ __align__(16) float sr[2][TTF], sp[2][TTF];
+    __shared__ float ss[TTF], sph[TTF];
     const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
     const bool kv = k < p.K;
     const int b = blockIdx.y, seg = blockIdx.z;
-    const int c_begin = seg * p.seg_chunks;
-    const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    const int TTe = min(TT, p.T);
+    const int TT = min(TTF, p.T);  // a tile never crosses a chunk end
+    const int t_begin = seg * p.seg_chunks * p.T;
+    const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
     float2 h = make_float2(0.0f, 0.0f), P = make_float2(1.0f, 0.0f);
     if (!SUMMARY && seg > 0 && kv)
@@ -63,33 +139,47 @@ __global__ void __launch_bounds__(kCplxKT) cplx_fwd_kernel(CplxArgs p) {
     const float* rb = p.r + boff;
     const float* pb = p.phi + boff;
 
-    for (int c = c_begin; c < c_end; ++c) {
-        for (int sub = 0; sub < p.T; sub += TTe) {
-            const int t0 = c * p.T + sub;
-            if (t0 >= p.L) break;
-            const int rows = min(TTe, p.L - t0);
-            __syncthreads();
-            load_tile<float2, KT>(su, ub, t0, rows, p.L, k0, p.K, tid, KT);
-            if (tid < rows) {
-                ss[tid] = softplus_acc(rb[t0 + tid]);
-                sph[tid] = pb[t0 + tid];
-            }
-            __syncthreads();
-            for (int r = 0; r < rows; ++r) {
-                const float2 a = transition(lam, om, ss[r], sph[r]);
-                const float2 uu = su[r * KT + tid];
-                const float2 ah = cmul(a, h);
-                h = make_float2(ah.x + uu.x, ah.y + uu.y);
-                if (SUMMARY)
-                    P = cmul(a, P);
-                else
-                    su[r * KT + tid] = h;
-            }
-            if (!SUMMARY) {
-                __syncthreads();
-                store_tile<float2, KT>(hb, su, t0, rows, p.L, k0, p.K, tid, KT);
+    auto issue = [&](int j, int st) {
+        const int t0 = t_begin + j * TT;
+        cp_async_tile<float2, KT>(su[st], ub, t0, TT, p.L, k0, p.K, tid, KT);
+        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_commit();
+    };
+    if (ntiles > 0) issue(0, 0);
+    for (int j = 0; j < ntiles; ++j) {
+        const int st = j & 1;
+        if (j + 1 < ntiles) {
+            issue(j + 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int t0 = t_begin + j * TT;
+        const int rows = min(TT, t_end - t0);
+        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        __syncthreads();
+        const float2* sut = su[st];
+        // transitions of CB steps at a time (independent of h), then their recurrence steps
+        for (int r0 = 0; r0 < rows; r0 += CB) {
+            float2 a[CB];
+            transitions<CB>(a, lam, om, ss, sph, r0);
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                const int r = r0 + u;
+                if (r < rows) {
+                    const float2 uu = sut[r * KT + tid];
+                    const float2 ah = cmul(a[u], h);
+                    h = make_float2(ah.x + uu.x, ah.y + uu.y);
+                    if (SUMMARY)
+                        P = cmul(a[u], P);
+                    else if (kv)
+                        hb[(size_t)(t0 + r) * p.K + k] = h;
+                }
             }
         }
+        __syncthreads();  // stage st and the step scalars are free again
     }
     if (SUMMARY) {
         if (kv) {
@@ -120,42 +210,59 @@ __global__ void cplx_carry_fwd_kernel(int B, int nseg, int K, const float2* __re
 
 // Backward summary for segments 1..nseg-1: local reverse sweep from zero, w <- conj(a)(g + w),
 // and P = prod conj(a) over the segment.
-__global__ void __launch_bounds__(kCplxKT) cplx_bwd_summary_kernel(CplxArgs p) {
-    constexpr int KT = kCplxKT, TT = kCplxTT;
-    __shared__ __align__(16) float2 sg[TT * KT];
-    __shared__ float ss[TT], sph[TT];
+__global__ void __launch_bounds__(KT) cplx_bwd_summary_kernel(CplxArgs p) {
+    __shared__ __align__(16) float2 sg[2][TTF * KT];
+    __shared__ __align__(16) float sr[2][TTF], sp[2][TTF];
+    __shared__ float ss[TTF], sph[TTF];
     const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
     const bool kv = k < p.K;
     const int b = blockIdx.y, seg = blockIdx.z + 1;
-    const int c_begin = seg * p.seg_chunks;
-    const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    const int TTe = min(TT, p.T);
+    const int TT = min(TTF, p.T);
+    const int t_begin = seg * p.seg_chunks * p.T;
+    const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
     float2 w = make_float2(0.0f, 0.0f), P = make_float2(1.0f, 0.0f);
     const size_t boff = (size_t)b * p.L;
     const float2* gb = reinterpret_cast<const float2*>(p.g) + boff * p.K;
     const float* rb = p.r + boff;
     const float* pb = p.phi + boff;
-    for (int c = c_end - 1; c >= c_begin; --c) {
-        for (int sub = ((p.T - 1) / TTe) * TTe; sub >= 0; sub -= TTe) {
-            const int t0 = c * p.T + sub;
-            if (t0 >= p.L) continue;
-            const int rows = min(TTe, p.L - t0);
-            __syncthreads();
-            load_tile<float2, KT>(sg, gb, t0, rows, p.L, k0, p.K, tid, KT);
-            if (tid < rows) {
-                ss[tid] = softplus_acc(rb[t0 + tid]);
-                sph[tid] = pb[t0 + tid];
-            }
-            __syncthreads();
-            for (int r = rows - 1; r >= 0; --r) {
-                const float2 a = transition(lam, om, ss[r], sph[r]);
-                const float2 gg = sg[r * KT + tid];
-                w = cmul_ca(a, make_float2(gg.x + w.x, gg.y + w.y));
-                P = cmul_ca(a, P);
+    auto issue = [&](int j, int st) {
+        const int t0 = t_begin + j * TT;
+        cp_async_tile<float2, KT>(sg[st], gb, t0, TT, p.L, k0, p.K, tid, KT);
+        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_commit();
+    };
+    if (ntiles > 0) issue(ntiles - 1, (ntiles - 1) & 1);
+    for (int j = ntiles - 1; j >= 0; --j) {
+        const int st = j & 1;
+        if (j > 0) {
+            issue(j - 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int t0 = t_begin + j * TT;
+        const int rows = min(TT, t_end - t0);
+        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        __syncthreads();
+        for (int r0 = ((rows - 1) / CB) * CB; r0 >= 0; r0 -= CB) {
+            float2 a[CB];
+            transitions<CB>(a, lam, om, ss, sph, r0);
+#pragma unroll
+            for (int u = CB - 1; u >= 0; --u) {
+                const int r = r0 + u;
+                if (r < rows) {
+                    const float2 gg = sg[st][r * KT + tid];
+                    w = cmul_ca(a[u], make_float2(gg.x + w.x, gg.y + w.y));
+                    P = cmul_ca(a[u], P);
+                }
             }
         }
+        __syncthreads();
     }
     if (kv) {
         const size_t o = ((size_t)b * (p.nseg - 1) + (seg - 1)) * p.K + k;
@@ -180,19 +287,21 @@ __global__ void cplx_carry_bwd_kernel(int B, int nseg, int K, const float2* __re
     }
 }
 
-__global__ void __launch_bounds__(kCplxKT) cplx_bwd_kernel(CplxArgs p) {
-    constexpr int KT = kCplxKT, TT = kCplxTT, NW = KT / 32;
-    __shared__ __align__(16) float2 sg[TT * KT];   // g, then du in place
-    __shared__ __align__(16) float2 shp[TT * KT];  // h_{t-1} for the tile's steps
+__global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
+    constexpr int TT = TTB;  // divides every chunk length, so tiles never cross a segment end
+    static_assert(TT * 4 == KT, "column sums: four threads per step");
+    __shared__ __align__(16) float2 sg[2][TT * KT];    // g of the tile's steps
+    __shared__ __align__(16) float2 shp[2][TT * KT];   // h_{t-1} of the tile's steps
+    __shared__ __align__(16) float sr[2][TT], sp[2][TT];
     __shared__ float ss[TT], sph[TT];
-    __shared__ float sred[TT * NW * 2];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ __align__(16) float2 red[TT * KT];      // (lambda Re q, omega Im q) per step, mode
+    const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
     const bool kv = k < p.K;
     const int b = blockIdx.y, seg = blockIdx.z;
-    const int c_begin = seg * p.seg_chunks;
-    const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    const int TTe = min(TT, p.T);
+    const int t_begin = seg * p.seg_chunks * p.T;
+    const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
     float2 w = make_float2(0.0f, 0.0f);
     if (seg < p.nseg - 1 && kv)
@@ -204,57 +313,79 @@ __global__ void __launch_bounds__(kCplxKT) cplx_bwd_kernel(CplxArgs p) {
     float2* dub = reinterpret_cast<float2*>(p.du) + boff * p.K;
     const float* rb = p.r + boff;
     const float* pb = p.phi + boff;
-    float* partb = p.rp_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L * 2;
+    float2* partb = reinterpret_cast<float2*>(p.rp_part) + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L;
+    // column-sum roles: step cs_r, a quarter of the modes each
+    const int cs_r = tid >> 2, cs_part = tid & 3;
 
-    for (int c = c_end - 1; c >= c_begin; --c) {
-        for (int sub = ((p.T - 1) / TTe) * TTe; sub >= 0; sub -= TTe) {
-            const int t0 = c * p.T + sub;
-            if (t0 >= p.L) continue;
-            const int rows = min(TTe, p.L - t0);
-            __syncthreads();
-            load_tile<float2, KT>(sg, gb, t0, rows, p.L, k0, p.K, tid, KT);
-            if (t0 > 0) {
-                load_tile<float2, KT>(shp, hb, t0 - 1, rows, p.L, k0, p.K, tid, KT);
-            } else {
-                shp[tid] = make_float2(0.0f, 0.0f);
-                if (rows > 1) load_tile<float2, KT>(shp + KT, hb, 0, rows - 1, p.L, k0, p.K, tid, KT);
-            }
-            if (tid < rows) {
-                ss[tid] = softplus_acc(rb[t0 + tid]);
-                sph[tid] = pb[t0 + tid];
-            }
-            __syncthreads();
-            for (int r = rows - 1; r >= 0; --r) {
-                const float s = ss[r], ph = sph[r];
-                const float2 a = transition(lam, om, s, ph);
-                const float2 gg = sg[r * KT + tid];
-                const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
-                w = cmul_ca(a, mu);
-                const float2 q = cmul_cb(w, shp[r * KT + tid]);
-                sg[r * KT + tid] = mu;
-                dlam = fmaf(-s, q.x, dlam);
-                dom = fmaf(ph, q.y, dom);
-                float rp = lam * q.x, pp = om * q.y;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    rp += __shfl_xor_sync(0xffffffffu, rp, o);
-                    pp += __shfl_xor_sync(0xffffffffu, pp, o);
-                }
-                if (lane == 0) {
-                    sred[(r * NW + warp) * 2 + 0] = rp;
-                    sred[(r * NW + warp) * 2 + 1] = pp;
-                }
-            }
-            __syncthreads();
-            for (int i = tid; i < rows * 2; i += KT) {
-                const int r = i >> 1, o = i & 1;
-                float s = 0.0f;
-#pragma unroll
-                for (int ww = 0; ww < NW; ++ww) s += sred[(r * NW + ww) * 2 + o];
-                partb[(size_t)(t0 + r) * 2 + o] = s;
-            }
-            store_tile<float2, KT>(dub, sg, t0, rows, p.L, k0, p.K, tid, KT);
+    auto issue = [&](int j, int st) {
+        const int t0 = t_begin + j * TT;
+        cp_async_tile<float2, KT>(sg[st], gb, t0, TT, p.L, k0, p.K, tid, KT);
+        if (t0 > 0) {
+            cp_async_tile<float2, KT>(shp[st], hb, t0 - 1, TT, p.L, k0, p.K, tid, KT);
+        } else {  // h_{-1} = 0
+            shp[st][tid] = make_float2(0.0f, 0.0f);
+            cp_async_tile<float2, KT>(shp[st] + KT, hb, 0, TT - 1, p.L, k0, p.K, tid, KT);
         }
+        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_commit();
+    };
+    if (ntiles > 0) issue(ntiles - 1, (ntiles - 1) & 1);
+    for (int j = ntiles - 1; j >= 0; --j) {
+        const int st = j & 1;
+        if (j > 0) {
+            issue(j - 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int t0 = t_begin + j * TT;
+        const int rows = min(TT, t_end - t0);
+        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        __syncthreads();
+        const float2* sgt = sg[st];
+        const float2* sht = shp[st];
+        // transitions of CB steps at a time, then their reverse steps (last first)
+        for (int r0 = ((rows - 1) / CB) * CB; r0 >= 0; r0 -= CB) {
+            float2 a[CB];
+            transitions<CB>(a, lam, om, ss, sph, r0);
+#pragma unroll
+            for (int u = CB - 1; u >= 0; --u) {
+                const int r = r0 + u;
+                if (r < rows) {
+                    const float s = ss[r], ph = sph[r];
+                    const float2 gg = sgt[r * KT + tid];
+                    const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
+                    w = cmul_ca(a[u], mu);
+                    const float2 q = cmul_cb(w, sht[r * KT + tid]);
+                    if (kv) dub[(size_t)(t0 + r) * p.K + k] = mu;
+                    dlam = fmaf(-s, q.x, dlam);
+                    dom = fmaf(ph, q.y, dom);
+                    red[r * KT + tid] = make_float2(lam * q.x, om * q.y);
+                }
+            }
+        }
+        __syncthreads();
+        // sums over the CTA's modes, one step per four threads; the rotation by tid keeps each
+        // half-warp's 8-byte loads in distinct banks
+        {
+            float2 acc = make_float2(0.0f, 0.0f);
+            const float2* row = red + cs_r * KT + cs_part * (KT / 4);
+#pragma unroll
+            for (int m = 0; m < KT / 4; ++m) {
+                const float2 v = row[(m + tid) & (KT / 4 - 1)];
+                acc.x += v.x;
+                acc.y += v.y;
+            }
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+            }
+            if (cs_part == 0 && cs_r < rows) partb[t0 + cs_r] = acc;
+        }
+        __syncthreads();  // stage st, red and the step scalars are free again
     }
     if (kv) {
         const size_t o = ((size_t)b * p.nseg + seg) * p.K + k;
@@ -297,7 +428,7 @@ __global__ void cplx_reduce_k_kernel(CplxArgs p) {
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st) {
     cudaError_t e;
     if (a.nseg > 1) {
-        cplx_fwd_kernel<true><<<dim3(a.nkt, a.B, a.nseg - 1), kCplxKT, 0, st>>>(a);
+        cplx_fwd_kernel<true><<<dim3(a.nkt, a.B, a.nseg - 1), KT, 0, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.K;
         cplx_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
@@ -305,14 +436,14 @@ cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st) {
             reinterpret_cast<const float2*>(a.sumS), reinterpret_cast<float2*>(a.hin));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    cplx_fwd_kernel<false><<<dim3(a.nkt, a.B, a.nseg), kCplxKT, 0, st>>>(a);
+    cplx_fwd_kernel<false><<<dim3(a.nkt, a.B, a.nseg), KT, 0, st>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st) {
     cudaError_t e;
     if (a.nseg > 1) {
-        cplx_bwd_summary_kernel<<<dim3(a.nkt, a.B, a.nseg - 1), kCplxKT, 0, st>>>(a);
+        cplx_bwd_summary_kernel<<<dim3(a.nkt, a.B, a.nseg - 1), KT, 0, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.K;
         cplx_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
@@ -320,7 +451,7 @@ cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st) {
             reinterpret_cast<const float2*>(a.gsumG), reinterpret_cast<float2*>(a.win));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    cplx_bwd_kernel<<<dim3(a.nkt, a.B, a.nseg), kCplxKT, 0, st>>>(a);
+    cplx_bwd_kernel<<<dim3(a.nkt, a.B, a.nseg), KT, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t n = (int64_t)a.B * a.L;
     if (n > 0) {
