@@ -43,9 +43,8 @@ __device__ __forceinline__ float2 cmul_cb(float2 a, float2 b) {
 // 1.1e-10 there.  Branch-free; `far` reports |th| beyond the reduction's range (|th| > ~6400),
 // where the result is not used (see transitions()).
 __device__ __forceinline__ void sincos_phase(float th, float& sn, float& cs, bool& far) {
-    float kq = rintf(th * 0x1.45f306p-1f);  // th * 2/pi
+    const float kq = rintf(th * 0x1.45f306p-1f);  // th * 2/pi
     far = fabsf(kq) >= 4096.0f;
-    kq = fminf(fmaxf(kq, -4095.0f), 4095.0f);
     float x = fmaf(-kq, 0x1.92p+0f, th);
     x = fmaf(-kq, 0x1.fb4p-12f, x);
     x = fmaf(-kq, 0x1.4442d2p-24f, x);
@@ -64,12 +63,12 @@ __device__ __forceinline__ void sincos_phase(float th, float& sn, float& cs, boo
     cs = q == 0 ? c : (q == 1 ? -s : (q == 2 ? -c : s));
 }
 
-// exp(-lam s + i om ph) from given sin/cos of the rounded phase th = om*ph.  The exact residual
+// exp(-lam s + i om ph) from given sin/cos of the rounded phase th = om*ph; lam2 = lam log2(e).  The exact residual
 // of the phase product (one fma) is applied to the sine/cosine to first order, so the phase
 // carries no fp32 rounding of om*ph.
-__device__ __forceinline__ float2 transition_from(float lam, float om, float s, float ph, float th,
+__device__ __forceinline__ float2 transition_from(float lam2, float om, float s, float ph, float th,
                                                   float sn, float cs) {
-    const float rho = expf(-lam * s);
+    const float rho = ex2_mufu(-lam2 * s);
     const float tl = fmaf(om, ph, -th);
     const float c2 = fmaf(-tl, sn, cs);
     const float s2 = fmaf(tl, cs, sn);
@@ -80,38 +79,37 @@ __device__ __forceinline__ float2 transition_from(float lam, float om, float s, 
 // they do not depend on the state, so their arithmetic overlaps.  Phases out of the reduction's
 // range (never for |omega phi| < 6400) are redone with the library sincosf, warp-uniformly.
 template <int CB>
-__device__ __forceinline__ void transitions(float2 (&a)[CB], float lam, float om, const float* ss,
-                                            const float* sph, int r0) {
+__device__ __forceinline__ void transitions(float2 (&a)[CB], float lam2, float om,
+                                            const float2* ssp, int r0) {
     bool any_far = false;
 #pragma unroll
     for (int u = 0; u < CB; ++u) {
-        const float ph = sph[r0 + u], th = om * ph;
+        const float2 sp = ssp[r0 + u];  // (s, phi)
+        const float th = om * sp.y;
         float sn, cs;
         bool far;
         sincos_phase(th, sn, cs, far);
         any_far |= far;
-        a[u] = transition_from(lam, om, ss[r0 + u], ph, th, sn, cs);
+        a[u] = transition_from(lam2, om, sp.x, sp.y, th, sn, cs);
     }
     if (__any_sync(0xffffffffu, any_far)) {
 #pragma unroll
         for (int u = 0; u < CB; ++u) {
-            const float ph = sph[r0 + u], th = om * ph;
-            if (fabsf(th * 0x1.45f306p-1f) >= 4095.5f) {
+            const float2 sp = ssp[r0 + u];
+            const float th = om * sp.y;
+            if (fabsf(rintf(th * 0x1.45f306p-1f)) >= 4096.0f) {
                 float sn, cs;
                 sincosf(th, &sn, &cs);
-                a[u] = transition_from(lam, om, ss[r0 + u], ph, th, sn, cs);
+                a[u] = transition_from(lam2, om, sp.x, sp.y, th, sn, cs);
             }
         }
     }
 }
 
 // Per-step scalars of a staged tile: s = softplus(r) and phi, for `rows` steps.
-__device__ __forceinline__ void step_scalars(const float* sr, const float* sp, float* ss, float* sph,
+__device__ __forceinline__ void step_scalars(const float* sr, const float* sp, float2* ssp,
                                              int rows, int tid) {
-    if (tid < rows) {
-        ss[tid] = softplus_acc(sr[tid]);
-        sph[tid] = sp[tid];
-    }
+    if (tid < rows) ssp[tid] = make_float2(softplus_acc(sr[tid]), sp[tid]);
 }
 
 // Forward.  SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end
@@ -120,7 +118,7 @@ template <bool SUMMARY>
 __global__ void __launch_bounds__(KT) cplx_fwd_kernel(CplxArgs p) {
     __shared__ __align__(16) float2 su[2][TTF * KT];
     __shared__ __align__(16) float sr[2][TTF], sp[2][TTF];
-    __shared__ float ss[TTF], sph[TTF];
+    __shared__ float2 ssp[TTF];  // (softplus(r), phi) per step
     const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
     const bool kv = k < p.K;
@@ -158,13 +156,13 @@ __global__ void __launch_bounds__(KT) cplx_fwd_kernel(CplxArgs p) {
         __syncthreads();
         const int t0 = t_begin + j * TT;
         const int rows = min(TT, t_end - t0);
-        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        step_scalars(sr[st], sp[st], ssp, rows, tid);
         __syncthreads();
         const float2* sut = su[st];
         // transitions of CB steps at a time (independent of h), then their recurrence steps
         for (int r0 = 0; r0 < rows; r0 += CB) {
             float2 a[CB];
-            transitions<CB>(a, lam, om, ss, sph, r0);
+            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
 #pragma unroll
             for (int u = 0; u < CB; ++u) {
                 const int r = r0 + u;
@@ -213,7 +211,7 @@ __global__ void cplx_carry_fwd_kernel(int B, int nseg, int K, const float2* __re
 __global__ void __launch_bounds__(KT) cplx_bwd_summary_kernel(CplxArgs p) {
     __shared__ __align__(16) float2 sg[2][TTF * KT];
     __shared__ __align__(16) float sr[2][TTF], sp[2][TTF];
-    __shared__ float ss[TTF], sph[TTF];
+    __shared__ float2 ssp[TTF];  // (softplus(r), phi) per step
     const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
     const bool kv = k < p.K;
@@ -247,11 +245,11 @@ __global__ void __launch_bounds__(KT) cplx_bwd_summary_kernel(CplxArgs p) {
         __syncthreads();
         const int t0 = t_begin + j * TT;
         const int rows = min(TT, t_end - t0);
-        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        step_scalars(sr[st], sp[st], ssp, rows, tid);
         __syncthreads();
         for (int r0 = ((rows - 1) / CB) * CB; r0 >= 0; r0 -= CB) {
             float2 a[CB];
-            transitions<CB>(a, lam, om, ss, sph, r0);
+            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
 #pragma unroll
             for (int u = CB - 1; u >= 0; --u) {
                 const int r = r0 + u;
@@ -293,7 +291,7 @@ __global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
     __shared__ __align__(16) float2 sg[2][TT * KT];    // g of the tile's steps
     __shared__ __align__(16) float2 shp[2][TT * KT];   // h_{t-1} of the tile's steps
     __shared__ __align__(16) float sr[2][TT], sp[2][TT];
-    __shared__ float ss[TT], sph[TT];
+    __shared__ float2 ssp[TT];  // (softplus(r), phi) per step
     __shared__ __align__(16) float2 red[TT * KT];      // (lambda Re q, omega Im q) per step, mode
     const int tid = threadIdx.x;
     const int k0 = blockIdx.x * KT, k = k0 + tid;
@@ -342,19 +340,20 @@ __global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
         __syncthreads();
         const int t0 = t_begin + j * TT;
         const int rows = min(TT, t_end - t0);
-        step_scalars(sr[st], sp[st], ss, sph, rows, tid);
+        step_scalars(sr[st], sp[st], ssp, rows, tid);
         __syncthreads();
         const float2* sgt = sg[st];
         const float2* sht = shp[st];
         // transitions of CB steps at a time, then their reverse steps (last first)
         for (int r0 = ((rows - 1) / CB) * CB; r0 >= 0; r0 -= CB) {
             float2 a[CB];
-            transitions<CB>(a, lam, om, ss, sph, r0);
+            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
 #pragma unroll
             for (int u = CB - 1; u >= 0; --u) {
                 const int r = r0 + u;
                 if (r < rows) {
-                    const float s = ss[r], ph = sph[r];
+                    const float2 sp2 = ssp[r];
+                    const float s = sp2.x, ph = sp2.y;
                     const float2 gg = sgt[r * KT + tid];
                     const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
                     w = cmul_ca(a[u], mu);

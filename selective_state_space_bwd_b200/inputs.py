@@ -13,6 +13,7 @@ Phase Gradient Flow abstract's 128,000-step impulse-response benchmark):
 * ``stiff_impulse``   B=1, L=128000, D=1024, N=16, fp32 (unit impulse at t=0 plus noise, stiff A)
 * ``mamba1p4b_layer`` B=4, L=8192,   D=4096, N=16, bf16
 * ``sparc_complex``   B=16, L=4096,  K=2048 complex modes (SPARC shared retention/phase control)
+* ``sparc_complex_b4`` the same with B=4 (a quarter of the data: profiling captures)
 
 Draw order (one ``numpy.random.default_rng(seed)`` stream, float32 draws): real mode
 A_log (stiff only), delta_raw, x, Bm, Cm, Dskip, dy; complex mode lambda, omega, r, phi, u, g.
@@ -56,6 +57,7 @@ WORKLOADS = {
     "stiff_impulse": RealWorkload("stiff_impulse", 1, 128000, 1024, 16, 128, F32, "stiff"),
     "mamba1p4b_layer": RealWorkload("mamba1p4b_layer", 4, 8192, 4096, 16, 128, BF16, "mamba"),
     "sparc_complex": ComplexWorkload("sparc_complex", 16, 4096, 2048, 128),
+    "sparc_complex_b4": ComplexWorkload("sparc_complex_b4", 4, 4096, 2048, 128),
 }
 
 
