@@ -50,6 +50,8 @@ def _load():
             lib.ssm_oracle_real_ex.restype = ctypes.c_int
             lib.ssm_oracle_complex.argtypes = [I64, I64, I64] + [P] * 6 + [I64, I64, ctypes.c_int] + [P] * 6
             lib.ssm_oracle_complex.restype = ctypes.c_int
+            lib.ssm_oracle_complex_rtrl.argtypes = [I64, I64, I64] + [P] * 6 + [ctypes.c_int] + [P] * 4
+            lib.ssm_oracle_complex_rtrl.restype = ctypes.c_int
             lib.ssm_oracle_max_threads.argtypes = []
             lib.ssm_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -145,4 +147,30 @@ def complex_(u, r, phi, lam, omega, g=None, k_range=None, threads=0):
                                 _ptr(out.get("dlambda")), _ptr(out.get("domega")))
     if rc != 0:
         raise RuntimeError("ssm_oracle_complex failed (bad argument or out of memory)")
+    return out
+
+
+def complex_rtrl(u, r, phi, lam, omega, g, state=None, want_h=False, threads=0):
+    """Complex-mode forward with exact structured RTRL: the state's sensitivities to lambda and
+    omega are carried forward and the gradient of Re sum conj(g) h accumulates online.
+
+    Shapes: u, g [B,L,K] complex; r, phi [B,L]; lam, omega [K]; state [B,3,K] complex holding
+    (h, dh/dlambda, dh/domega) before the first step (default zero).  Returns a dict with
+    dlambda, domega [K], state [B,3,K] (after the last step) and, if asked, h [B,L,K].
+    """
+    lib = _load()
+    u, g = _c128(u), _c128(g)
+    r, phi, lam, omega = map(_f64, (r, phi, lam, omega))
+    B, L, K = u.shape
+    assert g.shape == (B, L, K) and r.shape == (B, L) and phi.shape == (B, L)
+    st = np.zeros((B, 3, K), dtype=np.complex128) if state is None else _c128(state).copy()
+    assert st.shape == (B, 3, K)
+    out = {"dlambda": np.full((K,), np.nan), "domega": np.full((K,), np.nan), "state": st}
+    if want_h:
+        out["h"] = np.full((B, L, K), np.nan, dtype=np.complex128)
+    rc = lib.ssm_oracle_complex_rtrl(B, L, K, _ptr(u), _ptr(r), _ptr(phi), _ptr(lam),
+                                     _ptr(omega), _ptr(g), int(threads), _ptr(out.get("h")),
+                                     _ptr(st), _ptr(out["dlambda"]), _ptr(out["domega"]))
+    if rc != 0:
+        raise RuntimeError("ssm_oracle_complex_rtrl failed (bad argument)")
     return out

@@ -358,3 +358,64 @@ int ssm_oracle_complex(int64_t B, int64_t L, int64_t K,
     }
     return fail ? -1 : 0;
 }
+
+/*
+ * Complex mode, exact structured real-time recurrent learning (SPARC abstract: the diagonal
+ * recurrence admits exact structured RTRL for online credit assignment).  Forward-mode
+ * sensitivities of the state to each mode's own parameters are carried with the state:
+ *     S^lambda_t = dh_t/dlambda = a_t S^lambda_{t-1} + (da_t/dlambda) h_{t-1},  da/dlambda = -s_t a_t
+ *     S^omega_t  = dh_t/domega  = a_t S^omega_{t-1}  + (da_t/domega)  h_{t-1},  da/domega  = i phi_t a_t
+ * and the gradient of the online loss L = Re sum_t conj(g_t) h_t accumulates as the steps arrive:
+ *     dL/dlambda += Re(conj(g_t) S^lambda_t),   dL/domega += Re(conj(g_t) S^omega_t).
+ * No reverse pass and nothing of the trajectory is kept: the result equals the reverse-time
+ * adjoint's dlambda, domega (the same numbers by a different method).
+ * state [B,3,K] complex (h, S^lambda, S^omega) may be NULL (start from zero, final values not
+ * returned); when given it is read as the state before t = 0 and overwritten with the state after
+ * t = L-1, so consecutive calls continue one sequence.  h (optional) receives the trajectory.
+ * dlambda, domega [K] receive this call's sums over b and t.  Returns 0 or -1.
+ */
+int ssm_oracle_complex_rtrl(int64_t B, int64_t L, int64_t K,
+                            const double* u_, const double* r, const double* phi,
+                            const double* lambda, const double* omega, const double* g_,
+                            int nthreads, double* h_, double* state_,
+                            double* dlambda, double* domega) {
+    if (B < 0 || L < 0 || K <= 0 || !g_ || !dlambda || !domega) return -1;
+    const double complex* u = (const double complex*)u_;
+    const double complex* g = (const double complex*)g_;
+    double complex* hout = (double complex*)h_;
+    double complex* state = (double complex*)state_;
+    nthreads = pick_threads(nthreads);
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t k = 0; k < K; ++k) {
+        const double lam = lambda[k], om = omega[k];
+        double dlam = 0.0, dom = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            double complex h = 0.0, Sl = 0.0, So = 0.0;
+            if (state) {
+                h = state[(b * 3 + 0) * K + k];
+                Sl = state[(b * 3 + 1) * K + k];
+                So = state[(b * 3 + 2) * K + k];
+            }
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t j = b * L + t;
+                const double s = softplus(r[j]);
+                const double complex a = cexp(-lam * s + I * (om * phi[j]));
+                Sl = a * Sl + (-s * a) * h;          /* uses h_{t-1} */
+                So = a * So + (I * phi[j] * a) * h;
+                h = a * h + u[j * K + k];
+                if (hout) hout[j * K + k] = h;
+                const double complex gt = g[j * K + k];
+                dlam += creal(conj(gt) * Sl);
+                dom += creal(conj(gt) * So);
+            }
+            if (state) {
+                state[(b * 3 + 0) * K + k] = h;
+                state[(b * 3 + 1) * K + k] = Sl;
+                state[(b * 3 + 2) * K + k] = So;
+            }
+        }
+        dlambda[k] = dlam;
+        domega[k] = dom;
+    }
+    return 0;
+}
