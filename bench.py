@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--seg-chunks", type=int, default=0)
     ap.add_argument("--zoh", action="store_true",
                     help="zero-order-hold input term instead of Euler (ssm_scan_*_ex)")
+    ap.add_argument("--rtrl", action="store_true",
+                    help="complex workloads: time exact structured RTRL (one forward pass that "
+                         "accumulates dlambda, domega online) instead of fwd + bwd")
     ap.add_argument("--state", action="store_true",
                     help="pass an initial state h0 and an upstream final-state gradient dhL")
     ap.add_argument("--memory-curve", action="store_true",
@@ -282,7 +285,7 @@ def complex_algorithmic_bytes(w):
     return 16 * BLK + 8 * BL, 24 * BLK + 16 * BL
 
 
-def oracle_sample_complex(w, inp, budget_s=(10.0, 30.0)):
+def oracle_sample_complex(w, inp, budget_s=(10.0, 30.0), rtrl=False):
     """Time the float64 oracle's complex mode on whole batch rows (about budget_s[0] seconds)."""
     import oracle
     oracle.build()
@@ -291,8 +294,12 @@ def oracle_sample_complex(w, inp, budget_s=(10.0, 30.0)):
     while t_total < budget_s[0]:
         sl = slice(b, b + 1)
         t0 = time.perf_counter()
-        oracle.complex_(inp["u"][sl], inp["r"][sl], inp["phi"][sl], inp["lam"], inp["omega"],
-                        inp["g"][sl], threads=threads)
+        if rtrl:
+            oracle.complex_rtrl(inp["u"][sl], inp["r"][sl], inp["phi"][sl], inp["lam"],
+                                inp["omega"], inp["g"][sl], threads=threads)
+        else:
+            oracle.complex_(inp["u"][sl], inp["r"][sl], inp["phi"][sl], inp["lam"], inp["omega"],
+                            inp["g"][sl], threads=threads)
         dt = time.perf_counter() - t0
         t_total += dt
         rows += 1
@@ -301,8 +308,8 @@ def oracle_sample_complex(w, inp, budget_s=(10.0, 30.0)):
             break
     upd = rows * w.seqlen * w.modes
     return {"value": upd / t_total, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, K={w.modes}), fwd+bwd in "
-                      f"float64 / complex128, {t_total:.1f} s"}
+            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, K={w.modes}), "
+                      f"{'RTRL' if rtrl else 'fwd+bwd'} in float64 / complex128, {t_total:.1f} s"}
 
 
 def main_complex(args, w):
@@ -339,13 +346,23 @@ def main_complex(args, w):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    if args.rtrl:
+        out = dict(dlambda=out["dlambda"], domega=out["domega"])
+        wsr = torch.empty(S.complex_rtrl_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+
     def fwd():
-        S.ssm_scan_complex_fwd(d["u"], d["r"], d["phi"], d["lam"], d["omega"], chunk=w.chunk,
-                               seg_chunks=args.seg_chunks, h=h, ws=wsf, stream=stream)
+        if args.rtrl:  # the whole RTRL pass: trajectory sensitivities and online gradient
+            S.ssm_scan_complex_rtrl(d["u"], d["r"], d["phi"], d["lam"], d["omega"], d["g"],
+                                    chunk=w.chunk, out=out, ws=wsr, stream=stream)
+        else:
+            S.ssm_scan_complex_fwd(d["u"], d["r"], d["phi"], d["lam"], d["omega"], chunk=w.chunk,
+                                   seg_chunks=args.seg_chunks, h=h, ws=wsf, stream=stream)
 
     def bwd():
-        S.ssm_scan_complex_bwd(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"], chunk=w.chunk,
-                               seg_chunks=args.seg_chunks, out=out, ws=wsb, stream=stream)
+        if not args.rtrl:
+            S.ssm_scan_complex_bwd(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"],
+                                   chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
+                                   stream=stream)
 
     def allreduce():
         if world > 1:  # dlambda, domega sum over the batch rows of every rank
@@ -358,7 +375,7 @@ def main_complex(args, w):
     for _ in range(max(3, args.warmup)):
         fwd(); bwd(); allreduce()
     torch.cuda.synchronize()
-    if S.ssm_scan_status(wsb) != 0 or S.ssm_scan_status(wsf) != 0:
+    if S.ssm_scan_status(wsr if args.rtrl else wsb) != 0 or S.ssm_scan_status(wsf) != 0:
         raise SystemExit("device status word reports a non-finite state")
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -386,11 +403,16 @@ def main_complex(args, w):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = hh.numel() * hh.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
 
+    if args.rtrl:  # the RTRL pass returns only dlambda, domega
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+        h2d = sum(v.numel() * v.element_size() for k, v in host.items())
+
     def e2e_step():
         for k, v in host.items():
             d[k].copy_(v, non_blocking=True)
         fwd(); bwd(); allreduce()
-        hh.copy_(h, non_blocking=True)
+        if not args.rtrl:
+            hh.copy_(h, non_blocking=True)
         for k, v in out.items():
             hout[k].copy_(v, non_blocking=True)
 
@@ -414,9 +436,13 @@ def main_complex(args, w):
     value = world * upd_rank * args.steps / t_step
     hbm, peak_kind = peaks()
     fb, bb = complex_algorithmic_bytes(w)
-    bwd_gbs = bb / (t_bwd / args.steps) / 1e9
+    if args.rtrl:  # u and g read (8 B each per update), r and phi read (4 B each per (b, t))
+        fb, bb = 16 * w.batch * w.seqlen * w.modes + 8 * w.batch * w.seqlen, 0
+    bwd_gbs = bb / (t_bwd / args.steps) / 1e9 if bb else 0.0
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
     launches = (S.complex_kernel_launches(shape, False) + S.complex_kernel_launches(shape, True)) * args.steps
+    if args.rtrl:
+        launches = 2 * args.steps
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -425,13 +451,18 @@ def main_complex(args, w):
             "data": "synthetic (seeded generator, workload value distributions)",
             "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
                        "modes": w.modes, "chunk": w.chunk, "io": "complex64",
+                       "training": "rtrl (online, forward only)" if args.rtrl else "bptt (fwd + bwd)",
                        "l2": "flushed (256 MiB write) before every timed step",
                        "parallelism": f"dp{world} (weak: one full batch per rank; "
                                       "dlambda/domega all-reduced)" if world > 1 else "single GPU"},
-            "roofline": {"bound": "hbm", "kernel": "ssm_scan_complex_bwd call (cplx_bwd_kernel + "
-                         "reductions)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+            "roofline": ({"bound": "hbm", "kernel": "ssm_scan_complex_rtrl call (cplx_rtrl_kernel "
+                          "+ reduction over the batch)", "achieved": fwd_gbs, "peak": hbm,
+                          "unit": "GB/s", "frac": fwd_gbs / hbm, "peak_kind": peak_kind,
+                          "algorithmic_bytes_per_launch": fb, "traffic": None} if args.rtrl else
+                         {"bound": "hbm", "kernel": "ssm_scan_complex_bwd call (cplx_bwd_kernel + "
+                          "reductions)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
+                          "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
+                          "algorithmic_bytes_per_launch": bb, "traffic": None}),
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
@@ -440,7 +471,7 @@ def main_complex(args, w):
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_sample_complex(w, inp)
+            line["cpu_baseline"] = oracle_sample_complex(w, inp, rtrl=args.rtrl)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

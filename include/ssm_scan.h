@@ -230,6 +230,35 @@ int ssm_scan_complex_bwd(const ssm_cshape* shape,
                          void* du, float* dr, float* dphi, float* dlambda, float* domega,
                          void* ws, size_t ws_bytes, ssm_stream_t stream);
 
+/* Workspace bytes for ssm_scan_complex_rtrl (at least 256); 0 for an invalid shape. */
+size_t ssm_scan_complex_rtrl_workspace_bytes(const ssm_cshape* shape);
+
+/*
+ * Complex forward with exact structured real-time recurrent learning ("SPARC: Shared Phase and
+ * Retention Control for Efficient Adaptive Spectral Recurrence", abstract: the diagonal recurrence
+ * supports exact structured RTRL for online credit assignment).  The state's sensitivities to its
+ * mode's own parameters travel with it,
+ *     S^lambda_t = a_t S^lambda_{t-1} - s_t a_t h_{t-1},   S^omega_t = a_t S^omega_{t-1} + i phi_t a_t h_{t-1},
+ * and the gradient of the online loss Re sum_t conj(g_t) h_t accumulates step by step:
+ *     dlambda_k = sum_{b,t} Re(conj(g) S^lambda),  domega_k = sum_{b,t} Re(conj(g) S^omega).
+ * One forward pass; no reverse sweep; nothing of the trajectory is stored.  The result equals
+ * the lambda/omega gradients of ssm_scan_complex_bwd (to rounding).
+ *   u, g     [B, L, K] complex64      r, phi [B, L] fp32      lambda, omega [K] fp32
+ *   h        [B, L, K] complex64 trajectory out, or NULL (not written)
+ *   state    [B, 3, K] complex64 (h, dh/dlambda, dh/domega), or NULL (start from zero, final
+ *            values not returned).  When given it is read as the state before the first step and
+ *            overwritten with the state after the last, so consecutive calls on consecutive parts
+ *            of a sequence continue it; the caller sums their dlambda/domega.
+ *   dlambda, domega [K] fp32: this call's sums (overwritten; zero when B or L is 0).
+ * shape->chunk must be valid (16..256) but is not used; shape->seg_chunks is ignored (each CTA
+ * walks the whole sequence).  Enqueues 2 kernels (none when B or L is 0).  Returns an ssm_status.
+ */
+int ssm_scan_complex_rtrl(const ssm_cshape* shape,
+                          const void* u, const float* r, const float* phi,
+                          const float* lambda, const float* omega, const void* g,
+                          void* h, void* state, float* dlambda, float* domega,
+                          void* ws, size_t ws_bytes, ssm_stream_t stream);
+
 /* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);

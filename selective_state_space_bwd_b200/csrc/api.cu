@@ -137,6 +137,7 @@ struct CplxPlan {
     int B, L, K, T, nC, nkt, seg_chunks, nseg;
     size_t f_sumP, f_sumS, f_hin, f_end;
     size_t b_gP, b_gG, b_win, b_rp, b_lo, b_end;
+    size_t r_lo, r_end;  // RTRL: per-(batch, mode) gradient sums
 };
 
 int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
@@ -169,6 +170,9 @@ int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
     p->b_rp = o;  o = align256(o + (size_t)p->nkt * B * (size_t)p->L * 8);
     p->b_lo = o;  o = align256(o + B * S * K * 8);
     p->b_end = o;
+    o = kStatusBytes;
+    p->r_lo = o;  o = align256(o + B * K * 8);
+    p->r_end = o;
     return SSM_OK;
 }
 
@@ -357,6 +361,45 @@ int ssm_scan_complex_fwd(const ssm_cshape* shape, const void* u, const float* r,
     a.sumP = at<float>(ws, p.f_sumP); a.sumS = at<float>(ws, p.f_sumS); a.hin = at<float>(ws, p.f_hin);
     a.status = at<unsigned>(ws, 0);
     return ssm::launch_cplx_fwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+size_t ssm_scan_complex_rtrl_workspace_bytes(const ssm_cshape* shape) {
+    CplxPlan p;
+    if (plan_cplx(shape, &p) != SSM_OK) return 0;
+    return p.r_end;
+}
+
+int ssm_scan_complex_rtrl(const ssm_cshape* shape, const void* u, const float* r,
+                          const float* phi, const float* lambda, const float* omega, const void* g,
+                          void* h, void* state, float* dlambda, float* domega, void* ws,
+                          size_t ws_bytes, ssm_stream_t stream) {
+    CplxPlan p;
+    int st = plan_cplx(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLK = (size_t)p.B * p.L * p.K, BL = (size_t)p.B * p.L;
+    const void* ptrs[] = {u, r, phi, lambda, omega, g, dlambda, domega, ws, h, state};
+    const size_t counts[] = {BLK, BL, BL, (size_t)p.K, (size_t)p.K, BLK, (size_t)p.K, (size_t)p.K,
+                             1, h ? BLK : 0, state ? (size_t)p.B * 3 * p.K : 0};
+    if ((st = check_arrays(ptrs, counts, 11)) != SSM_OK) return st;
+    if (ws_bytes < p.r_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) {  // no steps: no gradient, the state is unchanged
+        if (cudaMemsetAsync(dlambda, 0, (size_t)p.K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (cudaMemsetAsync(domega, 0, (size_t)p.K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::CplxArgs a = {};
+    a.B = p.B; a.L = p.L; a.K = p.K; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.nC; a.nseg = 1; a.nkt = p.nkt;
+    a.u = static_cast<const float*>(u); a.r = r; a.phi = phi; a.lam = lambda; a.om = omega;
+    a.g = static_cast<const float*>(g);
+    a.h = static_cast<float*>(h);
+    a.state = static_cast<float*>(state);
+    a.lo_part = at<float>(ws, p.r_lo);
+    a.dlam = dlambda; a.dom = domega;
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_cplx_rtrl(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 int ssm_scan_complex_bwd(const ssm_cshape* shape, const void* h, const float* r, const float* phi,

@@ -393,6 +393,99 @@ __global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
     }
 }
 
+// Exact structured RTRL (SPARC abstract: exact structured real-time recurrent learning for online
+// credit assignment).  The state's forward-mode sensitivities to the mode's own lambda and omega
+// travel with it,
+//   S^lambda_t = a_t S^lambda_{t-1} - s_t a_t h_{t-1},   S^omega_t = a_t S^omega_{t-1} + i phi_t a_t h_{t-1},
+// and the gradient of Re sum conj(g) h accumulates as the steps arrive:
+//   dlambda += Re(conj(g_t) S^lambda_t),  domega += Re(conj(g_t) S^omega_t).
+// One forward pass, no reverse sweep, nothing of the trajectory kept (h is written only if asked).
+// Thread = one mode of one batch row over the whole sequence.
+__global__ void __launch_bounds__(KT) cplx_rtrl_kernel(CplxArgs p) {
+    constexpr int TT = 16;
+    __shared__ __align__(16) float2 su[2][TT * KT];
+    __shared__ __align__(16) float2 sgt[2][TT * KT];
+    __shared__ __align__(16) float sr[2][TT], sp[2][TT];
+    __shared__ float2 ssp[TT];  // (softplus(r), phi) per step
+    const int tid = threadIdx.x;
+    const int k0 = blockIdx.x * KT, k = k0 + tid;
+    const bool kv = k < p.K;
+    const int b = blockIdx.y;
+    const int ntiles = (p.L + TT - 1) / TT;
+    const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
+    float2* stb = p.state ? reinterpret_cast<float2*>(p.state) + (size_t)b * 3 * p.K : nullptr;
+    float2 h = make_float2(0.0f, 0.0f), Sl = h, So = h;
+    if (stb && kv) {
+        h = stb[k];
+        Sl = stb[p.K + k];
+        So = stb[2 * p.K + k];
+    }
+    float dl = 0.0f, dom = 0.0f;
+    const size_t boff = (size_t)b * p.L;
+    const float2* ub = reinterpret_cast<const float2*>(p.u) + boff * p.K;
+    const float2* gb = reinterpret_cast<const float2*>(p.g) + boff * p.K;
+    float2* hb = p.h ? reinterpret_cast<float2*>(p.h) + boff * p.K : nullptr;
+    const float* rb = p.r + boff;
+    const float* pb = p.phi + boff;
+
+    auto issue = [&](int j, int st) {
+        const int t0 = j * TT;
+        cp_async_tile<float2, KT>(su[st], ub, t0, TT, p.L, k0, p.K, tid, KT);
+        cp_async_tile<float2, KT>(sgt[st], gb, t0, TT, p.L, k0, p.K, tid, KT);
+        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+        cp_async_commit();
+    };
+    if (ntiles > 0) issue(0, 0);
+    for (int j = 0; j < ntiles; ++j) {
+        const int st = j & 1;
+        if (j + 1 < ntiles) {
+            issue(j + 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int t0 = j * TT;
+        const int rows = min(TT, p.L - t0);
+        step_scalars(sr[st], sp[st], ssp, rows, tid);
+        __syncthreads();
+        for (int r0 = 0; r0 < rows; r0 += CB) {
+            float2 a[CB];
+            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                const int r = r0 + u;
+                if (r < rows) {
+                    const float2 sp2 = ssp[r];  // (s, phi)
+                    const float2 ah = cmul(a[u], h);
+                    const float2 al = cmul(a[u], Sl), ao = cmul(a[u], So);
+                    Sl = make_float2(fmaf(-sp2.x, ah.x, al.x), fmaf(-sp2.x, ah.y, al.y));
+                    So = make_float2(fmaf(-sp2.y, ah.y, ao.x), fmaf(sp2.y, ah.x, ao.y));
+                    const float2 uu = su[st][r * KT + tid];
+                    h = make_float2(ah.x + uu.x, ah.y + uu.y);
+                    const float2 gg = sgt[st][r * KT + tid];
+                    dl = fmaf(gg.x, Sl.x, fmaf(gg.y, Sl.y, dl));
+                    dom = fmaf(gg.x, So.x, fmaf(gg.y, So.y, dom));
+                    if (hb && kv) hb[(size_t)(t0 + r) * p.K + k] = h;
+                }
+            }
+        }
+        __syncthreads();  // stage st and the step scalars are free again
+    }
+    if (kv) {
+        reinterpret_cast<float2*>(p.lo_part)[(size_t)b * p.K + k] = make_float2(dl, dom);
+        if (stb) {
+            stb[k] = h;
+            stb[p.K + k] = Sl;
+            stb[2 * p.K + k] = So;
+        }
+        if (!(isfinite(h.x) && isfinite(h.y) && isfinite(Sl.x) && isfinite(Sl.y) &&
+              isfinite(So.x) && isfinite(So.y)))
+            flag_status(p.status, kStatusNonFinite);
+    }
+}
+
 // dr = -sigmoid(r) * sum over mode tiles of sum_k lambda Re q;  dphi = sum of sum_k omega Im q.
 __global__ void cplx_reduce_bl_kernel(CplxArgs p) {
     const int64_t n = (int64_t)p.B * p.L;
@@ -436,6 +529,14 @@ cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     cplx_fwd_kernel<false><<<dim3(a.nkt, a.B, a.nseg), KT, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cplx_rtrl(const CplxArgs& a, cudaStream_t st) {
+    cudaError_t e;
+    cplx_rtrl_kernel<<<dim3(a.nkt, a.B, 1), KT, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cplx_reduce_k_kernel<<<(a.K + 255) / 256, 256, 0, st>>>(a);  // sums over b (nseg = 1)
     return cudaGetLastError();
 }
 

@@ -90,6 +90,7 @@ struct CplxArgs {
     float* win;         // [B][nseg][K][2] adjoint entering each segment from its end
     float* rp_part;     // [nkt][B][L][2] per-CTA sums of lambda*Re q and omega*Im q
     float* lo_part;     // [B][nseg][K][2] per-segment sums of -s Re q and phi Im q
+    float* state;       // RTRL: [B][3][K][2] (h, dh/dlambda, dh/domega) carried across calls, or null
     unsigned* status;
 };
 
@@ -97,6 +98,7 @@ struct CplxArgs {
 cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st);
 cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cudaStream_t st);
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st);
+cudaError_t launch_cplx_rtrl(const CplxArgs& a, cudaStream_t st);
 cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st);
 
 }  // namespace ssm

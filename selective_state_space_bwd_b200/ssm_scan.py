@@ -58,7 +58,8 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_complex_workspace_bytes",
             "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
             "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
-            "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex"]
+            "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex",
+            "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl"]
 
 
 def lib():
@@ -93,6 +94,10 @@ def lib():
             L.ssm_status_string.argtypes, L.ssm_status_string.restype = [I], ctypes.c_char_p
             L.ssm_scan_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P]
             L.ssm_scan_fwd_noalloc.restype = I
+            L.ssm_scan_complex_rtrl_workspace_bytes.argtypes = [CP]
+            L.ssm_scan_complex_rtrl_workspace_bytes.restype = Z
+            L.ssm_scan_complex_rtrl.argtypes = [CP] + [P] * 11 + [Z, P]
+            L.ssm_scan_complex_rtrl.restype = I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -320,3 +325,36 @@ def ssm_scan_complex_bwd(h, r, phi, lam, omega, g, chunk=128, seg_chunks=0, out=
 def ssm_scan_status(ws, stream=None) -> int:
     """Synchronise the stream and return the device status word a call left in ``ws``."""
     return int(lib().ssm_scan_status(_p(ws), _stream(stream)))
+
+
+def complex_rtrl_workspace_bytes(shape: SsmCShape) -> int:
+    return int(lib().ssm_scan_complex_rtrl_workspace_bytes(ctypes.byref(shape)))
+
+
+def ssm_scan_complex_rtrl(u, r, phi, lam, omega, g, state=None, want_h=False, chunk=128,
+                          h=None, out=None, ws=None, stream=None):
+    """Complex forward with exact structured RTRL: returns dict dlambda, domega [K] (the gradient
+    of Re sum conj(g) h accumulated online), and h [B,L,K] if ``want_h`` or ``h`` is given.
+    ``state`` [B,3,K] complex64 (h, dh/dlambda, dh/domega) is read before the first step and
+    updated in place after the last (None: start from zero)."""
+    _need_cuda(u, r, phi, lam, omega, g, state, h)
+    if u.dtype != torch.complex64 or g.dtype != torch.complex64:
+        raise ValueError("u and g must be complex64")
+    B, L, K = u.shape
+    shape = complex_shape(B, L, K, chunk, 0)
+    if h is None and want_h:
+        h = torch.empty_like(u)
+    if state is not None and (state.dtype != torch.complex64 or tuple(state.shape) != (B, 3, K)
+                              or not state.is_contiguous()):
+        raise ValueError("state must be a contiguous complex64 [B, 3, K] tensor")
+    if out is None:
+        out = dict(dlambda=torch.empty_like(lam), domega=torch.empty_like(omega))
+    ws = _workspace(complex_rtrl_workspace_bytes(shape), u.device, ws)
+    code = lib().ssm_scan_complex_rtrl(ctypes.byref(shape), _p(u), _p(r), _p(phi), _p(lam),
+                                       _p(omega), _p(g), _p(h), _p(state), _p(out["dlambda"]),
+                                       _p(out["domega"]), _p(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream))
+    _check(code, "ssm_scan_complex_rtrl")
+    if h is not None:
+        out["h"] = h
+    return out

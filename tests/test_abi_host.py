@@ -154,6 +154,23 @@ def test_option_validation(S):
     assert L.ssm_scan_bwd_ex(ctypes.byref(shp), None, *pb, needb - 256, None) == 4
 
 
+def test_rtrl_validation(S):
+    L = S.lib()
+    shp = S.complex_shape(2, 64, 128, 32)
+    need = S.complex_rtrl_workspace_bytes(shp)
+    assert need >= 256 + 2 * 128 * 8
+    p = _fake_ptrs(11)
+    assert L.ssm_scan_complex_rtrl(ctypes.byref(shp), *p, need - 1, None) == 4
+    q = list(p)
+    q[5] = None  # g
+    assert L.ssm_scan_complex_rtrl(ctypes.byref(shp), *q, need, None) == 1
+    q = list(p)
+    q[8] = ctypes.c_void_p(0x100008)  # state misaligned
+    assert L.ssm_scan_complex_rtrl(ctypes.byref(shp), *q, need, None) == 3
+    odd = S.complex_shape(2, 64, 127, 32)
+    assert L.ssm_scan_complex_rtrl(ctypes.byref(odd), *p, need, None) == 3
+
+
 def test_complex_validation(S):
     L = S.lib()
     shp = S.complex_shape(2, 64, 16, 32)
