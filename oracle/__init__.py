@@ -52,6 +52,9 @@ def _load():
             lib.ssm_oracle_complex.restype = ctypes.c_int
             lib.ssm_oracle_complex_rtrl.argtypes = [I64, I64, I64] + [P] * 6 + [ctypes.c_int] + [P] * 4
             lib.ssm_oracle_complex_rtrl.restype = ctypes.c_int
+            lib.ssm_oracle_pdssm.argtypes = ([I64] * 5 + [P] * 6 + [ctypes.c_double, ctypes.c_int] +
+                                             [P] * 6)
+            lib.ssm_oracle_pdssm.restype = ctypes.c_int
             lib.ssm_oracle_max_threads.argtypes = []
             lib.ssm_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -173,4 +176,35 @@ def complex_rtrl(u, r, phi, lam, omega, g, state=None, want_h=False, threads=0):
                                      _ptr(st), _ptr(out["dlambda"]), _ptr(out["domega"]))
     if rc != 0:
         raise RuntimeError("ssm_oracle_complex_rtrl failed (bad argument)")
+    return out
+
+
+def pdssm(scores, dictionary, d, bt, h0=None, g=None, tau=1.0, threads=0):
+    """Flash PD-SSM scan (hard selection forward, straight-through backward) in float64.
+
+    Shapes: scores [B,L,H,K]; dictionary [K,N] int (row of the single 1 in each column of each
+    dictionary matrix); d, bt, g [B,L,H,N]; h0 [B,H,N].  Returns h [B,L,H,N] and sel [B,L,H]
+    (int32), plus dd, dbt [B,L,H,N], dscores [B,L,H,K], dh0 [B,H,N] when ``g`` is given.
+    """
+    lib = _load()
+    scores, d, bt = _f64(scores), _f64(d), _f64(bt)
+    dic = np.ascontiguousarray(dictionary, dtype=np.int32)
+    B, L, H, K = scores.shape
+    N = d.shape[-1]
+    assert dic.shape == (K, N) and d.shape == (B, L, H, N) and bt.shape == (B, L, H, N)
+    if h0 is not None:
+        h0 = _f64(h0)
+        assert h0.shape == (B, H, N)
+    out = {"h": np.full((B, L, H, N), np.nan), "sel": np.full((B, L, H), -1, dtype=np.int32)}
+    if g is not None:
+        g = _f64(g)
+        assert g.shape == (B, L, H, N)
+        out.update(dd=np.full((B, L, H, N), np.nan), dbt=np.full((B, L, H, N), np.nan),
+                   dscores=np.full((B, L, H, K), np.nan), dh0=np.full((B, H, N), np.nan))
+    rc = lib.ssm_oracle_pdssm(B, L, H, N, K, _ptr(scores), _ptr(dic), _ptr(d), _ptr(bt), _ptr(h0),
+                              _ptr(g), float(tau), int(threads), _ptr(out["h"]), _ptr(out["sel"]),
+                              _ptr(out.get("dd")), _ptr(out.get("dbt")), _ptr(out.get("dscores")),
+                              _ptr(out.get("dh0")))
+    if rc != 0:
+        raise RuntimeError("ssm_oracle_pdssm failed (bad argument or out of memory)")
     return out

@@ -419,3 +419,114 @@ int ssm_oracle_complex_rtrl(int64_t B, int64_t L, int64_t K,
     }
     return 0;
 }
+
+/*
+ * Flash PD-SSM scan ("Flash PD-SSM: Memory-Optimized Structured Sparse State-Space Models",
+ * technical summary: hard selection and gradient propagation).  Per batch b and head e, a real
+ * state h in R^N; at every step the transition is A_t = P_{k_t} D_t, where
+ *   k_t = argmax_k scores[b,t,e,k]   (ties: the lowest k),
+ *   P_k is dictionary matrix k, a one-hot column selector: column j holds a single 1, in row
+ *       dict[k*N + j]  (so (P_k v)_i = sum over j with dict[k*N+j] == i of v_j),
+ *   D_t = diag(d[b,t,e,:]),
+ * and h_t = A_t h_{t-1} + bt[b,t,e,:], h_{-1} = h0 (NULL: zero).  Outputs h [B,L,H,N] and the
+ * selection sel [B,L,H] (k_t).
+ * Backward (g = dL/dh_t given for every t, so L = sum_t <g_t, h_t>): with the hard forward
+ * matrices the adjoint is mu_t = g_t + A_{t+1}^T mu_{t+1}, (A^T mu)_j = d_j mu_{dict[k*N+j]};
+ *   dbt_t = mu_t,   dd_t[j] = mu_t[dict[k_t*N+j]] h_{t-1}[j],   dh0 = A_0^T mu_0.
+ * The selection is discrete, so its gradient is the straight-through surrogate of the summary
+ * (the hard choice in the forward pass, a temperature-tau softmax p = softmax(scores_t / tau) in
+ * the backward pass):  c_k = <mu_t, P_k D_t h_{t-1}>,  dscores_t[k] = p_k (c_k - sum_k' p_k' c_k') / tau.
+ * g NULL: forward only.  Returns 0 or -1.
+ */
+int ssm_oracle_pdssm(int64_t B, int64_t L, int64_t H, int64_t N, int64_t K,
+                     const double* scores, const int32_t* dict, const double* d, const double* bt,
+                     const double* h0, const double* g, double tau, int nthreads,
+                     double* h_out, int32_t* sel_out, double* dd, double* dbt, double* dscores,
+                     double* dh0) {
+    if (B < 0 || L < 0 || H <= 0 || N <= 0 || K <= 0 || !scores || !dict || !d || !bt || !h_out)
+        return -1;
+    if (g && !(tau > 0.0)) return -1;
+    for (int64_t i = 0; i < K * N; ++i)
+        if (dict[i] < 0 || dict[i] >= N) return -1;
+    nthreads = pick_threads(nthreads);
+    int fail = 0;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* hprev = (double*)malloc(sizeof(double) * (size_t)N);
+        double* hnew = (double*)malloc(sizeof(double) * (size_t)N);
+        double* mu = (double*)malloc(sizeof(double) * (size_t)N);
+        double* w = (double*)malloc(sizeof(double) * (size_t)N);
+        double* c = (double*)malloc(sizeof(double) * (size_t)K);
+        double* p = (double*)malloc(sizeof(double) * (size_t)K);
+        if (!hprev || !hnew || !mu || !w || !c || !p) {
+#pragma omp atomic write
+            fail = 1;
+        }
+#pragma omp barrier
+        if (!fail) {
+#pragma omp for schedule(static)
+            for (int64_t be = 0; be < B * H; ++be) {
+                const int64_t b = be / H, e = be % H;
+                /* forward */
+                for (int64_t n = 0; n < N; ++n) hprev[n] = h0 ? h0[be * N + n] : 0.0;
+                for (int64_t t = 0; t < L; ++t) {
+                    const int64_t row = (b * L + t) * H + e;   /* (b, t, e) */
+                    const double* sc = scores + row * K;
+                    int64_t kb = 0;
+                    for (int64_t k = 1; k < K; ++k)
+                        if (sc[k] > sc[kb]) kb = k;
+                    if (sel_out) sel_out[row] = (int32_t)kb;
+                    for (int64_t n = 0; n < N; ++n) hnew[n] = bt[row * N + n];
+                    for (int64_t j = 0; j < N; ++j) hnew[dict[kb * N + j]] += d[row * N + j] * hprev[j];
+                    for (int64_t n = 0; n < N; ++n) {
+                        h_out[row * N + n] = hnew[n];
+                        hprev[n] = hnew[n];
+                    }
+                }
+                if (!g) continue;
+                /* backward: w = A_{t+1}^T mu_{t+1} */
+                for (int64_t n = 0; n < N; ++n) w[n] = 0.0;
+                for (int64_t t = L - 1; t >= 0; --t) {
+                    const int64_t row = (b * L + t) * H + e;
+                    const double* sc = scores + row * K;
+                    int64_t kb = 0;
+                    for (int64_t k = 1; k < K; ++k)
+                        if (sc[k] > sc[kb]) kb = k;
+                    for (int64_t n = 0; n < N; ++n) mu[n] = g[row * N + n] + w[n];
+                    const double* hp = t > 0 ? h_out + (row - H) * N : NULL;  /* (b, t-1, e) */
+                    for (int64_t n = 0; n < N; ++n) {
+                        const double hpn = t > 0 ? hp[n] : (h0 ? h0[be * N + n] : 0.0);
+                        if (dbt) dbt[row * N + n] = mu[n];
+                        if (dd) dd[row * N + n] = mu[dict[kb * N + n]] * hpn;
+                        w[n] = d[row * N + n] * mu[dict[kb * N + n]];
+                    }
+                    if (dscores) {
+                        double mx = sc[0];
+                        for (int64_t k = 1; k < K; ++k) mx = sc[k] > mx ? sc[k] : mx;
+                        double zs = 0.0;
+                        for (int64_t k = 0; k < K; ++k) {
+                            p[k] = exp((sc[k] - mx) / tau);
+                            zs += p[k];
+                        }
+                        double pc = 0.0;
+                        for (int64_t k = 0; k < K; ++k) {
+                            double ck = 0.0;
+                            for (int64_t j = 0; j < N; ++j) {
+                                const double hpj = t > 0 ? hp[j] : (h0 ? h0[be * N + j] : 0.0);
+                                ck += mu[dict[k * N + j]] * d[row * N + j] * hpj;
+                            }
+                            p[k] /= zs;
+                            c[k] = ck;
+                            pc += p[k] * ck;
+                        }
+                        for (int64_t k = 0; k < K; ++k) dscores[row * K + k] = p[k] * (c[k] - pc) / tau;
+                    }
+                }
+                if (dh0)
+                    for (int64_t n = 0; n < N; ++n) dh0[be * N + n] = w[n];
+            }
+        }
+        free(hprev); free(hnew); free(mu); free(w); free(c); free(p);
+    }
+    return fail ? -1 : 0;
+}

@@ -148,3 +148,21 @@ def workload_inputs(name, seed=0):
     if isinstance(w, ComplexWorkload):
         return complex_inputs(w.batch, w.seqlen, w.modes, seed)
     return real_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed)
+
+
+def pdssm_inputs(batch, seqlen, heads, nstate, ndict, seed=0):
+    """Draw one Flash PD-SSM problem.
+
+    scores ~ N(0,1) [B,L,H,K]; dictionary: K random maps of the N columns to rows (each column of
+    each matrix holds a single 1), [K,N] int32; d ~ U(0.3, 0.9) [B,L,H,N] (so every transition
+    shrinks the state's 1-norm); bt, g ~ N(0,1) [B,L,H,N]; h0 ~ N(0,1) [B,H,N].
+    """
+    rng = np.random.default_rng(seed)
+    B, L, H, N, K = int(batch), int(seqlen), int(heads), int(nstate), int(ndict)
+    dictionary = rng.integers(0, N, size=(K, N), dtype=np.int32)
+    scores = rng.standard_normal((B, L, H, K), dtype=np.float32)
+    d = rng.uniform(0.3, 0.9, size=(B, L, H, N)).astype(np.float32)
+    bt = rng.standard_normal((B, L, H, N), dtype=np.float32)
+    g = rng.standard_normal((B, L, H, N), dtype=np.float32)
+    h0 = rng.standard_normal((B, H, N), dtype=np.float32)
+    return dict(scores=scores, dictionary=dictionary, d=d, bt=bt, g=g, h0=h0)
