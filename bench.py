@@ -242,6 +242,8 @@ def run_reference(args, w):
     oracle.build()
     threads = oracle.max_threads()
     cplx = isinstance(w, gen.ComplexWorkload)
+    if isinstance(w, gen.PdWorkload):
+        return run_reference_pdssm(args, w)
     if cplx:
         inp = gen.complex_inputs(1, w.seqlen, w.modes, seed=0)
         upd = w.seqlen * w.modes
@@ -478,6 +480,196 @@ def main_complex(args, w):
         dist.destroy_process_group()
 
 
+def pdssm_algorithmic_bytes(w):
+    """Minimum bytes of one Flash PD-SSM fwd + bwd.  Forward: scores, d, bt read; h, sel written.
+    Backward: scores, d, h, sel, g read; dd, dbt, dscores written (fp32; sel int32)."""
+    BLH = w.batch * w.seqlen * w.heads
+    upd = BLH * w.nstate
+    return 12 * upd + (4 * w.ndict + 4) * BLH, 20 * upd + (8 * w.ndict + 4) * BLH
+
+
+def oracle_sample_pdssm(w, inp, budget_s=(10.0, 30.0)):
+    """Time the float64 oracle's Flash PD-SSM fwd + bwd on whole batch rows."""
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    rows, t_total, b = 0, 0.0, 0
+    while t_total < budget_s[0]:
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        oracle.pdssm(inp["scores"][sl], inp["dictionary"], inp["d"][sl], inp["bt"][sl],
+                     inp["h0"][sl], inp["g"][sl], tau=1.0, threads=threads)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        rows += 1
+        b = (b + 1) % w.batch
+        if t_total + dt > budget_s[1]:
+            break
+    upd = rows * w.seqlen * w.heads * w.nstate
+    return {"value": upd / t_total, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, H={w.heads}, "
+                      f"N={w.nstate}, K={w.ndict}), fwd+bwd in float64, {t_total:.1f} s"}
+
+
+def main_pdssm(args, w):
+    """Flash PD-SSM: ssm_pdssm_fwd + ssm_pdssm_bwd per step.  Batch rows are independent and no
+    parameter gradient is summed, so ranks exchange nothing but the timing."""
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_bwd_b200 import build, ssm_scan as S
+    from selective_state_space_bwd_b200 import inputs as gen
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    S.lib()
+    inp = gen.pdssm_inputs(w.batch, w.seqlen, w.heads, w.nstate, w.ndict, seed=rank)
+    host = {k: torch.from_numpy(v).pin_memory() for k, v in inp.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    h = torch.empty_like(d["d"])
+    sel = torch.empty((w.batch, w.seqlen, w.heads), dtype=torch.int32, device=dev)
+    out = dict(dd=torch.empty_like(d["d"]), dbt=torch.empty_like(d["d"]),
+               dscores=torch.empty_like(d["scores"]), dh0=torch.empty_like(d["h0"]))
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        S.ssm_pdssm_fwd(d["scores"], d["dictionary"], d["d"], d["bt"], h0=d["h0"], h=h, sel=sel,
+                        ws=ws, stream=stream)
+
+    def bwd():
+        S.ssm_pdssm_bwd(d["scores"], d["dictionary"], d["d"], h, sel, d["g"], tau=1.0, h0=d["h0"],
+                        out=out, ws=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        fwd(); bwd()
+    torch.cuda.synchronize()
+    if S.ssm_scan_status(ws) != 0:
+        raise SystemExit("device status word reports an error")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream); fwd(); e[1].record(stream); bwd(); e[2].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    tt = torch.tensor([t_fwd + t_bwd, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    t_step, t_fwd, t_bwd = tt.tolist()
+
+    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+    hh = torch.empty(h.shape, dtype=h.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = hh.numel() * hh.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+
+    def e2e_step():
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        fwd(); bwd()
+        hh.copy_(h, non_blocking=True)
+        for k, v in out.items():
+            hout[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    t_e2e = float(t_e2e)
+
+    upd_rank = w.batch * w.seqlen * w.heads * w.nstate
+    value = world * upd_rank * args.steps / t_step
+    hbm, peak_kind = peaks()
+    fb, bb = pdssm_algorithmic_bytes(w)
+    fwd_gbs = fb / (t_fwd / args.steps) / 1e9
+    bwd_gbs = bb / (t_bwd / args.steps) / 1e9
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded generator: random dictionary maps, N(0,1) scores)",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "heads": w.heads,
+                       "nstate": w.nstate, "ndict": w.ndict, "tau": 1.0,
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (weak: one full batch per rank, no exchange)"
+                                      if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": "ssm_pdssm_bwd call (reverse scan + score "
+                         "gradient)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+            "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
+            "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
+            "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_sample_pdssm(w, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference_pdssm(args, w):
+    """The oracle on one batch row of the Flash PD-SSM workload per step (rank 0 only)."""
+    from selective_state_space_bwd_b200 import inputs as gen
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    inp = gen.pdssm_inputs(1, w.seqlen, w.heads, w.nstate, w.ndict, seed=0)
+    upd = w.seqlen * w.heads * w.nstate
+    times = []
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.pdssm(inp["scores"], inp["dictionary"], inp["d"], inp["bt"], inp["h0"], inp["g"],
+                     tau=1.0, threads=threads)
+        if k >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = upd * len(times) / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "heads": w.heads,
+                       "nstate": w.nstate, "ndict": w.ndict, "sample": "one batch row per step",
+                       "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"1 of {w.batch} batch rows of {w.name} per step, float64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.memory_curve:
@@ -488,6 +680,8 @@ def main():
         return run_reference(args, w)
     if isinstance(w, gen.ComplexWorkload):
         return main_complex(args, w)
+    if isinstance(w, gen.PdWorkload):
+        return main_pdssm(args, w)
 
     import torch
     import torch.distributed as dist

@@ -259,6 +259,50 @@ int ssm_scan_complex_rtrl(const ssm_cshape* shape,
                           void* h, void* state, float* dlambda, float* domega,
                           void* ws, size_t ws_bytes, ssm_stream_t stream);
 
+/* ------------------------------------------------------------------------------------------
+ * Flash PD-SSM ("Flash PD-SSM: Memory-Optimized Structured Sparse State-Space Models",
+ * technical summary: hard selection, gradient propagation).  Per batch b and head e a real state
+ * h in R^N; at every step one of K dictionary matrices is chosen by the step's scores and
+ * multiplied by a diagonal:
+ *     k_t = argmax_k scores[b,t,e,k]   (ties: the lowest k)
+ *     h_t = P_{k_t} D_t h_{t-1} + bt_t,   D_t = diag(d[b,t,e,:]),   h_{-1} = h0 (NULL: zero)
+ * P_k is a one-hot column selector: column j holds a single 1, in row dict[k*N + j] (several
+ * columns may share a row).  Layout: scores [B,L,H,K], d, bt, h, g, dd, dbt [B,L,H,N] fp32,
+ * dict [K,N] int32 (entries in [0, N); an entry out of range is clamped and sets
+ * SSM_ERR_INVALID_ARG in the workspace status word), sel [B,L,H] int32, h0, dh0 [B,H,N] fp32.
+ */
+typedef struct ssm_pdshape {
+    int64_t batch;   /* B >= 0 */
+    int64_t seqlen;  /* L >= 0 */
+    int64_t heads;   /* H >= 1 */
+    int32_t nstate;  /* N, one of 4, 8, 16, 32 */
+    int32_t ndict;   /* K, 1..32 */
+    int32_t reserved; /* must be 0 */
+    int32_t reserved2; /* must be 0 */
+} ssm_pdshape;
+
+/* Workspace bytes of the PD-SSM calls (the status word: 256); 0 for an invalid shape. */
+size_t ssm_pdssm_workspace_bytes(const ssm_pdshape* shape);
+
+/* Forward: writes the trajectory h and the selection sel.  Enqueues 2 kernels (argmax, scan).
+ * Returns an ssm_status. */
+int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* dict,
+                  const float* d, const float* bt, const float* h0, float* h, int32_t* sel,
+                  void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/* Backward of L = sum_t <g_t, h_t> for the forward above (h and sel as it wrote them).  The
+ * adjoint runs through the hard forward matrices,
+ *     mu_t = g_t + A_{t+1}^T mu_{t+1},   (A^T mu)_j = d_j mu[dict[k*N + j]],
+ *     dbt = mu,   dd_t[j] = mu_t[dict[k_t*N + j]] h_{t-1}[j],   dh0 = A_0^T mu_0 (dh0 may be NULL),
+ * and the discrete selection gets the straight-through surrogate with temperature tau > 0
+ * (hard in the forward pass, softmax(scores / tau) in the backward pass):
+ *     c_k = <mu_t, P_k D_t h_{t-1}>,   dscores_t[k] = p_k (c_k - sum_k' p_k' c_k') / tau.
+ * Enqueues 2 kernels (reverse scan, score gradient).  Returns an ssm_status. */
+int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, const int32_t* dict,
+                  const float* d, const float* h0, const float* h, const int32_t* sel,
+                  const float* g, float* dd, float* dbt, float* dscores, float* dh0,
+                  void* ws, size_t ws_bytes, ssm_stream_t stream);
+
 /* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);

@@ -433,6 +433,79 @@ int ssm_scan_complex_bwd(const ssm_cshape* shape, const void* h, const float* r,
     return ssm::launch_cplx_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------------------ Flash PD-SSM
+namespace {
+int check_pdshape(const ssm_pdshape* s) {
+    if (!s) return SSM_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->heads < 1 || s->reserved != 0 || s->reserved2 != 0)
+        return SSM_ERR_INVALID_ARG;
+    if (s->nstate != 4 && s->nstate != 8 && s->nstate != 16 && s->nstate != 32) return SSM_ERR_UNSUPPORTED;
+    if (s->ndict < 1 || s->ndict > 32) return SSM_ERR_UNSUPPORTED;
+    if (s->batch > 65535 || s->seqlen > (int64_t)1 << 30 || s->heads > (int64_t)1 << 24 ||
+        (double)s->batch * s->seqlen * s->heads * s->nstate > 9.0e15)
+        return SSM_ERR_UNSUPPORTED;
+    return SSM_OK;
+}
+
+ssm::PdArgs pd_args(const ssm_pdshape* s, void* ws) {
+    ssm::PdArgs a = {};
+    a.B = (int)s->batch; a.L = (int)s->seqlen; a.H = (int)s->heads; a.N = s->nstate; a.K = s->ndict;
+    a.status = at<unsigned>(ws, 0);
+    return a;
+}
+}  // namespace
+
+size_t ssm_pdssm_workspace_bytes(const ssm_pdshape* shape) {
+    return check_pdshape(shape) == SSM_OK ? kStatusBytes : 0;
+}
+
+int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* dict,
+                  const float* d, const float* bt, const float* h0, float* h, int32_t* sel,
+                  void* ws, size_t ws_bytes, ssm_stream_t stream) {
+    int st = check_pdshape(shape);
+    if (st != SSM_OK) return st;
+    const size_t BLH = (size_t)shape->batch * shape->seqlen * shape->heads;
+    const size_t N = shape->nstate, K = shape->ndict, BH = (size_t)shape->batch * shape->heads;
+    const void* ptrs[] = {scores, dict, d, bt, h, sel, ws, h0};
+    const size_t counts[] = {BLH * K, K * N, BLH * N, BLH * N, BLH * N, BLH, 1, h0 ? BH * N : 0};
+    if ((st = check_arrays(ptrs, counts, 8)) != SSM_OK) return st;
+    if (ws_bytes < kStatusBytes) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (BLH == 0) return SSM_OK;
+    ssm::PdArgs a = pd_args(shape, ws);
+    a.scores = scores; a.dict = dict; a.d = d; a.bt = bt; a.h0 = h0; a.h = h; a.sel = sel;
+    return ssm::launch_pdssm_fwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, const int32_t* dict,
+                  const float* d, const float* h0, const float* h, const int32_t* sel,
+                  const float* g, float* dd, float* dbt, float* dscores, float* dh0, void* ws,
+                  size_t ws_bytes, ssm_stream_t stream) {
+    int st = check_pdshape(shape);
+    if (st != SSM_OK) return st;
+    if (!(tau > 0.0f && tau < 3.0e38f)) return SSM_ERR_INVALID_ARG;
+    const size_t BLH = (size_t)shape->batch * shape->seqlen * shape->heads;
+    const size_t N = shape->nstate, K = shape->ndict, BH = (size_t)shape->batch * shape->heads;
+    const void* ptrs[] = {scores, dict, d, h, sel, g, dd, dbt, dscores, ws, h0, dh0};
+    const size_t counts[] = {BLH * K, K * N, BLH * N, BLH * N, BLH, BLH * N, BLH * N, BLH * N,
+                             BLH * K, 1, h0 ? BH * N : 0, dh0 ? BH * N : 0};
+    if ((st = check_arrays(ptrs, counts, 12)) != SSM_OK) return st;
+    if (ws_bytes < kStatusBytes) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (BLH == 0) {  // no steps: dL/dh0 = 0
+        if (dh0 && BH && cudaMemsetAsync(dh0, 0, BH * N * sizeof(float), s) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::PdArgs a = pd_args(shape, ws);
+    a.tau = tau; a.scores = scores; a.dict = dict; a.d = d; a.h0 = h0;
+    a.h = const_cast<float*>(h); a.sel = const_cast<int32_t*>(sel); a.g = g;
+    a.dd = dd; a.dbt = dbt; a.dscores = dscores; a.dh0 = dh0;
+    return ssm::launch_pdssm_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 int ssm_scan_status(const void* ws, ssm_stream_t stream) {
     if (!ws) return SSM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -94,7 +94,30 @@ struct CplxArgs {
     unsigned* status;
 };
 
+// Flash PD-SSM: N lanes per (batch, head) sequence (lane = state), kPdThreads per CTA.
+constexpr int kPdThreads = 128;
+
+struct PdArgs {
+    int B, L, H, N, K;
+    float tau;
+    const float* scores;   // [B][L][H][K]
+    const int32_t* dict;   // [K][N]: row of the single 1 in column j of dictionary matrix k
+    const float* d;        // [B][L][H][N]
+    const float* bt;       // [B][L][H][N]
+    const float* h0;       // [B][H][N] or null
+    float* h;              // forward: trajectory out; backward: trajectory in
+    int32_t* sel;          // forward: selection out; backward: in
+    const float* g;        // backward: dL/dh [B][L][H][N]
+    float* dd;
+    float* dbt;            // backward: also the adjoint mu read by the score-gradient kernel
+    float* dscores;
+    float* dh0;
+    unsigned* status;
+};
+
 // Launchers (return cudaGetLastError() of the last launch).
+cudaError_t launch_pdssm_fwd(const PdArgs& a, cudaStream_t st);
+cudaError_t launch_pdssm_bwd(const PdArgs& a, cudaStream_t st);
 cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st);
 cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cudaStream_t st);
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st);

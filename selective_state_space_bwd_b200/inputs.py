@@ -14,6 +14,8 @@ Phase Gradient Flow abstract's 128,000-step impulse-response benchmark):
 * ``mamba1p4b_layer`` B=4, L=8192,   D=4096, N=16, bf16
 * ``sparc_complex``   B=16, L=4096,  K=2048 complex modes (SPARC shared retention/phase control)
 * ``sparc_complex_b4`` the same with B=4 (a quarter of the data: profiling captures)
+* ``pdssm_l5120``     Flash PD-SSM scan: B=8, L=5120 (the sequence length of the Flash PD-SSM
+                      throughput comparison), H=256 heads, N=16 states, K=8 dictionary matrices
 
 Draw order (one ``numpy.random.default_rng(seed)`` stream, float32 draws): real mode
 A_log (stiff only), delta_raw, x, Bm, Cm, Dskip, dy; complex mode lambda, omega, r, phi, u, g.
@@ -58,6 +60,7 @@ WORKLOADS = {
     "mamba1p4b_layer": RealWorkload("mamba1p4b_layer", 4, 8192, 4096, 16, 128, BF16, "mamba"),
     "sparc_complex": ComplexWorkload("sparc_complex", 16, 4096, 2048, 128),
     "sparc_complex_b4": ComplexWorkload("sparc_complex_b4", 4, 4096, 2048, 128),
+    "pdssm_l5120": None,  # filled below (PdWorkload is defined after this table)
 }
 
 
@@ -147,6 +150,8 @@ def workload_inputs(name, seed=0):
     w = WORKLOADS[name]
     if isinstance(w, ComplexWorkload):
         return complex_inputs(w.batch, w.seqlen, w.modes, seed)
+    if type(w).__name__ == "PdWorkload":
+        return pdssm_inputs(w.batch, w.seqlen, w.heads, w.nstate, w.ndict, seed)
     return real_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.io, w.kind, seed)
 
 
@@ -166,3 +171,16 @@ def pdssm_inputs(batch, seqlen, heads, nstate, ndict, seed=0):
     g = rng.standard_normal((B, L, H, N), dtype=np.float32)
     h0 = rng.standard_normal((B, H, N), dtype=np.float32)
     return dict(scores=scores, dictionary=dictionary, d=d, bt=bt, g=g, h0=h0)
+
+
+@dataclass(frozen=True)
+class PdWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    heads: int
+    nstate: int
+    ndict: int
+
+
+WORKLOADS["pdssm_l5120"] = PdWorkload("pdssm_l5120", 8, 5120, 256, 16, 8)

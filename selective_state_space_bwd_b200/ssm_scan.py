@@ -45,6 +45,12 @@ class SsmOptions(ctypes.Structure):
                 ("dh0", ctypes.c_void_p)]
 
 
+class SsmPdShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("heads", ctypes.c_int64),
+                ("nstate", ctypes.c_int32), ("ndict", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("reserved2", ctypes.c_int32)]
+
+
 class SsmError(RuntimeError):
     def __init__(self, code, what):
         self.code = code
@@ -59,7 +65,8 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
             "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
             "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex",
-            "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl"]
+            "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
+            "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd"]
 
 
 def lib():
@@ -98,6 +105,12 @@ def lib():
             L.ssm_scan_complex_rtrl_workspace_bytes.restype = Z
             L.ssm_scan_complex_rtrl.argtypes = [CP] + [P] * 11 + [Z, P]
             L.ssm_scan_complex_rtrl.restype = I
+            PP = ctypes.POINTER(SsmPdShape)
+            L.ssm_pdssm_workspace_bytes.argtypes, L.ssm_pdssm_workspace_bytes.restype = [PP], Z
+            L.ssm_pdssm_fwd.argtypes = [PP] + [P] * 8 + [Z, P]
+            L.ssm_pdssm_fwd.restype = I
+            L.ssm_pdssm_bwd.argtypes = [PP, ctypes.c_float] + [P] * 12 + [Z, P]
+            L.ssm_pdssm_bwd.restype = I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -357,4 +370,52 @@ def ssm_scan_complex_rtrl(u, r, phi, lam, omega, g, state=None, want_h=False, ch
     _check(code, "ssm_scan_complex_rtrl")
     if h is not None:
         out["h"] = h
+    return out
+
+
+def pdssm_shape(batch, seqlen, heads, nstate, ndict):
+    return SsmPdShape(int(batch), int(seqlen), int(heads), int(nstate), int(ndict), 0, 0)
+
+
+def pdssm_workspace_bytes(shape: SsmPdShape) -> int:
+    return int(lib().ssm_pdssm_workspace_bytes(ctypes.byref(shape)))
+
+
+def ssm_pdssm_fwd(scores, dictionary, d, bt, h0=None, h=None, sel=None, ws=None, stream=None):
+    """Flash PD-SSM forward: scores [B,L,H,K], dictionary [K,N] int32, d, bt [B,L,H,N] fp32,
+    h0 [B,H,N] (None: zero).  Returns (h [B,L,H,N], sel [B,L,H] int32)."""
+    _need_cuda(scores, dictionary, d, bt, h0)
+    B, L, H, K = scores.shape
+    N = d.shape[-1]
+    shape = pdssm_shape(B, L, H, N, K)
+    if h is None:
+        h = torch.empty_like(d)
+    if sel is None:
+        sel = torch.empty((B, L, H), dtype=torch.int32, device=d.device)
+    ws = _workspace(pdssm_workspace_bytes(shape), d.device, ws)
+    code = lib().ssm_pdssm_fwd(ctypes.byref(shape), _p(scores), _p(dictionary), _p(d), _p(bt),
+                               _p(h0), _p(h), _p(sel), _p(ws), ws.numel() * ws.element_size(),
+                               _stream(stream))
+    _check(code, "ssm_pdssm_fwd")
+    return h, sel
+
+
+def ssm_pdssm_bwd(scores, dictionary, d, h, sel, g, tau=1.0, h0=None, out=None, ws=None,
+                  stream=None):
+    """Flash PD-SSM backward of sum <g, h> (straight-through score gradient at temperature tau).
+    Returns dict dd, dbt [B,L,H,N], dscores [B,L,H,K], dh0 [B,H,N]."""
+    _need_cuda(scores, dictionary, d, h, sel, g, h0)
+    B, L, H, K = scores.shape
+    N = d.shape[-1]
+    shape = pdssm_shape(B, L, H, N, K)
+    if out is None:
+        out = dict(dd=torch.empty_like(d), dbt=torch.empty_like(d),
+                   dscores=torch.empty_like(scores),
+                   dh0=torch.empty((B, H, N), dtype=torch.float32, device=d.device))
+    ws = _workspace(pdssm_workspace_bytes(shape), d.device, ws)
+    code = lib().ssm_pdssm_bwd(ctypes.byref(shape), float(tau), _p(scores), _p(dictionary), _p(d),
+                               _p(h0), _p(h), _p(sel), _p(g), _p(out["dd"]), _p(out["dbt"]),
+                               _p(out["dscores"]), _p(out.get("dh0")), _p(ws),
+                               ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_pdssm_bwd")
     return out

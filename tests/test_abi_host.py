@@ -171,6 +171,29 @@ def test_rtrl_validation(S):
     assert L.ssm_scan_complex_rtrl(ctypes.byref(odd), *p, need, None) == 3
 
 
+def test_pdssm_validation(S):
+    L = S.lib()
+    shp = S.pdssm_shape(2, 64, 8, 16, 8)
+    assert S.pdssm_workspace_bytes(shp) == 256
+    assert S.pdssm_workspace_bytes(S.pdssm_shape(2, 64, 8, 12, 8)) == 0      # N not in {4,8,16,32}
+    assert S.pdssm_workspace_bytes(S.pdssm_shape(2, 64, 8, 16, 33)) == 0     # K > 32
+    p = _fake_ptrs(8)
+    assert L.ssm_pdssm_fwd(ctypes.byref(shp), *p, 255, None) == 4
+    bad = S.pdssm_shape(2, 64, 8, 16, 0)
+    assert L.ssm_pdssm_fwd(ctypes.byref(bad), *p, 256, None) == 2
+    q = list(p)
+    q[5] = None  # h
+    assert L.ssm_pdssm_fwd(ctypes.byref(shp), *q, 256, None) == 1
+    pb = _fake_ptrs(12)
+    assert L.ssm_pdssm_bwd(ctypes.byref(shp), ctypes.c_float(0.0), *pb, 256, None) == 1   # tau
+    qb = list(pb)
+    qb[6] = None  # g
+    assert L.ssm_pdssm_bwd(ctypes.byref(shp), ctypes.c_float(1.0), *qb, 256, None) == 1
+    qb = list(pb)
+    qb[10] = ctypes.c_void_p(0x100004)  # dh0 misaligned
+    assert L.ssm_pdssm_bwd(ctypes.byref(shp), ctypes.c_float(1.0), *qb, 256, None) == 3
+
+
 def test_complex_validation(S):
     L = S.lib()
     shp = S.complex_shape(2, 64, 16, 32)
