@@ -539,7 +539,8 @@ def main_pdssm(args, w):
     sel = torch.empty((w.batch, w.seqlen, w.heads), dtype=torch.int32, device=dev)
     out = dict(dd=torch.empty_like(d["d"]), dbt=torch.empty_like(d["d"]),
                dscores=torch.empty_like(d["scores"]), dh0=torch.empty_like(d["h0"]))
-    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    shape = S.pdssm_shape(w.batch, w.seqlen, w.heads, w.nstate, w.ndict)
+    ws = torch.empty(S.pdssm_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -629,7 +630,7 @@ def main_pdssm(args, w):
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (8 if S.pdssm_workspace_bytes(shape) > 256 else 4) * args.steps,
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:

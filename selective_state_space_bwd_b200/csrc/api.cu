@@ -447,16 +447,61 @@ int check_pdshape(const ssm_pdshape* s) {
     return SSM_OK;
 }
 
+// Time segments of the PD-SSM scans: when the (batch, head-group) CTAs cannot fill the GPU, the
+// sequence is cut into segments of a multiple of 16 steps (at least 64) so that about four CTAs
+// per SM run; the workspace holds their summaries and carries.
+struct PdPlan {
+    int nseg, seg_len;
+    size_t f_pi, f_w, f_s, hin, b_rho, b_v, b_w, win, end;
+};
+
+PdPlan plan_pd(const ssm_pdshape* s) {
+    PdPlan p = {};
+    const int64_t B = s->batch, L = s->seqlen, H = s->heads, N = s->nstate;
+    const int64_t seq = ssm::kPdThreads / N, ctas = B * ((H + seq - 1) / seq);
+    int64_t nseg = 1;
+    if (ctas > 0 && ctas < kTargetCtas && L >= 128) {
+        nseg = (2 * kTargetCtas + ctas - 1) / ctas;
+        nseg = nseg < L / 64 ? nseg : L / 64;
+        if (nseg < 1) nseg = 1;
+    }
+    int64_t seg_len = (L + nseg - 1) / nseg;
+    seg_len = (seg_len + 15) / 16 * 16;
+    if (seg_len < 16) seg_len = 16;
+    nseg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
+    p.nseg = (int)nseg;
+    p.seg_len = (int)seg_len;
+    const size_t BHN = (size_t)B * H * N, S = (size_t)nseg;
+    const size_t summ = S > 1 ? BHN * (S - 1) * 4 : 0, carry = S > 1 ? BHN * S * 4 : 0;
+    size_t o = kStatusBytes;
+    p.f_pi = o;  o = align256(o + summ);
+    p.f_w = o;   o = align256(o + summ);
+    p.f_s = o;   o = align256(o + summ);
+    p.hin = o;   o = align256(o + carry);
+    p.b_rho = o; o = align256(o + summ);
+    p.b_v = o;   o = align256(o + summ);
+    p.b_w = o;   o = align256(o + summ);
+    p.win = o;   o = align256(o + carry);
+    p.end = o;
+    return p;
+}
+
 ssm::PdArgs pd_args(const ssm_pdshape* s, void* ws) {
     ssm::PdArgs a = {};
     a.B = (int)s->batch; a.L = (int)s->seqlen; a.H = (int)s->heads; a.N = s->nstate; a.K = s->ndict;
     a.status = at<unsigned>(ws, 0);
+    const PdPlan p = plan_pd(s);
+    a.nseg = p.nseg; a.seg_len = p.seg_len;
+    a.f_pi = at<int32_t>(ws, p.f_pi); a.f_w = at<float>(ws, p.f_w); a.f_s = at<float>(ws, p.f_s);
+    a.hin = at<float>(ws, p.hin);
+    a.b_rho = at<int32_t>(ws, p.b_rho); a.b_v = at<float>(ws, p.b_v); a.b_w = at<float>(ws, p.b_w);
+    a.win = at<float>(ws, p.win);
     return a;
 }
 }  // namespace
 
 size_t ssm_pdssm_workspace_bytes(const ssm_pdshape* shape) {
-    return check_pdshape(shape) == SSM_OK ? kStatusBytes : 0;
+    return check_pdshape(shape) == SSM_OK ? plan_pd(shape).end : 0;
 }
 
 int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* dict,
@@ -469,7 +514,7 @@ int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* 
     const void* ptrs[] = {scores, dict, d, bt, h, sel, ws, h0};
     const size_t counts[] = {BLH * K, K * N, BLH * N, BLH * N, BLH * N, BLH, 1, h0 ? BH * N : 0};
     if ((st = check_arrays(ptrs, counts, 8)) != SSM_OK) return st;
-    if (ws_bytes < kStatusBytes) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < plan_pd(shape).end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
     if (BLH == 0) return SSM_OK;
@@ -491,7 +536,7 @@ int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, cons
     const size_t counts[] = {BLH * K, K * N, BLH * N, BLH * N, BLH, BLH * N, BLH * N, BLH * N,
                              BLH * K, 1, h0 ? BH * N : 0, dh0 ? BH * N : 0};
     if ((st = check_arrays(ptrs, counts, 12)) != SSM_OK) return st;
-    if (ws_bytes < kStatusBytes) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < plan_pd(shape).end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
     if (BLH == 0) {  // no steps: dL/dh0 = 0

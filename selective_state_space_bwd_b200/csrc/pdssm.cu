@@ -123,12 +123,20 @@ __global__ void __launch_bounds__(NT) pdssm_fwd_kernel(PdArgs p) {
     const bool ev = e < p.H;
     const size_t total = (size_t)p.B * p.L * p.H;  // (b, t, e) rows
     build_lists<N>(p.dict, p.K, s_start, s_src, tid, p.status);
-    float h = (p.h0 && ev) ? p.h0[((size_t)b * p.H + e) * N + j] : 0.0f;
-    const int ntiles = (p.L + TT - 1) / TT;
+    const int seg = blockIdx.z;
+    const int t_begin = seg * p.seg_len, t_end = min(p.L, t_begin + p.seg_len);
+    float h = 0.0f;
+    if (ev) {
+        if (p.nseg > 1)
+            h = p.hin[(((size_t)b * p.H + e) * p.nseg + seg) * N + j];
+        else if (p.h0)
+            h = p.h0[((size_t)b * p.H + e) * N + j];
+    }
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     auto row0 = [&](int t) { return ((size_t)b * p.L + t) * p.H + e0; };  // first (b,t,e) row
     const size_t rstride = (size_t)p.H * N;
     auto issue = [&](int jt, int st) {
-        const size_t o = row0(jt * TT);
+        const size_t o = row0(t_begin + jt * TT);
         tile_rows<TT>(sd[st], p.d, o * N, rstride, total * N, tid);
         tile_rows<TT>(sb[st], p.bt, o * N, rstride, total * N, tid);
         tile_sel<TT, SEQ>(ssel[st], p.sel, o, p.H, total, tid);
@@ -145,7 +153,7 @@ __global__ void __launch_bounds__(NT) pdssm_fwd_kernel(PdArgs p) {
             cp_async_wait<0>();
         }
         __syncthreads();
-        const int t0 = jt * TT, rows = min(TT, p.L - t0);
+        const int t0 = t_begin + jt * TT, rows = min(TT, t_end - t0);
         float* hout = p.h + (row0(t0) + sq) * N + j;
         for (int r = 0; r < rows; ++r) {
             const int k = min(max(ssel[st][r * SEQ + sq], 0), p.K - 1);
@@ -177,11 +185,13 @@ __global__ void __launch_bounds__(NT) pdssm_bwd_kernel(PdArgs p) {
     const bool ev = e < p.H;
     const size_t total = (size_t)p.B * p.L * p.H;
     for (int i = tid; i < p.K * N; i += NT) s_dict[i] = (unsigned char)dict_row<N>(p.dict, i, p.status);
-    const int ntiles = (p.L + TT - 1) / TT;
+    const int seg = blockIdx.z;
+    const int t_begin = seg * p.seg_len, t_end = min(p.L, t_begin + p.seg_len);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     auto row0 = [&](int t) { return ((size_t)b * p.L + t) * p.H + e0; };
     const size_t rstride = (size_t)p.H * N;
     auto issue = [&](int jt, int st) {
-        const int t0 = jt * TT;
+        const int t0 = t_begin + jt * TT;
         const size_t o = row0(t0);
         tile_rows<TT>(sg[st], p.g, o * N, rstride, total * N, tid);
         tile_rows<TT>(sd[st], p.d, o * N, rstride, total * N, tid);
@@ -200,7 +210,8 @@ __global__ void __launch_bounds__(NT) pdssm_bwd_kernel(PdArgs p) {
         cp_async_commit();
     };
     __syncthreads();  // dictionary
-    float w = 0.0f;   // A_{t+1}^T mu_{t+1}
+    float w = 0.0f;   // A_{t+1}^T mu_{t+1}: from the carry (or later segment), zero at the end
+    if (ev && seg < p.nseg - 1) w = p.win[(((size_t)b * p.H + e) * p.nseg + seg) * N + j];
     if (ntiles > 0) issue(ntiles - 1, (ntiles - 1) & 1);
     for (int jt = ntiles - 1; jt >= 0; --jt) {
         const int st = jt & 1;
@@ -211,7 +222,7 @@ __global__ void __launch_bounds__(NT) pdssm_bwd_kernel(PdArgs p) {
             cp_async_wait<0>();
         }
         __syncthreads();
-        const int t0 = jt * TT, rows = min(TT, p.L - t0);
+        const int t0 = t_begin + jt * TT, rows = min(TT, t_end - t0);
         const size_t base = (row0(t0) + sq) * N + j;
         for (int r = rows - 1; r >= 0; --r) {
             const int k = min(max(ssel[st][r * SEQ + sq], 0), p.K - 1);
@@ -230,8 +241,184 @@ __global__ void __launch_bounds__(NT) pdssm_bwd_kernel(PdArgs p) {
         __syncthreads();  // stage st is free again
     }
     if (ev) {
-        if (p.dh0) p.dh0[((size_t)b * p.H + e) * N + j] = w;
+        if (p.dh0 && seg == 0) p.dh0[((size_t)b * p.H + e) * N + j] = w;
         if (!isfinite(w)) flag_status(p.status, kStatusNonFinite);
+    }
+}
+
+// Phase A of the forward (segments 0..nseg-2): the scan of the segment from zero, and the
+// composition of its transitions.  A product of one-hot-column-times-diagonal matrices is again
+// one: column j of the composed map has weight f_w[j] in row f_pi[j], and one more step k gives
+// f_pi <- dict[k][f_pi], f_w <- f_w * d_t[f_pi].
+template <int N>
+__global__ void __launch_bounds__(NT) pdssm_fwd_summary_kernel(PdArgs p) {
+    constexpr int SEQ = NT / N, TT = 16;
+    __shared__ __align__(16) float sd[2][TT * NT];
+    __shared__ __align__(16) float sb[2][TT * NT];
+    __shared__ __align__(16) int ssel[2][TT * SEQ];
+    __shared__ float sv[NT];
+    __shared__ unsigned char s_start[KMAX * (N + 1)];
+    __shared__ unsigned char s_src[KMAX * N];
+    __shared__ unsigned char s_dict[KMAX * N];
+    const int tid = threadIdx.x, j = tid % N, sq = tid / N;
+    const int b = blockIdx.y, e0 = blockIdx.x * SEQ, e = e0 + sq, seg = blockIdx.z;
+    const bool ev = e < p.H;
+    const size_t total = (size_t)p.B * p.L * p.H;
+    build_lists<N>(p.dict, p.K, s_start, s_src, tid, p.status);
+    for (int i = tid; i < p.K * N; i += NT) s_dict[i] = (unsigned char)dict_row<N>(p.dict, i, p.status);
+    const int t_begin = seg * p.seg_len, t_end = min(p.L, t_begin + p.seg_len);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
+    auto row0 = [&](int t) { return ((size_t)b * p.L + t) * p.H + e0; };
+    const size_t rstride = (size_t)p.H * N;
+    auto issue = [&](int jt, int st) {
+        const size_t o = row0(t_begin + jt * TT);
+        tile_rows<TT>(sd[st], p.d, o * N, rstride, total * N, tid);
+        tile_rows<TT>(sb[st], p.bt, o * N, rstride, total * N, tid);
+        tile_sel<TT, SEQ>(ssel[st], p.sel, o, p.H, total, tid);
+        cp_async_commit();
+    };
+    __syncthreads();
+    float h = 0.0f, w = 1.0f;
+    int pi = j;
+    if (ntiles > 0) issue(0, 0);
+    for (int jt = 0; jt < ntiles; ++jt) {
+        const int st = jt & 1;
+        if (jt + 1 < ntiles) {
+            issue(jt + 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int rows = min(TT, t_end - (t_begin + jt * TT));
+        for (int r = 0; r < rows; ++r) {
+            const int k = min(max(ssel[st][r * SEQ + sq], 0), p.K - 1);
+            sv[tid] = sd[st][r * NT + tid] * h;
+            __syncwarp();
+            float acc = sb[st][r * NT + tid];
+            const int q1 = s_start[k * (N + 1) + j + 1];
+            for (int q = s_start[k * (N + 1) + j]; q < q1; ++q) acc += sv[sq * N + s_src[k * N + q]];
+            h = acc;
+            w *= sd[st][r * NT + sq * N + pi];
+            pi = s_dict[k * N + pi];
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+    if (ev) {
+        const size_t o = (((size_t)b * p.H + e) * (p.nseg - 1) + seg) * N + j;
+        p.f_pi[o] = pi;
+        p.f_w[o] = w;
+        p.f_s[o] = h;
+    }
+}
+
+// Phase B of the forward: h_in[0] = h0 (or zero), h_in[s+1] = M_s h_in[s] + S_s, one N-lane group
+// per (batch, head); the scatter of M_s is a fixed-order loop over the group's lanes.
+template <int N>
+__global__ void __launch_bounds__(NT) pdssm_carry_fwd_kernel(PdArgs p) {
+    const int tid = threadIdx.x, j = tid % N;
+    const int64_t be = ((int64_t)blockIdx.x * NT + tid) / N;  // (b, e) row
+    const bool ok = be < (int64_t)p.B * p.H;
+    const int lane = tid & 31, base = lane & ~(N - 1);
+    float h = (ok && p.h0) ? p.h0[be * N + j] : 0.0f;
+    for (int s = 0; s < p.nseg; ++s) {
+        if (ok) p.hin[(be * p.nseg + s) * N + j] = h;
+        if (s == p.nseg - 1) break;
+        const size_t o = ((size_t)be * (p.nseg - 1) + s) * N + j;
+        const int pi = ok ? p.f_pi[o] : 0;
+        const float x = ok ? p.f_w[o] * h : 0.0f;
+        float acc = ok ? p.f_s[o] : 0.0f;
+        for (int jj = 0; jj < N; ++jj) {
+            const int pj = __shfl_sync(0xffffffffu, pi, base + jj);
+            const float xj = __shfl_sync(0xffffffffu, x, base + jj);
+            if (pj == j) acc += xj;
+        }
+        h = acc;
+    }
+}
+
+// Phase A of the backward (segments 1..nseg-1): the adjoint sweep of the segment from zero, and
+// the composition of its transposed transitions, a gather map: (G x)_j = b_v[j] x[b_rho[j]];
+// one more step t (going backwards) gives b_rho <- b_rho[dict[k][j]], b_v <- d_t[j] b_v[dict[k][j]].
+template <int N>
+__global__ void __launch_bounds__(NT) pdssm_bwd_summary_kernel(PdArgs p) {
+    constexpr int SEQ = NT / N, TT = 8;
+    __shared__ __align__(16) float sg[2][TT * NT];
+    __shared__ __align__(16) float sd[2][TT * NT];
+    __shared__ __align__(16) int ssel[2][TT * SEQ];
+    __shared__ float sv[NT];
+    __shared__ unsigned char s_dict[KMAX * N];
+    const int tid = threadIdx.x, j = tid % N, sq = tid / N;
+    const int b = blockIdx.y, e0 = blockIdx.x * SEQ, e = e0 + sq, seg = blockIdx.z + 1;
+    const bool ev = e < p.H;
+    const int lane = tid & 31, gbase = lane & ~(N - 1);
+    const size_t total = (size_t)p.B * p.L * p.H;
+    for (int i = tid; i < p.K * N; i += NT) s_dict[i] = (unsigned char)dict_row<N>(p.dict, i, p.status);
+    const int t_begin = seg * p.seg_len, t_end = min(p.L, t_begin + p.seg_len);
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
+    auto row0 = [&](int t) { return ((size_t)b * p.L + t) * p.H + e0; };
+    const size_t rstride = (size_t)p.H * N;
+    auto issue = [&](int jt, int st) {
+        const size_t o = row0(t_begin + jt * TT);
+        tile_rows<TT>(sg[st], p.g, o * N, rstride, total * N, tid);
+        tile_rows<TT>(sd[st], p.d, o * N, rstride, total * N, tid);
+        tile_sel<TT, SEQ>(ssel[st], p.sel, o, p.H, total, tid);
+        cp_async_commit();
+    };
+    __syncthreads();
+    float w = 0.0f, v = 1.0f;
+    int rho = j;
+    if (ntiles > 0) issue(ntiles - 1, (ntiles - 1) & 1);
+    for (int jt = ntiles - 1; jt >= 0; --jt) {
+        const int st = jt & 1;
+        if (jt > 0) {
+            issue(jt - 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int rows = min(TT, t_end - (t_begin + jt * TT));
+        for (int r = rows - 1; r >= 0; --r) {
+            const int k = min(max(ssel[st][r * SEQ + sq], 0), p.K - 1);
+            const float dj = sd[st][r * NT + tid];
+            const float mu = sg[st][r * NT + tid] + w;
+            sv[tid] = mu;
+            __syncwarp();
+            const int src = s_dict[k * N + j];
+            w = dj * sv[sq * N + src];
+            const int rho_n = __shfl_sync(0xffffffffu, rho, gbase + src);
+            const float v_n = __shfl_sync(0xffffffffu, v, gbase + src);
+            rho = rho_n;
+            v = dj * v_n;
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+    if (ev) {
+        const size_t o = (((size_t)b * p.H + e) * (p.nseg - 1) + (seg - 1)) * N + j;
+        p.b_rho[o] = rho;
+        p.b_v[o] = v;
+        p.b_w[o] = w;
+    }
+}
+
+// Phase B of the backward: w_in[nseg-1] = 0, w_in[s-1] = W_s + G_s w_in[s] (a gather).
+template <int N>
+__global__ void __launch_bounds__(NT) pdssm_carry_bwd_kernel(PdArgs p) {
+    const int tid = threadIdx.x, j = tid % N;
+    const int64_t be = ((int64_t)blockIdx.x * NT + tid) / N;
+    const bool ok = be < (int64_t)p.B * p.H;
+    const int lane = tid & 31, base = lane & ~(N - 1);
+    float w = 0.0f;
+    for (int s = p.nseg - 1; s >= 0; --s) {
+        if (ok) p.win[(be * p.nseg + s) * N + j] = w;
+        if (s == 0) break;
+        const size_t o = ((size_t)be * (p.nseg - 1) + (s - 1)) * N + j;
+        const int rho = ok ? p.b_rho[o] : j;
+        const float g = __shfl_sync(0xffffffffu, w, base + rho);
+        w = ok ? fmaf(p.b_v[o], g, p.b_w[o]) : 0.0f;
     }
 }
 
@@ -296,15 +483,32 @@ cudaError_t fwd_impl(const PdArgs& a, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int seq = NT / N;
-    pdssm_fwd_kernel<N><<<dim3((a.H + seq - 1) / seq, a.B), NT, 0, st>>>(a);
+    const unsigned gx = (unsigned)((a.H + seq - 1) / seq);
+    if (a.nseg > 1) {
+        pdssm_fwd_summary_kernel<N><<<dim3(gx, a.B, a.nseg - 1), NT, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t groups = (int64_t)a.B * a.H * N;
+        pdssm_carry_fwd_kernel<N><<<(unsigned)((groups + NT - 1) / NT), NT, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    pdssm_fwd_kernel<N><<<dim3(gx, a.B, a.nseg), NT, 0, st>>>(a);
     return cudaGetLastError();
 }
 
 template <int N>
 cudaError_t bwd_impl(const PdArgs& a, cudaStream_t st) {
     const int seq = NT / N;
-    pdssm_bwd_kernel<N><<<dim3((a.H + seq - 1) / seq, a.B), NT, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    const unsigned gx = (unsigned)((a.H + seq - 1) / seq);
+    cudaError_t e;
+    if (a.nseg > 1) {
+        pdssm_bwd_summary_kernel<N><<<dim3(gx, a.B, a.nseg - 1), NT, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t groups = (int64_t)a.B * a.H * N;
+        pdssm_carry_bwd_kernel<N><<<(unsigned)((groups + NT - 1) / NT), NT, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    pdssm_bwd_kernel<N><<<dim3(gx, a.B, a.nseg), NT, 0, st>>>(a);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t n = (int64_t)a.B * a.L * a.H;
     pdssm_dscores_kernel<N><<<(unsigned)((n + NT - 1) / NT), NT, 0, st>>>(a);

@@ -113,6 +113,16 @@ struct PdArgs {
     float* dscores;
     float* dh0;
     unsigned* status;
+    // time segments (the three phases: local scans with composed maps, carry, rescan)
+    int nseg, seg_len;
+    int32_t* f_pi;  // forward summaries of segments 0..nseg-2 [B*H][nseg-1][N]: map of the
+    float* f_w;     //   composed transition (column j -> row f_pi, weight f_w) and local end state
+    float* f_s;
+    float* hin;     // state entering each segment [B*H][nseg][N]
+    int32_t* b_rho; // backward summaries of segments 1..nseg-1 [B*H][nseg-1][N]: composed
+    float* b_v;     //   transposed transitions (gather from b_rho, weight b_v) and local adjoint
+    float* b_w;
+    float* win;     // adjoint entering each segment from its end [B*H][nseg][N]
 };
 
 // Launchers (return cudaGetLastError() of the last launch).

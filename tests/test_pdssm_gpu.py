@@ -50,6 +50,9 @@ CASES = [  # B, L, H, N, K
     (3, 65, 17, 8, 1),
     (2, 130, 5, 32, 32),
     (1, 16, 32, 16, 5),
+    (1, 1000, 8, 16, 8),   # few CTAs: 13 time segments (summaries, carries, rescans)
+    (1, 300, 3, 4, 5),     # 4 segments, partial last segment
+    (2, 257, 20, 8, 6),    # 2 segments
 ]
 
 
