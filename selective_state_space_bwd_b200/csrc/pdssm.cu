@@ -109,20 +109,53 @@ __device__ __forceinline__ void build_lists(const int32_t* dict, int K, unsigned
     }
 }
 
+// Padded source table: every row gets the same number D of entries (the largest in-degree of the
+// dictionary), the missing ones pointing at slot N of its group, which holds zero.  With it every
+// lane of the scatter loops D times, so the lanes of a warp do not diverge.  Returns D, or 0 when
+// the table would not fit in PAD_BYTES (then the lists are used as they are).
+constexpr int PAD_BYTES = 4096;
+
+template <int N>
+__device__ __forceinline__ int build_pad(const unsigned char* start, const unsigned char* src, int K,
+                                         unsigned char* pad, int* s_deg, int tid) {
+    if (tid == 0) *s_deg = 0;
+    __syncthreads();
+    for (int i = tid; i < K * N; i += NT) {
+        const int k = i / N, r = i - k * N;
+        atomicMax(s_deg, start[k * (N + 1) + r + 1] - start[k * (N + 1) + r]);
+    }
+    __syncthreads();
+    const int D = *s_deg;
+    if (D == 0 || K * N * D > PAD_BYTES) return 0;
+    for (int i = tid; i < K * N; i += NT) {
+        const int k = i / N, r = i - k * N;
+        const int a = start[k * (N + 1) + r], c = start[k * (N + 1) + r + 1] - a;
+        for (int m = 0; m < D; ++m) pad[i * D + m] = m < c ? src[k * N + a + m] : (unsigned char)N;
+    }
+    __syncthreads();
+    return D;
+}
+
 template <int N>
 __global__ void __launch_bounds__(NT) pdssm_fwd_kernel(PdArgs p) {
     constexpr int SEQ = NT / N, TT = 16;
     __shared__ __align__(16) float sd[2][TT * NT];
     __shared__ __align__(16) float sb[2][TT * NT];
     __shared__ __align__(16) int ssel[2][TT * SEQ];
-    __shared__ float sv[NT];
+    __shared__ float sv[SEQ * (N + 1)];  // per group: N values and a zero slot
     __shared__ unsigned char s_start[KMAX * (N + 1)];
     __shared__ unsigned char s_src[KMAX * N];
+    __shared__ unsigned char s_pad[PAD_BYTES];
+    __shared__ int s_deg;
     const int tid = threadIdx.x, j = tid % N, sq = tid / N;
     const int b = blockIdx.y, e0 = blockIdx.x * SEQ, e = e0 + sq;
     const bool ev = e < p.H;
     const size_t total = (size_t)p.B * p.L * p.H;  // (b, t, e) rows
     build_lists<N>(p.dict, p.K, s_start, s_src, tid, p.status);
+    if (j == 0) sv[sq * (N + 1) + N] = 0.0f;
+    __syncthreads();
+    const int D = build_pad<N>(s_start, s_src, p.K, s_pad, &s_deg, tid);
+    float* svg = sv + sq * (N + 1);
     const int seg = blockIdx.z;
     const int t_begin = seg * p.seg_len, t_end = min(p.L, t_begin + p.seg_len);
     float h = 0.0f;
@@ -155,15 +188,22 @@ __global__ void __launch_bounds__(NT) pdssm_fwd_kernel(PdArgs p) {
         __syncthreads();
         const int t0 = t_begin + jt * TT, rows = min(TT, t_end - t0);
         float* hout = p.h + (row0(t0) + sq) * N + j;
+        const size_t hstep = (size_t)p.H * N;
         for (int r = 0; r < rows; ++r) {
             const int k = min(max(ssel[st][r * SEQ + sq], 0), p.K - 1);
-            sv[tid] = sd[st][r * NT + tid] * h;
+            svg[j] = sd[st][r * NT + tid] * h;
             __syncwarp();
             float acc = sb[st][r * NT + tid];
-            const int q1 = s_start[k * (N + 1) + j + 1];
-            for (int q = s_start[k * (N + 1) + j]; q < q1; ++q) acc += sv[sq * N + s_src[k * N + q]];
+            if (D > 0) {  // uniform trip count: no divergence
+                const unsigned char* row = s_pad + (k * N + j) * D;
+                for (int m = 0; m < D; ++m) acc += svg[row[m]];
+            } else {
+                const int q1 = s_start[k * (N + 1) + j + 1];
+                for (int q = s_start[k * (N + 1) + j]; q < q1; ++q) acc += svg[s_src[k * N + q]];
+            }
             h = acc;
-            if (ev) hout[(size_t)r * p.H * N] = h;
+            if (ev) *hout = h;
+            hout += hstep;
             __syncwarp();
         }
         __syncthreads();  // stage st is free again
