@@ -176,20 +176,25 @@ def oracle_sample(w, inp, budget_s=(10.0, 30.0), zoh=False):
                       f"fwd+bwd in float64, {t_total:.1f} s"}
 
 
-def measured_traffic(kernel_file, workload):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu capture summary,
-    if that capture was taken on the current kernel source; else None."""
+def measured_traffic(call, kernel_file, workload):
+    """DRAM bytes per launch of `call` (its kernels summed) on `workload`, from the committed ncu
+    capture records, if that capture was taken on the current source of `kernel_file`; else None.
+    A record captured on a smaller case of the same launch plan carries the factor that scales
+    it to the full workload's units."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        rec = json.load(open(p))
+        recs = json.load(open(p))["records"]
         src = open(os.path.join(ROOT, "selective_state_space_bwd_b200", "csrc", kernel_file), "rb").read()
-        if rec.get("workload") != workload or rec.get("source_sha256") != hashlib.sha256(src).hexdigest():
-            return None
-        return float(rec["dram_bytes_per_launch"])
-    except (OSError, ValueError, KeyError):
+        sha = hashlib.sha256(src).hexdigest()
+        for rec in recs:
+            if (rec["workload"] == workload and rec["call"] == call and rec["source"] == kernel_file
+                    and rec["source_sha256"] == sha):
+                return float(rec["dram_bytes_per_launch"])
+        return None
+    except (OSError, ValueError, KeyError, TypeError):
         return None
 
 
@@ -460,11 +465,15 @@ def main_complex(args, w):
             "roofline": ({"bound": "hbm", "kernel": "ssm_scan_complex_rtrl call (cplx_rtrl_kernel "
                           "+ reduction over the batch)", "achieved": fwd_gbs, "peak": hbm,
                           "unit": "GB/s", "frac": fwd_gbs / hbm, "peak_kind": peak_kind,
-                          "algorithmic_bytes_per_launch": fb, "traffic": None} if args.rtrl else
+                          "algorithmic_bytes_per_launch": fb,
+                          "traffic": measured_traffic("ssm_scan_complex_rtrl", "complex_scan.cu",
+                                                      w.name)} if args.rtrl else
                          {"bound": "hbm", "kernel": "ssm_scan_complex_bwd call (cplx_bwd_kernel + "
                           "reductions)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
-                          "algorithmic_bytes_per_launch": bb, "traffic": None}),
+                          "algorithmic_bytes_per_launch": bb,
+                          "traffic": measured_traffic("ssm_scan_complex_bwd", "complex_scan.cu",
+                                                      w.name)}),
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
@@ -625,7 +634,8 @@ def main_pdssm(args, w):
             "roofline": {"bound": "hbm", "kernel": "ssm_pdssm_bwd call (reverse scan + score "
                          "gradient)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": bb, "traffic": None},
+                         "algorithmic_bytes_per_launch": bb,
+                         "traffic": measured_traffic("ssm_pdssm_bwd", "pdssm.cu", w.name)},
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
@@ -896,7 +906,7 @@ def main():
                                       f"{alu_mhz:.0f} MHz (FMA = 1 op)",
                          "algorithmic_ops_per_launch": bo,
                          "algorithmic_bytes_per_launch": bb,
-                         "traffic": measured_traffic("real_bwd.cu", w.name)},
+                         "traffic": measured_traffic("ssm_scan_bwd", "real_bwd.cu", w.name)},
             "hbm": {"achieved_bwd": bwd_gbs, "achieved_fwd": fwd_gbs, "achieved_step": step_gbs,
                     "peak": hbm, "unit": "GB/s", "peak_kind": peak_kind},
             "hbm_frac_bwd": bwd_gbs / hbm,

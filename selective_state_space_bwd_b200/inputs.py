@@ -60,6 +60,8 @@ WORKLOADS = {
     "mamba1p4b_layer": RealWorkload("mamba1p4b_layer", 4, 8192, 4096, 16, 128, BF16, "mamba"),
     "sparc_complex": ComplexWorkload("sparc_complex", 16, 4096, 2048, 128),
     "sparc_complex_b4": ComplexWorkload("sparc_complex_b4", 4, 4096, 2048, 128),
+    # a quarter of sparc_complex along L with the same launch plan (profiling captures)
+    "sparc_complex_l1024": ComplexWorkload("sparc_complex_l1024", 16, 1024, 2048, 128),
     "pdssm_l5120": None,  # filled below (PdWorkload is defined after this table)
 }
 
@@ -184,3 +186,5 @@ class PdWorkload:
 
 
 WORKLOADS["pdssm_l5120"] = PdWorkload("pdssm_l5120", 8, 5120, 256, 16, 8)
+# a quarter of pdssm_l5120 along L with the same launch plan (profiling captures)
+WORKLOADS["pdssm_l1280"] = PdWorkload("pdssm_l1280", 8, 1280, 256, 16, 8)
