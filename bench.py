@@ -640,7 +640,7 @@ def main_pdssm(args, w):
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": (8 if S.pdssm_workspace_bytes(shape) > 256 else 4) * args.steps,
+            "gpu_launches": 2 * S.pdssm_kernel_launches(shape, False) * args.steps,
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:

@@ -274,7 +274,7 @@ int ssm_scan_complex_rtrl(const ssm_cshape* shape,
 typedef struct ssm_pdshape {
     int64_t batch;   /* B >= 0 */
     int64_t seqlen;  /* L >= 0 */
-    int64_t heads;   /* H >= 1 */
+    int64_t heads;   /* H >= 1, at most 2^21 */
     int32_t nstate;  /* N, one of 4, 8, 16, 32 */
     int32_t ndict;   /* K, 1..32 */
     int32_t reserved; /* must be 0 */
@@ -284,8 +284,8 @@ typedef struct ssm_pdshape {
 /* Workspace bytes of the PD-SSM calls (the status word: 256); 0 for an invalid shape. */
 size_t ssm_pdssm_workspace_bytes(const ssm_pdshape* shape);
 
-/* Forward: writes the trajectory h and the selection sel.  Enqueues 2 kernels (argmax, scan).
- * Returns an ssm_status. */
+/* Forward: writes the trajectory h and the selection sel (argmax of the scores, lowest index on
+ * ties).  Enqueues ssm_pdssm_kernel_launches(shape, 0) kernels.  Returns an ssm_status. */
 int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* dict,
                   const float* d, const float* bt, const float* h0, float* h, int32_t* sel,
                   void* ws, size_t ws_bytes, ssm_stream_t stream);
@@ -297,7 +297,7 @@ int ssm_pdssm_fwd(const ssm_pdshape* shape, const float* scores, const int32_t* 
  * and the discrete selection gets the straight-through surrogate with temperature tau > 0
  * (hard in the forward pass, softmax(scores / tau) in the backward pass):
  *     c_k = <mu_t, P_k D_t h_{t-1}>,   dscores_t[k] = p_k (c_k - sum_k' p_k' c_k') / tau.
- * Enqueues 2 kernels (reverse scan, score gradient).  Returns an ssm_status. */
+ * Enqueues ssm_pdssm_kernel_launches(shape, 1) kernels.  Returns an ssm_status. */
 int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, const int32_t* dict,
                   const float* d, const float* h0, const float* h, const int32_t* sel,
                   const float* g, float* dd, float* dbt, float* dscores, float* dh0,
@@ -309,6 +309,12 @@ int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);
 
 /* Same for the complex calls. */
 int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward);
+
+/* Same for the PD-SSM calls: 1 (one scan kernel, with the argmax fused into the forward and the
+ * score gradient into the backward), +2 when the sequence is cut into time segments (segment
+ * summaries and carry), +1 when ndict * (128 / nstate) > 256 (argmax or score gradient as a
+ * kernel of its own). */
+int ssm_pdssm_kernel_launches(const ssm_pdshape* shape, int backward);
 
 /* Waits for `stream`, then returns the status word the last call on `ws` left (SSM_OK,
  * SSM_ERR_NONFINITE or SSM_ERR_TIMEOUT), or SSM_ERR_CUDA if the copy itself fails. */

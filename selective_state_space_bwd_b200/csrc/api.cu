@@ -441,15 +441,18 @@ int check_pdshape(const ssm_pdshape* s) {
         return SSM_ERR_INVALID_ARG;
     if (s->nstate != 4 && s->nstate != 8 && s->nstate != 16 && s->nstate != 32) return SSM_ERR_UNSUPPORTED;
     if (s->ndict < 1 || s->ndict > 32) return SSM_ERR_UNSUPPORTED;
-    if (s->batch > 65535 || s->seqlen > (int64_t)1 << 30 || s->heads > (int64_t)1 << 24 ||
+    if (s->batch > 65535 || s->seqlen > (int64_t)1 << 30 || s->heads > (int64_t)1 << 21 ||
         (double)s->batch * s->seqlen * s->heads * s->nstate > 9.0e15)
         return SSM_ERR_UNSUPPORTED;
     return SSM_OK;
 }
 
-// Time segments of the PD-SSM scans: when the (batch, head-group) CTAs cannot fill the GPU, the
-// sequence is cut into segments of a multiple of 16 steps (at least 64) so that about four CTAs
-// per SM run; the workspace holds their summaries and carries.
+// Time segments of the PD-SSM scans: when the (batch, head-group) CTAs are fewer than kPdMinCtas
+// (each streams at most a few tens of GB/s, bounded by its per-step latency), the sequence is cut
+// into segments of a multiple of 16 steps (at least 64) so that about four CTAs per SM run; the
+// workspace holds their summaries and carries.
+constexpr int64_t kPdMinCtas = 128;
+
 struct PdPlan {
     int nseg, seg_len;
     size_t f_pi, f_w, f_s, hin, b_rho, b_v, b_w, win, end;
@@ -460,7 +463,7 @@ PdPlan plan_pd(const ssm_pdshape* s) {
     const int64_t B = s->batch, L = s->seqlen, H = s->heads, N = s->nstate;
     const int64_t seq = ssm::kPdThreads / N, ctas = B * ((H + seq - 1) / seq);
     int64_t nseg = 1;
-    if (ctas > 0 && ctas < kTargetCtas && L >= 128) {
+    if (ctas > 0 && ctas < kPdMinCtas && L >= 128) {
         nseg = (2 * kTargetCtas + ctas - 1) / ctas;
         nseg = nseg < L / 64 ? nseg : L / 64;
         if (nseg < 1) nseg = 1;
@@ -499,6 +502,13 @@ ssm::PdArgs pd_args(const ssm_pdshape* s, void* ws) {
     return a;
 }
 }  // namespace
+
+int ssm_pdssm_kernel_launches(const ssm_pdshape* shape, int backward) {
+    (void)backward;  // the forward and the backward launch the same number
+    if (check_pdshape(shape) != SSM_OK) return -1;
+    if (shape->batch == 0 || shape->seqlen == 0) return 0;
+    return ssm::pdssm_launches(pd_args(shape, nullptr));
+}
 
 size_t ssm_pdssm_workspace_bytes(const ssm_pdshape* shape) {
     return check_pdshape(shape) == SSM_OK ? plan_pd(shape).end : 0;

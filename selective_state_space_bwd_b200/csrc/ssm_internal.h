@@ -128,6 +128,7 @@ struct PdArgs {
 // Launchers (return cudaGetLastError() of the last launch).
 cudaError_t launch_pdssm_fwd(const PdArgs& a, cudaStream_t st);
 cudaError_t launch_pdssm_bwd(const PdArgs& a, cudaStream_t st);
+int pdssm_launches(const PdArgs& a);  // kernels per ssm_pdssm_fwd (and per ssm_pdssm_bwd) call
 cudaError_t launch_real_fwd(const RealArgs& a, int io_bf16, int N, cudaStream_t st);
 cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cudaStream_t st);
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st);

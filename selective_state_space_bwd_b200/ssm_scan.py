@@ -66,7 +66,8 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
             "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex",
             "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
-            "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd"]
+            "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd",
+            "ssm_pdssm_kernel_launches"]
 
 
 def lib():
@@ -111,6 +112,7 @@ def lib():
             L.ssm_pdssm_fwd.restype = I
             L.ssm_pdssm_bwd.argtypes = [PP, ctypes.c_float] + [P] * 12 + [Z, P]
             L.ssm_pdssm_bwd.restype = I
+            L.ssm_pdssm_kernel_launches.argtypes, L.ssm_pdssm_kernel_launches.restype = [PP, I], I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -379,6 +381,10 @@ def pdssm_shape(batch, seqlen, heads, nstate, ndict):
 
 def pdssm_workspace_bytes(shape: SsmPdShape) -> int:
     return int(lib().ssm_pdssm_workspace_bytes(ctypes.byref(shape)))
+
+
+def pdssm_kernel_launches(shape: SsmPdShape, backward: bool) -> int:
+    return int(lib().ssm_pdssm_kernel_launches(ctypes.byref(shape), int(bool(backward))))
 
 
 def ssm_pdssm_fwd(scores, dictionary, d, bt, h0=None, h=None, sel=None, ws=None, stream=None):

@@ -177,6 +177,8 @@ def test_pdssm_validation(S):
     assert S.pdssm_workspace_bytes(shp) == 256
     assert S.pdssm_workspace_bytes(S.pdssm_shape(2, 64, 8, 12, 8)) == 0      # N not in {4,8,16,32}
     assert S.pdssm_workspace_bytes(S.pdssm_shape(2, 64, 8, 16, 33)) == 0     # K > 32
+    assert S.pdssm_workspace_bytes(S.pdssm_shape(1, 64, (1 << 21) + 1, 4, 2)) == 0  # H > 2^21
+    assert S.pdssm_workspace_bytes(S.pdssm_shape(1, 64, 1 << 21, 4, 2)) == 256
     p = _fake_ptrs(8)
     assert L.ssm_pdssm_fwd(ctypes.byref(shp), *p, 255, None) == 4
     bad = S.pdssm_shape(2, 64, 8, 16, 0)
@@ -232,3 +234,14 @@ def test_kernel_launch_counts(S):
     assert S.kernel_launches(S.real_shape(2, 0, 32, 16, 128), True) == 0
     assert S.kernel_launches(S.real_shape(2, 8, 32, 12, 128), True) == -1
     assert S.complex_kernel_launches(S.complex_shape(16, 4096, 2048, 128), True) == 3
+    # PD-SSM: one scan kernel per call (argmax / score gradient fused) at the bench size; time
+    # segments below 128 CTAs add summary + carry; K * (128 / N) > 256 adds the separate kernel
+    pd = S.pdssm_shape(8, 5120, 256, 16, 8)
+    assert S.pdssm_kernel_launches(pd, False) == 1 and S.pdssm_kernel_launches(pd, True) == 1
+    assert S.pdssm_workspace_bytes(pd) == 256
+    few = S.pdssm_shape(1, 1000, 8, 16, 8)
+    assert S.pdssm_kernel_launches(few, False) == 3 and S.pdssm_kernel_launches(few, True) == 3
+    wide = S.pdssm_shape(2, 64, 8, 4, 9)
+    assert S.pdssm_kernel_launches(wide, False) == 2 and S.pdssm_kernel_launches(wide, True) == 2
+    assert S.pdssm_kernel_launches(S.pdssm_shape(2, 0, 8, 16, 8), False) == 0
+    assert S.pdssm_kernel_launches(S.pdssm_shape(2, 8, 8, 12, 8), False) == -1

@@ -53,6 +53,9 @@ CASES = [  # B, L, H, N, K
     (1, 1000, 8, 16, 8),   # few CTAs: 13 time segments (summaries, carries, rescans)
     (1, 300, 3, 4, 5),     # 4 segments, partial last segment
     (2, 257, 20, 8, 6),    # 2 segments
+    (2, 150, 9, 4, 9),     # K * heads-per-CTA > 256: argmax and score gradient as kernels of their own
+    (1, 200, 16, 8, 17),   # the same with N = 8
+    (3, 96, 64, 32, 32),   # largest state and dictionary
 ]
 
 
@@ -64,6 +67,21 @@ def test_pdssm_matches_oracle(S, oracle_mod, B, L, H, N, K, with_h0):
     got = run(S, c, tau, with_h0)
     ref = oracle_mod.pdssm(c["scores"], c["dictionary"], c["d"], c["bt"],
                            c["h0"] if with_h0 else None, c["g"], tau=tau)
+    np.testing.assert_array_equal(got["sel"], ref["sel"])
+    assert rel(got["h"], ref["h"]) <= FWD_TOL
+    for k in ("dd", "dbt", "dscores", "dh0"):
+        assert rel(got[k], ref[k]) <= GRAD_TOL, (k, rel(got[k], ref[k]))
+
+
+@pytest.mark.parametrize("N,K,B,L,H", [(16, 5, 2, 90, 11), (32, 3, 1, 70, 6), (8, 4, 2, 300, 40)])
+def test_pdssm_high_in_degree(S, oracle_mod, N, K, B, L, H):
+    """Dictionaries whose rows collect more than seven columns (all columns into one row, half of
+    them into another) take the plain in-list gather instead of the packed words."""
+    c = gen.pdssm_inputs(B, L, H, N, K, seed=N + K)
+    c["dictionary"][0, :] = 0
+    c["dictionary"][1, : N // 2] = N - 1
+    got = run(S, c, 0.7)
+    ref = oracle_mod.pdssm(c["scores"], c["dictionary"], c["d"], c["bt"], c["h0"], c["g"], tau=0.7)
     np.testing.assert_array_equal(got["sel"], ref["sel"])
     assert rel(got["h"], ref["h"]) <= FWD_TOL
     for k in ("dd", "dbt", "dscores", "dh0"):
