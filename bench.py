@@ -101,6 +101,61 @@ def algorithmic_bytes(w):
     return fwd, bwd                              # Bm, Cm in; dB, dC out; ckpt in
 
 
+def e2e_pipelined(torch, dev, stream, host, sets, compute, outputs, steps, world, dist):
+    """Seconds (max over ranks) for `steps` end-to-end steps.  Every step copies its inputs from
+    pinned host memory (`host` into set["d"]) on one copy stream, computes on `stream`, and copies
+    `outputs(set)` back into pinned host buffers on another; the steps alternate between the two
+    device buffer sets, so one step's copies run beside the next step's compute while every step
+    still moves all its bytes.  Returns (seconds, h2d bytes per step, d2h bytes per step)."""
+    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outputs(sets[0]).items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in hout.values())
+    s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def run(nsteps, start_event=None):
+        if start_event is not None:
+            s_h2d.wait_event(start_event)
+        for k in range(nsteps):
+            i = k % 2
+            bs = sets[i]
+            with torch.cuda.stream(s_h2d):
+                s_h2d.wait_event(ev_done[i])  # set i's inputs are free once its last compute ended
+                for key, v in host.items():
+                    bs["d"][key].copy_(v, non_blocking=True)
+                ev_in[i].record(s_h2d)
+            stream.wait_event(ev_in[i])
+            stream.wait_event(ev_out[i])  # set i's outputs were copied back
+            compute(bs)
+            ev_done[i].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_done[i])
+                for key, v in outputs(bs).items():
+                    hout[key].copy_(v, non_blocking=True)
+                ev_out[i].record(s_d2h)
+        stream.wait_event(ev_out[(nsteps - 1) % 2])
+
+    run(2)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    run(steps, start_event=e0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t), h2d, d2h
+
+
+E2E_OVERLAP = ("two buffer sets; each step's host-to-device and device-to-host copies run on their "
+               "own streams beside the next step's compute")
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
 
@@ -357,27 +412,34 @@ def main_complex(args, w):
         out = dict(dlambda=out["dlambda"], domega=out["domega"])
         wsr = torch.empty(S.complex_rtrl_workspace_bytes(shape), dtype=torch.uint8, device=dev)
 
-    def fwd():
-        if args.rtrl:  # the whole RTRL pass: trajectory sensitivities and online gradient
-            S.ssm_scan_complex_rtrl(d["u"], d["r"], d["phi"], d["lam"], d["omega"], d["g"],
-                                    chunk=w.chunk, out=out, ws=wsr, stream=stream)
-        else:
-            S.ssm_scan_complex_fwd(d["u"], d["r"], d["phi"], d["lam"], d["omega"], chunk=w.chunk,
-                                   seg_chunks=args.seg_chunks, h=h, ws=wsf, stream=stream)
+    sets = [dict(d=d, h=h, out=out)]
 
-    def bwd():
+    def fwd(bs=None):
+        bs = bs or sets[0]
+        dd, hh, oo = bs["d"], bs["h"], bs["out"]
+        if args.rtrl:  # the whole RTRL pass: trajectory sensitivities and online gradient
+            S.ssm_scan_complex_rtrl(dd["u"], dd["r"], dd["phi"], dd["lam"], dd["omega"], dd["g"],
+                                    chunk=w.chunk, out=oo, ws=wsr, stream=stream)
+        else:
+            S.ssm_scan_complex_fwd(dd["u"], dd["r"], dd["phi"], dd["lam"], dd["omega"], chunk=w.chunk,
+                                   seg_chunks=args.seg_chunks, h=hh, ws=wsf, stream=stream)
+
+    def bwd(bs=None):
+        bs = bs or sets[0]
+        dd, hh, oo = bs["d"], bs["h"], bs["out"]
         if not args.rtrl:
-            S.ssm_scan_complex_bwd(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"],
-                                   chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
+            S.ssm_scan_complex_bwd(hh, dd["r"], dd["phi"], dd["lam"], dd["omega"], dd["g"],
+                                   chunk=w.chunk, seg_chunks=args.seg_chunks, out=oo, ws=wsb,
                                    stream=stream)
 
-    def allreduce():
+    def allreduce(bs=None):
+        oo = (bs or sets[0])["out"]
         if world > 1:  # dlambda, domega sum over the batch rows of every rank
-            gbuf[:w.modes].copy_(out["dlambda"])
-            gbuf[w.modes:].copy_(out["domega"])
+            gbuf[:w.modes].copy_(oo["dlambda"])
+            gbuf[w.modes:].copy_(oo["domega"])
             dist.all_reduce(gbuf)
-            out["dlambda"].copy_(gbuf[:w.modes])
-            out["domega"].copy_(gbuf[w.modes:])
+            oo["dlambda"].copy_(gbuf[:w.modes])
+            oo["domega"].copy_(gbuf[w.modes:])
 
     for _ in range(max(3, args.warmup)):
         fwd(); bwd(); allreduce()
@@ -405,39 +467,17 @@ def main_complex(args, w):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     t_step, t_fwd, t_bwd = tt.tolist()
 
-    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
-    hh = torch.empty(h.shape, dtype=h.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = hh.numel() * hh.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+    sets.append(dict(d={k: torch.empty_like(v) for k, v in d.items()}, h=torch.empty_like(h),
+                     out={k: torch.empty_like(v) for k, v in out.items()}))
 
-    if args.rtrl:  # the RTRL pass returns only dlambda, domega
-        d2h = sum(v.numel() * v.element_size() for v in hout.values())
-        h2d = sum(v.numel() * v.element_size() for k, v in host.items())
+    def compute(bs):
+        fwd(bs); bwd(bs); allreduce(bs)
 
-    def e2e_step():
-        for k, v in host.items():
-            d[k].copy_(v, non_blocking=True)
-        fwd(); bwd(); allreduce()
-        if not args.rtrl:
-            hh.copy_(h, non_blocking=True)
-        for k, v in out.items():
-            hout[k].copy_(v, non_blocking=True)
+    def outputs(bs):  # the RTRL pass returns only dlambda, domega
+        return dict(bs["out"]) if args.rtrl else dict(h=bs["h"], **bs["out"])
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-    t_e2e = float(t_e2e)
+    t_e2e, h2d, d2h = e2e_pipelined(torch, dev, stream, host, sets, compute, outputs, args.steps,
+                                    world, dist)
 
     upd_rank = w.batch * w.seqlen * w.modes
     value = world * upd_rank * args.steps / t_step
@@ -477,7 +517,7 @@ def main_complex(args, w):
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": E2E_OVERLAP},
             "gpu_launches": launches,
             "clocks": clk,
         }
@@ -553,13 +593,19 @@ def main_pdssm(args, w):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def fwd():
-        S.ssm_pdssm_fwd(d["scores"], d["dictionary"], d["d"], d["bt"], h0=d["h0"], h=h, sel=sel,
-                        ws=ws, stream=stream)
+    sets = [dict(d=d, h=h, sel=sel, out=out)]
 
-    def bwd():
-        S.ssm_pdssm_bwd(d["scores"], d["dictionary"], d["d"], h, sel, d["g"], tau=1.0, h0=d["h0"],
-                        out=out, ws=ws, stream=stream)
+    def fwd(bs=None):
+        bs = bs or sets[0]
+        dd = bs["d"]
+        S.ssm_pdssm_fwd(dd["scores"], dd["dictionary"], dd["d"], dd["bt"], h0=dd["h0"], h=bs["h"],
+                        sel=bs["sel"], ws=ws, stream=stream)
+
+    def bwd(bs=None):
+        bs = bs or sets[0]
+        dd = bs["d"]
+        S.ssm_pdssm_bwd(dd["scores"], dd["dictionary"], dd["d"], bs["h"], bs["sel"], dd["g"], tau=1.0,
+                        h0=dd["h0"], out=bs["out"], ws=ws, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         fwd(); bwd()
@@ -585,34 +631,14 @@ def main_pdssm(args, w):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     t_step, t_fwd, t_bwd = tt.tolist()
 
-    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
-    hh = torch.empty(h.shape, dtype=h.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = hh.numel() * hh.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+    sets.append(dict(d={k: torch.empty_like(v) for k, v in d.items()}, h=torch.empty_like(h),
+                     sel=torch.empty_like(sel), out={k: torch.empty_like(v) for k, v in out.items()}))
 
-    def e2e_step():
-        for k, v in host.items():
-            d[k].copy_(v, non_blocking=True)
-        fwd(); bwd()
-        hh.copy_(h, non_blocking=True)
-        for k, v in out.items():
-            hout[k].copy_(v, non_blocking=True)
+    def compute(bs):
+        fwd(bs); bwd(bs)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-    t_e2e = float(t_e2e)
+    t_e2e, h2d, d2h = e2e_pipelined(torch, dev, stream, host, sets, compute,
+                                    lambda bs: dict(h=bs["h"], **bs["out"]), args.steps, world, dist)
 
     upd_rank = w.batch * w.seqlen * w.heads * w.nstate
     value = world * upd_rank * args.steps / t_step
@@ -639,7 +665,7 @@ def main_pdssm(args, w):
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": E2E_OVERLAP},
             "gpu_launches": 2 * S.pdssm_kernel_launches(shape, False) * args.steps,
             "clocks": clk,
         }
@@ -797,19 +823,10 @@ def main():
     t_step, t_fwd, t_bwd = tt.tolist()
 
     # end to end: every step's inputs come from pinned host memory and every output goes back,
-    # inside the timed region.  Two buffer sets and two copy streams overlap the copies of one
-    # step with the compute of the next (each step still moves all its bytes).
-    hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
-    hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = hy.numel() * hy.element_size() + sum(v.numel() * v.element_size() for v in hout.values())
+    # inside the timed region (two buffer sets: one step's copies run beside the next's compute)
     sets = [dict(d=d, y=y, ckpt=ckpt, out=out)]
     sets.append(dict(d={k: torch.empty_like(v) for k, v in d.items()}, y=torch.empty_like(y),
                      ckpt=torch.empty_like(ckpt), out={k: torch.empty_like(v) for k, v in out.items()}))
-    s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def compute(bs):
         if use_ex:
@@ -833,42 +850,8 @@ def main():
         if world > 1:
             dp.allreduce_param_grads(bs["out"]["dA_log"], bs["out"]["dD"], buf=gbuf)
 
-    def e2e_run(nsteps, start_event=None):
-        if start_event is not None:
-            s_h2d.wait_event(start_event)
-        for k in range(nsteps):
-            i = k % 2
-            bs = sets[i]
-            with torch.cuda.stream(s_h2d):
-                s_h2d.wait_event(ev_done[i])  # set i's inputs are free once its last compute ended
-                for key, v in host.items():
-                    bs["d"][key].copy_(v, non_blocking=True)
-                ev_in[i].record(s_h2d)
-            stream.wait_event(ev_in[i])
-            stream.wait_event(ev_out[i])  # set i's outputs were copied back
-            compute(bs)
-            ev_done[i].record(stream)
-            with torch.cuda.stream(s_d2h):
-                s_d2h.wait_event(ev_done[i])
-                hy.copy_(bs["y"], non_blocking=True)
-                for key, v in bs["out"].items():
-                    hout[key].copy_(v, non_blocking=True)
-                ev_out[i].record(s_d2h)
-        stream.wait_event(ev_out[(nsteps - 1) % 2])
-
-    e2e_run(2)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    e2e_run(args.steps, start_event=e0)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-    t_e2e = float(t_e2e)
+    t_e2e, h2d, d2h = e2e_pipelined(torch, dev, stream, host, sets, compute,
+                                    lambda bs: dict(y=bs["y"], **bs["out"]), args.steps, world, dist)
 
     upd_rank = w.batch * w.seqlen * w.dim * w.dstate
     value = world * upd_rank * args.steps / t_step
@@ -914,9 +897,7 @@ def main():
             "alu_frac_fwd": fo / (t_fwd / args.steps) / 1e12 / alu_peak,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "overlap": "two buffer sets; each step's host-to-device and device-to-host "
-                               "copies run on their own streams beside the next step's compute"},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": E2E_OVERLAP},
             "gpu_launches": launches,
             "clocks": clk,
         }
