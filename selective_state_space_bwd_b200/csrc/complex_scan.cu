@@ -6,10 +6,14 @@
 //   mu_t = g_t + w_{t+1},  w_t = conj(a_t) mu_t,  q_t = mu_t conj(a_t h_{t-1}) = w_t conj(h_{t-1}),
 //   du = mu,  dlambda = -sum s Re q,  dr = sigmoid(r) (-sum_k lambda Re q),
 //   domega = sum phi Im q,  dphi = sum_k omega Im q.
-// Thread = one mode of one batch row; CTA = kCplxKT modes x one time segment.  Tiles of steps are
-// streamed through a two-stage cp.async ring; the per-step sums over the modes (dr, dphi) go
-// through shared memory, one column per step.  Segments other than the first (forward) / last
-// (backward) take their entering carry from a summary + carry pass, as in the real mode.
+// A CTA takes kCplxKT modes of one batch row over one time segment and is warp-specialised: one
+// consumer thread per mode runs the recurrence (or the adjoint sweep) over 16-step tiles streamed
+// through its own cp.async ring, while two producer threads per mode compute the next tile's
+// transitions a = exp(-lambda s + i omega phi) (an exp2 and a sine/cosine per update, most of
+// the arithmetic, independent of the state) into one of two shared buffers, handed over with
+// named barriers.  The per-step sums over the modes (dr, dphi) go through shared memory, one
+// column per step.  Segments other than the first (forward) / last (backward) take their
+// entering carry from a summary + carry pass, as in the real mode.
 #include "real_common.cuh"
 
 namespace ssm {
@@ -22,7 +26,6 @@ using real::cp_async_wait;
 
 constexpr int KT = kCplxKT;
 constexpr int TTF = kCplxTT;   // forward tile: steps per stage
-constexpr int TTB = 16;        // backward tile (two input tiles per stage)
 constexpr int CB = 8;          // transitions computed together (independent of the state)
 
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
@@ -78,13 +81,13 @@ __device__ __forceinline__ float2 transition_from(float lam2, float om, float s,
 // The transitions a_{t,k} of CB consecutive steps (ss/sph at r0..r0+CB-1), computed together:
 // they do not depend on the state, so their arithmetic overlaps.  Phases out of the reduction's
 // range (never for |omega phi| < 6400) are redone with the library sincosf, warp-uniformly.
-template <int CB>
+template <int CB, int STRIDE = 1>
 __device__ __forceinline__ void transitions(float2 (&a)[CB], float lam2, float om,
                                             const float2* ssp, int r0) {
     bool any_far = false;
 #pragma unroll
     for (int u = 0; u < CB; ++u) {
-        const float2 sp = ssp[r0 + u];  // (s, phi)
+        const float2 sp = ssp[r0 + STRIDE * u];  // (s, phi)
         const float th = om * sp.y;
         float sn, cs;
         bool far;
@@ -95,7 +98,7 @@ __device__ __forceinline__ void transitions(float2 (&a)[CB], float lam2, float o
     if (__any_sync(0xffffffffu, any_far)) {
 #pragma unroll
         for (int u = 0; u < CB; ++u) {
-            const float2 sp = ssp[r0 + u];
+            const float2 sp = ssp[r0 + STRIDE * u];
             const float th = om * sp.y;
             if (fabsf(rintf(th * 0x1.45f306p-1f)) >= 4096.0f) {
                 float sn, cs;
@@ -112,72 +115,118 @@ __device__ __forceinline__ void step_scalars(const float* sr, const float* sp, f
     if (tid < rows) ssp[tid] = make_float2(softplus_acc(sr[tid]), sp[tid]);
 }
 
-// Forward.  SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end
-// state).  SUMMARY = false: the scan from the segment's entering state, writing h.
+// Forward, warp-specialised.  A CTA takes KT modes of one batch row over one time segment:
+// KT consumer threads (one per mode) run the recurrence h = a h + u, and 2 KT producer threads
+// (two per mode, alternate steps) compute the transitions a of the next 16-step tile into one of
+// two shared buffers.  The transitions (an exp2 and a sine/cosine per update, most of the
+// arithmetic) do not depend on the state, so the producers run ahead while the consumers' short
+// dependent chain and HBM stream proceed; FULL / EMPTY named barriers hand the buffers over.
+// SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end state).
+// SUMMARY = false: the scan from the segment's entering state, writing h.
+constexpr int FT = 16;                 // steps per tile (divides every chunk length)
+constexpr int F_CONS = KT;             // consumer threads
+constexpr int F_PROD = 2 * KT;         // producer threads
+constexpr int F_NT = F_CONS + F_PROD;
+constexpr int F_USTAGES = 3;           // u ring of the consumers
+constexpr int F_BAR_FULL = 1, F_BAR_EMPTY = 3, F_BAR_PROD = 5, F_BAR_CONS = 6;
+
+__device__ __forceinline__ void bar_sync_n(int id, int n) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_arrive_n(int id, int n) {
+    asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+
 template <bool SUMMARY>
-__global__ void __launch_bounds__(KT) cplx_fwd_kernel(CplxArgs p) {
-    __shared__ __align__(16) float2 su[2][TTF * KT];
-    __shared__ __align__(16) float sr[2][TTF], sp[2][TTF];
-    __shared__ float2 ssp[TTF];  // (softplus(r), phi) per step
+__global__ void __launch_bounds__(F_NT) cplx_fwd_kernel(CplxArgs p) {
+    __shared__ __align__(16) float2 sa[2][FT * KT];           // transitions of a tile
+    __shared__ __align__(16) float2 su[F_USTAGES][FT * KT];   // u of a tile
+    __shared__ float2 ssp[2][FT];                             // (softplus(r), phi) per step
     const int tid = threadIdx.x;
-    const int k0 = blockIdx.x * KT, k = k0 + tid;
-    const bool kv = k < p.K;
+    const int k0 = blockIdx.x * KT;
     const int b = blockIdx.y, seg = blockIdx.z;
-    const int TT = min(TTF, p.T);  // a tile never crosses a chunk end
     const int t_begin = seg * p.seg_chunks * p.T;
     const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
-    const int ntiles = (t_end - t_begin + TT - 1) / TT;
-    const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
+    const int ntiles = (t_end - t_begin + FT - 1) / FT;
+    const size_t boff = (size_t)b * p.L;
+
+    if (tid >= F_CONS) {
+        // ---------------------------------------------------------------- producers
+        const int pt = tid - F_CONS, kk = pt % KT, rp = pt / KT;  // mode, row parity
+        const int k = k0 + kk;
+        const bool kv = k < p.K;
+        const float lam2 = kv ? p.lam[k] * kLog2e : 0.0f, om = kv ? p.om[k] : 0.0f;
+        const float* rb = p.r + boff;
+        const float* pb = p.phi + boff;
+        // the step scalars of tile i + 1 are fetched while tile i is computed
+        float rn = 0.0f, pn = 0.0f;
+        if (pt < FT && t_begin + pt < t_end) {
+            rn = rb[t_begin + pt];
+            pn = pb[t_begin + pt];
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i & 1;
+            const int t0 = t_begin + i * FT, rows = min(FT, t_end - t0);
+            if (pt < FT) {
+                ssp[buf][pt] = pt < rows ? make_float2(softplus_acc(rn), pn) : make_float2(0.0f, 0.0f);
+                const int tn = t0 + FT + pt;
+                if (i + 1 < ntiles && tn < t_end) {
+                    rn = rb[tn];
+                    pn = pb[tn];
+                }
+            }
+            bar_sync_n(F_BAR_PROD, F_PROD);               // the step scalars are in
+            bar_sync_n(F_BAR_EMPTY + buf, F_NT);          // the consumers are done with buffer buf
+            float2 a[FT / 2];
+            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+#pragma unroll
+            for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
+            bar_arrive_n(F_BAR_FULL + buf, F_NT);         // buffer buf holds the tile's transitions
+        }
+        bar_sync_n(F_BAR_EMPTY + 0, F_NT);  // balance the consumers' last two releases
+        bar_sync_n(F_BAR_EMPTY + 1, F_NT);
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int k = k0 + tid;
+    const bool kv = k < p.K;
     float2 h = make_float2(0.0f, 0.0f), P = make_float2(1.0f, 0.0f);
     if (!SUMMARY && seg > 0 && kv)
         h = reinterpret_cast<const float2*>(p.hin)[((size_t)b * p.nseg + seg) * p.K + k];
-    const size_t boff = (size_t)b * p.L;
     const float2* ub = reinterpret_cast<const float2*>(p.u) + boff * p.K;
     float2* hb = SUMMARY ? nullptr : reinterpret_cast<float2*>(p.h) + boff * p.K;
-    const float* rb = p.r + boff;
-    const float* pb = p.phi + boff;
-
-    auto issue = [&](int j, int st) {
-        const int t0 = t_begin + j * TT;
-        cp_async_tile<float2, KT>(su[st], ub, t0, TT, p.L, k0, p.K, tid, KT);
-        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
-        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+    auto issue = [&](int i) {
+        if (i < ntiles)
+            cp_async_tile<float2, KT>(su[i % F_USTAGES], ub, t_begin + i * FT, FT, p.L, k0, p.K, tid,
+                                      F_CONS);
         cp_async_commit();
     };
-    if (ntiles > 0) issue(0, 0);
-    for (int j = 0; j < ntiles; ++j) {
-        const int st = j & 1;
-        if (j + 1 < ntiles) {
-            issue(j + 1, st ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    issue(0);
+    issue(1);
+    bar_arrive_n(F_BAR_EMPTY + 0, F_NT);  // both transition buffers start empty
+    bar_arrive_n(F_BAR_EMPTY + 1, F_NT);
+    for (int i = 0; i < ntiles; ++i) {
+        const int buf = i & 1;
+        const int t0 = t_begin + i * FT, rows = min(FT, t_end - t0);
+        cp_async_wait<F_USTAGES - 2>();
+        bar_sync_n(F_BAR_CONS, F_CONS);  // u of tile i is in; both consumer warps are past tile i-1
+        issue(i + 2);
+        const float2* sut = su[i % F_USTAGES];
+        const float2* sat = sa[buf];
+        bar_sync_n(F_BAR_FULL + buf, F_NT);  // the producers have written the tile's transitions
+#pragma unroll 4
+        for (int r = 0; r < rows; ++r) {
+            const float2 av = sat[r * KT + tid];
+            const float2 uu = sut[r * KT + tid];
+            const float2 ah = cmul(av, h);
+            h = make_float2(ah.x + uu.x, ah.y + uu.y);
+            if (SUMMARY)
+                P = cmul(av, P);
+            else if (kv)
+                hb[(size_t)(t0 + r) * p.K + k] = h;
         }
-        __syncthreads();
-        const int t0 = t_begin + j * TT;
-        const int rows = min(TT, t_end - t0);
-        step_scalars(sr[st], sp[st], ssp, rows, tid);
-        __syncthreads();
-        const float2* sut = su[st];
-        // transitions of CB steps at a time (independent of h), then their recurrence steps
-        for (int r0 = 0; r0 < rows; r0 += CB) {
-            float2 a[CB];
-            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
-#pragma unroll
-            for (int u = 0; u < CB; ++u) {
-                const int r = r0 + u;
-                if (r < rows) {
-                    const float2 uu = sut[r * KT + tid];
-                    const float2 ah = cmul(a[u], h);
-                    h = make_float2(ah.x + uu.x, ah.y + uu.y);
-                    if (SUMMARY)
-                        P = cmul(a[u], P);
-                    else if (kv)
-                        hb[(size_t)(t0 + r) * p.K + k] = h;
-                }
-            }
-        }
-        __syncthreads();  // stage st and the step scalars are free again
+        bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // buffer buf is consumed
     }
     if (SUMMARY) {
         if (kv) {
@@ -285,90 +334,131 @@ __global__ void cplx_carry_bwd_kernel(int B, int nseg, int K, const float2* __re
     }
 }
 
-__global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
-    constexpr int TT = TTB;  // divides every chunk length, so tiles never cross a segment end
-    static_assert(TT * 4 == KT, "column sums: four threads per step");
-    __shared__ __align__(16) float2 sg[2][TT * KT];    // g of the tile's steps
-    __shared__ __align__(16) float2 shp[2][TT * KT];   // h_{t-1} of the tile's steps
-    __shared__ __align__(16) float sr[2][TT], sp[2][TT];
-    __shared__ float2 ssp[TT];  // (softplus(r), phi) per step
-    __shared__ __align__(16) float2 red[TT * KT];      // (lambda Re q, omega Im q) per step, mode
+// Backward, warp-specialised like the forward: KT consumer threads (one per mode) sweep the
+// adjoint backwards over 16-step tiles of g and h_{t-1} (their own two-stage cp.async ring) and
+// sum (lambda Re q, omega Im q) over the CTA's modes per step; 2 KT producer threads compute the
+// transitions of the next (earlier) tile, and the tile's step scalars (softplus(r), phi), into
+// one of two shared buffers.
+constexpr int B_USTAGES = 2;
+constexpr int B_SMEM = ((2 + 2 * B_USTAGES) * FT * KT + 2 * FT) * (int)sizeof(float2);
+
+__global__ void __launch_bounds__(F_NT) cplx_bwd_kernel(CplxArgs p) {
+    static_assert(FT * 4 == KT, "column sums: four consumer threads per step");
+    // dynamic shared memory (49.4 KB): transitions [2][FT*KT], g and h_{t-1} [B_USTAGES][FT*KT],
+    // step scalars [2][FT].  The per-step (lambda Re q, omega Im q) overwrite the g of the tile
+    // being swept: each consumer reads g at (r, mode) and then writes there, and the stage is not
+    // refilled before the column sums that read them are done.
+    extern __shared__ __align__(16) float2 cdyn[];
+    float2 (*sa)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn);
+    float2 (*sg)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + 2 * FT * KT);
+    float2 (*shp)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + (2 + B_USTAGES) * FT * KT);
+    float2 (*ssp)[FT] = reinterpret_cast<float2 (*)[FT]>(cdyn + (2 + 2 * B_USTAGES) * FT * KT);
     const int tid = threadIdx.x;
-    const int k0 = blockIdx.x * KT, k = k0 + tid;
-    const bool kv = k < p.K;
+    const int k0 = blockIdx.x * KT;
     const int b = blockIdx.y, seg = blockIdx.z;
     const int t_begin = seg * p.seg_chunks * p.T;
     const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
-    const int ntiles = (t_end - t_begin + TT - 1) / TT;
+    const int ntiles = (t_end - t_begin + FT - 1) / FT;
+    const size_t boff = (size_t)b * p.L;
+
+    if (tid >= F_CONS) {
+        // ---------------------------------------------------------------- producers
+        const int pt = tid - F_CONS, kk = pt % KT, rp = pt / KT;
+        const int k = k0 + kk;
+        const bool kv = k < p.K;
+        const float lam2 = kv ? p.lam[k] * kLog2e : 0.0f, om = kv ? p.om[k] : 0.0f;
+        const float* rb = p.r + boff;
+        const float* pb = p.phi + boff;
+        float rn = 0.0f, pn = 0.0f;  // step scalars of the next tile, fetched a tile ahead
+        {
+            const int t = t_begin + (ntiles - 1) * FT + pt;
+            if (ntiles > 0 && pt < FT && t < t_end) {
+                rn = rb[t];
+                pn = pb[t];
+            }
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i & 1, jt = ntiles - 1 - i;
+            const int t0 = t_begin + jt * FT, rows = min(FT, t_end - t0);
+            bar_sync_n(F_BAR_EMPTY + buf, F_NT);  // the consumers are done with buffer buf
+            if (pt < FT) {
+                ssp[buf][pt] = pt < rows ? make_float2(softplus_acc(rn), pn) : make_float2(0.0f, 0.0f);
+                if (jt > 0) {  // the earlier tile is always full
+                    rn = rb[t0 - FT + pt];
+                    pn = pb[t0 - FT + pt];
+                }
+            }
+            bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
+            float2 a[FT / 2];
+            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+#pragma unroll
+            for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
+            bar_arrive_n(F_BAR_FULL + buf, F_NT);  // buffer buf holds the tile's transitions
+        }
+        bar_sync_n(F_BAR_EMPTY + 0, F_NT);  // balance the consumers' last two releases
+        bar_sync_n(F_BAR_EMPTY + 1, F_NT);
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int k = k0 + tid;
+    const bool kv = k < p.K;
     const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
     float2 w = make_float2(0.0f, 0.0f);
     if (seg < p.nseg - 1 && kv)
         w = reinterpret_cast<const float2*>(p.win)[((size_t)b * p.nseg + seg) * p.K + k];
     float dlam = 0.0f, dom = 0.0f;
-    const size_t boff = (size_t)b * p.L;
     const float2* gb = reinterpret_cast<const float2*>(p.g) + boff * p.K;
     const float2* hb = reinterpret_cast<const float2*>(p.h_in) + boff * p.K;
     float2* dub = reinterpret_cast<float2*>(p.du) + boff * p.K;
-    const float* rb = p.r + boff;
-    const float* pb = p.phi + boff;
     float2* partb = reinterpret_cast<float2*>(p.rp_part) + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L;
-    // column-sum roles: step cs_r, a quarter of the modes each
-    const int cs_r = tid >> 2, cs_part = tid & 3;
-
-    auto issue = [&](int j, int st) {
-        const int t0 = t_begin + j * TT;
-        cp_async_tile<float2, KT>(sg[st], gb, t0, TT, p.L, k0, p.K, tid, KT);
-        if (t0 > 0) {
-            cp_async_tile<float2, KT>(shp[st], hb, t0 - 1, TT, p.L, k0, p.K, tid, KT);
-        } else {  // h_{-1} = 0
-            shp[st][tid] = make_float2(0.0f, 0.0f);
-            cp_async_tile<float2, KT>(shp[st] + KT, hb, 0, TT - 1, p.L, k0, p.K, tid, KT);
-        }
-        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
-        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
-        cp_async_commit();
-    };
-    if (ntiles > 0) issue(ntiles - 1, (ntiles - 1) & 1);
-    for (int j = ntiles - 1; j >= 0; --j) {
-        const int st = j & 1;
-        if (j > 0) {
-            issue(j - 1, st ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const int t0 = t_begin + j * TT;
-        const int rows = min(TT, t_end - t0);
-        step_scalars(sr[st], sp[st], ssp, rows, tid);
-        __syncthreads();
-        const float2* sgt = sg[st];
-        const float2* sht = shp[st];
-        // transitions of CB steps at a time, then their reverse steps (last first)
-        for (int r0 = ((rows - 1) / CB) * CB; r0 >= 0; r0 -= CB) {
-            float2 a[CB];
-            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
-#pragma unroll
-            for (int u = CB - 1; u >= 0; --u) {
-                const int r = r0 + u;
-                if (r < rows) {
-                    const float2 sp2 = ssp[r];
-                    const float s = sp2.x, ph = sp2.y;
-                    const float2 gg = sgt[r * KT + tid];
-                    const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
-                    w = cmul_ca(a[u], mu);
-                    const float2 q = cmul_cb(w, sht[r * KT + tid]);
-                    if (kv) dub[(size_t)(t0 + r) * p.K + k] = mu;
-                    dlam = fmaf(-s, q.x, dlam);
-                    dom = fmaf(ph, q.y, dom);
-                    red[r * KT + tid] = make_float2(lam * q.x, om * q.y);
-                }
+    const int cs_r = tid >> 2, cs_part = tid & 3;  // column sums: step cs_r, a quarter of the modes
+    auto issue = [&](int jt) {
+        if (jt >= 0) {
+            const int st = jt % B_USTAGES, t0 = t_begin + jt * FT;
+            cp_async_tile<float2, KT>(sg[st], gb, t0, FT, p.L, k0, p.K, tid, F_CONS);
+            if (t0 > 0) {
+                cp_async_tile<float2, KT>(shp[st], hb, t0 - 1, FT, p.L, k0, p.K, tid, F_CONS);
+            } else {  // h_{-1} = 0
+                shp[st][tid] = make_float2(0.0f, 0.0f);
+                cp_async_tile<float2, KT>(shp[st] + KT, hb, 0, FT - 1, p.L, k0, p.K, tid, F_CONS);
             }
         }
-        __syncthreads();
-        // sums over the CTA's modes, one step per four threads; the rotation by tid keeps each
-        // half-warp's 8-byte loads in distinct banks
+        cp_async_commit();
+    };
+    issue(ntiles - 1);
+    bar_arrive_n(F_BAR_EMPTY + 0, F_NT);  // both transition buffers start empty
+    bar_arrive_n(F_BAR_EMPTY + 1, F_NT);
+    for (int i = 0; i < ntiles; ++i) {
+        const int buf = i & 1, jt = ntiles - 1 - i, st = jt % B_USTAGES;
+        const int t0 = t_begin + jt * FT, rows = min(FT, t_end - t0);
+        cp_async_wait<0>();
+        bar_sync_n(F_BAR_CONS, F_CONS);  // g, h of tile jt are in; both consumer warps are past jt+1
+        issue(jt - 1);
+        const float2* sgt = sg[st];
+        const float2* sht = shp[st];
+        const float2* sat = sa[buf];
+        const float2* sst = ssp[buf];
+        float2* red = sg[st];
+        bar_sync_n(F_BAR_FULL + buf, F_NT);  // the producers have written the tile's transitions
+#pragma unroll 4
+        for (int r = rows - 1; r >= 0; --r) {
+            const float2 sp2 = sst[r];
+            const float2 av = sat[r * KT + tid];
+            const float2 gg = sgt[r * KT + tid];
+            const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
+            w = cmul_ca(av, mu);
+            const float2 q = cmul_cb(w, sht[r * KT + tid]);
+            if (kv) dub[(size_t)(t0 + r) * p.K + k] = mu;
+            dlam = fmaf(-sp2.x, q.x, dlam);
+            dom = fmaf(sp2.y, q.y, dom);
+            red[r * KT + tid] = make_float2(lam * q.x, om * q.y);
+        }
+        bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // transitions and step scalars are consumed
+        bar_sync_n(F_BAR_CONS, F_CONS);         // the tile's (lambda Re q, omega Im q) are in
         {
+            // sums over the CTA's modes, one step per four threads; the rotation by tid keeps
+            // each half-warp's 8-byte loads in distinct banks
             float2 acc = make_float2(0.0f, 0.0f);
             const float2* row = red + cs_r * KT + cs_part * (KT / 4);
 #pragma unroll
@@ -384,7 +474,6 @@ __global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
             }
             if (cs_part == 0 && cs_r < rows) partb[t0 + cs_r] = acc;
         }
-        __syncthreads();  // stage st, red and the step scalars are free again
     }
     if (kv) {
         const size_t o = ((size_t)b * p.nseg + seg) * p.K + k;
@@ -400,19 +489,64 @@ __global__ void __launch_bounds__(KT) cplx_bwd_kernel(CplxArgs p) {
 // and the gradient of Re sum conj(g) h accumulates as the steps arrive:
 //   dlambda += Re(conj(g_t) S^lambda_t),  domega += Re(conj(g_t) S^omega_t).
 // One forward pass, no reverse sweep, nothing of the trajectory kept (h is written only if asked).
-// Thread = one mode of one batch row over the whole sequence.
-__global__ void __launch_bounds__(KT) cplx_rtrl_kernel(CplxArgs p) {
-    constexpr int TT = 16;
-    __shared__ __align__(16) float2 su[2][TT * KT];
-    __shared__ __align__(16) float2 sgt[2][TT * KT];
-    __shared__ __align__(16) float sr[2][TT], sp[2][TT];
-    __shared__ float2 ssp[TT];  // (softplus(r), phi) per step
+// A CTA takes KT modes of one batch row over the whole sequence.
+__global__ void __launch_bounds__(F_NT) cplx_rtrl_kernel(CplxArgs p) {
+    // warp-specialised like the forward: KT consumer threads carry (h, S^lambda, S^omega) of one
+    // mode each over 16-step tiles of u and g (their own two-stage cp.async ring); 2 KT producer
+    // threads compute the next tile's transitions and step scalars into one of two buffers.
+    // Dynamic shared memory (49.4 KB): transitions [2][FT*KT], u and g [B_USTAGES][FT*KT], step
+    // scalars [2][FT].
+    extern __shared__ __align__(16) float2 cdyn[];
+    float2 (*sa)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn);
+    float2 (*su)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + 2 * FT * KT);
+    float2 (*sgt)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + (2 + B_USTAGES) * FT * KT);
+    float2 (*ssp)[FT] = reinterpret_cast<float2 (*)[FT]>(cdyn + (2 + 2 * B_USTAGES) * FT * KT);
     const int tid = threadIdx.x;
-    const int k0 = blockIdx.x * KT, k = k0 + tid;
-    const bool kv = k < p.K;
+    const int k0 = blockIdx.x * KT;
     const int b = blockIdx.y;
-    const int ntiles = (p.L + TT - 1) / TT;
-    const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
+    const int ntiles = (p.L + FT - 1) / FT;
+    const size_t boff = (size_t)b * p.L;
+
+    if (tid >= F_CONS) {
+        // ---------------------------------------------------------------- producers
+        const int pt = tid - F_CONS, kk = pt % KT, rp = pt / KT;
+        const int k = k0 + kk;
+        const bool kv = k < p.K;
+        const float lam2 = kv ? p.lam[k] * kLog2e : 0.0f, om = kv ? p.om[k] : 0.0f;
+        const float* rb = p.r + boff;
+        const float* pb = p.phi + boff;
+        float rn = 0.0f, pn = 0.0f;  // step scalars of the next tile, fetched a tile ahead
+        if (pt < FT && pt < p.L) {
+            rn = rb[pt];
+            pn = pb[pt];
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i & 1;
+            const int t0 = i * FT, rows = min(FT, p.L - t0);
+            bar_sync_n(F_BAR_EMPTY + buf, F_NT);  // the consumers are done with buffer buf
+            if (pt < FT) {
+                ssp[buf][pt] = pt < rows ? make_float2(softplus_acc(rn), pn) : make_float2(0.0f, 0.0f);
+                const int tn = t0 + FT + pt;
+                if (tn < p.L) {
+                    rn = rb[tn];
+                    pn = pb[tn];
+                }
+            }
+            bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
+            float2 a[FT / 2];
+            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+#pragma unroll
+            for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
+            bar_arrive_n(F_BAR_FULL + buf, F_NT);
+        }
+        bar_sync_n(F_BAR_EMPTY + 0, F_NT);  // balance the consumers' last two releases
+        bar_sync_n(F_BAR_EMPTY + 1, F_NT);
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int k = k0 + tid;
+    const bool kv = k < p.K;
     float2* stb = p.state ? reinterpret_cast<float2*>(p.state) + (size_t)b * 3 * p.K : nullptr;
     float2 h = make_float2(0.0f, 0.0f), Sl = h, So = h;
     if (stb && kv) {
@@ -421,57 +555,47 @@ __global__ void __launch_bounds__(KT) cplx_rtrl_kernel(CplxArgs p) {
         So = stb[2 * p.K + k];
     }
     float dl = 0.0f, dom = 0.0f;
-    const size_t boff = (size_t)b * p.L;
     const float2* ub = reinterpret_cast<const float2*>(p.u) + boff * p.K;
     const float2* gb = reinterpret_cast<const float2*>(p.g) + boff * p.K;
     float2* hb = p.h ? reinterpret_cast<float2*>(p.h) + boff * p.K : nullptr;
-    const float* rb = p.r + boff;
-    const float* pb = p.phi + boff;
-
-    auto issue = [&](int j, int st) {
-        const int t0 = j * TT;
-        cp_async_tile<float2, KT>(su[st], ub, t0, TT, p.L, k0, p.K, tid, KT);
-        cp_async_tile<float2, KT>(sgt[st], gb, t0, TT, p.L, k0, p.K, tid, KT);
-        cp_async_flat<float>(sr[st], rb, (size_t)t0, TT, (size_t)p.L, tid, KT);
-        cp_async_flat<float>(sp[st], pb, (size_t)t0, TT, (size_t)p.L, tid, KT);
+    auto issue = [&](int i) {
+        if (i < ntiles) {
+            const int st = i % B_USTAGES;
+            cp_async_tile<float2, KT>(su[st], ub, i * FT, FT, p.L, k0, p.K, tid, F_CONS);
+            cp_async_tile<float2, KT>(sgt[st], gb, i * FT, FT, p.L, k0, p.K, tid, F_CONS);
+        }
         cp_async_commit();
     };
-    if (ntiles > 0) issue(0, 0);
-    for (int j = 0; j < ntiles; ++j) {
-        const int st = j & 1;
-        if (j + 1 < ntiles) {
-            issue(j + 1, st ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    issue(0);
+    bar_arrive_n(F_BAR_EMPTY + 0, F_NT);  // both transition buffers start empty
+    bar_arrive_n(F_BAR_EMPTY + 1, F_NT);
+    for (int i = 0; i < ntiles; ++i) {
+        const int buf = i & 1, st = i % B_USTAGES;
+        const int t0 = i * FT, rows = min(FT, p.L - t0);
+        cp_async_wait<0>();
+        bar_sync_n(F_BAR_CONS, F_CONS);  // u, g of tile i are in; both consumer warps are past i-1
+        issue(i + 1);
+        const float2* sut = su[st];
+        const float2* sgg = sgt[st];
+        const float2* sat = sa[buf];
+        const float2* sst = ssp[buf];
+        bar_sync_n(F_BAR_FULL + buf, F_NT);  // the producers have written the tile's transitions
+#pragma unroll 4
+        for (int r = 0; r < rows; ++r) {
+            const float2 sp2 = sst[r];  // (s, phi)
+            const float2 av = sat[r * KT + tid];
+            const float2 ah = cmul(av, h);
+            const float2 al = cmul(av, Sl), ao = cmul(av, So);
+            Sl = make_float2(fmaf(-sp2.x, ah.x, al.x), fmaf(-sp2.x, ah.y, al.y));
+            So = make_float2(fmaf(-sp2.y, ah.y, ao.x), fmaf(sp2.y, ah.x, ao.y));
+            const float2 uu = sut[r * KT + tid];
+            h = make_float2(ah.x + uu.x, ah.y + uu.y);
+            const float2 gg = sgg[r * KT + tid];
+            dl = fmaf(gg.x, Sl.x, fmaf(gg.y, Sl.y, dl));
+            dom = fmaf(gg.x, So.x, fmaf(gg.y, So.y, dom));
+            if (hb && kv) hb[(size_t)(t0 + r) * p.K + k] = h;
         }
-        __syncthreads();
-        const int t0 = j * TT;
-        const int rows = min(TT, p.L - t0);
-        step_scalars(sr[st], sp[st], ssp, rows, tid);
-        __syncthreads();
-        for (int r0 = 0; r0 < rows; r0 += CB) {
-            float2 a[CB];
-            transitions<CB>(a, lam * kLog2e, om, ssp, r0);
-#pragma unroll
-            for (int u = 0; u < CB; ++u) {
-                const int r = r0 + u;
-                if (r < rows) {
-                    const float2 sp2 = ssp[r];  // (s, phi)
-                    const float2 ah = cmul(a[u], h);
-                    const float2 al = cmul(a[u], Sl), ao = cmul(a[u], So);
-                    Sl = make_float2(fmaf(-sp2.x, ah.x, al.x), fmaf(-sp2.x, ah.y, al.y));
-                    So = make_float2(fmaf(-sp2.y, ah.y, ao.x), fmaf(sp2.y, ah.x, ao.y));
-                    const float2 uu = su[st][r * KT + tid];
-                    h = make_float2(ah.x + uu.x, ah.y + uu.y);
-                    const float2 gg = sgt[st][r * KT + tid];
-                    dl = fmaf(gg.x, Sl.x, fmaf(gg.y, Sl.y, dl));
-                    dom = fmaf(gg.x, So.x, fmaf(gg.y, So.y, dom));
-                    if (hb && kv) hb[(size_t)(t0 + r) * p.K + k] = h;
-                }
-            }
-        }
-        __syncthreads();  // stage st and the step scalars are free again
+        bar_arrive_n(F_BAR_EMPTY + buf, F_NT);
     }
     if (kv) {
         reinterpret_cast<float2*>(p.lo_part)[(size_t)b * p.K + k] = make_float2(dl, dom);
@@ -520,7 +644,7 @@ __global__ void cplx_reduce_k_kernel(CplxArgs p) {
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st) {
     cudaError_t e;
     if (a.nseg > 1) {
-        cplx_fwd_kernel<true><<<dim3(a.nkt, a.B, a.nseg - 1), KT, 0, st>>>(a);
+        cplx_fwd_kernel<true><<<dim3(a.nkt, a.B, a.nseg - 1), F_NT, 0, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.K;
         cplx_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
@@ -528,13 +652,15 @@ cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st) {
             reinterpret_cast<const float2*>(a.sumS), reinterpret_cast<float2*>(a.hin));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    cplx_fwd_kernel<false><<<dim3(a.nkt, a.B, a.nseg), KT, 0, st>>>(a);
+    cplx_fwd_kernel<false><<<dim3(a.nkt, a.B, a.nseg), F_NT, 0, st>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_cplx_rtrl(const CplxArgs& a, cudaStream_t st) {
     cudaError_t e;
-    cplx_rtrl_kernel<<<dim3(a.nkt, a.B, 1), KT, 0, st>>>(a);
+    e = cudaFuncSetAttribute(cplx_rtrl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM);
+    if (e != cudaSuccess) return e;
+    cplx_rtrl_kernel<<<dim3(a.nkt, a.B, 1), F_NT, B_SMEM, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cplx_reduce_k_kernel<<<(a.K + 255) / 256, 256, 0, st>>>(a);  // sums over b (nseg = 1)
     return cudaGetLastError();
@@ -551,7 +677,9 @@ cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st) {
             reinterpret_cast<const float2*>(a.gsumG), reinterpret_cast<float2*>(a.win));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    cplx_bwd_kernel<<<dim3(a.nkt, a.B, a.nseg), KT, 0, st>>>(a);
+    e = cudaFuncSetAttribute(cplx_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM);
+    if (e != cudaSuccess) return e;
+    cplx_bwd_kernel<<<dim3(a.nkt, a.B, a.nseg), F_NT, B_SMEM, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t n = (int64_t)a.B * a.L;
     if (n > 0) {
