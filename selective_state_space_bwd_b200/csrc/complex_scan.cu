@@ -109,6 +109,71 @@ __device__ __forceinline__ void transitions(float2 (&a)[CB], float lam2, float o
     }
 }
 
+// The same transitions, two steps per packed fp32x2 operation (the producers' path): the
+// reduction, both polynomials, the residual rotation and the decay exponent run as FFMA2 / FMUL2
+// on (step u, step u+1), component by component the same roundings as transitions(), so the
+// results are identical; the quadrant selection stays scalar.
+template <int CB, int STRIDE>
+__device__ __forceinline__ void transitions_pk(float2 (&a)[CB], float lam2, float om,
+                                               const float2* ssp, int r0) {
+    static_assert(CB % 2 == 0, "steps in pairs");
+    using real::f2;
+    bool any_far = false;
+#pragma unroll
+    for (int u = 0; u < CB; u += 2) {
+        const float2 sp0 = ssp[r0 + STRIDE * u], sp1 = ssp[r0 + STRIDE * (u + 1)];  // (s, phi)
+        const float2 ph = make_float2(sp0.y, sp1.y);
+        const float2 th = __fmul2_rn(f2(om), ph);
+        const float2 tq = __fmul2_rn(th, f2(0x1.45f306p-1f));  // th * 2/pi
+        const float2 kq = make_float2(rintf(tq.x), rintf(tq.y));
+        any_far |= fabsf(kq.x) >= 4096.0f || fabsf(kq.y) >= 4096.0f;
+        const float2 nk = make_float2(-kq.x, -kq.y);
+        float2 x = __ffma2_rn(nk, f2(0x1.92p+0f), th);
+        x = __ffma2_rn(nk, f2(0x1.fb4p-12f), x);
+        x = __ffma2_rn(nk, f2(0x1.4442d2p-24f), x);
+        const float2 x2 = __fmul2_rn(x, x);
+        float2 ps = __ffma2_rn(x2, f2(1.0f / 362880.0f), f2(-1.0f / 5040.0f));
+        ps = __ffma2_rn(x2, ps, f2(1.0f / 120.0f));
+        ps = __ffma2_rn(x2, ps, f2(-1.0f / 6.0f));
+        const float2 sv = __ffma2_rn(__fmul2_rn(x, x2), ps, x);
+        float2 pc = __ffma2_rn(x2, f2(-1.0f / 3628800.0f), f2(1.0f / 40320.0f));
+        pc = __ffma2_rn(x2, pc, f2(-1.0f / 720.0f));
+        pc = __ffma2_rn(x2, pc, f2(1.0f / 24.0f));
+        pc = __ffma2_rn(x2, pc, f2(-0.5f));
+        const float2 cv = __ffma2_rn(x2, pc, f2(1.0f));
+        float2 sn, cs;
+        {
+            const int q = static_cast<int>(kq.x) & 3;
+            sn.x = q == 0 ? sv.x : (q == 1 ? cv.x : (q == 2 ? -sv.x : -cv.x));
+            cs.x = q == 0 ? cv.x : (q == 1 ? -sv.x : (q == 2 ? -cv.x : sv.x));
+        }
+        {
+            const int q = static_cast<int>(kq.y) & 3;
+            sn.y = q == 0 ? sv.y : (q == 1 ? cv.y : (q == 2 ? -sv.y : -cv.y));
+            cs.y = q == 0 ? cv.y : (q == 1 ? -sv.y : (q == 2 ? -cv.y : sv.y));
+        }
+        const float2 ls = __fmul2_rn(f2(-lam2), make_float2(sp0.x, sp1.x));
+        const float2 rho = make_float2(ex2_mufu(ls.x), ex2_mufu(ls.y));
+        const float2 tl = __ffma2_rn(f2(om), ph, make_float2(-th.x, -th.y));
+        const float2 c2 = __ffma2_rn(make_float2(-tl.x, -tl.y), sn, cs);
+        const float2 s2 = __ffma2_rn(tl, cs, sn);
+        a[u] = make_float2(rho.x * c2.x, rho.x * s2.x);
+        a[u + 1] = make_float2(rho.y * c2.y, rho.y * s2.y);
+    }
+    if (__any_sync(0xffffffffu, any_far)) {
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const float2 sp = ssp[r0 + STRIDE * u];
+            const float th = om * sp.y;
+            if (fabsf(rintf(th * 0x1.45f306p-1f)) >= 4096.0f) {
+                float sn, cs;
+                sincosf(th, &sn, &cs);
+                a[u] = transition_from(lam2, om, sp.x, sp.y, th, sn, cs);
+            }
+        }
+    }
+}
+
 // Per-step scalars of a staged tile: s = softplus(r) and phi, for `rows` steps.
 __device__ __forceinline__ void step_scalars(const float* sr, const float* sp, float2* ssp,
                                              int rows, int tid) {
@@ -178,7 +243,7 @@ __global__ void __launch_bounds__(F_NT) cplx_fwd_kernel(CplxArgs p) {
             bar_sync_n(F_BAR_PROD, F_PROD);               // the step scalars are in
             bar_sync_n(F_BAR_EMPTY + buf, F_NT);          // the consumers are done with buffer buf
             float2 a[FT / 2];
-            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+            transitions_pk<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
 #pragma unroll
             for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
             bar_arrive_n(F_BAR_FULL + buf, F_NT);         // buffer buf holds the tile's transitions
@@ -390,7 +455,7 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_kernel(CplxArgs p) {
             }
             bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
             float2 a[FT / 2];
-            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+            transitions_pk<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
 #pragma unroll
             for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
             bar_arrive_n(F_BAR_FULL + buf, F_NT);  // buffer buf holds the tile's transitions
@@ -534,7 +599,7 @@ __global__ void __launch_bounds__(F_NT) cplx_rtrl_kernel(CplxArgs p) {
             }
             bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
             float2 a[FT / 2];
-            transitions<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+            transitions_pk<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
 #pragma unroll
             for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
             bar_arrive_n(F_BAR_FULL + buf, F_NT);
