@@ -11,9 +11,10 @@
 // through its own cp.async ring, while two producer threads per mode compute the next tile's
 // transitions a = exp(-lambda s + i omega phi) (an exp2 and a sine/cosine per update, most of
 // the arithmetic, independent of the state) into one of two shared buffers, handed over with
-// named barriers.  The per-step sums over the modes (dr, dphi) go through shared memory, one
-// column per step.  Segments other than the first (forward) / last (backward) take their
-// entering carry from a summary + carry pass, as in the real mode.
+// named barriers (the barrier sequences of both roles are model-checked on the host by
+// tests/test_barrier_protocol.py).  The per-step sums over the modes (dr, dphi) go through
+// shared memory, one column per step.  Segments other than the first (forward) / last
+// (backward) take their entering carry from a summary + carry pass, as in the real mode.
 #include "real_common.cuh"
 
 namespace ssm {

@@ -421,8 +421,9 @@ __global__ void __launch_bounds__(NT) pdssm_carry_fwd_kernel(PdArgs p) {
 // cp.async ring) and leaves mu and x = d h_{t-1} of each tile in one of two shared buffers; the
 // score-gradient warp takes the tile from there (one lane per (step, head) entry, the scores
 // through its own ring) while the scan warp goes on with the next tile.  The two hand the buffers
-// over with named barriers (FULL: written, EMPTY: read).  The latency-bound scan and the
-// arithmetic-bound score gradient so run side by side instead of in turn.
+// over with named barriers (FULL: written, EMPTY: read; the sequence of barrier operations of
+// both roles is model-checked on the host by tests/test_barrier_protocol.py).  The latency-bound
+// scan and the arithmetic-bound score gradient so run side by side instead of in turn.
 //
 // Shared memory per scan warp: g, d, h_{t-1} [2][TT][32] floats and sel [2][TT*SPW]; per pair:
 // mu and x [2 buffers][TT][RS] with RS = SPW*(N+1) = 32 + SPW (state i of entry (r, c) at
