@@ -55,6 +55,10 @@ def _load():
             lib.ssm_oracle_pdssm.argtypes = ([I64] * 5 + [P] * 6 + [ctypes.c_double, ctypes.c_int] +
                                              [P] * 6)
             lib.ssm_oracle_pdssm.restype = ctypes.c_int
+            lib.ssm_oracle_dtproj.argtypes = [I64, I64, I64] + [P] * 4
+            lib.ssm_oracle_dtproj.restype = ctypes.c_int
+            lib.ssm_oracle_dtproj_bwd.argtypes = [I64, I64, I64] + [P] * 6
+            lib.ssm_oracle_dtproj_bwd.restype = ctypes.c_int
             lib.ssm_oracle_max_threads.argtypes = []
             lib.ssm_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -208,3 +212,33 @@ def pdssm(scores, dictionary, d, bt, h0=None, g=None, tau=1.0, threads=0):
     if rc != 0:
         raise RuntimeError("ssm_oracle_pdssm failed (bad argument or out of memory)")
     return out
+
+
+def dtproj(u, w, bias=None, g=None):
+    """Step-size projection delta_raw[m, d] = sum_r u[m, r] w[d, r] + bias[d] over the rows of u
+    ([M, R] or [B, L, R]); with g = dL/d delta_raw also du, dw and dbias (see ssm_oracle.c)."""
+    lib = _load()
+    u = _f64(u)
+    lead = u.shape[:-1]
+    R = u.shape[-1]
+    u2 = u.reshape(-1, R)
+    w = _f64(w)
+    D = w.shape[0]
+    assert w.shape == (D, R)
+    M = u2.shape[0]
+    b = _f64(bias) if bias is not None else None
+    out = np.empty((M, D))
+    if lib.ssm_oracle_dtproj(M, D, R, _ptr(u2), _ptr(w), _ptr(b) if b is not None else None,
+                             _ptr(out)) != 0:
+        raise RuntimeError("ssm_oracle_dtproj failed")
+    res = {"delta_raw": out.reshape(*lead, D)}
+    if g is not None:
+        g2 = _f64(g).reshape(M, D)
+        du = np.empty((M, R))
+        dw = np.empty((D, R))
+        dbias = np.empty(D)
+        if lib.ssm_oracle_dtproj_bwd(M, D, R, _ptr(u2), _ptr(w), _ptr(g2), _ptr(du), _ptr(dw),
+                                     _ptr(dbias)) != 0:
+            raise RuntimeError("ssm_oracle_dtproj_bwd failed")
+        res.update(du=du.reshape(*lead, R), dw=dw, dbias=dbias)
+    return res

@@ -530,3 +530,53 @@ int ssm_oracle_pdssm(int64_t B, int64_t L, int64_t H, int64_t N, int64_t K,
     }
     return fail ? -1 : 0;
 }
+
+/*
+ * Step-size projection in front of the real scan ("选择性状态空间模型(S3M)原理与工程实践" §1.1:
+ * delta = softplus(projection(x)); §4.1 merges the discretisation with this matrix product).  Per
+ * row m (one (batch, step) pair) the pre-activation of every channel d is a rank-R linear map of
+ * the row's low-rank input u:
+ *     delta_raw[m, d] = sum_r u[m, r] w[d, r] + bias[d]
+ * and for an upstream gradient g = dL/d delta_raw:
+ *     du[m, r] = sum_d g[m, d] w[d, r],   dw[d, r] = sum_m g[m, d] u[m, r],   dbias[d] = sum_m g[m, d].
+ * Plain loops in float64, rows split across threads (forward, du) or channels split across threads
+ * (dw, dbias); every sum runs in index order.  bias and dbias may be NULL.
+ */
+int ssm_oracle_dtproj(int64_t M, int64_t D, int64_t R, const double* u, const double* w,
+                      const double* bias, double* out) {
+    if (M < 0 || D < 1 || R < 1 || !u || !w || !out) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int64_t r = 0; r < R; ++r) acc += u[m * R + r] * w[d * R + r];
+            out[m * D + d] = acc + (bias ? bias[d] : 0.0);
+        }
+    return 0;
+}
+
+int ssm_oracle_dtproj_bwd(int64_t M, int64_t D, int64_t R, const double* u, const double* w,
+                          const double* g, double* du, double* dw, double* dbias) {
+    if (M < 0 || D < 1 || R < 1 || !u || !w || !g || !du || !dw) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t r = 0; r < R; ++r) {
+            double acc = 0.0;
+            for (int64_t d = 0; d < D; ++d) acc += g[m * D + d] * w[d * R + r];
+            du[m * R + r] = acc;
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t d = 0; d < D; ++d) {
+        for (int64_t r = 0; r < R; ++r) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += g[m * D + d] * u[m * R + r];
+            dw[d * R + r] = acc;
+        }
+        if (dbias) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += g[m * D + d];
+            dbias[d] = acc;
+        }
+    }
+    return 0;
+}

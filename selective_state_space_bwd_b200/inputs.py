@@ -125,6 +125,23 @@ def real_inputs(batch, seqlen, dim, dstate, io=F32, kind="mamba", seed=0):
     return out
 
 
+def dtproj_inputs(batch, seqlen, dim, rank, seed=0):
+    """Draw the step-size projection of one real-mode problem (bf16 I/O).
+
+    u ~ N(0,1) [B,L,R] (the low-rank per-token input), w ~ N(0, 1/(4R)) [D,R], bias ~ U(lo, hi)
+    [D] with lo, hi the raw values whose softplus is 2e-3 and 5e-2, so that u w^T + bias (spread
+    ~0.5 about the bias) keeps softplus(delta_raw) near the workload's [1e-3, 1e-1]; the upstream
+    gradient ddelta_raw ~ N(0,1) [B,L,D].  u, w, ddelta_raw are rounded to bf16; bias is fp32.
+    """
+    rng = np.random.default_rng(seed)
+    B, L, D, R = int(batch), int(seqlen), int(dim), int(rank)
+    u = round_to_bf16(rng.standard_normal((B, L, R), dtype=np.float32))
+    w = round_to_bf16((rng.standard_normal((D, R)) / (2.0 * math.sqrt(R))).astype(np.float32))
+    bias = rng.uniform(_inv_softplus(2e-3), _inv_softplus(5e-2), size=(D,)).astype(np.float32)
+    g = round_to_bf16(rng.standard_normal((B, L, D), dtype=np.float32))
+    return dict(u=u, w=w, bias=bias, g=g)
+
+
 def complex_inputs(batch, seqlen, modes, seed=0):
     """Draw one complex-mode problem (SPARC-style shared control).
 
