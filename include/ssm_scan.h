@@ -303,6 +303,40 @@ int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, cons
                   const float* g, float* dd, float* dbt, float* dscores, float* dh0,
                   void* ws, size_t ws_bytes, ssm_stream_t stream);
 
+/*
+ * Step-size projection in front of the real scan ("选择性状态空间模型(S3M)原理与工程实践" §1.1:
+ * delta = softplus(projection(x)); §4.1 merges the discretisation with this matrix product).  One
+ * row m per (batch, step); each row's low-rank input u[m, :] maps to the pre-activation of every
+ * channel:
+ *     delta_raw[m, d] = sum_r u[m, r] w[d, r] + bias[d]
+ * which ssm_scan_fwd / ssm_scan_bwd then take as delta_raw ([B, L, D] is [M, D] with M = B*L).
+ * The backward of L for an upstream g = dL/d delta_raw (ssm_scan_bwd's ddelta_raw):
+ *     du[m, r] = sum_d g[m, d] w[d, r],   dw[d, r] = sum_m g[m, d] u[m, r],   dbias[d] = sum_m g[m, d].
+ * Tensor-core GEMMs with bf16 operands and fp32 accumulation; delta_raw and du are rounded to bf16
+ * once, dw and dbias are fp32.  Layout: u, du [M, R], w [D, R], delta_raw, g [M, D] bf16;
+ * bias, dbias [D], dw [D, R] fp32; bias and dbias may be NULL.
+ */
+typedef struct ssm_dtshape {
+    int64_t rows;   /* M >= 0 (0 is a valid empty problem), at most 65535 * 128 */
+    int64_t dim;    /* D, a multiple of 8 in 8..2^22 */
+    int32_t rank;   /* R, a multiple of 16 in 16..256 */
+    int32_t io;     /* SSM_BF16 (the only supported I/O type: SSM_ERR_UNSUPPORTED otherwise) */
+} ssm_dtshape;
+
+/* Workspace bytes of ssm_dtproj_bwd (fp32 partial sums of dw and dbias over splits of 512 rows;
+ * at least 256); 0 for an invalid shape. */
+size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape);
+
+/* delta_raw = u w^T + bias.  Enqueues 1 kernel.  Returns an ssm_status. */
+int ssm_dtproj_fwd(const ssm_dtshape* shape, const void* u, const void* w, const float* bias,
+                   void* delta_raw, ssm_stream_t stream);
+
+/* du, dw, dbias for g = dL/d delta_raw.  Enqueues 3 kernels (du; dw and dbias partial sums;
+ * their fixed-order reduction).  Returns an ssm_status. */
+int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const void* g,
+                   void* du, float* dw, float* dbias, void* ws, size_t ws_bytes,
+                   ssm_stream_t stream);
+
 /* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);

@@ -561,6 +561,66 @@ int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, cons
     return ssm::launch_pdssm_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+namespace {
+int check_dtshape(const ssm_dtshape* s) {
+    if (!s) return SSM_ERR_INVALID_ARG;
+    if (s->rows < 0 || s->dim < 1 || s->rank < 1) return SSM_ERR_INVALID_ARG;
+    if (s->io != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (s->dim % 8 != 0 || s->dim < 8 || s->rank % 16 != 0 || s->rank > 256) return SSM_ERR_UNSUPPORTED;
+    if (s->rows > (int64_t)65535 * 128 || s->dim > ((int64_t)1 << 22)) return SSM_ERR_UNSUPPORTED;
+    return SSM_OK;
+}
+
+int dt_splits(const ssm_dtshape* s) {
+    const int64_t k = ssm::dtproj_rows_per_split();
+    return (int)((s->rows + k - 1) / k);
+}
+}  // namespace
+
+size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape) {
+    if (check_dtshape(shape) != SSM_OK) return 0;
+    const size_t b = (size_t)dt_splits(shape) * shape->dim * (shape->rank + 1) * sizeof(float);
+    return b < 256 ? 256 : align256(b);
+}
+
+int ssm_dtproj_fwd(const ssm_dtshape* shape, const void* u, const void* w, const float* bias,
+                   void* delta_raw, ssm_stream_t stream) {
+    int st = check_dtshape(shape);
+    if (st != SSM_OK) return st;
+    const size_t M = shape->rows, D = shape->dim, R = shape->rank;
+    const void* ptrs[] = {u, w, delta_raw, bias};
+    const size_t counts[] = {M * R, D * R, M * D, bias ? D : 0};
+    if ((st = check_arrays(ptrs, counts, 4)) != SSM_OK) return st;
+    if (M == 0) return SSM_OK;
+    ssm::DtArgs a = {};
+    a.M = (int64_t)M; a.D = (int64_t)D; a.R = (int)R;
+    a.u = u; a.w = w; a.bias = bias; a.delta_raw = delta_raw;
+    return ssm::launch_dtproj_fwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const void* g,
+                   void* du, float* dw, float* dbias, void* ws, size_t ws_bytes,
+                   ssm_stream_t stream) {
+    int st = check_dtshape(shape);
+    if (st != SSM_OK) return st;
+    const size_t M = shape->rows, D = shape->dim, R = shape->rank;
+    const void* ptrs[] = {u, w, g, du, dw, ws, dbias};
+    const size_t counts[] = {M * R, D * R, M * D, M * R, D * R, 1, dbias ? D : 0};
+    if ((st = check_arrays(ptrs, counts, 7)) != SSM_OK) return st;
+    if (ws_bytes < ssm_dtproj_workspace_bytes(shape)) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (M == 0) {  // no rows: the sums are empty
+        if (cudaMemsetAsync(dw, 0, D * R * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (dbias && cudaMemsetAsync(dbias, 0, D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::DtArgs a = {};
+    a.M = (int64_t)M; a.D = (int64_t)D; a.R = (int)R; a.splits = dt_splits(shape);
+    a.u = u; a.w = w; a.g = g; a.du = du; a.dw = dw; a.dbias = dbias;
+    a.part = static_cast<float*>(ws);
+    return ssm::launch_dtproj_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 int ssm_scan_status(const void* ws, ssm_stream_t stream) {
     if (!ws) return SSM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -125,6 +125,25 @@ struct PdArgs {
     float* win;     // adjoint entering each segment from its end [B*H][nseg][N]
 };
 
+// Step-size projection (csrc/dtproj.cu): bf16 u [M, R], w [D, R], delta_raw / g [M, D],
+// du [M, R]; fp32 bias, dw [D, R], dbias [D]; part: `splits` x D x (R+1) fp32 partial sums.
+struct DtArgs {
+    int64_t M, D;
+    int R, splits;
+    const void* u;
+    const void* w;
+    const float* bias;
+    void* delta_raw;
+    const void* g;
+    void* du;
+    float* dw;
+    float* dbias;
+    float* part;
+};
+int64_t dtproj_rows_per_split();
+cudaError_t launch_dtproj_fwd(const DtArgs& a, cudaStream_t st);
+cudaError_t launch_dtproj_bwd(const DtArgs& a, cudaStream_t st);
+
 // Launchers (return cudaGetLastError() of the last launch).
 cudaError_t launch_pdssm_fwd(const PdArgs& a, cudaStream_t st);
 cudaError_t launch_pdssm_bwd(const PdArgs& a, cudaStream_t st);

@@ -51,6 +51,11 @@ class SsmPdShape(ctypes.Structure):
                 ("reserved2", ctypes.c_int32)]
 
 
+class SsmDtShape(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("dim", ctypes.c_int64), ("rank", ctypes.c_int32),
+                ("io", ctypes.c_int32)]
+
+
 class SsmError(RuntimeError):
     def __init__(self, code, what):
         self.code = code
@@ -67,7 +72,8 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex",
             "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
             "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd",
-            "ssm_pdssm_kernel_launches"]
+            "ssm_pdssm_kernel_launches", "ssm_dtproj_workspace_bytes", "ssm_dtproj_fwd",
+            "ssm_dtproj_bwd"]
 
 
 def lib():
@@ -113,6 +119,11 @@ def lib():
             L.ssm_pdssm_bwd.argtypes = [PP, ctypes.c_float] + [P] * 12 + [Z, P]
             L.ssm_pdssm_bwd.restype = I
             L.ssm_pdssm_kernel_launches.argtypes, L.ssm_pdssm_kernel_launches.restype = [PP, I], I
+            DP = ctypes.POINTER(SsmDtShape)
+            L.ssm_dtproj_workspace_bytes.argtypes, L.ssm_dtproj_workspace_bytes.restype = [DP], Z
+            L.ssm_dtproj_fwd.argtypes, L.ssm_dtproj_fwd.restype = [DP] + [P] * 4 + [P], I
+            L.ssm_dtproj_bwd.argtypes = [DP] + [P] * 7 + [Z, P]
+            L.ssm_dtproj_bwd.restype = I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -424,4 +435,47 @@ def ssm_pdssm_bwd(scores, dictionary, d, h, sel, g, tau=1.0, h0=None, out=None, 
                                _p(out["dscores"]), _p(out.get("dh0")), _p(ws),
                                ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_pdssm_bwd")
+    return out
+
+
+def dtproj_shape(rows, dim, rank, io=SSM_BF16):
+    return SsmDtShape(int(rows), int(dim), int(rank), int(io))
+
+
+def dtproj_workspace_bytes(shape: SsmDtShape) -> int:
+    return int(lib().ssm_dtproj_workspace_bytes(ctypes.byref(shape)))
+
+
+def ssm_dtproj_fwd(u, w, bias=None, delta_raw=None, stream=None):
+    """Step-size projection delta_raw = u w^T + bias.  u [..., R] and w [D, R] bf16, bias [D] fp32
+    (or None).  Returns delta_raw [..., D] bf16."""
+    _need_cuda(u, w, bias)
+    R = u.shape[-1]
+    D = w.shape[0]
+    M = u.numel() // R if R else 0
+    shape = dtproj_shape(M, D, R, _io_of(u))
+    if delta_raw is None:
+        delta_raw = torch.empty((*u.shape[:-1], D), dtype=u.dtype, device=u.device)
+    code = lib().ssm_dtproj_fwd(ctypes.byref(shape), _p(u), _p(w), _p(bias), _p(delta_raw),
+                                _stream(stream))
+    _check(code, "ssm_dtproj_fwd")
+    return delta_raw
+
+
+def ssm_dtproj_bwd(u, w, g, want_dbias=True, out=None, ws=None, stream=None):
+    """Backward of the projection for g = dL/d delta_raw [..., D] bf16.  Returns dict du [..., R]
+    bf16, dw [D, R] fp32, dbias [D] fp32 (None if not wanted)."""
+    _need_cuda(u, w, g)
+    R = u.shape[-1]
+    D = w.shape[0]
+    M = u.numel() // R if R else 0
+    shape = dtproj_shape(M, D, R, _io_of(u))
+    if out is None:
+        out = dict(du=torch.empty_like(u), dw=torch.empty((D, R), dtype=torch.float32, device=u.device),
+                   dbias=torch.empty(D, dtype=torch.float32, device=u.device) if want_dbias else None)
+    ws = _workspace(dtproj_workspace_bytes(shape), u.device, ws)
+    code = lib().ssm_dtproj_bwd(ctypes.byref(shape), _p(u), _p(w), _p(g), _p(out["du"]),
+                                _p(out["dw"]), _p(out.get("dbias")), _p(ws),
+                                ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_dtproj_bwd")
     return out

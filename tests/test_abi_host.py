@@ -245,3 +245,23 @@ def test_kernel_launch_counts(S):
     assert S.pdssm_kernel_launches(wide, False) == 2 and S.pdssm_kernel_launches(wide, True) == 2
     assert S.pdssm_kernel_launches(S.pdssm_shape(2, 0, 8, 16, 8), False) == 0
     assert S.pdssm_kernel_launches(S.pdssm_shape(2, 8, 8, 12, 8), False) == -1
+
+
+def test_dtproj_validation(S):
+    import ctypes
+    L = S.lib()
+    ok = S.dtproj_shape(1000, 1536, 48)
+    assert S.dtproj_workspace_bytes(ok) == 2 * 1536 * 49 * 4  # two splits of 512 rows, R + 1 columns
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1536, 40)) == 0   # R not a multiple of 16
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1532, 48)) == 0   # D not a multiple of 8
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 64, 272)) == 0    # R > 256
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 64, 16, S.SSM_F32)) == 0
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(0, 64, 16)) == 256
+    p16 = [ctypes.c_void_p(4096)] * 4
+    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 16, S.SSM_F32)), *p16, None) == 2
+    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 40)), *p16, None) == 2
+    assert L.ssm_dtproj_fwd(ctypes.byref(ok), None, *p16[:3], None) == 1       # u missing
+    odd = [ctypes.c_void_p(4096), ctypes.c_void_p(4104), ctypes.c_void_p(4096), None]
+    assert L.ssm_dtproj_fwd(ctypes.byref(ok), *odd, None) == 3                 # w misaligned
+    pb = [ctypes.c_void_p(4096)] * 7
+    assert L.ssm_dtproj_bwd(ctypes.byref(ok), *pb, 255, None) == 4             # workspace
