@@ -51,6 +51,9 @@ def parse():
                          "accumulates dlambda, domega online) instead of fwd + bwd")
     ap.add_argument("--state", action="store_true",
                     help="pass an initial state h0 and an upstream final-state gradient dhL")
+    ap.add_argument("--dtproj", type=int, default=0, metavar="R",
+                    help="bf16 real workloads: compute delta_raw every step with the rank-R step-size "
+                         "projection (ssm_dtproj_fwd) and its gradient (ssm_dtproj_bwd)")
     ap.add_argument("--memory-curve", action="store_true",
                     help="peak device memory of fwd+bwd vs L for the stiff workload's shape")
     return ap.parse_args()
@@ -99,6 +102,16 @@ def algorithmic_bytes(w):
     fwd = 3 * E * s + 2 * BLN * s + ck           # x, delta_raw in; y out; Bm, Cm in; ckpt out
     bwd = 5 * E * s + 4 * BLN * s + ck           # x, delta_raw, dy in; dx, ddelta_raw out;
     return fwd, bwd                              # Bm, Cm in; dB, dC out; ckpt in
+
+
+def dtproj_algorithmic(w, R):
+    """Minimum bytes of the step-size projection's forward (u, w read, bias read, delta_raw
+    written; bf16 except the fp32 bias) and backward (g = ddelta_raw read once, u and w read, du
+    written bf16, dw and dbias written fp32), and the FLOPs of one of its GEMMs (2 M D R)."""
+    M, D = w.batch * w.seqlen, w.dim
+    fwd = 2 * M * R + 2 * D * R + 4 * D + 2 * M * D
+    bwd = 2 * M * D + 2 * M * R + 2 * D * R + 2 * M * R + 4 * D * R + 4 * D
+    return fwd, bwd, 2 * M * D * R
 
 
 def e2e_pipelined(torch, dev, stream, host, sets, compute, outputs, steps, world, dist):
@@ -744,7 +757,20 @@ def main():
     host = {k: torch.from_numpy(v).to(dt if k not in ("A_log", "Dskip") else torch.float32)
             for k, v in inp.items()}
     host = {k: v.pin_memory() for k, v in host.items()}
+    R = args.dtproj
+    if R:  # delta_raw comes from the projection of a rank-R input every step
+        if w.io != gen.BF16:
+            raise SystemExit("--dtproj needs a bf16 workload")
+        pin = gen.dtproj_inputs(w.batch, w.seqlen, w.dim, R, seed=100 + rank)
+        del host["delta_raw"]
+        host["u"] = torch.from_numpy(pin["u"]).to(torch.bfloat16).pin_memory()
+        host["w"] = torch.from_numpy(pin["w"]).to(torch.bfloat16).pin_memory()
+        host["bias"] = torch.from_numpy(pin["bias"]).pin_memory()
     d = {k: v.to(dev) for k, v in host.items()}
+    if R:
+        d["delta_raw"] = torch.empty_like(d["x"])
+        dshape = S.dtproj_shape(w.batch * w.seqlen, w.dim, R)
+        wsp = torch.empty(S.dtproj_workspace_bytes(dshape), dtype=torch.uint8, device=dev)
     shape = S.real_shape(w.batch, w.seqlen, w.dim, w.dstate, w.chunk,
                          S.SSM_BF16 if w.io == gen.BF16 else S.SSM_F32, args.seg_chunks)
     nC = -(-w.seqlen // w.chunk)
@@ -768,6 +794,24 @@ def main():
     if use_ex:
         hL = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
         out["dh0"] = torch.empty_like(hL)
+    if R:
+        out["du"] = torch.empty_like(d["u"])
+        out["dw"] = torch.empty((w.dim, R), dtype=torch.float32, device=dev)
+        out["dbias"] = torch.empty(w.dim, dtype=torch.float32, device=dev)
+        gbuf = torch.empty(w.dim * w.dstate + w.dim + w.dim * (R + 1), dtype=torch.float32, device=dev)
+
+    def proj_fwd(dd=None):
+        dd = d if dd is None else dd
+        if R:
+            S.ssm_dtproj_fwd(dd["u"], dd["w"], dd["bias"], delta_raw=dd["delta_raw"], stream=stream)
+
+    def proj_bwd(dd=None, oo=None):
+        dd = d if dd is None else dd
+        oo = out if oo is None else oo
+        if R:
+            S.ssm_dtproj_bwd(dd["u"], dd["w"], oo["ddelta_raw"],
+                             out=dict(du=oo["du"], dw=oo["dw"], dbias=oo["dbias"]), ws=wsp,
+                             stream=stream)
 
     def fwd():
         if use_ex:
@@ -789,17 +833,27 @@ def main():
                            d["dy"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
                            stream=stream)
 
-    def allreduce():
+    def allreduce(oo=None):
+        oo = out if oo is None else oo
         if world > 1:
-            dp.allreduce_param_grads(out["dA_log"], out["dD"], buf=gbuf)
+            if R:  # the projection's parameter gradients travel in the same collective
+                n1, n2 = w.dim * w.dstate + w.dim, w.dim * R
+                gbuf[n1:n1 + n2].copy_(oo["dw"].reshape(-1))
+                gbuf[n1 + n2:].copy_(oo["dbias"])
+                dp.allreduce_param_grads(oo["dA_log"], oo["dD"], buf=gbuf[:n1])
+                dist.all_reduce(gbuf[n1:])
+                oo["dw"].copy_(gbuf[n1:n1 + n2].view_as(oo["dw"]))
+                oo["dbias"].copy_(gbuf[n1 + n2:])
+            else:
+                dp.allreduce_param_grads(oo["dA_log"], oo["dD"], buf=gbuf)
 
     for _ in range(max(3, args.warmup)):
-        fwd(); bwd(); allreduce()
+        proj_fwd(); fwd(); bwd(); proj_bwd(); allreduce()
     torch.cuda.synchronize()
     if S.ssm_scan_status(wsb) != 0 or S.ssm_scan_status(wsf) != 0:
         raise SystemExit("device status word reports a non-finite state")
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -808,19 +862,22 @@ def main():
     for k in range(args.steps):
         flush.zero_()
         e = ev[k]
-        e[0].record(stream); fwd(); e[1].record(stream); bwd(); e[2].record(stream)
-        allreduce(); e[3].record(stream)
+        e[0].record(stream); proj_fwd(); e[1].record(stream); fwd(); e[2].record(stream)
+        bwd(); e[3].record(stream); proj_bwd(); e[4].record(stream)
+        allreduce(); e[5].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / 1e3
-    tt = torch.tensor([t_step, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+    t_pf = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_fwd = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_bwd = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_pb = sum(e[3].elapsed_time(e[4]) for e in ev) / 1e3
+    t_step = sum(e[0].elapsed_time(e[5]) for e in ev) / 1e3
+    tt = torch.tensor([t_step, t_fwd, t_bwd, t_pf, t_pb], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t_step, t_fwd, t_bwd = tt.tolist()
+    t_step, t_fwd, t_bwd, t_pf, t_pb = tt.tolist()
 
     # end to end: every step's inputs come from pinned host memory and every output goes back,
     # inside the timed region (two buffer sets: one step's copies run beside the next's compute)
@@ -829,6 +886,7 @@ def main():
                      ckpt=torch.empty_like(ckpt), out={k: torch.empty_like(v) for k, v in out.items()}))
 
     def compute(bs):
+        proj_fwd(bs["d"])
         if use_ex:
             S.ssm_scan_fwd_ex(bs["d"]["x"], bs["d"]["delta_raw"], bs["d"]["A_log"], bs["d"]["Bm"],
                               bs["d"]["Cm"], bs["d"]["Dskip"], zoh=args.zoh, h0=h0, chunk=w.chunk,
@@ -847,8 +905,8 @@ def main():
                            bs["d"]["Cm"], bs["d"]["Dskip"], bs["ckpt"], bs["d"]["dy"],
                            chunk=w.chunk, seg_chunks=args.seg_chunks, out=bs["out"], ws=wsb,
                            stream=stream)
-        if world > 1:
-            dp.allreduce_param_grads(bs["out"]["dA_log"], bs["out"]["dD"], buf=gbuf)
+        proj_bwd(bs["d"], bs["out"])
+        allreduce(bs["out"])
 
     t_e2e, h2d, d2h = e2e_pipelined(torch, dev, stream, host, sets, compute,
                                     lambda bs: dict(y=bs["y"], **bs["out"]), args.steps, world, dist)
@@ -857,7 +915,8 @@ def main():
     value = world * upd_rank * args.steps / t_step
     hbm, peak_kind = peaks()
     fb, bb = algorithmic_bytes(w)
-    launches = (S.kernel_launches(shape, False) + S.kernel_launches(shape, True)) * args.steps
+    launches = (S.kernel_launches(shape, False) + S.kernel_launches(shape, True) +
+                (4 if R else 0)) * args.steps
     bwd_gbs = bb / (t_bwd / args.steps) / 1e9
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
     step_gbs = (fb + bb) / ((t_fwd + t_bwd) / args.steps) / 1e9
@@ -901,6 +960,17 @@ def main():
             "gpu_launches": launches,
             "clocks": clk,
         }
+        if R:
+            line["config"]["dt_rank"] = R
+            pfb, pbb, pfl = dtproj_algorithmic(w, R)
+            line["dtproj"] = {
+                "rank": R, "ms_fwd": 1e3 * t_pf / args.steps, "ms_bwd": 1e3 * t_pb / args.steps,
+                "algorithmic_bytes_fwd": pfb, "algorithmic_bytes_bwd": pbb, "flop_per_gemm": pfl,
+                "hbm_frac_fwd": pfb / (t_pf / args.steps) / 1e9 / hbm,
+                "hbm_frac_bwd": pbb / (t_pb / args.steps) / 1e9 / hbm,
+                "tensor_tflops_fwd": pfl / (t_pf / args.steps) / 1e12,
+                "tensor_tflops_bwd": 2 * pfl / (t_pb / args.steps) / 1e12,
+                "note": "bf16 mma.sync GEMMs; ms_per_step and value include both projections"}
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = oracle_sample(w, inp, zoh=args.zoh)
         print(json.dumps(line), flush=True)

@@ -20,7 +20,6 @@ namespace ssm {
 namespace {
 
 constexpr int GT = 256;  // threads per CTA (8 warps)
-constexpr int BK = 32;   // k per pipeline stage
 constexpr int PAD = 8;   // bf16 padding per shared row (16 bytes: ldmatrix rows hit distinct banks)
 
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
@@ -64,19 +63,34 @@ struct GemmArgs {
     const float* bias;
 };
 
+// Shared-memory bytes of one configuration: a STAGES-deep ring of A and B tiles, reused for the
+// bf16 output tile after the main loop.
+template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int EPI>
+struct GemmSmem {
+    static constexpr int SA = AT ? BM + PAD : BK + PAD;  // shared row lengths (bf16)
+    static constexpr int SB = BT ? BN + PAD : BK + PAD;
+    static constexpr int A_ELEMS = AT ? BK * SA : BM * SA;
+    static constexpr int B_ELEMS = BT ? BK * SB : BN * SB;
+    static constexpr int SC = BN + PAD;  // bf16 output tile staged for 16-byte row stores
+    static constexpr int PIPE_BYTES = STAGES * (A_ELEMS + B_ELEMS) * 2;
+    static constexpr int C_BYTES = EPI == EPI_F32_PART ? 0 : BM * SC * 2;
+    static constexpr int BYTES = PIPE_BYTES > C_BYTES ? PIPE_BYTES : C_BYTES;
+};
+
 // C tile [BM x BN] of blockIdx (y: m, x: n, z: k split).  Warps WM x WN, warp tile
-// (BM/WM) x (BN/WN) of m16 x n8 mma tiles.
-template <bool AT, bool BT, int BM, int BN, int WM, int WN, int EPI>
+// (BM/WM) x (BN/WN) of m16 x n8 mma tiles; k in steps of BK through a STAGES-deep cp.async ring.
+template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int WM, int WN, int EPI>
 __global__ void __launch_bounds__(GT) dtp_gemm_kernel(GemmArgs p) {
     static_assert(WM * WN * 32 == GT, "eight warps");
+    static_assert(BK % 16 == 0 && STAGES >= 2, "k steps of whole mma blocks");
     constexpr int TM = BM / WM, TN = BN / WN, MT = TM / 16, NT8 = TN / 8;
     static_assert(TM % 16 == 0 && TN % 16 == 0, "warp tile of whole m16 x n16 blocks");
-    constexpr int SA = AT ? BM + PAD : BK + PAD;       // shared row lengths (bf16)
-    constexpr int SB = BT ? BN + PAD : BK + PAD;
-    constexpr int A_ELEMS = AT ? BK * SA : BM * SA;
-    constexpr int B_ELEMS = BT ? BK * SB : BN * SB;
-    __shared__ __align__(16) __nv_bfloat16 sA[2][A_ELEMS];
-    __shared__ __align__(16) __nv_bfloat16 sB[2][B_ELEMS];
+    using Sm = GemmSmem<AT, BT, BM, BN, BK, STAGES, EPI>;
+    constexpr int SA = Sm::SA, SB = Sm::SB, A_ELEMS = Sm::A_ELEMS, B_ELEMS = Sm::B_ELEMS, SC = Sm::SC;
+    extern __shared__ __align__(16) unsigned char smem[];
+    __nv_bfloat16 (*sA)[A_ELEMS] = reinterpret_cast<__nv_bfloat16 (*)[A_ELEMS]>(smem);
+    __nv_bfloat16 (*sB)[B_ELEMS] =
+        reinterpret_cast<__nv_bfloat16 (*)[B_ELEMS]>(smem + STAGES * A_ELEMS * 2);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wm = warp / WN, wn = warp % WN;
@@ -130,6 +144,16 @@ __global__ void __launch_bounds__(GT) dtp_gemm_kernel(GemmArgs p) {
         asm volatile("cp.async.commit_group;\n" ::);
     };
 
+    const int g = lane >> 2, t4 = lane & 3;
+    float bias_r[NT8][2];  // the bias of this thread's output columns, fetched before the main loop
+#pragma unroll
+    for (int jn = 0; jn < NT8; ++jn) {
+        const int64_t col = n0 + wn * TN + 8 * jn + 2 * t4;
+        const bool on = EPI == EPI_BIAS_BF16 && p.bias != nullptr && col < p.N;
+        bias_r[jn][0] = on ? p.bias[col] : 0.0f;
+        bias_r[jn][1] = on ? p.bias[col + 1] : 0.0f;
+    }
+
     float acc[MT][NT8][4];
 #pragma unroll
     for (int i = 0; i < MT; ++i)
@@ -138,16 +162,26 @@ __global__ void __launch_bounds__(GT) dtp_gemm_kernel(GemmArgs p) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
 
-    if (nk > 0) load(0, kb);
+    // ring: STAGES - 1 tiles in flight ahead of the one being multiplied (empty groups past the
+    // end keep the group count uniform)
+#pragma unroll
+    for (int s0 = 0; s0 < STAGES - 1; ++s0) {
+        if (s0 < nk)
+            load(s0, kb + (int64_t)s0 * BK);
+        else
+            asm volatile("cp.async.commit_group;\n" ::);
+    }
     for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt & 1;
-        if (kt + 1 < nk) {
-            load(st ^ 1, kb + (int64_t)(kt + 1) * BK);
-            asm volatile("cp.async.wait_group 1;\n" ::);
-        } else {
-            asm volatile("cp.async.wait_group 0;\n" ::);
+        const int st = kt % STAGES;
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(STAGES - 2));
+        __syncthreads();  // tile kt is in; every thread is done with tile kt - 1
+        {
+            const int kn = kt + STAGES - 1;
+            if (kn < nk)
+                load(kn % STAGES, kb + (int64_t)kn * BK);
+            else
+                asm volatile("cp.async.commit_group;\n" ::);
         }
-        __syncthreads();
         const __nv_bfloat16* a = sA[st];
         const __nv_bfloat16* b = sB[st];
 #pragma unroll
@@ -178,40 +212,53 @@ __global__ void __launch_bounds__(GT) dtp_gemm_kernel(GemmArgs p) {
                 }
             }
         }
-        __syncthreads();  // stage st is free again
     }
+    __syncthreads();  // every thread is done with the ring (the output tile reuses it)
 
     // epilogue: c0, c1 at (row g, cols 2t, 2t+1), c2, c3 at row g + 8
-    const int g = lane >> 2, t4 = lane & 3;
+    if (EPI == EPI_F32_PART) {
 #pragma unroll
-    for (int i = 0; i < MT; ++i) {
+        for (int i = 0; i < MT; ++i)
 #pragma unroll
-        for (int jn = 0; jn < NT8; ++jn) {
-            const int64_t col = n0 + wn * TN + 8 * jn + 2 * t4;
+            for (int jn = 0; jn < NT8; ++jn) {
+                const int64_t col = n0 + wn * TN + 8 * jn + 2 * t4;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t row = m0 + wm * TM + 16 * i + g + 8 * h;
-                float v0 = acc[i][jn][2 * h], v1 = acc[i][jn][2 * h + 1];
-                if (row >= p.M || col >= p.N) continue;
-                if (EPI == EPI_F32_PART) {
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t row = m0 + wm * TM + 16 * i + g + 8 * h;
+                    if (row >= p.M || col >= p.N) continue;
                     float* c = static_cast<float*>(p.C) + (int64_t)blockIdx.z * p.M * p.ldc + row * p.ldc;
-                    c[col] = v0;
-                    if (col + 1 < p.N) c[col + 1] = v1;
-                } else {
-                    if (EPI == EPI_BIAS_BF16 && p.bias) {
-                        v0 += p.bias[col];
-                        v1 += p.bias[col + 1];
-                    }
-                    // N is a multiple of 8 for these outputs, so col + 1 < N
-                    *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col) =
-                        __floats2bfloat162_rn(v0, v1);
+                    c[col] = acc[i][jn][2 * h];
+                    if (col + 1 < p.N) c[col + 1] = acc[i][jn][2 * h + 1];
                 }
             }
+        return;
+    }
+    // bf16 outputs (N a multiple of 8): the tile goes through shared memory (the pipeline buffers
+    // are free after the last barrier) and leaves as 16-byte row pieces
+    __nv_bfloat16* sC = reinterpret_cast<__nv_bfloat16*>(smem);
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int jn = 0; jn < NT8; ++jn) {
+            const int cl = wn * TN + 8 * jn + 2 * t4;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int rl = wm * TM + 16 * i + g + 8 * h;
+                *reinterpret_cast<__nv_bfloat162*>(sC + rl * SC + cl) = __floats2bfloat162_rn(
+                    acc[i][jn][2 * h] + bias_r[jn][0], acc[i][jn][2 * h + 1] + bias_r[jn][1]);
+            }
         }
+    __syncthreads();
+    for (int q = tid; q < BM * (BN / 8); q += GT) {
+        const int rl = q / (BN / 8), c8 = q % (BN / 8);
+        const int64_t row = m0 + rl, col = n0 + 8 * c8;
+        if (row < p.M && col < p.N)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col) =
+                *reinterpret_cast<const uint4*>(sC + rl * SC + 8 * c8);
     }
 }
 
-// dw[d, r] = sum_s part[s, d, r] (r < R), dbias[d] = sum_s part[s, d, R], in split order.
+// dw[d, r] = sum_s part[s, d, r] (r < R), dbias[d] = sum_s part[s, d, R], in a fixed order.
 __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, int64_t D, int R,
                                   float* __restrict__ dw, float* __restrict__ dbias) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -219,24 +266,39 @@ __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, in
     if (i >= n) return;
     const int64_t d = i / (R + 1);
     const int r = (int)(i - d * (R + 1));
-    float s = 0.0f;
-    for (int k = 0; k < splits; ++k) s += part[(int64_t)k * n + i];
+    // four interleaved running sums (independent loads in flight), combined in a fixed order
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    int k = 0;
+    for (; k + 4 <= splits; k += 4) {
+        s0 += part[(int64_t)k * n + i];
+        s1 += part[(int64_t)(k + 1) * n + i];
+        s2 += part[(int64_t)(k + 2) * n + i];
+        s3 += part[(int64_t)(k + 3) * n + i];
+    }
+    for (; k < splits; ++k) s0 += part[(int64_t)k * n + i];
+    const float s = (s0 + s1) + (s2 + s3);
     if (r < R)
         dw[d * R + r] = s;
     else if (dbias)
         dbias[d] = s;
 }
 
-template <bool AT, bool BT, int BM, int BN, int WM, int WN, int EPI>
+template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int WM, int WN, int EPI>
 cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
     const dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + BM - 1) / BM), (unsigned)splits);
-    dtp_gemm_kernel<AT, BT, BM, BN, WM, WN, EPI><<<grid, GT, 0, st>>>(a);
+    constexpr int bytes = GemmSmem<AT, BT, BM, BN, BK, STAGES, EPI>::BYTES;
+    auto kern = dtp_gemm_kernel<AT, BT, BM, BN, BK, STAGES, WM, WN, EPI>;
+    if (bytes > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<grid, GT, bytes, st>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int64_t dtproj_rows_per_split() { return 512; }
+int64_t dtproj_rows_per_split() { return 256; }
 
 cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     GemmArgs a = {};
@@ -247,7 +309,7 @@ cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     a.ones_col = -1;
     a.C = d.delta_raw;
     a.bias = d.bias;
-    return run_gemm<false, false, 128, 128, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    return run_gemm<false, false, 64, 128, 32, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
 }
 
 cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
@@ -259,7 +321,7 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     a.M = d.M; a.N = d.R; a.K = d.D; a.kchunk = d.D;
     a.ones_col = -1;
     a.C = d.du;
-    cudaError_t e = run_gemm<false, true, 128, 64, 4, 2, EPI_BF16>(a, 1, st);
+    cudaError_t e = run_gemm<false, true, 64, 64, 64, 4, 4, 2, EPI_BF16>(a, 1, st);
     if (e != cudaSuccess) return e;
     // partials [split][D][R+1] = g^T [D x M] . (u | 1) [M x (R+1)]   (A stored [k = m][d], B [m][r])
     GemmArgs b = {};
@@ -269,7 +331,7 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     b.M = d.D; b.N = d.R + 1; b.K = d.M; b.kchunk = dtproj_rows_per_split();
     b.ones_col = d.R;
     b.C = d.part;
-    e = run_gemm<true, true, 128, 64, 4, 2, EPI_F32_PART>(b, d.splits, st);
+    e = run_gemm<true, true, 128, 64, 32, 3, 4, 2, EPI_F32_PART>(b, d.splits, st);
     if (e != cudaSuccess) return e;
     const int64_t n = d.D * (d.R + 1);
     dtp_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(d.part, d.splits, d.D, d.R, d.dw,
