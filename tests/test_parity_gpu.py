@@ -222,6 +222,18 @@ def test_complex_shapes(S, oracle_mod, B, L, K, T, sc):
     check_complex(got, ref)
 
 
+def test_complex_far_phases(S, oracle_mod):
+    """Phases |omega phi| beyond the pi/2 reduction's range (~6400) take the library sine/cosine,
+    warp-uniformly, inside the producers' packed transitions; the rest of the tile keeps the
+    series.  Forward and backward against the oracle, with and without time segments."""
+    c = gen.complex_inputs(2, 260, 130, seed=11)
+    c["phi"][0, 40:52] = np.linspace(-7000.0, 9000.0, 12, dtype=np.float32)
+    c["phi"][1, 200] = 12345.0
+    ref = oracle_mod.complex_(c["u"], c["r"], c["phi"], c["lam"], c["omega"], c["g"])
+    for sc in (0, 1):
+        check_complex(run_complex(S, c, 64, sc), ref)
+
+
 # ------------------------------------------------------------------------------ full-size workloads
 
 def _channel_sample(D, n=24):

@@ -106,3 +106,15 @@ def test_rtrl_empty_sequence(S):
     torch.cuda.synchronize()
     assert not got["dlambda"].any() and not got["domega"].any()
     assert torch.equal(state, before)
+
+
+def test_rtrl_far_phases(S, oracle_mod):
+    """Phases beyond the pi/2 reduction's range go through the library sine/cosine."""
+    c = gen.complex_inputs(2, 150, 64, seed=12)
+    c["phi"][0, 10:20] = np.linspace(-8000.0, 8000.0, 10, dtype=np.float32)
+    d = dev(c)
+    got = S.ssm_scan_complex_rtrl(d["u"], d["r"], d["phi"], d["lam"], d["omega"], d["g"])
+    torch.cuda.synchronize()
+    ref = oracle_mod.complex_rtrl(c["u"], c["r"], c["phi"], c["lam"], c["omega"], c["g"])
+    for k in ("dlambda", "domega"):
+        assert rel(got[k].cpu().numpy(), ref[k]) <= GRAD_TOL, k
