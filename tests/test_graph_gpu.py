@@ -1,5 +1,6 @@
-"""The scan calls can be captured in a CUDA graph: a captured forward + backward replayed on new
-inputs (copied into the captured buffers) gives bitwise the outputs of eager calls."""
+"""The library's calls can be captured in a CUDA graph: a captured forward + backward (real mode;
+complex mode; Flash PD-SSM; the step-size projection) replayed on new inputs copied into the
+captured buffers gives bitwise the outputs of eager calls."""
 
 import numpy as np
 import pytest
@@ -65,3 +66,91 @@ def test_captured_fwd_bwd_replays_bitwise(S):
     for k, v in ref.items():
         assert torch.equal(got[k], v), k
     assert S.ssm_scan_status(wsb) == 0
+
+
+def _capture_and_replay(step, bufs, fresh):
+    """Warm up `step` eagerly, capture it, copy `fresh` into the captured input buffers `bufs`,
+    replay; returns nothing (the outputs live in the captured buffers)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for k in bufs:
+        bufs[k].copy_(fresh[k])
+    g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
+def test_captured_complex_and_pdssm_and_projection_replay_bitwise(S):
+    # complex mode (warp-specialised kernels with named barriers)
+    c1, c2 = gen.complex_inputs(2, 300, 128, seed=1), gen.complex_inputs(2, 300, 128, seed=2)
+    a = {k: torch.from_numpy(v).cuda() for k, v in c1.items()}
+    h = torch.empty_like(a["u"])
+    outc = dict(du=torch.empty_like(a["g"]), dr=torch.empty_like(a["r"]), dphi=torch.empty_like(a["phi"]),
+                dlambda=torch.empty_like(a["lam"]), domega=torch.empty_like(a["omega"]))
+
+    def cstep():
+        S.ssm_scan_complex_fwd(a["u"], a["r"], a["phi"], a["lam"], a["omega"], h=h)
+        S.ssm_scan_complex_bwd(h, a["r"], a["phi"], a["lam"], a["omega"], a["g"], out=outc)
+
+    _capture_and_replay(cstep, a, {k: torch.from_numpy(v).cuda() for k, v in c2.items()})
+    got = {"h": h.clone(), **{k: v.clone() for k, v in outc.items()}}
+    b = {k: torch.from_numpy(v).cuda() for k, v in c2.items()}
+    h2 = S.ssm_scan_complex_fwd(b["u"], b["r"], b["phi"], b["lam"], b["omega"])
+    o2 = S.ssm_scan_complex_bwd(h2, b["r"], b["phi"], b["lam"], b["omega"], b["g"])
+    torch.cuda.synchronize()
+    assert torch.equal(got["h"], h2)
+    for k in o2:
+        assert torch.equal(got[k], o2[k]), k
+
+    # Flash PD-SSM (fused argmax / score gradient, warp-specialised backward)
+    p1, p2 = gen.pdssm_inputs(2, 400, 32, 16, 8, seed=1), gen.pdssm_inputs(2, 400, 32, 16, 8, seed=2)
+    q = {k: torch.from_numpy(v).cuda() for k, v in p1.items()}
+    hp = torch.empty_like(q["d"])
+    sel = torch.empty(q["scores"].shape[:3], dtype=torch.int32, device="cuda")
+    outp = dict(dd=torch.empty_like(q["d"]), dbt=torch.empty_like(q["d"]),
+                dscores=torch.empty_like(q["scores"]), dh0=torch.empty_like(q["h0"]))
+
+    def pstep():
+        S.ssm_pdssm_fwd(q["scores"], q["dictionary"], q["d"], q["bt"], h0=q["h0"], h=hp, sel=sel)
+        S.ssm_pdssm_bwd(q["scores"], q["dictionary"], q["d"], hp, sel, q["g"], tau=0.5, h0=q["h0"],
+                        out=outp)
+
+    _capture_and_replay(pstep, q, {k: torch.from_numpy(v).cuda() for k, v in p2.items()})
+    got = {"h": hp.clone(), "sel": sel.clone(), **{k: v.clone() for k, v in outp.items()}}
+    r = {k: torch.from_numpy(v).cuda() for k, v in p2.items()}
+    h3, s3 = S.ssm_pdssm_fwd(r["scores"], r["dictionary"], r["d"], r["bt"], h0=r["h0"])
+    o3 = S.ssm_pdssm_bwd(r["scores"], r["dictionary"], r["d"], h3, s3, r["g"], tau=0.5, h0=r["h0"])
+    torch.cuda.synchronize()
+    assert torch.equal(got["h"], h3) and torch.equal(got["sel"], s3)
+    for k in o3:
+        assert torch.equal(got[k], o3[k]), k
+
+    # step-size projection
+    j1, j2 = gen.dtproj_inputs(2, 700, 256, 48, seed=1), gen.dtproj_inputs(2, 700, 256, 48, seed=2)
+    bfk = ("u", "w", "g")
+    t = {k: torch.from_numpy(v).cuda().to(torch.bfloat16 if k in bfk else torch.float32)
+         for k, v in j1.items()}
+    dr = torch.empty((2, 700, 256), dtype=torch.bfloat16, device="cuda")
+    outj = dict(du=torch.empty_like(t["u"]), dw=torch.empty((256, 48), device="cuda"),
+                dbias=torch.empty(256, device="cuda"))
+
+    def jstep():
+        S.ssm_dtproj_fwd(t["u"], t["w"], t["bias"], delta_raw=dr)
+        S.ssm_dtproj_bwd(t["u"], t["w"], t["g"], out=outj)
+
+    _capture_and_replay(jstep, t, {k: torch.from_numpy(v).cuda().to(torch.bfloat16 if k in bfk else torch.float32)
+                                   for k, v in j2.items()})
+    got = {"dr": dr.clone(), **{k: v.clone() for k, v in outj.items()}}
+    u = {k: torch.from_numpy(v).cuda().to(torch.bfloat16 if k in bfk else torch.float32) for k, v in j2.items()}
+    dr2 = S.ssm_dtproj_fwd(u["u"], u["w"], u["bias"])
+    o4 = S.ssm_dtproj_bwd(u["u"], u["w"], u["g"])
+    torch.cuda.synchronize()
+    assert torch.equal(got["dr"], dr2)
+    for k in o4:
+        assert torch.equal(got[k], o4[k]), k
