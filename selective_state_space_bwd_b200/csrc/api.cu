@@ -10,6 +10,13 @@ namespace {
 
 constexpr size_t kStatusBytes = 256;
 constexpr int kTargetCtas = 296;  // 2 x 148 SMs: below this many CTAs, split time into segments
+// Real forward, once split: enough segments for about 2368 CTAs (two waves at the eight CTAs per
+// SM its registers and shared memory allow), so that every SM keeps several CTAs busy.
+constexpr int64_t kRealFwdSplitCtas = 2368;
+// Real backward: 3 CTAs per SM (registers and shared memory) on 148 SMs
+constexpr int64_t kRealBwdSlots = 444;
+// Real backward: per-launch bound on the per-CTA scratch (window-start states, (delta, sigma))
+constexpr size_t kRealBwdScratchCap = (size_t)192 << 20;
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -17,7 +24,9 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 bool valid_chunk(int T) { return T == 16 || T == 32 || T == 64 || T == 128 || T == 256; }
 
-int pick_segments(int64_t ctas_per_seg, int nC, int forced, int* seg_chunks) {
+// Time segments of a forward: none when ctas_per_seg reaches kTargetCtas, else enough for about
+// `split_ctas` CTAs in all.
+int pick_segments(int64_t ctas_per_seg, int nC, int forced, int64_t split_ctas, int* seg_chunks) {
     if (nC <= 0) {
         *seg_chunks = 1;
         return 1;
@@ -27,7 +36,7 @@ int pick_segments(int64_t ctas_per_seg, int nC, int forced, int* seg_chunks) {
         sc = forced < nC ? forced : nC;
     } else {
         int64_t nseg = 1;
-        if (ctas_per_seg < kTargetCtas) nseg = (kTargetCtas + ctas_per_seg - 1) / ctas_per_seg;
+        if (ctas_per_seg < kTargetCtas) nseg = (split_ctas + ctas_per_seg - 1) / ctas_per_seg;
         if (nseg > nC) nseg = nC;
         sc = (int)((nC + nseg - 1) / nseg);
     }
@@ -42,7 +51,7 @@ struct RealPlan {
     int b_nseg, b_seg_chunks, b_seq, b_group, b_rows, b_launches;
     // workspace offsets (bytes); fwd and bwd use separate layouts
     size_t f_sumP, f_sumS, f_hin, f_end;
-    size_t b_gP, b_gG, b_vin, b_part, b_dA, b_dD, b_bnd, b_end;
+    size_t b_gP, b_gG, b_part, b_dA, b_dD, b_bnd, b_end;
 };
 
 int plan_real(const ssm_shape* s, RealPlan* p) {
@@ -65,7 +74,8 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->nC = (p->L + p->T - 1) / p->T;
     const int DT = ssm::real_dt(p->N);
     p->ndt = (p->D + DT - 1) / DT;
-    p->nseg = pick_segments((int64_t)p->B * p->ndt, p->nC, s->seg_chunks, &p->seg_chunks);
+    p->nseg = pick_segments((int64_t)p->B * p->ndt, p->nC, s->seg_chunks, kRealFwdSplitCtas,
+                            &p->seg_chunks);
     if (p->nseg > 65535) return SSM_ERR_UNSUPPORTED;
 
     const size_t B = p->B, DN = (size_t)p->D * p->N, S = p->nseg;
@@ -86,15 +96,27 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     const size_t chunks_cap = per_chunk > 0 ? cap / per_chunk : (size_t)p->nC;  // per launch
     const int nC1 = p->nC > 0 ? p->nC : 1;
     auto clampi = [](size_t v, size_t lo, size_t hi) { return (int)(v < lo ? lo : (v > hi ? hi : v)); };
+    // CTAs per launch are bounded by the scratch cap as well as by the partial-sum cap
+    const size_t scr_cta = ssm::real_bwd_scratch_floats(p->N, p->T) * 4;
+    const int64_t ctas_cap = scr_cta > 0 ? (int64_t)(kRealBwdScratchCap / scr_cta) : ctas_per_seg;
+    const size_t segs_cap = (size_t)(ctas_cap / ctas_per_seg > 1 ? ctas_cap / ctas_per_seg : 1);
+    // one wave of CTAs (kTargetCtas..kRealBwdSlots), or several waves that fill the SMs to at
+    // least 80 %: no time split.  Otherwise (too few CTAs, or a partial last wave that would
+    // leave most SMs idle) concurrent segments of at most 4 chunks, each launch holding as many
+    // segments as the caps allow.
+    const int64_t waves = (ctas_per_seg + kRealBwdSlots - 1) / kRealBwdSlots;
+    const bool fill = ctas_per_seg >= kTargetCtas &&
+                      (ctas_per_seg <= kRealBwdSlots || 5 * ctas_per_seg >= 4 * waves * kRealBwdSlots);
     if (s->seg_chunks > 0) {
-        // forced time split: concurrent segments, as many per launch as the cap allows
+        // forced time split: concurrent segments, as many per launch as the caps allow
         p->b_seg_chunks = s->seg_chunks < nC1 ? s->seg_chunks : nC1;
         p->b_nseg = (nC1 + p->b_seg_chunks - 1) / p->b_seg_chunks;
         p->b_seq = 0;
-        p->b_group = clampi(chunks_cap / p->b_seg_chunks, 1, p->b_nseg);
-    } else if (ctas_per_seg >= kTargetCtas || nC1 <= 1) {
-        // enough CTAs without splitting time: one pass, or sequential blocks if the partial sums
-        // of the whole sequence would exceed the cap
+        const size_t g = chunks_cap / p->b_seg_chunks;
+        p->b_group = clampi(g < segs_cap ? g : segs_cap, 1, p->b_nseg);
+    } else if (fill || nC1 <= 1) {
+        // no time split: one pass, or sequential blocks if the partial sums of the whole
+        // sequence would exceed the cap
         if (chunks_cap >= (size_t)nC1) {
             p->b_nseg = 1;
             p->b_seg_chunks = nC1;
@@ -106,13 +128,18 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
         }
         p->b_group = 1;
     } else {
-        // few CTAs: concurrent segments (summary + carry), `g` of them per launch for
-        // parallelism, each short enough that a launch's partial sums fit the cap
-        const int g = (int)((kTargetCtas + ctas_per_seg - 1) / ctas_per_seg);
-        p->b_seg_chunks = clampi(chunks_cap / g, 1, (size_t)((nC1 + g - 1) / g));
+        // concurrent segments of 4 chunks when there are at least 2 x 4 CTA-chunks of work per
+        // CTA slot (the summary pass then stays a small share of the work), shorter for smaller
+        // problems so that more of them run at once; launches of equal size
+        const int64_t work = (int64_t)nC1 * ctas_per_seg / (2 * kRealBwdSlots);
+        p->b_seg_chunks = (int)(work < 1 ? 1 : (work > 4 ? 4 : work));
+        if (p->b_seg_chunks > nC1) p->b_seg_chunks = nC1;
         p->b_nseg = (nC1 + p->b_seg_chunks - 1) / p->b_seg_chunks;
         p->b_seq = 0;
-        p->b_group = g < p->b_nseg ? g : p->b_nseg;
+        const size_t g = chunks_cap / p->b_seg_chunks;
+        const int gmax = clampi(g < segs_cap ? g : segs_cap, 1, p->b_nseg);
+        const int nl = (p->b_nseg + gmax - 1) / gmax;
+        p->b_group = (p->b_nseg + nl - 1) / nl;
     }
     if (p->b_nseg > 65535) return SSM_ERR_UNSUPPORTED;
     const size_t BS = p->b_nseg;
@@ -120,11 +147,12 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->b_launches = (p->b_nseg + per - 1) / per;
     const size_t rows = (size_t)per * p->b_seg_chunks * p->T;
     p->b_rows = (int)(rows < (size_t)p->L ? rows : (size_t)p->L);
-    const size_t bsumm = (BS > 1 && !p->b_seq) ? B * (BS - 1) * DN * 4 : 0;
+    // gG holds the summaries' local adjoints and then, overwritten by the carry, the adjoint
+    // entering each segment but the last (sequential blocks hand it over through gG too)
+    const size_t bvin = BS > 1 ? B * (BS - 1) * DN * 4 : 0;
     o = kStatusBytes;
-    p->b_gP = o;   o = align256(o + bsumm);
-    p->b_gG = o;   o = align256(o + bsumm);
-    p->b_vin = o;  o = align256(o + (BS > 1 ? B * BS * DN * 4 : 0));
+    p->b_gP = o;   o = align256(o + (p->b_seq ? 0 : bvin));
+    p->b_gG = o;   o = align256(o + bvin);
     p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->b_rows * 2 * p->N * 4);
     p->b_dA = o;   o = align256(o + B * BS * DN * 4);
     p->b_dD = o;   o = align256(o + B * BS * (size_t)p->D * 4);
@@ -154,7 +182,7 @@ int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
     p->T = s->chunk;
     p->nC = (p->L + p->T - 1) / p->T;
     p->nkt = (p->K + ssm::kCplxKT - 1) / ssm::kCplxKT;
-    p->nseg = pick_segments((int64_t)p->B * p->nkt, p->nC, s->seg_chunks, &p->seg_chunks);
+    p->nseg = pick_segments((int64_t)p->B * p->nkt, p->nC, s->seg_chunks, kTargetCtas, &p->seg_chunks);
     if (p->nseg > 65535) return SSM_ERR_UNSUPPORTED;
     const size_t B = p->B, K = p->K, S = p->nseg;
     const size_t summ = S > 1 ? B * (S - 1) * K * 8 : 0;
@@ -296,7 +324,7 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const 
     a.seq_blocks = p.b_seq; a.part_rows = p.b_rows;
     a.x = x; a.draw = delta_raw; a.A_log = A_log; a.Bm = Bm; a.Cm = Cm; a.Dskip = Dskip;
     a.ckpt_in = ckpt; a.dy = dy; a.dx = dx; a.ddraw = ddelta_raw;
-    a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.vin = at<float>(ws, p.b_vin);
+    a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.vin = a.gsumG;
     a.dBC_part = at<float>(ws, p.b_part); a.dA_part = at<float>(ws, p.b_dA);
     a.dD_part = at<float>(ws, p.b_dD);
     a.bnd_scratch = at<float>(ws, p.b_bnd);

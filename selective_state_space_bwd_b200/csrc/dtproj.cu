@@ -309,7 +309,13 @@ cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     a.ones_col = -1;
     a.C = d.delta_raw;
     a.bias = d.bias;
-    return run_gemm<false, false, 64, 128, 32, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    // R <= 64: the whole k range in one shared tile (no ring turnover); larger R: 128-row tiles
+    // so each w tile serves twice the rows
+    if (d.R <= 16) return run_gemm<false, false, 64, 128, 16, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    if (d.R <= 32) return run_gemm<false, false, 64, 128, 32, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    if (d.R <= 48) return run_gemm<false, false, 64, 128, 48, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    if (d.R <= 64) return run_gemm<false, false, 64, 128, 64, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    return run_gemm<false, false, 128, 128, 64, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
 }
 
 cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
@@ -321,7 +327,7 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     a.M = d.M; a.N = d.R; a.K = d.D; a.kchunk = d.D;
     a.ones_col = -1;
     a.C = d.du;
-    cudaError_t e = run_gemm<false, true, 64, 64, 64, 4, 4, 2, EPI_BF16>(a, 1, st);
+    cudaError_t e = run_gemm<false, true, 128, 64, 64, 3, 4, 2, EPI_BF16>(a, 1, st);
     if (e != cudaSuccess) return e;
     // partials [split][D][R+1] = g^T [D x M] . (u | 1) [M x (R+1)]   (A stored [k = m][d], B [m][r])
     GemmArgs b = {};

@@ -87,21 +87,19 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(Rea
     }
 }
 
-// Scaled adjoint entering each segment from its end: v_in[nseg-1] = dhL (or 0),
-// v_in[s-1] = G_s + P_s v_in[s].
+// Scaled adjoint entering each segment from its end: v_in[nseg-1] = dhL (or 0, read by the last
+// segment directly), v_in[s-1] = G_s + P_s v_in[s].  v_in[s-1] overwrites G_s in place (slot s-1
+// of the summaries), so the hand-over needs no buffer of its own.
 __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __restrict__ P,
-                                      const float* __restrict__ G, float* __restrict__ vin,
-                                      const float* __restrict__ dhL) {
+                                      float* __restrict__ G, const float* __restrict__ dhL) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)B * DN) return;
     const int b = (int)(i / DN), k = (int)(i % DN);
     float v = dhL ? dhL[i] : 0.0f;
-    for (int s = nseg - 1; s >= 0; --s) {
-        vin[((size_t)b * nseg + s) * DN + k] = v;
-        if (s > 0) {
-            const size_t j = ((size_t)b * (nseg - 1) + (s - 1)) * DN + k;
-            v = fmaf(P[j], v, G[j]);
-        }
+    for (int s = nseg - 1; s > 0; --s) {
+        const size_t j = ((size_t)b * (nseg - 1) + (s - 1)) * DN + k;
+        v = fmaf(P[j], v, G[j]);
+        G[j] = v;
     }
 }
 
@@ -196,7 +194,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
     if (dv) {
         // the adjoint entering from the segment's end: handed over by the carry or by the later
         // block, or, for the last segment, the upstream gradient of the final state (or zero)
-        const float* src = seg < p.nseg - 1 ? p.vin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0
+        const float* src = seg < p.nseg - 1 ? p.vin + (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N + n0
                            : p.dhL          ? p.dhL + ((size_t)b * p.D + d) * N + n0
                                             : nullptr;
         if (src) ld_pairs<4>(v, src);
@@ -504,7 +502,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
         if (ng == 0) p.dD_part[((size_t)b * p.nseg + seg) * p.D + d] = dDacc;
         // sequential blocks: the adjoint leaving this block's start enters the previous block
         if (p.seq_blocks && seg > 0)
-            st_pairs<4>(p.vin + (((size_t)b * p.nseg + (seg - 1)) * p.D + d) * N + n0, v);
+            st_pairs<4>(p.vin + (((size_t)b * (p.nseg - 1) + (seg - 1)) * p.D + d) * N + n0, v);
         // the first segment ends at t = -1: its adjoint a_0 g_0 is the gradient of h0
         if (p.dh0 && seg == 0) st_pairs<4>(p.dh0 + ((size_t)b * p.D + d) * N + n0, v);
         if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
@@ -577,8 +575,7 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
-                                                                            a.gsumP, a.gsumG, a.vin,
-                                                                            a.dhL);
+                                                                            a.gsumP, a.vin, a.dhL);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const size_t sm = BwdSmem<E, N>::BYTES;

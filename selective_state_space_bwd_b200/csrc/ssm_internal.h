@@ -42,7 +42,9 @@ struct RealArgs {
     float* hin;       // state entering each segment [B][nseg][D][N]
     float* gsumP;     // backward segment summaries [B][nseg-1][D][N] (segments 1..nseg-1)
     float* gsumG;
-    float* vin;       // scaled adjoint a_{t+1} g_{t+1} entering each segment from its end
+    float* vin;       // scaled adjoint a_{t+1} g_{t+1} entering segments 0..nseg-2 from their
+                      // ends, [B][nseg-1][D][N]; the same buffer as gsumG (the carry overwrites
+                      // each summary with it); the last segment takes dhL
     float* dBC_part;  // [ndt][B][part_rows][2N] per-CTA sums over its channels (dB then dC),
                       // rows relative to part_t0 (the first step of the current launch)
     float* dA_part;   // [B][nseg][D][N] sum over the segment of delta * q

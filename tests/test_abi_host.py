@@ -60,9 +60,10 @@ def test_checkpoint_and_workspace_sizes(S, B, L, D, N, T):
     fw, bw = S.workspace_bytes(shp, False), S.workspace_bytes(shp, True)
     assert fw >= 256 and bw >= 256 and fw % 256 == 0 and bw % 256 == 0
     # the backward's dB/dC partial sums cover one launch's steps, capped at
-    # max(checkpoint bytes, 128 MiB); the rest of its workspace is per-CTA scratch
+    # max(checkpoint bytes, 128 MiB); its per-CTA scratch is capped at 192 MiB per launch; the
+    # segment summaries take at most as much as the checkpoints
     cap = max(S.checkpoint_bytes(shp), 128 << 20)
-    assert bw <= cap + (160 << 20)
+    assert bw <= 2 * cap + (193 << 20)
 
 
 def test_backward_workspace_is_o_of_l_over_t(S):
@@ -223,13 +224,17 @@ def test_status_null_workspace(S):
 def test_kernel_launch_counts(S):
     one = S.real_shape(8, 2048, 1536, 16, 128, S.SSM_BF16)        # enough CTAs: no time split
     assert S.kernel_launches(one, False) == 1 and S.kernel_launches(one, True) == 3
-    # few CTAs: concurrent segments + carry; the backward uses 40 shorter segments (25 chunks),
-    # 10 per launch (320 CTAs) so that each launch's dB/dC partial sums stay under the cap:
-    # summary + carry + 4 x (main + reduce) + params = 11
+    # few CTAs: concurrent segments + carry; the backward uses 250 segments of 4 chunks, 63 per
+    # launch (2016 CTAs) so that each launch's dB/dC partial sums and scratch stay under their
+    # caps: summary + carry + 4 x (main + reduce) + params = 11
     split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
     assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 11
-    # long and wide: the backward walks time in 4 sequential blocks
-    blocks = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)
+    # 512 CTAs would leave a second wave of 68 CTAs on 444 slots: 16 concurrent segments of
+    # 4 chunks instead, 4 per launch
+    wave = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)
+    assert S.kernel_launches(wave, False) == 1 and S.kernel_launches(wave, True) == 11
+    # wide enough to fill the SMs: no split; time in 4 sequential blocks under the partial cap
+    blocks = S.real_shape(16, 2048, 4096, 16, 128, S.SSM_BF16)
     assert S.kernel_launches(blocks, False) == 1 and S.kernel_launches(blocks, True) == 9
     assert S.kernel_launches(S.real_shape(2, 0, 32, 16, 128), True) == 0
     assert S.kernel_launches(S.real_shape(2, 8, 32, 12, 128), True) == -1

@@ -35,7 +35,8 @@ def bf(a):
 
 
 @pytest.mark.parametrize("B,L,D,R", [(1, 300, 40, 16), (2, 500, 1536, 48), (1, 129, 8, 256),
-                                     (3, 7, 64, 32), (1, 4096, 4096, 128), (8, 2048, 1536, 48)])
+                                     (3, 7, 64, 32), (1, 4096, 4096, 128), (8, 2048, 1536, 48),
+                                     (2, 333, 200, 64), (1, 1000, 264, 80)])
 def test_dtproj_matches_oracle(S, oracle_mod, B, L, D, R):
     p = gen.dtproj_inputs(B, L, D, R, seed=B + L + D + R)
     u, w, g = bf(p["u"]), bf(p["w"]), bf(p["g"])
