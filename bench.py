@@ -970,7 +970,7 @@ def main():
                 "hbm_frac_bwd": pbb / (t_pb / args.steps) / 1e9 / hbm,
                 "tensor_tflops_fwd": pfl / (t_pf / args.steps) / 1e12,
                 "tensor_tflops_bwd": 2 * pfl / (t_pb / args.steps) / 1e12,
-                "note": "bf16 mma.sync GEMMs; ms_per_step and value include both projections"}
+                "note": "bf16 tcgen05 GEMMs (TMA operands, TMEM accumulators); ms_per_step and value include both projections"}
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = oracle_sample(w, inp, zoh=args.zoh)
         print(json.dumps(line), flush=True)

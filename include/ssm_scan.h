@@ -68,7 +68,7 @@ typedef enum ssm_status {
     SSM_ERR_MISALIGNED = 3,           /* pointer not 16-byte aligned, or dim*sizeof(io) % 16 != 0 */
     SSM_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the size query's answer */
     SSM_ERR_CUDA = 5,                 /* a kernel launch or CUDA runtime call failed */
-    SSM_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (reserved) */
+    SSM_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (ssm_dtproj_status) */
     SSM_ERR_NONFINITE = 7             /* a NaN or Inf reached a carried state (device-side) */
 } ssm_status;
 
@@ -323,8 +323,8 @@ typedef struct ssm_dtshape {
     int32_t io;     /* SSM_BF16 (the only supported I/O type: SSM_ERR_UNSUPPORTED otherwise) */
 } ssm_dtshape;
 
-/* Workspace bytes of ssm_dtproj_bwd (fp32 partial sums of dw and dbias over splits of 512 rows;
- * at least 256); 0 for an invalid shape. */
+/* Workspace bytes of ssm_dtproj_bwd (fp32 partial sums of dw and dbias over splits of 1024 rows:
+ * ceil(M / 1024) * D * (R + 1) * 4 bytes, at least 256); 0 for an invalid shape. */
 size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape);
 
 /* delta_raw = u w^T + bias.  Enqueues 1 kernel.  Returns an ssm_status. */
@@ -336,6 +336,12 @@ int ssm_dtproj_fwd(const ssm_dtshape* shape, const void* u, const void* w, const
 int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const void* g,
                    void* du, float* dw, float* dbias, void* ws, size_t ws_bytes,
                    ssm_stream_t stream);
+
+/* Device status of the projection kernels, which wait on their tensor-core MMAs through bounded
+ * mbarrier waits: SSM_OK, or SSM_ERR_TIMEOUT once any such wait gave up (the kernel then writes no
+ * output) since the last reset.  reset != 0 clears it.  Synchronises `stream`; SSM_ERR_CUDA if the
+ * copy fails. */
+int ssm_dtproj_status(int reset, ssm_stream_t stream);
 
 /* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */

@@ -600,7 +600,7 @@ int check_dtshape(const ssm_dtshape* s) {
 }
 
 int dt_splits(const ssm_dtshape* s) {
-    const int64_t k = ssm::dtproj_rows_per_split();
+    const int64_t k = ssm::dtproj_rows_per_split(s->rank);
     return (int)((s->rows + k - 1) / k);
 }
 }  // namespace
@@ -647,6 +647,13 @@ int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const
     a.u = u; a.w = w; a.g = g; a.du = du; a.dw = dw; a.dbias = dbias;
     a.part = static_cast<float*>(ws);
     return ssm::launch_dtproj_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_dtproj_status(int reset, ssm_stream_t stream) {
+    unsigned v = 0;
+    if (ssm::dtproj_read_status(&v, reset != 0, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    return v ? SSM_ERR_TIMEOUT : SSM_OK;
 }
 
 int ssm_scan_status(const void* ws, ssm_stream_t stream) {

@@ -2,16 +2,26 @@
 // delta = softplus(projection(x)); §4.1 fuses the discretisation with this matrix product).  Per
 // row m = (batch, step):  delta_raw[m, d] = sum_r u[m, r] w[d, r] + bias[d],  with backward
 //   du = g w,   dw = g^T u,   dbias = sum_m g       (g = dL / d delta_raw).
-// Three tensor-core GEMMs, bf16 operands and fp32 accumulation (mma.sync m16n8k16, operands
-// staged through shared memory by cp.async and loaded into fragments with ldmatrix, transposed
-// where the operand is stored the other way round):
-//   forward   [M x D] = u [M x R] . w [D x R]^T, epilogue + bias, bf16 out;
-//   du        [M x R] = g [M x D] . w [D x R];
-//   dw, dbias [D x (R+1)] = g^T [D x M] . (u | 1) [M x (R+1)], split over M into fixed-order
-//             partial sums (the ones column gives dbias), then a reduction.
+// Three GEMMs on the fifth-generation tensor cores (tcgen05.mma, kind::f16: bf16 operands from
+// shared memory, fp32 accumulator in tensor memory), all from one kernel template:
+//   forward   C [M x D]   = u [M x R] . w [D x R]^T  (both operands k-major), + bias, bf16 out;
+//   du        C [M x R]   = g [M x D] . w [D x R]    (w read n-major: its rows run along k);
+//   dw, dbias C [D x R+1] = g^T [D x M] . (u | 1)    (both operands m/n-major; split over M into
+//             fixed-order fp32 partial sums; a second MMA per step against a static shared block
+//             whose first column is ones gives dbias), then a reduction.
+// Operand tiles are 64 elements wide (one 128-byte swizzle atom of bf16) and reach shared memory by
+// TMA (cp.async.bulk.tensor, 128-byte swizzle, out-of-range rows and columns filled with zeros) in
+// the canonical layouts the tensor core reads through its shared-memory descriptors: k-major
+// tiles as rows of 64 k-elements, m/n-major tiles as rows of 64 m/n-elements per k, so every box is
+// a plain 2-D window of a global array.  One thread issues the copies and the MMAs (four k16 steps
+// per stage); mbarriers carry "stage full" (TMA transaction bytes) and "stage free" / "accumulator
+// ready" (tcgen05.commit); the other warps only drain the accumulator from tensor memory.
 // The rank R is small (tens to a few hundred), so each GEMM moves far more bytes than it does
 // arithmetic per byte: they are bound by HBM (writing delta_raw, reading g), not by the tensor pipe.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <stdint.h>
 
 #include "ssm_device.cuh"
 #include "ssm_internal.h"
@@ -19,253 +29,517 @@
 namespace ssm {
 namespace {
 
-constexpr int GT = 256;  // threads per CTA (8 warps)
-constexpr int PAD = 8;   // bf16 padding per shared row (16 bytes: ldmatrix rows hit distinct banks)
+constexpr int TM = 128;    // UMMA M: tile rows = tensor-memory lanes
+constexpr int BK = 64;     // k depth of one stage: one 128-byte swizzle atom of bf16
+constexpr int NTH = 128;   // 4 warps: loaders and epilogue; thread 0 also issues the MMAs
+constexpr int A_BYTES = TM * 128;          // one A stage (either layout)
+constexpr unsigned kSpinLimit = 1u << 20;  // bounded mbarrier waits (well above any MMA)
+
+// Set (never cleared by a kernel) when a bounded wait gave up; read by ssm_dtproj_status.
+__device__ unsigned int g_dtp_status;
 
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
     return (unsigned)__cvta_generic_to_shared(p);
 }
-__device__ __forceinline__ void cp16(void* dst, const void* src, bool ok) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(ok ? 16 : 0));
-}
-__device__ __forceinline__ void ldsm4(unsigned (&r)[4], const void* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(p))
+__device__ __forceinline__ void st_shared_v4(unsigned a, unsigned x, unsigned y, unsigned z, unsigned w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
 }
-__device__ __forceinline__ void ldsm4t(unsigned (&r)[4], const void* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(p))
-                 : "memory");
+// generic-proxy writes of this thread (plain shared stores) become visible to the tensor core's
+// reads through the async proxy
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
-// D = A (16x16 bf16, row) . B (16x8 bf16, col) + C, fp32
-__device__ __forceinline__ void mma16816(float (&c)[4], const unsigned (&a)[4], unsigned b0, unsigned b1) {
+
+__device__ __forceinline__ void mbar_init(unsigned a, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned a, unsigned parity) {
+    unsigned ok;
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// arrival that also announces `bytes` of TMA transactions still to land on this phase
+__device__ __forceinline__ void mbar_expect_tx(unsigned a, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(a), "r"(bytes) : "memory");
+}
+// 2-D tensor-map box at (x innermost, y) into shared memory, completing on mbarrier `bar`
+__device__ __forceinline__ void tma_load_2d(unsigned dst, const CUtensorMap* map, int x, int y, unsigned bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+// 2-D tensor-map box from shared memory to (x innermost, y); rows and columns outside the array
+// are not written
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, unsigned src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// this thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// this thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// true once the phase of parity `parity` has completed; false if the bounded wait gave up.  The
+// caller must not be two or more phases behind (parity alone cannot tell those apart).
+__device__ __forceinline__ bool mbar_wait(unsigned a, unsigned parity) {
+    for (unsigned i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(a, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// D[tmem] (+)= A[smem] . B[smem]^T, one kind::f16 instruction (M = 128, N, K = 16)
+__device__ __forceinline__ void umma_bf16(unsigned d, uint64_t adesc, uint64_t bdesc, unsigned idesc,
+                                          unsigned accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+// arrive on the mbarrier once every MMA this thread issued so far has completed
+__device__ __forceinline__ void umma_commit(unsigned mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mbar)
+                 : "memory");
+}
+// 32 consecutive fp32 accumulator columns of this warp's 32 tensor-memory lanes (one row per lane)
+__device__ __forceinline__ void tmem_ld32(unsigned taddr, float (&v)[32]) {
+    unsigned r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start, leading and stride
+// byte offsets in 16-byte units at bits 0, 16, 32; version 1 at bit 46; layout 2 at bit 61).
+__device__ __forceinline__ uint64_t sw128_desc(unsigned saddr, unsigned lbo, unsigned sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, operand majors, N, M = 128.
+__host__ __device__ constexpr unsigned idesc_bf16(int n, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((unsigned)a_mn << 15) | ((unsigned)b_mn << 16) |
+           ((unsigned)(n >> 3) << 17) | ((unsigned)(TM >> 4) << 24);
 }
 
 enum Epi { EPI_BIAS_BF16 = 0, EPI_BF16 = 1, EPI_F32_PART = 2 };
 
-struct GemmArgs {
-    const __nv_bfloat16* A;  // logical [M][K]: AT ? A[k*lda + m] : A[m*lda + k]
-    const __nv_bfloat16* B;  // logical [N][K]: BT ? B[k*ldb + n] : B[n*ldb + k]
-    int64_t lda, ldb, ldc;
-    int64_t M, N, K;         // N counts the ones column when ones_col >= 0
-    int64_t kchunk;          // k range of one split (blockIdx.z)
-    int ones_col;            // logical column of B that is all ones (dbias), or -1
-    void* C;
+struct TcArgs {
+    int64_t M, N, K;         // logical C [M][N] = sum_k A(m, k) B(n, k); N counts the column sums
+    int64_t ldc;             // bf16 outputs: row stride of C
+    int64_t kchunk;          // k range of one split (blockIdx.z), a multiple of 64
+    int64_t ones_out;        // EPI_F32_PART: data columns below it; the column sums (dbias) go to it
+    void* C;                 // EPI_F32_PART: [split][N][M] fp32; else [M][N] bf16
     const float* bias;
 };
 
-// Shared-memory bytes of one configuration: a STAGES-deep ring of A and B tiles, reused for the
-// bf16 output tile after the main loop.
-template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int EPI>
-struct GemmSmem {
-    static constexpr int SA = AT ? BM + PAD : BK + PAD;  // shared row lengths (bf16)
-    static constexpr int SB = BT ? BN + PAD : BK + PAD;
-    static constexpr int A_ELEMS = AT ? BK * SA : BM * SA;
-    static constexpr int B_ELEMS = BT ? BK * SB : BN * SB;
-    static constexpr int SC = BN + PAD;  // bf16 output tile staged for 16-byte row stores
-    static constexpr int PIPE_BYTES = STAGES * (A_ELEMS + B_ELEMS) * 2;
-    static constexpr int C_BYTES = EPI == EPI_F32_PART ? 0 : BM * SC * 2;
-    static constexpr int BYTES = PIPE_BYTES > C_BYTES ? PIPE_BYTES : C_BYTES;
+__host__ __device__ constexpr int tmem_cols(int bn) {
+    return bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : bn <= 256 ? 256 : 512;
+}
+
+// Shared layout of the k-loop kernel: STAGES x (A tile, B tile), the static block of ones (when
+// the column sums are wanted), then the mbarriers.
+template <int BN, int STAGES, bool ONES>
+struct TcSmem {
+    static constexpr int B_BYTES = BN * 128;                 // one B stage (either layout)
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int PIPE = STAGES * STAGE;
+    static constexpr int ONE_BLK = PIPE;                     // 64 k rows x 64 columns, column 0 = 1
+    static constexpr int FULL = ONE_BLK + (ONES ? BK * 128 : 0);  // STAGES "stage loaded"
+    static constexpr int FREE = FULL + STAGES * 8;           // STAGES "stage consumed"
+    static constexpr int DONE = FREE + STAGES * 8;           // all MMAs done
+    static constexpr int SLOT = DONE + 8;                    // tensor-memory address
+    static constexpr int BYTES = SLOT + 8 + 1024;            // + slack to align the base to 1024
+    static constexpr int SROW = BN * 2 + 16;                 // bf16 output row staged for stores
+    static_assert(TM * SROW <= PIPE, "output staging fits the pipeline buffers");
 };
 
-// C tile [BM x BN] of blockIdx (y: m, x: n, z: k split).  Warps WM x WN, warp tile
-// (BM/WM) x (BN/WN) of m16 x n8 mma tiles; k in steps of BK through a STAGES-deep cp.async ring.
-template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int WM, int WN, int EPI>
-__global__ void __launch_bounds__(GT) dtp_gemm_kernel(GemmArgs p) {
-    static_assert(WM * WN * 32 == GT, "eight warps");
-    static_assert(BK % 16 == 0 && STAGES >= 2, "k steps of whole mma blocks");
-    constexpr int TM = BM / WM, TN = BN / WN, MT = TM / 16, NT8 = TN / 8;
-    static_assert(TM % 16 == 0 && TN % 16 == 0, "warp tile of whole m16 x n16 blocks");
-    using Sm = GemmSmem<AT, BT, BM, BN, BK, STAGES, EPI>;
-    constexpr int SA = Sm::SA, SB = Sm::SB, A_ELEMS = Sm::A_ELEMS, B_ELEMS = Sm::B_ELEMS, SC = Sm::SC;
-    extern __shared__ __align__(16) unsigned char smem[];
-    __nv_bfloat16 (*sA)[A_ELEMS] = reinterpret_cast<__nv_bfloat16 (*)[A_ELEMS]>(smem);
-    __nv_bfloat16 (*sB)[B_ELEMS] =
-        reinterpret_cast<__nv_bfloat16 (*)[B_ELEMS]>(smem + STAGES * A_ELEMS * 2);
+__device__ __forceinline__ void tmem_alloc_cta(unsigned slot, unsigned cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_cta(unsigned taddr, unsigned cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(cols) : "memory");
+}
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int wm = warp / WN, wn = warp % WN;
-    const int64_t m0 = (int64_t)blockIdx.y * BM, n0 = (int64_t)blockIdx.x * BN;
+// C tile [128 x BN] of blockIdx (y: m, x: n, z: k split), the k range in 64-deep stages.
+// mA, mB: tensor maps of A and B with 64-element-wide boxes (k-major: {64 k, rows}; m/n-major:
+// {64 m/n, 64 k}).  ONES: one more 64-wide accumulator block multiplies A by a static block whose
+// first column is all ones, giving A's column sums (dbias) in accumulator column BN.
+template <bool A_MN, bool B_MN, int BN, int STAGES, bool ONES, int EPI>
+__global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUtensorMap mA,
+                                                     const __grid_constant__ CUtensorMap mB, TcArgs p) {
+    static_assert(BN % 64 == 0 && BN <= 256 && STAGES >= 3, "n tile of whole 64-wide blocks");
+    static_assert(!ONES || EPI == EPI_F32_PART, "column sums go to the fp32 partial sums");
+    using Sm = TcSmem<BN, STAGES, ONES>;
+    constexpr int TCOLS = tmem_cols(BN + (ONES ? 64 : 0));
+    constexpr int PF = STAGES - 2;  // stages loading ahead of the one being multiplied
+    extern __shared__ unsigned char smem_raw[];
+    const unsigned raw = smem_u32(smem_raw);
+    const unsigned base = (raw + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
+    unsigned char* gbase = smem_raw + (base - raw);
+    const unsigned full = base + Sm::FULL, free_ = base + Sm::FREE, done = base + Sm::DONE;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t m0 = (int64_t)blockIdx.y * TM, n0 = (int64_t)blockIdx.x * BN;
     const int64_t kb = (int64_t)blockIdx.z * p.kchunk;
     const int64_t ke = min(p.K, kb + p.kchunk);
-    const int nk = (int)((ke - kb + BK - 1) / BK);
+    const int nk = ke > kb ? (int)((ke - kb + BK - 1) / BK) : 0;
 
-    auto load = [&](int st, int64_t k0) {
-        __nv_bfloat16* a = sA[st];
-        __nv_bfloat16* b = sB[st];
-        if (AT) {  // BK rows of k, BM/8 chunks of m
-            for (int q = tid; q < BK * (BM / 8); q += GT) {
-                const int r = q / (BM / 8), c = q % (BM / 8);
-                const int64_t k = k0 + r, m = m0 + 8 * c;
-                const bool ok = k < ke && m + 8 <= p.M;
-                cp16(a + r * SA + 8 * c, ok ? p.A + k * p.lda + m : p.A, ok);
-            }
-        } else {   // BM rows of m, BK/8 chunks of k
-            for (int q = tid; q < BM * (BK / 8); q += GT) {
-                const int r = q / (BK / 8), c = q % (BK / 8);
-                const int64_t m = m0 + r, k = k0 + 8 * c;
-                const bool ok = m < p.M && k + 8 <= ke;
-                cp16(a + r * SA + 8 * c, ok ? p.A + m * p.lda + k : p.A, ok);
-            }
+    if (warp == 0) tmem_alloc_cta(base + Sm::SLOT, TCOLS);
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + 8 * s, 1);
+            mbar_init(free_ + 8 * s, 1);
         }
-        if (BT) {  // BK rows of k, BN/8 chunks of n; the ones column's chunk is written directly
-            for (int q = tid; q < BK * (BN / 8); q += GT) {
-                const int r = q / (BN / 8), c = q % (BN / 8);
-                const int64_t k = k0 + r, n = n0 + 8 * c;
-                __nv_bfloat16* dst = b + r * SB + 8 * c;
-                if (p.ones_col >= 0 && n == p.ones_col) {
-                    const __nv_bfloat16 one = __float2bfloat16(k < ke ? 1.0f : 0.0f);
-                    const __nv_bfloat16 zero = __float2bfloat16(0.0f);
-                    dst[0] = one;
-#pragma unroll
-                    for (int i = 1; i < 8; ++i) dst[i] = zero;
-                } else {
-                    const bool ok = k < ke && n + 8 <= (p.ones_col >= 0 ? p.ones_col : p.N);
-                    cp16(dst, ok ? p.B + k * p.ldb + n : p.B, ok);
-                }
-            }
-        } else {   // BN rows of n, BK/8 chunks of k
-            for (int q = tid; q < BN * (BK / 8); q += GT) {
-                const int r = q / (BK / 8), c = q % (BK / 8);
-                const int64_t n = n0 + r, k = k0 + 8 * c;
-                const bool ok = n < p.N && k + 8 <= ke;
-                cp16(b + r * SB + 8 * c, ok ? p.B + n * p.ldb + k : p.B, ok);
-            }
-        }
-        asm volatile("cp.async.commit_group;\n" ::);
-    };
-
-    const int g = lane >> 2, t4 = lane & 3;
-    float bias_r[NT8][2];  // the bias of this thread's output columns, fetched before the main loop
-#pragma unroll
-    for (int jn = 0; jn < NT8; ++jn) {
-        const int64_t col = n0 + wn * TN + 8 * jn + 2 * t4;
-        const bool on = EPI == EPI_BIAS_BF16 && p.bias != nullptr && col < p.N;
-        bias_r[jn][0] = on ? p.bias[col] : 0.0f;
-        bias_r[jn][1] = on ? p.bias[col + 1] : 0.0f;
+        mbar_init(done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-
-    float acc[MT][NT8][4];
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-#pragma unroll
-        for (int j = 0; j < NT8; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
-
-    // ring: STAGES - 1 tiles in flight ahead of the one being multiplied (empty groups past the
-    // end keep the group count uniform)
-#pragma unroll
-    for (int s0 = 0; s0 < STAGES - 1; ++s0) {
-        if (s0 < nk)
-            load(s0, kb + (int64_t)s0 * BK);
-        else
-            asm volatile("cp.async.commit_group;\n" ::);
-    }
-    for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt % STAGES;
-        asm volatile("cp.async.wait_group %0;\n" ::"n"(STAGES - 2));
-        __syncthreads();  // tile kt is in; every thread is done with tile kt - 1
-        {
-            const int kn = kt + STAGES - 1;
-            if (kn < nk)
-                load(kn % STAGES, kb + (int64_t)kn * BK);
-            else
-                asm volatile("cp.async.commit_group;\n" ::);
+    if (ONES) {
+        // 64 k rows x 64 columns (m/n-major, 128-byte swizzle), bf16 1.0 in column 0 of every row:
+        // chunk 0 of row r sits at chunk (0 ^ (r & 7)).  Rows past K meet zeros in A.
+        for (int q = tid; q < BK * 8; q += NTH) {
+            const int r = q >> 3, c = q & 7;
+            st_shared_v4(base + Sm::ONE_BLK + r * 128 + ((c ^ (r & 7)) << 4), c == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
         }
-        const __nv_bfloat16* a = sA[st];
-        const __nv_bfloat16* b = sB[st];
-#pragma unroll
-        for (int ks = 0; ks < BK / 16; ++ks) {
-            unsigned af[MT][4];
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-                const int mr = wm * TM + 16 * i;
-                const int j = lane >> 3;
-                if (AT)  // stored [k][m]: matrix j = (m block j&1, k block j>>1)
-                    ldsm4t(af[i], a + (ks * 16 + 8 * (j >> 1) + (lane & 7)) * SA + mr + 8 * (j & 1));
-                else     // stored [m][k]: lanes 0-15 rows m, lanes 16-31 the upper k half
-                    ldsm4(af[i], a + (mr + (lane & 15)) * SA + ks * 16 + 8 * (lane >> 4));
-            }
-#pragma unroll
-            for (int jn = 0; jn < NT8; jn += 2) {
-                const int nc = wn * TN + 8 * jn;
-                const int j = lane >> 3;
-                unsigned bf[4];  // (b0b1, b2b3) of n8 tile jn, then of tile jn + 1
-                if (BT)  // stored [k][n]: matrix j = (k block j&1, n block j>>1)
-                    ldsm4t(bf, b + (ks * 16 + 8 * (j & 1) + (lane & 7)) * SB + nc + 8 * (j >> 1));
-                else     // stored [n][k]: matrix j = (n block j>>1, k block j&1)
-                    ldsm4(bf, b + (nc + 8 * (j >> 1) + (lane & 7)) * SB + ks * 16 + 8 * (j & 1));
-#pragma unroll
-                for (int i = 0; i < MT; ++i) {
-                    mma16816(acc[i][jn], af[i], bf[0], bf[1]);
-                    mma16816(acc[i][jn + 1], af[i], bf[2], bf[3]);
-                }
-            }
-        }
+        fence_async_smem();
     }
-    __syncthreads();  // every thread is done with the ring (the output tile reuses it)
-
-    // epilogue: c0, c1 at (row g, cols 2t, 2t+1), c2, c3 at row g + 8
-    if (EPI == EPI_F32_PART) {
-#pragma unroll
-        for (int i = 0; i < MT; ++i)
-#pragma unroll
-            for (int jn = 0; jn < NT8; ++jn) {
-                const int64_t col = n0 + wn * TN + 8 * jn + 2 * t4;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int64_t row = m0 + wm * TM + 16 * i + g + 8 * h;
-                    if (row >= p.M || col >= p.N) continue;
-                    float* c = static_cast<float*>(p.C) + (int64_t)blockIdx.z * p.M * p.ldc + row * p.ldc;
-                    c[col] = acc[i][jn][2 * h];
-                    if (col + 1 < p.N) c[col + 1] = acc[i][jn][2 * h + 1];
-                }
-            }
-        return;
-    }
-    // bf16 outputs (N a multiple of 8): the tile goes through shared memory (the pipeline buffers
-    // are free after the last barrier) and leaves as 16-byte row pieces
-    __nv_bfloat16* sC = reinterpret_cast<__nv_bfloat16*>(smem);
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-#pragma unroll
-        for (int jn = 0; jn < NT8; ++jn) {
-            const int cl = wn * TN + 8 * jn + 2 * t4;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int rl = wm * TM + 16 * i + g + 8 * h;
-                *reinterpret_cast<__nv_bfloat162*>(sC + rl * SC + cl) = __floats2bfloat162_rn(
-                    acc[i][jn][2 * h] + bias_r[jn][0], acc[i][jn][2 * h + 1] + bias_r[jn][1]);
-            }
-        }
+    tc_fence_before();
     __syncthreads();
-    for (int q = tid; q < BM * (BN / 8); q += GT) {
-        const int rl = q / (BN / 8), c8 = q % (BN / 8);
-        const int64_t row = m0 + rl, col = n0 + 8 * c8;
-        if (row < p.M && col < p.N)
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col) =
-                *reinterpret_cast<const uint4*>(sC + rl * SC + 8 * c8);
+    tc_fence_after();
+    const unsigned tmem = *reinterpret_cast<volatile unsigned*>(gbase + Sm::SLOT);
+
+    bool ok = true;
+    if (tid == 0) {
+        auto issue = [&](int t, int st) {
+            const unsigned a = base + st * Sm::STAGE, b = a + A_BYTES, f = full + 8 * st;
+            const int k0 = (int)(kb + (int64_t)t * BK);
+            mbar_expect_tx(f, Sm::STAGE);
+            if (!A_MN) {
+                tma_load_2d(a, &mA, k0, (int)m0, f);
+            } else {
+                tma_load_2d(a, &mA, (int)m0, k0, f);
+                tma_load_2d(a + BK * 128, &mA, (int)m0 + 64, k0, f);
+            }
+            if (!B_MN) {
+                tma_load_2d(b, &mB, k0, (int)n0, f);
+            } else {
+#pragma unroll
+                for (int blk = 0; blk < BN / 64; ++blk) tma_load_2d(b + blk * (BK * 128), &mB, (int)n0 + 64 * blk, k0, f);
+            }
+        };
+        for (int t = 0; t < PF && t < nk; ++t) issue(t, t);
+        for (int kt = 0; kt < nk && ok; ++kt) {
+            const int nx = kt + PF;
+            if (nx < nk) {
+                const int st = nx % STAGES;
+                // the stage last held tile nx - STAGES = kt - 2, multiplied a step ago
+                if (nx >= STAGES) ok = mbar_wait(free_ + 8 * st, (unsigned)((nx / STAGES - 1) & 1));
+                if (!ok) break;
+                issue(nx, st);
+            }
+            const int s = kt % STAGES;
+            if (!(ok = mbar_wait(full + 8 * s, (unsigned)((kt / STAGES) & 1)))) break;
+            const unsigned a = base + s * Sm::STAGE, b = a + A_BYTES;
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < BK / 16; ++j) {
+                // k16 step j: 32 bytes into each k-major row, or two 8-row groups of k rows
+                const uint64_t ad = A_MN ? sw128_desc(a + j * 2048, BK * 128, 1024)
+                                         : sw128_desc(a + j * 32, 16, 1024);
+                const uint64_t bd = B_MN ? sw128_desc(b + j * 2048, BK * 128, 1024)
+                                         : sw128_desc(b + j * 32, 16, 1024);
+                umma_bf16(tmem, ad, bd, idesc_bf16(BN, A_MN, B_MN), (kt | j) != 0);
+                if (ONES)
+                    umma_bf16(tmem + BN, ad, sw128_desc(base + Sm::ONE_BLK + j * 2048, BK * 128, 1024),
+                              idesc_bf16(64, A_MN, true), (kt | j) != 0);
+            }
+            umma_commit(free_ + 8 * s);
+        }
+        umma_commit(done);  // arrives once every MMA issued above has completed
+        if (ok) ok = mbar_wait(done, 0);
+        tc_fence_before();
+    }
+    // the other threads wait here (not spinning on the mbarrier beside thread 0)
+    const bool bad = __syncthreads_or(!ok);
+    tc_fence_after();
+
+    if (!bad) {
+        const int row = warp * 32 + lane;  // tile row = tensor-memory lane
+        const unsigned tl = tmem + ((unsigned)(warp * 32) << 16);
+        if (EPI == EPI_F32_PART) {
+            // partial sums [split][N][M]: one column per store, the warp's 32 rows contiguous; tile
+            // columns below ones_out are data columns, accumulator column BN the column sums
+            float* out = static_cast<float*>(p.C) + (int64_t)blockIdx.z * p.N * p.M;
+            const int64_t m = m0 + row;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN + (ONES ? 32 : 0); c0 += 32) {
+                float v[32];
+                if (nk > 0) {
+                    tmem_ld32(tl + c0, v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
+                if (m < p.M) {
+                    if (c0 < BN) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int64_t col = n0 + c0 + i;
+                            if (col < p.ones_out) out[col * p.M + m] = v[i];
+                        }
+                    } else {
+                        out[(int64_t)p.ones_out * p.M + m] = v[0];
+                    }
+                }
+            }
+        } else {
+            // bf16 rows staged in shared memory (the pipeline buffers are free), then stored as
+            // 16-byte row pieces
+            const unsigned srow = base + row * Sm::SROW;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float v[32];
+                if (nk > 0) {
+                    tmem_ld32(tl + c0, v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    unsigned w4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
+                        w4[i] = *reinterpret_cast<const unsigned*>(&h);
+                    }
+                    st_shared_v4(srow + (c0 + 8 * q) * 2, w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            __syncthreads();
+            for (int q = tid; q < TM * (BN / 8); q += NTH) {
+                const int rl = q / (BN / 8), c8 = q % (BN / 8);
+                const int64_t m = m0 + rl, col = n0 + 8 * c8;
+                if (m < p.M && col < p.N)
+                    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + m * p.ldc + col) =
+                        *reinterpret_cast<const uint4*>(gbase + rl * Sm::SROW + 16 * c8);
+            }
+        }
+    } else if (tid == 0) {
+        atomicOr(&g_dtp_status, 1u);
+        mbar_wait(done, 0);  // the MMAs already issued get a last bounded chance to finish
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_cta(tmem, TCOLS);
     }
 }
 
-// dw[d, r] = sum_s part[s, d, r] (r < R), dbias[d] = sum_s part[s, d, R], in a fixed order.
+// Forward GEMM, persistent: CTA c handles output tiles c, c + G, c + 2G, ... (tile = 128 rows of u
+// x BN rows of w, the whole k range R <= 64 KA in one stage).  Two stages and two tensor-memory
+// accumulators: while the tensor core multiplies tile i into one accumulator, the eight warps
+// drain tile i - 1 from the other (+ bias, bf16, into a 128-byte-swizzled staging tile that one
+// TMA store writes out) and the copies of tile i + 1 are in flight.
+constexpr int FWD_NTH = 256;
+template <int KA, int BN>
+struct FwdSm {
+    static constexpr int A_ST = KA * TM * 128;     // KA swizzle atoms of 128 rows
+    static constexpr int B_ST = KA * BN * 128;
+    static constexpr int STAGE = A_ST + B_ST;
+    static constexpr int STG = 2 * STAGE;          // output tile: BN / 64 atoms of 128 rows
+    static constexpr int FULL = STG + BN * 256;    // 2 "stage loaded" mbarriers
+    static constexpr int ACC = FULL + 16;          // 2 "accumulator ready" mbarriers
+    static constexpr int SLOT = ACC + 16;
+    static constexpr int BYTES = SLOT + 16 + 1024;
+};
+
+template <int KA, int BN>
+__global__ void __launch_bounds__(FWD_NTH) dtp_fwd_kernel(const __grid_constant__ CUtensorMap mA,
+                                                          const __grid_constant__ CUtensorMap mB,
+                                                          const __grid_constant__ CUtensorMap mC, TcArgs p,
+                                                          int64_t n_nt, int64_t ntiles) {
+    static_assert(BN % 64 == 0 && 2 * BN <= 512, "two accumulators of whole 64-wide blocks");
+    using Sm = FwdSm<KA, BN>;
+    constexpr int TCOLS = tmem_cols(2 * BN);
+    extern __shared__ unsigned char smem_raw[];
+    const unsigned raw = smem_u32(smem_raw);
+    const unsigned base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    const unsigned full = base + Sm::FULL, acc = base + Sm::ACC, stg = base + Sm::STG;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int T = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+
+    if (warp == 0) tmem_alloc_cta(base + Sm::SLOT, TCOLS);
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(full + 8 * s, 1);
+            mbar_init(acc + 8 * s, 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tmem = *reinterpret_cast<volatile unsigned*>(gbase + Sm::SLOT);
+
+    auto tile_m0 = [&](int i) { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) / n_nt * TM; };
+    auto tile_n0 = [&](int i) { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) % n_nt * BN; };
+    auto issue = [&](int i, int s) {  // thread 0: both operands of tile i, every k atom
+        const unsigned a = base + s * Sm::STAGE, b = a + Sm::A_ST, f = full + 8 * s;
+        const int m0 = (int)tile_m0(i), n0 = (int)tile_n0(i);
+        mbar_expect_tx(f, Sm::STAGE);
+#pragma unroll
+        for (int at = 0; at < KA; ++at) {
+            tma_load_2d(a + at * (TM * 128), &mA, 64 * at, m0, f);
+            tma_load_2d(b + at * (BN * 128), &mB, 64 * at, n0, f);
+        }
+    };
+    // accumulator of tile i -> + bias -> bf16 -> swizzled staging tile -> TMA store (thread 0)
+    auto drain = [&](int i) {
+        const int64_t m0 = tile_m0(i), n0 = tile_n0(i);
+        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+        const unsigned tl = tmem + (i & 1) * BN + ((unsigned)((warp & 3) * 32) << 16);
+#pragma unroll
+        for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
+            float v[32];
+            tmem_ld32(tl + c0, v);
+            if (p.bias != nullptr) {
+                if (n0 + c0 + 32 <= p.N) {
+                    const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + c0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = __ldg(b4 + q);
+                        v[4 * q] += bb.x;
+                        v[4 * q + 1] += bb.y;
+                        v[4 * q + 2] += bb.z;
+                        v[4 * q + 3] += bb.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (n0 + c0 + j < p.N) v[j] += __ldg(p.bias + n0 + c0 + j);
+                }
+            }
+            // columns c0 .. c0 + 31: 16-byte chunks (c0 % 64) / 8 + q of the 64-column atom c0 / 64
+            const unsigned atom = stg + (c0 / 64) * (TM * 128) + row * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                unsigned w4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
+                    w4[j] = *reinterpret_cast<const unsigned*>(&h);
+                }
+                const int cc = (c0 % 64) / 8 + q;
+                st_shared_v4(atom + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int hb = 0; hb < BN / 64; ++hb) tma_store_2d(&mC, stg + hb * (TM * 128), (int)n0 + 64 * hb, (int)m0);
+            bulk_commit();
+        }
+    };
+
+    bool ok = true;
+    if (tid == 0 && T > 0) issue(0, 0);
+    for (int i = 0; i < T; ++i) {
+        const int s = i & 1;
+        if (tid == 0) {
+            // stage s ^ 1 and accumulator s ^ 1 held tile i - 1: once its MMAs are done the stage
+            // takes tile i + 1 and the accumulator can be drained
+            if (i >= 1) ok = mbar_wait(acc + 8 * (s ^ 1), (unsigned)(((i - 1) >> 1) & 1));
+            if (ok && i + 1 < T) issue(i + 1, s ^ 1);
+            if (ok) ok = mbar_wait(full + 8 * s, (unsigned)((i >> 1) & 1));
+            if (ok) {
+                tc_fence_after();
+                const unsigned a = base + s * Sm::STAGE, b = a + Sm::A_ST;
+#pragma unroll
+                for (int j = 0; j < 4 * KA; ++j)
+                    umma_bf16(tmem + s * BN, sw128_desc(a + (j >> 2) * (TM * 128) + (j & 3) * 32, 16, 1024),
+                              sw128_desc(b + (j >> 2) * (BN * 128) + (j & 3) * 32, 16, 1024),
+                              idesc_bf16(BN, false, false), j != 0);
+                umma_commit(acc + 8 * s);
+            }
+            bulk_wait_read();  // the staging tile of the previous drain has been read out
+            tc_fence_before();
+        }
+        if (__syncthreads_or(!ok)) {
+            ok = false;
+            break;
+        }
+        if (i >= 1) {
+            tc_fence_after();
+            drain(i - 1);
+        }
+    }
+    if (tid == 0 && ok && T > 0) {
+        ok = mbar_wait(acc + 8 * ((T - 1) & 1), (unsigned)(((T - 1) >> 1) & 1));
+        bulk_wait_read();
+        tc_fence_before();
+    }
+    if (!__syncthreads_or(!ok)) {
+        if (T > 0) {
+            tc_fence_after();
+            drain(T - 1);
+        }
+    } else if (tid == 0) {
+        atomicOr(&g_dtp_status, 1u);
+        // the MMAs already issued get a last bounded chance to finish
+        if (T > 0) mbar_wait(acc + 8 * ((T - 1) & 1), (unsigned)(((T - 1) >> 1) & 1));
+    }
+    if (tid == 0) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_cta(tmem, TCOLS);
+    }
+}
+
+// dw[d, r] = sum_s part[s, r, d] (r < R), dbias[d] = sum_s part[s, R, d], in a fixed order.
 __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, int64_t D, int R,
                                   float* __restrict__ dw, float* __restrict__ dbias) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // r * D + d
     const int64_t n = D * (R + 1);
     if (i >= n) return;
-    const int64_t d = i / (R + 1);
-    const int r = (int)(i - d * (R + 1));
+    const int r = (int)(i / D);
+    const int64_t d = i - (int64_t)r * D;
     // four interleaved running sums (independent loads in flight), combined in a fixed order
     float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
     int k = 0;
@@ -283,61 +557,148 @@ __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, in
         dbias[d] = s;
 }
 
-template <bool AT, bool BT, int BM, int BN, int BK, int STAGES, int WM, int WN, int EPI>
-cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
-    const dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + BM - 1) / BM), (unsigned)splits);
-    constexpr int bytes = GemmSmem<AT, BT, BM, BN, BK, STAGES, EPI>::BYTES;
-    auto kern = dtp_gemm_kernel<AT, BT, BM, BN, BK, STAGES, WM, WN, EPI>;
-    if (bytes > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e != cudaSuccess) return e;
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no link to libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
     }
-    kern<<<grid, GT, bytes, st>>>(a);
+    return fn;
+}
+
+// Tensor map of a row-major bf16 array [rows][cols] (row stride ld elements) with boxes of
+// 64 columns x box_rows rows, 128-byte swizzle, zeros outside the array.
+cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+    const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <bool A_MN, bool B_MN, int BN, int STAGES, bool ONES, int EPI>
+cudaError_t run_tc(const CUtensorMap& mA, const CUtensorMap& mB, const TcArgs& a, int splits, cudaStream_t st) {
+    const int64_t ncols = ONES ? a.ones_out : a.N;  // data columns (the column sums ride along)
+    const dim3 grid((unsigned)((ncols + BN - 1) / BN), (unsigned)((a.M + TM - 1) / TM), (unsigned)splits);
+    constexpr int bytes = TcSmem<BN, STAGES, ONES>::BYTES;
+    auto kern = dtp_tc_kernel<A_MN, B_MN, BN, STAGES, ONES, EPI>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NTH, bytes, st>>>(mA, mB, a);
+    return cudaGetLastError();
+}
+
+template <int KA, int BN>
+cudaError_t run_fwd(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC, const TcArgs& a,
+                    cudaStream_t st) {
+    constexpr int bytes = FwdSm<KA, BN>::BYTES;
+    auto kern = dtp_fwd_kernel<KA, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // CTAs per SM: shared memory (with the per-CTA reservation) and the two accumulators in the
+    // SM's 512 tensor-memory columns bound it (registers do not, at 256 threads)
+    int smem_sm = 0, resv = 0;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+    per_sm = smem_sm / (bytes + resv);
+    const int tcap = 512 / tmem_cols(2 * BN);
+    if (per_sm > tcap) per_sm = tcap;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t n_nt = (a.N + BN - 1) / BN;
+    const int64_t ntiles = n_nt * ((a.M + TM - 1) / TM);
+    const int64_t grid = ntiles < (int64_t)sms * per_sm ? ntiles : (int64_t)sms * per_sm;
+    kern<<<(unsigned)grid, FWD_NTH, bytes, st>>>(mA, mB, mC, a, n_nt, ntiles);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int64_t dtproj_rows_per_split() { return 256; }
+// Rows of one dw / dbias split (a multiple of the 64-row stage)
+int64_t dtproj_rows_per_split(int) { return 1024; }
+
+cudaError_t dtproj_read_status(unsigned* status, bool reset, cudaStream_t st) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(status, g_dtp_status, sizeof(unsigned), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && reset) {
+        static const unsigned zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_dtp_status, &zero, sizeof(unsigned), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    return e;
+}
 
 cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
-    GemmArgs a = {};
-    a.A = static_cast<const __nv_bfloat16*>(d.u);
-    a.B = static_cast<const __nv_bfloat16*>(d.w);
-    a.lda = d.R; a.ldb = d.R; a.ldc = d.D;
-    a.M = d.M; a.N = d.D; a.K = d.R; a.kchunk = d.R;
-    a.ones_col = -1;
+    // delta_raw [M x D] = u [M x R] . w [D x R]^T + bias: both operands k-major
+    const int ka = (d.R + 63) / 64;              // 64-deep k atoms covering R, all in one stage
+    const int bn = ka <= 2 ? 128 : 64;
+    CUtensorMap mA, mB, mC;
+    cudaError_t e = make_map(&mA, d.u, d.M, d.R, d.R, TM);
+    if (e == cudaSuccess) e = make_map(&mB, d.w, d.D, d.R, d.R, bn);
+    if (e == cudaSuccess) e = make_map(&mC, d.delta_raw, d.M, d.D, d.D, TM);
+    if (e != cudaSuccess) return e;
+    TcArgs a = {};
+    a.M = d.M; a.N = d.D; a.K = d.R; a.ldc = d.D; a.kchunk = d.R;
+    a.ones_out = d.D;
     a.C = d.delta_raw;
     a.bias = d.bias;
-    // R <= 64: the whole k range in one shared tile (no ring turnover); larger R: 128-row tiles
-    // so each w tile serves twice the rows
-    if (d.R <= 16) return run_gemm<false, false, 64, 128, 16, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
-    if (d.R <= 32) return run_gemm<false, false, 64, 128, 32, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
-    if (d.R <= 48) return run_gemm<false, false, 64, 128, 48, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
-    if (d.R <= 64) return run_gemm<false, false, 64, 128, 64, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
-    return run_gemm<false, false, 128, 128, 64, 2, 2, 4, EPI_BIAS_BF16>(a, 1, st);
+    switch (ka) {
+        case 1: return run_fwd<1, 128>(mA, mB, mC, a, st);
+        case 2: return run_fwd<2, 128>(mA, mB, mC, a, st);
+        case 3: return run_fwd<3, 64>(mA, mB, mC, a, st);
+        default: return run_fwd<4, 64>(mA, mB, mC, a, st);
+    }
 }
 
 cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
-    // du [M x R] = g [M x D] . w [D x R]   (B stored [k = d][n = r])
-    GemmArgs a = {};
-    a.A = static_cast<const __nv_bfloat16*>(d.g);
-    a.B = static_cast<const __nv_bfloat16*>(d.w);
-    a.lda = d.D; a.ldb = d.R; a.ldc = d.R;
-    a.M = d.M; a.N = d.R; a.K = d.D; a.kchunk = d.D;
-    a.ones_col = -1;
-    a.C = d.du;
-    cudaError_t e = run_gemm<false, true, 128, 64, 64, 3, 4, 2, EPI_BF16>(a, 1, st);
+    // du [M x R] = g [M x D] . w [D x R]: A = g k-major ({64 d, 128 rows} boxes), B = w read with its
+    // rows along k (n-major, {64 r, 64 d} boxes)
+    CUtensorMap gK, wN, gM, uN;
+    cudaError_t e = make_map(&gK, d.g, d.M, d.D, d.D, TM);
+    if (e == cudaSuccess) e = make_map(&wN, d.w, d.D, d.R, d.R, BK);
+    // dw partials [split][R+1][D] = g^T [D x M] . (u | 1) [M x (R+1)]: A = g m-major and B = u
+    // n-major ({64 d or r, 64 rows} boxes)
+    if (e == cudaSuccess) e = make_map(&gM, d.g, d.M, d.D, d.D, BK);
+    if (e == cudaSuccess) e = make_map(&uN, d.u, d.M, d.R, d.R, BK);
     if (e != cudaSuccess) return e;
-    // partials [split][D][R+1] = g^T [D x M] . (u | 1) [M x (R+1)]   (A stored [k = m][d], B [m][r])
-    GemmArgs b = {};
-    b.A = static_cast<const __nv_bfloat16*>(d.g);
-    b.B = static_cast<const __nv_bfloat16*>(d.u);
-    b.lda = d.D; b.ldb = d.R; b.ldc = d.R + 1;
-    b.M = d.D; b.N = d.R + 1; b.K = d.M; b.kchunk = dtproj_rows_per_split();
-    b.ones_col = d.R;
+    TcArgs a = {};
+    a.M = d.M; a.N = d.R; a.K = d.D; a.ldc = d.R; a.kchunk = d.D;
+    a.ones_out = d.R;
+    a.C = d.du;
+    switch ((d.R + 63) / 64) {  // 64-wide n blocks covering R
+        case 1: e = run_tc<false, true, 64, 8, false, EPI_BF16>(gK, wN, a, 1, st); break;
+        case 2: e = run_tc<false, true, 128, 6, false, EPI_BF16>(gK, wN, a, 1, st); break;
+        case 3: e = run_tc<false, true, 192, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
+        default: e = run_tc<false, true, 256, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
+    }
+    if (e != cudaSuccess) return e;
+    // dw partials [split][R+1][D]: data columns 0..R-1, then the column sums of g (dbias) from the
+    // static block of ones
+    TcArgs b = {};
+    b.M = d.D; b.N = d.R + 1; b.K = d.M; b.ldc = 0; b.kchunk = dtproj_rows_per_split(d.R);
+    b.ones_out = d.R;
     b.C = d.part;
-    e = run_gemm<true, true, 128, 64, 32, 3, 4, 2, EPI_F32_PART>(b, d.splits, st);
+    switch ((d.R + 63) / 64) {
+        case 1: e = run_tc<true, true, 64, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
+        case 2: e = run_tc<true, true, 128, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
+        case 3: e = run_tc<true, true, 192, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
+        default: e = run_tc<true, true, 256, 3, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
+    }
     if (e != cudaSuccess) return e;
     const int64_t n = d.D * (d.R + 1);
     dtp_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(d.part, d.splits, d.D, d.R, d.dw,

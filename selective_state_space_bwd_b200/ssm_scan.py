@@ -73,7 +73,7 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
             "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd",
             "ssm_pdssm_kernel_launches", "ssm_dtproj_workspace_bytes", "ssm_dtproj_fwd",
-            "ssm_dtproj_bwd"]
+            "ssm_dtproj_bwd", "ssm_dtproj_status"]
 
 
 def lib():
@@ -124,6 +124,7 @@ def lib():
             L.ssm_dtproj_fwd.argtypes, L.ssm_dtproj_fwd.restype = [DP] + [P] * 4 + [P], I
             L.ssm_dtproj_bwd.argtypes = [DP] + [P] * 7 + [Z, P]
             L.ssm_dtproj_bwd.restype = I
+            L.ssm_dtproj_status.argtypes, L.ssm_dtproj_status.restype = [I, P], I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -479,3 +480,8 @@ def ssm_dtproj_bwd(u, w, g, want_dbias=True, out=None, ws=None, stream=None):
                                 ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_dtproj_bwd")
     return out
+
+
+def dtproj_status(reset=False, stream=None) -> int:
+    """SSM_OK, or SSM_ERR_TIMEOUT once a projection kernel's bounded wait gave up (synchronises)."""
+    return int(lib().ssm_dtproj_status(1 if reset else 0, _stream(stream)))

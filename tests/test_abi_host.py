@@ -256,7 +256,8 @@ def test_dtproj_validation(S):
     import ctypes
     L = S.lib()
     ok = S.dtproj_shape(1000, 1536, 48)
-    assert S.dtproj_workspace_bytes(ok) == 4 * 1536 * 49 * 4  # four splits of 256 rows, R + 1 columns
+    assert S.dtproj_workspace_bytes(ok) == 1536 * 49 * 4  # one split of 1024 rows, R + 1 columns
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(3000, 64, 128)) == 3 * 64 * 129 * 4
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1536, 40)) == 0   # R not a multiple of 16
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1532, 48)) == 0   # D not a multiple of 8
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 64, 272)) == 0    # R > 256

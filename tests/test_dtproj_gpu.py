@@ -36,7 +36,7 @@ def bf(a):
 
 @pytest.mark.parametrize("B,L,D,R", [(1, 300, 40, 16), (2, 500, 1536, 48), (1, 129, 8, 256),
                                      (3, 7, 64, 32), (1, 4096, 4096, 128), (8, 2048, 1536, 48),
-                                     (2, 333, 200, 64), (1, 1000, 264, 80)])
+                                     (2, 333, 200, 64), (1, 1000, 264, 80), (2, 1000, 520, 192)])
 def test_dtproj_matches_oracle(S, oracle_mod, B, L, D, R):
     p = gen.dtproj_inputs(B, L, D, R, seed=B + L + D + R)
     u, w, g = bf(p["u"]), bf(p["w"]), bf(p["g"])
@@ -95,3 +95,13 @@ def test_projection_scan_pipeline(S, oracle_mod):
     assert rel(y.float().cpu().numpy(), sc["y"]) <= 2e-2
     for k in ("du", "dw", "dbias"):
         assert rel(pg[k].float().cpu().numpy(), ref[k]) <= 2e-2, k
+
+
+def test_dtproj_status_clean(S):
+    """No bounded tensor-core wait of the projection kernels gave up in this process."""
+    p = gen.dtproj_inputs(2, 700, 320, 64, seed=11)
+    u, w, g = bf(p["u"]), bf(p["w"]), bf(p["g"])
+    S.ssm_dtproj_fwd(u, w, torch.from_numpy(p["bias"]).cuda())
+    S.ssm_dtproj_bwd(u, w, g)
+    assert S.dtproj_status() == S.SSM_OK
+    assert S.dtproj_status(reset=True) == S.SSM_OK
