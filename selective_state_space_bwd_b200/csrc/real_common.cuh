@@ -29,21 +29,31 @@ __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 // exp2 of both halves on the MUFU unit
 __device__ __forceinline__ float2 ex2_pair(float2 e) { return make_float2(ex2_mufu(e.x), ex2_mufu(e.y)); }
 
-// S consecutive floats from shared / global memory as S/2 pairs (16-byte vector accesses)
+// S consecutive floats from shared / global memory as S/2 pairs (16-byte vector accesses; one
+// 8-byte access for S = 2)
 template <int S>
 __device__ __forceinline__ void ld_pairs(float2 (&o)[S / 2], const float* p) {
+    if constexpr (S == 2) {
+        o[0] = *reinterpret_cast<const float2*>(p);
+    } else {
 #pragma unroll
-    for (int i = 0; i < S / 4; ++i) {
-        const float4 v = reinterpret_cast<const float4*>(p)[i];
-        o[2 * i] = make_float2(v.x, v.y);
-        o[2 * i + 1] = make_float2(v.z, v.w);
+        for (int i = 0; i < S / 4; ++i) {
+            const float4 v = reinterpret_cast<const float4*>(p)[i];
+            o[2 * i] = make_float2(v.x, v.y);
+            o[2 * i + 1] = make_float2(v.z, v.w);
+        }
     }
 }
 template <int S>
 __device__ __forceinline__ void st_pairs(float* p, const float2 (&o)[S / 2]) {
+    if constexpr (S == 2) {
+        *reinterpret_cast<float2*>(p) = o[0];
+    } else {
 #pragma unroll
-    for (int i = 0; i < S / 4; ++i)
-        reinterpret_cast<float4*>(p)[i] = make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
+        for (int i = 0; i < S / 4; ++i)
+            reinterpret_cast<float4*>(p)[i] =
+                make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
+    }
 }
 template <int S>
 __device__ __forceinline__ void st_pairs_cg(float* p, const float2 (&o)[S / 2]) {

@@ -7,8 +7,9 @@
 // backward recomputes from; "Breaking the Memory Wall ... Tiled Operator-Space Evolution",
 // abstract).
 //
-// Work decomposition.  Thread = (channel, 4 consecutive states), state pairs in packed fp32x2
-// arithmetic, NG = N / 4 adjacent lanes per channel, 32 channels per CTA.  Each CTA streams its
+// Work decomposition.  Thread = (channel, S consecutive states), state pairs in packed fp32x2
+// arithmetic, NG = N / S adjacent lanes per channel, 32 channels per CTA; S = 4, or S = 2 when the
+// grid is too small to fill the SMs.  Each CTA streams its
 // time segment through shared memory in 32-step sub-tiles: while sub-tile j is processed, the
 // raw inputs of sub-tile j+1 arrive by asynchronous copies (two-stage ring), so no warp waits on
 // global memory.  Per sub-tile: softplus once per (t, d) into a (delta, delta*x) tile, B and C to
@@ -23,20 +24,23 @@ namespace ssm {
 namespace real {
 namespace {
 
-template <int N>
+// S states per thread: 4 (two packed pairs), or 2 (one pair) for grids too small to fill the SMs,
+// which doubles the warps per SM; the y group of U steps is reduce-scattered over the NG lanes.
+template <int N, int S_>
 struct FwdCfg {
-    static constexpr int S = 4;           // states per thread
+    static constexpr int S = S_;          // states per thread
     static constexpr int P2 = S / 2;      // state pairs per thread
     static constexpr int NG = N / S;      // lanes per channel
     static constexpr int DT = kRealDT;    // channels per CTA
     static constexpr int NT = DT * NG;    // threads per CTA
     static constexpr int TT = 32;         // steps per staged sub-tile
-    static constexpr int U = 4;           // steps per unrolled group
+    static constexpr int U = S == 2 ? 8 : 4;  // steps per unrolled group (>= NG)
+    static_assert(U >= NG, "one y value per lane at least");
 };
 
 template <typename E, int N>
 struct FwdSmem {
-    static constexpr int TT = FwdCfg<N>::TT, DT = FwdCfg<N>::DT;
+    static constexpr int TT = FwdCfg<N, 4>::TT, DT = FwdCfg<N, 4>::DT;
     static constexpr int XE = TT * DT;                                  // elements of an x tile
     static constexpr int BE = TT * N;                                   // elements of a B tile
     static constexpr int STAGE = (2 * XE + 2 * BE) * (int)sizeof(E);    // x, delta_raw, B, C
@@ -49,9 +53,9 @@ struct FwdSmem {
 
 // SUMMARY = true: local scan from zero over segments 0..nseg-2, emitting (prod a, end state).
 // SUMMARY = false: the scan from the segment's entering state, writing y and checkpoints.
-template <typename E, int N, bool SUMMARY, bool ZOH>
-__global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
-    using Cfg = FwdCfg<N>;
+template <typename E, int N, int S, bool SUMMARY, bool ZOH>
+__global__ void __launch_bounds__(FwdCfg<N, S>::NT) real_fwd_kernel(RealArgs p) {
+    using Cfg = FwdCfg<N, S>;
     using Sm = FwdSmem<E, N>;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TT = Cfg::TT, U = Cfg::U;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
         const float* src = p.nseg > 1 ? p.hin + (((size_t)b * p.nseg + seg) * p.D + d) * N + n0
                            : p.h0   ? p.h0 + ((size_t)b * p.D + d) * N + n0
                                     : nullptr;
-        if (src) ld_pairs<4>(h, src);
+        if (src) ld_pairs<S>(h, src);
     }
     const size_t boff = (size_t)b * p.L;
     const E* xb = static_cast<const E*>(p.x) + boff * p.D;
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
                 const int r = r0 + u;
                 const float2 dd = sdd[r * DT + dl];
                 float2 bq[P2];
-                ld_pairs<4>(bq, sBf + r * N + n0);
+                ld_pairs<S>(bq, sBf + r * N + n0);
                 if (SUMMARY) {
 #pragma unroll
                     for (int i = 0; i < P2; ++i) {
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
                     }
                 } else {
                     float2 cq[P2];
-                    ld_pairs<4>(cq, sCf + r * N + n0);
+                    ld_pairs<S>(cq, sCf + r * N + n0);
                     float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
                     for (int i = 0; i < P2; ++i) {
@@ -194,8 +198,8 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
         }
         const bool chunk_end = (t0 + rows) % T == 0 || t0 + rows == p.L;
         if (!SUMMARY && dv && chunk_end) {
-            st_pairs<4>(p.ckpt + (((size_t)b * p.nC + t0 / T) * p.D + d) * N + n0, h);
-            if (p.hL && t0 + rows == p.L) st_pairs<4>(p.hL + ((size_t)b * p.D + d) * N + n0, h);
+            st_pairs<S>(p.ckpt + (((size_t)b * p.nC + t0 / T) * p.D + d) * N + n0, h);
+            if (p.hL && t0 + rows == p.L) st_pairs<S>(p.hL + ((size_t)b * p.D + d) * N + n0, h);
         }
         __syncthreads();
         if (!SUMMARY) store_tile<E, DT>(yb, sy, t0, rows, p.L, d0, p.D, tid, NT);
@@ -203,10 +207,10 @@ __global__ void __launch_bounds__(FwdCfg<N>::NT) real_fwd_kernel(RealArgs p) {
     if (SUMMARY) {
         if (dv) {
             const size_t o = (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N + n0;
-            st_pairs<4>(p.sumP + o, P);
-            st_pairs<4>(p.sumS + o, h);
+            st_pairs<S>(p.sumP + o, P);
+            st_pairs<S>(p.sumS + o, h);
         }
-    } else if (dv && !all_finite<4>(h)) {
+    } else if (dv && !all_finite<S>(h)) {
         flag_status(p.status, kStatusNonFinite);
     }
 }
@@ -233,14 +237,14 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename E, int N, bool ZOH>
+template <typename E, int N, int S, bool ZOH>
 cudaError_t real_fwd_impl(const RealArgs& a, cudaStream_t st) {
-    const dim3 block(FwdCfg<N>::NT);
+    const dim3 block(FwdCfg<N, S>::NT);
     const size_t sm = FwdSmem<E, N>::BYTES;
     cudaError_t e;
     if (a.nseg > 1) {
-        if ((e = set_smem(real_fwd_kernel<E, N, true, ZOH>, sm)) != cudaSuccess) return e;
-        real_fwd_kernel<E, N, true, ZOH><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
+        if ((e = set_smem(real_fwd_kernel<E, N, S, true, ZOH>, sm)) != cudaSuccess) return e;
+        real_fwd_kernel<E, N, S, true, ZOH><<<dim3(a.ndt, a.B, a.nseg - 1), block, sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t n = (int64_t)a.B * a.D * N;
         real_carry_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.B, a.nseg, a.D * N,
@@ -248,16 +252,28 @@ cudaError_t real_fwd_impl(const RealArgs& a, cudaStream_t st) {
                                                                             a.h0);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = set_smem(real_fwd_kernel<E, N, false, ZOH>, sm)) != cudaSuccess) return e;
-    real_fwd_kernel<E, N, false, ZOH><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
+    if ((e = set_smem(real_fwd_kernel<E, N, S, false, ZOH>, sm)) != cudaSuccess) return e;
+    real_fwd_kernel<E, N, S, false, ZOH><<<dim3(a.ndt, a.B, a.nseg), block, sm, st>>>(a);
     return cudaGetLastError();
+}
+
+// Two states per thread when the main launch has fewer CTAs than 3 per SM on 148 SMs (444): the
+// grid then gives under 12 warps per SM at four states per thread, too few to hide the latency
+// of the exp / FMA chain; above that the extra per-step work of the narrower threads costs more
+// than the latency it hides.
+constexpr int64_t kFwdNarrowCtas = 444;
+
+template <typename E, int N, bool ZOH>
+cudaError_t real_fwd_pick(const RealArgs& a, cudaStream_t st) {
+    if ((int64_t)a.ndt * a.B * a.nseg < kFwdNarrowCtas) return real_fwd_impl<E, N, 2, ZOH>(a, st);
+    return real_fwd_impl<E, N, 4, ZOH>(a, st);
 }
 
 template <typename E, bool ZOH>
 cudaError_t fwd_dispatch_n(const RealArgs& a, int N, cudaStream_t st) {
-    if (N == 4) return real_fwd_impl<E, 4, ZOH>(a, st);
-    if (N == 8) return real_fwd_impl<E, 8, ZOH>(a, st);
-    return real_fwd_impl<E, 16, ZOH>(a, st);
+    if (N == 4) return real_fwd_pick<E, 4, ZOH>(a, st);
+    if (N == 8) return real_fwd_pick<E, 8, ZOH>(a, st);
+    return real_fwd_pick<E, 16, ZOH>(a, st);
 }
 
 template <typename E>
