@@ -770,7 +770,8 @@ def main():
     if R:
         d["delta_raw"] = torch.empty_like(d["x"])
         dshape = S.dtproj_shape(w.batch * w.seqlen, w.dim, R)
-        wsp = torch.empty(S.dtproj_workspace_bytes(dshape), dtype=torch.uint8, device=dev)
+        wsp = torch.empty(S.dtproj_workspace_bytes(dshape, True), dtype=torch.uint8, device=dev)
+        wspf = torch.empty(S.dtproj_workspace_bytes(dshape, False), dtype=torch.uint8, device=dev)
     shape = S.real_shape(w.batch, w.seqlen, w.dim, w.dstate, w.chunk,
                          S.SSM_BF16 if w.io == gen.BF16 else S.SSM_F32, args.seg_chunks)
     nC = -(-w.seqlen // w.chunk)
@@ -803,7 +804,8 @@ def main():
     def proj_fwd(dd=None):
         dd = d if dd is None else dd
         if R:
-            S.ssm_dtproj_fwd(dd["u"], dd["w"], dd["bias"], delta_raw=dd["delta_raw"], stream=stream)
+            S.ssm_dtproj_fwd(dd["u"], dd["w"], dd["bias"], delta_raw=dd["delta_raw"], ws=wspf,
+                             stream=stream)
 
     def proj_bwd(dd=None, oo=None):
         dd = d if dd is None else dd

@@ -68,7 +68,7 @@ typedef enum ssm_status {
     SSM_ERR_MISALIGNED = 3,           /* pointer not 16-byte aligned, or dim*sizeof(io) % 16 != 0 */
     SSM_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the size query's answer */
     SSM_ERR_CUDA = 5,                 /* a kernel launch or CUDA runtime call failed */
-    SSM_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (ssm_dtproj_status) */
+    SSM_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (device-side) */
     SSM_ERR_NONFINITE = 7             /* a NaN or Inf reached a carried state (device-side) */
 } ssm_status;
 
@@ -314,7 +314,9 @@ int ssm_pdssm_bwd(const ssm_pdshape* shape, float tau, const float* scores, cons
  *     du[m, r] = sum_d g[m, d] w[d, r],   dw[d, r] = sum_m g[m, d] u[m, r],   dbias[d] = sum_m g[m, d].
  * Tensor-core GEMMs with bf16 operands and fp32 accumulation; delta_raw and du are rounded to bf16
  * once, dw and dbias are fp32.  Layout: u, du [M, R], w [D, R], delta_raw, g [M, D] bf16;
- * bias, dbias [D], dw [D, R] fp32; bias and dbias may be NULL.
+ * bias, dbias [D], dw [D, R] fp32; bias and dbias may be NULL.  The kernels wait on their
+ * tensor-core work through bounded waits; one that gives up writes no output and records
+ * SSM_ERR_TIMEOUT in the workspace status word (ssm_scan_status reads it; each call resets it).
  */
 typedef struct ssm_dtshape {
     int64_t rows;   /* M >= 0 (0 is a valid empty problem), at most 65535 * 128 */
@@ -323,25 +325,22 @@ typedef struct ssm_dtshape {
     int32_t io;     /* SSM_BF16 (the only supported I/O type: SSM_ERR_UNSUPPORTED otherwise) */
 } ssm_dtshape;
 
-/* Workspace bytes of ssm_dtproj_bwd (fp32 partial sums of dw and dbias over splits of 1024 rows:
- * ceil(M / 1024) * D * (R + 1) * 4 bytes, at least 256); 0 for an invalid shape. */
-size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape);
+/* Workspace bytes of ssm_dtproj_fwd (backward == 0: the 256-byte status word) or ssm_dtproj_bwd
+ * (backward != 0: the status word, then fp32 partial sums of dw and dbias over splits of 1024
+ * rows, ceil(M / 1024) * D * (R + 1) * 4 bytes rounded up to 256); 0 for an invalid shape. */
+size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape, int backward);
 
-/* delta_raw = u w^T + bias.  Enqueues 1 kernel.  Returns an ssm_status. */
+/* delta_raw = u w^T + bias.  Enqueues 1 kernel.  ws: caller-owned device workspace of at least
+ * ssm_dtproj_workspace_bytes(shape, 0) bytes, 16-byte aligned.  Returns an ssm_status. */
 int ssm_dtproj_fwd(const ssm_dtshape* shape, const void* u, const void* w, const float* bias,
-                   void* delta_raw, ssm_stream_t stream);
+                   void* delta_raw, void* ws, size_t ws_bytes, ssm_stream_t stream);
 
 /* du, dw, dbias for g = dL/d delta_raw.  Enqueues 3 kernels (du; dw and dbias partial sums;
- * their fixed-order reduction).  Returns an ssm_status. */
+ * their fixed-order reduction).  ws: at least ssm_dtproj_workspace_bytes(shape, 1) bytes.
+ * Returns an ssm_status. */
 int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const void* g,
                    void* du, float* dw, float* dbias, void* ws, size_t ws_bytes,
                    ssm_stream_t stream);
-
-/* Device status of the projection kernels, which wait on their tensor-core MMAs through bounded
- * mbarrier waits: SSM_OK, or SSM_ERR_TIMEOUT once any such wait gave up (the kernel then writes no
- * output) since the last reset.  reset != 0 clears it.  Synchronises `stream`; SSM_ERR_CUDA if the
- * copy fails. */
-int ssm_dtproj_status(int reset, ssm_stream_t stream);
 
 /* Number of kernels one ssm_scan_fwd (backward == 0) / ssm_scan_bwd (backward != 0) call
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */

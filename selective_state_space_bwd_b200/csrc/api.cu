@@ -605,25 +605,30 @@ int dt_splits(const ssm_dtshape* s) {
 }
 }  // namespace
 
-size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape) {
+size_t ssm_dtproj_workspace_bytes(const ssm_dtshape* shape, int backward) {
     if (check_dtshape(shape) != SSM_OK) return 0;
+    if (!backward) return kStatusBytes;
     const size_t b = (size_t)dt_splits(shape) * shape->dim * (shape->rank + 1) * sizeof(float);
-    return b < 256 ? 256 : align256(b);
+    return kStatusBytes + align256(b);
 }
 
 int ssm_dtproj_fwd(const ssm_dtshape* shape, const void* u, const void* w, const float* bias,
-                   void* delta_raw, ssm_stream_t stream) {
+                   void* delta_raw, void* ws, size_t ws_bytes, ssm_stream_t stream) {
     int st = check_dtshape(shape);
     if (st != SSM_OK) return st;
     const size_t M = shape->rows, D = shape->dim, R = shape->rank;
-    const void* ptrs[] = {u, w, delta_raw, bias};
-    const size_t counts[] = {M * R, D * R, M * D, bias ? D : 0};
-    if ((st = check_arrays(ptrs, counts, 4)) != SSM_OK) return st;
+    const void* ptrs[] = {u, w, delta_raw, ws, bias};
+    const size_t counts[] = {M * R, D * R, M * D, 1, bias ? D : 0};
+    if ((st = check_arrays(ptrs, counts, 5)) != SSM_OK) return st;
+    if (ws_bytes < ssm_dtproj_workspace_bytes(shape, 0)) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
     if (M == 0) return SSM_OK;
     ssm::DtArgs a = {};
     a.M = (int64_t)M; a.D = (int64_t)D; a.R = (int)R;
     a.u = u; a.w = w; a.bias = bias; a.delta_raw = delta_raw;
-    return ssm::launch_dtproj_fwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_dtproj_fwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const void* g,
@@ -635,8 +640,9 @@ int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const
     const void* ptrs[] = {u, w, g, du, dw, ws, dbias};
     const size_t counts[] = {M * R, D * R, M * D, M * R, D * R, 1, dbias ? D : 0};
     if ((st = check_arrays(ptrs, counts, 7)) != SSM_OK) return st;
-    if (ws_bytes < ssm_dtproj_workspace_bytes(shape)) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < ssm_dtproj_workspace_bytes(shape, 1)) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
     if (M == 0) {  // no rows: the sums are empty
         if (cudaMemsetAsync(dw, 0, D * R * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
         if (dbias && cudaMemsetAsync(dbias, 0, D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
@@ -645,15 +651,9 @@ int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const
     ssm::DtArgs a = {};
     a.M = (int64_t)M; a.D = (int64_t)D; a.R = (int)R; a.splits = dt_splits(shape);
     a.u = u; a.w = w; a.g = g; a.du = du; a.dw = dw; a.dbias = dbias;
-    a.part = static_cast<float*>(ws);
+    a.part = at<float>(ws, kStatusBytes);
+    a.status = at<unsigned>(ws, 0);
     return ssm::launch_dtproj_bwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
-}
-
-int ssm_dtproj_status(int reset, ssm_stream_t stream) {
-    unsigned v = 0;
-    if (ssm::dtproj_read_status(&v, reset != 0, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    return v ? SSM_ERR_TIMEOUT : SSM_OK;
 }
 
 int ssm_scan_status(const void* ws, ssm_stream_t stream) {

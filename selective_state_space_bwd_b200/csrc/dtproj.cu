@@ -35,9 +35,6 @@ constexpr int NTH = 128;   // 4 warps: loaders and epilogue; thread 0 also issue
 constexpr int A_BYTES = TM * 128;          // one A stage (either layout)
 constexpr unsigned kSpinLimit = 1u << 20;  // bounded mbarrier waits (well above any MMA)
 
-// Set (never cleared by a kernel) when a bounded wait gave up; read by ssm_dtproj_status.
-__device__ unsigned int g_dtp_status;
-
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
     return (unsigned)__cvta_generic_to_shared(p);
 }
@@ -159,6 +156,7 @@ struct TcArgs {
     int64_t ones_out;        // EPI_F32_PART: data columns below it; the column sums (dbias) go to it
     void* C;                 // EPI_F32_PART: [split][N][M] fp32; else [M][N] bf16
     const float* bias;
+    unsigned* status;        // workspace status word: SSM_ERR_TIMEOUT when a bounded wait gives up
 };
 
 __host__ __device__ constexpr int tmem_cols(int bn) {
@@ -356,7 +354,7 @@ __global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUt
             }
         }
     } else if (tid == 0) {
-        atomicOr(&g_dtp_status, 1u);
+        flag_status(p.status, kStatusTimeout);
         mbar_wait(done, 0);  // the MMAs already issued get a last bounded chance to finish
     }
     tc_fence_before();
@@ -519,7 +517,7 @@ __global__ void __launch_bounds__(FWD_NTH) dtp_fwd_kernel(const __grid_constant_
             drain(T - 1);
         }
     } else if (tid == 0) {
-        atomicOr(&g_dtp_status, 1u);
+        flag_status(p.status, kStatusTimeout);
         // the MMAs already issued get a last bounded chance to finish
         if (T > 0) mbar_wait(acc + 8 * ((T - 1) & 1), (unsigned)(((T - 1) >> 1) & 1));
     }
@@ -631,18 +629,6 @@ cudaError_t run_fwd(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensor
 // Rows of one dw / dbias split (a multiple of the 64-row stage)
 int64_t dtproj_rows_per_split(int) { return 1024; }
 
-cudaError_t dtproj_read_status(unsigned* status, bool reset, cudaStream_t st) {
-    cudaError_t e = cudaMemcpyFromSymbolAsync(status, g_dtp_status, sizeof(unsigned), 0,
-                                              cudaMemcpyDeviceToHost, st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e == cudaSuccess && reset) {
-        static const unsigned zero = 0;
-        e = cudaMemcpyToSymbolAsync(g_dtp_status, &zero, sizeof(unsigned), 0, cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    }
-    return e;
-}
-
 cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     // delta_raw [M x D] = u [M x R] . w [D x R]^T + bias: both operands k-major
     const int ka = (d.R + 63) / 64;              // 64-deep k atoms covering R, all in one stage
@@ -657,6 +643,7 @@ cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     a.ones_out = d.D;
     a.C = d.delta_raw;
     a.bias = d.bias;
+    a.status = d.status;
     switch (ka) {
         case 1: return run_fwd<1, 128>(mA, mB, mC, a, st);
         case 2: return run_fwd<2, 128>(mA, mB, mC, a, st);
@@ -680,6 +667,7 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     a.M = d.M; a.N = d.R; a.K = d.D; a.ldc = d.R; a.kchunk = d.D;
     a.ones_out = d.R;
     a.C = d.du;
+    a.status = d.status;
     switch ((d.R + 63) / 64) {  // 64-wide n blocks covering R
         case 1: e = run_tc<false, true, 64, 8, false, EPI_BF16>(gK, wN, a, 1, st); break;
         case 2: e = run_tc<false, true, 128, 6, false, EPI_BF16>(gK, wN, a, 1, st); break;
@@ -693,6 +681,7 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     b.M = d.D; b.N = d.R + 1; b.K = d.M; b.ldc = 0; b.kchunk = dtproj_rows_per_split(d.R);
     b.ones_out = d.R;
     b.C = d.part;
+    b.status = d.status;
     switch ((d.R + 63) / 64) {
         case 1: e = run_tc<true, true, 64, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
         case 2: e = run_tc<true, true, 128, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;

@@ -12,6 +12,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Status codes written into the workspace status word (mirror of ssm_status in ssm_scan.h).
+constexpr unsigned kStatusTimeout = 6u;
 constexpr unsigned kStatusNonFinite = 7u;
 
 __device__ __forceinline__ void flag_status(unsigned* status, unsigned code) {

@@ -141,11 +141,9 @@ struct DtArgs {
     float* dw;
     float* dbias;
     float* part;
+    unsigned* status;  // workspace status word (SSM_ERR_TIMEOUT when a bounded wait gave up)
 };
 int64_t dtproj_rows_per_split(int R);
-// Copies (and with reset clears) the projection kernels' device status: nonzero once a bounded
-// wait gave up.  Synchronises the stream.
-cudaError_t dtproj_read_status(unsigned* status, bool reset, cudaStream_t st);
 cudaError_t launch_dtproj_fwd(const DtArgs& a, cudaStream_t st);
 cudaError_t launch_dtproj_bwd(const DtArgs& a, cudaStream_t st);
 

@@ -73,7 +73,7 @@ EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_works
             "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
             "ssm_pdssm_workspace_bytes", "ssm_pdssm_fwd", "ssm_pdssm_bwd",
             "ssm_pdssm_kernel_launches", "ssm_dtproj_workspace_bytes", "ssm_dtproj_fwd",
-            "ssm_dtproj_bwd", "ssm_dtproj_status"]
+            "ssm_dtproj_bwd"]
 
 
 def lib():
@@ -120,11 +120,10 @@ def lib():
             L.ssm_pdssm_bwd.restype = I
             L.ssm_pdssm_kernel_launches.argtypes, L.ssm_pdssm_kernel_launches.restype = [PP, I], I
             DP = ctypes.POINTER(SsmDtShape)
-            L.ssm_dtproj_workspace_bytes.argtypes, L.ssm_dtproj_workspace_bytes.restype = [DP], Z
-            L.ssm_dtproj_fwd.argtypes, L.ssm_dtproj_fwd.restype = [DP] + [P] * 4 + [P], I
+            L.ssm_dtproj_workspace_bytes.argtypes, L.ssm_dtproj_workspace_bytes.restype = [DP, I], Z
+            L.ssm_dtproj_fwd.argtypes, L.ssm_dtproj_fwd.restype = [DP] + [P] * 5 + [Z, P], I
             L.ssm_dtproj_bwd.argtypes = [DP] + [P] * 7 + [Z, P]
             L.ssm_dtproj_bwd.restype = I
-            L.ssm_dtproj_status.argtypes, L.ssm_dtproj_status.restype = [I, P], I
             OP = ctypes.POINTER(SsmOptions)
             L.ssm_scan_fwd_ex.argtypes = [SP, OP] + [P] * 9 + [Z, P]
             L.ssm_scan_fwd_ex.restype = I
@@ -443,13 +442,14 @@ def dtproj_shape(rows, dim, rank, io=SSM_BF16):
     return SsmDtShape(int(rows), int(dim), int(rank), int(io))
 
 
-def dtproj_workspace_bytes(shape: SsmDtShape) -> int:
-    return int(lib().ssm_dtproj_workspace_bytes(ctypes.byref(shape)))
+def dtproj_workspace_bytes(shape: SsmDtShape, backward: bool = True) -> int:
+    return int(lib().ssm_dtproj_workspace_bytes(ctypes.byref(shape), 1 if backward else 0))
 
 
-def ssm_dtproj_fwd(u, w, bias=None, delta_raw=None, stream=None):
+def ssm_dtproj_fwd(u, w, bias=None, delta_raw=None, ws=None, stream=None):
     """Step-size projection delta_raw = u w^T + bias.  u [..., R] and w [D, R] bf16, bias [D] fp32
-    (or None).  Returns delta_raw [..., D] bf16."""
+    (or None).  Returns delta_raw [..., D] bf16.  ``ws`` (optional) holds the status word that
+    ssm_scan_status reads."""
     _need_cuda(u, w, bias)
     R = u.shape[-1]
     D = w.shape[0]
@@ -457,8 +457,9 @@ def ssm_dtproj_fwd(u, w, bias=None, delta_raw=None, stream=None):
     shape = dtproj_shape(M, D, R, _io_of(u))
     if delta_raw is None:
         delta_raw = torch.empty((*u.shape[:-1], D), dtype=u.dtype, device=u.device)
-    code = lib().ssm_dtproj_fwd(ctypes.byref(shape), _p(u), _p(w), _p(bias), _p(delta_raw),
-                                _stream(stream))
+    ws = _workspace(dtproj_workspace_bytes(shape, False), u.device, ws)
+    code = lib().ssm_dtproj_fwd(ctypes.byref(shape), _p(u), _p(w), _p(bias), _p(delta_raw), _p(ws),
+                                ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_dtproj_fwd")
     return delta_raw
 
@@ -474,14 +475,10 @@ def ssm_dtproj_bwd(u, w, g, want_dbias=True, out=None, ws=None, stream=None):
     if out is None:
         out = dict(du=torch.empty_like(u), dw=torch.empty((D, R), dtype=torch.float32, device=u.device),
                    dbias=torch.empty(D, dtype=torch.float32, device=u.device) if want_dbias else None)
-    ws = _workspace(dtproj_workspace_bytes(shape), u.device, ws)
+    ws = _workspace(dtproj_workspace_bytes(shape, True), u.device, ws)
     code = lib().ssm_dtproj_bwd(ctypes.byref(shape), _p(u), _p(w), _p(g), _p(out["du"]),
                                 _p(out["dw"]), _p(out.get("dbias")), _p(ws),
                                 ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_dtproj_bwd")
     return out
 
-
-def dtproj_status(reset=False, stream=None) -> int:
-    """SSM_OK, or SSM_ERR_TIMEOUT once a projection kernel's bounded wait gave up (synchronises)."""
-    return int(lib().ssm_dtproj_status(1 if reset else 0, _stream(stream)))

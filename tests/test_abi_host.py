@@ -256,18 +256,21 @@ def test_dtproj_validation(S):
     import ctypes
     L = S.lib()
     ok = S.dtproj_shape(1000, 1536, 48)
-    assert S.dtproj_workspace_bytes(ok) == 1536 * 49 * 4  # one split of 1024 rows, R + 1 columns
-    assert S.dtproj_workspace_bytes(S.dtproj_shape(3000, 64, 128)) == 3 * 64 * 129 * 4
+    # status word (256 bytes), then one split of 1024 rows x (R + 1) columns x D
+    assert S.dtproj_workspace_bytes(ok) == 256 + 1536 * 49 * 4
+    assert S.dtproj_workspace_bytes(ok, backward=False) == 256
+    assert S.dtproj_workspace_bytes(S.dtproj_shape(3000, 64, 128)) == 256 + 3 * 64 * 129 * 4
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1536, 40)) == 0   # R not a multiple of 16
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 1532, 48)) == 0   # D not a multiple of 8
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 64, 272)) == 0    # R > 256
     assert S.dtproj_workspace_bytes(S.dtproj_shape(10, 64, 16, S.SSM_F32)) == 0
     assert S.dtproj_workspace_bytes(S.dtproj_shape(0, 64, 16)) == 256
-    p16 = [ctypes.c_void_p(4096)] * 4
-    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 16, S.SSM_F32)), *p16, None) == 2
-    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 40)), *p16, None) == 2
-    assert L.ssm_dtproj_fwd(ctypes.byref(ok), None, *p16[:3], None) == 1       # u missing
-    odd = [ctypes.c_void_p(4096), ctypes.c_void_p(4104), ctypes.c_void_p(4096), None]
-    assert L.ssm_dtproj_fwd(ctypes.byref(ok), *odd, None) == 3                 # w misaligned
+    p16 = [ctypes.c_void_p(4096)] * 5
+    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 16, S.SSM_F32)), *p16, 256, None) == 2
+    assert L.ssm_dtproj_fwd(ctypes.byref(S.dtproj_shape(10, 64, 40)), *p16, 256, None) == 2
+    assert L.ssm_dtproj_fwd(ctypes.byref(ok), None, *p16[:4], 256, None) == 1       # u missing
+    odd = [ctypes.c_void_p(4096), ctypes.c_void_p(4104), ctypes.c_void_p(4096), None, ctypes.c_void_p(4096)]
+    assert L.ssm_dtproj_fwd(ctypes.byref(ok), *odd, 256, None) == 3                 # w misaligned
+    assert L.ssm_dtproj_fwd(ctypes.byref(ok), *p16, 255, None) == 4                 # workspace
     pb = [ctypes.c_void_p(4096)] * 7
-    assert L.ssm_dtproj_bwd(ctypes.byref(ok), *pb, 255, None) == 4             # workspace
+    assert L.ssm_dtproj_bwd(ctypes.byref(ok), *pb, 255, None) == 4                  # workspace

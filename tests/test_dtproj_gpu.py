@@ -98,10 +98,14 @@ def test_projection_scan_pipeline(S, oracle_mod):
 
 
 def test_dtproj_status_clean(S):
-    """No bounded tensor-core wait of the projection kernels gave up in this process."""
+    """No bounded tensor-core wait of the projection kernels gives up: the workspace status word
+    reads SSM_OK after each call."""
     p = gen.dtproj_inputs(2, 700, 320, 64, seed=11)
     u, w, g = bf(p["u"]), bf(p["w"]), bf(p["g"])
-    S.ssm_dtproj_fwd(u, w, torch.from_numpy(p["bias"]).cuda())
-    S.ssm_dtproj_bwd(u, w, g)
-    assert S.dtproj_status() == S.SSM_OK
-    assert S.dtproj_status(reset=True) == S.SSM_OK
+    shp = S.dtproj_shape(2 * 700, 320, 64)
+    wsf = torch.full((S.dtproj_workspace_bytes(shp, False),), 0xFF, dtype=torch.uint8, device="cuda")
+    wsb = torch.full((S.dtproj_workspace_bytes(shp, True),), 0xFF, dtype=torch.uint8, device="cuda")
+    S.ssm_dtproj_fwd(u, w, torch.from_numpy(p["bias"]).cuda(), ws=wsf)
+    assert S.ssm_scan_status(wsf) == S.SSM_OK  # the call reset the word, no wait gave up
+    S.ssm_dtproj_bwd(u, w, g, ws=wsb)
+    assert S.ssm_scan_status(wsb) == S.SSM_OK
