@@ -112,9 +112,11 @@ __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __re
 //   pass B: stream the sub-tiles in reverse.  For each 4-step window, last first: recompute
 //           (a_t, a_t h_{t-1}) forward from the window's start state into registers, then sweep
 //           the adjoint back through the window.
+//           After each step: the step's dB / dC values (4 states each) summed over the warp's
+//           channels by a shuffle reduce-scatter that leaves one (dB or dC, state) sum per lane.
 //           After each window: reduce-scatter of the per-channel sums over the NG lanes, dx and
-//           ddelta_raw stored directly, and the window's dB / dC values (double-buffered shared
-//           memory) summed over the CTA's 32 channels into its partial-sum rows.
+//           ddelta_raw stored directly, and the warps' dB / dC sums (double-buffered shared
+//           memory, one 16-byte store per lane) added over the CTA's warps into its partial rows.
 template <int N>
 struct BwdCfg {
     static constexpr int S = 4;            // states per thread
@@ -124,16 +126,7 @@ struct BwdCfg {
     static constexpr int NT = DT * NG;     // threads per CTA
     static constexpr int W = 4;            // steps per window
     static constexpr int TT = 32;          // steps per staged sub-tile
-    static constexpr int Q = NT / (2 * N); // channel parts in the dB/dC column sums
 };
-
-// Quad swizzle of the dB/dC rows: a quarter-warp (8 lanes) covers 32/N channels; channel rows are
-// N/2 quads long, so rows 16/N apart start on the same bank.  XOR-ing the quad index with N/4 for
-// every other such group spreads the quarter-warp over all 32 banks.
-template <int N>
-__host__ __device__ constexpr int red_swz(int ch) {
-    return ((ch / (16 / N)) & 1) * (N / 4);
-}
 
 template <typename E, int N>
 struct BwdSmem {
@@ -148,8 +141,8 @@ struct BwdSmem {
     static constexpr int B_STAGE = XE * 8 + (2 * XE + 2 * BE) * (int)sizeof(E);
     static constexpr int B_BF = 2 * B_STAGE;              // B fp32
     static constexpr int B_CF = B_BF + BE * 4;            // C fp32
-    static constexpr int B_RED = B_CF + BE * 4;           // dB/dC values, 2 x [W][DT][2N]
-    static constexpr int B_END = B_RED + 2 * W * DT * 2 * N * 4;
+    static constexpr int B_RED = B_CF + BE * 4;           // warp sums of dB/dC, 2 x [warps][W][2N]
+    static constexpr int B_END = B_RED + 2 * (BwdCfg<N>::NT / 32) * 2 * N * W * 4;
     static constexpr int BYTES = A_END > B_END ? A_END : B_END;
 };
 
@@ -161,7 +154,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
     // per-step channel sums over the states: sum g w' B (dx), sum A q, and for zero-order hold
     // also sum g a B (ddelta; with Euler it equals the first)
     constexpr int SV = ZOH ? 3 : 2;
-    constexpr int TT = Cfg::TT, Q = Cfg::Q, N2 = 2 * N;
+    constexpr int TT = Cfg::TT, N2 = 2 * N;
     extern __shared__ __align__(16) unsigned char smem[];
 
     const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
@@ -172,10 +165,6 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
     const int TTe = T < TT ? T : TT;
     const int c_begin = seg * p.seg_chunks;
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
-    // column-sum roles: `cs_part` sums channels [cs_part*DT/Q, ...) of output quad `cs_quad`
-    const int cs_part = (tid >> 3) % Q;
-    const int cs_quad = (tid & 7) + 8 * (tid / (8 * Q));
-    const int cs_u = cs_quad / (N2 / 4), cs_o = 4 * (cs_quad % (N2 / 4));
 
     float2 A[P2], A2[P2], v[P2], dA[P2];
     float2 Ar[P2];  // zero-order hold: 1 / A
@@ -368,35 +357,16 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
                             dDacc = fmaf(dyv, xv, dDacc);
                         }
                     }
-                    __syncthreads();  // the window's dB/dC values are in `red`
-                    const float* src = red + (cs_u * DT + cs_part * (DT / Q)) * N2;
-                    const int cq = cs_o >> 2;
-                    float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
+                    __syncthreads();  // the warps' dB/dC sums of the window are in `red`
+                    {
+                        // output (step u, dB or dC, state n) = sum over the warps
+                        const int u = tid / N2, wh = (tid / N) % 2, n = tid % N;
+                        float s = 0.0f;
 #pragma unroll
-                    for (int ch = 0; ch < DT / Q; ch += 2) {
-                        // DT / Q is a multiple of 8, so the swizzle of channel ch is red_swz(ch)
-                        const float4 a0 = *reinterpret_cast<const float4*>(
-                            src + ch * N2 + 4 * (cq ^ red_swz<N>(ch)));
-                        const float4 a1 = *reinterpret_cast<const float4*>(
-                            src + (ch + 1) * N2 + 4 * (cq ^ red_swz<N>(ch + 1)));
-                        s0 = __fadd2_rn(s0, make_float2(a0.x, a0.y));
-                        s1 = __fadd2_rn(s1, make_float2(a0.z, a0.w));
-                        s2 = __fadd2_rn(s2, make_float2(a1.x, a1.y));
-                        s3 = __fadd2_rn(s3, make_float2(a1.z, a1.w));
+                        for (int w = 0; w < NT / 32; ++w) s += red[(w * W + u) * N2 + wh * N + n];
+                        const int r = q * W + u;
+                        if (r < rows) partb[(size_t)(t0 + r) * N2 + wh * N + n] = s;
                     }
-                    s0 = __fadd2_rn(s0, s2);
-                    s1 = __fadd2_rn(s1, s3);
-#pragma unroll
-                    for (int m = 8; m < 8 * Q; m <<= 1) {
-                        s0.x += __shfl_xor_sync(kFull, s0.x, m);
-                        s0.y += __shfl_xor_sync(kFull, s0.y, m);
-                        s1.x += __shfl_xor_sync(kFull, s1.x, m);
-                        s1.y += __shfl_xor_sync(kFull, s1.y, m);
-                    }
-                    const int r = q * W + cs_u;
-                    if (cs_part == 0 && r < rows)
-                        *reinterpret_cast<float4*>(partb + (size_t)(t0 + r) * N2 + cs_o) =
-                            make_float4(s0.x, s0.y, s1.x, s1.y);
                 };
 
                 // windows in reverse: recompute (a_t, a_t h_{t-1}) forward from the window's start
@@ -434,7 +404,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
                         }
                     }
                     float sv[SV * W];
-                    float* red = sred + (q & 1) * W * DT * N2;
+                    float* red = sred + (q & 1) * (NT / 32) * 2 * N * W;
+                    float dbc[W];  // this lane's channel-summed dB or dC element, per step
 #pragma unroll
                     for (int uu = W - 1; uu >= 0; --uu) {
                         const int r = q * W + uu;
@@ -478,12 +449,43 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) 
                         sv[SV * uu] = sg.x + sg.y;
                         sv[SV * uu + 1] = sa.x + sa.y;
                         if constexpr (ZOH) sv[SV * uu + 2] = sga.x + sga.y;
-                        // rows of 2N floats; odd channel groups swap their dB and dC halves so
-                        // that a quarter-warp's 16-byte stores fall in distinct banks
-                        float* sr = red + (uu * DT + dl) * N2;
-                        const int sw = red_swz<N>(dl);
-                        st_pairs<4>(sr + 4 * (ng ^ sw), rB);
-                        st_pairs<4>(sr + 4 * ((NG + ng) ^ sw), rC);
+                        // sum over the warp's channels (lane bits above the NG state lanes):
+                        // the first three halvings scatter the 8 values (dB, dC of 4 states) so
+                        // that lane element e = (lane >> 2) & 7 remains, further ones just sum
+                        {
+                            float vv[8] = {rB[0].x, rB[0].y, rB[1].x, rB[1].y,
+                                           rC[0].x, rC[0].y, rC[1].x, rC[1].y};
+                            int c = 8;
+#pragma unroll
+                            for (int m = 16; m >= NG; m >>= 1) {
+                                if (c > 1) {
+                                    const bool up = (threadIdx.x & m) != 0;
+                                    const int h = c / 2;
+#pragma unroll
+                                    for (int i2 = 0; i2 < 4; ++i2) {
+                                        if (i2 < h) {
+                                            const float send = up ? vv[i2] : vv[i2 + h];
+                                            const float keep = up ? vv[i2 + h] : vv[i2];
+                                            vv[i2] = keep + __shfl_xor_sync(kFull, send, m);
+                                        }
+                                    }
+                                    c = h;
+                                } else {
+                                    vv[0] += __shfl_xor_sync(kFull, vv[0], m);
+                                }
+                            }
+                            dbc[uu] = vv[0];
+                        }
+                    }
+                    {
+                        const int lane = tid & 31, e = (lane >> 2) & 7;
+                        // one lane per (dB or dC, state) writes the warp's sums of the window's
+                        // steps: rows of 2N floats, a warp's lanes contiguous
+                        if ((lane & 3 & ~(NG - 1)) == 0) {
+                            float* wr = red + (tid >> 5) * W * N2 + (e >> 2) * N + ng * 4 + (e & 3);
+#pragma unroll
+                            for (int u = 0; u < W; ++u) wr[u * N2] = dbc[u];
+                        }
                     }
                     finish_window(q, sv, red);
                 }
