@@ -13,8 +13,8 @@ constexpr int kTargetCtas = 296;  // 2 x 148 SMs: below this many CTAs, split ti
 // Real forward, once split: enough segments for about 2368 CTAs (two waves at the eight CTAs per
 // SM its registers and shared memory allow), so that every SM keeps several CTAs busy.
 constexpr int64_t kRealFwdSplitCtas = 2368;
-// Real backward: 3 CTAs per SM (registers and shared memory) on 148 SMs
-constexpr int64_t kRealBwdSlots = 444;
+// Real backward: 4 CTAs per SM (126 registers per thread, 37 KB of shared memory) on 148 SMs
+constexpr int64_t kRealBwdSlots = 592;
 // Real backward: per-launch bound on the per-CTA scratch (window-start states, (delta, sigma))
 constexpr size_t kRealBwdScratchCap = (size_t)192 << 20;
 

@@ -147,7 +147,7 @@ struct BwdSmem {
 };
 
 template <typename E, int N, bool ZOH>
-__global__ void __launch_bounds__(BwdCfg<N>::NT, 3) real_bwd_kernel(RealArgs p) {
+__global__ void __launch_bounds__(BwdCfg<N>::NT, ZOH ? 3 : 4) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N>;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;

@@ -229,10 +229,14 @@ def test_kernel_launch_counts(S):
     # caps: summary + carry + 4 x (main + reduce) + params = 11
     split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
     assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 11
-    # 512 CTAs would leave a second wave of 68 CTAs on 444 slots: 16 concurrent segments of
-    # 4 chunks instead, 4 per launch
+    # 512 CTAs fit one wave (4 CTAs per SM on 148 SMs = 592 slots): no time split, time in 4
+    # sequential blocks under the partial cap
     wave = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)
-    assert S.kernel_launches(wave, False) == 1 and S.kernel_launches(wave, True) == 11
+    assert S.kernel_launches(wave, False) == 1 and S.kernel_launches(wave, True) == 9
+    # 640 CTAs would leave a second wave of 48 on 592 slots: 16 concurrent segments of 4 chunks
+    # instead, 3 per launch (summary + carry + 6 x (main + reduce) + params)
+    part = S.real_shape(5, 8192, 4096, 16, 128, S.SSM_BF16)
+    assert S.kernel_launches(part, True) == 15
     # wide enough to fill the SMs: no split; time in 4 sequential blocks under the partial cap
     blocks = S.real_shape(16, 2048, 4096, 16, 128, S.SSM_BF16)
     assert S.kernel_launches(blocks, False) == 1 and S.kernel_launches(blocks, True) == 9
