@@ -146,8 +146,11 @@ struct BwdSmem {
     static constexpr int BYTES = A_END > B_END ? A_END : B_END;
 };
 
-template <typename E, int N, bool ZOH>
-__global__ void __launch_bounds__(BwdCfg<N>::NT, ZOH ? 3 : 4) real_bwd_kernel(RealArgs p) {
+// MINB: CTAs per SM the register allocation must allow.  4 (126 registers for the Euler N = 16
+// kernel) lets grids of up to 592 CTAs run in one wave; 3 leaves the compiler more registers,
+// which is 2 % faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
+template <typename E, int N, bool ZOH, int MINB>
+__global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N>;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;
@@ -581,7 +584,9 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const size_t sm = BwdSmem<E, N>::BYTES;
-    if ((e = set_smem(real_bwd_kernel<E, N, ZOH>, sm)) != cudaSuccess) return e;
+    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3>, sm)) != cudaSuccess) return e;
+    if constexpr (N == 16 && !ZOH)
+        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4>, sm)) != cudaSuccess) return e;
     const int per = a.seq_blocks ? 1 : group;
     for (int hi = a.nseg; hi > 0; hi -= per) {
         const int lo = hi - per > 0 ? hi - per : 0;
@@ -589,7 +594,15 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         a.part_t0 = lo * a.seg_chunks * a.T;
         const int t_hi = min(a.L, hi * a.seg_chunks * a.T);
         const int rows = t_hi - a.part_t0;
-        real_bwd_kernel<E, N, ZOH><<<dim3(a.ndt, a.B, hi - lo), dim3(BwdCfg<N>::NT), sm, st>>>(a);
+        const dim3 grid(a.ndt, a.B, hi - lo);
+        bool wide = false;  // more CTAs than 3 per SM on 148 SMs
+        if constexpr (N == 16 && !ZOH) wide = (int64_t)a.ndt * a.B * (hi - lo) > 444;
+        if (wide) {
+            if constexpr (N == 16 && !ZOH)
+                real_bwd_kernel<E, N, ZOH, 4><<<grid, dim3(BwdCfg<N>::NT), sm, st>>>(a);
+        } else {
+            real_bwd_kernel<E, N, ZOH, 3><<<grid, dim3(BwdCfg<N>::NT), sm, st>>>(a);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t nbc = (int64_t)a.B * rows * 2 * N;
         if (nbc > 0) {
