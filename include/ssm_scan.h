@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define SSM_SCAN_ABI_VERSION 2
+#define SSM_SCAN_ABI_VERSION 3  /* 3: ssm_dtproj_fwd takes a workspace (its status word) */
 
 /* Same underlying type as cudaStream_t (NULL = the legacy default stream). */
 typedef struct CUstream_st* ssm_stream_t;

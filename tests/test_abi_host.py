@@ -44,7 +44,7 @@ def test_exports_every_declared_symbol(S):
 
 def test_abi_version_and_status_strings(S):
     L = S.lib()
-    assert L.ssm_scan_abi_version() == 2
+    assert L.ssm_scan_abi_version() == 3
     for code in range(8):
         assert L.ssm_status_string(code).decode().startswith(S.STATUS_NAMES[code])
     assert L.ssm_status_string(99) == b"unknown ssm_status"
