@@ -147,7 +147,8 @@ __host__ __device__ constexpr unsigned idesc_bf16(int n, bool a_mn, bool b_mn) {
            ((unsigned)(n >> 3) << 17) | ((unsigned)(TM >> 4) << 24);
 }
 
-enum Epi { EPI_BIAS_BF16 = 0, EPI_BF16 = 1, EPI_F32_PART = 2 };
+// k-loop kernel epilogues: bf16 rows of C, or fp32 partial sums of one split
+enum Epi { EPI_BF16 = 1, EPI_F32_PART = 2 };
 
 struct TcArgs {
     int64_t M, N, K;         // logical C [M][N] = sum_k A(m, k) B(n, k); N counts the column sums
