@@ -244,22 +244,32 @@ def oracle_sample(w, inp, budget_s=(10.0, 30.0), zoh=False):
                       f"fwd+bwd in float64, {t_total:.1f} s"}
 
 
+def code_digest(path):
+    """sha256 of a C++/CUDA source's code: `//` comments, surrounding blanks and empty lines
+    dropped, so that an edit of the comments alone keeps a traffic record valid."""
+    import hashlib
+    lines = []
+    for line in open(path, encoding="utf-8").read().splitlines():
+        code = line.split("//", 1)[0].strip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def measured_traffic(call, kernel_file, workload):
     """DRAM bytes per launch of `call` (its kernels summed) on `workload`, from the committed ncu
-    capture records, if that capture was taken on the current source of `kernel_file`; else None.
+    capture records, if that capture was taken on the current code of `kernel_file`; else None.
     A record captured on a smaller case of the same launch plan carries the factor that scales
     it to the full workload's units."""
-    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         recs = json.load(open(p))["records"]
-        src = open(os.path.join(ROOT, "selective_state_space_bwd_b200", "csrc", kernel_file), "rb").read()
-        sha = hashlib.sha256(src).hexdigest()
+        sha = code_digest(os.path.join(ROOT, "selective_state_space_bwd_b200", "csrc", kernel_file))
         for rec in recs:
             if (rec["workload"] == workload and rec["call"] == call and rec["source"] == kernel_file
-                    and rec["source_sha256"] == sha):
+                    and rec["code_sha256"] == sha):
                 return float(rec["dram_bytes_per_launch"])
         return None
     except (OSError, ValueError, KeyError, TypeError):
