@@ -556,16 +556,17 @@ __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, in
         dbias[d] = s;
 }
 
-// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no link to libcuda)
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no link to libcuda);
+// looked up once (thread-safe initialisation of the function-local static)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        return nullptr;
+    }();
     return fn;
 }
 
