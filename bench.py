@@ -170,7 +170,8 @@ E2E_OVERLAP = ("two buffer sets; each step's host-to-device and device-to-host c
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs.  The raw
+    samples go to clocks_rank<i>.csv in $SSM_BENCH_CLOCKS_DIR (default: the system temp dir)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -179,7 +180,9 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        import tempfile
+        out = os.environ.get("SSM_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out, f"clocks_rank{index}.csv")
 
     def start(self):
         try:
