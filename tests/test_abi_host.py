@@ -278,3 +278,22 @@ def test_dtproj_validation(S):
     assert L.ssm_dtproj_fwd(ctypes.byref(ok), *p16, 255, None) == 4                 # workspace
     pb = [ctypes.c_void_p(4096)] * 7
     assert L.ssm_dtproj_bwd(ctypes.byref(ok), *pb, 255, None) == 4                  # workspace
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    """include/ssm_scan.h is a plain C header (usable from C and C++ callers alike)."""
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "ssm_scan.h"\n'
+                   "int main(void) {\n"
+                   "    ssm_shape s = {1, 16, 8, 4, 128, SSM_F32, 0, 0};\n"
+                   "    ssm_dtshape d = {0, 8, 16, SSM_BF16};\n"
+                   "    return (int)(ssm_scan_checkpoint_bytes(&s) * 0 + ssm_dtproj_workspace_bytes(&d, 0) * 0);\n"
+                   "}\n")
+    inc = os.path.join(ROOT, "include")
+    for cmd in (["gcc", "-std=c11", "-Wall", "-Werror", "-I", inc, "-c", str(src), "-o", str(tmp_path / "a.o")],
+                ["g++", "-std=c++17", "-Wall", "-Werror", "-I", inc, "-x", "c++", "-c", str(src),
+                 "-o", str(tmp_path / "b.o")]):
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
