@@ -404,7 +404,7 @@ def main_complex(args, w):
     """The complex-mode (shared retention/phase) scan: ssm_scan_complex_fwd + _bwd per step."""
     import torch
     import torch.distributed as dist
-    from selective_state_space_bwd_b200 import build, ssm_scan as S
+    from selective_state_space_bwd_b200 import build, dp, ssm_scan as S
     from selective_state_space_bwd_b200 import inputs as gen
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -461,11 +461,7 @@ def main_complex(args, w):
     def allreduce(bs=None):
         oo = (bs or sets[0])["out"]
         if world > 1:  # dlambda, domega sum over the batch rows of every rank
-            gbuf[:w.modes].copy_(oo["dlambda"])
-            gbuf[w.modes:].copy_(oo["domega"])
-            dist.all_reduce(gbuf)
-            oo["dlambda"].copy_(gbuf[:w.modes])
-            oo["domega"].copy_(gbuf[w.modes:])
+            dp.allreduce_grads([oo["dlambda"], oo["domega"]], buf=gbuf)
 
     for _ in range(max(3, args.warmup)):
         fwd(); bwd(); allreduce()
@@ -850,17 +846,9 @@ def main():
 
     def allreduce(oo=None):
         oo = out if oo is None else oo
-        if world > 1:
-            if R:  # the projection's parameter gradients travel in the same collective
-                n1, n2 = w.dim * w.dstate + w.dim, w.dim * R
-                gbuf[n1:n1 + n2].copy_(oo["dw"].reshape(-1))
-                gbuf[n1 + n2:].copy_(oo["dbias"])
-                dp.allreduce_param_grads(oo["dA_log"], oo["dD"], buf=gbuf[:n1])
-                dist.all_reduce(gbuf[n1:])
-                oo["dw"].copy_(gbuf[n1:n1 + n2].view_as(oo["dw"]))
-                oo["dbias"].copy_(gbuf[n1 + n2:])
-            else:
-                dp.allreduce_param_grads(oo["dA_log"], oo["dD"], buf=gbuf)
+        if world > 1:  # one collective; the projection's gradients travel in it when present
+            grads = [oo["dA_log"], oo["dD"]] + ([oo["dw"], oo["dbias"]] if R else [])
+            dp.allreduce_grads(grads, buf=gbuf)
 
     for _ in range(max(3, args.warmup)):
         proj_fwd(); fwd(); bwd(); proj_bwd(); allreduce()
