@@ -28,3 +28,26 @@ def test_reference_arm_json_line(workload):
     assert d["impl"] == "reference" and d["value"] > 0 and d["config"]["workload"] == workload
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_traffic_records_follow_kernel_code_not_comments(tmp_path):
+    """The committed ncu traffic records are keyed to the kernel file's code: an edit of comments
+    alone keeps the key, a code edit changes it, and every committed record matches the current
+    source (so the bench's `traffic` field is not null)."""
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    a = tmp_path / "a.cu"
+    a.write_text("// header\nint f(int x) {  // doubles\n    return 2 * x;\n}\n")
+    b = tmp_path / "b.cu"
+    b.write_text("// another header\n\nint f(int x) {\n    return 2 * x;   // twice\n}\n")
+    c = tmp_path / "c.cu"
+    c.write_text("int f(int x) {\n    return 3 * x;\n}\n")
+    assert bench.code_digest(a) == bench.code_digest(b)
+    assert bench.code_digest(a) != bench.code_digest(c)
+    recs = json.load(open(os.path.join(root, "profiles", "traffic.json")))["records"]
+    for rec in recs:
+        assert bench.measured_traffic(rec["call"], rec["source"], rec["workload"]) == \
+            float(rec["dram_bytes_per_launch"]), rec["source"]
