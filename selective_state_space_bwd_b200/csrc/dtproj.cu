@@ -15,7 +15,9 @@
 // tiles as rows of 64 k-elements, m/n-major tiles as rows of 64 m/n-elements per k, so every box is
 // a plain 2-D window of a global array.  One thread issues the copies and the MMAs (four k16 steps
 // per stage); mbarriers carry "stage full" (TMA transaction bytes) and "stage free" / "accumulator
-// ready" (tcgen05.commit); the other warps only drain the accumulator from tensor memory.
+// ready" (tcgen05.commit); the other warps only drain the accumulator from tensor memory.  The
+// issue / wait order and the phase parities are model-checked on the host by
+// tests/test_mbarrier_protocol.py.
 // The rank R is small (tens to a few hundred), so each GEMM moves far more bytes than it does
 // arithmetic per byte: they are bound by HBM (writing delta_raw, reading g), not by the tensor pipe.
 #include <cuda.h>
