@@ -22,7 +22,10 @@ static __device__ __align__(256) unsigned char g_fwd_scratch[kNoAllocScratchByte
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices];  // device address of g_fwd_scratch per device; null until set up
+// Device address of g_fwd_scratch per device; null until set up.  Kept for the life of the
+// process (a cudaDeviceReset would reload the module and may move the array: the header tells
+// callers not to use this entry point on a device after resetting it).
+void* g_scratch_addr[kMaxDevices];
 
 // In host code `g_fwd_scratch` names a host-side stand-in, not device memory, so the kernels get
 // the address the runtime reports for the current device (looked up once per device).
