@@ -27,7 +27,8 @@
  *     h_t,k = a_t,k h_{t-1,k} + u_t,k                                   h_{-1} = 0
  *
  * and ssm_scan_complex_bwd returns the gradient of Re sum conj(g)·h with respect to u (complex,
- * as d/dRe + i d/dIm), r, phi, lambda and omega.
+ * as d/dRe + i d/dIm), r, phi, lambda and omega, recomputing each chunk from the checkpoints the
+ * forward wrote (ssm_scan_complex_bwd_traj computes the same from a stored trajectory h).
  *
  * Conventions (all calls)
  * -----------------------
@@ -56,7 +57,9 @@
 extern "C" {
 #endif
 
-#define SSM_SCAN_ABI_VERSION 3  /* 3: ssm_dtproj_fwd takes a workspace (its status word) */
+#define SSM_SCAN_ABI_VERSION 4  /* 4: complex forward writes checkpoints; checkpointed complex
+                                  backward (ssm_scan_complex_bwd); the trajectory-reading one
+                                  is ssm_scan_complex_bwd_traj */
 
 /* Same underlying type as cudaStream_t (NULL = the legacy default stream). */
 typedef struct CUstream_st* ssm_stream_t;
@@ -74,7 +77,9 @@ typedef enum ssm_status {
 
 typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
 
-/* Real-mode problem size. */
+/* Real-mode problem size.  Beyond the sizes the method itself needs (batch, seqlen, dim, dstate,
+ * chunk, io) it carries seg_chunks, a performance knob that never changes the result beyond
+ * rounding, and a reserved word kept for later fields. */
 typedef struct ssm_shape {
     int64_t batch;      /* B >= 0 */
     int64_t seqlen;     /* L >= 0 (0 is a valid empty problem) */
@@ -87,12 +92,12 @@ typedef struct ssm_shape {
     int32_t reserved;   /* must be 0 */
 } ssm_shape;
 
-/* Complex-mode problem size. */
+/* Complex-mode problem size (with the same seg_chunks knob as ssm_shape). */
 typedef struct ssm_cshape {
     int64_t batch;      /* B >= 0 */
     int64_t seqlen;     /* L >= 0 */
     int64_t modes;      /* K >= 1, even */
-    int32_t chunk;      /* time-split granularity in steps, one of 16..256 */
+    int32_t chunk;      /* T, one of 16..256: checkpoint spacing and time-split granularity */
     int32_t seg_chunks; /* chunks per time segment; 0 = automatic (tuning knob only) */
 } ssm_cshape;
 
@@ -189,7 +194,9 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts,
  *   rejected with SSM_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  Only problems that
  *   the library splits into many time segments need more than 256 bytes.
  * - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *   that device current; make that first call before any stream capture.
+ *   that device current; make that first call before any stream capture.  The address is kept
+ *   for the life of the process: after cudaDeviceReset on a device, do not call this entry point
+ *   on that device again (the array may have moved).
  * - Every call on a device shares the one array and leaves its contents behind; calls that
  *   overlap on the GPU (other streams, other host threads) race on it.  Serialise them.
  * - The device status word is kept in that array and is not readable through ssm_scan_status.
@@ -200,35 +207,67 @@ int ssm_scan_fwd_noalloc(const ssm_shape* shape,
                          const void* Bm, const void* Cm, const float* Dskip,
                          void* y, float* ckpt, ssm_stream_t stream);
 
-/* Workspace bytes for the complex calls (at least 256); 0 for an invalid shape. */
+/* Workspace bytes for the complex calls (at least 256); 0 for an invalid shape.  backward != 0
+ * covers both backward calls (the checkpointed one needs the larger workspace: it adds a
+ * per-CTA chunk-trajectory scratch capped at max(64 MiB, the checkpoint bytes)). */
 size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward);
 
+/* Bytes of the complex checkpoints: B * ceil(L / T) * K * 8 (complex64); 0 for an invalid shape. */
+size_t ssm_scan_complex_checkpoint_bytes(const ssm_cshape* shape);
+
 /*
- * Complex forward.
+ * Complex forward ("SPARC: Shared Phase and Retention Control for Efficient Adaptive Spectral
+ * Recurrence", abstract: two input-dependent scalars shared by every mode, diagonal recurrence):
+ *     s_t = softplus(r_t),  a_{t,k} = exp(-lambda_k s_t + i omega_k phi_t),  h_t = a_t h_{t-1} + u_t.
  *   u       [B, L, K] complex64 (interleaved re, im fp32)
  *   r, phi  [B, L] fp32          lambda, omega [K] fp32
- * Output:
+ * Outputs (either may be NULL, not both; SSM_ERR_INVALID_ARG when both are):
  *   h       [B, L, K] complex64: the whole state trajectory (the output of this mode)
+ *   ckpt    [B, ceil(L/T), K] complex64: the state at the last step of every chunk of T steps,
+ *           what ssm_scan_complex_bwd recomputes from
  */
 int ssm_scan_complex_fwd(const ssm_cshape* shape,
                          const void* u, const float* r, const float* phi,
                          const float* lambda, const float* omega,
-                         void* h, void* ws, size_t ws_bytes, ssm_stream_t stream);
+                         void* h, void* ckpt, void* ws, size_t ws_bytes, ssm_stream_t stream);
 
 /*
- * Complex backward: gradient of Re sum conj(g)·h.
- *   h       [B, L, K] complex64, the trajectory written by ssm_scan_complex_fwd.  Because the
- *           trajectory is this mode's output it is already resident, so the backward reads it
- *           (h_{t-1} at step t) instead of recomputing it.
- *   r, phi, lambda, omega as for the forward;  g [B, L, K] complex64 (dLoss/dh).
+ * Complex backward from checkpoints: the gradient of Re sum conj(g)·h, where only the chunk-end
+ * states are kept ("Breaking the Memory Wall: Exact Analytical Differentiation via Tiled
+ * Operator-Space Evolution", abstract).  Each chunk's trajectory is recomputed from its entering
+ * checkpoint into an L2-resident workspace region, then the adjoint
+ *     mu_t = g_t + conj(a_{t+1}) mu_{t+1},   q_t = mu_t conj(a_t h_{t-1})
+ * is swept back through it:  du = mu,  dlambda = -sum s Re q,  dr = sigmoid(r) (-sum_k lambda Re q),
+ * domega = sum phi Im q,  dphi = sum_k omega Im q.  The trajectory h need not be kept: memory
+ * beyond inputs and outputs is O(L / T).  Every transition is evaluated twice (recompute and
+ * sweep), so this is slower than ssm_scan_complex_bwd_traj, which reads a stored h instead.
+ *   u       [B, L, K] complex64, the forward's input
+ *   r, phi, lambda, omega as for the forward
+ *   ckpt    [B, ceil(L/T), K] complex64, written by ssm_scan_complex_fwd with the same shape
+ *   g       [B, L, K] complex64 (dLoss/dh)
  * Outputs (overwritten):
  *   du [B, L, K] complex64;  dr, dphi [B, L] fp32;  dlambda, domega [K] fp32.
+ * Enqueues ssm_scan_complex_kernel_launches(shape, 1) kernels.  Returns an ssm_status.
  */
 int ssm_scan_complex_bwd(const ssm_cshape* shape,
-                         const void* h, const float* r, const float* phi,
-                         const float* lambda, const float* omega, const void* g,
-                         void* du, float* dr, float* dphi, float* dlambda, float* domega,
-                         void* ws, size_t ws_bytes, ssm_stream_t stream);
+                         const void* u, const float* r, const float* phi,
+                         const float* lambda, const float* omega, const void* ckpt,
+                         const void* g, void* du, float* dr, float* dphi, float* dlambda,
+                         float* domega, void* ws, size_t ws_bytes, ssm_stream_t stream);
+
+/*
+ * Complex backward from the stored trajectory (the fast path when h is resident anyway, e.g.
+ * because it is this mode's output): the same gradient as ssm_scan_complex_bwd, with h_{t-1}
+ * read from h at every step instead of recomputed, so each transition is evaluated once.
+ *   h       [B, L, K] complex64, the trajectory written by ssm_scan_complex_fwd
+ *   r, phi, lambda, omega, g, outputs as for ssm_scan_complex_bwd.
+ * Enqueues ssm_scan_complex_kernel_launches(shape, 2) kernels.  Returns an ssm_status.
+ */
+int ssm_scan_complex_bwd_traj(const ssm_cshape* shape,
+                              const void* h, const float* r, const float* phi,
+                              const float* lambda, const float* omega, const void* g,
+                              void* du, float* dr, float* dphi, float* dlambda, float* domega,
+                              void* ws, size_t ws_bytes, ssm_stream_t stream);
 
 /* Workspace bytes for ssm_scan_complex_rtrl (at least 256); 0 for an invalid shape. */
 size_t ssm_scan_complex_rtrl_workspace_bytes(const ssm_cshape* shape);
@@ -346,7 +385,8 @@ int ssm_dtproj_bwd(const ssm_dtshape* shape, const void* u, const void* w, const
  * enqueues for this shape (0 for an empty problem, -1 for an invalid shape). */
 int ssm_scan_kernel_launches(const ssm_shape* shape, int backward);
 
-/* Same for the complex calls. */
+/* Same for the complex calls: backward = 0 ssm_scan_complex_fwd, 1 ssm_scan_complex_bwd (from
+ * checkpoints), 2 ssm_scan_complex_bwd_traj (-1 for any other value). */
 int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward);
 
 /* Same for the PD-SSM calls: 1 (one scan kernel, with the argmax fused into the forward and the

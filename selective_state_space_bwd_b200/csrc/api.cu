@@ -163,10 +163,15 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
 
 struct CplxPlan {
     int B, L, K, T, nC, nkt, seg_chunks, nseg;
+    int b_group;  // checkpointed backward: segments per launch (the trajectory scratch holds one)
     size_t f_sumP, f_sumS, f_hin, f_end;
-    size_t b_gP, b_gG, b_win, b_rp, b_lo, b_end;
+    size_t b_gP, b_gG, b_win, b_rp, b_lo, b_traj, b_end;
     size_t r_lo, r_end;  // RTRL: per-(batch, mode) gradient sums
 };
+
+// Checkpointed complex backward: per-launch cap on the chunk-trajectory scratch
+// (max(checkpoint bytes, this)), so the backward's memory stays O(L / T).
+constexpr size_t kCplxTrajCap = (size_t)64 << 20;
 
 int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
     if (!s) return SSM_ERR_INVALID_ARG;
@@ -197,6 +202,13 @@ int plan_cplx(const ssm_cshape* s, CplxPlan* p) {
     p->b_win = o; o = align256(o + (S > 1 ? B * S * K * 8 : 0));
     p->b_rp = o;  o = align256(o + (size_t)p->nkt * B * (size_t)p->L * 8);
     p->b_lo = o;  o = align256(o + B * S * K * 8);
+    // checkpointed backward: [group][B][nkt] CTAs' chunk trajectories
+    const size_t traj_seg = B * (size_t)p->nkt * ssm::cplx_traj_floats(p->T) * 4;
+    const size_t ckpt = B * (size_t)p->nC * K * 8;
+    const size_t cap = ckpt > kCplxTrajCap ? ckpt : kCplxTrajCap;
+    const size_t g = traj_seg > 0 ? cap / traj_seg : S;
+    p->b_group = (int)(g < 1 ? 1 : (g > S ? S : g));
+    p->b_traj = o; o = align256(o + (size_t)p->b_group * traj_seg);
     p->b_end = o;
     o = kStatusBytes;
     p->r_lo = o;  o = align256(o + B * K * 8);
@@ -355,10 +367,17 @@ int ssm_scan_kernel_launches(const ssm_shape* shape, int backward) {
 
 int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward) {
     CplxPlan p;
-    if (plan_cplx(shape, &p) != SSM_OK) return -1;
+    if (plan_cplx(shape, &p) != SSM_OK || backward < 0 || backward > 2) return -1;
     if (p.B == 0 || p.L == 0) return 0;
     const int seg = p.nseg > 1 ? 2 : 0;
+    if (backward == 1) return seg + (p.nseg + p.b_group - 1) / p.b_group + 2;
     return backward ? 3 + seg : 1 + seg;
+}
+
+size_t ssm_scan_complex_checkpoint_bytes(const ssm_cshape* shape) {
+    CplxPlan p;
+    if (plan_cplx(shape, &p) != SSM_OK) return 0;
+    return (size_t)p.B * p.nC * p.K * 8;
 }
 
 size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward) {
@@ -368,15 +387,17 @@ size_t ssm_scan_complex_workspace_bytes(const ssm_cshape* shape, int backward) {
 }
 
 int ssm_scan_complex_fwd(const ssm_cshape* shape, const void* u, const float* r, const float* phi,
-                         const float* lambda, const float* omega, void* h, void* ws,
+                         const float* lambda, const float* omega, void* h, void* ckpt, void* ws,
                          size_t ws_bytes, ssm_stream_t stream) {
     CplxPlan p;
     int st = plan_cplx(shape, &p);
     if (st != SSM_OK) return st;
     const size_t BLK = (size_t)p.B * p.L * p.K, BL = (size_t)p.B * p.L;
-    const void* ptrs[] = {u, r, phi, lambda, omega, h, ws};
-    const size_t counts[] = {BLK, BL, BL, (size_t)p.K, (size_t)p.K, BLK, 1};
-    if ((st = check_arrays(ptrs, counts, 7)) != SSM_OK) return st;
+    const size_t CK = (size_t)p.B * p.nC * p.K;
+    if (!h && !ckpt) return SSM_ERR_INVALID_ARG;  // nothing to write
+    const void* ptrs[] = {u, r, phi, lambda, omega, h, ckpt, ws};
+    const size_t counts[] = {BLK, BL, BL, (size_t)p.K, (size_t)p.K, h ? BLK : 0, ckpt ? CK : 0, 1};
+    if ((st = check_arrays(ptrs, counts, 8)) != SSM_OK) return st;
     if (ws_bytes < p.f_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
@@ -386,6 +407,7 @@ int ssm_scan_complex_fwd(const ssm_cshape* shape, const void* u, const float* r,
     a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.nkt = p.nkt;
     a.u = static_cast<const float*>(u); a.r = r; a.phi = phi; a.lam = lambda; a.om = omega;
     a.h = static_cast<float*>(h);
+    a.ckpt = static_cast<float*>(ckpt);
     a.sumP = at<float>(ws, p.f_sumP); a.sumS = at<float>(ws, p.f_sumS); a.hin = at<float>(ws, p.f_hin);
     a.status = at<unsigned>(ws, 0);
     return ssm::launch_cplx_fwd(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -430,10 +452,43 @@ int ssm_scan_complex_rtrl(const ssm_cshape* shape, const void* u, const float* r
     return ssm::launch_cplx_rtrl(a, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-int ssm_scan_complex_bwd(const ssm_cshape* shape, const void* h, const float* r, const float* phi,
-                         const float* lambda, const float* omega, const void* g, void* du,
-                         float* dr, float* dphi, float* dlambda, float* domega, void* ws,
+int ssm_scan_complex_bwd(const ssm_cshape* shape, const void* u, const float* r, const float* phi,
+                         const float* lambda, const float* omega, const void* ckpt, const void* g,
+                         void* du, float* dr, float* dphi, float* dlambda, float* domega, void* ws,
                          size_t ws_bytes, ssm_stream_t stream) {
+    CplxPlan p;
+    int st = plan_cplx(shape, &p);
+    if (st != SSM_OK) return st;
+    const size_t BLK = (size_t)p.B * p.L * p.K, BL = (size_t)p.B * p.L, K = p.K;
+    const size_t CK = (size_t)p.B * p.nC * p.K;
+    const void* ptrs[] = {u, r, phi, lambda, omega, ckpt, g, du, dr, dphi, dlambda, domega, ws};
+    const size_t counts[] = {BLK, BL, BL, K, K, CK, BLK, BLK, BL, BL, K, K, 1};
+    if ((st = check_arrays(ptrs, counts, 13)) != SSM_OK) return st;
+    if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.B == 0 || p.L == 0) {
+        if (cudaMemsetAsync(dlambda, 0, K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (cudaMemsetAsync(domega, 0, K * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    ssm::CplxArgs a = {};
+    a.B = p.B; a.L = p.L; a.K = p.K; a.T = p.T; a.nC = p.nC;
+    a.seg_chunks = p.seg_chunks; a.nseg = p.nseg; a.nkt = p.nkt;
+    a.u = static_cast<const float*>(u); a.r = r; a.phi = phi; a.lam = lambda; a.om = omega;
+    a.ckpt_in = static_cast<const float*>(ckpt); a.g = static_cast<const float*>(g);
+    a.du = static_cast<float*>(du); a.dr = dr; a.dphi = dphi; a.dlam = dlambda; a.dom = domega;
+    a.gsumP = at<float>(ws, p.b_gP); a.gsumG = at<float>(ws, p.b_gG); a.win = at<float>(ws, p.b_win);
+    a.rp_part = at<float>(ws, p.b_rp); a.lo_part = at<float>(ws, p.b_lo);
+    a.traj = at<float>(ws, p.b_traj);
+    a.status = at<unsigned>(ws, 0);
+    return ssm::launch_cplx_bwd_ckpt(a, p.b_group, s) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_scan_complex_bwd_traj(const ssm_cshape* shape, const void* h, const float* r,
+                              const float* phi, const float* lambda, const float* omega,
+                              const void* g, void* du, float* dr, float* dphi, float* dlambda,
+                              float* domega, void* ws, size_t ws_bytes, ssm_stream_t stream) {
     CplxPlan p;
     int st = plan_cplx(shape, &p);
     if (st != SSM_OK) return st;

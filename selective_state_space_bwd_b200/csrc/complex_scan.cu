@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(F_NT) cplx_fwd_kernel(CplxArgs p) {
     if (!SUMMARY && seg > 0 && kv)
         h = reinterpret_cast<const float2*>(p.hin)[((size_t)b * p.nseg + seg) * p.K + k];
     const float2* ub = reinterpret_cast<const float2*>(p.u) + boff * p.K;
-    float2* hb = SUMMARY ? nullptr : reinterpret_cast<float2*>(p.h) + boff * p.K;
+    float2* hb = SUMMARY || !p.h ? nullptr : reinterpret_cast<float2*>(p.h) + boff * p.K;
     auto issue = [&](int i) {
         if (i < ntiles)
             cp_async_tile<float2, KT>(su[i % F_USTAGES], ub, t_begin + i * FT, FT, p.L, k0, p.K, tid,
@@ -289,10 +289,15 @@ __global__ void __launch_bounds__(F_NT) cplx_fwd_kernel(CplxArgs p) {
             h = make_float2(ah.x + uu.x, ah.y + uu.y);
             if (SUMMARY)
                 P = cmul(av, P);
-            else if (kv)
+            else if (kv && hb)
                 hb[(size_t)(t0 + r) * p.K + k] = h;
         }
         bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // buffer buf is consumed
+        // tiles never cross a chunk end (FT divides T): the state after the tile's last step is
+        // the chunk's checkpoint when the tile ends the chunk
+        const int te = t0 + rows;
+        if (!SUMMARY && p.ckpt && kv && (te % p.T == 0 || te == p.L))
+            reinterpret_cast<float2*>(p.ckpt)[((size_t)b * p.nC + (te - 1) / p.T) * p.K + k] = h;
     }
     if (SUMMARY) {
         if (kv) {
@@ -400,6 +405,56 @@ __global__ void cplx_carry_bwd_kernel(int B, int nseg, int K, const float2* __re
     }
 }
 
+// Producer side of the backward kernels: for the items i = 0..n-1 of the CTA's tile sequence
+// (tile(i, t0, rows): the steps t0 .. t0+rows-1 of item i), the step scalars (softplus(r), phi)
+// and the transitions a of the item's steps go into buffer i & 1, handed over with the FULL /
+// EMPTY named barriers; the step scalars of item i + 1 are fetched while item i is computed.
+template <typename TileFn>
+__device__ __forceinline__ void cplx_produce(const CplxArgs& p, int n, TileFn tile, int tid, int k0,
+                                             size_t boff, float2 (*sa)[FT * KT],
+                                             float2 (*ssp)[FT]) {
+    const int pt = tid - F_CONS, kk = pt % KT, rp = pt / KT;
+    const int k = k0 + kk;
+    const bool kv = k < p.K;
+    const float lam2 = kv ? p.lam[k] * kLog2e : 0.0f, om = kv ? p.om[k] : 0.0f;
+    const float* rb = p.r + boff;
+    const float* pb = p.phi + boff;
+    float rn = 0.0f, pn = 0.0f;
+    if (n > 0 && pt < FT) {
+        int t0, rows;
+        tile(0, t0, rows);
+        if (pt < rows) {
+            rn = rb[t0 + pt];
+            pn = pb[t0 + pt];
+        }
+    }
+    for (int i = 0; i < n; ++i) {
+        const int buf = i & 1;
+        int t0, rows;
+        tile(i, t0, rows);
+        bar_sync_n(F_BAR_EMPTY + buf, F_NT);  // the consumers are done with buffer buf
+        if (pt < FT) {
+            ssp[buf][pt] = pt < rows ? make_float2(softplus_acc(rn), pn) : make_float2(0.0f, 0.0f);
+            if (i + 1 < n) {
+                int t1, r1;
+                tile(i + 1, t1, r1);
+                if (pt < r1) {
+                    rn = rb[t1 + pt];
+                    pn = pb[t1 + pt];
+                }
+            }
+        }
+        bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
+        float2 a[FT / 2];
+        transitions_pk<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
+#pragma unroll
+        for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
+        bar_arrive_n(F_BAR_FULL + buf, F_NT);  // buffer buf holds the item's transitions
+    }
+    bar_sync_n(F_BAR_EMPTY + 0, F_NT);  // balance the consumers' last two releases
+    bar_sync_n(F_BAR_EMPTY + 1, F_NT);
+}
+
 // Backward, warp-specialised like the forward: KT consumer threads (one per mode) sweep the
 // adjoint backwards over 16-step tiles of g and h_{t-1} (their own two-stage cp.async ring) and
 // sum (lambda Re q, omega Im q) over the CTA's modes per step; 2 KT producer threads compute the
@@ -428,41 +483,11 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_kernel(CplxArgs p) {
     const size_t boff = (size_t)b * p.L;
 
     if (tid >= F_CONS) {
-        // ---------------------------------------------------------------- producers
-        const int pt = tid - F_CONS, kk = pt % KT, rp = pt / KT;
-        const int k = k0 + kk;
-        const bool kv = k < p.K;
-        const float lam2 = kv ? p.lam[k] * kLog2e : 0.0f, om = kv ? p.om[k] : 0.0f;
-        const float* rb = p.r + boff;
-        const float* pb = p.phi + boff;
-        float rn = 0.0f, pn = 0.0f;  // step scalars of the next tile, fetched a tile ahead
-        {
-            const int t = t_begin + (ntiles - 1) * FT + pt;
-            if (ntiles > 0 && pt < FT && t < t_end) {
-                rn = rb[t];
-                pn = pb[t];
-            }
-        }
-        for (int i = 0; i < ntiles; ++i) {
-            const int buf = i & 1, jt = ntiles - 1 - i;
-            const int t0 = t_begin + jt * FT, rows = min(FT, t_end - t0);
-            bar_sync_n(F_BAR_EMPTY + buf, F_NT);  // the consumers are done with buffer buf
-            if (pt < FT) {
-                ssp[buf][pt] = pt < rows ? make_float2(softplus_acc(rn), pn) : make_float2(0.0f, 0.0f);
-                if (jt > 0) {  // the earlier tile is always full
-                    rn = rb[t0 - FT + pt];
-                    pn = pb[t0 - FT + pt];
-                }
-            }
-            bar_sync_n(F_BAR_PROD, F_PROD);  // the step scalars are in
-            float2 a[FT / 2];
-            transitions_pk<FT / 2, 2>(a, lam2, om, ssp[buf], rp);
-#pragma unroll
-            for (int u = 0; u < FT / 2; ++u) sa[buf][(rp + 2 * u) * KT + kk] = a[u];
-            bar_arrive_n(F_BAR_FULL + buf, F_NT);  // buffer buf holds the tile's transitions
-        }
-        bar_sync_n(F_BAR_EMPTY + 0, F_NT);  // balance the consumers' last two releases
-        bar_sync_n(F_BAR_EMPTY + 1, F_NT);
+        // producers: the segment's tiles from the last one back
+        cplx_produce(p, ntiles, [&](int i, int& t0, int& rows) {
+            t0 = t_begin + (ntiles - 1 - i) * FT;
+            rows = min(FT, t_end - t0);
+        }, tid, k0, boff, sa, ssp);
         return;
     }
 
@@ -525,6 +550,169 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_kernel(CplxArgs p) {
         {
             // sums over the CTA's modes, one step per four threads; the rotation by tid keeps
             // each half-warp's 8-byte loads in distinct banks
+            float2 acc = make_float2(0.0f, 0.0f);
+            const float2* row = red + cs_r * KT + cs_part * (KT / 4);
+#pragma unroll
+            for (int m = 0; m < KT / 4; ++m) {
+                const float2 v = row[(m + tid) & (KT / 4 - 1)];
+                acc.x += v.x;
+                acc.y += v.y;
+            }
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+            }
+            if (cs_part == 0 && cs_r < rows) partb[t0 + cs_r] = acc;
+        }
+    }
+    if (kv) {
+        const size_t o = ((size_t)b * p.nseg + seg) * p.K + k;
+        reinterpret_cast<float2*>(p.lo_part)[o] = make_float2(dlam, dom);
+        if (!(isfinite(w.x) && isfinite(w.y))) flag_status(p.status, kStatusNonFinite);
+    }
+}
+
+// Checkpointed backward: the same adjoint sweep, with the trajectory recomputed chunk by chunk
+// from the forward's checkpoints instead of read from a stored h ("Breaking the Memory Wall ...
+// Tiled Operator-Space Evolution", abstract: only chunk-boundary states are kept).  For each chunk
+// of the segment, last first, the CTA's tile sequence holds the chunk's tiles twice: forward, where
+// the consumers run h = a h + u from the chunk's entering checkpoint and leave h_{t-1} of every step
+// in the CTA's scratch region ([T][KT] complex, L2-resident), then backward, where they sweep the
+// adjoint exactly as cplx_bwd_kernel does with h_{t-1} read back from that region.  The producers
+// compute the transitions of every item, so each transition is evaluated twice.
+__global__ void __launch_bounds__(F_NT) cplx_bwd_ckpt_kernel(CplxArgs p) {
+    static_assert(FT * 4 == KT, "column sums: four consumer threads per step");
+    // dynamic shared memory as cplx_bwd_kernel: transitions [2][FT*KT], u (forward items) or g
+    // (sweep items) [B_USTAGES][FT*KT], h_{t-1} [B_USTAGES][FT*KT], step scalars [2][FT]
+    extern __shared__ __align__(16) float2 cdyn[];
+    float2 (*sa)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn);
+    float2 (*sx)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + 2 * FT * KT);
+    float2 (*shp)[FT * KT] = reinterpret_cast<float2 (*)[FT * KT]>(cdyn + (2 + B_USTAGES) * FT * KT);
+    float2 (*ssp)[FT] = reinterpret_cast<float2 (*)[FT]>(cdyn + (2 + 2 * B_USTAGES) * FT * KT);
+    const int tid = threadIdx.x;
+    const int k0 = blockIdx.x * KT;
+    const int b = blockIdx.y, seg = p.seg0 + blockIdx.z;
+    const int c_begin = seg * p.seg_chunks;
+    const int c_end = min(p.nC, c_begin + p.seg_chunks);
+    const int ntT = p.T / FT;                                   // tiles of a full chunk
+    const int nt0 = (min(p.T, p.L - (c_end - 1) * p.T) + FT - 1) / FT;  // of the segment's last
+    const int n = c_end > c_begin ? 2 * nt0 + 2 * ntT * (c_end - 1 - c_begin) : 0;
+    const size_t boff = (size_t)b * p.L;
+    // item i: chunk c, forward (sweep = false) or sweep item, tile j of the chunk's nt tiles
+    auto item = [&](int i, int& c, bool& sweep, int& j, int& nt) {
+        if (i < 2 * nt0) {
+            c = c_end - 1;
+            nt = nt0;
+            j = i;
+        } else {
+            const int i2 = i - 2 * nt0;
+            c = c_end - 2 - i2 / (2 * ntT);
+            nt = ntT;
+            j = i2 % (2 * ntT);
+        }
+        sweep = j >= nt;
+        if (sweep) j = 2 * nt - 1 - j;
+    };
+
+    if (tid >= F_CONS) {
+        cplx_produce(p, n, [&](int i, int& t0, int& rows) {
+            int c, j, nt;
+            bool sw;
+            item(i, c, sw, j, nt);
+            t0 = c * p.T + j * FT;
+            rows = min(FT, p.L - t0);
+        }, tid, k0, boff, sa, ssp);
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int k = k0 + tid;
+    const bool kv = k < p.K;
+    const float lam = kv ? p.lam[k] : 0.0f, om = kv ? p.om[k] : 0.0f;
+    float2 w = make_float2(0.0f, 0.0f), h = make_float2(0.0f, 0.0f);
+    if (seg < p.nseg - 1 && kv)
+        w = reinterpret_cast<const float2*>(p.win)[((size_t)b * p.nseg + seg) * p.K + k];
+    float dlam = 0.0f, dom = 0.0f;
+    const float2* ub = reinterpret_cast<const float2*>(p.u) + boff * p.K;
+    const float2* gb = reinterpret_cast<const float2*>(p.g) + boff * p.K;
+    const float2* ckb = reinterpret_cast<const float2*>(p.ckpt_in) + (size_t)b * p.nC * p.K;
+    float2* dub = reinterpret_cast<float2*>(p.du) + boff * p.K;
+    float2* partb = reinterpret_cast<float2*>(p.rp_part) + ((size_t)blockIdx.x * p.B + b) * (size_t)p.L;
+    const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    float2* traj = reinterpret_cast<float2*>(p.traj) + cta * (cplx_traj_floats(p.T) / 2);
+    const int cs_r = tid >> 2, cs_part = tid & 3;  // column sums: step cs_r, a quarter of the modes
+    auto issue = [&](int i) {
+        if (i < n) {
+            int c, j, nt;
+            bool sw;
+            item(i, c, sw, j, nt);
+            const int st = i % B_USTAGES, t0 = c * p.T + j * FT;
+            if (!sw) {
+                cp_async_tile<float2, KT>(sx[st], ub, t0, FT, p.L, k0, p.K, tid, F_CONS);
+            } else {
+                cp_async_tile<float2, KT>(sx[st], gb, t0, FT, p.L, k0, p.K, tid, F_CONS);
+                cp_async_tile<float2, KT>(shp[st], traj, j * FT, FT, min(p.T, p.L - c * p.T), 0,
+                                          KT, tid, F_CONS);
+            }
+        }
+        cp_async_commit();
+    };
+    issue(0);
+    bar_arrive_n(F_BAR_EMPTY + 0, F_NT);  // both transition buffers start empty
+    bar_arrive_n(F_BAR_EMPTY + 1, F_NT);
+    for (int i = 0; i < n; ++i) {
+        int c, j, nt;
+        bool sweep;
+        item(i, c, sweep, j, nt);
+        const int buf = i & 1, st = i % B_USTAGES;
+        const int t0 = c * p.T + j * FT, rows = min(FT, p.L - t0);
+        cp_async_wait<0>();
+        bar_sync_n(F_BAR_CONS, F_CONS);  // item i's tiles are in; every consumer is past item i-1
+        // the first sweep item of a chunk reads the h_{t-1} that the item before it writes, so its
+        // copies are issued once that item is done
+        const bool defer = !sweep && j == nt - 1;
+        if (!defer) issue(i + 1);
+        const float2* sat = sa[buf];
+        bar_sync_n(F_BAR_FULL + buf, F_NT);  // the producers have written the item's transitions
+        if (!sweep) {
+            if (j == 0 && kv) h = c > 0 ? ckb[(size_t)(c - 1) * p.K + k] : make_float2(0.0f, 0.0f);
+            const float2* sut = sx[st];
+            float2* tr = traj + (size_t)(j * FT) * KT + tid;
+#pragma unroll 4
+            for (int r = 0; r < rows; ++r) {
+                tr[r * KT] = h;  // h_{t-1} of step t = t0 + r
+                const float2 ah = cmul(sat[r * KT + tid], h);
+                const float2 uu = sut[r * KT + tid];
+                h = make_float2(ah.x + uu.x, ah.y + uu.y);
+            }
+            bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // transitions consumed
+            if (defer) {
+                bar_sync_n(F_BAR_CONS, F_CONS);  // the chunk's h_{t-1} are all written
+                issue(i + 1);
+            }
+            continue;
+        }
+        const float2* sgt = sx[st];
+        const float2* sht = shp[st];
+        const float2* sst = ssp[buf];
+        float2* red = sx[st];
+#pragma unroll 4
+        for (int r = rows - 1; r >= 0; --r) {
+            const float2 sp2 = sst[r];
+            const float2 av = sat[r * KT + tid];
+            const float2 gg = sgt[r * KT + tid];
+            const float2 mu = make_float2(gg.x + w.x, gg.y + w.y);
+            w = cmul_ca(av, mu);
+            const float2 q = cmul_cb(w, sht[r * KT + tid]);
+            if (kv) dub[(size_t)(t0 + r) * p.K + k] = mu;
+            dlam = fmaf(-sp2.x, q.x, dlam);
+            dom = fmaf(sp2.y, q.y, dom);
+            red[r * KT + tid] = make_float2(lam * q.x, om * q.y);
+        }
+        bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // transitions and step scalars are consumed
+        bar_sync_n(F_BAR_CONS, F_CONS);         // the item's (lambda Re q, omega Im q) are in
+        {
             float2 acc = make_float2(0.0f, 0.0f);
             const float2* row = red + cs_r * KT + cs_part * (KT / 4);
 #pragma unroll
@@ -729,6 +917,35 @@ cudaError_t launch_cplx_rtrl(const CplxArgs& a, cudaStream_t st) {
     cplx_rtrl_kernel<<<dim3(a.nkt, a.B, 1), F_NT, B_SMEM, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cplx_reduce_k_kernel<<<(a.K + 255) / 256, 256, 0, st>>>(a);  // sums over b (nseg = 1)
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cplx_bwd_ckpt(const CplxArgs& a0, int group, cudaStream_t st) {
+    cudaError_t e;
+    CplxArgs a = a0;
+    if (a.nseg > 1) {
+        cplx_bwd_summary_kernel<<<dim3(a.nkt, a.B, a.nseg - 1), KT, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t n = (int64_t)a.B * a.K;
+        cplx_carry_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            a.B, a.nseg, a.K, reinterpret_cast<const float2*>(a.gsumP),
+            reinterpret_cast<const float2*>(a.gsumG), reinterpret_cast<float2*>(a.win));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(cplx_bwd_ckpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM);
+    if (e != cudaSuccess) return e;
+    for (int lo = 0; lo < a.nseg; lo += group) {
+        a.seg0 = lo;
+        const int ns = a.nseg - lo < group ? a.nseg - lo : group;
+        cplx_bwd_ckpt_kernel<<<dim3(a.nkt, a.B, ns), F_NT, B_SMEM, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const int64_t n = (int64_t)a.B * a.L;
+    if (n > 0) {
+        cplx_reduce_bl_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    cplx_reduce_k_kernel<<<(a.K + 255) / 256, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -94,7 +94,17 @@ struct CplxArgs {
     float* lo_part;     // [B][nseg][K][2] per-segment sums of -s Re q and phi Im q
     float* state;       // RTRL: [B][3][K][2] (h, dh/dlambda, dh/domega) carried across calls, or null
     unsigned* status;
+    // checkpoints: the state at the last step of every chunk, [B][nC][K][2].  The forward writes
+    // them when ckpt is not null; the checkpointed backward reads ckpt_in and recomputes each
+    // chunk's trajectory into a per-CTA scratch region of cplx_traj_floats(T) floats (L2-resident),
+    // running segments [seg0, seg0 + gridDim.z) per launch
+    float* ckpt;
+    const float* ckpt_in;
+    float* traj;
+    int seg0;
 };
+// Floats of one CTA's chunk-trajectory scratch in the checkpointed complex backward.
+__host__ __device__ inline size_t cplx_traj_floats(int T) { return (size_t)T * kCplxKT * 2; }
 
 // Flash PD-SSM: N lanes per (batch, head) sequence (lane = state), kPdThreads per CTA.
 constexpr int kPdThreads = 128;
@@ -156,5 +166,7 @@ cudaError_t launch_real_bwd(const RealArgs& a, int io_bf16, int N, int group, cu
 cudaError_t launch_cplx_fwd(const CplxArgs& a, cudaStream_t st);
 cudaError_t launch_cplx_rtrl(const CplxArgs& a, cudaStream_t st);
 cudaError_t launch_cplx_bwd(const CplxArgs& a, cudaStream_t st);
+// checkpointed backward: segments in launches of `group` (the trajectory scratch holds one launch)
+cudaError_t launch_cplx_bwd_ckpt(const CplxArgs& a, int group, cudaStream_t st);
 
 }  // namespace ssm

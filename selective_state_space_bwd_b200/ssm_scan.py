@@ -3,7 +3,7 @@
 Argument marshalling only: every step of the scan runs in the library's CUDA kernels.  If the
 library is missing, or the tensors are not on a CUDA device, the calls raise — there is no CPU
 fallback.  Names mirror the C ABI: ``ssm_scan_fwd``, ``ssm_scan_bwd``, ``ssm_scan_complex_fwd``,
-``ssm_scan_complex_bwd``, ``ssm_scan_status``; the workspace / checkpoint size queries are exposed
+``ssm_scan_complex_bwd``, ``ssm_scan_complex_bwd_traj``, ``ssm_scan_status``; the workspace / checkpoint size queries are exposed
 as ``workspace_bytes`` and friends.
 """
 
@@ -67,7 +67,8 @@ _lib = None
 
 EXPORTED = ["ssm_scan_abi_version", "ssm_scan_checkpoint_bytes", "ssm_scan_workspace_bytes",
             "ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_complex_workspace_bytes",
-            "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_kernel_launches",
+            "ssm_scan_complex_fwd", "ssm_scan_complex_bwd", "ssm_scan_complex_bwd_traj",
+            "ssm_scan_complex_checkpoint_bytes", "ssm_scan_kernel_launches",
             "ssm_scan_complex_kernel_launches", "ssm_scan_status", "ssm_status_string",
             "ssm_scan_fwd_noalloc", "ssm_scan_fwd_ex", "ssm_scan_bwd_ex",
             "ssm_scan_complex_rtrl_workspace_bytes", "ssm_scan_complex_rtrl",
@@ -96,10 +97,14 @@ def lib():
             L.ssm_scan_bwd.restype = I
             L.ssm_scan_complex_workspace_bytes.argtypes = [CP, I]
             L.ssm_scan_complex_workspace_bytes.restype = Z
-            L.ssm_scan_complex_fwd.argtypes = [CP] + [P] * 7 + [Z, P]
+            L.ssm_scan_complex_checkpoint_bytes.argtypes = [CP]
+            L.ssm_scan_complex_checkpoint_bytes.restype = Z
+            L.ssm_scan_complex_fwd.argtypes = [CP] + [P] * 8 + [Z, P]
             L.ssm_scan_complex_fwd.restype = I
-            L.ssm_scan_complex_bwd.argtypes = [CP] + [P] * 12 + [Z, P]
+            L.ssm_scan_complex_bwd.argtypes = [CP] + [P] * 13 + [Z, P]
             L.ssm_scan_complex_bwd.restype = I
+            L.ssm_scan_complex_bwd_traj.argtypes = [CP] + [P] * 12 + [Z, P]
+            L.ssm_scan_complex_bwd_traj.restype = I
             L.ssm_scan_kernel_launches.argtypes = [SP, I]
             L.ssm_scan_kernel_launches.restype = I
             L.ssm_scan_complex_kernel_launches.argtypes = [CP, I]
@@ -178,8 +183,14 @@ def kernel_launches(shape: SsmShape, backward: bool) -> int:
     return int(lib().ssm_scan_kernel_launches(ctypes.byref(shape), int(bool(backward))))
 
 
-def complex_kernel_launches(shape: SsmCShape, backward: bool) -> int:
-    return int(lib().ssm_scan_complex_kernel_launches(ctypes.byref(shape), int(bool(backward))))
+def complex_checkpoint_bytes(shape: SsmCShape) -> int:
+    return int(lib().ssm_scan_complex_checkpoint_bytes(ctypes.byref(shape)))
+
+
+def complex_kernel_launches(shape: SsmCShape, backward) -> int:
+    """backward: 0 / False the forward, 1 / True ssm_scan_complex_bwd (from checkpoints),
+    2 ssm_scan_complex_bwd_traj (from the stored trajectory)."""
+    return int(lib().ssm_scan_complex_kernel_launches(ctypes.byref(shape), int(backward)))
 
 
 def _io_of(t):
@@ -312,39 +323,69 @@ def ssm_scan_bwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, zoh=False, h0=
     return out
 
 
-def ssm_scan_complex_fwd(u, r, phi, lam, omega, chunk=128, seg_chunks=0, h=None, ws=None,
-                         stream=None):
-    """Complex forward.  u [B,L,K] complex64; r, phi [B,L]; lam, omega [K].  Returns h."""
+def ssm_scan_complex_fwd(u, r, phi, lam, omega, chunk=128, seg_chunks=0, h=None, ckpt=None,
+                         want_h=True, want_ckpt=False, ws=None, stream=None):
+    """Complex forward.  u [B,L,K] complex64; r, phi [B,L]; lam, omega [K].  Returns h (the
+    trajectory, or None when ``want_h`` is false and no ``h`` is given), or (h, ckpt) when
+    ``want_ckpt`` is true or a ``ckpt`` [B, ceil(L/chunk), K] complex64 buffer is given."""
     _need_cuda(u, r, phi, lam, omega)
     if u.dtype != torch.complex64:
         raise ValueError("u must be complex64")
     B, L, K = u.shape
     shape = complex_shape(B, L, K, chunk, seg_chunks)
-    if h is None:
+    if h is None and want_h:
         h = torch.empty_like(u)
+    ret_ck = want_ckpt or ckpt is not None
+    if ckpt is None and want_ckpt:
+        ckpt = torch.empty((B, -(-L // chunk), K), dtype=torch.complex64, device=u.device)
     ws = _workspace(complex_workspace_bytes(shape, False), u.device, ws)
     code = lib().ssm_scan_complex_fwd(ctypes.byref(shape), _p(u), _p(r), _p(phi), _p(lam),
-                                      _p(omega), _p(h), _p(ws), ws.numel() * ws.element_size(),
-                                      _stream(stream))
+                                      _p(omega), _p(h), _p(ckpt), _p(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_scan_complex_fwd")
-    return h
+    return (h, ckpt) if ret_ck else h
 
 
-def ssm_scan_complex_bwd(h, r, phi, lam, omega, g, chunk=128, seg_chunks=0, out=None, ws=None,
-                         stream=None):
-    """Complex backward of Re sum conj(g) h.  Returns dict du, dr, dphi, dlambda, domega."""
-    _need_cuda(h, r, phi, lam, omega, g)
-    B, L, K = h.shape
-    shape = complex_shape(B, L, K, chunk, seg_chunks)
+def _complex_grads(g, r, phi, lam, omega, out):
     if out is None:
         out = dict(du=torch.empty_like(g), dr=torch.empty_like(r), dphi=torch.empty_like(phi),
                    dlambda=torch.empty_like(lam), domega=torch.empty_like(omega))
-    ws = _workspace(complex_workspace_bytes(shape, True), h.device, ws)
-    code = lib().ssm_scan_complex_bwd(ctypes.byref(shape), _p(h), _p(r), _p(phi), _p(lam),
-                                      _p(omega), _p(g), _p(out["du"]), _p(out["dr"]),
+    return out
+
+
+def ssm_scan_complex_bwd(u, r, phi, lam, omega, ckpt, g, chunk=128, seg_chunks=0, out=None,
+                         ws=None, stream=None):
+    """Complex backward of Re sum conj(g) h from the forward's checkpoints (each chunk's
+    trajectory recomputed from its entering checkpoint).  Returns dict du, dr, dphi, dlambda,
+    domega."""
+    _need_cuda(u, r, phi, lam, omega, ckpt, g)
+    B, L, K = u.shape
+    shape = complex_shape(B, L, K, chunk, seg_chunks)
+    out = _complex_grads(g, r, phi, lam, omega, out)
+    ws = _workspace(complex_workspace_bytes(shape, True), u.device, ws)
+    code = lib().ssm_scan_complex_bwd(ctypes.byref(shape), _p(u), _p(r), _p(phi), _p(lam),
+                                      _p(omega), _p(ckpt), _p(g), _p(out["du"]), _p(out["dr"]),
                                       _p(out["dphi"]), _p(out["dlambda"]), _p(out["domega"]),
                                       _p(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(code, "ssm_scan_complex_bwd")
+    return out
+
+
+def ssm_scan_complex_bwd_traj(h, r, phi, lam, omega, g, chunk=128, seg_chunks=0, out=None,
+                              ws=None, stream=None):
+    """Complex backward of Re sum conj(g) h reading the stored trajectory h.  Returns dict du,
+    dr, dphi, dlambda, domega."""
+    _need_cuda(h, r, phi, lam, omega, g)
+    B, L, K = h.shape
+    shape = complex_shape(B, L, K, chunk, seg_chunks)
+    out = _complex_grads(g, r, phi, lam, omega, out)
+    ws = _workspace(complex_workspace_bytes(shape, True), h.device, ws)
+    code = lib().ssm_scan_complex_bwd_traj(ctypes.byref(shape), _p(h), _p(r), _p(phi), _p(lam),
+                                           _p(omega), _p(g), _p(out["du"]), _p(out["dr"]),
+                                           _p(out["dphi"]), _p(out["dlambda"]),
+                                           _p(out["domega"]), _p(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "ssm_scan_complex_bwd_traj")
     return out
 
 

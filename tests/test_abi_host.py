@@ -44,7 +44,7 @@ def test_exports_every_declared_symbol(S):
 
 def test_abi_version_and_status_strings(S):
     L = S.lib()
-    assert L.ssm_scan_abi_version() == 3
+    assert L.ssm_scan_abi_version() == 4
     for code in range(8):
         assert L.ssm_status_string(code).decode().startswith(S.STATUS_NAMES[code])
     assert L.ssm_status_string(99) == b"unknown ssm_status"
@@ -207,14 +207,51 @@ def test_complex_validation(S):
     assert S.complex_workspace_bytes(odd, True) == 0
     badT = S.complex_shape(2, 64, 16, 48)
     assert S.complex_workspace_bytes(badT, False) == 0
-    p = _fake_ptrs(7)
+    p = _fake_ptrs(8)  # u, r, phi, lambda, omega, h, ckpt, ws
     assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *p, need_f - 1, None) == 4
     q = list(p)
     q[1] = None
     assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *q, need_f, None) == 1
-    pb = _fake_ptrs(12)
+    q = list(p)
+    q[5] = q[6] = None  # neither the trajectory nor the checkpoints: nothing to write
+    assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *q, need_f, None) == 1
+    q = list(p)
+    q[5] = None  # checkpoints only is a valid forward
+    q[6] = ctypes.c_void_p(0x100004)
+    assert L.ssm_scan_complex_fwd(ctypes.byref(shp), *q, need_f, None) == 3
+    pb = _fake_ptrs(13)  # checkpointed backward: u, r, phi, lambda, omega, ckpt, g, 5 outputs, ws
     pb[5] = ctypes.c_void_p(0x100004)
     assert L.ssm_scan_complex_bwd(ctypes.byref(shp), *pb, need_b, None) == 3
+    pb = _fake_ptrs(13)
+    pb[5] = None  # the checkpoints are required
+    assert L.ssm_scan_complex_bwd(ctypes.byref(shp), *pb, need_b, None) == 1
+    pb = _fake_ptrs(13)
+    assert L.ssm_scan_complex_bwd(ctypes.byref(shp), *pb, need_b - 1, None) == 4
+    pt = _fake_ptrs(12)  # trajectory backward: h, r, phi, lambda, omega, g, 5 outputs, ws
+    pt[5] = ctypes.c_void_p(0x100004)
+    assert L.ssm_scan_complex_bwd_traj(ctypes.byref(shp), *pt, need_b, None) == 3
+
+
+def test_complex_checkpoint_bytes(S):
+    # B * ceil(L / T) * K complex64 values
+    assert S.complex_checkpoint_bytes(S.complex_shape(16, 4096, 2048, 128)) == 16 * 32 * 2048 * 8
+    assert S.complex_checkpoint_bytes(S.complex_shape(3, 517, 130, 32)) == 3 * 17 * 130 * 8
+    assert S.complex_checkpoint_bytes(S.complex_shape(2, 0, 64, 64)) == 0
+    assert S.complex_checkpoint_bytes(S.complex_shape(2, 64, 15, 32)) == 0  # odd K: invalid
+    # the backward workspace covers the chunk-trajectory scratch, which stays O(L / T): doubling
+    # L at a fixed problem width never more than doubles it, and it is capped at 64 MiB or the
+    # checkpoints, whichever is larger
+    for B, K in ((16, 2048), (1, 64), (2, 256)):
+        prev = None
+        for L in (4096, 8192, 16384, 32768):
+            shp = S.complex_shape(B, L, K, 128)
+            ws = S.complex_workspace_bytes(shp, True)
+            ck = S.complex_checkpoint_bytes(shp)
+            traj_cap = max(64 << 20, ck)
+            assert ws <= traj_cap + B * L * 8 * ((K + 63) // 64) + 8 * B * K * (L // 128) * 4 + (1 << 20)
+            if prev is not None:
+                assert ws <= 2 * prev + (1 << 20)
+            prev = ws
 
 
 def test_status_null_workspace(S):
@@ -242,7 +279,11 @@ def test_kernel_launch_counts(S):
     assert S.kernel_launches(blocks, False) == 1 and S.kernel_launches(blocks, True) == 9
     assert S.kernel_launches(S.real_shape(2, 0, 32, 16, 128), True) == 0
     assert S.kernel_launches(S.real_shape(2, 8, 32, 12, 128), True) == -1
-    assert S.complex_kernel_launches(S.complex_shape(16, 4096, 2048, 128), True) == 3
+    big = S.complex_shape(16, 4096, 2048, 128)
+    # checkpointed backward: one main launch (512 CTAs, no time split) + the two reductions;
+    # the trajectory backward: main + two reductions as well
+    assert S.complex_kernel_launches(big, 1) == 3 and S.complex_kernel_launches(big, 2) == 3
+    assert S.complex_kernel_launches(big, 0) == 1 and S.complex_kernel_launches(big, 3) == -1
     # PD-SSM: one scan kernel per call (argmax / score gradient fused) at the bench size; time
     # segments below 128 CTAs add summary + carry; K * (128 / N) > 256 adds the separate kernel
     pd = S.pdssm_shape(8, 5120, 256, 16, 8)

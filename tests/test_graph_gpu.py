@@ -96,17 +96,34 @@ def test_captured_complex_and_pdssm_and_projection_replay_bitwise(S):
 
     def cstep():
         S.ssm_scan_complex_fwd(a["u"], a["r"], a["phi"], a["lam"], a["omega"], h=h)
-        S.ssm_scan_complex_bwd(h, a["r"], a["phi"], a["lam"], a["omega"], a["g"], out=outc)
+        S.ssm_scan_complex_bwd_traj(h, a["r"], a["phi"], a["lam"], a["omega"], a["g"], out=outc)
 
     _capture_and_replay(cstep, a, {k: torch.from_numpy(v).cuda() for k, v in c2.items()})
     got = {"h": h.clone(), **{k: v.clone() for k, v in outc.items()}}
     b = {k: torch.from_numpy(v).cuda() for k, v in c2.items()}
     h2 = S.ssm_scan_complex_fwd(b["u"], b["r"], b["phi"], b["lam"], b["omega"])
-    o2 = S.ssm_scan_complex_bwd(h2, b["r"], b["phi"], b["lam"], b["omega"], b["g"])
+    o2 = S.ssm_scan_complex_bwd_traj(h2, b["r"], b["phi"], b["lam"], b["omega"], b["g"])
     torch.cuda.synchronize()
     assert torch.equal(got["h"], h2)
     for k in o2:
         assert torch.equal(got[k], o2[k]), k
+
+    # complex mode from checkpoints (forward writing checkpoints, checkpointed backward)
+    ck = torch.empty((2, -(-300 // 128), 128), dtype=torch.complex64, device="cuda")
+    outk = {k: torch.empty_like(v) for k, v in outc.items()}
+
+    def kstep():
+        S.ssm_scan_complex_fwd(a["u"], a["r"], a["phi"], a["lam"], a["omega"], h=h, ckpt=ck)
+        S.ssm_scan_complex_bwd(a["u"], a["r"], a["phi"], a["lam"], a["omega"], ck, a["g"], out=outk)
+
+    _capture_and_replay(kstep, a, {k: torch.from_numpy(v).cuda() for k, v in c1.items()})
+    b1 = {k: torch.from_numpy(v).cuda() for k, v in c1.items()}
+    _, ck1 = S.ssm_scan_complex_fwd(b1["u"], b1["r"], b1["phi"], b1["lam"], b1["omega"], want_ckpt=True)
+    o1 = S.ssm_scan_complex_bwd(b1["u"], b1["r"], b1["phi"], b1["lam"], b1["omega"], ck1, b1["g"])
+    torch.cuda.synchronize()
+    assert torch.equal(ck, ck1)
+    for k in o1:
+        assert torch.equal(outk[k], o1[k]), k
 
     # Flash PD-SSM (fused argmax / score gradient, warp-specialised backward)
     p1, p2 = gen.pdssm_inputs(2, 400, 32, 16, 8, seed=1), gen.pdssm_inputs(2, 400, 32, 16, 8, seed=2)

@@ -184,17 +184,30 @@ def test_nonfinite_status(S):
 
 # ------------------------------------------------------------------------------ complex cases
 
-def run_complex(S, c, T, seg_chunks=0):
+def run_complex(S, c, T, seg_chunks=0, bwd="ckpt"):
+    """Complex forward (trajectory and checkpoints) and one of the two backward calls: from the
+    checkpoints (ssm_scan_complex_bwd) or from the stored trajectory (ssm_scan_complex_bwd_traj)."""
     u = to_dev(c["u"], torch.complex64)
     g = to_dev(c["g"], torch.complex64)
     r, phi = to_dev(c["r"], torch.float32), to_dev(c["phi"], torch.float32)
     lam, om = to_dev(c["lam"], torch.float32), to_dev(c["omega"], torch.float32)
-    h = S.ssm_scan_complex_fwd(u, r, phi, lam, om, chunk=T, seg_chunks=seg_chunks)
-    gr = S.ssm_scan_complex_bwd(h, r, phi, lam, om, g, chunk=T, seg_chunks=seg_chunks)
+    h, ck = S.ssm_scan_complex_fwd(u, r, phi, lam, om, chunk=T, seg_chunks=seg_chunks,
+                                   want_ckpt=True)
+    if bwd == "ckpt":
+        gr = S.ssm_scan_complex_bwd(u, r, phi, lam, om, ck, g, chunk=T, seg_chunks=seg_chunks)
+    else:
+        gr = S.ssm_scan_complex_bwd_traj(h, r, phi, lam, om, g, chunk=T, seg_chunks=seg_chunks)
     torch.cuda.synchronize()
-    out = {"h": np64(h)}
+    out = {"h": np64(h), "ckpt": np64(ck)}
     out.update({k: np64(v) for k, v in gr.items()})
     return out
+
+
+def check_complex_ckpt(got, T):
+    """The forward's checkpoints are its own trajectory at every chunk's last step, bit for bit."""
+    L = got["h"].shape[1]
+    ends = [min(L, (c + 1) * T) - 1 for c in range(got["ckpt"].shape[1])]
+    assert np.array_equal(got["ckpt"], got["h"][:, ends, :])
 
 
 def check_complex(got, ref, sel=None):
@@ -215,11 +228,42 @@ def check_complex(got, ref, sel=None):
 @pytest.mark.parametrize("B,L,K,T,sc", [(2, 300, 64, 128, 0), (3, 517, 130, 32, 2),
                                         (1, 1000, 64, 64, 3), (2, 77, 2, 16, 0),
                                         (1, 1, 64, 128, 0), (2, 600, 200, 256, 1)])
-def test_complex_shapes(S, oracle_mod, B, L, K, T, sc):
+@pytest.mark.parametrize("bwd", ["ckpt", "traj"])
+def test_complex_shapes(S, oracle_mod, B, L, K, T, sc, bwd):
     c = gen.complex_inputs(B, L, K, seed=L + K)
-    got = run_complex(S, c, T, sc)
+    got = run_complex(S, c, T, sc, bwd)
     ref = oracle_mod.complex_(c["u"], c["r"], c["phi"], c["lam"], c["omega"], c["g"])
     check_complex(got, ref)
+    check_complex_ckpt(got, T)
+
+
+def test_complex_backward_variants_agree(S):
+    """Both backward calls sweep the same adjoint with the same transitions; the checkpointed one
+    recomputes h_{t-1} from the checkpoints, so they agree to fp32 recurrence rounding."""
+    c = gen.complex_inputs(2, 700, 130, seed=5)
+    a = run_complex(S, c, 64, 3, "ckpt")
+    b = run_complex(S, c, 64, 3, "traj")
+    for k in ("du", "dr", "dphi", "dlambda", "domega"):
+        assert rel_l2(a[k], b[k]) <= 1e-5, k
+
+
+def test_complex_forward_checkpoints_only(S, oracle_mod):
+    """With no trajectory buffer the forward writes only the checkpoints, and the checkpointed
+    backward needs nothing else: the O(L/T) path."""
+    c = gen.complex_inputs(2, 333, 64, seed=9)
+    u = to_dev(c["u"], torch.complex64)
+    g = to_dev(c["g"], torch.complex64)
+    r, phi = to_dev(c["r"], torch.float32), to_dev(c["phi"], torch.float32)
+    lam, om = to_dev(c["lam"], torch.float32), to_dev(c["omega"], torch.float32)
+    h, ck = S.ssm_scan_complex_fwd(u, r, phi, lam, om, chunk=32, want_h=False, want_ckpt=True)
+    assert h is None
+    gr = S.ssm_scan_complex_bwd(u, r, phi, lam, om, ck, g, chunk=32)
+    torch.cuda.synchronize()
+    ref = oracle_mod.complex_(c["u"], c["r"], c["phi"], c["lam"], c["omega"], c["g"])
+    ends = [min(333, (i + 1) * 32) - 1 for i in range(ck.shape[1])]
+    assert rel_l2(np64(ck), ref["h"][:, ends, :]) <= FWD_TOL_F32
+    for k in ("du", "dr", "dphi", "dlambda", "domega"):
+        assert rel_l2(np64(gr[k]), ref[k]) <= GRAD_TOL_F32, k
 
 
 def test_complex_far_phases(S, oracle_mod):
@@ -231,7 +275,8 @@ def test_complex_far_phases(S, oracle_mod):
     c["phi"][1, 200] = 12345.0
     ref = oracle_mod.complex_(c["u"], c["r"], c["phi"], c["lam"], c["omega"], c["g"])
     for sc in (0, 1):
-        check_complex(run_complex(S, c, 64, sc), ref)
+        for bwd in ("ckpt", "traj"):
+            check_complex(run_complex(S, c, 64, sc, bwd), ref)
 
 
 # ------------------------------------------------------------------------------ full-size workloads
@@ -284,7 +329,8 @@ def test_full_size_real_identities(S, name):
     assert abs(np.sum(inp["Dskip"] * got["dD"]) - skip) <= 1e-4 * abs(skip)
 
 
-def test_full_size_complex_sampled(S, oracle_mod):
+@pytest.mark.parametrize("bwd", ["ckpt", "traj"])
+def test_full_size_complex_sampled(S, oracle_mod, bwd):
     w = gen.WORKLOADS["sparc_complex"]
     c = gen.workload_inputs("sparc_complex")
     sel = _channel_sample(w.modes)
@@ -292,7 +338,8 @@ def test_full_size_complex_sampled(S, oracle_mod):
     mask[sel] = 1.0
     cm = dict(c)
     cm["g"] = (c["g"] * mask).astype(np.complex64)
-    got = run_complex(S, cm, w.chunk)
+    got = run_complex(S, cm, w.chunk, 0, bwd)
+    check_complex_ckpt(got, w.chunk)
     ref = oracle_mod.complex_(c["u"][..., sel], c["r"], c["phi"], c["lam"][sel],
                               c["omega"][sel], cm["g"][..., sel])
     pick = {"h": got["h"][..., sel], "du": got["du"][..., sel], "dr": got["dr"],

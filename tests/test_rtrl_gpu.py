@@ -55,7 +55,7 @@ def test_rtrl_matches_gpu_adjoint(S):
     d = dev(c)
     rt = S.ssm_scan_complex_rtrl(d["u"], d["r"], d["phi"], d["lam"], d["omega"], d["g"])
     h = S.ssm_scan_complex_fwd(d["u"], d["r"], d["phi"], d["lam"], d["omega"])
-    adj = S.ssm_scan_complex_bwd(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"])
+    adj = S.ssm_scan_complex_bwd_traj(h, d["r"], d["phi"], d["lam"], d["omega"], d["g"])
     torch.cuda.synchronize()
     for k in ("dlambda", "domega"):
         assert rel(rt[k].cpu().numpy(), adj[k].cpu().numpy()) <= GRAD_TOL, k
