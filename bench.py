@@ -21,7 +21,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -40,7 +39,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mamba130m_layer")
+    ap.add_argument("--workload", default="mamba1p4b_layer",
+                    help="default: the largest single-GPU real workload (B=4, L=8192, D=4096, N=16, bf16)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seg-chunks", type=int, default=0)
@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--rtrl", action="store_true",
                     help="complex workloads: time exact structured RTRL (one forward pass that "
                          "accumulates dlambda, domega online) instead of fwd + bwd")
+    ap.add_argument("--ckpt", action="store_true",
+                    help="complex workloads: the forward also writes chunk checkpoints and the "
+                         "backward recomputes from them (ssm_scan_complex_bwd) instead of reading "
+                         "the stored trajectory (ssm_scan_complex_bwd_traj)")
     ap.add_argument("--state", action="store_true",
                     help="pass an initial state h0 and an upstream final-state gradient dhL")
     ap.add_argument("--dtproj", type=int, default=0, metavar="R",
@@ -80,6 +84,11 @@ BWD_OPS_PER_UPDATE = 11
 ZOH_FWD_OPS_PER_UPDATE = 7
 ZOH_BWD_OPS_PER_UPDATE = 19
 SMS, FP32_LANES_PER_SM = 148, 128
+# MUFU ex2 results per SM per clock (measured with a microbenchmark on this B200), and the exp2
+# the kernels evaluate per update: the forward one, the backward two (the chunk walk that finds
+# each window's start state, and the window's own recompute)
+MUFU_EX2_PER_SM = 16
+FWD_EXP2_PER_UPDATE, BWD_EXP2_PER_UPDATE = 1, 2
 
 
 def alu_peak_tops():
@@ -89,6 +98,20 @@ def alu_peak_tops():
     if os.path.exists(p):
         mhz = float(json.load(open(p)).get("sm_max_mhz", mhz))
     return SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12, mhz
+
+
+def clock_roofs(clk, achieved_tops, updates_per_s, exp2_per_update):
+    """The FP32-pipe and MUFU roofs at the SM clock sampled during the timed region (the fixed
+    peak above assumes the maximum clock), and the fractions of them achieved."""
+    mhz = clk.get("sm_mhz") if clk else None
+    if not mhz:
+        return {}
+    fp32 = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
+    mufu = SMS * MUFU_EX2_PER_SM * mhz * 1e6  # exp2 per second
+    return {"sampled_sm_mhz": mhz, "peak_at_sampled_clock": fp32,
+            "frac_at_sampled_clock": achieved_tops / fp32,
+            "mufu_ex2_per_s_at_sampled_clock": mufu,
+            "mufu_frac_at_sampled_clock": updates_per_s * exp2_per_update / mufu}
 
 
 def algorithmic_bytes(w):
@@ -170,55 +193,82 @@ E2E_OVERLAP = ("two buffer sets; each step's host-to-device and device-to-host c
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs.  The raw
+    """SM clock and throttle reasons sampled through NVML every 2 ms while the timed region runs
+    (a background thread), so even a timed region of a few tens of milliseconds gets tens of
+    samples.  The GPU is found by its PCI bus id (falling back to the device index).  The raw
     samples go to clocks_rank<i>.csv in $SSM_BENCH_CLOCKS_DIR (default: the system temp dir)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
+        self.handle = None
+        self.samples = []
         import tempfile
         out = os.environ.get("SSM_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
         self.path = os.path.join(out, f"clocks_rank{index}.csv")
 
-    def start(self):
+    def _open(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        h = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.index)], stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, ValueError):
-            self.proc = None
+            import torch
+            pr = torch.cuda.get_device_properties(self.index)
+            bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = None
+        return nv, (h if h is not None else nv.nvmlDeviceGetHandleByIndex(self.index))
+
+    def start(self):
+        import threading
+        try:
+            self.nv, self.handle = self._open()
+            self.smax = float(self.nv.nvmlDeviceGetMaxClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+            return
+        nv = self.nv
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        self.stop_flag = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1e3
+                except Exception:
+                    break
+                self.samples.append((time.time(), float(mhz), pw, [bool(rs & b) for b in bits]))
+                time.sleep(self.PERIOD_S)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        self.proc.terminate()
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        reasons = set()
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as fh:
+                fh.write("time_s,sm_mhz,power_w," + ",".join(self.NAMES) + "\n")
+                for t, mhz, pw, act in self.samples:
+                    fh.write(f"{t:.4f},{mhz:.0f},{pw:.1f}," + ",".join(str(int(a)) for a in act) + "\n")
+        except OSError:
+            pass
+        for _, _, _, act in self.samples:
+            reasons.update(n for n, a in zip(self.NAMES, act) if a)
+        sm = [s[1] for s in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "reasons": sorted(reasons), "samples": len(sm), "sampler": "NVML, 2 ms period",
+                "power_w_max": max((s[2] for s in self.samples), default=None)}
 
 
 def oracle_sample(w, inp, budget_s=(10.0, 30.0), zoh=False):
@@ -366,9 +416,10 @@ def run_reference(args, w):
 
 
 def complex_algorithmic_bytes(w):
-    """Minimum bytes of one complex fwd + bwd: u read and h written by the forward; h and g read,
-    du written by the backward (8 B each, complex64); r and phi read by both, dr and dphi
-    written (4 B each)."""
+    """Minimum bytes of one complex fwd + bwd: u read and h written by the forward; h (or, from
+    checkpoints, u) and g read, du written by the backward (8 B each, complex64); r and phi read
+    by both, dr and dphi written (4 B each).  The checkpoints (1/T of the trajectory) are left
+    out."""
     BLK, BL = w.batch * w.seqlen * w.modes, w.batch * w.seqlen
     return 16 * BLK + 8 * BL, 24 * BLK + 16 * BL
 
@@ -438,7 +489,10 @@ def main_complex(args, w):
         out = dict(dlambda=out["dlambda"], domega=out["domega"])
         wsr = torch.empty(S.complex_rtrl_workspace_bytes(shape), dtype=torch.uint8, device=dev)
 
-    sets = [dict(d=d, h=h, out=out)]
+    nC = -(-w.seqlen // w.chunk)
+    ck = (torch.empty((w.batch, nC, w.modes), dtype=torch.complex64, device=dev)
+          if args.ckpt else None)
+    sets = [dict(d=d, h=h, ck=ck, out=out)]
 
     def fwd(bs=None):
         bs = bs or sets[0]
@@ -448,15 +502,22 @@ def main_complex(args, w):
                                     chunk=w.chunk, out=oo, ws=wsr, stream=stream)
         else:
             S.ssm_scan_complex_fwd(dd["u"], dd["r"], dd["phi"], dd["lam"], dd["omega"], chunk=w.chunk,
-                                   seg_chunks=args.seg_chunks, h=hh, ws=wsf, stream=stream)
+                                   seg_chunks=args.seg_chunks, h=hh, ckpt=bs["ck"], ws=wsf,
+                                   stream=stream)
 
     def bwd(bs=None):
         bs = bs or sets[0]
         dd, hh, oo = bs["d"], bs["h"], bs["out"]
-        if not args.rtrl:
-            S.ssm_scan_complex_bwd(hh, dd["r"], dd["phi"], dd["lam"], dd["omega"], dd["g"],
-                                   chunk=w.chunk, seg_chunks=args.seg_chunks, out=oo, ws=wsb,
-                                   stream=stream)
+        if args.rtrl:
+            return
+        if args.ckpt:  # recompute every chunk from its checkpoint
+            S.ssm_scan_complex_bwd(dd["u"], dd["r"], dd["phi"], dd["lam"], dd["omega"], bs["ck"],
+                                   dd["g"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=oo,
+                                   ws=wsb, stream=stream)
+        else:  # read h_{t-1} from the stored trajectory
+            S.ssm_scan_complex_bwd_traj(hh, dd["r"], dd["phi"], dd["lam"], dd["omega"], dd["g"],
+                                        chunk=w.chunk, seg_chunks=args.seg_chunks, out=oo, ws=wsb,
+                                        stream=stream)
 
     def allreduce(bs=None):
         oo = (bs or sets[0])["out"]
@@ -490,6 +551,7 @@ def main_complex(args, w):
     t_step, t_fwd, t_bwd = tt.tolist()
 
     sets.append(dict(d={k: torch.empty_like(v) for k, v in d.items()}, h=torch.empty_like(h),
+                     ck=torch.empty_like(ck) if ck is not None else None,
                      out={k: torch.empty_like(v) for k, v in out.items()}))
 
     def compute(bs):
@@ -509,7 +571,8 @@ def main_complex(args, w):
         fb, bb = 16 * w.batch * w.seqlen * w.modes + 8 * w.batch * w.seqlen, 0
     bwd_gbs = bb / (t_bwd / args.steps) / 1e9 if bb else 0.0
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
-    launches = (S.complex_kernel_launches(shape, False) + S.complex_kernel_launches(shape, True)) * args.steps
+    launches = (S.complex_kernel_launches(shape, 0) +
+                S.complex_kernel_launches(shape, 1 if args.ckpt else 2)) * args.steps
     if args.rtrl:
         launches = 2 * args.steps
     if rank == 0:
@@ -521,6 +584,8 @@ def main_complex(args, w):
             "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
                        "modes": w.modes, "chunk": w.chunk, "io": "complex64",
                        "training": "rtrl (online, forward only)" if args.rtrl else "bptt (fwd + bwd)",
+                       "backward": ("from chunk checkpoints (ssm_scan_complex_bwd)" if args.ckpt
+                                    else "from the stored trajectory (ssm_scan_complex_bwd_traj)"),
                        "l2": "flushed (256 MiB write) before every timed step",
                        "parallelism": f"dp{world} (weak: one full batch per rank; "
                                       "dlambda/domega all-reduced)" if world > 1 else "single GPU"},
@@ -530,12 +595,16 @@ def main_complex(args, w):
                           "algorithmic_bytes_per_launch": fb,
                           "traffic": measured_traffic("ssm_scan_complex_rtrl", "complex_scan.cu",
                                                       w.name)} if args.rtrl else
-                         {"bound": "hbm", "kernel": "ssm_scan_complex_bwd call (cplx_bwd_kernel + "
-                          "reductions)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
+                         {"bound": "hbm",
+                          "kernel": ("ssm_scan_complex_bwd call (cplx_bwd_ckpt_kernel + reductions)"
+                                     if args.ckpt else "ssm_scan_complex_bwd_traj call "
+                                     "(cplx_bwd_kernel + reductions)"),
+                          "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
                           "algorithmic_bytes_per_launch": bb,
-                          "traffic": measured_traffic("ssm_scan_complex_bwd", "complex_scan.cu",
-                                                      w.name)}),
+                          "traffic": measured_traffic("ssm_scan_complex_bwd" if args.ckpt else
+                                                      "ssm_scan_complex_bwd_traj",
+                                                      "complex_scan.cu", w.name)}),
             "hbm_frac_fwd": fwd_gbs / hbm, "hbm_frac_bwd": bwd_gbs / hbm,
             "ms_fwd": 1e3 * t_fwd / args.steps, "ms_bwd": 1e3 * t_bwd / args.steps,
             "e2e": {"value": world * upd_rank * args.steps / t_e2e, "unit": UNIT,
@@ -951,7 +1020,9 @@ def main():
                                       f"{alu_mhz:.0f} MHz (FMA = 1 op)",
                          "algorithmic_ops_per_launch": bo,
                          "algorithmic_bytes_per_launch": bb,
-                         "traffic": measured_traffic("ssm_scan_bwd", "real_bwd.cu", w.name)},
+                         "traffic": measured_traffic("ssm_scan_bwd", "real_bwd.cu", w.name),
+                         **clock_roofs(clk, bwd_tops, upd_rank / (t_bwd / args.steps),
+                                       BWD_EXP2_PER_UPDATE)},
             "hbm": {"achieved_bwd": bwd_gbs, "achieved_fwd": fwd_gbs, "achieved_step": step_gbs,
                     "peak": hbm, "unit": "GB/s", "peak_kind": peak_kind},
             "hbm_frac_bwd": bwd_gbs / hbm,
