@@ -106,17 +106,20 @@ __global__ void real_carry_bwd_kernel(int B, int nseg, int DN, const float* __re
 // ------------------------------------------------------------------------------------------------
 // Backward main kernel.  Chunks of the segment in reverse order; per chunk:
 //   pass A: stream the chunk forward in 32-step sub-tiles (asynchronous two-stage ring).  Per
-//           sub-tile: delta and sigmoid(delta_raw) from one exp per (t, d); (delta, delta) and
+//           sub-tile: delta and sigmoid(delta_raw) from one exp per (t, d); (delta, sigma) and
 //           the state at every 4-step window start go to this CTA's L2-resident workspace region;
 //           the recurrence advances through the sub-tile.
 //   pass B: stream the sub-tiles in reverse.  For each 4-step window, last first: recompute
 //           (a_t, a_t h_{t-1}) forward from the window's start state into registers, then sweep
 //           the adjoint back through the window.
-//           After each step: the step's dB / dC values (4 states each) summed over the warp's
-//           channels by a shuffle reduce-scatter that leaves one (dB or dC, state) sum per lane.
-//           After each window: reduce-scatter of the per-channel sums over the NG lanes, dx and
-//           ddelta_raw stored directly, and the warps' dB / dC sums (double-buffered shared
-//           memory, one 16-byte store per lane) added over the CTA's warps into its partial rows.
+// Channel sums of dB and dC.  A thread's four state slots are rotated by its position `rot` among
+// four neighbouring channel lanes (slot j holds state n0 + ((j + rot) & 3)), so after each step
+// the four lanes exchange their per-slot values in three shuffle rounds that all send the same
+// slot (an all-to-all with uniform register indices): each lane ends with the sum over the four
+// channels of one state, for dB and for dC.  After each window the eight four-channel groups of
+// the CTA meet in shared memory and one thread per (step, dB or dC, state) adds them into the
+// CTA's partial row.  The per-(t, d) sums over the states (dx, ddelta_raw) are a reduce-scatter
+// over the NG lanes of a channel, per window.
 template <int N>
 struct BwdCfg {
     static constexpr int S = 4;            // states per thread
@@ -126,34 +129,84 @@ struct BwdCfg {
     static constexpr int NT = DT * NG;     // threads per CTA
     static constexpr int W = 4;            // steps per window
     static constexpr int TT = 32;          // steps per staged sub-tile
+    static constexpr int GRP = DT / 4;     // four-channel groups per CTA
+    static constexpr int RS = 9 * N;       // stride (floats) of a group's window sums in shared memory
+    static_assert(W * 2 * N == NT, "one (step, dB or dC, state) output of a window per thread");
 };
 
 template <typename E, int N>
 struct BwdSmem {
-    static constexpr int TT = BwdCfg<N>::TT, DT = BwdCfg<N>::DT, W = BwdCfg<N>::W;
+    using Cfg = BwdCfg<N>;
+    static constexpr int TT = Cfg::TT, DT = Cfg::DT;
     static constexpr int XE = TT * DT, BE = TT * N;
+    static constexpr int RE = TT * 4 * N;  // fp32 tile of B or C with the four slot rotations
     // pass A stage: x, delta_raw, B (raw)
     static constexpr int A_STAGE = (2 * XE + BE) * (int)sizeof(E);
     static constexpr int A_DD = 2 * A_STAGE;              // (delta, delta*x) float2 [TT][DT]
-    static constexpr int A_BF = A_DD + XE * 8;            // B fp32 [TT][N]
-    static constexpr int A_END = A_BF + BE * 4;
+    static constexpr int A_BR = A_DD + XE * 8;            // B rotated fp32 [TT][4][N]
+    static constexpr int A_END = A_BR + RE * 4;
     // pass B stage: (delta, sigma) float2, x, dy, B, C (raw)
     static constexpr int B_STAGE = XE * 8 + (2 * XE + 2 * BE) * (int)sizeof(E);
-    static constexpr int B_BF = 2 * B_STAGE;              // B fp32
-    static constexpr int B_CF = B_BF + BE * 4;            // C fp32
-    static constexpr int B_RED = B_CF + BE * 4;           // warp sums of dB/dC, 2 x [warps][W][2N]
-    static constexpr int B_END = B_RED + 2 * (BwdCfg<N>::NT / 32) * 2 * N * W * 4;
+    static constexpr int B_BR = 2 * B_STAGE;              // B rotated fp32
+    static constexpr int B_CR = B_BR + RE * 4;            // C rotated fp32
+    static constexpr int B_RED = B_CR + RE * 4;           // window sums, 2 x [GRP][RS] floats
+    static constexpr int B_END = B_RED + 2 * Cfg::GRP * Cfg::RS * 4;
     static constexpr int BYTES = A_END > B_END ? A_END : B_END;
+    static_assert(A_STAGE % 16 == 0 && B_STAGE % 16 == 0, "16-byte aligned stages");
 };
+
+// Rows [0, rows) of a staged [rows][N] tile to fp32 with the four slot rotations of every group of
+// four states: dst[(row * 4 + k) * N + 4 g + j] = src[row * N + 4 g + ((j + k) & 3)], so a thread
+// of rotation k reads its four slots with one 16-byte load.
+template <typename E, int N>
+__device__ __forceinline__ void rotate_rows(float* __restrict__ dst, const E* __restrict__ src,
+                                            int rows, int tid, int nthreads) {
+    constexpr int G = N / 4;
+    for (int i = tid; i < rows * G; i += nthreads) {
+        const int row = i / G, g = i - row * G;
+        float v[4];
+        if constexpr (sizeof(E) == 2) {
+            const uint2 w = *reinterpret_cast<const uint2*>(src + row * N + 4 * g);
+            v[0] = __uint_as_float(w.x << 16);
+            v[1] = __uint_as_float(w.x & 0xffff0000u);
+            v[2] = __uint_as_float(w.y << 16);
+            v[3] = __uint_as_float(w.y & 0xffff0000u);
+        } else {
+            const float4 w = *reinterpret_cast<const float4*>(src + row * N + 4 * g);
+            v[0] = w.x;
+            v[1] = w.y;
+            v[2] = w.z;
+            v[3] = w.w;
+        }
+        float* o = dst + row * 4 * N + 4 * g;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4*>(o + k * N) =
+                make_float4(v[k & 3], v[(k + 1) & 3], v[(k + 2) & 3], v[(k + 3) & 3]);
+    }
+}
+
+// The thread's four slots of one state row (a [.., N] row of a [*, D, N] array), in slot order.
+__device__ __forceinline__ void ld_slots(float2 (&o)[2], const float* row, const int (&sidx)[4]) {
+    o[0] = make_float2(row[sidx[0]], row[sidx[1]]);
+    o[1] = make_float2(row[sidx[2]], row[sidx[3]]);
+}
+__device__ __forceinline__ void st_slots(float* row, const float2 (&o)[2], const int (&sidx)[4]) {
+    row[sidx[0]] = o[0].x;
+    row[sidx[1]] = o[0].y;
+    row[sidx[2]] = o[1].x;
+    row[sidx[3]] = o[1].y;
+}
 
 // MINB: CTAs per SM the register allocation must allow.  4 (126 registers for the Euler N = 16
 // kernel) lets grids of up to 592 CTAs run in one wave; 3 leaves the compiler more registers,
-// which is 2 % faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
+// which is faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
 template <typename E, int N, bool ZOH, int MINB>
 __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N>;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;
+    constexpr int GRP = Cfg::GRP, RS = Cfg::RS;
     // per-step channel sums over the states: sum g w' B (dx), sum A q, and for zero-order hold
     // also sum g a B (ddelta; with Euler it equals the first)
     constexpr int SV = ZOH ? 3 : 2;
@@ -164,6 +217,14 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     const int b = blockIdx.y, seg = p.seg0 + blockIdx.z;
     const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * Cfg::S;
     const bool dv = d < p.D;
+    // slot rotation and the all-to-all partners among the four channel lanes of this group
+    const int cl = (tid & 31) / NG, rot = cl & 3, grp = dl >> 2;
+    const int src1 = ng + NG * ((cl & ~3) | ((rot - 1) & 3));
+    const int src2 = ng + NG * ((cl & ~3) | ((rot - 2) & 3));
+    const int src3 = ng + NG * ((cl & ~3) | ((rot - 3) & 3));
+    int sidx[4];  // state held by each slot
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sidx[j] = n0 + ((j + rot) & 3);
     const int T = p.T;
     const int TTe = T < TT ? T : TT;
     const int c_begin = seg * p.seg_chunks;
@@ -171,25 +232,27 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
 
     float2 A[P2], A2[P2], v[P2], dA[P2];
     float2 Ar[P2];  // zero-order hold: 1 / A
+    {
+        const float* al = p.A_log + (size_t)(dv ? d : 0) * N;
 #pragma unroll
-    for (int i = 0; i < P2; ++i) {
-        A[i] = dv ? make_float2(-expf(p.A_log[d * N + n0 + 2 * i]), -expf(p.A_log[d * N + n0 + 2 * i + 1]))
-                  : make_float2(0.0f, 0.0f);
-        A2[i] = __fmul2_rn(A[i], f2(kLog2e));
-        if (ZOH)
-            Ar[i] = dv ? make_float2(-expf(-p.A_log[d * N + n0 + 2 * i]),
-                                     -expf(-p.A_log[d * N + n0 + 2 * i + 1]))
-                       : make_float2(0.0f, 0.0f);
-        v[i] = make_float2(0.0f, 0.0f);
-        dA[i] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < P2; ++i) {
+            A[i] = dv ? make_float2(-expf(al[sidx[2 * i]]), -expf(al[sidx[2 * i + 1]]))
+                      : make_float2(0.0f, 0.0f);
+            A2[i] = __fmul2_rn(A[i], f2(kLog2e));
+            if (ZOH)
+                Ar[i] = dv ? make_float2(-expf(-al[sidx[2 * i]]), -expf(-al[sidx[2 * i + 1]]))
+                           : make_float2(0.0f, 0.0f);
+            v[i] = make_float2(0.0f, 0.0f);
+            dA[i] = make_float2(0.0f, 0.0f);
+        }
     }
     if (dv) {
         // the adjoint entering from the segment's end: handed over by the carry or by the later
         // block, or, for the last segment, the upstream gradient of the final state (or zero)
-        const float* src = seg < p.nseg - 1 ? p.vin + (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N + n0
-                           : p.dhL          ? p.dhL + ((size_t)b * p.D + d) * N + n0
+        const float* src = seg < p.nseg - 1 ? p.vin + (((size_t)b * (p.nseg - 1) + seg) * p.D + d) * N
+                           : p.dhL          ? p.dhL + ((size_t)b * p.D + d) * N
                                             : nullptr;
-        if (src) ld_pairs<4>(v, src);
+        if (src) ld_slots(v, src, sidx);
     }
     float dDacc = 0.0f;
     const float dsk = dv ? p.Dskip[d] : 0.0f;
@@ -207,6 +270,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     float* scr = p.bnd_scratch + cta * real_bwd_scratch_floats(N, T);
     float* bnd = scr + (size_t)tid * 4;                        // window starts: [T/W][NT][4]
     float2* dsg = reinterpret_cast<float2*>(scr + (size_t)(T / W) * NT * 4);  // (delta, sigma) [T][DT]
+    const int roff = rot * N + n0;  // this thread's slots within a rotated row of 4N floats
 
     for (int c = c_end - 1; c >= c_begin; --c) {
         const int tc = c * T;
@@ -217,15 +281,15 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
         {
             float2 h[P2];
             if (c > 0 && dv) {
-                ld_pairs<4>(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N + n0);
+                ld_slots(h, p.ckpt_in + (((size_t)b * p.nC + (c - 1)) * p.D + d) * N, sidx);
             } else if (p.h0 && dv) {
-                ld_pairs<4>(h, p.h0 + ((size_t)b * p.D + d) * N + n0);
+                ld_slots(h, p.h0 + ((size_t)b * p.D + d) * N, sidx);
             } else {
 #pragma unroll
                 for (int i = 0; i < P2; ++i) h[i] = make_float2(0.0f, 0.0f);
             }
             float2* sdd = reinterpret_cast<float2*>(smem + Sm::A_DD);
-            float* sBf = reinterpret_cast<float*>(smem + Sm::A_BF);
+            float* sBr = reinterpret_cast<float*>(smem + Sm::A_BR);
             auto stage = [&](int k) { return reinterpret_cast<E*>(smem + k * Sm::A_STAGE); };
             auto issue = [&](int j, int k) {
                 const int t0 = tc + j * TTe;
@@ -262,7 +326,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                     sdd[i] = make_float2(dlt, dlt * Elem<E>::to_f(sx[i]));
                     __stcg(&dsg[(size_t)(j * TTe) * DT + i], make_float2(dlt, sig));
                 }
-                for (int i = tid; i < TTe * N; i += NT) sBf[i] = Elem<E>::to_f(sB[i]);
+                rotate_rows<E, N>(sBr, sB, TTe, tid, NT);
                 __syncthreads();
                 for (int w = 0; w < TTe / W; ++w) {
                     __stcg(reinterpret_cast<float4*>(bnd + (size_t)((j * TTe) / W + w) * NT * 4),
@@ -272,7 +336,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         const int r = w * W + u;
                         const float2 dd = sdd[r * DT + dl];
                         float2 bq[P2];
-                        ld_pairs<4>(bq, sBf + r * N + n0);
+                        ld_pairs<4>(bq, sBr + r * 4 * N + roff);
 #pragma unroll
                         for (int i = 0; i < P2; ++i) {
                             const float2 zl2 = __fmul2_rn(f2(dd.x), A2[i]);
@@ -291,8 +355,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
 
         // ------------------------------------------------------------------ pass B
         {
-            float* sBf = reinterpret_cast<float*>(smem + Sm::B_BF);
-            float* sCf = reinterpret_cast<float*>(smem + Sm::B_CF);
+            float* sBr = reinterpret_cast<float*>(smem + Sm::B_BR);
+            float* sCr = reinterpret_cast<float*>(smem + Sm::B_CR);
             float* sred = reinterpret_cast<float*>(smem + Sm::B_RED);
             auto stage = [&](int k) { return smem + k * Sm::B_STAGE; };
             auto issue = [&](int j, int k) {
@@ -332,17 +396,22 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                 const E* sdy = sx + Sm::XE;
                 const E* sB = sx + 2 * Sm::XE;
                 const E* sC = sB + Sm::BE;
-                for (int i = tid; i < TTe * N; i += NT) {
-                    sBf[i] = Elem<E>::to_f(sB[i]);
-                    sCf[i] = Elem<E>::to_f(sC[i]);
-                }
+                rotate_rows<E, N>(sBr, sB, TTe, tid, NT);
+                rotate_rows<E, N>(sCr, sC, TTe, tid, NT);
                 __syncthreads();
                 const int nw = TTe / W;  // 4 or 8 windows, even
                 const int wbase = (j * TTe) / W;
 
                 float2 aa[W][P2], pp[W][P2];  // (a_t, a_t h_{t-1}) of the current window
-                // after a window's reverse sweep: outputs, then its dB/dC column sums
-                auto finish_window = [&](int q, float (&sv)[SV * W], const float* red) {
+                // after a window's reverse sweep: outputs, then its dB/dC sums over the CTA
+                auto finish_window = [&](int q, float (&sv)[SV * W], const float (&sbv)[W],
+                                         const float (&scv)[W]) {
+                    float* red = sred + (q & 1) * GRP * RS;
+#pragma unroll
+                    for (int u = 0; u < W; ++u) {
+                        red[grp * RS + u * N2 + n0 + rot] = sbv[u];
+                        red[grp * RS + u * N2 + N + n0 + rot] = scv[u];
+                    }
                     reduce_scatter<SV * W, NG>(sv, ng);
 #pragma unroll
                     for (int jj = 0; jj < W / NG; ++jj) {
@@ -360,15 +429,14 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                             dDacc = fmaf(dyv, xv, dDacc);
                         }
                     }
-                    __syncthreads();  // the warps' dB/dC sums of the window are in `red`
+                    __syncthreads();  // every group's sums of the window are in `red`
                     {
-                        // output (step u, dB or dC, state n) = sum over the warps
-                        const int u = tid / N2, wh = (tid / N) % 2, n = tid % N;
+                        // output (step u, dB or dC, state) = sum over the CTA's groups
                         float s = 0.0f;
 #pragma unroll
-                        for (int w = 0; w < NT / 32; ++w) s += red[(w * W + u) * N2 + wh * N + n];
-                        const int r = q * W + u;
-                        if (r < rows) partb[(size_t)(t0 + r) * N2 + wh * N + n] = s;
+                        for (int g = 0; g < GRP; ++g) s += red[g * RS + tid];
+                        const int r = q * W + tid / N2;
+                        if (r < rows) partb[(size_t)(t0 + r) * N2 + (tid % N2)] = s;
                     }
                 };
 
@@ -385,7 +453,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         const int r = q * W + u;
                         const float dlt = sds[r * DT + dl].x;
                         const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                        ld_pairs<4>(bqs[u], sBf + r * N + n0);
+                        ld_pairs<4>(bqs[u], sBr + r * 4 * N + roff);
                         dls[u] = dlt;
                         dxs[u] = dxv;
                         if constexpr (ZOH) rds[u] = __fdividef(1.0f, dlt);
@@ -407,15 +475,14 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         }
                     }
                     float sv[SV * W];
-                    float* red = sred + (q & 1) * (NT / 32) * 2 * N * W;
-                    float dbc[W];  // this lane's channel-summed dB or dC element, per step
+                    float sbv[W], scv[W];  // this lane's state: dB, dC summed over its group, per step
 #pragma unroll
                     for (int uu = W - 1; uu >= 0; --uu) {
                         const int r = q * W + uu;
                         const float dlt = dls[uu], dxv = dxs[uu];
                         const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
                         float2 cq[P2];
-                        ld_pairs<4>(cq, sCf + r * N + n0);
+                        ld_pairs<4>(cq, sCr + r * 4 * N + roff);
                         float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
                         float2 sga = make_float2(0.0f, 0.0f);
                         float2 rB[P2], rC[P2];
@@ -452,49 +519,18 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         sv[SV * uu] = sg.x + sg.y;
                         sv[SV * uu + 1] = sa.x + sa.y;
                         if constexpr (ZOH) sv[SV * uu + 2] = sga.x + sga.y;
-                        // sum over the warp's channels (lane bits above the NG state lanes):
-                        // the first three halvings scatter the 8 values (dB, dC of 4 states) so
-                        // that lane element e = (lane >> 2) & 7 remains, further ones just sum
-                        {
-                            float vv[8] = {rB[0].x, rB[0].y, rB[1].x, rB[1].y,
-                                           rC[0].x, rC[0].y, rC[1].x, rC[1].y};
-                            int c = 8;
-#pragma unroll
-                            for (int m = 16; m >= NG; m >>= 1) {
-                                if (c > 1) {
-                                    const bool up = (threadIdx.x & m) != 0;
-                                    const int h = c / 2;
-#pragma unroll
-                                    for (int i2 = 0; i2 < 4; ++i2) {
-                                        if (i2 < h) {
-                                            const float send = up ? vv[i2] : vv[i2 + h];
-                                            const float keep = up ? vv[i2 + h] : vv[i2];
-                                            vv[i2] = keep + __shfl_xor_sync(kFull, send, m);
-                                        }
-                                    }
-                                    c = h;
-                                } else {
-                                    vv[0] += __shfl_xor_sync(kFull, vv[0], m);
-                                }
-                            }
-                            dbc[uu] = vv[0];
-                        }
+                        // all-to-all over the four channel lanes of the group: round k sends
+                        // slot k, which the partner (rotation rot - k) holds for this lane's state
+                        sbv[uu] = (rB[0].x + __shfl_sync(kFull, rB[0].y, src1)) +
+                                  (__shfl_sync(kFull, rB[1].x, src2) + __shfl_sync(kFull, rB[1].y, src3));
+                        scv[uu] = (rC[0].x + __shfl_sync(kFull, rC[0].y, src1)) +
+                                  (__shfl_sync(kFull, rC[1].x, src2) + __shfl_sync(kFull, rC[1].y, src3));
                     }
-                    {
-                        const int lane = tid & 31, e = (lane >> 2) & 7;
-                        // one lane per (dB or dC, state) writes the warp's sums of the window's
-                        // steps: rows of 2N floats, a warp's lanes contiguous
-                        if ((lane & 3 & ~(NG - 1)) == 0) {
-                            float* wr = red + (tid >> 5) * W * N2 + (e >> 2) * N + ng * 4 + (e & 3);
-#pragma unroll
-                            for (int u = 0; u < W; ++u) wr[u * N2] = dbc[u];
-                        }
-                    }
-                    finish_window(q, sv, red);
+                    finish_window(q, sv, sbv, scv);
                 }
                 // state at the start of the last window of the previous sub-tile
                 if (j > 0) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase - 1) * NT * 4);
-                __syncthreads();  // stage k, sBf/sCf and sred are free again
+                __syncthreads();  // stage k, sBr/sCr and sred are free again
             }
         }
     }
@@ -502,14 +538,14 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
 #pragma unroll
     for (int m = 1; m < NG; m <<= 1) dDacc += __shfl_xor_sync(kFull, dDacc, m);
     if (dv) {
-        const size_t o = (((size_t)b * p.nseg + seg) * p.D + d) * N + n0;
-        st_pairs<4>(p.dA_part + o, dA);
+        const size_t o = (((size_t)b * p.nseg + seg) * p.D + d) * N;
+        st_slots(p.dA_part + o, dA, sidx);
         if (ng == 0) p.dD_part[((size_t)b * p.nseg + seg) * p.D + d] = dDacc;
         // sequential blocks: the adjoint leaving this block's start enters the previous block
         if (p.seq_blocks && seg > 0)
-            st_pairs<4>(p.vin + (((size_t)b * (p.nseg - 1) + (seg - 1)) * p.D + d) * N + n0, v);
+            st_slots(p.vin + (((size_t)b * (p.nseg - 1) + (seg - 1)) * p.D + d) * N, v, sidx);
         // the first segment ends at t = -1: its adjoint a_0 g_0 is the gradient of h0
-        if (p.dh0 && seg == 0) st_pairs<4>(p.dh0 + ((size_t)b * p.D + d) * N + n0, v);
+        if (p.dh0 && seg == 0) st_slots(p.dh0 + ((size_t)b * p.D + d) * N, v, sidx);
         if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
     }
 }

@@ -1,0 +1,77 @@
+"""Host model check of the lane arithmetic the real backward uses for its dB / dC channel sums.
+
+A thread of the backward holds four states of one channel.  Its state slots are rotated by its
+position `rot` among four neighbouring channel lanes (slot j holds state n0 + ((j + rot) & 3)),
+and after each step the four lanes run an all-to-all in three shuffle rounds, round k sending
+slot k to the partner whose rotation is rot - k.  This test replays those index formulas (as
+written in csrc/real_bwd.cu) for every lane of a warp and every supported state size and checks
+that each lane ends with the sum over its group's four channels of one state, that the four lanes
+of a group cover the group's four states, and that the shared-memory layout of the window sums
+is free of bank conflicts on both the writes and the reads.
+"""
+
+import numpy as np
+import pytest
+
+
+def lane_layout(N):
+    NG = N // 4
+    out = []
+    for lane in range(32):
+        ng, cl = lane % NG, lane // NG
+        rot = cl & 3
+        n0 = 4 * ng
+        srcs = [ng + NG * ((cl & ~3) | ((rot - k) & 3)) for k in (1, 2, 3)]
+        sidx = [n0 + ((j + rot) & 3) for j in range(4)]
+        out.append(dict(ng=ng, cl=cl, rot=rot, n0=n0, srcs=srcs, sidx=sidx))
+    return NG, out
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_all_to_all_sums_each_state_over_its_group(N):
+    NG, lay = lane_layout(N)
+    rng = np.random.default_rng(N)
+    val = rng.normal(size=(32 // NG, N))  # value[channel lane][state]
+    slot = np.array([[val[L["cl"], s] for s in L["sidx"]] for L in lay])
+    for lane, L in enumerate(lay):
+        got = slot[lane, 0] + sum(slot[src, k + 1] for k, src in enumerate(L["srcs"]))
+        # every source lane is in the same state group and the same four-channel group
+        for src in L["srcs"]:
+            assert lay[src]["ng"] == L["ng"] and lay[src]["cl"] // 4 == L["cl"] // 4
+        group = [(L["cl"] & ~3) + i for i in range(4)]
+        want = sum(val[c, L["n0"] + L["rot"]] for c in group)
+        assert got == pytest.approx(want, rel=1e-12, abs=1e-12)
+    # the four lanes of a group hold the group's four states, one each
+    for ng in range(NG):
+        for c0 in range(0, 32 // NG, 4):
+            states = sorted(L["n0"] + L["rot"] for L in lay if L["ng"] == ng and L["cl"] // 4 == c0 // 4)
+            assert states == list(range(4 * ng, 4 * ng + 4))
+
+
+def banks(addrs):
+    """Shared-memory wavefronts of one warp-wide 4-byte access (distinct words per bank)."""
+    per_bank = {}
+    for a in set(addrs):
+        per_bank.setdefault(a % 32, set()).add(a)
+    return max(len(v) for v in per_bank.values())
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_window_sums_layout_is_conflict_free(N):
+    NG, lay = lane_layout(N)
+    W, DT = 4, 32
+    NT = DT * NG
+    RS, GRP, N2 = 9 * N, DT // 4, 2 * N
+    assert W * N2 == NT
+    for warp in range(NT // 32):
+        for u in range(W):
+            for kind in range(2):
+                addrs = []
+                for lane, L in enumerate(lay):
+                    dl = (warp * 32 + lane) // NG
+                    grp = dl >> 2
+                    addrs.append(grp * RS + u * N2 + kind * N + L["n0"] + L["rot"])
+                assert banks(addrs) == 1
+        # the readers: thread tid sums red[g * RS + tid] over the groups
+        for g in range(GRP):
+            assert banks([g * RS + warp * 32 + lane for lane in range(32)]) == 1
