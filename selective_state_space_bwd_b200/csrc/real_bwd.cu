@@ -134,12 +134,18 @@ struct BwdCfg {
     static_assert(W * 2 * N == NT, "one (step, dB or dC, state) output of a window per thread");
 };
 
-template <typename E, int N>
+// A2A selects the channel sums of dB / dC: the four-lane all-to-all over rotated slots (fewer
+// instructions; B and C are staged in their four rotations and the CTA adds eight group partials
+// per output) or a shuffle reduce-scatter over the warp's eight channels with natural slot order
+// (plain B / C tiles, four warp partials per output), which needs fewer registers and less shared
+// memory and is used by the instance compiled for four CTAs per SM.
+template <typename E, int N, bool A2A>
 struct BwdSmem {
     using Cfg = BwdCfg<N>;
     static constexpr int TT = Cfg::TT, DT = Cfg::DT;
     static constexpr int XE = TT * DT, BE = TT * N;
-    static constexpr int RE = TT * 4 * N;  // fp32 tile of B or C with the four slot rotations
+    static constexpr int ROT = A2A ? 4 : 1;  // slot rotations staged per B / C row
+    static constexpr int RE = TT * ROT * N;  // fp32 tile of B or C
     // pass A stage: x, delta_raw, B (raw)
     static constexpr int A_STAGE = (2 * XE + BE) * (int)sizeof(E);
     static constexpr int A_DD = 2 * A_STAGE;              // (delta, delta*x) float2 [TT][DT]
@@ -149,8 +155,9 @@ struct BwdSmem {
     static constexpr int B_STAGE = XE * 8 + (2 * XE + 2 * BE) * (int)sizeof(E);
     static constexpr int B_BR = 2 * B_STAGE;              // B rotated fp32
     static constexpr int B_CR = B_BR + RE * 4;            // C rotated fp32
-    static constexpr int B_RED = B_CR + RE * 4;           // window sums, 2 x [GRP][RS] floats
-    static constexpr int B_END = B_RED + 2 * Cfg::GRP * Cfg::RS * 4;
+    static constexpr int B_RED = B_CR + RE * 4;           // window sums, double-buffered
+    static constexpr int RED = A2A ? Cfg::GRP * Cfg::RS : (Cfg::NT / 32) * 2 * N * Cfg::W;
+    static constexpr int B_END = B_RED + 2 * RED * 4;
     static constexpr int BYTES = A_END > B_END ? A_END : B_END;
     static_assert(A_STAGE % 16 == 0 && B_STAGE % 16 == 0, "16-byte aligned stages");
 };
@@ -158,7 +165,7 @@ struct BwdSmem {
 // Rows [0, rows) of a staged [rows][N] tile to fp32 with the four slot rotations of every group of
 // four states: dst[(row * 4 + k) * N + 4 g + j] = src[row * N + 4 g + ((j + k) & 3)], so a thread
 // of rotation k reads its four slots with one 16-byte load.
-template <typename E, int N>
+template <typename E, int N, int ROT>
 __device__ __forceinline__ void rotate_rows(float* __restrict__ dst, const E* __restrict__ src,
                                             int rows, int tid, int nthreads) {
     constexpr int G = N / 4;
@@ -178,9 +185,9 @@ __device__ __forceinline__ void rotate_rows(float* __restrict__ dst, const E* __
             v[2] = w.z;
             v[3] = w.w;
         }
-        float* o = dst + row * 4 * N + 4 * g;
+        float* o = dst + row * ROT * N + 4 * g;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < ROT; ++k)
             *reinterpret_cast<float4*>(o + k * N) =
                 make_float4(v[k & 3], v[(k + 1) & 3], v[(k + 2) & 3], v[(k + 3) & 3]);
     }
@@ -201,10 +208,11 @@ __device__ __forceinline__ void st_slots(float* row, const float2 (&o)[2], const
 // MINB: CTAs per SM the register allocation must allow.  4 (126 registers for the Euler N = 16
 // kernel) lets grids of up to 592 CTAs run in one wave; 3 leaves the compiler more registers,
 // which is faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
-template <typename E, int N, bool ZOH, int MINB>
+template <typename E, int N, bool ZOH, int MINB, bool A2A>
 __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
-    using Sm = BwdSmem<E, N>;
+    using Sm = BwdSmem<E, N, A2A>;
+    constexpr int ROT = Sm::ROT;
     constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, W = Cfg::W;
     constexpr int GRP = Cfg::GRP, RS = Cfg::RS;
     // per-step channel sums over the states: sum g w' B (dx), sum A q, and for zero-order hold
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * Cfg::S;
     const bool dv = d < p.D;
     // slot rotation and the all-to-all partners among the four channel lanes of this group
-    const int cl = (tid & 31) / NG, rot = cl & 3, grp = dl >> 2;
+    const int cl = (tid & 31) / NG, rot = A2A ? cl & 3 : 0, grp = dl >> 2;
     const int src1 = ng + NG * ((cl & ~3) | ((rot - 1) & 3));
     const int src2 = ng + NG * ((cl & ~3) | ((rot - 2) & 3));
     const int src3 = ng + NG * ((cl & ~3) | ((rot - 3) & 3));
@@ -270,7 +278,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     float* scr = p.bnd_scratch + cta * real_bwd_scratch_floats(N, T);
     float* bnd = scr + (size_t)tid * 4;                        // window starts: [T/W][NT][4]
     float2* dsg = reinterpret_cast<float2*>(scr + (size_t)(T / W) * NT * 4);  // (delta, sigma) [T][DT]
-    const int roff = rot * N + n0;  // this thread's slots within a rotated row of 4N floats
+    const int roff = rot * N + n0;  // this thread's slots within a staged row of ROT * N floats
 
     for (int c = c_end - 1; c >= c_begin; --c) {
         const int tc = c * T;
@@ -303,13 +311,9 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
             issue(0, 0);
             for (int j = 0; j < nsub; ++j) {
                 const int k = j & 1;
-                if (j + 1 < nsub) {
-                    issue(j + 1, k ^ 1);
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
-                }
-                __syncthreads();
+                cp_async_wait<0>();
+                __syncthreads();  // sub-tile j is in; every thread is past sub-tile j-1
+                if (j + 1 < nsub) issue(j + 1, k ^ 1);
                 const int t0 = tc + j * TTe;
                 const int rows = min(TTe, p.L - t0);
                 const E* sx = stage(k);
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                     sdd[i] = make_float2(dlt, dlt * Elem<E>::to_f(sx[i]));
                     __stcg(&dsg[(size_t)(j * TTe) * DT + i], make_float2(dlt, sig));
                 }
-                rotate_rows<E, N>(sBr, sB, TTe, tid, NT);
+                rotate_rows<E, N, ROT>(sBr, sB, TTe, tid, NT);
                 __syncthreads();
                 for (int w = 0; w < TTe / W; ++w) {
                     __stcg(reinterpret_cast<float4*>(bnd + (size_t)((j * TTe) / W + w) * NT * 4),
@@ -336,7 +340,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         const int r = w * W + u;
                         const float2 dd = sdd[r * DT + dl];
                         float2 bq[P2];
-                        ld_pairs<4>(bq, sBr + r * 4 * N + roff);
+                        ld_pairs<4>(bq, sBr + r * ROT * N + roff);
 #pragma unroll
                         for (int i = 0; i < P2; ++i) {
                             const float2 zl2 = __fmul2_rn(f2(dd.x), A2[i]);
@@ -349,7 +353,6 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         }
                     }
                 }
-                __syncthreads();  // stage k and sdd are free again
             }
         }
 
@@ -382,13 +385,9 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
             ld_pairs_cg<4>(hw, bnd + (size_t)((nsub - 1) * TTe / W + TTe / W - 1) * NT * 4);
             for (int j = nsub - 1; j >= 0; --j) {
                 const int k = j & 1;
-                if (j > 0) {
-                    issue(j - 1, k ^ 1);
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
-                }
-                __syncthreads();
+                cp_async_wait<0>();
+                __syncthreads();  // sub-tile j is in; every thread is past sub-tile j+1
+                if (j > 0) issue(j - 1, k ^ 1);
                 const int t0 = tc + j * TTe;
                 const int rows = min(TTe, p.L - t0);
                 const float2* sds = reinterpret_cast<const float2*>(stage(k));
@@ -396,8 +395,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                 const E* sdy = sx + Sm::XE;
                 const E* sB = sx + 2 * Sm::XE;
                 const E* sC = sB + Sm::BE;
-                rotate_rows<E, N>(sBr, sB, TTe, tid, NT);
-                rotate_rows<E, N>(sCr, sC, TTe, tid, NT);
+                rotate_rows<E, N, ROT>(sBr, sB, TTe, tid, NT);
+                rotate_rows<E, N, ROT>(sCr, sC, TTe, tid, NT);
                 __syncthreads();
                 const int nw = TTe / W;  // 4 or 8 windows, even
                 const int wbase = (j * TTe) / W;
@@ -406,11 +405,22 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                 // after a window's reverse sweep: outputs, then its dB/dC sums over the CTA
                 auto finish_window = [&](int q, float (&sv)[SV * W], const float (&sbv)[W],
                                          const float (&scv)[W]) {
-                    float* red = sred + (q & 1) * GRP * RS;
+                    float* red = sred + (q & 1) * Sm::RED;
+                    if constexpr (A2A) {
 #pragma unroll
-                    for (int u = 0; u < W; ++u) {
-                        red[grp * RS + u * N2 + n0 + rot] = sbv[u];
-                        red[grp * RS + u * N2 + N + n0 + rot] = scv[u];
+                        for (int u = 0; u < W; ++u) {
+                            red[grp * RS + u * N2 + n0 + rot] = sbv[u];
+                            red[grp * RS + u * N2 + N + n0 + rot] = scv[u];
+                        }
+                    } else {
+                        // one lane per (dB or dC, state) writes the warp's sums of the window's
+                        // steps: rows of 2N floats, a warp's lanes contiguous
+                        const int lane = tid & 31, e = (lane >> 2) & 7;
+                        if ((lane & 3 & ~(NG - 1)) == 0) {
+                            float* wr = red + (tid >> 5) * W * N2 + (e >> 2) * N + ng * 4 + (e & 3);
+#pragma unroll
+                            for (int u = 0; u < W; ++u) wr[u * N2] = sbv[u];
+                        }
                     }
                     reduce_scatter<SV * W, NG>(sv, ng);
 #pragma unroll
@@ -431,10 +441,16 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                     }
                     __syncthreads();  // every group's sums of the window are in `red`
                     {
-                        // output (step u, dB or dC, state) = sum over the CTA's groups
+                        // output (step u, dB or dC, state) = sum over the CTA's groups or warps
                         float s = 0.0f;
+                        if constexpr (A2A) {
 #pragma unroll
-                        for (int g = 0; g < GRP; ++g) s += red[g * RS + tid];
+                            for (int g = 0; g < GRP; ++g) s += red[g * RS + tid];
+                        } else {
+                            const int u = tid / N2, e2 = tid % N2;
+#pragma unroll
+                            for (int w = 0; w < NT / 32; ++w) s += red[(w * W + u) * N2 + e2];
+                        }
                         const int r = q * W + tid / N2;
                         if (r < rows) partb[(size_t)(t0 + r) * N2 + (tid % N2)] = s;
                     }
@@ -453,7 +469,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         const int r = q * W + u;
                         const float dlt = sds[r * DT + dl].x;
                         const float dxv = dlt * Elem<E>::to_f(sx[r * DT + dl]);
-                        ld_pairs<4>(bqs[u], sBr + r * 4 * N + roff);
+                        ld_pairs<4>(bqs[u], sBr + r * ROT * N + roff);
                         dls[u] = dlt;
                         dxs[u] = dxv;
                         if constexpr (ZOH) rds[u] = __fdividef(1.0f, dlt);
@@ -482,7 +498,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         const float dlt = dls[uu], dxv = dxs[uu];
                         const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
                         float2 cq[P2];
-                        ld_pairs<4>(cq, sCr + r * 4 * N + roff);
+                        ld_pairs<4>(cq, sCr + r * ROT * N + roff);
                         float2 sg = make_float2(0.0f, 0.0f), sa = make_float2(0.0f, 0.0f);
                         float2 sga = make_float2(0.0f, 0.0f);
                         float2 rB[P2], rC[P2];
@@ -519,18 +535,47 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         sv[SV * uu] = sg.x + sg.y;
                         sv[SV * uu + 1] = sa.x + sa.y;
                         if constexpr (ZOH) sv[SV * uu + 2] = sga.x + sga.y;
-                        // all-to-all over the four channel lanes of the group: round k sends
-                        // slot k, which the partner (rotation rot - k) holds for this lane's state
-                        sbv[uu] = (rB[0].x + __shfl_sync(kFull, rB[0].y, src1)) +
-                                  (__shfl_sync(kFull, rB[1].x, src2) + __shfl_sync(kFull, rB[1].y, src3));
-                        scv[uu] = (rC[0].x + __shfl_sync(kFull, rC[0].y, src1)) +
-                                  (__shfl_sync(kFull, rC[1].x, src2) + __shfl_sync(kFull, rC[1].y, src3));
+                        if constexpr (A2A) {
+                            // all-to-all over the four channel lanes of the group: round k sends
+                            // slot k, which the partner (rotation rot - k) holds for this lane's
+                            // state
+                            sbv[uu] = (rB[0].x + __shfl_sync(kFull, rB[0].y, src1)) +
+                                      (__shfl_sync(kFull, rB[1].x, src2) + __shfl_sync(kFull, rB[1].y, src3));
+                            scv[uu] = (rC[0].x + __shfl_sync(kFull, rC[0].y, src1)) +
+                                      (__shfl_sync(kFull, rC[1].x, src2) + __shfl_sync(kFull, rC[1].y, src3));
+                        } else {
+                            // sum over the warp's channels (lane bits above the NG state lanes):
+                            // the first three halvings scatter the 8 values (dB, dC of 4 states)
+                            // so that lane element e = (lane >> 2) & 7 remains, further ones sum
+                            float vv[8] = {rB[0].x, rB[0].y, rB[1].x, rB[1].y,
+                                           rC[0].x, rC[0].y, rC[1].x, rC[1].y};
+                            int c = 8;
+#pragma unroll
+                            for (int m = 16; m >= NG; m >>= 1) {
+                                if (c > 1) {
+                                    const bool up = (threadIdx.x & m) != 0;
+                                    const int h = c / 2;
+#pragma unroll
+                                    for (int i2 = 0; i2 < 4; ++i2) {
+                                        if (i2 < h) {
+                                            const float send = up ? vv[i2] : vv[i2 + h];
+                                            const float keep = up ? vv[i2 + h] : vv[i2];
+                                            vv[i2] = keep + __shfl_xor_sync(kFull, send, m);
+                                        }
+                                    }
+                                    c = h;
+                                } else {
+                                    vv[0] += __shfl_xor_sync(kFull, vv[0], m);
+                                }
+                            }
+                            sbv[uu] = vv[0];
+                            scv[uu] = 0.0f;
+                        }
                     }
                     finish_window(q, sv, sbv, scv);
                 }
                 // state at the start of the last window of the previous sub-tile
                 if (j > 0) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase - 1) * NT * 4);
-                __syncthreads();  // stage k, sBr/sCr and sred are free again
             }
         }
     }
@@ -619,10 +664,12 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
                                                                             a.gsumP, a.vin, a.dhL);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t sm = BwdSmem<E, N>::BYTES;
-    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3>, sm)) != cudaSuccess) return e;
+    // at most three CTAs per SM: the all-to-all instance; four: the reduce-scatter instance, whose
+    // registers and shared memory fit four
+    const size_t sm3 = BwdSmem<E, N, true>::BYTES, sm4 = BwdSmem<E, N, false>::BYTES;
+    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true>, sm3)) != cudaSuccess) return e;
     if constexpr (N == 16 && !ZOH)
-        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4>, sm)) != cudaSuccess) return e;
+        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false>, sm4)) != cudaSuccess) return e;
     const int per = a.seq_blocks ? 1 : group;
     for (int hi = a.nseg; hi > 0; hi -= per) {
         const int lo = hi - per > 0 ? hi - per : 0;
@@ -635,9 +682,9 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         if constexpr (N == 16 && !ZOH) wide = (int64_t)a.ndt * a.B * (hi - lo) > 444;
         if (wide) {
             if constexpr (N == 16 && !ZOH)
-                real_bwd_kernel<E, N, ZOH, 4><<<grid, dim3(BwdCfg<N>::NT), sm, st>>>(a);
+                real_bwd_kernel<E, N, ZOH, 4, false><<<grid, dim3(BwdCfg<N>::NT), sm4, st>>>(a);
         } else {
-            real_bwd_kernel<E, N, ZOH, 3><<<grid, dim3(BwdCfg<N>::NT), sm, st>>>(a);
+            real_bwd_kernel<E, N, ZOH, 3, true><<<grid, dim3(BwdCfg<N>::NT), sm3, st>>>(a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t nbc = (int64_t)a.B * rows * 2 * N;
