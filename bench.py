@@ -193,12 +193,12 @@ E2E_OVERLAP = ("two buffer sets; each step's host-to-device and device-to-host c
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled through NVML every 2 ms while the timed region runs
+    """SM clock and throttle reasons sampled through NVML every 1 ms while the timed region runs
     (a background thread), so even a timed region of a few tens of milliseconds gets tens of
     samples.  The GPU is found by its PCI bus id (falling back to the device index).  The raw
     samples go to clocks_rank<i>.csv in $SSM_BENCH_CLOCKS_DIR (default: the system temp dir)."""
 
-    PERIOD_S = 0.002
+    PERIOD_S = 0.001
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
@@ -267,7 +267,7 @@ class ClockSampler:
             reasons.update(n for n, a in zip(self.NAMES, act) if a)
         sm = [s[1] for s in self.samples]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
-                "reasons": sorted(reasons), "samples": len(sm), "sampler": "NVML, 2 ms period",
+                "reasons": sorted(reasons), "samples": len(sm), "sampler": "NVML, 1 ms period",
                 "power_w_max": max((s[2] for s in self.samples), default=None)}
 
 
@@ -293,8 +293,8 @@ def oracle_sample(w, inp, budget_s=(10.0, 30.0), zoh=False):
             break
     upd = rows * w.seqlen * w.dim * w.dstate
     return {"value": upd / t_total, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{rows} batch row(s) of {w.name} (L={w.seqlen}, D={w.dim}, N={w.dstate}), "
-                      f"fwd+bwd in float64, {t_total:.1f} s"}
+            "sample": f"{rows} batch-row runs, cycling over the {w.batch} rows of {w.name} "
+                      f"(L={w.seqlen}, D={w.dim}, N={w.dstate}), fwd+bwd in float64, {t_total:.1f} s"}
 
 
 def code_digest(path):
@@ -369,6 +369,40 @@ def memory_curve():
                       "curve": rows}), flush=True)
 
 
+L2_NOTE = "flushed (256 MiB write) before every timed step"
+
+
+def real_config(args, w, world):
+    """The workload a real-mode line measures (both arms print the same dict)."""
+    c = {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+         "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
+         "discretization": "zoh" if args.zoh else "euler",
+         "initial_state": bool(args.state), "state": "fp32", "l2": L2_NOTE,
+         "parallelism": f"dp{world} (weak: one full batch per rank; dA_log/dD all-reduced)"
+                        if world > 1 else "single GPU"}
+    if args.dtproj:
+        c["dt_rank"] = args.dtproj
+    return c
+
+
+def complex_config(args, w, world):
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+            "modes": w.modes, "chunk": w.chunk, "io": "complex64",
+            "training": "rtrl (online, forward only)" if args.rtrl else "bptt (fwd + bwd)",
+            "backward": ("from chunk checkpoints (ssm_scan_complex_bwd)" if args.ckpt
+                         else "from the stored trajectory (ssm_scan_complex_bwd_traj)"),
+            "l2": L2_NOTE,
+            "parallelism": f"dp{world} (weak: one full batch per rank; dlambda/domega all-reduced)"
+                           if world > 1 else "single GPU"}
+
+
+def pdssm_config(args, w, world):
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "heads": w.heads,
+            "nstate": w.nstate, "ndict": w.ndict, "tau": 1.0, "l2": L2_NOTE,
+            "parallelism": f"dp{world} (weak: one full batch per rank, no exchange)"
+                           if world > 1 else "single GPU"}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -394,7 +428,7 @@ def run_reference(args, w):
                             threads=threads)
         else:
             oracle.real(inp["x"], inp["delta_raw"], inp["A_log"], inp["Bm"], inp["Cm"],
-                        inp["Dskip"], inp["dy"], chunk=w.chunk, threads=threads)
+                        inp["Dskip"], inp["dy"], chunk=w.chunk, threads=threads, zoh=args.zoh)
         dt = time.perf_counter() - t0
         if k >= args.warmup:
             times.append(dt)
@@ -404,13 +438,10 @@ def run_reference(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
-            "config": ({"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
-                        "modes": w.modes, "chunk": w.chunk, "io": "complex64"} if cplx else
-                       {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
-                        "dstate": w.dstate, "chunk": w.chunk, "io": w.io})
-                      | {"sample": "one batch row per step", "l2": "n/a (CPU)"},
+            "config": (complex_config if cplx else real_config)(args, w, args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"1 of {w.batch} batch rows of {w.name} per step, float64"},
+                             "sample": f"1 of {w.batch} batch rows of {w.name} per step (fwd + "
+                                       f"bwd in float64 on the host cores; no L2 flush)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -581,14 +612,7 @@ def main_complex(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "c64",
             "data": "synthetic (seeded generator, workload value distributions)",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
-                       "modes": w.modes, "chunk": w.chunk, "io": "complex64",
-                       "training": "rtrl (online, forward only)" if args.rtrl else "bptt (fwd + bwd)",
-                       "backward": ("from chunk checkpoints (ssm_scan_complex_bwd)" if args.ckpt
-                                    else "from the stored trajectory (ssm_scan_complex_bwd_traj)"),
-                       "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"dp{world} (weak: one full batch per rank; "
-                                      "dlambda/domega all-reduced)" if world > 1 else "single GPU"},
+            "config": complex_config(args, w, world),
             "roofline": ({"bound": "hbm", "kernel": "ssm_scan_complex_rtrl call (cplx_rtrl_kernel "
                           "+ reduction over the batch)", "achieved": fwd_gbs, "peak": hbm,
                           "unit": "GB/s", "frac": fwd_gbs / hbm, "peak_kind": peak_kind,
@@ -743,11 +767,7 @@ def main_pdssm(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded generator: random dictionary maps, N(0,1) scores)",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "heads": w.heads,
-                       "nstate": w.nstate, "ndict": w.ndict, "tau": 1.0,
-                       "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"dp{world} (weak: one full batch per rank, no exchange)"
-                                      if world > 1 else "single GPU"},
+            "config": pdssm_config(args, w, world),
             "roofline": {"bound": "hbm", "kernel": "ssm_pdssm_bwd call (reverse scan + score "
                          "gradient)", "achieved": bwd_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": bwd_gbs / hbm, "peak_kind": peak_kind,
@@ -789,11 +809,10 @@ def run_reference_pdssm(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "heads": w.heads,
-                       "nstate": w.nstate, "ndict": w.ndict, "sample": "one batch row per step",
-                       "l2": "n/a (CPU)"},
+            "config": pdssm_config(args, w, args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"1 of {w.batch} batch rows of {w.name} per step, float64"},
+                             "sample": f"1 of {w.batch} batch rows of {w.name} per step (fwd + "
+                                       f"bwd in float64 on the host cores; no L2 flush)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -1006,13 +1025,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.io == gen.BF16 else "f32",
             "data": "synthetic (seeded generator, workload value distributions)",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
-                       "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
-                       "discretization": "zoh" if args.zoh else "euler",
-                       "initial_state": bool(args.state),
-                       "state": "fp32", "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"dp{world} (weak: one full batch per rank; "
-                                      "dA_log/dD all-reduced)" if world > 1 else "single GPU"},
+            "config": real_config(args, w, world),
             "roofline": {"bound": "alu", "kernel": "ssm_scan_bwd call (real_bwd_kernel + "
                          "dB/dC and parameter reductions)", "achieved": bwd_tops, "peak": alu_peak,
                          "unit": "Top/s", "frac": bwd_tops / alu_peak,
@@ -1035,7 +1048,6 @@ def main():
             "clocks": clk,
         }
         if R:
-            line["config"]["dt_rank"] = R
             pfb, pbb, pfl = dtproj_algorithmic(w, R)
             line["dtproj"] = {
                 "rank": R, "ms_fwd": 1e3 * t_pf / args.steps, "ms_bwd": 1e3 * t_pb / args.steps,
