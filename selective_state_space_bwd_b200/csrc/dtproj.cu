@@ -192,27 +192,28 @@ __device__ __forceinline__ void tmem_dealloc_cta(unsigned taddr, unsigned cols) 
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(cols) : "memory");
 }
 
-// C tile [128 x BN] of blockIdx (y: m, x: n, z: k split), the k range in 64-deep stages.
-// mA, mB: tensor maps of A and B with 64-element-wide boxes (k-major: {64 k, rows}; m/n-major:
-// {64 m/n, 64 k}).  ONES: one more 64-wide accumulator block multiplies A by a static block whose
-// first column is all ones, giving A's column sums (dbias) in accumulator column BN.
+// C tile [128 x BN] at tile coordinates (bn: n, bm: m, bz: k split), the k range in 64-deep
+// stages.  mA, mB: tensor maps of A and B with 64-element-wide boxes (k-major: {64 k, rows};
+// m/n-major: {64 m/n, 64 k}); they are kernel parameters (__grid_constant__), passed on by
+// reference so the copies read them in parameter space.  ONES: one more 64-wide accumulator block
+// multiplies A by a static block whose first column is all ones, giving A's column sums (dbias) in
+// accumulator column BN.  The dynamic shared memory holds at least TcSmem<BN, STAGES, ONES>::BYTES.
 template <bool A_MN, bool B_MN, int BN, int STAGES, bool ONES, int EPI>
-__global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUtensorMap mA,
-                                                     const __grid_constant__ CUtensorMap mB, TcArgs p) {
+__device__ __forceinline__ void tc_tile(const CUtensorMap& mA, const CUtensorMap& mB, const TcArgs& p,
+                                        int bn, int bm, int bz, unsigned char* smem_raw) {
     static_assert(BN % 64 == 0 && BN <= 256 && STAGES >= 3, "n tile of whole 64-wide blocks");
     static_assert(!ONES || EPI == EPI_F32_PART, "column sums go to the fp32 partial sums");
     using Sm = TcSmem<BN, STAGES, ONES>;
     constexpr int TCOLS = tmem_cols(BN + (ONES ? 64 : 0));
     constexpr int PF = STAGES - 2;  // stages loading ahead of the one being multiplied
-    extern __shared__ unsigned char smem_raw[];
     const unsigned raw = smem_u32(smem_raw);
     const unsigned base = (raw + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
     unsigned char* gbase = smem_raw + (base - raw);
     const unsigned full = base + Sm::FULL, free_ = base + Sm::FREE, done = base + Sm::DONE;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t m0 = (int64_t)blockIdx.y * TM, n0 = (int64_t)blockIdx.x * BN;
-    const int64_t kb = (int64_t)blockIdx.z * p.kchunk;
+    const int64_t m0 = (int64_t)bm * TM, n0 = (int64_t)bn * BN;
+    const int64_t kb = (int64_t)bz * p.kchunk;
     const int64_t ke = min(p.K, kb + p.kchunk);
     const int nk = ke > kb ? (int)((ke - kb + BK - 1) / BK) : 0;
 
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUt
         if (EPI == EPI_F32_PART) {
             // partial sums [split][N][M]: one column per store, the warp's 32 rows contiguous; tile
             // columns below ones_out are data columns, accumulator column BN the column sums
-            float* out = static_cast<float*>(p.C) + (int64_t)blockIdx.z * p.N * p.M;
+            float* out = static_cast<float*>(p.C) + (int64_t)bz * p.N * p.M;
             const int64_t m = m0 + row;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN + (ONES ? 32 : 0); c0 += 32) {
@@ -365,6 +366,34 @@ __global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUt
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc_cta(tmem, TCOLS);
+    }
+}
+
+// One GEMM: tile (blockIdx.x: n, blockIdx.y: m, blockIdx.z: k split)
+template <bool A_MN, bool B_MN, int BN, int STAGES, bool ONES, int EPI>
+__global__ void __launch_bounds__(NTH) dtp_tc_kernel(const __grid_constant__ CUtensorMap mA,
+                                                     const __grid_constant__ CUtensorMap mB, TcArgs p) {
+    extern __shared__ unsigned char smem_raw[];
+    tc_tile<A_MN, B_MN, BN, STAGES, ONES, EPI>(mA, mB, p, blockIdx.x, blockIdx.y, blockIdx.z, smem_raw);
+}
+
+// The projection's two backward GEMMs in one launch, so that both stream g at once: CTAs
+// [0, n_du) compute du (one 128-row tile of g each, the whole k = D range), the others one
+// (d tile, row split) of the dw / dbias partial sums.  For R <= 64.
+constexpr int BWD_DU_STAGES = 4, BWD_DW_STAGES = 4;
+__global__ void __launch_bounds__(NTH) dtp_bwd_kernel(const __grid_constant__ CUtensorMap gK,
+                                                      const __grid_constant__ CUtensorMap wN,
+                                                      const __grid_constant__ CUtensorMap gM,
+                                                      const __grid_constant__ CUtensorMap uN, TcArgs du,
+                                                      TcArgs dw, int n_du, int dw_mt) {
+    extern __shared__ unsigned char smem_raw[];
+    const int c = blockIdx.x;
+    if (c < n_du) {
+        tc_tile<false, true, 64, BWD_DU_STAGES, false, EPI_BF16>(gK, wN, du, 0, c, 0, smem_raw);
+    } else {
+        const int j = c - n_du;
+        tc_tile<true, true, 64, BWD_DW_STAGES, true, EPI_F32_PART>(gM, uN, dw, 0, j % dw_mt, j / dw_mt,
+                                                                   smem_raw);
     }
 }
 
@@ -541,17 +570,15 @@ __global__ void dtp_reduce_kernel(const float* __restrict__ part, int splits, in
     if (i >= n) return;
     const int r = (int)(i / D);
     const int64_t d = i - (int64_t)r * D;
-    // four interleaved running sums (independent loads in flight), combined in a fixed order
-    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-    int k = 0;
-    for (; k + 4 <= splits; k += 4) {
-        s0 += part[(int64_t)k * n + i];
-        s1 += part[(int64_t)(k + 1) * n + i];
-        s2 += part[(int64_t)(k + 2) * n + i];
-        s3 += part[(int64_t)(k + 3) * n + i];
+    // splits in groups of 16 loads issued before any is used, summed in split order
+    float s = 0.0f;
+    for (int k0 = 0; k0 < splits; k0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = k0 + k < splits ? __ldcs(part + (int64_t)(k0 + k) * n + i) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) s += v[k];
     }
-    for (; k < splits; ++k) s0 += part[(int64_t)k * n + i];
-    const float s = (s0 + s1) + (s2 + s3);
     if (r < R)
         dw[d * R + r] = s;
     else if (dbias)
@@ -631,12 +658,17 @@ cudaError_t run_fwd(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensor
 }  // namespace
 
 // Rows of one dw / dbias split (a multiple of the 64-row stage)
-int64_t dtproj_rows_per_split(int) { return 1024; }
+// Rows of one dw / dbias split (a multiple of the 64-row stage).  R <= 64 runs du and dw in one
+// launch: 1536-row splits give a dw CTA about the bytes of g of a du CTA, and both kinds fit one
+// wave at two CTAs per SM for the workloads' row counts.
+int64_t dtproj_rows_per_split(int R) { return R <= 64 ? 1536 : 1024; }
 
 cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     // delta_raw [M x D] = u [M x R] . w [D x R]^T + bias: both operands k-major
     const int ka = (d.R + 63) / 64;              // 64-deep k atoms covering R, all in one stage
-    const int bn = ka <= 2 ? 128 : 64;
+    // n tile: 64 for one k atom (three CTAs per SM instead of two), 128 for two (a wider tile
+    // amortises the second atom's copies), 64 beyond
+    const int bn = ka == 2 ? 128 : 64;
     CUtensorMap mA, mB, mC;
     cudaError_t e = make_map(&mA, d.u, d.M, d.R, d.R, TM);
     if (e == cudaSuccess) e = make_map(&mB, d.w, d.D, d.R, d.R, bn);
@@ -649,7 +681,7 @@ cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     a.bias = d.bias;
     a.status = d.status;
     switch (ka) {
-        case 1: return run_fwd<1, 128>(mA, mB, mC, a, st);
+        case 1: return run_fwd<1, 64>(mA, mB, mC, a, st);
         case 2: return run_fwd<2, 128>(mA, mB, mC, a, st);
         case 3: return run_fwd<3, 64>(mA, mB, mC, a, st);
         default: return run_fwd<4, 64>(mA, mB, mC, a, st);
@@ -672,13 +704,6 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     a.ones_out = d.R;
     a.C = d.du;
     a.status = d.status;
-    switch ((d.R + 63) / 64) {  // 64-wide n blocks covering R
-        case 1: e = run_tc<false, true, 64, 8, false, EPI_BF16>(gK, wN, a, 1, st); break;
-        case 2: e = run_tc<false, true, 128, 6, false, EPI_BF16>(gK, wN, a, 1, st); break;
-        case 3: e = run_tc<false, true, 192, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
-        default: e = run_tc<false, true, 256, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
-    }
-    if (e != cudaSuccess) return e;
     // dw partials [split][R+1][D]: data columns 0..R-1, then the column sums of g (dbias) from the
     // static block of ones
     TcArgs b = {};
@@ -686,14 +711,37 @@ cudaError_t launch_dtproj_bwd(const DtArgs& d, cudaStream_t st) {
     b.ones_out = d.R;
     b.C = d.part;
     b.status = d.status;
+    const int64_t n = d.D * (d.R + 1);
+    if (d.R <= 64) {
+        // du and dw side by side in one launch
+        constexpr int b_du = TcSmem<64, BWD_DU_STAGES, false>::BYTES;
+        constexpr int b_dw = TcSmem<64, BWD_DW_STAGES, true>::BYTES;
+        constexpr int bytes = b_du > b_dw ? b_du : b_dw;
+        if ((e = cudaFuncSetAttribute(dtp_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) !=
+            cudaSuccess)
+            return e;
+        const int n_du = (int)((d.M + TM - 1) / TM);
+        const int dw_mt = (int)((d.D + TM - 1) / TM);
+        const int64_t ctas = (int64_t)n_du + (int64_t)dw_mt * d.splits;
+        if (ctas > 0x7fffffff) return cudaErrorInvalidConfiguration;
+        dtp_bwd_kernel<<<(unsigned)ctas, NTH, bytes, st>>>(gK, wN, gM, uN, a, b, n_du, dw_mt);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        dtp_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(d.part, d.splits, d.D, d.R, d.dw,
+                                                                        d.dbias);
+        return cudaGetLastError();
+    }
+    switch ((d.R + 63) / 64) {  // 64-wide n blocks covering R
+        case 2: e = run_tc<false, true, 128, 6, false, EPI_BF16>(gK, wN, a, 1, st); break;
+        case 3: e = run_tc<false, true, 192, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
+        default: e = run_tc<false, true, 256, 4, false, EPI_BF16>(gK, wN, a, 1, st); break;
+    }
+    if (e != cudaSuccess) return e;
     switch ((d.R + 63) / 64) {
-        case 1: e = run_tc<true, true, 64, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
         case 2: e = run_tc<true, true, 128, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
         case 3: e = run_tc<true, true, 192, 4, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
         default: e = run_tc<true, true, 256, 3, true, EPI_F32_PART>(gM, uN, b, d.splits, st); break;
     }
     if (e != cudaSuccess) return e;
-    const int64_t n = d.D * (d.R + 1);
     dtp_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(d.part, d.splits, d.D, d.R, d.dw,
                                                                     d.dbias);
     return cudaGetLastError();
