@@ -9,14 +9,17 @@
 namespace {
 
 constexpr size_t kStatusBytes = 256;
+// The real backward keeps its scratch-slot mask in the status block, after the status word:
+// (kStatusBytes - kSlotMaskOffset) * 8 = 1984 slots at most.
+constexpr size_t kSlotMaskOffset = 32;
 constexpr int kTargetCtas = 296;  // 2 x 148 SMs: below this many CTAs, split time into segments
 // Real forward, once split: enough segments for about 2368 CTAs (two waves at the eight CTAs per
 // SM its registers and shared memory allow), so that every SM keeps several CTAs busy.
 constexpr int64_t kRealFwdSplitCtas = 2368;
-// Real backward: 4 CTAs per SM (126 registers per thread, 37 KB of shared memory) on 148 SMs
+// Real backward: 4 CTAs per SM (126 registers per thread, 48 KB of shared memory) on 148 SMs.
+// Also the number of scratch slots (window-start states, (delta, sigma)) of a launch with more
+// CTAs: a CTA holds one from its start to its end.
 constexpr int64_t kRealBwdSlots = 592;
-// Real backward: per-launch bound on the per-CTA scratch (window-start states, (delta, sigma))
-constexpr size_t kRealBwdScratchCap = (size_t)192 << 20;
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -52,6 +55,7 @@ struct RealPlan {
     // workspace offsets (bytes); fwd and bwd use separate layouts
     size_t f_sumP, f_sumS, f_hin, f_end;
     size_t b_gP, b_gG, b_part, b_dA, b_dD, b_bnd, b_end;
+    int b_nslot;  // backward scratch slots: CTAs per launch, at most the resident CTAs
 };
 
 int plan_real(const ssm_shape* s, RealPlan* p) {
@@ -87,19 +91,17 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     p->f_end = o;
 
     // Backward.  The per-CTA dB/dC partial sums cover the steps of one launch; time is walked
-    // in launches whose partial buffer fits max(checkpoint bytes, 128 MiB), so the backward's
-    // memory stays O(L / T) however long the sequence.
+    // in launches whose partial buffer fits max(half the checkpoint bytes, 128 MiB), so the
+    // backward's memory stays O(L / T) however long the sequence.
     const size_t per_chunk = (size_t)p->ndt * B * p->T * 2 * p->N * 4;
     const size_t ckpt = B * (size_t)p->nC * DN * 4;
-    const size_t cap = ckpt > ((size_t)128 << 20) ? ckpt : ((size_t)128 << 20);
+    const size_t cap = ckpt / 2 > ((size_t)128 << 20) ? ckpt / 2 : ((size_t)128 << 20);
     const int64_t ctas_per_seg = (int64_t)B * p->ndt;
     const size_t chunks_cap = per_chunk > 0 ? cap / per_chunk : (size_t)p->nC;  // per launch
     const int nC1 = p->nC > 0 ? p->nC : 1;
     auto clampi = [](size_t v, size_t lo, size_t hi) { return (int)(v < lo ? lo : (v > hi ? hi : v)); };
-    // CTAs per launch are bounded by the scratch cap as well as by the partial-sum cap
-    const size_t scr_cta = ssm::real_bwd_scratch_floats(p->N, p->T) * 4;
-    const int64_t ctas_cap = scr_cta > 0 ? (int64_t)(kRealBwdScratchCap / scr_cta) : ctas_per_seg;
-    const size_t segs_cap = (size_t)(ctas_cap / ctas_per_seg > 1 ? ctas_cap / ctas_per_seg : 1);
+    // launches as large as the partial-sum cap allows: the scratch is one slot per resident CTA
+    const size_t segs_cap = (size_t)p->nC + 1;
     // one wave of CTAs (kTargetCtas..kRealBwdSlots), or several waves that fill the SMs to at
     // least 80 %: no time split.  Otherwise (too few CTAs, or a partial last wave that would
     // leave most SMs idle) concurrent segments of at most 4 chunks, each launch holding as many
@@ -150,13 +152,17 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     // gG holds the summaries' local adjoints and then, overwritten by the carry, the adjoint
     // entering each segment but the last (sequential blocks hand it over through gG too)
     const size_t bvin = BS > 1 ? B * (BS - 1) * DN * 4 : 0;
+    // gP (the summaries' products) is dead once the carry has run, before any scan CTA writes its
+    // dA_log partial sum: the two share one region
     o = kStatusBytes;
-    p->b_gP = o;   o = align256(o + (p->b_seq ? 0 : bvin));
+    p->b_gP = o;   o = align256(o + B * BS * DN * 4);
+    p->b_dA = p->b_gP;
     p->b_gG = o;   o = align256(o + bvin);
     p->b_part = o; o = align256(o + (size_t)p->ndt * B * (size_t)p->b_rows * 2 * p->N * 4);
-    p->b_dA = o;   o = align256(o + B * BS * DN * 4);
     p->b_dD = o;   o = align256(o + B * BS * (size_t)p->D * 4);
-    p->b_bnd = o;  o = align256(o + (size_t)p->ndt * B * per * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
+    const int64_t ctas = (int64_t)p->ndt * p->B * per;
+    p->b_nslot = (int)(ctas < kRealBwdSlots ? (ctas > 0 ? ctas : 1) : kRealBwdSlots);
+    p->b_bnd = o;  o = align256(o + (size_t)p->b_nslot * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
     p->b_end = o;
     return SSM_OK;
 }
@@ -324,7 +330,8 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const 
     if ((st = check_arrays(ptrs, counts, 18)) != SSM_OK) return st;
     if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), s) != cudaSuccess) return SSM_ERR_CUDA;
+    // status word and scratch-slot mask
+    if (cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) return SSM_ERR_CUDA;
     if (p.B == 0 || p.L == 0) {
         if (cudaMemsetAsync(dA_log, 0, DN * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
         if (cudaMemsetAsync(dD, 0, (size_t)p.D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
@@ -340,6 +347,8 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const 
     a.dBC_part = at<float>(ws, p.b_part); a.dA_part = at<float>(ws, p.b_dA);
     a.dD_part = at<float>(ws, p.b_dD);
     a.bnd_scratch = at<float>(ws, p.b_bnd);
+    a.slot_mask = at<unsigned>(ws, kSlotMaskOffset);
+    a.nslot = p.b_nslot;
     a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
     a.status = at<unsigned>(ws, 0);
     a.h0 = o.h0; a.dhL = o.dhL; a.dh0 = o.dh0; a.zoh = o.discretization == SSM_ZOH;

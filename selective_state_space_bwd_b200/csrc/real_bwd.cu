@@ -205,10 +205,45 @@ __device__ __forceinline__ void st_slots(float* row, const float2 (&o)[2], const
     row[sidx[3]] = o[1].y;
 }
 
+// A scratch slot for this CTA: claims a clear bit of the slot mask (the search starts at `start`),
+// or returns -1 once the bounded wait gives up.  A slot is held from a CTA's start to its end, so
+// with at least as many slots as resident CTAs a clear bit exists whenever a CTA starts; with
+// fewer, a CTA waits for a holder to finish (holders never wait), which the bound allows for.
+constexpr unsigned kSlotSpinLimit = 1u << 22;  // x 256 ns sleeps: about a second
+__device__ int claim_slot(unsigned* mask, int nslot, int start) {
+    // first the CTA's own slot (CTAs of a launch with no more CTAs than slots never meet)
+    {
+        const unsigned bit = 1u << (start & 31);
+        if (!(atomicOr(mask + start / 32, bit) & bit)) {
+            __threadfence();
+            return start;
+        }
+    }
+    const int nw = (nslot + 31) / 32;
+    for (unsigned it = 0; it < kSlotSpinLimit; ++it) {
+        for (int k = 0; k < nw; ++k) {
+            const int w = (start / 32 + k) % nw;
+            const unsigned valid = (w == nw - 1 && (nslot & 31)) ? (1u << (nslot & 31)) - 1u : ~0u;
+            unsigned clear = ~*reinterpret_cast<volatile unsigned*>(mask + w) & valid;
+            while (clear) {
+                const unsigned bit = 1u << (__ffs(clear) - 1);
+                const unsigned old = atomicOr(mask + w, bit);
+                if (!(old & bit)) {
+                    __threadfence();  // the previous holder's accesses come first
+                    return w * 32 + (__ffs(bit) - 1);
+                }
+                clear = ~old & valid;
+            }
+        }
+        __nanosleep(256);
+    }
+    return -1;
+}
+
 // MINB: CTAs per SM the register allocation must allow.  4 (126 registers for the Euler N = 16
 // kernel) lets grids of up to 592 CTAs run in one wave; 3 leaves the compiler more registers,
 // which is faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
-template <typename E, int N, bool ZOH, int MINB, bool A2A>
+template <typename E, int N, bool ZOH, int MINB, bool A2A, bool POOL>
 __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N, A2A>;
@@ -218,6 +253,9 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     // per-step channel sums over the states: sum g w' B (dx), sum A q, and for zero-order hold
     // also sum g a B (ddelta; with Euler it equals the first)
     constexpr int SV = ZOH ? 3 : 2;
+    // zero-order hold: E1 of a window's steps kept in registers from the recompute, or (the
+    // instance for four CTAs per SM, within 128 registers) evaluated again in the sweep
+    constexpr bool KEEP_E1 = ZOH && MINB < 4;
     constexpr int TT = Cfg::TT, N2 = 2 * N;
     extern __shared__ __align__(16) unsigned char smem[];
 
@@ -239,7 +277,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     const int c_end = min(p.nC, c_begin + p.seg_chunks);
 
     float2 A[P2], A2[P2], v[P2], dA[P2];
-    float2 Ar[P2];  // zero-order hold: 1 / A
+    float2 Ar[P2];  // zero-order hold: 1 / A (the instance keeping E1; the other takes 1 / z per use)
     {
         const float* al = p.A_log + (size_t)(dv ? d : 0) * N;
 #pragma unroll
@@ -274,8 +312,21 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     E* ddrb = static_cast<E*>(p.ddraw) + boff * p.D;
     float* partb = p.dBC_part + ((size_t)blockIdx.x * p.B + b) * (size_t)p.part_rows * N2 -
                    (size_t)p.part_t0 * N2;  // indexed by absolute step t
-    const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    float* scr = p.bnd_scratch + cta * real_bwd_scratch_floats(N, T);
+    // scratch slot: the CTA's own index when the launch has no more CTAs than slots; else (POOL)
+    // one claimed from the slot mask for the CTA's lifetime
+    const int cta = (int)(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x);
+    int slot = cta;
+    if constexpr (POOL) {
+        __shared__ int s_slot;
+        if (tid == 0) s_slot = claim_slot(p.slot_mask, p.nslot, cta % p.nslot);
+        __syncthreads();
+        slot = s_slot;
+        if (slot < 0) {  // no slot within the bound: this CTA's outputs stay unwritten, the call fails
+            if (tid == 0) flag_status(p.status, kStatusTimeout);
+            return;
+        }
+    }
+    float* scr = p.bnd_scratch + (size_t)slot * real_bwd_scratch_floats(N, T);
     float* bnd = scr + (size_t)tid * 4;                        // window starts: [T/W][NT][4]
     float2* dsg = reinterpret_cast<float2*>(scr + (size_t)(T / W) * NT * 4);  // (delta, sigma) [T][DT]
     const int roff = rot * N + n0;  // this thread's slots within a staged row of ROT * N floats
@@ -462,8 +513,8 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                     float2 hc[P2] = {hw[0], hw[1]};
                     if (q >= 1) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase + q - 1) * NT * 4);
                     float2 bqs[W][P2];
-                    float2 e1s[ZOH ? W : 1][P2];  // zero-order hold: E1(delta A) per step
-                    float dls[W], dxs[W], rds[ZOH ? W : 1];
+                    float2 e1s[KEEP_E1 ? W : 1][P2];  // zero-order hold: E1(delta A) per step
+                    float dls[W], dxs[W], rds[KEEP_E1 ? W : 1];
 #pragma unroll
                     for (int u = 0; u < W; ++u) {
                         const int r = q * W + u;
@@ -472,7 +523,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                         ld_pairs<4>(bqs[u], sBr + r * ROT * N + roff);
                         dls[u] = dlt;
                         dxs[u] = dxv;
-                        if constexpr (ZOH) rds[u] = __fdividef(1.0f, dlt);
+                        if constexpr (KEEP_E1) rds[u] = __fdividef(1.0f, dlt);
 #pragma unroll
                         for (int i = 0; i < P2; ++i) {
                             const float2 zl2 = __fmul2_rn(f2(dlt), A2[i]);
@@ -481,9 +532,9 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                             aa[u][i] = a;
                             pp[u][i] = pr;
                             if constexpr (ZOH) {
-                                const float2 e1 = zoh_e1(__fmul2_rn(zl2, f2(kLn2)), a,
-                                                         __fmul2_rn(f2(rds[u]), Ar[i]));
-                                e1s[u][i] = e1;
+                                const float2 z = __fmul2_rn(zl2, f2(kLn2));
+                                const float2 e1 = zoh_e1(z, a, KEEP_E1 ? __fmul2_rn(f2(rds[u]), Ar[i]) : rcp_pair(z));
+                                if constexpr (KEEP_E1) e1s[u][i] = e1;
                                 hc[i] = __ffma2_rn(__fmul2_rn(f2(dxv), e1), bqs[u][i], pr);
                             } else {
                                 hc[i] = __ffma2_rn(f2(dxv), bqs[u][i], pr);
@@ -511,12 +562,16 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                             if constexpr (ZOH) {
                                 // input weight phi = delta E1; d phi / ddelta = a;
                                 // d phi / dA = delta^2 E2
-                                const float2 e1 = e1s[uu][i];
+                                const float2 z = __fmul2_rn(__fmul2_rn(f2(dlt), A2[i]), f2(kLn2));
+                                const float2 rz = KEEP_E1 ? __fmul2_rn(f2(rds[uu]), Ar[i]) : rcp_pair(z);
+                                float2 e1;
+                                if constexpr (KEEP_E1)
+                                    e1 = e1s[uu][i];
+                                else
+                                    e1 = zoh_e1(z, aa[uu][i], rz);  // as in the recompute
                                 const float2 hj = __ffma2_rn(__fmul2_rn(f2(dxv), e1), bqs[uu][i],
                                                              pp[uu][i]);           // h_t
-                                const float2 e2 = zoh_e2(
-                                    __fmul2_rn(__fmul2_rn(f2(dlt), A2[i]), f2(kLn2)), aa[uu][i],
-                                    e1, __fmul2_rn(f2(rds[uu]), Ar[i]));
+                                const float2 e2 = zoh_e2(z, aa[uu][i], e1, rz);
                                 const float2 gb = __fmul2_rn(g, bqs[uu][i]);
                                 dA[i] = __ffma2_rn(gb, __fmul2_rn(f2(dxv * dlt), e2), dA[i]);
                                 sg = __ffma2_rn(gb, e1, sg);
@@ -593,6 +648,13 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
         if (p.dh0 && seg == 0) st_slots(p.dh0 + ((size_t)b * p.D + d) * N, v, sidx);
         if (!all_finite<4>(v)) flag_status(p.status, kStatusNonFinite);
     }
+    if constexpr (POOL) {
+        __syncthreads();  // every thread is done with the scratch slot
+        if (tid == 0) {
+            __threadfence();
+            atomicAnd(p.slot_mask + slot / 32, ~(1u << (slot & 31)));
+        }
+    }
 }
 
 // dB, dC for the steps [part_t0, part_t0 + rows) of the current launch: fixed-order sums of the
@@ -667,9 +729,12 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
     // at most three CTAs per SM: the all-to-all instance; four: the reduce-scatter instance, whose
     // registers and shared memory fit four
     const size_t sm3 = BwdSmem<E, N, true>::BYTES, sm4 = BwdSmem<E, N, false>::BYTES;
-    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true>, sm3)) != cudaSuccess) return e;
-    if constexpr (N == 16 && !ZOH)
-        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false>, sm4)) != cudaSuccess) return e;
+    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true, false>, sm3)) != cudaSuccess) return e;
+    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true, true>, sm3)) != cudaSuccess) return e;
+    if constexpr (N == 16) {
+        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false, false>, sm4)) != cudaSuccess) return e;
+        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false, true>, sm4)) != cudaSuccess) return e;
+    }
     const int per = a.seq_blocks ? 1 : group;
     for (int hi = a.nseg; hi > 0; hi -= per) {
         const int lo = hi - per > 0 ? hi - per : 0;
@@ -678,13 +743,22 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         const int t_hi = min(a.L, hi * a.seg_chunks * a.T);
         const int rows = t_hi - a.part_t0;
         const dim3 grid(a.ndt, a.B, hi - lo);
-        bool wide = false;  // more CTAs than 3 per SM on 148 SMs
-        if constexpr (N == 16 && !ZOH) wide = (int64_t)a.ndt * a.B * (hi - lo) > 444;
+        const int64_t ctas = (int64_t)a.ndt * a.B * (hi - lo);
+        const bool pool = ctas > a.nslot;  // more CTAs than scratch slots: claim them
+        bool wide = false;                 // more CTAs than 3 per SM on 148 SMs
+        if constexpr (N == 16) wide = ctas > 444;
+        const dim3 blk(BwdCfg<N>::NT);
         if (wide) {
-            if constexpr (N == 16 && !ZOH)
-                real_bwd_kernel<E, N, ZOH, 4, false><<<grid, dim3(BwdCfg<N>::NT), sm4, st>>>(a);
+            if constexpr (N == 16) {
+                if (pool)
+                    real_bwd_kernel<E, N, ZOH, 4, false, true><<<grid, blk, sm4, st>>>(a);
+                else
+                    real_bwd_kernel<E, N, ZOH, 4, false, false><<<grid, blk, sm4, st>>>(a);
+            }
+        } else if (pool) {
+            real_bwd_kernel<E, N, ZOH, 3, true, true><<<grid, blk, sm3, st>>>(a);
         } else {
-            real_bwd_kernel<E, N, ZOH, 3, true><<<grid, dim3(BwdCfg<N>::NT), sm3, st>>>(a);
+            real_bwd_kernel<E, N, ZOH, 3, true, false><<<grid, blk, sm3, st>>>(a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t nbc = (int64_t)a.B * rows * 2 * N;

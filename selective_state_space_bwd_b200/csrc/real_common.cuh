@@ -84,16 +84,21 @@ __device__ __forceinline__ bool all_finite(const float2 (&v)[S / 2]) {
 // For a pair of exponents z = delta * A <= 0 (natural units), with a = exp(z) and rz = 1 / z:
 //   E1(z) = expm1(z) / z           the input weight is phi = (exp(delta A) - 1) / A = delta E1(z)
 //   E2(z) = (exp(z) - E1(z)) / z   d phi / dA = (delta a - phi) / A = delta^2 E2(z)
-// Below |z| = 1/2 both come from their Taylor series about 0 (E1 = sum_k z^k / (k+1)!,
-// E2 = sum_k z^(k-1) k / (k+1)!, eight terms each, remainder under 3e-8 relative); above it from
-// the quotients, where a - 1 and a - E1 do not cancel.  delta = 0 (padding) gives rz = inf and
-// z = 0, which selects the series.
-constexpr float kZohSeries = -0.5f;
+// Below |z| = 1/4 both come from their Taylor series about 0 (E1 = sum_k z^k / (k+1)!,
+// E2 = sum_k z^(k-1) k / (k+1)!), six terms each: the first omitted terms, z^6 / 5040 and
+// z^6 / 5760, are under 1.1e-7 of E1 and E2 there.  From |z| = 1/4 on they come from the
+// quotients: a's relative error (about 2^-22 from the exp2 unit) then costs E1 at most
+// 2.4e-7 / (0.25 * 0.88) = 1.1e-6 relative and E2, through a - E1 >= 0.1, about 1.2e-5.  delta = 0
+// (padding) gives rz = inf and z = 0, which selects the series.
+constexpr float kZohSeries = -0.25f;
+
+// 1 / z of a pair (fast reciprocal; only the quotient branch, |z| >= 1/4, uses it)
+__device__ __forceinline__ float2 rcp_pair(float2 z) {
+    return make_float2(__fdividef(1.0f, z.x), __fdividef(1.0f, z.y));
+}
 
 __device__ __forceinline__ float2 zoh_e1(float2 z, float2 a, float2 rz) {
-    float2 p = f2(1.0f / 40320.0f);
-    p = __ffma2_rn(p, z, f2(1.0f / 5040.0f));
-    p = __ffma2_rn(p, z, f2(1.0f / 720.0f));
+    float2 p = f2(1.0f / 720.0f);
     p = __ffma2_rn(p, z, f2(1.0f / 120.0f));
     p = __ffma2_rn(p, z, f2(1.0f / 24.0f));
     p = __ffma2_rn(p, z, f2(1.0f / 6.0f));
@@ -104,9 +109,7 @@ __device__ __forceinline__ float2 zoh_e1(float2 z, float2 a, float2 rz) {
 }
 
 __device__ __forceinline__ float2 zoh_e2(float2 z, float2 a, float2 e1, float2 rz) {
-    float2 p = f2(1.0f / 45360.0f);
-    p = __ffma2_rn(p, z, f2(1.0f / 5760.0f));
-    p = __ffma2_rn(p, z, f2(1.0f / 840.0f));
+    float2 p = f2(1.0f / 840.0f);
     p = __ffma2_rn(p, z, f2(1.0f / 144.0f));
     p = __ffma2_rn(p, z, f2(1.0f / 30.0f));
     p = __ffma2_rn(p, z, f2(1.0f / 8.0f));

@@ -49,7 +49,10 @@ struct RealArgs {
                       // rows relative to part_t0 (the first step of the current launch)
     float* dA_part;   // [B][nseg][D][N] sum over the segment of delta * q
     float* dD_part;   // [B][nseg][D]
-    float* bnd_scratch;  // per-CTA backward scratch (L2-resident), real_bwd_scratch_floats each
+    float* bnd_scratch;  // backward scratch (L2-resident): nslot slots of real_bwd_scratch_floats,
+                         // each held by one resident CTA at a time
+    unsigned* slot_mask; // bit i set while slot i is held; zero when a launch starts and ends
+    int nslot;
     int seg0;         // backward: first segment handled by this launch (blockIdx.z offset)
     int seq_blocks;   // backward: segments run as sequential launches, each handing its
                       // entering adjoint to the next through vin

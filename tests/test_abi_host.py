@@ -262,8 +262,8 @@ def test_kernel_launch_counts(S):
     one = S.real_shape(8, 2048, 1536, 16, 128, S.SSM_BF16)        # enough CTAs: no time split
     assert S.kernel_launches(one, False) == 1 and S.kernel_launches(one, True) == 3
     # few CTAs: concurrent segments + carry; the backward uses 250 segments of 4 chunks, 63 per
-    # launch (2016 CTAs) so that each launch's dB/dC partial sums and scratch stay under their
-    # caps: summary + carry + 4 x (main + reduce) + params = 11
+    # launch (2016 CTAs) so that each launch's dB/dC partial sums stay under their cap:
+    # summary + carry + 4 x (main + reduce) + params = 11
     split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
     assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 11
     # 512 CTAs fit one wave (4 CTAs per SM on 148 SMs = 592 slots): no time split, time in 4

@@ -88,6 +88,9 @@ CASES = [
     (3, 129, 40, 4, 16, gen.F32, "mamba", 0),
     (2, 520, 96, 16, 128, gen.BF16, "mamba", 0),
     (1, 1000, 64, 16, 128, gen.F32, "stiff", 0),
+    # more than 444 CTAs of 32 channels: the backward instance for four CTAs per SM
+    (15, 200, 1024, 16, 64, gen.F32, "stiff", 0),
+    (4, 260, 4096, 16, 128, gen.BF16, "mamba", 0),
 ]
 
 
