@@ -13,11 +13,11 @@
 // TMA (cp.async.bulk.tensor, 128-byte swizzle, out-of-range rows and columns filled with zeros) in
 // the canonical layouts the tensor core reads through its shared-memory descriptors: k-major
 // tiles as rows of 64 k-elements, m/n-major tiles as rows of 64 m/n-elements per k, so every box is
-// a plain 2-D window of a global array.  One thread issues the copies and the MMAs (four k16 steps
-// per stage); mbarriers carry "stage full" (TMA transaction bytes) and "stage free" / "accumulator
-// ready" (tcgen05.commit); the other warps only drain the accumulator from tensor memory.  The
-// issue / wait order and the phase parities are model-checked on the host by
-// tests/test_mbarrier_protocol.py.
+// a plain 2-D window of a global array.  One thread issues the copies and another the MMAs (four
+// k16 steps per stage); mbarriers carry "stage full" (TMA transaction bytes) and "stage free" /
+// "accumulator ready" (tcgen05.commit); the forward also has drain warps of its own (see
+// dtp_fwd_ws_kernel).  The issue / wait order and the phase parities are model-checked on the host
+// by tests/test_mbarrier_protocol.py.
 // The rank R is small (tens to a few hundred), so each GEMM moves far more bytes than it does
 // arithmetic per byte: they are bound by HBM (writing delta_raw, reading g), not by the tensor pipe.
 #include <cuda.h>
@@ -201,11 +201,10 @@ __device__ __forceinline__ void tmem_dealloc_cta(unsigned taddr, unsigned cols) 
 template <bool A_MN, bool B_MN, int BN, int STAGES, bool ONES, int EPI>
 __device__ __forceinline__ void tc_tile(const CUtensorMap& mA, const CUtensorMap& mB, const TcArgs& p,
                                         int bn, int bm, int bz, unsigned char* smem_raw) {
-    static_assert(BN % 64 == 0 && BN <= 256 && STAGES >= 3, "n tile of whole 64-wide blocks");
+    static_assert(BN % 64 == 0 && BN <= 256 && STAGES >= 2, "n tile of whole 64-wide blocks");
     static_assert(!ONES || EPI == EPI_F32_PART, "column sums go to the fp32 partial sums");
     using Sm = TcSmem<BN, STAGES, ONES>;
     constexpr int TCOLS = tmem_cols(BN + (ONES ? 64 : 0));
-    constexpr int PF = STAGES - 2;  // stages loading ahead of the one being multiplied
     const unsigned raw = smem_u32(smem_raw);
     const unsigned base = (raw + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
     unsigned char* gbase = smem_raw + (base - raw);
@@ -241,34 +240,33 @@ __device__ __forceinline__ void tc_tile(const CUtensorMap& mA, const CUtensorMap
     const unsigned tmem = *reinterpret_cast<volatile unsigned*>(gbase + Sm::SLOT);
 
     bool ok = true;
-    if (tid == 0) {
-        auto issue = [&](int t, int st) {
-            const unsigned a = base + st * Sm::STAGE, b = a + A_BYTES, f = full + 8 * st;
-            const int k0 = (int)(kb + (int64_t)t * BK);
-            mbar_expect_tx(f, Sm::STAGE);
-            if (!A_MN) {
-                tma_load_2d(a, &mA, k0, (int)m0, f);
-            } else {
-                tma_load_2d(a, &mA, (int)m0, k0, f);
-                tma_load_2d(a + BK * 128, &mA, (int)m0 + 64, k0, f);
-            }
-            if (!B_MN) {
-                tma_load_2d(b, &mB, k0, (int)n0, f);
-            } else {
+    auto issue = [&](int t, int st) {
+        const unsigned a = base + st * Sm::STAGE, b = a + A_BYTES, f = full + 8 * st;
+        const int k0 = (int)(kb + (int64_t)t * BK);
+        mbar_expect_tx(f, Sm::STAGE);
+        if (!A_MN) {
+            tma_load_2d(a, &mA, k0, (int)m0, f);
+        } else {
+            tma_load_2d(a, &mA, (int)m0, k0, f);
+            tma_load_2d(a + BK * 128, &mA, (int)m0 + 64, k0, f);
+        }
+        if (!B_MN) {
+            tma_load_2d(b, &mB, k0, (int)n0, f);
+        } else {
 #pragma unroll
-                for (int blk = 0; blk < BN / 64; ++blk) tma_load_2d(b + blk * (BK * 128), &mB, (int)n0 + 64 * blk, k0, f);
-            }
-        };
-        for (int t = 0; t < PF && t < nk; ++t) issue(t, t);
-        for (int kt = 0; kt < nk && ok; ++kt) {
-            const int nx = kt + PF;
-            if (nx < nk) {
-                const int st = nx % STAGES;
-                // the stage last held tile nx - STAGES = kt - 2, multiplied a step ago
-                if (nx >= STAGES) ok = mbar_wait(free_ + 8 * st, (unsigned)((nx / STAGES - 1) & 1));
-                if (!ok) break;
-                issue(nx, st);
-            }
+            for (int blk = 0; blk < BN / 64; ++blk) tma_load_2d(b + blk * (BK * 128), &mB, (int)n0 + 64 * blk, k0, f);
+        }
+    };
+    if (tid == 0) {
+        // copies: tile t into stage t % STAGES once the MMAs of tile t - STAGES have read it
+        for (int t = 0; t < nk; ++t) {
+            const int st = t % STAGES;
+            if (t >= STAGES && !(ok = mbar_wait(free_ + 8 * st, (unsigned)((t / STAGES - 1) & 1)))) break;
+            issue(t, st);
+        }
+    } else if (tid == 32) {
+        // MMAs, one stage at a time as its copies land
+        for (int kt = 0; kt < nk; ++kt) {
             const int s = kt % STAGES;
             if (!(ok = mbar_wait(full + 8 * s, (unsigned)((kt / STAGES) & 1)))) break;
             const unsigned a = base + s * Sm::STAGE, b = a + A_BYTES;
@@ -291,7 +289,7 @@ __device__ __forceinline__ void tc_tile(const CUtensorMap& mA, const CUtensorMap
         if (ok) ok = mbar_wait(done, 0);
         tc_fence_before();
     }
-    // the other threads wait here (not spinning on the mbarrier beside thread 0)
+    // the other threads wait here (not spinning on the mbarriers beside threads 0 and 32)
     const bool bad = __syncthreads_or(!ok);
     tc_fence_after();
 
@@ -357,9 +355,9 @@ __device__ __forceinline__ void tc_tile(const CUtensorMap& mA, const CUtensorMap
                         *reinterpret_cast<const uint4*>(gbase + rl * Sm::SROW + 16 * c8);
             }
         }
-    } else if (tid == 0) {
-        flag_status(p.status, kStatusTimeout);
-        mbar_wait(done, 0);  // the MMAs already issued get a last bounded chance to finish
+    } else {
+        if (tid == 0) flag_status(p.status, kStatusTimeout);
+        if (tid == 32) mbar_wait(done, 0);  // the MMAs already issued get a last bounded chance
     }
     tc_fence_before();
     __syncthreads();
@@ -397,46 +395,90 @@ __global__ void __launch_bounds__(NTH) dtp_bwd_kernel(const __grid_constant__ CU
     }
 }
 
-// Forward GEMM, persistent: CTA c handles output tiles c, c + G, c + 2G, ... (tile = 128 rows of u
-// x BN rows of w, the whole k range R <= 64 KA in one stage).  Two stages and two tensor-memory
-// accumulators: while the tensor core multiplies tile i into one accumulator, the eight warps
-// drain tile i - 1 from the other (+ bias, bf16, into a 128-byte-swizzled staging tile that one
-// TMA store writes out) and the copies of tile i + 1 are in flight.
-constexpr int FWD_NTH = 256;
-template <int KA, int BN>
-struct FwdSm {
-    static constexpr int A_ST = KA * TM * 128;     // KA swizzle atoms of 128 rows
-    static constexpr int B_ST = KA * BN * 128;
-    static constexpr int STAGE = A_ST + B_ST;
-    static constexpr int STG = 2 * STAGE;          // output tile: BN / 64 atoms of 128 rows
-    static constexpr int FULL = STG + BN * 256;    // 2 "stage loaded" mbarriers
-    static constexpr int ACC = FULL + 16;          // 2 "accumulator ready" mbarriers
-    static constexpr int SLOT = ACC + 16;
-    static constexpr int BYTES = SLOT + 16 + 1024;
+// Forward GEMM, warp-specialised and persistent.  Work unit = one 128-row tile of u times a run of
+// up to NCH consecutive 64-row tiles of w (one output tile each); CTA c takes units c, c + G, ...
+//   warp 0, one thread: TMA copies: the unit's u tile into one of two A buffers (once per unit),
+//                       each w tile into a ring of STAGES stages;
+//   warp 1, one thread: each output tile's MMAs into one of ACC tensor-memory accumulators (the
+//                       warp also allocates and frees the tensor memory);
+//   warps 2-5: drain.  Warp w reads accumulator lanes 32 (w % 4) .. + 31 (the quarter a warp may
+//              reach), adds the bias, packs bf16 into its own 128-byte-swizzled staging box of
+//              32 rows x 64 columns (two, alternating) and stores it with one TMA copy.
+// No CTA-wide barrier inside the loop: "full" (TMA transaction bytes), "free" and "accumulator
+// full" (tcgen05.commit) and "accumulator free" (one arrival per drain warp) mbarriers hand the
+// tiles on, so copies, MMAs and drains of different tiles overlap.  Copying u once per unit rather
+// than once per output tile matters: u's rows are R bf16 (96 bytes at R = 48), short, unaligned
+// rows that the copy engine moves at a fraction of its rate for long ones.
+constexpr int WS_NTH = 192;
+constexpr int WS_BN = 64;
+template <int KA, int STAGES, int ACC>
+struct WsSm {
+    static constexpr int A_ST = KA * TM * 128;          // u tile: KA swizzle atoms of 128 rows
+    static constexpr int B_ST = KA * WS_BN * 128;       // w tile: KA atoms of 64 rows
+    static constexpr int BST = 2 * A_ST;                // the ring of w stages after two A buffers
+    static constexpr int BOX = 32 * 128;                // staging box: 32 rows x 64 bf16
+    static constexpr int EPI = BST + STAGES * B_ST;     // 4 warps x 2 boxes
+    // afull, afree [2]; full, free [STAGES]; accf, acce [ACC]; done
+    static constexpr int BAR = EPI + 4 * 2 * BOX;
+    static constexpr int SLOT = BAR + (4 + 2 * STAGES + 2 * ACC + 1) * 8;
+    static constexpr int BYTES = SLOT + 8 + 1024;       // + slack to align the base to 1024
 };
 
-template <int KA, int BN>
-__global__ void __launch_bounds__(FWD_NTH) dtp_fwd_kernel(const __grid_constant__ CUtensorMap mA,
-                                                          const __grid_constant__ CUtensorMap mB,
-                                                          const __grid_constant__ CUtensorMap mC, TcArgs p,
-                                                          int64_t n_nt, int64_t ntiles) {
-    static_assert(BN % 64 == 0 && 2 * BN <= 512, "two accumulators of whole 64-wide blocks");
-    using Sm = FwdSm<KA, BN>;
-    constexpr int TCOLS = tmem_cols(2 * BN);
+__device__ __forceinline__ void mbar_arrive(unsigned a) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(a) : "memory");
+}
+// this thread's bulk stores but the most recent one have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory");
+}
+
+template <int KA, int STAGES, int ACC>
+__global__ void __launch_bounds__(WS_NTH, 1) dtp_fwd_ws_kernel(const __grid_constant__ CUtensorMap mA,
+                                                               const __grid_constant__ CUtensorMap mB,
+                                                               const __grid_constant__ CUtensorMap mC,
+                                                               TcArgs p, int n_nt, int nch, int64_t nunits) {
+    using Sm = WsSm<KA, STAGES, ACC>;
+    constexpr int BN = WS_BN;
+    constexpr int TCOLS = tmem_cols(ACC * BN);
+    static_assert(ACC * BN <= 512 && STAGES >= 2, "accumulators fit tensor memory");
     extern __shared__ unsigned char smem_raw[];
     const unsigned raw = smem_u32(smem_raw);
     const unsigned base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    const unsigned full = base + Sm::FULL, acc = base + Sm::ACC, stg = base + Sm::STG;
+    const unsigned bar = base + Sm::BAR;
+    auto afull = [&](int k) { return bar + 8 * k; };
+    auto afree = [&](int k) { return bar + 8 * (2 + k); };
+    auto full = [&](int s) { return bar + 8 * (4 + s); };
+    auto freeb = [&](int s) { return bar + 8 * (4 + STAGES + s); };
+    auto accf = [&](int a) { return bar + 8 * (4 + 2 * STAGES + a); };
+    auto acce = [&](int a) { return bar + 8 * (4 + 2 * STAGES + ACC + a); };
+    const unsigned done = bar + 8 * (4 + 2 * STAGES + 2 * ACC);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int T = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+    const int nchk = (n_nt + nch - 1) / nch;  // n runs per 128-row tile of u
+    // unit k of this CTA: 128-row tile of u and first n tile, number of n tiles
+    auto unit = [&](int64_t k, int64_t& m0, int& nt0, int& nj) {
+        const int64_t g = (int64_t)blockIdx.x + k * gridDim.x;
+        m0 = g / nchk * TM;
+        nt0 = (int)(g % nchk) * nch;
+        nj = n_nt - nt0 < nch ? n_nt - nt0 : nch;
+    };
+    const int64_t U = (int64_t)blockIdx.x < nunits ? (nunits - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    if (warp == 0) tmem_alloc_cta(base + Sm::SLOT, TCOLS);
+    if (warp == 1) tmem_alloc_cta(base + Sm::SLOT, TCOLS);
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(full + 8 * s, 1);
-            mbar_init(acc + 8 * s, 1);
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(afull(k), 1);
+            mbar_init(afree(k), 1);
         }
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(freeb(s), 1);
+        }
+        for (int a = 0; a < ACC; ++a) {
+            mbar_init(accf(a), 1);
+            mbar_init(acce(a), 4);
+        }
+        mbar_init(done, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     tc_fence_before();
@@ -444,119 +486,142 @@ __global__ void __launch_bounds__(FWD_NTH) dtp_fwd_kernel(const __grid_constant_
     tc_fence_after();
     const unsigned tmem = *reinterpret_cast<volatile unsigned*>(gbase + Sm::SLOT);
 
-    auto tile_m0 = [&](int i) { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) / n_nt * TM; };
-    auto tile_n0 = [&](int i) { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) % n_nt * BN; };
-    auto issue = [&](int i, int s) {  // thread 0: both operands of tile i, every k atom
-        const unsigned a = base + s * Sm::STAGE, b = a + Sm::A_ST, f = full + 8 * s;
-        const int m0 = (int)tile_m0(i), n0 = (int)tile_n0(i);
-        mbar_expect_tx(f, Sm::STAGE);
-#pragma unroll
-        for (int at = 0; at < KA; ++at) {
-            tma_load_2d(a + at * (TM * 128), &mA, 64 * at, m0, f);
-            tma_load_2d(b + at * (BN * 128), &mB, 64 * at, n0, f);
-        }
-    };
-    // accumulator of tile i -> + bias -> bf16 -> swizzled staging tile -> TMA store (thread 0)
-    auto drain = [&](int i) {
-        const int64_t m0 = tile_m0(i), n0 = tile_n0(i);
-        const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-        const unsigned tl = tmem + (i & 1) * BN + ((unsigned)((warp & 3) * 32) << 16);
-#pragma unroll
-        for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
-            float v[32];
-            tmem_ld32(tl + c0, v);
-            if (p.bias != nullptr) {
-                if (n0 + c0 + 32 <= p.N) {
-                    const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + c0);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 bb = __ldg(b4 + q);
-                        v[4 * q] += bb.x;
-                        v[4 * q + 1] += bb.y;
-                        v[4 * q + 2] += bb.z;
-                        v[4 * q + 3] += bb.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (n0 + c0 + j < p.N) v[j] += __ldg(p.bias + n0 + c0 + j);
-                }
-            }
-            // columns c0 .. c0 + 31: 16-byte chunks (c0 % 64) / 8 + q of the 64-column atom c0 / 64
-            const unsigned atom = stg + (c0 / 64) * (TM * 128) + row * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                unsigned w4[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
-                    w4[j] = *reinterpret_cast<const unsigned*>(&h);
-                }
-                const int cc = (c0 % 64) / 8 + q;
-                st_shared_v4(atom + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-#pragma unroll
-            for (int hb = 0; hb < BN / 64; ++hb) tma_store_2d(&mC, stg + hb * (TM * 128), (int)n0 + 64 * hb, (int)m0);
-            bulk_commit();
-        }
-    };
-
     bool ok = true;
-    if (tid == 0 && T > 0) issue(0, 0);
-    for (int i = 0; i < T; ++i) {
-        const int s = i & 1;
-        if (tid == 0) {
-            // stage s ^ 1 and accumulator s ^ 1 held tile i - 1: once its MMAs are done the stage
-            // takes tile i + 1 and the accumulator can be drained
-            if (i >= 1) ok = mbar_wait(acc + 8 * (s ^ 1), (unsigned)(((i - 1) >> 1) & 1));
-            if (ok && i + 1 < T) issue(i + 1, s ^ 1);
-            if (ok) ok = mbar_wait(full + 8 * s, (unsigned)((i >> 1) & 1));
-            if (ok) {
-                tc_fence_after();
-                const unsigned a = base + s * Sm::STAGE, b = a + Sm::A_ST;
+    if (warp == 0) {
+        if (lane == 0) {
+            int i = 0;  // output tiles so far
+            for (int64_t k = 0; k < U && ok; ++k) {
+                int64_t m0;
+                int nt0, nj;
+                unit(k, m0, nt0, nj);
+                const int ab = (int)(k & 1);
+                // the A buffer last held unit k - 2: its MMAs must be done
+                if (k >= 2 && !(ok = mbar_wait(afree(ab), (unsigned)(((k >> 1) - 1) & 1)))) break;
+                const unsigned a = base + ab * Sm::A_ST;
+                mbar_expect_tx(afull(ab), Sm::A_ST);
 #pragma unroll
-                for (int j = 0; j < 4 * KA; ++j)
-                    umma_bf16(tmem + s * BN, sw128_desc(a + (j >> 2) * (TM * 128) + (j & 3) * 32, 16, 1024),
-                              sw128_desc(b + (j >> 2) * (BN * 128) + (j & 3) * 32, 16, 1024),
-                              idesc_bf16(BN, false, false), j != 0);
-                umma_commit(acc + 8 * s);
+                for (int at = 0; at < KA; ++at) tma_load_2d(a + at * (TM * 128), &mA, 64 * at, (int)m0, afull(ab));
+                for (int j = 0; j < nj; ++j, ++i) {
+                    const int s = i % STAGES, r = i / STAGES;
+                    // the stage last held tile i - STAGES: its MMAs must be done
+                    if (r >= 1 && !(ok = mbar_wait(freeb(s), (unsigned)((r - 1) & 1)))) break;
+                    const unsigned b = base + Sm::BST + s * Sm::B_ST;
+                    mbar_expect_tx(full(s), Sm::B_ST);
+#pragma unroll
+                    for (int at = 0; at < KA; ++at)
+                        tma_load_2d(b + at * (BN * 128), &mB, 64 * at, (nt0 + j) * BN, full(s));
+                }
             }
-            bulk_wait_read();  // the staging tile of the previous drain has been read out
-            tc_fence_before();
         }
-        if (__syncthreads_or(!ok)) {
-            ok = false;
-            break;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int i = 0;
+            for (int64_t k = 0; k < U && ok; ++k) {
+                int64_t m0;
+                int nt0, nj;
+                unit(k, m0, nt0, nj);
+                const int ab = (int)(k & 1);
+                if (!(ok = mbar_wait(afull(ab), (unsigned)((k >> 1) & 1)))) break;
+                const unsigned a = base + ab * Sm::A_ST;
+                for (int j = 0; j < nj; ++j, ++i) {
+                    const int s = i % STAGES, ac = i % ACC;
+                    if (!(ok = mbar_wait(full(s), (unsigned)((i / STAGES) & 1)))) break;
+                    // the accumulator last held tile i - ACC: all four drain warps must have read it
+                    if (i >= ACC && !(ok = mbar_wait(acce(ac), (unsigned)((i / ACC - 1) & 1)))) break;
+                    tc_fence_after();
+                    const unsigned b = base + Sm::BST + s * Sm::B_ST;
+#pragma unroll
+                    for (int jj = 0; jj < 4 * KA; ++jj)
+                        umma_bf16(tmem + ac * BN,
+                                  sw128_desc(a + (jj >> 2) * (TM * 128) + (jj & 3) * 32, 16, 1024),
+                                  sw128_desc(b + (jj >> 2) * (BN * 128) + (jj & 3) * 32, 16, 1024),
+                                  idesc_bf16(BN, false, false), jj != 0);
+                    umma_commit(freeb(s));
+                    umma_commit(accf(ac));
+                }
+                umma_commit(afree(ab));  // once the unit's MMAs are done, its A buffer is free
+            }
+            umma_commit(done);  // arrives once every MMA issued above has completed
         }
-        if (i >= 1) {
-            tc_fence_after();
-            drain(i - 1);
+    } else {
+        const int q = warp & 3;                               // accumulator lane quarter
+        const unsigned tq = tmem + ((unsigned)(q * 32) << 16);
+        const unsigned box0 = base + Sm::EPI + (warp - 2) * 2 * Sm::BOX;
+        const bool has_bias = p.bias != nullptr;
+        // bias of the tile's columns n0 + 2 lane and + 1 (lane pairs; a drain takes the other
+        // lanes' pairs by shuffles), loaded one tile ahead so that its latency stays off the drain
+        auto bias_pair = [&](int64_t n0) {
+            const int64_t c = n0 + 2 * lane;  // N is a multiple of 8: c < N gives c + 1 < N
+            return has_bias && c < p.N ? __ldg(reinterpret_cast<const float2*>(p.bias + c))
+                                       : make_float2(0.0f, 0.0f);
+        };
+        int64_t m0n = 0;
+        int nt0n = 0, njn = 0;
+        if (U > 0) unit(0, m0n, nt0n, njn);
+        float2 bnext = bias_pair((int64_t)nt0n * BN);
+        int i = 0;
+        for (int64_t k = 0; k < U && ok; ++k) {
+            int64_t m0;
+            int nt0, nj;
+            unit(k, m0, nt0, nj);
+            for (int j = 0; j < nj; ++j, ++i) {
+                const int ac = i % ACC;
+                const float2 bcur = bnext;
+                // the next tile's bias: the next run of this unit, or the next unit's first
+                if (j + 1 < nj) {
+                    bnext = bias_pair((int64_t)(nt0 + j + 1) * BN);
+                } else if (k + 1 < U) {
+                    unit(k + 1, m0n, nt0n, njn);
+                    bnext = bias_pair((int64_t)nt0n * BN);
+                }
+                if (!(ok = mbar_wait(accf(ac), (unsigned)((i / ACC) & 1)))) break;
+                tc_fence_after();
+                const int64_t n0 = (int64_t)(nt0 + j) * BN;
+                const unsigned box = box0 + (i & 1) * Sm::BOX;
+                if (lane == 0) bulk_wait_read_1();  // the store of tile i - 2 has read this box
+                __syncwarp();
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tq + ac * BN + c0, v);
+                    if (has_bias) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            v[e] += __shfl_sync(0xffffffffu, bcur.x, (c0 + e) >> 1);
+                            v[e + 1] += __shfl_sync(0xffffffffu, bcur.y, (c0 + e) >> 1);
+                        }
+                    }
+                    // columns c0 .. c0 + 31: 16-byte chunks c0 / 8 + e of the box row `lane`, swizzled
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        unsigned w4[4];
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * e + 2 * f], v[8 * e + 2 * f + 1]);
+                            w4[f] = *reinterpret_cast<const unsigned*>(&h);
+                        }
+                        const int cc = c0 / 8 + e;
+                        st_shared_v4(box + lane * 128 + ((cc ^ (lane & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+                tc_fence_before();
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(acce(ac));  // this warp's lanes of the accumulator are read
+                    tma_store_2d(&mC, box, (int)n0, (int)m0 + q * 32);
+                    bulk_commit();
+                }
+            }
         }
+        if (lane == 0) bulk_wait_all();
     }
-    if (tid == 0 && ok && T > 0) {
-        ok = mbar_wait(acc + 8 * ((T - 1) & 1), (unsigned)(((T - 1) >> 1) & 1));
-        bulk_wait_read();
-        tc_fence_before();
-    }
-    if (!__syncthreads_or(!ok)) {
-        if (T > 0) {
-            tc_fence_after();
-            drain(T - 1);
-        }
-    } else if (tid == 0) {
-        flag_status(p.status, kStatusTimeout);
-        // the MMAs already issued get a last bounded chance to finish
-        if (T > 0) mbar_wait(acc + 8 * ((T - 1) & 1), (unsigned)(((T - 1) >> 1) & 1));
-    }
-    if (tid == 0) bulk_wait_all();
+    if (__syncthreads_or(!ok) && tid == 0) flag_status(p.status, kStatusTimeout);
+    // every MMA issued has completed (bounded wait) before the tensor memory is freed
+    if (warp == 1 && lane == 0) mbar_wait(done, 0);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_cta(tmem, TCOLS);
     }
@@ -626,32 +691,48 @@ cudaError_t run_tc(const CUtensorMap& mA, const CUtensorMap& mB, const TcArgs& a
     return cudaGetLastError();
 }
 
-template <int KA, int BN>
+template <int KA, int STAGES, int ACC>
 cudaError_t run_fwd(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC, const TcArgs& a,
                     cudaStream_t st) {
-    constexpr int bytes = FwdSm<KA, BN>::BYTES;
-    auto kern = dtp_fwd_kernel<KA, BN>;
+    constexpr int bytes = WsSm<KA, STAGES, ACC>::BYTES;
+    auto kern = dtp_fwd_ws_kernel<KA, STAGES, ACC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100)) != cudaSuccess)
         return e;
-    int dev = 0, sms = 0, per_sm = 0;
+    int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    // CTAs per SM: shared memory (with the per-CTA reservation) and the two accumulators in the
-    // SM's 512 tensor-memory columns bound it (registers do not, at 256 threads)
+    // CTAs per SM: shared memory (with the per-CTA reservation) and the accumulators in the SM's
+    // 512 tensor-memory columns bound it
     int smem_sm = 0, resv = 0;
     if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
         return e;
     if ((e = cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
-    per_sm = smem_sm / (bytes + resv);
-    const int tcap = 512 / tmem_cols(2 * BN);
+    int per_sm = smem_sm / (bytes + resv);
+    const int tcap = 512 / tmem_cols(ACC * WS_BN);
     if (per_sm > tcap) per_sm = tcap;
     if (per_sm < 1) per_sm = 1;
-    const int64_t n_nt = (a.N + BN - 1) / BN;
-    const int64_t ntiles = n_nt * ((a.M + TM - 1) / TM);
-    const int64_t grid = ntiles < (int64_t)sms * per_sm ? ntiles : (int64_t)sms * per_sm;
-    kern<<<(unsigned)grid, FWD_NTH, bytes, st>>>(mA, mB, mC, a, n_nt, ntiles);
+    const int64_t slots = (int64_t)sms * per_sm;
+    const int n_nt = (int)((a.N + WS_BN - 1) / WS_BN);
+    const int64_t n_mt = (a.M + TM - 1) / TM;
+    // n tiles per unit: the run length that puts the fewest output tiles (plus one u copy per
+    // unit, weighted as half a tile) on the busiest CTA
+    int nch = n_nt;
+    double best = -1.0;
+    for (int k = 1; k <= n_nt && k <= 64; ++k) {  // k runs per u tile
+        const int c = (n_nt + k - 1) / k;
+        const int64_t units = n_mt * ((n_nt + c - 1) / c);
+        const int64_t per = (units + slots - 1) / slots;
+        const double cost = (double)per * c + 0.5 * (double)per;
+        if (best < 0.0 || cost < best) {
+            best = cost;
+            nch = c;
+        }
+    }
+    const int64_t nunits = n_mt * ((n_nt + nch - 1) / nch);
+    const int64_t grid = nunits < slots ? nunits : slots;
+    kern<<<(unsigned)grid, WS_NTH, bytes, st>>>(mA, mB, mC, a, n_nt, nch, nunits);
     return cudaGetLastError();
 }
 
@@ -666,13 +747,10 @@ int64_t dtproj_rows_per_split(int R) { return R <= 64 ? 1536 : 1024; }
 cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     // delta_raw [M x D] = u [M x R] . w [D x R]^T + bias: both operands k-major
     const int ka = (d.R + 63) / 64;              // 64-deep k atoms covering R, all in one stage
-    // n tile: 64 for one k atom (three CTAs per SM instead of two), 128 for two (a wider tile
-    // amortises the second atom's copies), 64 beyond
-    const int bn = ka == 2 ? 128 : 64;
     CUtensorMap mA, mB, mC;
     cudaError_t e = make_map(&mA, d.u, d.M, d.R, d.R, TM);
-    if (e == cudaSuccess) e = make_map(&mB, d.w, d.D, d.R, d.R, bn);
-    if (e == cudaSuccess) e = make_map(&mC, d.delta_raw, d.M, d.D, d.D, TM);
+    if (e == cudaSuccess) e = make_map(&mB, d.w, d.D, d.R, d.R, WS_BN);
+    if (e == cudaSuccess) e = make_map(&mC, d.delta_raw, d.M, d.D, d.D, 32);  // a drain warp's box
     if (e != cudaSuccess) return e;
     TcArgs a = {};
     a.M = d.M; a.N = d.D; a.K = d.R; a.ldc = d.D; a.kchunk = d.R;
@@ -680,11 +758,13 @@ cudaError_t launch_dtproj_fwd(const DtArgs& d, cudaStream_t st) {
     a.C = d.delta_raw;
     a.bias = d.bias;
     a.status = d.status;
+    // w stages: four for one or two k atoms (two CTAs per SM for one), three and two beyond (one
+    // CTA per SM)
     switch (ka) {
-        case 1: return run_fwd<1, 64>(mA, mB, mC, a, st);
-        case 2: return run_fwd<2, 128>(mA, mB, mC, a, st);
-        case 3: return run_fwd<3, 64>(mA, mB, mC, a, st);
-        default: return run_fwd<4, 64>(mA, mB, mC, a, st);
+        case 1: return run_fwd<1, 4, 4>(mA, mB, mC, a, st);
+        case 2: return run_fwd<2, 4, 4>(mA, mB, mC, a, st);
+        case 3: return run_fwd<3, 3, 4>(mA, mB, mC, a, st);
+        default: return run_fwd<4, 2, 4>(mA, mB, mC, a, st);
     }
 }
 
