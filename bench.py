@@ -446,12 +446,16 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def complex_algorithmic_bytes(w):
-    """Minimum bytes of one complex fwd + bwd: u read and h written by the forward; h (or, from
-    checkpoints, u) and g read, du written by the backward (8 B each, complex64); r and phi read
-    by both, dr and dphi written (4 B each).  The checkpoints (1/T of the trajectory) are left
-    out."""
+def complex_algorithmic_bytes(w, ckpt=False):
+    """Minimum bytes of one complex fwd + bwd (8 B per complex64 element, 4 B per real one).
+    From the stored trajectory: the forward reads u and writes h, the backward reads h and g and
+    writes du.  From chunk checkpoints (ckpt): the forward reads u and writes the checkpoints, the
+    backward reads them, u and g and writes du.  Both read r and phi; the backward writes dr and
+    dphi."""
     BLK, BL = w.batch * w.seqlen * w.modes, w.batch * w.seqlen
+    if ckpt:
+        ck = w.batch * (-(-w.seqlen // w.chunk)) * w.modes * 8
+        return 8 * BLK + 8 * BL + ck, 24 * BLK + 16 * BL + ck
     return 16 * BLK + 8 * BL, 24 * BLK + 16 * BL
 
 
@@ -597,7 +601,7 @@ def main_complex(args, w):
     upd_rank = w.batch * w.seqlen * w.modes
     value = world * upd_rank * args.steps / t_step
     hbm, peak_kind = peaks()
-    fb, bb = complex_algorithmic_bytes(w)
+    fb, bb = complex_algorithmic_bytes(w, ckpt=args.ckpt)
     if args.rtrl:  # u and g read (8 B each per update), r and phi read (4 B each per (b, t))
         fb, bb = 16 * w.batch * w.seqlen * w.modes + 8 * w.batch * w.seqlen, 0
     bwd_gbs = bb / (t_bwd / args.steps) / 1e9 if bb else 0.0
