@@ -266,6 +266,11 @@ def test_kernel_launch_counts(S):
     # summary + carry + 4 x (main + reduce) + params = 11
     split = S.real_shape(1, 128000, 1024, 16, 128, S.SSM_F32)
     assert S.kernel_launches(split, False) == 3 and S.kernel_launches(split, True) == 11
+    # 40 segments of 4 chunks x 64 CTAs, 20 per launch: 1280 CTAs per launch, more than the 592
+    # resident ones, so the scratch is 592 slots that CTAs claim (58.2 MB, not 125.8 MB)
+    multi = S.real_shape(2, 20000, 1024, 16, 128, S.SSM_F32)
+    assert S.kernel_launches(multi, True) == 7
+    assert S.workspace_bytes(multi, True) - 592 * 98304 < 95_000_000
     # 512 CTAs fit one wave (4 CTAs per SM on 148 SMs = 592 slots): no time split, time in 4
     # sequential blocks under the partial cap
     wave = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)

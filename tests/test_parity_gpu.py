@@ -182,6 +182,33 @@ def test_nonfinite_status(S):
     assert S.ssm_scan_status(ws) == 0
 
 
+def test_multiwave_backward_scratch_slots(S, oracle_mod):
+    """A time-split backward whose launches hold more CTAs than the 592 resident ones (B=2,
+    L=20000, D=1024: segments of 4 chunks x 64 CTAs, 20 segments = 1280 CTAs per launch), so
+    its CTAs claim scratch slots from the workspace's slot mask.  Every output against the
+    oracle, the status word clean after each call, and a second call on the same workspace
+    (whose mask the first left clear) bitwise equal."""
+    B, L, D, N, T = 2, 20000, 1024, 16, 128
+    inp = gen.real_inputs(B, L, D, N, gen.F32, "stiff", seed=23)
+    shape = S.real_shape(B, L, D, N, T, S.SSM_F32)
+    assert S.kernel_launches(shape, True) == 7  # summary, carry, 2 x (scan + dB/dC sums), params
+    wsb = torch.empty(S.workspace_bytes(shape, True), dtype=torch.uint8, device="cuda")
+    dt = torch.float32
+    x, dr, dy = (to_dev(inp[k], dt) for k in ("x", "delta_raw", "dy"))
+    Bm, Cm, A_log, Dskip = (to_dev(inp[k], dt) for k in ("Bm", "Cm", "A_log", "Dskip"))
+    y, ckpt = S.ssm_scan_fwd(x, dr, A_log, Bm, Cm, Dskip, chunk=T)
+    g1 = S.ssm_scan_bwd(x, dr, A_log, Bm, Cm, Dskip, ckpt, dy, chunk=T, ws=wsb)
+    g1 = {k: v.clone() for k, v in g1.items()}
+    assert S.ssm_scan_status(wsb) == 0
+    g2 = S.ssm_scan_bwd(x, dr, A_log, Bm, Cm, Dskip, ckpt, dy, chunk=T, ws=wsb)
+    assert S.ssm_scan_status(wsb) == 0
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+    got = {"y": np64(y), "ckpt": np64(ckpt)}
+    got.update({k: np64(v) for k, v in g1.items()})
+    check_real(got, run_oracle(oracle_mod, inp, T), gen.F32)
+
+
 # ------------------------------------------------------------------------------ complex cases
 
 def run_complex(S, c, T, seg_chunks=0, bwd="ckpt"):
