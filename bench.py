@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--seg-chunks", type=int, default=0)
     ap.add_argument("--zoh", action="store_true",
                     help="zero-order-hold input term instead of Euler (ssm_scan_*_ex)")
+    ap.add_argument("--fused-sums", action="store_true",
+                    help="real backward with SSM_FUSED_SUMS: dB/dC sums inside the scan kernel "
+                         "(cooperative launches), less DRAM traffic, no reduction launch")
     ap.add_argument("--rtrl", action="store_true",
                     help="complex workloads: time exact structured RTRL (one forward pass that "
                          "accumulates dlambda, domega online) instead of fwd + bwd")
@@ -377,6 +380,7 @@ def real_config(args, w, world):
     c = {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
          "dstate": w.dstate, "chunk": w.chunk, "io": w.io,
          "discretization": "zoh" if args.zoh else "euler",
+         "dbc_sums": "fused into the scan kernel (SSM_FUSED_SUMS)" if args.fused_sums else "reduction kernel",
          "initial_state": bool(args.state), "state": "fp32", "l2": L2_NOTE,
          "parallelism": f"dp{world} (weak: one full batch per rank; dA_log/dD all-reduced)"
                         if world > 1 else "single GPU"}
@@ -887,7 +891,7 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    use_ex = args.zoh or args.state
+    use_ex = args.zoh or args.state or args.fused_sums
     h0 = dhL = hL = None
     if args.state:
         g = torch.Generator(device="cpu").manual_seed(1234 + rank)
@@ -930,7 +934,8 @@ def main():
         if use_ex:
             S.ssm_scan_bwd_ex(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"],
                               ckpt, d["dy"], zoh=args.zoh, h0=h0, dhL=dhL, chunk=w.chunk,
-                              seg_chunks=args.seg_chunks, out=out, ws=wsb, stream=stream)
+                              seg_chunks=args.seg_chunks, out=out, ws=wsb, stream=stream,
+                              fused_sums=args.fused_sums)
         else:
             S.ssm_scan_bwd(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"], ckpt,
                            d["dy"], chunk=w.chunk, seg_chunks=args.seg_chunks, out=out, ws=wsb,
@@ -990,7 +995,8 @@ def main():
             S.ssm_scan_bwd_ex(bs["d"]["x"], bs["d"]["delta_raw"], bs["d"]["A_log"], bs["d"]["Bm"],
                               bs["d"]["Cm"], bs["d"]["Dskip"], bs["ckpt"], bs["d"]["dy"],
                               zoh=args.zoh, h0=h0, dhL=dhL, chunk=w.chunk,
-                              seg_chunks=args.seg_chunks, out=bs["out"], ws=wsb, stream=stream)
+                              seg_chunks=args.seg_chunks, out=bs["out"], ws=wsb, stream=stream,
+                              fused_sums=args.fused_sums)
         else:
             S.ssm_scan_fwd(bs["d"]["x"], bs["d"]["delta_raw"], bs["d"]["A_log"], bs["d"]["Bm"],
                            bs["d"]["Cm"], bs["d"]["Dskip"], chunk=w.chunk,
@@ -1010,8 +1016,9 @@ def main():
     value = world * upd_rank * args.steps / t_step
     hbm, peak_kind = peaks()
     fb, bb = algorithmic_bytes(w)
-    launches = (S.kernel_launches(shape, False) + S.kernel_launches(shape, True) +
-                (4 if R else 0)) * args.steps
+    # the projection: forward + (du and dw in one launch for R <= 64, else two) + dw reduction
+    launches = (S.kernel_launches(shape, False) + S.kernel_launches(shape, True, args.fused_sums) +
+                ((3 if R <= 64 else 4) if R else 0)) * args.steps
     bwd_gbs = bb / (t_bwd / args.steps) / 1e9
     fwd_gbs = fb / (t_fwd / args.steps) / 1e9
     step_gbs = (fb + bb) / ((t_fwd + t_bwd) / args.steps) / 1e9
@@ -1037,7 +1044,8 @@ def main():
                                       f"{alu_mhz:.0f} MHz (FMA = 1 op)",
                          "algorithmic_ops_per_launch": bo,
                          "algorithmic_bytes_per_launch": bb,
-                         "traffic": measured_traffic("ssm_scan_bwd", "real_bwd.cu", w.name),
+                         "traffic": measured_traffic("ssm_scan_bwd (SSM_FUSED_SUMS)" if args.fused_sums
+                                                     else "ssm_scan_bwd", "real_bwd.cu", w.name),
                          **clock_roofs(clk, bwd_tops, upd_rank / (t_bwd / args.steps),
                                        BWD_EXP2_PER_UPDATE)},
             "hbm": {"achieved_bwd": bwd_gbs, "achieved_fwd": fwd_gbs, "achieved_step": step_gbs,

@@ -54,7 +54,7 @@ struct RealPlan {
     int b_nseg, b_seg_chunks, b_seq, b_group, b_rows, b_launches;
     // workspace offsets (bytes); fwd and bwd use separate layouts
     size_t f_sumP, f_sumS, f_hin, f_end;
-    size_t b_gP, b_gG, b_part, b_dA, b_dD, b_bnd, b_end;
+    size_t b_gP, b_gG, b_part, b_dA, b_dD, b_bnd, b_cnt, b_end;
     int b_nslot;  // backward scratch slots: CTAs per launch, at most the resident CTAs
 };
 
@@ -163,6 +163,7 @@ int plan_real(const ssm_shape* s, RealPlan* p) {
     const int64_t ctas = (int64_t)p->ndt * p->B * per;
     p->b_nslot = (int)(ctas < kRealBwdSlots ? (ctas > 0 ? ctas : 1) : kRealBwdSlots);
     p->b_bnd = o;  o = align256(o + (size_t)p->b_nslot * ssm::real_bwd_scratch_floats(p->N, p->T) * 4);
+    p->b_cnt = o;  o = align256(o + BS * B * 4);  // chunks finished per (segment, batch row)
     p->b_end = o;
     return SSM_OK;
 }
@@ -234,7 +235,7 @@ int check_arrays(const void* const* ptrs, const size_t* counts, int n) {
 }
 
 int check_options(const ssm_scan_options& o) {
-    if (o.reserved != 0) return SSM_ERR_INVALID_ARG;
+    if ((o.flags & ~SSM_FUSED_SUMS) != 0) return SSM_ERR_INVALID_ARG;
     if (o.discretization != SSM_EULER && o.discretization != SSM_ZOH) return SSM_ERR_INVALID_ARG;
     return SSM_OK;
 }
@@ -330,8 +331,11 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const 
     if ((st = check_arrays(ptrs, counts, 18)) != SSM_OK) return st;
     if (ws_bytes < p.b_end) return SSM_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // status word and scratch-slot mask
+    // status word and scratch-slot mask; the chunk counters of the fused dB/dC sums when asked for
     if (cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) return SSM_ERR_CUDA;
+    if ((o.flags & SSM_FUSED_SUMS) && p.B > 0 && p.L > 0 &&
+        cudaMemsetAsync(at<unsigned char>(ws, p.b_cnt), 0, (size_t)p.b_nseg * p.B * 4, s) != cudaSuccess)
+        return SSM_ERR_CUDA;
     if (p.B == 0 || p.L == 0) {
         if (cudaMemsetAsync(dA_log, 0, DN * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
         if (cudaMemsetAsync(dD, 0, (size_t)p.D * sizeof(float), s) != cudaSuccess) return SSM_ERR_CUDA;
@@ -349,6 +353,8 @@ int ssm_scan_bwd_ex(const ssm_shape* shape, const ssm_scan_options* opts, const 
     a.bnd_scratch = at<float>(ws, p.b_bnd);
     a.slot_mask = at<unsigned>(ws, kSlotMaskOffset);
     a.nslot = p.b_nslot;
+    a.grp_cnt = at<unsigned>(ws, p.b_cnt);
+    a.fused_sums = (o.flags & SSM_FUSED_SUMS) != 0;
     a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
     a.status = at<unsigned>(ws, 0);
     a.h0 = o.h0; a.dhL = o.dhL; a.dh0 = o.dh0; a.zoh = o.discretization == SSM_ZOH;
@@ -370,8 +376,18 @@ int ssm_scan_kernel_launches(const ssm_shape* shape, int backward) {
     if (plan_real(shape, &p) != SSM_OK) return -1;
     if (p.B == 0 || p.L == 0) return 0;
     if (!backward) return p.nseg > 1 ? 3 : 1;  // [segment summary + carry] + scan
-    // [summary + carry] + per launch (main + dB/dC reduce) + dA_log/dD reduce
-    return (p.b_nseg > 1 && !p.b_seq ? 2 : 0) + 2 * p.b_launches + 1;
+    // [summary + carry] + per launch (main + dB/dC reduce) + dA_log/dD reduce; with
+    // SSM_FUSED_SUMS (backward == 2) no reduce for a launch whose CTAs are all resident at once
+    // on 148 SMs (3 per SM, 4 for the N = 16 instance)
+    int n = (p.b_nseg > 1 && !p.b_seq ? 2 : 0) + 1;
+    const int per = p.b_seq ? 1 : p.b_group;
+    for (int hi = p.b_nseg; hi > 0; hi -= per) {
+        const int segs = hi - per > 0 ? per : hi;
+        const int64_t ctas = (int64_t)p.ndt * p.B * segs;
+        const int64_t resident = p.N == 16 ? kRealBwdSlots : 444;
+        n += (backward == 2 && ctas <= p.b_nslot && ctas <= resident) ? 1 : 2;
+    }
+    return n;
 }
 
 int ssm_scan_complex_kernel_launches(const ssm_cshape* shape, int backward) {

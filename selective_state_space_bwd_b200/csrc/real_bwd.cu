@@ -243,7 +243,93 @@ __device__ int claim_slot(unsigned* mask, int nslot, int start) {
 // MINB: CTAs per SM the register allocation must allow.  4 (126 registers for the Euler N = 16
 // kernel) lets grids of up to 592 CTAs run in one wave; 3 leaves the compiler more registers,
 // which is faster when the grid fits 3 per SM anyway (zero-order hold always uses 3).
-template <typename E, int N, bool ZOH, int MINB, bool A2A, bool POOL>
+// Fused dB/dC sums (FUSED, launches whose CTAs are all resident: cooperative launches).  The
+// CTAs of one (segment, batch row) walk the same chunks in the same order.  After a chunk's pass B
+// a CTA counts itself finished with that chunk; after the next chunk's pass A (or at its end) it
+// waits until all ndt CTAs of its row have finished the chunk, then sums its share of the
+// chunk's partial rows (rows [rows * dt / ndt, rows * (dt + 1) / ndt)) over the channel tiles
+// into dB / dC: the share's float4 units times P parts of the tiles spread over the threads (about
+// eight tiles each, their loads issued together), the parts added in part order.  With N = 16 a
+// partial row is one 128-byte line; those lines are then dead and are discarded from L2, so that
+// they are never written back.  Kept out of line: the scan kernel's registers stay its own.
+template <typename E, int N>
+__device__ __noinline__ void fused_dbc_share(const float* __restrict__ part, int part_rows, int part_t0,
+                                             int B, int L, int T, int ndt, E* __restrict__ dB,
+                                             E* __restrict__ dC, int b, int chunk, int dt, int tid,
+                                             int nthreads, float4* comb) {
+    constexpr int N2 = 2 * N, U4 = N2 / 4;            // float4 columns of a partial row
+    const int t0 = chunk * T;
+    const int rows = min(T, L - t0);
+    const int r0 = (int)((int64_t)rows * dt / ndt), r1 = (int)((int64_t)rows * (dt + 1) / ndt);
+    const int U = (r1 - r0) * U4;                      // float4 units of the share
+    const size_t stride = (size_t)B * part_rows * N2;  // between channel tiles' partials
+    const float* base = part + ((size_t)b * part_rows + (t0 - part_t0) + r0) * N2;
+    for (int ub = 0; ub < U; ub += nthreads) {
+        const int nu = min(nthreads, U - ub);
+        const int P = nthreads / nu;                   // parts of the tiles
+        const int tp = (ndt + P - 1) / P;
+        const int unit = tid % nu, pq = tid / nu;
+        const int u = ub + unit;
+        if (pq < P) {
+            float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const float* src = base + (size_t)(u / U4) * N2 + (u % U4) * 4;
+            const int j0 = min(ndt, pq * tp), j1 = min(ndt, j0 + tp);
+            int j = j0;
+            for (; j + 8 <= j1; j += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)(j + k) * stride));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    s.x += v[k].x;
+                    s.y += v[k].y;
+                    s.z += v[k].z;
+                    s.w += v[k].w;
+                }
+            }
+            for (; j < j1; ++j) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)j * stride));
+                s.x += v.x;
+                s.y += v.y;
+                s.z += v.z;
+                s.w += v.w;
+            }
+            comb[pq * nu + unit] = s;
+        }
+        __syncthreads();
+        if (pq == 0) {
+            float4 t = comb[unit];
+            for (int w = 1; w < P; ++w) {
+                const float4 v = comb[w * nu + unit];
+                t.x += v.x;
+                t.y += v.y;
+                t.z += v.z;
+                t.w += v.w;
+            }
+            const float o[4] = {t.x, t.y, t.z, t.w};
+            const int r = r0 + u / U4, e = (u % U4) * 4;
+            const size_t bl = (size_t)b * L + t0 + r;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (e + k < N)
+                    dB[bl * N + e + k] = Elem<E>::from_f(o[k]);
+                else
+                    dC[bl * N + (e + k - N)] = Elem<E>::from_f(o[k]);
+            }
+        }
+        __syncthreads();
+    }
+    if constexpr (N2 * 4 == 128) {
+        // every tile's partial rows of the share, one line each, are dead: drop them unwritten
+        for (int i = tid; i < (r1 - r0) * ndt; i += nthreads) {
+            const int jt = i / (r1 - r0), r = i % (r1 - r0);
+            const float* a = base + (size_t)jt * stride + (size_t)r * N2;
+            asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(a) : "memory");
+        }
+    }
+}
+
+template <typename E, int N, bool ZOH, int MINB, bool A2A, bool POOL, bool FUSED>
 __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs p) {
     using Cfg = BwdCfg<N>;
     using Sm = BwdSmem<E, N, A2A>;
@@ -331,6 +417,31 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
     float2* dsg = reinterpret_cast<float2*>(scr + (size_t)(T / W) * NT * 4);  // (delta, sigma) [T][DT]
     const int roff = rot * N + n0;  // this thread's slots within a staged row of ROT * N floats
 
+    // fused dB/dC sums: the chunk whose sums are pending and this CTA's finished-chunk count
+    static_assert(!FUSED || 2 * Sm::RED * 4 >= NT * 16, "the warps' part sums fit the window-sum buffer");
+    int pend = -1, nfin = 0;
+    unsigned* gcnt = FUSED ? p.grp_cnt + (size_t)seg * p.B + b : nullptr;
+    auto sum_pending = [&]() {
+        if constexpr (FUSED) {
+            __shared__ int s_ok;
+            if (tid == 0) {
+                const unsigned target = (unsigned)nfin * (unsigned)p.ndt;
+                unsigned it = 0;
+                while (*reinterpret_cast<volatile unsigned*>(gcnt) < target && ++it < kSlotSpinLimit)
+                    __nanosleep(128);
+                s_ok = it < kSlotSpinLimit;
+                __threadfence();  // the other CTAs' partial rows come first
+                if (!s_ok) flag_status(p.status, kStatusTimeout);
+            }
+            __syncthreads();
+            if (s_ok)
+                fused_dbc_share<E, N>(p.dBC_part, p.part_rows, p.part_t0, p.B, p.L, p.T, p.ndt,
+                                      static_cast<E*>(p.dB), static_cast<E*>(p.dC), b, pend,
+                                      (int)blockIdx.x, tid, NT, reinterpret_cast<float4*>(smem + Sm::B_RED));
+            pend = -1;
+        }
+    };
+
     for (int c = c_end - 1; c >= c_begin; --c) {
         const int tc = c * T;
         const int rows_c = min(T, p.L - tc);
@@ -405,6 +516,10 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                     }
                 }
             }
+        }
+
+        if constexpr (FUSED) {
+            if (pend >= 0) sum_pending();  // the previous chunk's sums, behind this pass A
         }
 
         // ------------------------------------------------------------------ pass B
@@ -633,6 +748,18 @@ __global__ void __launch_bounds__(BwdCfg<N>::NT, MINB) real_bwd_kernel(RealArgs 
                 if (j > 0) ld_pairs_cg<4>(hw, bnd + (size_t)(wbase - 1) * NT * 4);
             }
         }
+        if constexpr (FUSED) {
+            __syncthreads();  // every partial row of chunk c is written
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(gcnt, 1u);
+            }
+            pend = c;
+            ++nfin;
+        }
+    }
+    if constexpr (FUSED) {
+        if (pend >= 0) sum_pending();
     }
     // each lane of a channel accumulated dD over its own subset of steps
 #pragma unroll
@@ -727,13 +854,30 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // at most three CTAs per SM: the all-to-all instance; four: the reduce-scatter instance, whose
-    // registers and shared memory fit four
+    // registers and shared memory fit four.  Instances: plain, claiming scratch slots (POOL, more
+    // CTAs than slots), and with the fused dB/dC sums (FUSED, every CTA resident: cooperative)
     const size_t sm3 = BwdSmem<E, N, true>::BYTES, sm4 = BwdSmem<E, N, false>::BYTES;
-    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true, false>, sm3)) != cudaSuccess) return e;
-    if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 3, true, true>, sm3)) != cudaSuccess) return e;
+    auto k3 = real_bwd_kernel<E, N, ZOH, 3, true, false, false>;
+    auto k3p = real_bwd_kernel<E, N, ZOH, 3, true, true, false>;
+    auto k3f = real_bwd_kernel<E, N, ZOH, 3, true, false, true>;
+    if ((e = set_smem(k3, sm3)) != cudaSuccess || (e = set_smem(k3p, sm3)) != cudaSuccess ||
+        (e = set_smem(k3f, sm3)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0, coop = 0, res3 = 0, res4 = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&res3, k3f, BwdCfg<N>::NT, sm3)) != cudaSuccess)
+        return e;
     if constexpr (N == 16) {
-        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false, false>, sm4)) != cudaSuccess) return e;
-        if ((e = set_smem(real_bwd_kernel<E, N, ZOH, 4, false, true>, sm4)) != cudaSuccess) return e;
+        auto k4 = real_bwd_kernel<E, N, ZOH, 4, false, false, false>;
+        auto k4p = real_bwd_kernel<E, N, ZOH, 4, false, true, false>;
+        auto k4f = real_bwd_kernel<E, N, ZOH, 4, false, false, true>;
+        if ((e = set_smem(k4, sm4)) != cudaSuccess || (e = set_smem(k4p, sm4)) != cudaSuccess ||
+            (e = set_smem(k4f, sm4)) != cudaSuccess)
+            return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&res4, k4f, BwdCfg<N>::NT, sm4)) != cudaSuccess)
+            return e;
     }
     const int per = a.seq_blocks ? 1 : group;
     for (int hi = a.nseg; hi > 0; hi -= per) {
@@ -747,18 +891,42 @@ cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
         const bool pool = ctas > a.nslot;  // more CTAs than scratch slots: claim them
         bool wide = false;                 // more CTAs than 3 per SM on 148 SMs
         if constexpr (N == 16) wide = ctas > 444;
+        // asked for, and every CTA resident at once: the dB/dC sums run inside the scan kernel
+        const bool fused = a.fused_sums && coop && !pool && ctas <= (int64_t)sms * (wide ? res4 : res3);
         const dim3 blk(BwdCfg<N>::NT);
+        if (fused) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.gridDim = grid;
+            cfg.blockDim = blk;
+            cfg.stream = st;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (wide) {
+                if constexpr (N == 16) {
+                    cfg.dynamicSmemBytes = sm4;
+                    e = cudaLaunchKernelEx(&cfg, real_bwd_kernel<E, N, ZOH, 4, false, false, true>, a);
+                }
+            } else {
+                cfg.dynamicSmemBytes = sm3;
+                e = cudaLaunchKernelEx(&cfg, k3f, a);
+            }
+            if (e != cudaSuccess) return e;
+            continue;  // dB and dC are written: no reduction launch
+        }
         if (wide) {
             if constexpr (N == 16) {
                 if (pool)
-                    real_bwd_kernel<E, N, ZOH, 4, false, true><<<grid, blk, sm4, st>>>(a);
+                    real_bwd_kernel<E, N, ZOH, 4, false, true, false><<<grid, blk, sm4, st>>>(a);
                 else
-                    real_bwd_kernel<E, N, ZOH, 4, false, false><<<grid, blk, sm4, st>>>(a);
+                    real_bwd_kernel<E, N, ZOH, 4, false, false, false><<<grid, blk, sm4, st>>>(a);
             }
         } else if (pool) {
-            real_bwd_kernel<E, N, ZOH, 3, true, true><<<grid, blk, sm3, st>>>(a);
+            k3p<<<grid, blk, sm3, st>>>(a);
         } else {
-            real_bwd_kernel<E, N, ZOH, 3, true, false><<<grid, blk, sm3, st>>>(a);
+            k3<<<grid, blk, sm3, st>>>(a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t nbc = (int64_t)a.B * rows * 2 * N;

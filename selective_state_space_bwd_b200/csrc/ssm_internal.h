@@ -53,6 +53,9 @@ struct RealArgs {
                          // each held by one resident CTA at a time
     unsigned* slot_mask; // bit i set while slot i is held; zero when a launch starts and ends
     int nslot;
+    unsigned* grp_cnt;   // backward, fused dB/dC sums: chunks finished per (segment, batch row)
+                         // [nseg][B], zero when the call starts
+    int fused_sums;      // backward: SSM_FUSED_SUMS asked for
     int seg0;         // backward: first segment handled by this launch (blockIdx.z offset)
     int seq_blocks;   // backward: segments run as sequential launches, each handing its
                       // entering adjoint to the next through vin

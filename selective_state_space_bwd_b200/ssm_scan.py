@@ -37,10 +37,11 @@ class SsmCShape(ctypes.Structure):
 
 
 SSM_EULER, SSM_ZOH = 0, 1
+SSM_FUSED_SUMS = 1  # ssm_scan_options.flags: dB/dC sums inside the backward's scan kernel
 
 
 class SsmOptions(ctypes.Structure):
-    _fields_ = [("discretization", ctypes.c_int32), ("reserved", ctypes.c_int32),
+    _fields_ = [("discretization", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("h0", ctypes.c_void_p), ("hL", ctypes.c_void_p), ("dhL", ctypes.c_void_p),
                 ("dh0", ctypes.c_void_p)]
 
@@ -179,8 +180,9 @@ def complex_workspace_bytes(shape: SsmCShape, backward: bool) -> int:
     return int(lib().ssm_scan_complex_workspace_bytes(ctypes.byref(shape), int(bool(backward))))
 
 
-def kernel_launches(shape: SsmShape, backward: bool) -> int:
-    return int(lib().ssm_scan_kernel_launches(ctypes.byref(shape), int(bool(backward))))
+def kernel_launches(shape: SsmShape, backward: bool, fused_sums: bool = False) -> int:
+    mode = (2 if fused_sums else 1) if backward else 0
+    return int(lib().ssm_scan_kernel_launches(ctypes.byref(shape), mode))
 
 
 def complex_checkpoint_bytes(shape: SsmCShape) -> int:
@@ -265,11 +267,12 @@ def ssm_scan_bwd(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, chunk=128, seg_ch
     return out
 
 
-def _options(zoh, h0=None, hL=None, dhL=None, dh0=None):
+def _options(zoh, h0=None, hL=None, dhL=None, dh0=None, fused_sums=False):
     for t in (h0, hL, dhL, dh0):
         if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
             raise ValueError("h0, hL, dhL, dh0 must be contiguous float32 [B, D, N]")
-    return SsmOptions(SSM_ZOH if zoh else SSM_EULER, 0, None if h0 is None else h0.data_ptr(),
+    return SsmOptions(SSM_ZOH if zoh else SSM_EULER, SSM_FUSED_SUMS if fused_sums else 0,
+                      None if h0 is None else h0.data_ptr(),
                       None if hL is None else hL.data_ptr(), None if dhL is None else dhL.data_ptr(),
                       None if dh0 is None else dh0.data_ptr())
 
@@ -299,9 +302,10 @@ def ssm_scan_fwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, zoh=False, h0=None, chun
 
 
 def ssm_scan_bwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, zoh=False, h0=None, dhL=None,
-                    chunk=128, seg_chunks=0, out=None, ws=None, stream=None):
+                    chunk=128, seg_chunks=0, out=None, ws=None, stream=None, fused_sums=False):
     """Backward with options: the gradient of sum(dy y) + sum(dhL hL).  Returns the dict of
-    ssm_scan_bwd plus dh0 [B,D,N] (the gradient with respect to h0)."""
+    ssm_scan_bwd plus dh0 [B,D,N] (the gradient with respect to h0).  ``fused_sums`` sets
+    SSM_FUSED_SUMS (dB/dC sums inside the scan kernel where its CTAs can all be resident)."""
     _need_cuda(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, h0, dhL)
     B, L, D = x.shape
     N = A_log.shape[1]
@@ -312,7 +316,7 @@ def ssm_scan_bwd_ex(x, delta_raw, A_log, Bm, Cm, Dskip, ckpt, dy, zoh=False, h0=
                    dD=torch.empty_like(Dskip))
     if out.get("dh0") is None:
         out["dh0"] = torch.empty((B, D, N), dtype=torch.float32, device=x.device)
-    opts = _options(zoh, h0=h0, dhL=dhL, dh0=out["dh0"])
+    opts = _options(zoh, h0=h0, dhL=dhL, dh0=out["dh0"], fused_sums=fused_sums)
     ws = _workspace(workspace_bytes(shape, True), x.device, ws)
     code = lib().ssm_scan_bwd_ex(ctypes.byref(shape), ctypes.byref(opts), _p(x), _p(delta_raw),
                                  _p(A_log), _p(Bm), _p(Cm), _p(Dskip), _p(ckpt), _p(dy),

@@ -44,7 +44,7 @@ def test_exports_every_declared_symbol(S):
 
 def test_abi_version_and_status_strings(S):
     L = S.lib()
-    assert L.ssm_scan_abi_version() == 4
+    assert L.ssm_scan_abi_version() == 5
     for code in range(8):
         assert L.ssm_status_string(code).decode().startswith(S.STATUS_NAMES[code])
     assert L.ssm_status_string(99) == b"unknown ssm_status"
@@ -134,7 +134,7 @@ def test_null_misaligned_and_small_workspace(S):
 
 
 def test_option_validation(S):
-    """The option-taking calls reject an unknown discretization, a non-zero reserved field and a
+    """The option-taking calls reject an unknown discretization, an unknown flag and a
     misaligned state pointer before anything is enqueued; NULL options equal the plain calls'
     validation."""
     L = S.lib()
@@ -142,14 +142,18 @@ def test_option_validation(S):
     need, needb = S.workspace_bytes(shp, False), S.workspace_bytes(shp, True)
     p, pb = _fake_ptrs(9), _fake_ptrs(15)
     bad_disc = S.SsmOptions(2, 0, None, None, None, None)
-    bad_res = S.SsmOptions(S.SSM_ZOH, 7, None, None, None, None)
+    bad_res = S.SsmOptions(S.SSM_ZOH, 7, None, None, None, None)     # bits beyond SSM_FUSED_SUMS
+    bad_flag = S.SsmOptions(S.SSM_EULER, 2, None, None, None, None)
     mis_h0 = S.SsmOptions(S.SSM_EULER, 0, 0x100004, None, None, None)
     mis_dh0 = S.SsmOptions(S.SSM_ZOH, 0, None, None, None, 0x100008)
-    for o in (bad_disc, bad_res):
+    for o in (bad_disc, bad_res, bad_flag):
         assert L.ssm_scan_fwd_ex(ctypes.byref(shp), ctypes.byref(o), *p, need, None) == 1
         assert L.ssm_scan_bwd_ex(ctypes.byref(shp), ctypes.byref(o), *pb, needb, None) == 1
     assert L.ssm_scan_fwd_ex(ctypes.byref(shp), ctypes.byref(mis_h0), *p, need, None) == 3
     assert L.ssm_scan_bwd_ex(ctypes.byref(shp), ctypes.byref(mis_dh0), *pb, needb, None) == 3
+    # SSM_FUSED_SUMS is a valid flag: the call gets as far as the workspace check
+    fused = S.SsmOptions(S.SSM_EULER, S.SSM_FUSED_SUMS, None, None, None, None)
+    assert L.ssm_scan_bwd_ex(ctypes.byref(shp), ctypes.byref(fused), *pb, needb - 256, None) == 4
     # NULL options: same checks as the plain calls (here: workspace too small)
     assert L.ssm_scan_fwd_ex(ctypes.byref(shp), None, *p, need - 1, None) == 4
     assert L.ssm_scan_bwd_ex(ctypes.byref(shp), None, *pb, needb - 256, None) == 4
@@ -261,6 +265,8 @@ def test_status_null_workspace(S):
 def test_kernel_launch_counts(S):
     one = S.real_shape(8, 2048, 1536, 16, 128, S.SSM_BF16)        # enough CTAs: no time split
     assert S.kernel_launches(one, False) == 1 and S.kernel_launches(one, True) == 3
+    # with SSM_FUSED_SUMS its 384 CTAs are all resident: the scan kernel adds the dB/dC sums
+    assert S.kernel_launches(one, True, fused_sums=True) == 2
     # few CTAs: concurrent segments + carry; the backward uses 250 segments of 4 chunks, 63 per
     # launch (2016 CTAs) so that each launch's dB/dC partial sums stay under their cap:
     # summary + carry + 4 x (main + reduce) + params = 11
@@ -270,11 +276,13 @@ def test_kernel_launch_counts(S):
     # resident ones, so the scratch is 592 slots that CTAs claim (58.2 MB, not 125.8 MB)
     multi = S.real_shape(2, 20000, 1024, 16, 128, S.SSM_F32)
     assert S.kernel_launches(multi, True) == 7
+    assert S.kernel_launches(multi, True, fused_sums=True) == 7   # not resident: unchanged
     assert S.workspace_bytes(multi, True) - 592 * 98304 < 95_000_000
     # 512 CTAs fit one wave (4 CTAs per SM on 148 SMs = 592 slots): no time split, time in 4
     # sequential blocks under the partial cap
     wave = S.real_shape(4, 8192, 4096, 16, 128, S.SSM_BF16)
     assert S.kernel_launches(wave, False) == 1 and S.kernel_launches(wave, True) == 9
+    assert S.kernel_launches(wave, True, fused_sums=True) == 5
     # 640 CTAs would leave a second wave of 48 on 592 slots: 16 concurrent segments of 4 chunks
     # instead, 3 per launch (summary + carry + 6 x (main + reduce) + params)
     part = S.real_shape(5, 8192, 4096, 16, 128, S.SSM_BF16)

@@ -25,7 +25,10 @@ def _dev(inp):
             for k, v in inp.items()}
 
 
-def test_captured_fwd_bwd_replays_bitwise(S):
+@pytest.mark.parametrize("fused", [False, True])
+def test_captured_fwd_bwd_replays_bitwise(S, fused):
+    """fused: the backward with SSM_FUSED_SUMS (cooperative launches and the chunk counters'
+    memset in the graph)."""
     B, L, D, N, T = 2, 1000, 128, 16, 128
     a = _dev(gen.real_inputs(B, L, D, N, gen.BF16, "mamba", seed=1))
     shape = S.real_shape(B, L, D, N, T, S.SSM_BF16)
@@ -40,8 +43,12 @@ def test_captured_fwd_bwd_replays_bitwise(S):
     def step():
         S.ssm_scan_fwd(a["x"], a["delta_raw"], a["A_log"], a["Bm"], a["Cm"], a["Dskip"], chunk=T,
                        y=y, ckpt=ck, ws=wsf)
-        S.ssm_scan_bwd(a["x"], a["delta_raw"], a["A_log"], a["Bm"], a["Cm"], a["Dskip"], ck, a["dy"],
-                       chunk=T, out=out, ws=wsb)
+        if fused:
+            S.ssm_scan_bwd_ex(a["x"], a["delta_raw"], a["A_log"], a["Bm"], a["Cm"], a["Dskip"], ck,
+                              a["dy"], chunk=T, out=out, ws=wsb, fused_sums=True)
+        else:
+            S.ssm_scan_bwd(a["x"], a["delta_raw"], a["A_log"], a["Bm"], a["Cm"], a["Dskip"], ck,
+                           a["dy"], chunk=T, out=out, ws=wsb)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -59,12 +66,17 @@ def test_captured_fwd_bwd_replays_bitwise(S):
     torch.cuda.synchronize()
     got = {"y": y.clone(), **{k: v.clone() for k, v in out.items()}}
     y2, ck2 = S.ssm_scan_fwd(b["x"], b["delta_raw"], b["A_log"], b["Bm"], b["Cm"], b["Dskip"], chunk=T)
-    ref = S.ssm_scan_bwd(b["x"], b["delta_raw"], b["A_log"], b["Bm"], b["Cm"], b["Dskip"], ck2, b["dy"],
-                         chunk=T)
+    if fused:
+        ref = S.ssm_scan_bwd_ex(b["x"], b["delta_raw"], b["A_log"], b["Bm"], b["Cm"], b["Dskip"], ck2,
+                                b["dy"], chunk=T, fused_sums=True)
+    else:
+        ref = S.ssm_scan_bwd(b["x"], b["delta_raw"], b["A_log"], b["Bm"], b["Cm"], b["Dskip"], ck2,
+                             b["dy"], chunk=T)
     torch.cuda.synchronize()
     assert torch.equal(got["y"], y2)
     for k, v in ref.items():
-        assert torch.equal(got[k], v), k
+        if k in out:
+            assert torch.equal(got[k], v), k
     assert S.ssm_scan_status(wsb) == 0
 
 

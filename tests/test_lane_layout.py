@@ -10,6 +10,7 @@ of a group cover the group's four states, and that the shared-memory layout of t
 is free of bank conflicts on both the writes and the reads.
 """
 
+import itertools
 import numpy as np
 import pytest
 
@@ -75,3 +76,36 @@ def test_window_sums_layout_is_conflict_free(N):
         # the readers: thread tid sums red[g * RS + tid] over the groups
         for g in range(GRP):
             assert banks([g * RS + warp * 32 + lane for lane in range(32)]) == 1
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_fused_dbc_share_partition(N):
+    """Model of the backward's fused dB/dC sums (fused_dbc_share in real_bwd.cu): channel tile dt
+    of a batch row sums rows [rows*dt/ndt, rows*(dt+1)/ndt) of a chunk; the share's float4 units
+    times P = threads / units parts of the tiles spread over the CTA's threads.  Every output of
+    the chunk is written exactly once, and every tile's partial of it is read exactly once."""
+    N2, U4 = 2 * N, 2 * N // 4
+    NT = 32 * N // 4
+    for ndt, rows in itertools.product((1, 3, 32, 48, 128), (1, 5, 16, 127, 128)):
+        written, reads = {}, {}
+        for dt in range(ndt):
+            r0, r1 = rows * dt // ndt, rows * (dt + 1) // ndt
+            U = (r1 - r0) * U4
+            for ub in range(0, U, NT):
+                nu = min(NT, U - ub)
+                P = NT // nu
+                tp = (ndt + P - 1) // P
+                for tid in range(NT):
+                    unit, pq = tid % nu, tid // nu
+                    u = ub + unit
+                    if pq < P:
+                        j0 = min(ndt, pq * tp)
+                        for j in range(j0, min(ndt, j0 + tp)):
+                            key = (j, r0 + u // U4, (u % U4) * 4)
+                            reads[key] = reads.get(key, 0) + 1
+                    if pq == 0:
+                        for k in range(4):
+                            o = (r0 + u // U4, (u % U4) * 4 + k)
+                            written[o] = written.get(o, 0) + 1
+        assert written == {(r, e): 1 for r in range(rows) for e in range(N2)}
+        assert reads == {(j, r, e): 1 for j in range(ndt) for r in range(rows) for e in range(0, N2, 4)}

@@ -160,3 +160,44 @@ def test_empty_sequence_passes_the_state_through(S):
     np.testing.assert_array_equal(got["hL"], inp["h0"])
     np.testing.assert_array_equal(got["dh0"], inp["dhL"])
     assert not got["dA_log"].any() and not got["dD"].any()
+
+
+FUSED_CASES = [
+    # B, L, D, N, T, io, kind, seg_chunks: backward launches whose CTAs all fit at once
+    (2, 300, 64, 16, 64, gen.F32, "mamba", 0),
+    (2, 300, 64, 16, 64, gen.F32, "mamba", 2),     # time segments (summary + carry)
+    (3, 517, 72, 8, 32, gen.F32, "stiff", 0),
+    (2, 129, 136, 4, 16, gen.BF16, "mamba", 0),
+    (4, 700, 1024, 16, 128, gen.BF16, "mamba", 0),  # 128 CTAs, 6 chunks
+    (15, 200, 1024, 16, 64, gen.F32, "stiff", 0),  # 480 CTAs: the four-CTA-per-SM instance
+]
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("B,L,D,N,T,io,kind,seg", FUSED_CASES)
+def test_fused_sums_parity(S, oracle_mod, zoh, B, L, D, N, T, io, kind, seg):
+    """SSM_FUSED_SUMS: dB and dC summed inside the scan kernel (cooperative launches) against the
+    oracle; the other gradients bitwise equal to the call without the flag; the status clean; a
+    second call bitwise equal (a fixed order of the channel tiles)."""
+    inp = _inputs(B, L, D, N, io, kind, seed=B * 7 + L + N)
+    d = _dev(inp, io)
+    y, ckpt, hL = S.ssm_scan_fwd_ex(d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"],
+                                    d["Dskip"], zoh=zoh, h0=d["h0"], chunk=T, seg_chunks=seg)
+    args = (d["x"], d["delta_raw"], d["A_log"], d["Bm"], d["Cm"], d["Dskip"], ckpt, d["dy"])
+    shape = S.real_shape(B, L, D, N, T, S._io_of(d["x"]), seg)
+    ws = torch.empty(S.workspace_bytes(shape, True), dtype=torch.uint8, device="cuda")
+    g1 = S.ssm_scan_bwd_ex(*args, zoh=zoh, h0=d["h0"], dhL=d["dhL"], chunk=T, seg_chunks=seg,
+                           ws=ws, fused_sums=True)
+    g1 = {k: v.clone() for k, v in g1.items()}
+    assert S.ssm_scan_status(ws) == 0
+    g2 = S.ssm_scan_bwd_ex(*args, zoh=zoh, h0=d["h0"], dhL=d["dhL"], chunk=T, seg_chunks=seg,
+                           ws=ws, fused_sums=True)
+    plain = S.ssm_scan_bwd_ex(*args, zoh=zoh, h0=d["h0"], dhL=d["dhL"], chunk=T, seg_chunks=seg)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+        if k not in ("dB", "dC"):
+            assert torch.equal(g1[k], plain[k]), k
+    got = {"y": _np(y), "ckpt": _np(ckpt), "hL": _np(hL)}
+    got.update({k: _np(v) for k, v in g1.items()})
+    check(got, run_oracle(oracle_mod, inp, zoh, T), io)

@@ -118,6 +118,10 @@ REAL_CASES = [
     (1, 127, 32, 16, 128, gen.F32, 0),
     (1, 129, 32, 16, 128, gen.F32, 1),
     (4, 2048, 96, 16, 128, gen.BF16, 0),
+    # 512 CTAs of N = 8: more than the 444 the three-CTA-per-SM instance holds at once, so the
+    # backward runs as a plain launch followed by its dB/dC reduction kernel (the small cases
+    # above run cooperatively, their sums fused into the scan kernel)
+    (16, 150, 1024, 8, 64, gen.F32, 0),
 ]
 
 

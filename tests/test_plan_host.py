@@ -34,8 +34,8 @@ def test_backward_plan_caps_and_launches(S, B, L, D):
     ckpt = S.checkpoint_bytes(shp)
     cap = max(ckpt, 128 << 20)
     bw = S.workspace_bytes(shp, True)
-    # capped dB/dC partial sums + capped per-CTA scratch (192 MiB) + segment summaries (at most
-    # the checkpoints) + small per-(batch, segment) sums
+    # capped dB/dC partial sums + scratch slots (592 x 96 KB at most) + segment summaries (at
+    # most the checkpoints) + small per-(batch, segment) sums
     assert bw <= 2 * cap + (193 << 20)
     nf, nb = S.kernel_launches(shp, False), S.kernel_launches(shp, True)
     # forward: one scan launch, or summary + carry + scan when split in time
