@@ -1044,8 +1044,11 @@ def main():
                                       f"{alu_mhz:.0f} MHz (FMA = 1 op)",
                          "algorithmic_ops_per_launch": bo,
                          "algorithmic_bytes_per_launch": bb,
-                         "traffic": measured_traffic("ssm_scan_bwd (SSM_FUSED_SUMS)" if args.fused_sums
-                                                     else "ssm_scan_bwd", "real_bwd.cu", w.name),
+                         # records exist for the Euler path without options (and with the fused
+                         # sums); zero-order hold and an initial state run other instances
+                         "traffic": (None if args.zoh or args.state else
+                                     measured_traffic("ssm_scan_bwd (SSM_FUSED_SUMS)" if args.fused_sums
+                                                      else "ssm_scan_bwd", "real_bwd.cu", w.name)),
                          **clock_roofs(clk, bwd_tops, upd_rank / (t_bwd / args.steps),
                                        BWD_EXP2_PER_UPDATE)},
             "hbm": {"achieved_bwd": bwd_gbs, "achieved_fwd": fwd_gbs, "achieved_step": step_gbs,
