@@ -30,14 +30,30 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source whose object is stale to an object, in parallel (one nvcc process
+    each; no device code crosses files), then link the shared library."""
     if not force and up_to_date():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
+    obj_dir = os.path.join(HERE, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+             "-I", os.path.join(ROOT, "include")]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+        flags.append("-Xptxas=-v")
+    objs = [os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o") for src in sources()]
+    headers = [p for p in deps() if not p.endswith(".cu")]
+
+    def stale(src, obj):
+        return force or not os.path.exists(obj) or any(
+            os.path.getmtime(p) > os.path.getmtime(obj) for p in [src, *headers])
+
+    procs = [subprocess.Popen([nvcc, *flags, "-c", src, "-o", obj])
+             for src, obj in zip(sources(), objs) if stale(src, obj)]
+    failed = [p.args for p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    subprocess.run([nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *objs], check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

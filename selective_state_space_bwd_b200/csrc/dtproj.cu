@@ -84,10 +84,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, unsigned sr
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-// this thread's bulk stores have finished reading shared memory
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-}
 // this thread's bulk stores are complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 // true once the phase of parity `parity` has completed; false if the bounded wait gave up.  The
