@@ -34,7 +34,7 @@ struct FwdCfg {
     static constexpr int DT = kRealDT;    // channels per CTA
     static constexpr int NT = DT * NG;    // threads per CTA
     static constexpr int TT = 32;         // steps per staged sub-tile
-    static constexpr int U = S == 2 ? 8 : 4;  // steps per unrolled group (>= NG)
+    static constexpr int U = 8;           // steps per unrolled group (>= NG)
     static_assert(U >= NG, "one y value per lane at least");
 };
 
