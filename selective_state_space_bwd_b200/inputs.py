@@ -58,6 +58,8 @@ WORKLOADS = {
     "mamba130m_layer": RealWorkload("mamba130m_layer", 8, 2048, 1536, 16, 128, BF16, "mamba"),
     "stiff_impulse": RealWorkload("stiff_impulse", 1, 128000, 1024, 16, 128, F32, "stiff"),
     "mamba1p4b_layer": RealWorkload("mamba1p4b_layer", 4, 8192, 4096, 16, 128, BF16, "mamba"),
+    # a quarter of mamba1p4b_layer along L: the same grids and kernel instances (profiling captures)
+    "mamba1p4b_layer_l2048": RealWorkload("mamba1p4b_layer_l2048", 4, 2048, 4096, 16, 128, BF16, "mamba"),
     "sparc_complex": ComplexWorkload("sparc_complex", 16, 4096, 2048, 128),
     "sparc_complex_b4": ComplexWorkload("sparc_complex_b4", 4, 4096, 2048, 128),
     # a quarter of sparc_complex along L with the same launch plan (profiling captures)
