@@ -12,6 +12,7 @@ Phase Gradient Flow abstract's 128,000-step impulse-response benchmark):
 * ``mamba130m_layer`` B=8, L=2048,   D=1536, N=16, bf16
 * ``stiff_impulse``   B=1, L=128000, D=1024, N=16, fp32 (unit impulse at t=0 plus noise, stiff A)
 * ``mamba1p4b_layer`` B=4, L=8192,   D=4096, N=16, bf16
+* ``mamba1p4b_layer_l2048`` the same with L=2048 (same grids and kernel instances: profiling)
 * ``sparc_complex``   B=16, L=4096,  K=2048 complex modes (SPARC shared retention/phase control)
 * ``sparc_complex_b4`` the same with B=4 (a quarter of the data: profiling captures)
 * ``pdssm_l5120``     Flash PD-SSM scan: B=8, L=5120 (the sequence length of the Flash PD-SSM
