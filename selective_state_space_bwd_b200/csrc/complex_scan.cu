@@ -642,19 +642,18 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_ckpt_kernel(CplxArgs p) {
     const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
     float2* traj = reinterpret_cast<float2*>(p.traj) + cta * (cplx_traj_floats(p.T) / 2);
     const int cs_r = tid >> 2, cs_part = tid & 3;  // column sums: step cs_r, a quarter of the modes
-    auto issue = [&](int i) {
+    // copies of item i: part 1 = its u or g tile, part 2 = its h_{t-1} rows (sweep items); both
+    // parts by default
+    auto issue = [&](int i, int parts = 3) {
         if (i < n) {
             int c, j, nt;
             bool sw;
             item(i, c, sw, j, nt);
             const int st = i % B_USTAGES, t0 = c * p.T + j * FT;
-            if (!sw) {
-                cp_async_tile<float2, KT>(sx[st], ub, t0, FT, p.L, k0, p.K, tid, F_CONS);
-            } else {
-                cp_async_tile<float2, KT>(sx[st], gb, t0, FT, p.L, k0, p.K, tid, F_CONS);
+            if (parts & 1) cp_async_tile<float2, KT>(sx[st], sw ? gb : ub, t0, FT, p.L, k0, p.K, tid, F_CONS);
+            if (sw && (parts & 2))
                 cp_async_tile<float2, KT>(shp[st], traj, j * FT, FT, min(p.T, p.L - c * p.T), 0,
                                           KT, tid, F_CONS);
-            }
         }
         cp_async_commit();
     };
@@ -669,10 +668,10 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_ckpt_kernel(CplxArgs p) {
         const int t0 = c * p.T + j * FT, rows = min(FT, p.L - t0);
         cp_async_wait<0>();
         bar_sync_n(F_BAR_CONS, F_CONS);  // item i's tiles are in; every consumer is past item i-1
-        // the first sweep item of a chunk reads the h_{t-1} that the item before it writes, so its
-        // copies are issued once that item is done
+        // the first sweep item of a chunk reads the h_{t-1} that the item before it writes, so
+        // those rows are copied once that item is done (its g tile right away)
         const bool defer = !sweep && j == nt - 1;
-        if (!defer) issue(i + 1);
+        issue(i + 1, defer ? 1 : 3);
         const float2* sat = sa[buf];
         bar_sync_n(F_BAR_FULL + buf, F_NT);  // the producers have written the item's transitions
         if (!sweep) {
@@ -689,7 +688,7 @@ __global__ void __launch_bounds__(F_NT) cplx_bwd_ckpt_kernel(CplxArgs p) {
             bar_arrive_n(F_BAR_EMPTY + buf, F_NT);  // transitions consumed
             if (defer) {
                 bar_sync_n(F_BAR_CONS, F_CONS);  // the chunk's h_{t-1} are all written
-                issue(i + 1);
+                issue(i + 1, 2);
             }
             continue;
         }
