@@ -13,7 +13,7 @@
 // time segment through shared memory in 32-step sub-tiles: while sub-tile j is processed, the
 // raw inputs of sub-tile j+1 arrive by asynchronous copies (two-stage ring), so no warp waits on
 // global memory.  Per sub-tile: softplus once per (t, d) into a (delta, delta*x) tile, B and C to
-// fp32, then the sequential scan in groups of 4 steps; the per-channel sums of y over the NG
+// fp32, then the sequential scan in groups of 8 steps; the per-channel sums of y over the NG
 // lanes are a reduce-scatter, and y leaves through a staged tile with 16-byte stores.
 // When the grid has too few CTAs, time is split into segments whose entering states come from a
 // summary + carry pass (the local-scan / carry / correction structure of the three-phase scan in
