@@ -18,24 +18,37 @@ namespace {
 
 // ------------------------------------------------------------------------------------------------
 // Backward segment summary (segments 1..nseg-1): local reverse adjoint from zero over the
-// segment, v <- a_t (C_t dy_t + v), and P = prod a over the segment.
+// segment, v <- a_t (C_t dy_t + v), and P = prod a over the segment.  The segment streams through
+// shared memory from its end backwards in 32-step sub-tiles of dy, delta_raw and C, copied
+// asynchronously two sub-tiles ahead (three-stage ring), so the copies' latency stays off the
+// scan.
+template <typename E, int N>
+struct BwdSumSmem {
+    static constexpr int TS = 32, DT = kRealDT;
+    static constexpr int XE = TS * DT, CE = TS * N;
+    static constexpr int RAW = 3;                                      // raw stages
+    static constexpr int STAGE = (2 * XE + CE) * (int)sizeof(E);       // dy, delta_raw, C as stored
+    static constexpr int DEL = RAW * STAGE;                            // delta [TS][DT] fp32
+    static constexpr int CF = DEL + XE * 4;                            // C [TS][N] fp32
+    static constexpr int BYTES = CF + CE * 4;
+};
+
 template <typename E, int N, int S>
 __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(RealArgs p) {
     using Cfg = RealCfg<N, S>;
-    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, U = Cfg::U;
+    using Sm = BwdSumSmem<E, N>;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, U = Cfg::U, TS = Sm::TS;
     extern __shared__ __align__(16) unsigned char smem[];
-    const int T = p.T;
-    E* sdy = reinterpret_cast<E*>(smem);
-    E* sdr = sdy + T * DT;
-    float* sC = reinterpret_cast<float*>(sdr + T * DT);
-    float* sdel = sC + T * N;
+    float* sdel = reinterpret_cast<float*>(smem + Sm::DEL);
+    float* sCf = reinterpret_cast<float*>(smem + Sm::CF);
 
     const int tid = threadIdx.x, ng = tid % NG, dl = tid / NG;
     const int b = blockIdx.y, seg = blockIdx.z + 1;
     const int d0 = blockIdx.x * DT, d = d0 + dl, n0 = ng * S;
     const bool dv = d < p.D;
-    const int c_begin = seg * p.seg_chunks;
-    const int c_end = min(p.nC, c_begin + p.seg_chunks);
+    const int t_begin = seg * p.seg_chunks * p.T;
+    const int t_end = min(p.L, min(p.nC, (seg + 1) * p.seg_chunks) * p.T);
+    const int nsub = t_end > t_begin ? (t_end - t_begin + TS - 1) / TS : 0;
 
     float2 A2[P2], v[P2], P[P2];
 #pragma unroll
@@ -51,17 +64,37 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(Rea
     const E* drb = static_cast<const E*>(p.draw) + boff * p.D;
     const E* Cb = static_cast<const E*>(p.Cm) + boff * N;
 
-    for (int c = c_end - 1; c >= c_begin; --c) {
-        const int t0 = c * T;
-        const int rows = min(T, p.L - t0);
+    auto raw = [&](int k) { return reinterpret_cast<E*>(smem + (k % Sm::RAW) * Sm::STAGE); };
+    // sub-tile k holds steps [t_begin + k TS, min(t_end, t_begin + (k + 1) TS)), rounded up to
+    // whole groups of U; the rounding only reaches past the sequence end (segment ends are
+    // multiples of the chunk length), where the copies read zeros
+    auto issue = [&](int k) {
+        if (k >= 0) {
+            const int t0 = t_begin + k * TS;
+            const int rows4 = (min(TS, t_end - t0) + U - 1) / U * U;
+            E* sr = raw(k);
+            cp_async_tile<E, DT>(sr, dyb, t0, rows4, p.L, d0, p.D, tid, NT);
+            cp_async_tile<E, DT>(sr + Sm::XE, drb, t0, rows4, p.L, d0, p.D, tid, NT);
+            cp_async_flat<E>(sr + 2 * Sm::XE, Cb, (size_t)t0 * N, rows4 * N, (size_t)p.L * N, tid, NT);
+        }
+        cp_async_commit();  // an empty group before the first sub-tile keeps the wait counts uniform
+    };
+    issue(nsub - 1);
+    issue(nsub - 2);
+    for (int k = nsub - 1; k >= 0; --k) {
+        cp_async_wait<1>();  // sub-tile k is in (k - 1 may still be in flight)
+        __syncthreads();     // ... for every thread, and every thread is past the scan of k + 1
+        issue(k - 2);
+        const int t0 = t_begin + k * TS;
+        const int rows = min(TS, t_end - t0);
         const int rows4 = (rows + U - 1) / U * U;
-        __syncthreads();
-        load_tile<E, DT>(sdy, dyb, t0, rows4, p.L, d0, p.D, tid, NT);
-        load_tile<E, DT>(sdr, drb, t0, rows4, p.L, d0, p.D, tid, NT);
-        load_rows_f32<E, N>(sC, Cb, t0, rows4, p.L, tid, NT);
-        __syncthreads();
+        const E* sdy = raw(k);
+        const E* sdr = sdy + Sm::XE;
+        const E* sC = sdy + 2 * Sm::XE;
+        // steps past the sequence end get delta = 0 (a = 1; their dy reads zero)
         for (int i = tid; i < rows4 * DT; i += NT)
             sdel[i] = i < rows * DT ? softplus_fast(Elem<E>::to_f(sdr[i])) : 0.0f;
+        for (int i = tid; i < rows4 * N; i += NT) sCf[i] = Elem<E>::to_f(sC[i]);
         __syncthreads();
         for (int r0 = rows4 - U; r0 >= 0; r0 -= U) {
 #pragma unroll
@@ -70,7 +103,7 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(Rea
                 const float dlt = sdel[r * DT + dl];
                 const float dyv = Elem<E>::to_f(sdy[r * DT + dl]);
                 float2 cq[P2];
-                ld_pairs<S>(cq, sC + r * N + n0);
+                ld_pairs<S>(cq, sCf + r * N + n0);
 #pragma unroll
                 for (int i = 0; i < P2; ++i) {
                     const float2 a = ex2_pair(__fmul2_rn(f2(dlt), A2[i]));
@@ -80,6 +113,7 @@ __global__ void __launch_bounds__(RealCfg<N, S>::NT) real_bwd_summary_kernel(Rea
             }
         }
     }
+    cp_async_wait<0>();  // no copy outlives the CTA
     if (dv) {
         const size_t o = (((size_t)b * (p.nseg - 1) + (seg - 1)) * p.D + d) * N + n0;
         st_pairs<S>(p.gsumP + o, P);
@@ -823,10 +857,6 @@ __global__ void real_reduce_params_kernel(RealArgs p, int N) {
     }
 }
 
-template <int N, int S>
-size_t bwd_summary_smem(int T, int esz) {
-    return (size_t)T * kRealDT * esz * 2 + (size_t)T * N * 4 + (size_t)T * kRealDT * 4;
-}
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -839,12 +869,11 @@ cudaError_t set_smem(K kern, size_t bytes) {
 // launch only, so its size does not grow with L.
 template <typename E, int N, bool ZOH>
 cudaError_t real_bwd_impl(const RealArgs& a0, int group, cudaStream_t st) {
-    const int esz = (int)sizeof(E);
     cudaError_t e;
     RealArgs a = a0;
     if (a.nseg > 1 && !a.seq_blocks) {
         a.seg0 = 1;
-        const size_t sm = bwd_summary_smem<N, 4>(a.T, esz);
+        const size_t sm = BwdSumSmem<E, N>::BYTES;
         if ((e = set_smem(real_bwd_summary_kernel<E, N, 4>, sm)) != cudaSuccess) return e;
         real_bwd_summary_kernel<E, N, 4><<<dim3(a.ndt, a.B, a.nseg - 1), dim3(RealCfg<N, 4>::NT), sm, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
