@@ -57,7 +57,8 @@ template <typename E, int N, int S, bool SUMMARY, bool ZOH>
 __global__ void __launch_bounds__(FwdCfg<N, S>::NT) real_fwd_kernel(RealArgs p) {
     using Cfg = FwdCfg<N, S>;
     using Sm = FwdSmem<E, N>;
-    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TT = Cfg::TT, U = Cfg::U;
+    constexpr int P2 = Cfg::P2, NG = Cfg::NG, DT = Cfg::DT, NT = Cfg::NT, TT = Cfg::TT;
+    constexpr int U = SUMMARY ? 16 : Cfg::U;  // the segment summaries (no y) scan 16-step groups
     extern __shared__ __align__(16) unsigned char smem[];
     float2* sdd = reinterpret_cast<float2*>(smem + Sm::DD);
     float* sBf = reinterpret_cast<float*>(smem + Sm::BF);
