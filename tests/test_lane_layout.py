@@ -1,4 +1,6 @@
-"""Host model check of the lane arithmetic the real backward uses for its dB / dC channel sums.
+"""Host model checks of the index arithmetic of the real kernels: the lanes of the backward's
+dB / dC channel sums, the partition of its fused sums, and the sub-tile walk of the segment
+summaries.
 
 A thread of the backward holds four states of one channel.  Its state slots are rotated by its
 position `rot` among four neighbouring channel lanes (slot j holds state n0 + ((j + rot) & 3)),
@@ -109,3 +111,46 @@ def test_fused_dbc_share_partition(N):
                             written[o] = written.get(o, 0) + 1
         assert written == {(r, e): 1 for r in range(rows) for e in range(N2)}
         assert reads == {(j, r, e): 1 for j in range(ndt) for r in range(rows) for e in range(0, N2, 4)}
+
+
+def summary_subtiles(L, T, seg_chunks, seg, TS, U):
+    """The sub-tile walk of a segment summary, as the backward summary kernel
+    (`real_bwd_summary_kernel`, TS = 32, U = 4) and the forward's summary instance (TS = min(T,
+    32), U = 16) index it: (t0, rows, rows4) of sub-tiles k = 0..nsub-1 and, for the backward's
+    three-stage ring, the raw stage each one occupies."""
+    nC = -(-L // T)
+    t_begin = seg * seg_chunks * T
+    t_end = min(L, min(nC, (seg + 1) * seg_chunks) * T)
+    nsub = -(-(t_end - t_begin) // TS) if t_end > t_begin else 0
+    tiles = []
+    for k in range(nsub):
+        t0 = t_begin + k * TS
+        rows = min(TS, t_end - t0)
+        rows4 = -(-rows // U) * U
+        tiles.append((t0, rows, rows4, k % 3))
+    return t_begin, t_end, tiles
+
+
+@pytest.mark.parametrize("T", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("TS,U", [(32, 4), ("fwd", 16)])
+def test_segment_summary_subtiles_cover_each_step_once(T, TS, U):
+    """Every step of a summarised segment lies in exactly one sub-tile; the rounding of a
+    sub-tile to whole U-step groups stays inside the staged tile (32 rows) and reaches only past
+    the sequence end, where the copies read zeros (so the rounded steps, with delta = 0, change
+    nothing); and in the backward's ring the stage a sub-tile's copies are issued into (two
+    ahead, k - 2, walking k downwards) is the one the sub-tile processed just before (k + 1)
+    occupied."""
+    ts = min(T, 32) if TS == "fwd" else TS
+    for L, sc in itertools.product((1, 15, 16, 17, 100, 257, 1000, 4099), (1, 2, 3, 7)):
+        nseg = -(-(-(-L // T)) // sc)
+        for seg in range(1, nseg):
+            t_begin, t_end, tiles = summary_subtiles(L, T, sc, seg, ts, U)
+            covered = []
+            for t0, rows, rows4, _ in tiles:
+                assert 0 < rows <= ts and rows4 <= 32
+                covered.extend(range(t0, t0 + rows))
+                assert all(t >= L for t in range(t0 + rows, t0 + rows4))
+            assert covered == list(range(t_begin, t_end))
+            if TS != "fwd":
+                for k in range(2, len(tiles) - 1):
+                    assert tiles[k - 2][3] == tiles[k + 1][3]
