@@ -55,3 +55,22 @@ def test_traffic_records_follow_kernel_code_not_comments(tmp_path):
             assert got == float(rec["dram_bytes_per_launch"]), rec["source"]
         else:
             assert got is None
+
+
+def test_l2_flush_writes_then_reads_buffers_larger_than_l2():
+    """The flush between timed steps: a write of 256 MiB (twice the 126 MB L2) and a read of
+    another 256 MiB buffer, so that the written lines are evicted (and written back) before the
+    step's events start; checked on the host's device-independent tensors."""
+    import importlib.util
+    import torch
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    f = bench.L2Flush("cpu")
+    assert f.wr.numel() * f.wr.element_size() == 256 << 20
+    assert f.rd.numel() * f.rd.element_size() == 256 << 20
+    assert f.wr.data_ptr() != f.rd.data_ptr()
+    f.wr.fill_(7)
+    f()
+    assert int(f.wr.max()) == 0 and float(f.acc) == 0.0
