@@ -60,9 +60,8 @@ def test_traffic_records_follow_kernel_code_not_comments(tmp_path):
 def test_l2_flush_writes_then_reads_buffers_larger_than_l2():
     """The flush between timed steps: a write of 256 MiB (twice the 126 MB L2) and a read of
     another 256 MiB buffer, so that the written lines are evicted (and written back) before the
-    step's events start; checked on the host's device-independent tensors."""
+    step's events start; checked here with CPU tensors."""
     import importlib.util
-    import torch
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
     bench = importlib.util.module_from_spec(spec)
